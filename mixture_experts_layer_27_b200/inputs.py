@@ -1,0 +1,148 @@
+"""Seeded synthetic inputs for the MoE layer (shared by tests, bench and smoke).
+
+This module holds no arithmetic of the layer itself: it only draws tensors.
+Both the CUDA path and the CPU oracle consume the exact bits it produces.
+
+Workloads (the pages name model families and print no shapes; these stand in):
+
+* ``tiny``      T=128,  d=256,  E=8,   k=2, I=512
+* ``dsv3``      T=2048, d=7168, E=256, k=8, I=2048   (DeepSeek-V3-like, near-uniform routing)
+* ``kimi``      T=4096, d=7168, E=384, k=8, I=2048   (Kimi-K2-like, Zipf(1.2)-skewed load)
+* ``kimi_mx``   ``kimi`` in MXFP8 mode
+* ``ep64``      6 local experts of 384, 16 minibatches x 2048 tokens, ring buffer
+
+Distributions: X, dY ~ N(0, 1); W_gate, W_up ~ N(0, 1/d) (std 1/sqrt(fan_in));
+W_down ~ N(0, 1/I); W_r ~ N(0, 0.02^2); every tensor rounded once to bf16 (RNE).
+Every tensor (and every expert's slice) has its own seed derived from the
+workload seed and the tensor name, so tensors can be regenerated one by one.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import hashlib
+import math
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    T: int
+    d: int
+    E: int
+    k: int
+    I: int
+    mxfp8: bool = False
+    zipf: bool = False          # per-expert router bias giving a Zipf(1.2)-shaped load
+    first_local: int = 0
+    num_local: int = 0          # 0 = all experts are local
+    seed: int = 0
+
+    @property
+    def El(self) -> int:
+        return self.num_local or self.E
+
+    def model_flops(self) -> float:
+        """fwd+bwd model FLOPs: 18 d I per assignment (6 fwd, 12 bwd) + 6 T d E router."""
+        return 18.0 * self.d * self.I * self.T * self.k + 6.0 * self.T * self.d * self.E
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", 128, 256, 8, 2, 512),
+    "dsv3": Workload("dsv3", 2048, 7168, 256, 8, 2048),
+    "kimi": Workload("kimi", 4096, 7168, 384, 8, 2048, zipf=True),
+    "kimi_mx": Workload("kimi_mx", 4096, 7168, 384, 8, 2048, mxfp8=True, zipf=True),
+}
+
+
+def _seed(base: int, *names) -> int:
+    h = hashlib.sha256(("%d/" % base + "/".join(str(n) for n in names)).encode()).digest()
+    return int.from_bytes(h[:8], "little") & ((1 << 63) - 1)
+
+
+def _normal(shape, std, seed, device):
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(torch.bfloat16)
+
+
+def expert_weights(w: Workload, name: str, e: int, device="cpu") -> torch.Tensor:
+    """One expert's slice of W_gate / W_up ([d, I]) or W_down ([I, d]), bf16."""
+    if name in ("W_gate", "W_up"):
+        return _normal((w.d, w.I), 1.0 / math.sqrt(w.d), _seed(w.seed, w.name, name, e), device)
+    if name == "W_down":
+        return _normal((w.I, w.d), 1.0 / math.sqrt(w.I), _seed(w.seed, w.name, name, e), device)
+    raise KeyError(name)
+
+
+def make_inputs(w: Workload, device="cpu", T: int | None = None) -> dict:
+    """All layer inputs for workload w (T may be overridden to sub-sample tokens)."""
+    T = T or w.T
+    out = {
+        "X": _normal((T, w.d), 1.0, _seed(w.seed, w.name, "X"), device),
+        "W_r": _normal((w.d, w.E), 0.02, _seed(w.seed, w.name, "W_r"), device),
+        "dY": _normal((T, w.d), 1.0, _seed(w.seed, w.name, "dY"), device),
+    }
+    El = w.El
+    for name in ("W_gate", "W_up", "W_down"):
+        shape = (El, w.d, w.I) if name != "W_down" else (El, w.I, w.d)
+        t = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        for el in range(El):
+            t[el] = expert_weights(w, name, w.first_local + el, device)
+        out[name] = t
+    out["bias"] = zipf_bias(w, out["X"], out["W_r"]) if w.zipf else None
+    return out
+
+
+def zipf_target_shares(E: int, s: float = 1.2, hot_over_mean: float = 10.0) -> torch.Tensor:
+    """Shares q_r proportional to (r + r0)^-s, r = 1..E, with r0 chosen so max/mean = hot_over_mean.
+
+    Pure Zipf(1.2) at E = 384 would put ~94x the mean load on the hottest
+    expert, more than one expert can take (T tokens = 48x the mean at k = 8),
+    and the workload asks for ~10x; the offset r0 reconciles the two.
+    """
+    r = torch.arange(1, E + 1, dtype=torch.float64)
+
+    def ratio(r0):
+        q = (r + r0) ** (-s)
+        return float(q[0] / q.mean())
+
+    lo, hi = 0.0, 1e4
+    for _ in range(200):
+        mid = 0.5 * (lo + hi)
+        if ratio(mid) > hot_over_mean:
+            lo = mid
+        else:
+            hi = mid
+    q = (r + 0.5 * (lo + hi)) ** (-s)
+    return q / q.sum()
+
+
+def zipf_bias(w: Workload, X: torch.Tensor, W_r: torch.Tensor, iters: int = 60) -> torch.Tensor:
+    """Per-expert router bias (fp32 [E]) that skews top-k load toward Zipf shares.
+
+    Fixed-count calibration on the seeded logits: b_e += 0.5 (log target_e -
+    log max(observed_e, 0.5)).  The rank -> expert map is a seeded permutation.
+    torch.topk only measures load here; the layer's own selection rule is not used.
+    """
+    dev = X.device
+    logits = X.float() @ W_r.float()
+    q = zipf_target_shares(w.E)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(_seed(w.seed, w.name, "zipf_perm"))
+    perm = torch.randperm(w.E, generator=g)
+    target = torch.empty(w.E, dtype=torch.float64)
+    target[perm] = q * X.shape[0] * w.k
+    target = target.to(dev)
+    b = torch.zeros(w.E, dtype=torch.float64, device=dev)
+    for _ in range(iters):
+        idx = torch.topk(logits + b.float(), w.k, dim=1).indices
+        obs = torch.bincount(idx.flatten(), minlength=w.E).double()
+        b += 0.5 * (torch.log(target) - torch.log(torch.clamp(obs, min=0.5)))
+        b -= b.mean()
+    return b.float()

@@ -1,0 +1,390 @@
+"""Oracle: a plain, slow, fp64 CPU statement of the MoE layer forward and backward.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg
+use it.  It shares no code, table or helper with the CUDA path.
+
+What it follows
+---------------
+The pages ("Cursor open-sources Mixture-of-Kittens (MoK)...", page 1) describe a
+mixture-of-experts training layer:
+
+* "MoE layer as the bottleneck" and the toknow.ai summary (page 2): every token is
+  routed to a few experts (router scores -> top-k experts).
+* "Three design decisions that matter", bullet 1: one schedule table drives the
+  forward dispatch / combine and the backward reverse-combine / reverse-dispatch.
+* "Three design decisions that matter", bullet 2: experts run as an
+  expert-grouped GEMM.
+* same section, closing paragraph: the experts are SwiGLU MLPs, and the router
+  weight gradient is computed "SonicMoE-style" inside the SwiGLU backward; the
+  layer supports BF16 and MXFP8 precision modes and is fully deterministic.
+
+The pages print no formula.  The layer's arithmetic is therefore the plain
+definition of a top-k softmax-gated SwiGLU mixture of experts:
+
+    l   = X W_r + b                         router logits            [T, E]
+    S_t = the k largest entries of l_t      (descending; ties -> lower expert id)
+    g   = exp(l_t,e) / sum_{e' in S_t} exp(l_t,e')   for e in S_t     (gates)
+    A   = X_t W_gate[e],  B = X_t W_up[e],  H = silu(A) * B
+    O   = H W_down[e]
+    Y_t = sum_{e in S_t} g_t,e O_t,e
+
+and its exact gradient (the selection is piecewise constant, so no gradient
+flows through it; the bias b is an input without gradient):
+
+    dO  = g dY_t,  dH = dO W_down[e]^T
+    dA  = dH * B * silu'(A),  dB = dH * silu(A)
+    dg  = <dY_t, O_t,e>
+    dl_t,e = g_t,e (dg_t,e - sum_m g_t,m dg_t,m) on S_t, 0 elsewhere
+    dX_t  = sum_e (dA W_gate[e]^T + dB W_up[e]^T) + dl_t W_r^T
+    dW_r  = X^T dl
+    dW_gate[e] = sum_t X_t^T dA,  dW_up[e] = sum_t X_t^T dB,
+    dW_down[e] = sum_t H^T dO.
+
+Readings where the pages are silent (each is listed in the design notes):
+
+* selection runs on the (biased) logits, ties broken by the lower expert id,
+  values compared as numbers (-0 == +0), NaN ranked lowest;
+* ids inside a token are ordered by descending logit (ties: ascending id);
+* "softmax over E then renormalise over the top k" equals a softmax over the
+  selected k logits, which is what is computed;
+* the schedule: counts per expert, exclusive prefix sums (unpadded and padded
+  to P = 128 rows), a stable per-expert token order (ascending token id);
+* experts outside [first_local, first_local + num_local) are excluded (their
+  assignments belong to another rank): they add nothing to Y, dX or dl;
+* dg is computed the direct way, <dY, O>; the fused "SonicMoE-style" form
+  <dY W_down^T, H> is an identity the tests check, not something shared.
+
+Every floating-point step is fp64; inputs are the exact values the GPU gets.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+P_PAD = 128  # rows per expert segment are padded to a multiple of this
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+def _f64(a) -> np.ndarray:
+    return np.asarray(a, dtype=np.float64)
+
+
+def _expert(W, e: int) -> np.ndarray:
+    """Weights of expert e as fp64; W is an [E, ...] array or a callable e -> array."""
+    return _f64(W(e) if callable(W) else W[e])
+
+
+def silu(a: np.ndarray) -> np.ndarray:
+    """silu(a) = a * sigmoid(a) = a / (1 + exp(-a)), written overflow-safely."""
+    return a * _sigmoid(a)
+
+
+def _sigmoid(a: np.ndarray) -> np.ndarray:
+    out = np.empty_like(a)
+    pos = a >= 0
+    out[pos] = 1.0 / (1.0 + np.exp(-a[pos]))
+    ea = np.exp(a[~pos])
+    out[~pos] = ea / (1.0 + ea)
+    return out
+
+
+def silu_grad(a: np.ndarray) -> np.ndarray:
+    """d silu / da = s (1 + a (1 - s)), s = sigmoid(a)."""
+    s = _sigmoid(a)
+    return s * (1.0 + a * (1.0 - s))
+
+
+# ----------------------------------------------------------------------------
+# routing (page 2 "routes each input to a few of them"; page 1 closing
+# paragraph of "Three design decisions": deterministic)
+# ----------------------------------------------------------------------------
+def router_logits(X, W_r, bias=None) -> np.ndarray:
+    """l = X W_r (+ b).  X [T, d], W_r [d, E], b [E] or None -> [T, E] fp64."""
+    l = _f64(X) @ _f64(W_r)
+    if bias is not None:
+        l = l + _f64(bias)[None, :]
+    return l
+
+
+def topk_ids(logits, k: int) -> np.ndarray:
+    """Top-k expert ids per row, by descending logit; equal logits -> lower id first.
+
+    Values are compared as numbers, so -0 and +0 tie; NaN ranks below everything
+    (also below -inf).  Returns int32 [T, k].
+    """
+    l = np.asarray(logits)
+    T, E = l.shape
+    if not 1 <= k <= E:
+        raise ValueError("top_k must be in [1, E]")
+    ids = np.empty((T, k), dtype=np.int32)
+    idx = np.arange(E)
+    for t in range(T):
+        row = l[t].astype(np.float64)
+        nan = np.isnan(row)
+        key = np.where(nan, 0.0, -row)  # descending value ...
+        # lexsort: last key is primary.  NaN first pushed to the back, then value, then id.
+        order = np.lexsort((idx, key, nan.astype(np.int8)))
+        ids[t] = order[:k]
+    return ids
+
+
+def gates(logits, ids) -> np.ndarray:
+    """Softmax over the k selected logits of each row (fp64 [T, k])."""
+    l = _f64(logits)
+    sel = np.take_along_axis(l, ids.astype(np.int64), axis=1)
+    m = sel.max(axis=1, keepdims=True)
+    ex = np.exp(sel - m)
+    return ex / ex.sum(axis=1, keepdims=True)
+
+
+def schedule(ids, E: int, first_local: int = 0, num_local: int | None = None, P: int = P_PAD) -> dict:
+    """The routing table shared by dispatch, combine and their backward mirrors.
+
+    counts[e]          number of (token, slot) assignments to local expert e
+    offsets[E_l+1]     exclusive prefix sum of counts (unpadded rows)
+    padded_offsets     exclusive prefix sum of ceil(counts / P) * P
+    perm[rows]         token of each unpadded row; inside an expert, ascending token id
+    slot_row[T, k]     padded row of each assignment, -1 for non-local experts
+    Here e runs over the local experts only (index e - first_local).
+    """
+    ids = np.asarray(ids)
+    T, k = ids.shape
+    if num_local is None:
+        num_local = E - first_local
+    El = num_local
+    local = (ids >= first_local) & (ids < first_local + El)
+    le = np.where(local, ids - first_local, -1)
+    counts = np.zeros(El, dtype=np.int64)
+    for e in le[local]:
+        counts[e] += 1
+    offsets = np.zeros(El + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    padded = ((counts + P - 1) // P) * P
+    padded_offsets = np.zeros(El + 1, dtype=np.int64)
+    padded_offsets[1:] = np.cumsum(padded)
+    perm = np.empty(int(offsets[-1]), dtype=np.int64)
+    slot_row = np.full((T, k), -1, dtype=np.int64)
+    fill = np.zeros(El, dtype=np.int64)
+    for t in range(T):  # ascending token order gives the stable per-expert order
+        for j in range(k):
+            e = le[t, j]
+            if e < 0:
+                continue
+            pos = fill[e]
+            fill[e] += 1
+            perm[offsets[e] + pos] = t
+            slot_row[t, j] = padded_offsets[e] + pos
+    return dict(counts=counts, offsets=offsets, padded_offsets=padded_offsets,
+                perm=perm, slot_row=slot_row, first_local=first_local, num_local=El)
+
+
+def _expert_rows(ids, sched, e_local: int):
+    """(tokens, slots) assigned to local expert e_local, in the schedule's row order."""
+    o0, o1 = sched["offsets"][e_local], sched["offsets"][e_local + 1]
+    toks = sched["perm"][o0:o1]
+    e = e_local + sched["first_local"]
+    slots = np.array([int(np.nonzero(ids[t] == e)[0][0]) for t in toks], dtype=np.int64)
+    return toks, slots
+
+
+# ----------------------------------------------------------------------------
+# forward / backward (page 1, "Three design decisions that matter")
+# ----------------------------------------------------------------------------
+def forward(X, W_r, bias, W_gate, W_up, W_down, top_k: int,
+            first_local: int = 0, num_local: int | None = None, keep=True):
+    """MoE layer forward in fp64.  Returns (Y [T, d], ctx for backward)."""
+    X64 = _f64(X)
+    T, d = X64.shape
+    E = np.asarray(W_r).shape[1]
+    logits = router_logits(X64, W_r, bias)
+    ids = topk_ids(logits, top_k)
+    g = gates(logits, ids)
+    sched = schedule(ids, E, first_local, num_local)
+    Y = np.zeros((T, d))
+    saved = []
+    for el in range(sched["num_local"]):
+        toks, slots = _expert_rows(ids, sched, el)
+        if toks.size == 0:
+            saved.append(None)
+            continue
+        e = el + sched["first_local"]
+        Xe = X64[toks]
+        A = Xe @ _expert(W_gate, e)
+        B = Xe @ _expert(W_up, e)
+        H = silu(A) * B
+        O = H @ _expert(W_down, e)
+        ge = g[toks, slots]
+        Y[toks] += ge[:, None] * O  # each token appears once per expert
+        saved.append((toks, slots, A, B) if keep else None)
+    ctx = dict(X=X64, W_r=_f64(W_r), W_gate=W_gate, W_up=W_up, W_down=W_down,
+               logits=logits, ids=ids, g=g, sched=sched, saved=saved, E=E)
+    return Y, ctx
+
+
+def backward(ctx, dY):
+    """Exact gradient of the forward (selection held fixed).  All fp64."""
+    dY64 = _f64(dY)
+    X64, ids, g, sched = ctx["X"], ctx["ids"], ctx["g"], ctx["sched"]
+    T, d = X64.shape
+    k = ids.shape[1]
+    E = ctx["E"]
+    dX = np.zeros((T, d))
+    dg = np.zeros((T, k))
+    dW_gate, dW_up, dW_down = {}, {}, {}
+    for el in range(sched["num_local"]):
+        e = el + sched["first_local"]
+        item = ctx["saved"][el]
+        Wg, Wu, Wd = _expert(ctx["W_gate"], e), _expert(ctx["W_up"], e), _expert(ctx["W_down"], e)
+        if item is None:
+            toks, slots = _expert_rows(ids, sched, el)
+            if toks.size == 0:
+                I = Wg.shape[1]
+                dW_gate[e] = np.zeros((d, I)); dW_up[e] = np.zeros((d, I)); dW_down[e] = np.zeros((I, d))
+                continue
+            Xe = X64[toks]
+            A, B = Xe @ Wg, Xe @ Wu
+        else:
+            toks, slots, A, B = item
+            Xe = X64[toks]
+        H = silu(A) * B
+        O = H @ Wd
+        dYe = dY64[toks]
+        ge = g[toks, slots]
+        dg[toks, slots] = np.sum(dYe * O, axis=1)  # <dY_t, O_t,e>
+        dO = ge[:, None] * dYe
+        dH = dO @ Wd.T
+        dA = dH * B * silu_grad(A)
+        dB = dH * silu(A)
+        dX[toks] += dA @ Wg.T + dB @ Wu.T
+        dW_gate[e] = Xe.T @ dA
+        dW_up[e] = Xe.T @ dB
+        dW_down[e] = H.T @ dO
+    # router: softmax-over-selected Jacobian, scattered to the selected experts
+    dl = np.zeros((T, E))
+    s = np.sum(g * dg, axis=1, keepdims=True)
+    np.put_along_axis(dl, ids.astype(np.int64), g * (dg - s), axis=1)
+    dX += dl @ ctx["W_r"].T
+    dW_r = X64.T @ dl
+    return dict(dX=dX, dW_gate=dW_gate, dW_up=dW_up, dW_down=dW_down, dW_r=dW_r,
+                dl=dl, dg=dg)
+
+
+def token_forward_backward(t: int, X, W_r, bias, W_gate, W_up, W_down, top_k: int, dY,
+                           first_local: int = 0, num_local: int | None = None):
+    """Y_t, dX_t and dl_t for one token: each depends on that token's data alone.
+
+    Used to check full-size GPU results at sampled tokens without running the
+    whole layer on the CPU.  Same definition as forward/backward, one row.
+    """
+    x = _f64(X)[t:t + 1]
+    E = np.asarray(W_r).shape[1]
+    l = router_logits(x, W_r, bias)
+    ids = topk_ids(l, top_k)
+    g = gates(l, ids)[0]
+    lo = first_local
+    hi = E if num_local is None else first_local + num_local
+    dy = _f64(dY)[t]
+    y = np.zeros(x.shape[1])
+    dx = np.zeros(x.shape[1])
+    dg = np.zeros(top_k)
+    for j, e in enumerate(ids[0]):
+        if not lo <= e < hi:
+            continue
+        Wg, Wu, Wd = _expert(W_gate, e), _expert(W_up, e), _expert(W_down, e)
+        a = x[0] @ Wg
+        b = x[0] @ Wu
+        h = silu(a) * b
+        o = h @ Wd
+        y += g[j] * o
+        dg[j] = dy @ o
+        dh = (g[j] * dy) @ Wd.T
+        dx += (dh * b * silu_grad(a)) @ Wg.T + (dh * silu(a)) @ Wu.T
+    dl = np.zeros(E)
+    dl[ids[0]] = g * (dg - np.sum(g * dg))
+    dx += dl @ _f64(W_r).T
+    return y, dx, dl, ids[0], g
+
+
+# ----------------------------------------------------------------------------
+# MXFP8 (page 1: "It supports BF16 and MXFP8 precision modes").  The block
+# format (E4M3 payload, one E8M0 power-of-two scale per 32 values along the
+# contraction dimension) is the OCP Microscaling v1.0 format; the scale rule is
+# that format's: shared exponent = floor(log2(amax)) - emax(E4M3) = ... - 8.
+# ----------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """E4M3 (OCP 'FN': bias 7, no infinities, S.1111.111 = NaN) bytes -> fp64."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    s = np.where(c & 0x80, -1.0, 1.0)
+    ex = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(ex == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * 2.0 ** (ex - 7))
+    val = np.where((ex == 0xF) & (m == 0x7), np.nan, val)
+    return s * val
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """fp64 -> E4M3 byte, round to nearest even, saturating to +-448 (satfinite)."""
+    x = _f64(x)
+    out = np.zeros(x.shape, dtype=np.uint8)
+    sign = (np.signbit(x)).astype(np.int64) << 7
+    a = np.abs(x)
+    a = np.minimum(a, E4M3_MAX)  # satfinite (NaN input is not produced by the layer)
+    nz = a > 0
+    # exponent of the binade, at least the subnormal exponent -6
+    e = np.full(a.shape, -6, dtype=np.int64)
+    e[nz] = np.maximum(np.floor(np.log2(a[nz])).astype(np.int64), -6)
+    quantum = np.ldexp(1.0, (e - 3).astype(np.int64))
+    q = np.round(a / quantum) * quantum  # np.round rounds halves to even
+    q = np.minimum(q, E4M3_MAX)
+    # encode q exactly
+    code = np.zeros(a.shape, dtype=np.int64)
+    qnz = q > 0
+    eq = np.full(a.shape, -6, dtype=np.int64)
+    eq[qnz] = np.floor(np.log2(q[qnz])).astype(np.int64)
+    normal = qnz & (eq >= -6) & (q >= 2.0 ** -6)
+    sub = qnz & ~normal
+    mant_n = np.rint(q / np.ldexp(1.0, eq) * 8.0 - 8.0).astype(np.int64)
+    code = np.where(normal, ((eq + 7) << 3) | mant_n, code)
+    code = np.where(sub, np.rint(q / 2.0 ** -9).astype(np.int64), code)
+    out[...] = (code | sign).astype(np.uint8)
+    return out
+
+
+def mx_quantize(v, axis: int = -1, block: int = 32):
+    """MX block quantisation of v along `axis` in blocks of `block` values.
+
+    Returns (codes uint8 [same shape], scale bytes uint8 [..., n/block, ...]).
+    scale byte = shared exponent + 127; a block whose amax is 0 gets byte 0 and
+    all-zero codes.  Value represented: e4m3_decode(code) * 2**(byte - 127).
+    """
+    v = np.moveaxis(_f64(v), axis, -1)
+    n = v.shape[-1]
+    if n % block:
+        raise ValueError("length along the block axis must be a multiple of the block")
+    vb = v.reshape(v.shape[:-1] + (n // block, block))
+    amax = np.max(np.abs(vb), axis=-1)
+    zero = amax == 0
+    se = np.zeros(amax.shape, dtype=np.int64)
+    se[~zero] = np.floor(np.log2(amax[~zero])).astype(np.int64) - 8
+    se = np.clip(se, -127, 127)
+    scaled = vb * np.ldexp(1.0, -se)[..., None]
+    codes = e4m3_encode(scaled)
+    codes[zero] = 0
+    sbytes = np.where(zero, 0, se + 127).astype(np.uint8)
+    codes = np.moveaxis(codes.reshape(v.shape), -1, axis)
+    sbytes = np.moveaxis(sbytes, -1, axis)
+    return codes, sbytes
+
+
+def mx_dequantize(codes, sbytes, axis: int = -1, block: int = 32) -> np.ndarray:
+    c = np.moveaxis(np.asarray(codes), axis, -1)
+    s = np.moveaxis(np.asarray(sbytes), axis, -1).astype(np.int64)
+    vals = e4m3_decode(c).reshape(c.shape[:-1] + (c.shape[-1] // block, block))
+    vals = vals * np.ldexp(1.0, s - 127)[..., None]
+    return np.moveaxis(vals.reshape(c.shape), -1, axis)

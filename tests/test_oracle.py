@@ -1,0 +1,353 @@
+"""Pins for the fp64 oracle, each against something other than the oracle itself.
+
+* central finite differences of the forward (brute force) pin every gradient;
+* torch autograd / torch.topk / torch float8 casts (library routines) pin the
+  closed-form special cases (identical experts, k = E, E = 1) and the encoders;
+* invariants of the routing table (counts, prefix sums, a stable bijection).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+
+def _rand_layer(rng, T, d, E, I, k, scale_r=0.5):
+    X = rng.standard_normal((T, d))
+    W_r = rng.standard_normal((d, E)) * scale_r
+    Wg = rng.standard_normal((E, d, I)) / np.sqrt(d)
+    Wu = rng.standard_normal((E, d, I)) / np.sqrt(d)
+    Wd = rng.standard_normal((E, I, d)) / np.sqrt(I)
+    dY = rng.standard_normal((T, d))
+    return X, W_r, Wg, Wu, Wd, dY
+
+
+def _loss(X, W_r, b, Wg, Wu, Wd, k, dY):
+    Y, _ = O.forward(X, W_r, b, Wg, Wu, Wd, k)
+    return float(np.sum(Y * dY))
+
+
+def _margin_ok(X, W_r, b, k, tol):
+    l = O.router_logits(X, W_r, b)
+    s = -np.sort(-l, axis=1)
+    return np.all(s[:, k - 1] - s[:, k] > tol) if k < l.shape[1] else True
+
+
+# --------------------------------------------------------------------------
+# finite differences (brute force) on a tiny layer
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_gradients_match_central_differences(seed):
+    rng = np.random.default_rng(seed)
+    T, d, E, I, k = 4, 8, 4, 16, 2
+    X, W_r, Wg, Wu, Wd, dY = _rand_layer(rng, T, d, E, I, k)
+    b = rng.standard_normal(E) * 0.1
+    assert _margin_ok(X, W_r, b, k, 1e-3), "selection too close to a tie for FD"
+    _, ctx = O.forward(X, W_r, b, Wg, Wu, Wd, k)
+    gr = O.backward(ctx, dY)
+    h = 1e-6
+
+    def fd(arr, idx):
+        old = arr[idx]
+        arr[idx] = old + h
+        lp = _loss(X, W_r, b, Wg, Wu, Wd, k, dY)
+        arr[idx] = old - h
+        lm = _loss(X, W_r, b, Wg, Wu, Wd, k, dY)
+        arr[idx] = old
+        return (lp - lm) / (2 * h)
+
+    def check(arr, grad):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            num[idx] = fd(arr, idx)
+        err = np.max(np.abs(num - grad)) / max(np.max(np.abs(num)), 1e-30)
+        assert err < 1e-6, err
+
+    check(X, gr["dX"])
+    check(W_r, gr["dW_r"])
+    check(Wg, np.stack([gr["dW_gate"][e] for e in range(E)]))
+    check(Wu, np.stack([gr["dW_up"][e] for e in range(E)]))
+    check(Wd, np.stack([gr["dW_down"][e] for e in range(E)]))
+
+
+# --------------------------------------------------------------------------
+# closed forms, against torch autograd in float64
+# --------------------------------------------------------------------------
+def _dense_swiglu_torch(X, Wg, Wu, Wd, dY):
+    x = torch.tensor(X, requires_grad=True)
+    wg = torch.tensor(Wg, requires_grad=True)
+    wu = torch.tensor(Wu, requires_grad=True)
+    wd = torch.tensor(Wd, requires_grad=True)
+    y = (torch.nn.functional.silu(x @ wg) * (x @ wu)) @ wd
+    (y * torch.tensor(dY)).sum().backward()
+    return y.detach().numpy(), x.grad.numpy(), wg.grad.numpy(), wu.grad.numpy(), wd.grad.numpy()
+
+
+def test_identical_experts_equal_one_dense_swiglu_mlp():
+    rng = np.random.default_rng(3)
+    T, d, E, I, k = 37, 16, 6, 24, 3
+    X, W_r, Wg, Wu, Wd, dY = _rand_layer(rng, T, d, E, I, k)
+    Wg[:] = Wg[0]; Wu[:] = Wu[0]; Wd[:] = Wd[0]
+    Y, ctx = O.forward(X, W_r, None, Wg, Wu, Wd, k)
+    gr = O.backward(ctx, dY)
+    y, dx, dwg, dwu, dwd = _dense_swiglu_torch(X, Wg[0], Wu[0], Wd[0], dY)
+    np.testing.assert_allclose(Y, y, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(gr["dX"], dx, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(sum(gr["dW_gate"].values()), dwg, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(sum(gr["dW_up"].values()), dwu, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(sum(gr["dW_down"].values()), dwd, rtol=1e-10, atol=1e-11)
+    # every selected expert returns the same output, so the router gets no gradient
+    assert np.max(np.abs(gr["dl"])) < 1e-12
+    assert np.max(np.abs(gr["dW_r"])) < 1e-11
+
+
+def test_single_expert_is_dense_mlp_with_unit_gate():
+    rng = np.random.default_rng(4)
+    T, d, E, I, k = 9, 8, 1, 16, 1
+    X, W_r, Wg, Wu, Wd, dY = _rand_layer(rng, T, d, E, I, k)
+    Y, ctx = O.forward(X, W_r, None, Wg, Wu, Wd, k)
+    assert np.all(ctx["g"] == 1.0)
+    gr = O.backward(ctx, dY)
+    y, dx, dwg, dwu, dwd = _dense_swiglu_torch(X, Wg[0], Wu[0], Wd[0], dY)
+    np.testing.assert_allclose(Y, y, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(gr["dX"], dx, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(gr["dW_gate"][0], dwg, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(gr["dW_down"][0], dwd, rtol=1e-10, atol=1e-11)
+    assert np.all(gr["dW_r"] == 0)
+
+
+def test_k_equals_E_is_dense_softmax_mixture():
+    """With every expert selected the gates are a full softmax and differentiable."""
+    rng = np.random.default_rng(5)
+    T, d, E, I = 11, 8, 4, 12
+    X, W_r, Wg, Wu, Wd, dY = _rand_layer(rng, T, d, E, I, E)
+    b = rng.standard_normal(E) * 0.3
+    Y, ctx = O.forward(X, W_r, b, Wg, Wu, Wd, E)
+    gr = O.backward(ctx, dY)
+    x = torch.tensor(X, requires_grad=True)
+    wr = torch.tensor(W_r, requires_grad=True)
+    wg = torch.tensor(Wg, requires_grad=True)
+    wu = torch.tensor(Wu, requires_grad=True)
+    wd = torch.tensor(Wd, requires_grad=True)
+    p = torch.softmax(x @ wr + torch.tensor(b), dim=1)  # [T, E]
+    outs = torch.stack([(torch.nn.functional.silu(x @ wg[e]) * (x @ wu[e])) @ wd[e] for e in range(E)], 1)
+    y = (p[:, :, None] * outs).sum(1)
+    (y * torch.tensor(dY)).sum().backward()
+    np.testing.assert_allclose(Y, y.detach().numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(gr["dX"], x.grad.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(gr["dW_r"], wr.grad.numpy(), rtol=1e-10, atol=1e-11)
+    for e in range(E):
+        np.testing.assert_allclose(gr["dW_gate"][e], wg.grad[e].numpy(), rtol=1e-10, atol=1e-11)
+        np.testing.assert_allclose(gr["dW_up"][e], wu.grad[e].numpy(), rtol=1e-10, atol=1e-11)
+        np.testing.assert_allclose(gr["dW_down"][e], wd.grad[e].numpy(), rtol=1e-10, atol=1e-11)
+
+
+def test_topk_gating_matches_torch_autograd_through_selected_softmax():
+    """k < E: torch autograd through topk-selected softmax equals the oracle."""
+    rng = np.random.default_rng(6)
+    T, d, E, I, k = 13, 8, 7, 12, 3
+    X, W_r, Wg, Wu, Wd, dY = _rand_layer(rng, T, d, E, I, k)
+    Y, ctx = O.forward(X, W_r, None, Wg, Wu, Wd, k)
+    gr = O.backward(ctx, dY)
+    x = torch.tensor(X, requires_grad=True)
+    wr = torch.tensor(W_r, requires_grad=True)
+    logits = x @ wr
+    vals, idx = torch.topk(logits, k, dim=1)
+    assert np.array_equal(idx.numpy(), ctx["ids"])
+    g = torch.softmax(vals, dim=1)
+    y = torch.zeros(T, d, dtype=torch.float64)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            xt = x[t:t + 1]
+            o = (torch.nn.functional.silu(xt @ torch.tensor(Wg[e])) * (xt @ torch.tensor(Wu[e]))) @ torch.tensor(Wd[e])
+            y = y.index_add(0, torch.tensor([t]), g[t, j] * o)
+    (y * torch.tensor(dY)).sum().backward()
+    np.testing.assert_allclose(Y, y.detach().numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(gr["dX"], x.grad.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(gr["dW_r"], wr.grad.numpy(), rtol=1e-10, atol=1e-11)
+
+
+def test_sonicmoe_identity_router_grad_from_swiglu_backward():
+    """<dY, H W_down> == <dY W_down^T, H>: the fused form of the router gradient."""
+    rng = np.random.default_rng(7)
+    T, d, E, I, k = 40, 16, 5, 32, 2
+    X, W_r, Wg, Wu, Wd, dY = _rand_layer(rng, T, d, E, I, k)
+    _, ctx = O.forward(X, W_r, None, Wg, Wu, Wd, k)
+    gr = O.backward(ctx, dY)
+    ids = ctx["ids"]
+    for t in range(T):
+        for j in range(k):
+            e = ids[t, j]
+            a, b_ = X[t] @ Wg[e], X[t] @ Wu[e]
+            h = O.silu(a) * b_
+            fused = float((dY[t] @ Wd[e].T) @ h)
+            assert abs(fused - gr["dg"][t, j]) < 1e-12 * max(1.0, abs(fused))
+
+
+def test_token_path_equals_full_layer():
+    rng = np.random.default_rng(8)
+    T, d, E, I, k = 21, 8, 6, 16, 3
+    X, W_r, Wg, Wu, Wd, dY = _rand_layer(rng, T, d, E, I, k)
+    b = rng.standard_normal(E) * 0.2
+    for fl, nl in [(0, None), (2, 3)]:
+        Y, ctx = O.forward(X, W_r, b, Wg, Wu, Wd, k, first_local=fl, num_local=nl)
+        gr = O.backward(ctx, dY)
+        for t in [0, 5, 20]:
+            y, dx, dl, ids, g = O.token_forward_backward(t, X, W_r, b, Wg, Wu, Wd, k, dY, fl, nl)
+            np.testing.assert_allclose(y, Y[t], rtol=1e-13, atol=1e-13)
+            np.testing.assert_allclose(dx, gr["dX"][t], rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(dl, gr["dl"][t], rtol=1e-12, atol=1e-13)
+
+
+def test_local_expert_slices_sum_to_full_layer():
+    """Y, dX, dl and dW_r are linear in the experts' contributions: slices add up."""
+    rng = np.random.default_rng(9)
+    T, d, E, I, k = 30, 8, 6, 16, 3
+    X, W_r, Wg, Wu, Wd, dY = _rand_layer(rng, T, d, E, I, k)
+    Yf, cf = O.forward(X, W_r, None, Wg, Wu, Wd, k)
+    gf = O.backward(cf, dY)
+    Ys, dXs, dWrs = 0, 0, 0
+    for fl in range(0, E, 2):
+        Y, c = O.forward(X, W_r, None, Wg, Wu, Wd, k, first_local=fl, num_local=2)
+        g = O.backward(c, dY)
+        Ys, dXs, dWrs = Ys + Y, dXs + g["dX"], dWrs + g["dW_r"]
+        for e in range(fl, fl + 2):
+            np.testing.assert_allclose(g["dW_gate"][e], gf["dW_gate"][e], rtol=1e-12, atol=1e-13)
+    # the router term dl W_r^T is added once per slice; the dense part sums exactly
+    np.testing.assert_allclose(Ys, Yf, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(dWrs, gf["dW_r"], rtol=1e-11, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# routing: selection, ties, invariants of the table
+# --------------------------------------------------------------------------
+def test_topk_matches_torch_topk_on_distinct_values():
+    rng = np.random.default_rng(10)
+    l = rng.standard_normal((200, 64))
+    for k in [1, 2, 8, 64]:
+        ids = O.topk_ids(l, k)
+        _, ti = torch.topk(torch.tensor(l), k, dim=1, sorted=True)
+        assert np.array_equal(ids, ti.numpy())
+
+
+def test_topk_tie_break_lower_id_and_signed_zero_and_nan():
+    l = np.array([
+        [1.0, 1.0, 1.0, 1.0],          # all tied -> 0,1,2
+        [0.0, -0.0, 0.5, -0.0],        # -0 == +0 -> 2,0,1
+        [np.nan, -np.inf, 3.0, np.nan],  # NaN lowest, below -inf
+        [2.0, 5.0, 5.0, 1.0],          # tie at top -> 1,2,0
+    ])
+    ids = O.topk_ids(l, 3)
+    assert ids.tolist() == [[0, 1, 2], [2, 0, 1], [2, 1, 0], [1, 2, 0]]
+
+
+def test_gates_sum_to_one_and_equal_renormalised_full_softmax():
+    rng = np.random.default_rng(11)
+    l = rng.standard_normal((50, 16)) * 3
+    ids = O.topk_ids(l, 4)
+    g = O.gates(l, ids)
+    assert np.max(np.abs(g.sum(1) - 1)) < 1e-15
+    p = torch.softmax(torch.tensor(l), dim=1).numpy()
+    ps = np.take_along_axis(p, ids.astype(np.int64), 1)
+    np.testing.assert_allclose(g, ps / ps.sum(1, keepdims=True), rtol=1e-13)
+    assert np.all(np.diff(g, axis=1) <= 0)  # descending logits -> descending gates
+
+
+@pytest.mark.parametrize("T,E,k,fl,nl", [(300, 16, 4, 0, None), (257, 8, 2, 0, None),
+                                          (100, 12, 3, 4, 5), (64, 1, 1, 0, None)])
+def test_schedule_invariants_and_brute_force(T, E, k, fl, nl):
+    rng = np.random.default_rng(T + E)
+    l = rng.standard_normal((T, E))
+    l[:, 0] += 1.5  # a hot expert: some segments span several padded tiles
+    ids = O.topk_ids(l, k)
+    s = O.schedule(ids, E, fl, nl)
+    El = s["num_local"]
+    # exactly k distinct ids per token
+    assert all(len(set(r)) == k for r in ids.tolist())
+    loc = (ids >= fl) & (ids < fl + El)
+    assert s["counts"].sum() == loc.sum()
+    if nl is None:
+        assert s["counts"].sum() == T * k
+    assert np.array_equal(s["offsets"], np.concatenate([[0], np.cumsum(s["counts"])]))
+    pc = -(-s["counts"] // O.P_PAD) * O.P_PAD
+    assert np.array_equal(s["padded_offsets"], np.concatenate([[0], np.cumsum(pc)]))
+    # brute force: a stable sort of (expert, token) pairs gives perm
+    pairs = sorted((int(ids[t, j]) - fl, t) for t in range(T) for j in range(k) if loc[t, j])
+    assert [t for _, t in pairs] == s["perm"].tolist()
+    # slot_row points to the row holding that token inside its expert's padded segment
+    for t in range(T):
+        for j in range(k):
+            r = s["slot_row"][t, j]
+            if not loc[t, j]:
+                assert r == -1
+                continue
+            e = ids[t, j] - fl
+            assert s["padded_offsets"][e] <= r < s["padded_offsets"][e] + s["counts"][e]
+            pos = r - s["padded_offsets"][e]
+            assert s["perm"][s["offsets"][e] + pos] == t
+    # tokens strictly increasing inside each segment
+    for e in range(El):
+        seg = s["perm"][s["offsets"][e]:s["offsets"][e + 1]]
+        assert np.all(np.diff(seg) > 0)
+
+
+# --------------------------------------------------------------------------
+# MX (E4M3 + E8M0) quantiser
+# --------------------------------------------------------------------------
+def test_e4m3_decode_matches_torch_float8():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = O.e4m3_decode(codes)
+    both_nan = np.isnan(ref) & np.isnan(mine)
+    assert np.all(both_nan | (ref == mine))
+    assert O.e4m3_decode([0x7E])[0] == 448.0 and O.e4m3_decode([0x01])[0] == 2.0 ** -9
+
+
+def test_e4m3_encode_round_trips_and_matches_torch_rne():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    vals = O.e4m3_decode(codes)
+    back = O.e4m3_encode(vals)
+    assert np.array_equal(back, codes)
+    rng = np.random.default_rng(12)
+    x = np.concatenate([rng.standard_normal(20000) * s for s in (1e-3, 0.05, 1, 30, 120)])
+    x = x[np.abs(x) < 440]
+    # exact midpoints between neighbours exercise ties-to-even
+    mids = (vals[:-1] + vals[1:]) / 2
+    mids = mids[np.isfinite(mids) & (np.abs(mids) < 440)]
+    x = np.concatenate([x, mids, -mids])
+    ref = torch.tensor(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_encode(x), ref)
+
+
+def test_e4m3_saturates():
+    assert O.e4m3_encode([500.0, -1e9, 449.0])[0] == 0x7E
+    assert O.e4m3_encode([-1e9])[0] == 0xFE
+
+
+def test_mx_quantize_scale_rule_and_edges():
+    v = np.zeros((2, 64))
+    v[0, :32] = np.linspace(-3, 3, 32)          # amax 3 -> floor(log2 3) - 8 = -7
+    v[0, 32:] = 0.0                              # all-zero block
+    v[1, :32] = 2.0 ** 5                         # amax a power of two -> -3, value 256
+    v[1, 32:] = np.linspace(-1, 1, 32) * 2.0 ** -20
+    codes, sc = O.mx_quantize(v, axis=1)
+    assert sc.tolist() == [[127 - 7, 0], [127 - 3, 127 - 20 - 8]]
+    assert np.all(codes[0, 32:] == 0)
+    assert np.all(O.e4m3_decode(codes[1, :32]) == 256.0)
+    back = O.mx_dequantize(codes, sc, axis=1)
+    # E4M3 has 3 mantissa bits: relative error at most 2^-4 inside the normal range
+    nz = np.abs(v) > 2.0 ** -6 * 2.0 ** (sc.repeat(32, axis=1).astype(int) - 127)
+    assert np.all(np.abs(back - v)[nz] <= np.abs(v)[nz] * 2.0 ** -4 + 1e-30)
+    # amax * 2^-s lies in [256, 512): the largest element may saturate to 448
+    big = np.full((1, 32), 1.0); big[0, 0] = 1.99
+    c2, s2 = O.mx_quantize(big, axis=1)
+    assert s2[0, 0] == 127 - 8 and c2[0, 0] == 0x7E
+
+
+def test_mx_quantize_axis0_equals_transposed_axis1():
+    rng = np.random.default_rng(13)
+    v = rng.standard_normal((64, 96))
+    c0, s0 = O.mx_quantize(v, axis=0)
+    c1, s1 = O.mx_quantize(v.T, axis=1)
+    assert np.array_equal(c0, c1.T) and np.array_equal(s0, s1.T)
