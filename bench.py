@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""MoE layer forward+backward throughput on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload dsv3] [--impl moe|reference]
+
+One step = one forward + one backward of the whole layer (router GEMM, top-k
+gating, histogram/scan, stable scatter + dispatch, grouped gate/up GEMM with
+SwiGLU, grouped down GEMM with the gate multiply, combine; reverse-combine,
+dgrad with the SwiGLU backward and router-gate gradient, router backward,
+dgrad gate/up, reverse-dispatch, wgrad) over one batch of synthetic tokens.
+
+* value: tokens/s over all ranks, inputs resident in HBM, CUDA-event timed on
+  the launch stream, max over ranks.  The expert weights (>= 22 GB) exceed
+  L2 and are streamed every step, so no explicit L2 flush is needed.
+* e2e: the same steps through the C ABI from pinned HOST buffers: X and dY
+  copied in, Y and dX copied out, inside the timed region.
+* roofline: the kernel with the largest share of the timed region, its
+  algorithmic bytes per launch / its CUDA-event duration, against the
+  measured HBM copy bandwidth.
+* cpu_baseline: the fp64 CPU oracle on a bounded sample of the workload.
+* --impl reference: times that oracle alone, as the comparison arm.
+
+Multi-GPU (torchrun, N > 1): N independent replicas of the single-GPU layer
+(weak scaling, no data-path collective); only the timing is reduced (max).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from mixture_experts_layer_27_b200 import inputs as IN  # noqa: E402
+
+METRIC = "MoE layer fwd+bwd tokens/s and TFLOP/s (% of B200 BF16/FP8 tensor peak)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def workload_config(w: IN.Workload) -> dict:
+    routing = "zipf(1.2) bias, hottest ~10x mean" if w.zipf else "near-uniform (W_r ~ N(0, 0.02^2))"
+    return {"workload": f"{w.name}: T={w.T} d={w.d} E={w.E} top_k={w.k} I={w.I} bf16, {routing}",
+            "T": w.T, "d": w.d, "E": w.E, "top_k": w.k, "I": w.I, "precision": "mxfp8" if w.mxfp8 else "bf16",
+            "seed": w.seed, "l2": "no flush: expert weights (%.1f GB) exceed the 126 MB L2 and stream every step"
+            % (3 * w.El * w.d * w.I * 2 / 1e9), "parallelism": "replicas"}
+
+
+# ----------------------------------------------------------------------------
+# algorithmic bytes per launch of each kernel (minimum HBM traffic of its job)
+# rows = T*k routed assignments; weights of all local experts; bf16 = 2 bytes
+# ----------------------------------------------------------------------------
+def algorithmic_bytes(w: IN.Workload) -> dict:
+    T, d, E, I, k, El = w.T, w.d, w.E, w.I, w.k, w.El
+    rows = T * k
+    W1 = El * d * I * 2  # one expert weight matrix family (gate, up or down), bytes
+    return {
+        "router_logits": T * d * 2 + d * E * 2 + T * E * 4,
+        "topk_gating": T * E * 4 + rows * 8,
+        "dispatch": T * d * 2 + rows * d * 2,
+        "gemm_gateup_swiglu": 2 * W1 + rows * d * 2 + 3 * rows * I * 2,
+        "gemm_down_combw": W1 + rows * I * 2 + rows * d * 2,
+        "combine": rows * d * 2 + T * d * 2,
+        "reverse_combine": T * d * 2 + rows * d * 2,
+        "gemm_dgrad_down_swiglu_bwd": W1 + rows * d * 2 + 2 * rows * I * 2 + 3 * rows * I * 2,
+        "router_wgrad": rows * d * 2 + d * E * 4,
+        "gemm_dgrad_gateup": 2 * W1 + 2 * rows * I * 2 + rows * d * 2,
+        "reverse_dispatch": rows * d * 2 + T * d * 2 + E * d * 2,
+        "gemm_wgrad_gateup": rows * d * 2 + 2 * rows * I * 2 + 2 * W1,
+        "gemm_wgrad_down": rows * I * 2 + rows * d * 2 + W1,
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: torch.device):
+        try:
+            self.dev = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            self.dev = str(device.index or 0)
+        self.proc = None
+        self.path = os.path.join("/tmp", f"moe_clocks_{os.getpid()}_{device.index or 0}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.dev)], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 9:
+                    rows.append(p)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = max((num(r[2]) for r in rows if num(r[2]) is not None), default=None)
+        loaded = [r for r in rows if (num(r[3]) or 0) > 250] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i in range(4) if r[5 + i].lower().startswith("active")})
+        sm_load = [num(r[1]) for r in loaded if num(r[1]) is not None]
+        return {"sm_mhz": statistics.median(sm_load) if sm_load else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max((num(r[3]) or 0) for r in rows)}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle on a bounded sample (the baseline and the reference arm)
+# ----------------------------------------------------------------------------
+def oracle_sample(w: IN.Workload, x_cpu: dict, m: int) -> float:
+    """Seconds for the fp64 oracle: routing of all T tokens + fwd/bwd of experts [0, m)."""
+    import numpy as np
+    import oracle as O
+
+    def f64(t):
+        return t.float().numpy().astype(np.float64)
+
+    X, Wr, dY = f64(x_cpu["X"]), f64(x_cpu["W_r"]), f64(x_cpu["dY"])
+    b = None if x_cpu["bias"] is None else f64(x_cpu["bias"])
+    Wg, Wu, Wd = (f64(x_cpu[n][:m]) for n in ("W_gate", "W_up", "W_down"))
+    t0 = time.perf_counter()
+    _, ctx = O.forward(X, Wr, b, Wg, Wu, Wd, w.k, first_local=0, num_local=m)
+    O.backward(ctx, dY)
+    return time.perf_counter() - t0
+
+
+def cpu_inputs(w: IN.Workload, m: int) -> dict:
+    """Host copies of the inputs the sample needs (CPU generator; same distributions)."""
+    x = {"X": IN._normal((w.T, w.d), 1.0, IN._seed(w.seed, w.name, "X"), "cpu"),
+         "W_r": IN._normal((w.d, w.E), 0.02, IN._seed(w.seed, w.name, "W_r"), "cpu"),
+         "dY": IN._normal((w.T, w.d), 1.0, IN._seed(w.seed, w.name, "dY"), "cpu")}
+    for n in ("W_gate", "W_up", "W_down"):
+        x[n] = torch.stack([IN.expert_weights(w, n, e, "cpu") for e in range(m)])
+    x["bias"] = IN.zipf_bias(w, x["X"], x["W_r"]) if w.zipf else None
+    return x
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(w: IN.Workload, m1: int = 4, m2: int = 8) -> dict:
+    x = cpu_inputs(w, m2)
+    t1 = oracle_sample(w, x, m1)
+    t2 = oracle_sample(w, x, m2)
+    per_expert = max(t2 - t1, 0.0) / (m2 - m1)
+    t_full = t1 + per_expert * (w.El - m1)
+    return {"value": w.T / t_full, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"fp64 numpy oracle, all {w.T} tokens routed, fwd+bwd of {m1} and {m2} of {w.El} experts "
+                       f"({t1:.1f} s, {t2:.1f} s); time extrapolated linearly to {w.El} experts = {t_full:.1f} s "
+                       "per full fwd+bwd")}
+
+
+# ----------------------------------------------------------------------------
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_reference(args, w: IN.Workload, world: int, rank: int):
+    if rank != 0:
+        return
+    x = cpu_inputs(w, 4)
+    for _ in range(args.warmup):
+        oracle_sample(w, x, 1)
+    ts = [oracle_sample(w, x, 2) for _ in range(args.steps)]
+    # each step: routing of all tokens + 2 experts' fwd+bwd; the per-expert cost is
+    # measured once more with 4 experts and the step time extrapolated to all experts
+    t4 = oracle_sample(w, x, 4)
+    t2 = statistics.median(ts)
+    t_full = t2 + max(t4 - t2, 0.0) / 2 * (w.El - 2)
+    value = w.T / t_full
+    cores = blas_threads()
+    sample = (f"fp64 numpy oracle per step: all {w.T} tokens routed + fwd/bwd of 2 of {w.El} experts "
+              f"(median {t2:.2f} s over {args.steps} steps); per-expert cost from a 4-expert run, "
+              f"extrapolated to {w.El} experts = {t_full:.1f} s per layer fwd+bwd")
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_full * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(w),
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
+    from mixture_experts_layer_27_b200 import binding as B
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_kind = load_peaks()
+    x = IN.make_inputs(w, device=dev)
+    layer = B.MoELayer(w.T, w.d, w.E, w.I, w.k, device=dev)
+    Y = torch.empty(w.T, w.d, dtype=torch.bfloat16, device=dev)
+    grads = dict(dX=torch.empty(w.T, w.d, dtype=torch.bfloat16, device=dev),
+                 dW_gate=torch.empty_like(x["W_gate"]), dW_up=torch.empty_like(x["W_up"]),
+                 dW_down=torch.empty_like(x["W_down"]),
+                 dW_r=torch.empty(w.d, w.E, dtype=torch.float32, device=dev))
+    stream = torch.cuda.current_stream(dev)
+
+    def step(X, dY, Yout, g):
+        layer.forward(X, x["W_r"], x["bias"], x["W_gate"], x["W_up"], x["W_down"], Y=Yout)
+        layer.backward(X, x["W_r"], x["W_gate"], x["W_up"], x["W_down"], dY, out=g)
+
+    for _ in range(args.warmup):
+        step(x["X"], x["dY"], Y, grads)
+    torch.cuda.synchronize()
+    st = layer.error()
+    if st != B.MOE_OK:
+        raise RuntimeError("device error during warm-up: " + B.status_string(st))
+
+    # ---------------- device-resident timed region ----------------
+    clocks = ClockSampler(dev)
+    B.moe_profile_read()  # drop anything recorded so far
+    B.moe_profile_enable(True)
+    launches0 = B.moe_kernel_launches()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(x["X"], x["dY"], Y, grads)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    launches = B.moe_kernel_launches() - launches0
+    B.moe_profile_enable(False)
+    prof = B.moe_profile_read()
+    st = layer.error()
+    if st != B.MOE_OK:
+        raise RuntimeError("device error in the timed region: " + B.status_string(st))
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+
+    # ---------------- end to end through host buffers ----------------
+    hX = torch.empty(w.T, w.d, dtype=torch.bfloat16, pin_memory=True)
+    hdY = torch.empty_like(hX, pin_memory=True)
+    hY = torch.empty_like(hX, pin_memory=True)
+    hdX = torch.empty_like(hX, pin_memory=True)
+    hX.copy_(x["X"].cpu())
+    hdY.copy_(x["dY"].cpu())
+    dX_in = torch.empty_like(x["X"])
+    dY_in = torch.empty_like(x["dY"])
+
+    def e2e_step():
+        dX_in.copy_(hX, non_blocking=True)
+        dY_in.copy_(hdY, non_blocking=True)
+        step(dX_in, dY_in, Y, grads)
+        hY.copy_(Y, non_blocking=True)
+        hdX.copy_(grads["dX"], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e3.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    t_e2e = max_over_ranks(e2.elapsed_time(e3) / 1e3, world)
+    st = layer.error()
+    if st != B.MOE_OK:
+        raise RuntimeError("device error in the e2e region: " + B.status_string(st))
+
+    if rank != 0:
+        return
+    tokens = w.T * args.steps * world
+    flops = w.model_flops() * args.steps * world
+    value = tokens / t
+    tflops = flops / t / 1e12
+    per_gpu_tflops = tflops / world
+    algo = algorithmic_bytes(w)
+    kern = {}
+    for name, (ms, n) in sorted(prof.items(), key=lambda kv: -kv[1][0]):
+        avg = ms / n
+        e = {"ms_per_launch": avg, "launches": n, "share": ms / (t * 1e3)}
+        if name in algo:
+            e["algorithmic_GB"] = algo[name] / 1e9
+            e["achieved_GBs"] = algo[name] / (avg / 1e3) / 1e9
+        kern[name] = e
+    top = max(kern.items(), key=lambda kv: kv[1]["share"])[0]
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    ach = kern[top].get("achieved_GBs")
+    roof = {"kernel": top, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+            "frac": (ach / hbm) if ach else None, "traffic": None,
+            "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+            if peak_kind == "measured" else "fallback 6.65 TB/s"}
+    bf16 = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, random-init weights)",
+        "config": workload_config(w),
+        "tflops": tflops, "pct_of_bf16_peak": 100.0 * per_gpu_tflops / bf16,
+        "peak_note": f"bf16 sustained {bf16} TFLOP/s ({peak_kind}); model FLOPs 18 d I T k + 6 T d E per step",
+        "roofline": roof,
+        "e2e": {"value": tokens / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": 2 * w.T * w.d * 2,
+                "d2h_bytes_per_step": 2 * w.T * w.d * 2,
+                "note": "X, dY copied in from pinned host memory; Y, dX copied back; weights and their gradients "
+                        "stay in HBM"},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "kernels": kern,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="dsv3", choices=sorted(IN.WORKLOADS))
+    ap.add_argument("--impl", default="moe", choices=["moe", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = IN.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, w, world, rank)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_moe(args, w, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,154 @@
+/*
+ * moe.h -- C ABI of libmoe.so: a deterministic mixture-of-experts layer
+ * (forward and backward) on one B200 GPU.
+ *
+ * The operation is the MoE layer described by "Cursor open-sources
+ * Mixture-of-Kittens (MoK): a deterministic MoE training megakernel"
+ * (page 1, sections "MoE layer as the bottleneck" and "Three design decisions
+ * that matter"): tokens are routed to their top-k experts, dispatched into an
+ * expert-contiguous layout, run through SwiGLU experts as expert-grouped
+ * GEMMs, and combined back with their gate weights; the backward mirrors it
+ * (reverse-combine, grouped dgrad/wgrad, reverse-dispatch), with the router
+ * weight gradient taken inside the SwiGLU backward.  The pages print no
+ * formula; the arithmetic is the plain top-k softmax-gated SwiGLU mixture:
+ *
+ *   l = X W_r + b,  S_t = top-k(l_t) (descending, ties -> lower expert id)
+ *   g_t,e = softmax over the k selected logits
+ *   H = silu(X_t W_gate[e]) * (X_t W_up[e]),   Y_t = sum_{e in S_t} g_t,e H W_down[e]
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *   never allocates, frees or keeps them after the call returns.
+ * - bf16 tensors are row-major, 16-byte aligned, and passed as void*.
+ * - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is only
+ *   enqueued: no entry point except moe_get_error synchronises the stream or
+ *   reads device memory on the host.
+ * - Argument errors are returned synchronously and nothing is enqueued.
+ * - Device-side errors (a bounded wait that ran out, non-finite router logits)
+ *   set a status word inside `ctx`; moe_get_error reads it.  moe_fwd clears it.
+ * - Results are bit-reproducible: fixed reduction orders, no float atomics.
+ *
+ * Limits: 1 <= E <= 512; 1 <= top_k <= min(E, 16); d and I multiples of 256;
+ * 0 <= T and T * top_k < 2^31; 0 <= first_local_expert,
+ * first_local_expert + num_local_experts <= E.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,          /* null pointer, bad shape, misaligned tensor */
+  MOE_ERR_UNSUPPORTED = 2,          /* shape or mode outside the limits above */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 3,  /* ctx or workspace smaller than the *_size() call says */
+  MOE_ERR_CUDA = 4,                 /* a CUDA runtime call failed (launch, attribute, ...) */
+  MOE_ERR_DEVICE_TIMEOUT = 5,       /* a bounded device-side wait ran out */
+  MOE_ERR_NONFINITE = 6             /* a router logit was NaN or +-Inf */
+} moe_status;
+
+typedef enum moe_precision {
+  MOE_BF16 = 0,  /* bf16 operands, fp32 accumulation */
+  MOE_MXFP8 = 1  /* E4M3 operands with one E8M0 scale per 32 along each GEMM's contraction dim */
+} moe_precision;
+
+/* Layer shape.  Experts [first_local_expert, first_local_expert + num_local_experts)
+ * are computed here (num_local_experts = 0 means all E).  Assignments to other
+ * experts belong to another rank: they add nothing to Y or to the expert part of dX. */
+typedef struct moe_shape {
+  int64_t T;       /* tokens */
+  int32_t d;       /* model (hidden) dimension */
+  int32_t E;       /* experts the router scores (router width) */
+  int32_t I;       /* expert SwiGLU intermediate dimension */
+  int32_t top_k;   /* experts per token */
+  int32_t prec;    /* moe_precision */
+  int32_t first_local_expert;
+  int32_t num_local_experts;
+} moe_shape;
+
+/* Bytes of the saved-for-backward context that moe_fwd writes and moe_bwd reads
+ * (routing table, dispatched tokens, SwiGLU pre-activations, status word).
+ * Depends on the shape only.  0 for an invalid shape. */
+size_t moe_ctx_size(const moe_shape* shape);
+
+/* Bytes of scratch workspace moe_fwd / moe_bwd need (worst case over routings:
+ * padded rows <= T*k + 127*num_local).  0 for an invalid shape. */
+size_t moe_workspace_size(const moe_shape* shape);
+
+/* Forward.
+ *   X       [T, d]   bf16   tokens
+ *   W_r     [d, E]   bf16   router weight
+ *   bias    [E]      fp32   router bias added before selection and gating; may be NULL
+ *   W_gate  [El, d, I] bf16, W_up [El, d, I] bf16, W_down [El, I, d] bf16  (El = local experts)
+ *   Y       [T, d]   bf16   output (written)
+ *   ctx     ctx_bytes        saved for moe_bwd (written)
+ *   ws      ws_bytes         scratch
+ * Implements: router GEMM, top-k + softmax gating, histogram + prefix sums,
+ * stable scatter/dispatch (page 1, "Three design decisions", pull dispatch),
+ * grouped gate/up GEMM + SwiGLU, grouped down GEMM with the gate multiply,
+ * combine (push combine). */
+moe_status moe_fwd(const moe_shape* shape, const void* X, const void* W_r, const float* bias,
+                   const void* W_gate, const void* W_up, const void* W_down, void* Y,
+                   void* ctx, size_t ctx_bytes, void* ws, size_t ws_bytes, void* stream);
+
+/* Backward of the last moe_fwd that wrote `ctx` (same shape, X, W_r, weights).
+ *   dY      [T, d]   bf16   upstream gradient
+ *   dX      [T, d]   bf16   written
+ *   dW_gate, dW_up [El, d, I] bf16, dW_down [El, I, d] bf16   written (not accumulated)
+ *   dW_r    [d, E]   fp32   written
+ * Implements the mirror of the forward (page 1, "Three design decisions":
+ * pull reverse-combine, push reverse-dispatch), grouped dgrad and wgrad with
+ * fixed-order reductions, and the router-weight gradient computed inside the
+ * SwiGLU backward from <dY W_down^T, H> ("SonicMoE-style", same page). */
+moe_status moe_bwd(const moe_shape* shape, const void* X, const void* W_r, const void* W_gate,
+                   const void* W_up, const void* W_down, const void* dY, void* ctx, size_t ctx_bytes,
+                   void* dX, void* dW_gate, void* dW_up, void* dW_down, float* dW_r,
+                   void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, returns the device status word held in `ctx`
+ * (MOE_OK if no device error since the last moe_fwd), and clears it.
+ * Returns MOE_ERR_CUDA if the synchronisation itself failed. */
+moe_status moe_get_error(void* ctx, void* stream);
+
+/* Test hook: copies the routing table of the last moe_fwd into caller buffers
+ * (device pointers; any may be NULL to skip), local experts only:
+ *   ids [T, k] int32, gates [T, k] fp32, counts [El] int32, offsets [El+1] int32,
+ *   padded_offsets [El+1] int32 (segments padded to 128 rows), perm [sum counts] int32
+ *   (token of each row, ascending token id inside an expert), slot_row [T, k] int32
+ *   (padded row of each assignment, -1 for a non-local expert). */
+moe_status moe_debug_routing(const moe_shape* shape, const void* ctx, int32_t* ids, float* gates,
+                             int32_t* counts, int32_t* offsets, int32_t* padded_offsets,
+                             int32_t* perm, int32_t* slot_row, void* stream);
+
+/* Test hook: copies the fp32 router logits [T, E] (bias included) that the last
+ * moe_fwd computed in `ws` into `logits` (device pointer). */
+moe_status moe_debug_logits(const moe_shape* shape, const void* ws, float* logits, void* stream);
+
+/* Benchmark support (no counterpart on the pages).  When enabled, every
+ * kernel launch of the library is bracketed by two CUDA events recorded on the
+ * launch stream.  moe_profile_read synchronises the device, writes per kernel
+ * id the summed milliseconds and launch counts recorded since the last read
+ * (arrays of max_kernels entries; either may be NULL), clears the records and
+ * returns the number of kernel ids (or -1 if the synchronisation failed).
+ * moe_kernel_name gives a kernel id's name; moe_kernel_launches counts every
+ * kernel this library has launched in the process.  Not thread-safe against
+ * concurrent enabling. */
+moe_status moe_profile_enable(int on);
+int moe_profile_read(int max_kernels, double* total_ms, int* launches);
+const char* moe_kernel_name(int kernel_id);
+unsigned long long moe_kernel_launches(void);
+
+/* Static string naming a status code. */
+const char* moe_status_string(moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,226 @@
+"""Thin ctypes binding of libmoe.so: the C entry points under the same names.
+
+Only argument marshalling happens here (tensor -> device pointer, stream ->
+handle).  Every step of the layer runs in the library's CUDA kernels; there
+is no Python or CPU fallback: if the library is missing, loading it raises.
+PyTorch is used for device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from .build import LIB
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_WORKSPACE_TOO_SMALL = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_DEVICE_TIMEOUT = 5
+MOE_ERR_NONFINITE = 6
+MOE_BF16 = 0
+MOE_MXFP8 = 1
+
+
+class moe_shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("prec", ctypes.c_int32), ("first_local_expert", ctypes.c_int32),
+                ("num_local_experts", ctypes.c_int32)]
+
+
+def make_shape(T, d, E, I, top_k, prec=MOE_BF16, first_local_expert=0, num_local_experts=0) -> moe_shape:
+    return moe_shape(T, d, E, I, top_k, prec, first_local_expert, num_local_experts)
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+        self.status = status
+
+
+_lib = None
+_P = ctypes.c_void_p
+_S = ctypes.POINTER(moe_shape)
+
+_SIGS = {
+    "moe_ctx_size": (ctypes.c_size_t, [_S]),
+    "moe_workspace_size": (ctypes.c_size_t, [_S]),
+    "moe_fwd": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, ctypes.c_size_t, _P]),
+    "moe_bwd": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, _P, _P, _P, _P,
+                               ctypes.c_size_t, _P]),
+    "moe_get_error": (ctypes.c_int, [_P, _P]),
+    "moe_debug_routing": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_debug_logits": (ctypes.c_int, [_S, _P, _P, _P]),
+    "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
+    "moe_profile_read": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
+    "moe_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
+    "moe_kernel_launches": (ctypes.c_ulonglong, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libmoe.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB):
+            raise RuntimeError(f"{LIB} is missing: build it with `python -m mixture_experts_layer_27_b200.build`")
+        h = ctypes.CDLL(LIB)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(h, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = h
+    return _lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+def status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+def moe_ctx_size(shape: moe_shape) -> int:
+    return int(lib().moe_ctx_size(ctypes.byref(shape)))
+
+
+def moe_workspace_size(shape: moe_shape) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(shape)))
+
+
+def moe_fwd(shape, X, W_r, bias, W_gate, W_up, W_down, Y, ctx, ws, stream=None, ctx_bytes=None, ws_bytes=None):
+    return int(lib().moe_fwd(ctypes.byref(shape), _ptr(X), _ptr(W_r), _ptr(bias), _ptr(W_gate), _ptr(W_up),
+                             _ptr(W_down), _ptr(Y), _ptr(ctx), ctx_bytes if ctx_bytes is not None else _nbytes(ctx),
+                             _ptr(ws), ws_bytes if ws_bytes is not None else _nbytes(ws), _stream(stream)))
+
+
+def moe_bwd(shape, X, W_r, W_gate, W_up, W_down, dY, ctx, dX, dW_gate, dW_up, dW_down, dW_r, ws, stream=None,
+            ctx_bytes=None, ws_bytes=None):
+    return int(lib().moe_bwd(ctypes.byref(shape), _ptr(X), _ptr(W_r), _ptr(W_gate), _ptr(W_up), _ptr(W_down),
+                             _ptr(dY), _ptr(ctx), ctx_bytes if ctx_bytes is not None else _nbytes(ctx), _ptr(dX),
+                             _ptr(dW_gate), _ptr(dW_up), _ptr(dW_down), _ptr(dW_r), _ptr(ws),
+                             ws_bytes if ws_bytes is not None else _nbytes(ws), _stream(stream)))
+
+
+def moe_get_error(ctx, stream=None) -> int:
+    return int(lib().moe_get_error(_ptr(ctx), _stream(stream)))
+
+
+def moe_debug_routing(shape, ctx, ids=None, gates=None, counts=None, offsets=None, padded_offsets=None, perm=None,
+                      slot_row=None, stream=None) -> int:
+    return int(lib().moe_debug_routing(ctypes.byref(shape), _ptr(ctx), _ptr(ids), _ptr(gates), _ptr(counts),
+                                       _ptr(offsets), _ptr(padded_offsets), _ptr(perm), _ptr(slot_row),
+                                       _stream(stream)))
+
+
+def moe_debug_logits(shape, ws, logits, stream=None) -> int:
+    return int(lib().moe_debug_logits(ctypes.byref(shape), _ptr(ws), _ptr(logits), _stream(stream)))
+
+
+def moe_profile_enable(on: bool) -> int:
+    return int(lib().moe_profile_enable(1 if on else 0))
+
+
+def moe_profile_read(max_kernels: int = 64) -> dict:
+    """{kernel name: (total ms, launches)} since the last read (synchronises the device)."""
+    ms = (ctypes.c_double * max_kernels)()
+    n = (ctypes.c_int * max_kernels)()
+    k = int(lib().moe_profile_read(max_kernels, ms, n))
+    if k < 0:
+        raise MoeError(MOE_ERR_CUDA, "moe_profile_read")
+    return {moe_kernel_name(i): (ms[i], n[i]) for i in range(k) if n[i] > 0}
+
+
+def moe_kernel_name(kernel_id: int) -> str:
+    return lib().moe_kernel_name(int(kernel_id)).decode()
+
+
+def moe_kernel_launches() -> int:
+    return int(lib().moe_kernel_launches())
+
+
+def check(status: int, what: str = "moe"):
+    if status != MOE_OK:
+        raise MoeError(status, what)
+
+
+class MoELayer:
+    """Convenience owner of ctx / workspace buffers (allocated by torch) for one shape."""
+
+    def __init__(self, T, d, E, I, top_k, prec=MOE_BF16, first_local_expert=0, num_local_experts=0,
+                 device="cuda"):
+        import torch
+        self.shape = make_shape(T, d, E, I, top_k, prec, first_local_expert, num_local_experts)
+        nc, nw = moe_ctx_size(self.shape), moe_workspace_size(self.shape)
+        if nc == 0 or nw == 0:
+            raise MoeError(MOE_ERR_UNSUPPORTED, "shape")
+        self.ctx = torch.empty(nc, dtype=torch.uint8, device=device)
+        self.ws = torch.empty(nw, dtype=torch.uint8, device=device)
+        self.T, self.d, self.E, self.I, self.k = T, d, E, I, top_k
+        self.El = num_local_experts or (E - first_local_expert)
+
+    def forward(self, X, W_r, bias, W_gate, W_up, W_down, Y=None, stream=None):
+        import torch
+        if Y is None:
+            Y = torch.empty(self.T, self.d, dtype=torch.bfloat16, device=X.device)
+        check(moe_fwd(self.shape, X, W_r, bias, W_gate, W_up, W_down, Y, self.ctx, self.ws, stream), "moe_fwd")
+        return Y
+
+    def backward(self, X, W_r, W_gate, W_up, W_down, dY, out=None, stream=None):
+        import torch
+        if out is None:
+            dev = X.device
+            out = dict(dX=torch.empty(self.T, self.d, dtype=torch.bfloat16, device=dev),
+                       dW_gate=torch.empty(self.El, self.d, self.I, dtype=torch.bfloat16, device=dev),
+                       dW_up=torch.empty(self.El, self.d, self.I, dtype=torch.bfloat16, device=dev),
+                       dW_down=torch.empty(self.El, self.I, self.d, dtype=torch.bfloat16, device=dev),
+                       dW_r=torch.empty(self.d, self.E, dtype=torch.float32, device=dev))
+        check(moe_bwd(self.shape, X, W_r, W_gate, W_up, W_down, dY, self.ctx, out["dX"], out["dW_gate"],
+                      out["dW_up"], out["dW_down"], out["dW_r"], self.ws, stream), "moe_bwd")
+        return out
+
+    def routing(self):
+        import torch
+        T, k, El, dev = self.T, self.k, self.El, self.ctx.device
+        r = dict(ids=torch.empty(T, k, dtype=torch.int32, device=dev),
+                 gates=torch.empty(T, k, dtype=torch.float32, device=dev),
+                 counts=torch.empty(El, dtype=torch.int32, device=dev),
+                 offsets=torch.empty(El + 1, dtype=torch.int32, device=dev),
+                 padded_offsets=torch.empty(El + 1, dtype=torch.int32, device=dev),
+                 perm=torch.empty(max(T * k, 1), dtype=torch.int32, device=dev),
+                 slot_row=torch.empty(T, k, dtype=torch.int32, device=dev))
+        check(moe_debug_routing(self.shape, self.ctx, r["ids"], r["gates"], r["counts"], r["offsets"],
+                                r["padded_offsets"], r["perm"], r["slot_row"]), "moe_debug_routing")
+        torch.cuda.synchronize()
+        n = int(r["offsets"][-1].item())
+        r["perm"] = r["perm"][:n]
+        return r
+
+    def logits(self):
+        import torch
+        out = torch.empty(self.T, self.E, dtype=torch.float32, device=self.ws.device)
+        check(moe_debug_logits(self.shape, self.ws, out), "moe_debug_logits")
+        return out
+
+    def error(self, stream=None) -> int:
+        return moe_get_error(self.ctx, stream)

@@ -1,0 +1,438 @@
+// Expert-grouped GEMMs of the MoE layer on sm_100a tensor cores.
+//
+// One persistent, warp-specialised kernel template serves all six GEMMs of
+// the forward and backward ("expert-grouped GEMM", page 1 of the MoK pages,
+// "Three design decisions that matter", bullet 2):
+//
+//   warp 0      one thread issues TMA tile loads into a 4-stage smem ring
+//   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
+//   warps 2..5  epilogue: tcgen05.ld from TMEM, fused math, global stores
+//
+// The output tile is 128 x 256 (fp32 in TMEM), K advances 64 at a time
+// (one 128-byte swizzle atom of bf16).  Two accumulators let the epilogue of
+// tile i overlap the MMAs of tile i+1.  Every output tile is produced by one
+// CTA with one fixed K order, so results are bit-reproducible (no split-K,
+// no atomics).  Tiles are listed on the device from the padded expert
+// offsets, so the host never needs the routing result.
+#include <cstdio>
+
+#include "moe_internal.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+template <int KIND>
+struct Traits;
+template <> struct Traits<G_GATEUP>       { static constexpr bool A_MN = false, B_MN = true; };
+template <> struct Traits<G_DOWN>         { static constexpr bool A_MN = false, B_MN = true; };
+template <> struct Traits<G_DGRAD_DOWN>   { static constexpr bool A_MN = false, B_MN = false; };
+template <> struct Traits<G_DGRAD_GATEUP> { static constexpr bool A_MN = false, B_MN = false; };
+template <> struct Traits<G_WGRAD_GATEUP> { static constexpr bool A_MN = true, B_MN = true; };
+template <> struct Traits<G_WGRAD_DOWN>   { static constexpr bool A_MN = true, B_MN = true; };
+
+struct Tile {
+  int el;   // local expert
+  int m0;   // first output row (padded token row, or weight row for wgrad)
+  int n0;   // first output column
+  int nt;   // n-tile index
+  int kb0;  // first 64-wide K block (wgrad: first padded row / 64)
+  int nk;   // number of K blocks
+};
+
+template <int KIND>
+__device__ __forceinline__ int ntiles_n(const GemmParams& p) {
+  if (KIND == G_GATEUP) return p.I / 128;  // 128 gate + 128 up columns per tile
+  if (KIND == G_DOWN || KIND == G_DGRAD_GATEUP || KIND == G_WGRAD_DOWN) return p.d / 256;
+  if (KIND == G_DGRAD_DOWN) return p.I / 256;
+  return 2 * p.I / 256;  // G_WGRAD_GATEUP: gate n-tiles then up n-tiles
+}
+template <int KIND>
+__device__ __forceinline__ int mtiles_w(const GemmParams& p) {
+  return KIND == G_WGRAD_GATEUP ? p.d / 128 : p.I / 128;
+}
+
+// Local expert whose padded segment [poff[e], poff[e+1]) holds row R.
+__device__ __forceinline__ int expert_of_row(const int* poff, int El, int R) {
+  int lo = 0, hi = El - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(poff + mid) <= R) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int KIND>
+__device__ __forceinline__ int num_tiles(const GemmParams& p) {
+  if (KIND <= G_DGRAD_GATEUP) return (__ldg(p.hdr + HDR_ROWS_P) / 128) * ntiles_n<KIND>(p);
+  return p.El * mtiles_w<KIND>(p) * ntiles_n<KIND>(p);
+}
+
+template <int KIND>
+__device__ __forceinline__ Tile decode(const GemmParams& p, int t) {
+  Tile tl;
+  const int NT = ntiles_n<KIND>(p);
+  if constexpr (KIND <= G_DGRAD_GATEUP) {
+    // Tiles of expert e are [NT*poff[e]/128, NT*poff[e+1]/128), n-tile major so that
+    // the m-tiles of a hot expert sharing one weight tile run back to back.
+    const int el = expert_of_row(p.poff, p.El, (t / NT) * 128);
+    const int p0 = __ldg(p.poff + el), p1 = __ldg(p.poff + el + 1);
+    const int mte = (p1 - p0) / 128;
+    const int local = t - NT * (p0 / 128);
+    const int nt = local / mte, mi = local - nt * mte;
+    tl.el = el;
+    tl.m0 = p0 + mi * 128;
+    tl.nt = nt;
+    tl.n0 = nt * (KIND == G_GATEUP ? 128 : 256);
+    tl.kb0 = 0;
+    tl.nk = (KIND == G_GATEUP || KIND == G_DGRAD_DOWN) ? p.d / 64 : (KIND == G_DOWN ? p.I / 64 : 2 * p.I / 64);
+  } else {
+    const int tpe = mtiles_w<KIND>(p) * NT;
+    const int el = t / tpe, local = t - el * tpe;
+    const int mt = local / NT, nt = local - mt * NT;
+    const int p0 = __ldg(p.poff + el), p1 = __ldg(p.poff + el + 1);
+    tl.el = el;
+    tl.m0 = mt * 128;
+    tl.nt = nt;
+    tl.n0 = nt * 256;
+    tl.kb0 = p0 / 64;
+    tl.nk = (p1 - p0) / 64;
+  }
+  return tl;
+}
+
+// Issue the TMA loads of K block kb of tile tl into one stage.
+template <int KIND>
+__device__ __forceinline__ void load_stage(const GemmParams& p, const Tile& tl, int kb, uint8_t* sA, uint8_t* sB,
+                                           uint64_t* bar, uint64_t pol_act, uint64_t pol_w) {
+  const int k0 = kb * 64;
+  if constexpr (KIND == G_GATEUP) {
+    tma_load_2d(sA, &p.ta0, bar, k0, tl.m0, pol_act);  // X_perm [rows, d] (K-major)
+    const int krow = tl.el * p.d + k0;                 // W_gate / W_up as [El*d, I] (N contiguous)
+    tma_load_2d(sB, &p.tb0, bar, tl.n0, krow, pol_w);
+    tma_load_2d(sB + 8192, &p.tb0, bar, tl.n0 + 64, krow, pol_w);
+    tma_load_2d(sB + 16384, &p.tb1, bar, tl.n0, krow, pol_w);
+    tma_load_2d(sB + 24576, &p.tb1, bar, tl.n0 + 64, krow, pol_w);
+  } else if constexpr (KIND == G_DOWN) {
+    tma_load_2d(sA, &p.ta0, bar, k0, tl.m0, pol_act);  // H [rows, I]
+    const int krow = tl.el * p.I + k0;                 // W_down as [El*I, d]
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tma_load_2d(sB + j * 8192, &p.tb0, bar, tl.n0 + 64 * j, krow, pol_w);
+  } else if constexpr (KIND == G_DGRAD_DOWN) {
+    tma_load_2d(sA, &p.ta0, bar, k0, tl.m0, pol_act);                  // dY_perm [rows, d]
+    tma_load_2d(sB, &p.tb0, bar, k0, tl.el * p.I + tl.n0, pol_w);      // W_down rows = n (I), cols = k (d)
+  } else if constexpr (KIND == G_DGRAD_GATEUP) {
+    if (k0 < p.I) {
+      tma_load_2d(sA, &p.ta0, bar, k0, tl.m0, pol_act);                // dA [rows, I]
+      tma_load_2d(sB, &p.tb0, bar, k0, tl.el * p.d + tl.n0, pol_w);    // W_gate rows = n (d), cols = k (I)
+    } else {
+      tma_load_2d(sA, &p.ta1, bar, k0 - p.I, tl.m0, pol_act);          // dB
+      tma_load_2d(sB, &p.tb1, bar, k0 - p.I, tl.el * p.d + tl.n0, pol_w);  // W_up
+    }
+  } else if constexpr (KIND == G_WGRAD_GATEUP) {
+    const int row = (tl.kb0 + kb) * 64;                                // contraction over padded rows
+    tma_load_2d(sA, &p.ta0, bar, tl.m0, row, pol_act);                 // X_perm, M = d (contiguous)
+    tma_load_2d(sA + 8192, &p.ta0, bar, tl.m0 + 64, row, pol_act);
+    const int NTg = p.I / 256;
+    const CUtensorMap* mb = tl.nt < NTg ? &p.tb0 : &p.tb1;             // dA for gate, dB for up
+    const int nb = (tl.nt < NTg ? tl.nt : tl.nt - NTg) * 256;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tma_load_2d(sB + j * 8192, mb, bar, nb + 64 * j, row, pol_act);
+  } else {  // G_WGRAD_DOWN
+    const int row = (tl.kb0 + kb) * 64;
+    tma_load_2d(sA, &p.ta0, bar, tl.m0, row, pol_act);                 // Hg, M = I (contiguous)
+    tma_load_2d(sA + 8192, &p.ta0, bar, tl.m0 + 64, row, pol_act);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tma_load_2d(sB + j * 8192, &p.tb0, bar, tl.n0 + 64 * j, row, pol_act);  // dY_perm
+  }
+}
+
+__device__ __forceinline__ float sigmoidf_(float a) { return 1.0f / (1.0f + expf(-a)); }
+
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 u;
+    u.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
+    u.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+    u.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+    u.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+    d4[q] = u;
+  }
+}
+__device__ __forceinline__ void load_row32(const __nv_bfloat16* src, float (&v)[32]) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = s4[q];
+    float2 f;
+    f = unpack_bf16(u.x); v[8 * q + 0] = f.x; v[8 * q + 1] = f.y;
+    f = unpack_bf16(u.y); v[8 * q + 2] = f.x; v[8 * q + 3] = f.y;
+    f = unpack_bf16(u.z); v[8 * q + 4] = f.x; v[8 * q + 5] = f.y;
+    f = unpack_bf16(u.w); v[8 * q + 6] = f.x; v[8 * q + 7] = f.y;
+  }
+}
+
+// Epilogue for one output row (this thread's TMEM lane) of tile tl.
+template <int KIND>
+__device__ __forceinline__ void epilogue_row(const GemmParams& p, const Tile& tl, int row, uint32_t taddr) {
+  if constexpr (KIND == G_GATEUP) {
+    const size_t R = static_cast<size_t>(tl.m0 + row);
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float a[32], b[32], h[32];
+      tmem_ld32(taddr + c * 32, a);        // gate columns
+      tmem_ld32(taddr + 128 + c * 32, b);  // up columns
+#pragma unroll
+      for (int i = 0; i < 32; ++i) h[i] = a[i] * sigmoidf_(a[i]) * b[i];  // SwiGLU
+      const size_t off = R * p.I + tl.n0 + c * 32;
+      store_row32(p.out0 + off, a);
+      store_row32(p.out1 + off, b);
+      store_row32(p.out2 + off, h);
+    }
+  } else if constexpr (KIND == G_DOWN) {
+    const size_t R = static_cast<size_t>(tl.m0 + row);
+    const float g = p.row_gate[R];  // combine weight, 0 on pad rows
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      float o[32];
+      tmem_ld32(taddr + c * 32, o);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] *= g;
+      store_row32(p.out0 + R * p.d + tl.n0 + c * 32, o);
+    }
+  } else if constexpr (KIND == G_DGRAD_DOWN) {
+    // dH' = dY W_down^T arrives in TMEM.  With H = silu(A) B rebuilt from the saved A, B:
+    //   dg partial = sum_i dH'_i H_i          (router-gate gradient, "SonicMoE-style")
+    //   dH = g dH',  dA = dH B silu'(A),  dB = dH silu(A),  Hg = g H (wgrad operand)
+    const size_t R = static_cast<size_t>(tl.m0 + row);
+    const float g = p.row_gate[R];
+    float dg = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      float dh[32], a[32], b[32];
+      tmem_ld32(taddr + c * 32, dh);
+      const size_t off = R * p.I + tl.n0 + c * 32;
+      load_row32(p.in0 + off, a);
+      load_row32(p.in1 + off, b);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float s = sigmoidf_(a[i]);
+        const float sl = a[i] * s;
+        const float hh = sl * b[i];
+        dg = fmaf(dh[i], hh, dg);
+        const float dhg = g * dh[i];
+        const float da = dhg * b[i] * (s * (1.0f + a[i] * (1.0f - s)));
+        const float db = dhg * sl;
+        a[i] = da;
+        b[i] = db;
+        dh[i] = g * hh;
+      }
+      store_row32(p.out0 + off, a);   // dA
+      store_row32(p.out1 + off, b);   // dB
+      store_row32(p.out2 + off, dh);  // Hg
+    }
+    p.outf[R * (p.I / 256) + tl.nt] = dg;
+  } else if constexpr (KIND == G_DGRAD_GATEUP) {
+    const size_t R = static_cast<size_t>(tl.m0 + row);
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      float v[32];
+      tmem_ld32(taddr + c * 32, v);
+      store_row32(p.out0 + R * p.d + tl.n0 + c * 32, v);
+    }
+  } else {
+    __nv_bfloat16* out;
+    size_t base;
+    if constexpr (KIND == G_WGRAD_GATEUP) {
+      const int NTg = p.I / 256;
+      out = tl.nt < NTg ? p.out0 : p.out1;
+      const int nb = (tl.nt < NTg ? tl.nt : tl.nt - NTg) * 256;
+      base = static_cast<size_t>(tl.el) * p.d * p.I + static_cast<size_t>(tl.m0 + row) * p.I + nb;
+    } else {
+      out = p.out0;
+      base = static_cast<size_t>(tl.el) * p.I * p.d + static_cast<size_t>(tl.m0 + row) * p.d + tl.n0;
+    }
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      float v[32];
+      if (tl.nk > 0) {
+        tmem_ld32(taddr + c * 32, v);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;  // expert without tokens: zero gradient
+      }
+      store_row32(out + base + c * 32, v);
+    }
+  }
+}
+
+// Wait bounded by time only (used while draining after an error).
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > MOE_SPIN_CYCLES) return;
+  }
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + GEMM_STAGES * GEMM_STAGE_BYTES);
+  uint64_t* empty = full + GEMM_STAGES;
+  uint64_t* tfull = empty + GEMM_STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < GEMM_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&p.ta0);
+    prefetch_tmap(&p.ta1);
+    prefetch_tmap(&p.tb0);
+    prefetch_tmap(&p.tb1);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const int ntiles = num_tiles<KIND>(p);
+  constexpr uint32_t IDESC = idesc_bf16(GEMM_BM, GEMM_BN, Traits<KIND>::A_MN, Traits<KIND>::B_MN);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      const uint64_t pol_act = policy_evict_last();
+      const uint64_t pol_w = policy_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_parity[GEMM_STAGES];
+      for (int s = 0; s < GEMM_STAGES; ++s) last_parity[s] = -1;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const Tile tl = decode<KIND>(p, t);
+        for (int kb = 0; kb < tl.nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, p.status)) { ok = false; break; }
+          uint8_t* sA = smem + stage * GEMM_STAGE_BYTES;
+          uint8_t* sB = sA + GEMM_A_BYTES;
+          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(GEMM_STAGE_BYTES));
+          load_stage<KIND>(p, tl, kb, sA, sB, &full[stage], pol_act, pol_w);
+          last_parity[stage] = static_cast<int>(phase);
+          if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {  // let copies already in flight land before the CTA's smem goes away
+        for (int s = 0; s < GEMM_STAGES; ++s)
+          if (last_parity[s] >= 0) mbar_wait_drain(&full[s], static_cast<uint32_t>(last_parity[s]));
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
+        const Tile tl = decode<KIND>(p, t);
+        const int acc = it & 1;
+        const uint32_t accp = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], accp ^ 1, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dtm = tbase + acc * GEMM_BN;
+        for (int kb = 0; kb < tl.nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * GEMM_STAGE_BYTES);
+          const uint32_t b0 = a0 + static_cast<uint32_t>(GEMM_A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // 4 x K16 per 64-wide block
+            const uint64_t ad = Traits<KIND>::A_MN ? sdesc_sw128(a0 + kk * 2048, 8192, 1024)
+                                                   : sdesc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t bd = Traits<KIND>::B_MN ? sdesc_sw128(b0 + kk * 2048, 8192, 1024)
+                                                   : sdesc_sw128(b0 + kk * 32, 16, 1024);
+            umma_bf16(dtm, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+          if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        if (tl.nk > 0) umma_commit(&tfull[acc]);
+        else mbar_arrive(&tfull[acc]);
+      }
+      umma_commit(drain);  // all MMAs issued by this thread are complete once this lands
+      mbar_wait_drain(drain, 0);
+    }
+  } else {
+    // ---------------- epilogue warps 2..5 ----------------
+    const int quarter = warp & 3;  // TMEM lanes this warp may access: 32*quarter ..
+    const int row = quarter * 32 + lane;
+    int it = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+      const Tile tl = decode<KIND>(p, t);
+      const int acc = it & 1;
+      const uint32_t accp = (it >> 1) & 1;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&tfull[acc], accp, p.status) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t taddr = tbase + (static_cast<uint32_t>(quarter * 32) << 16) + acc * GEMM_BN;
+      epilogue_row<KIND>(p, tl, row, taddr);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+template <int KIND>
+static cudaError_t launch_kind(const GemmParams& p, int grid, cudaStream_t st) {
+  static bool configured = false;
+  if (!configured) {
+    const cudaError_t e = cudaFuncSetAttribute(k_moe_gemm<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(GEMM_SMEM_BYTES));
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  k_moe_gemm<KIND><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream_t st) {
+  switch (kind) {
+    case G_GATEUP: return launch_kind<G_GATEUP>(p, grid, st);
+    case G_DOWN: return launch_kind<G_DOWN>(p, grid, st);
+    case G_DGRAD_DOWN: return launch_kind<G_DGRAD_DOWN>(p, grid, st);
+    case G_DGRAD_GATEUP: return launch_kind<G_DGRAD_GATEUP>(p, grid, st);
+    case G_WGRAD_GATEUP: return launch_kind<G_WGRAD_GATEUP>(p, grid, st);
+    case G_WGRAD_DOWN: return launch_kind<G_WGRAD_DOWN>(p, grid, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

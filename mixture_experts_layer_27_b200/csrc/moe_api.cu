@@ -1,0 +1,500 @@
+// Host side of libmoe.so: argument validation, the ctx / workspace layout,
+// TMA tensor-map encoding and the launch sequences of moe_fwd / moe_bwd.
+// Every step of the layer runs in this library's kernels; the host only
+// enqueues work and never waits on the device (except in moe_get_error).
+#include <cstdint>
+#include <cstring>
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool make_layout(const moe_shape& s, Layout* L) {
+  if (s.T < 0 || s.d <= 0 || s.E <= 0 || s.I <= 0 || s.top_k <= 0) return false;
+  if (s.E > kMaxE || s.top_k > kMaxK || s.top_k > s.E) return false;
+  if (s.d % 256 || s.I % 256) return false;
+  const int El = s.num_local_experts == 0 ? s.E - s.first_local_expert : s.num_local_experts;
+  if (s.first_local_expert < 0 || El <= 0 || s.first_local_expert + El > s.E) return false;
+  if (s.T * static_cast<int64_t>(s.top_k) >= (int64_t(1) << 31)) return false;
+  L->T = s.T;
+  L->d = s.d;
+  L->E = s.E;
+  L->I = s.I;
+  L->k = s.top_k;
+  L->first = s.first_local_expert;
+  L->El = El;
+  const int64_t A = s.T * s.top_k;
+  L->RP = static_cast<int64_t>(align_up(static_cast<size_t>(A + int64_t(kPad - 1) * El), kPad));
+  if (L->RP < kPad) L->RP = kPad;
+  if (L->RP * static_cast<int64_t>(s.d > s.I ? s.d : s.I) >= (int64_t(1) << 40)) return false;
+  L->nblk = static_cast<int>((s.T + kTokensPerBlock - 1) / kTokensPerBlock);
+  if (L->nblk < 1) L->nblk = 1;
+
+  const size_t RP = static_cast<size_t>(L->RP), T = static_cast<size_t>(s.T), k = s.top_k;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, 256);
+    return at;
+  };
+  L->hdr = take(HDR_WORDS * 4);
+  L->ids = take(T * k * 4);
+  L->gates = take(T * k * 4);
+  L->counts = take(static_cast<size_t>(s.E) * 4);
+  L->offsets = take(static_cast<size_t>(s.E + 1) * 4);
+  L->poff = take(static_cast<size_t>(El + 1) * 4);
+  L->perm_tok = take(T * k * 4);
+  L->perm_asg = take(T * k * 4);
+  L->slot_row = take(T * k * 4);
+  L->row_asg = take(RP * 4);
+  L->row_gate = take(RP * 4);
+  L->xperm = take(RP * s.d * 2);
+  L->abuf = take(RP * s.I * 2);
+  L->bbuf = take(RP * s.I * 2);
+  L->ctx_bytes = o;
+
+  o = 0;
+  L->hist = take(static_cast<size_t>(L->nblk) * s.E * 4);
+  L->logits = take(T * s.E * 4);
+  L->hbuf = take(RP * s.I * 2);
+  L->obuf = take(RP * s.d * 2);
+  L->dyperm = take(RP * s.d * 2);
+  L->dabuf = take(RP * s.I * 2);
+  L->dbbuf = take(RP * s.I * 2);
+  L->hgbuf = take(RP * s.I * 2);
+  L->dgpart = take(RP * (s.I / 256) * 4);
+  L->dlasg = take(T * k * 4);
+  L->wrt = take(static_cast<size_t>(s.E) * s.d * 2);
+  L->dxperm = take(RP * s.d * 2);
+  L->ws_bytes = o;
+  return true;
+}
+
+Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
+  auto C = [&](size_t off) { return static_cast<char*>(ctx) + off; };
+  auto W = [&](size_t off) { return static_cast<char*>(ws) + off; };
+  Ctx c;
+  c.hdr = reinterpret_cast<int*>(C(L.hdr));
+  c.ids = reinterpret_cast<int*>(C(L.ids));
+  c.gates = reinterpret_cast<float*>(C(L.gates));
+  c.counts = reinterpret_cast<int*>(C(L.counts));
+  c.offsets = reinterpret_cast<int*>(C(L.offsets));
+  c.poff = reinterpret_cast<int*>(C(L.poff));
+  c.perm_tok = reinterpret_cast<int*>(C(L.perm_tok));
+  c.perm_asg = reinterpret_cast<int*>(C(L.perm_asg));
+  c.slot_row = reinterpret_cast<int*>(C(L.slot_row));
+  c.row_asg = reinterpret_cast<int*>(C(L.row_asg));
+  c.row_gate = reinterpret_cast<float*>(C(L.row_gate));
+  c.xperm = reinterpret_cast<__nv_bfloat16*>(C(L.xperm));
+  c.abuf = reinterpret_cast<__nv_bfloat16*>(C(L.abuf));
+  c.bbuf = reinterpret_cast<__nv_bfloat16*>(C(L.bbuf));
+  if (ws) {
+    c.hist = reinterpret_cast<int*>(W(L.hist));
+    c.logits = reinterpret_cast<float*>(W(L.logits));
+    c.hbuf = reinterpret_cast<__nv_bfloat16*>(W(L.hbuf));
+    c.obuf = reinterpret_cast<__nv_bfloat16*>(W(L.obuf));
+    c.dyperm = reinterpret_cast<__nv_bfloat16*>(W(L.dyperm));
+    c.dabuf = reinterpret_cast<__nv_bfloat16*>(W(L.dabuf));
+    c.dbbuf = reinterpret_cast<__nv_bfloat16*>(W(L.dbbuf));
+    c.hgbuf = reinterpret_cast<__nv_bfloat16*>(W(L.hgbuf));
+    c.dgpart = reinterpret_cast<float*>(W(L.dgpart));
+    c.dlasg = reinterpret_cast<float*>(W(L.dlasg));
+    c.wrt = reinterpret_cast<__nv_bfloat16*>(W(L.wrt));
+    c.dxperm = reinterpret_cast<__nv_bfloat16*>(W(L.dxperm));
+  }
+  return c;
+}
+
+// ---------------------------------------------------------------------------
+// TMA tensor maps (driver entry point fetched through the runtime, so the
+// library does not link libcuda directly)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [outer, inner] (inner contiguous, row pitch in elements),
+// box {box_inner, box_outer}, 128-byte swizzle, zero fill out of bounds.
+static bool tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch_elems,
+                    uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch_elems * 2};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess)
+      n = 148;
+  }
+  return n;
+}
+
+// ---------------------------------------------------------------------------
+// optional per-kernel timing: each launch bracketed by CUDA events on its stream
+// ---------------------------------------------------------------------------
+enum KernelId {
+  K_ROUTER_LOGITS, K_TOPK, K_SCAN, K_SCATTER, K_DISPATCH, K_GEMM_GATEUP, K_GEMM_DOWN, K_COMBINE,
+  K_REV_COMBINE, K_GEMM_DGRAD_DOWN, K_ROUTER_BWD, K_DWR, K_TRANSPOSE_WR, K_GEMM_DGRAD_GATEUP, K_REV_DISPATCH,
+  K_GEMM_WGRAD_GATEUP, K_GEMM_WGRAD_DOWN, K_NUM
+};
+static const char* kKernelNames[K_NUM] = {
+    "router_logits", "topk_gating", "hist_scan", "stable_scatter", "dispatch", "gemm_gateup_swiglu",
+    "gemm_down_combw", "combine", "reverse_combine", "gemm_dgrad_down_swiglu_bwd", "router_bwd", "router_wgrad",
+    "transpose_wr", "gemm_dgrad_gateup", "reverse_dispatch", "gemm_wgrad_gateup", "gemm_wgrad_down"};
+
+struct ProfRec {
+  int kid;
+  cudaEvent_t a, b;
+};
+static std::mutex g_mu;
+static bool g_prof_on = false;
+static std::vector<ProfRec> g_prof;
+static std::vector<cudaEvent_t> g_pool;
+static std::atomic<unsigned long long> g_launches{0};
+
+static cudaEvent_t pool_event() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Launches one kernel through `fn`, counting it and (when enabled) timing it.
+template <class F>
+static cudaError_t timed(int kid, cudaStream_t st, F fn) {
+  cudaEvent_t a = nullptr, b = nullptr;
+  if (g_prof_on) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    a = pool_event();
+    b = pool_event();
+    if (a && b) cudaEventRecord(a, st);
+  }
+  const cudaError_t e = fn();
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (g_prof_on && a && b) {
+    cudaEventRecord(b, st);
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_prof.push_back({kid, a, b});
+  }
+  return e;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static GemmParams base_params(const Layout& L, const Ctx& c, int* status) {
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.hdr = c.hdr;
+  p.poff = c.poff;
+  p.row_gate = c.row_gate;
+  p.El = L.El;
+  p.d = L.d;
+  p.I = L.I;
+  p.status = status;
+  return p;
+}
+
+#define MOE_TRY(x)                                   \
+  do {                                               \
+    if ((x) != cudaSuccess) return MOE_ERR_CUDA;     \
+  } while (0)
+#define MOE_TMAP(x)                                  \
+  do {                                               \
+    if (!(x)) return MOE_ERR_CUDA;                   \
+  } while (0)
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_ctx_size(const moe_shape* s) {
+  Layout L;
+  if (!s || !make_layout(*s, &L)) return 0;
+  return L.ctx_bytes;
+}
+
+size_t moe_workspace_size(const moe_shape* s) {
+  Layout L;
+  if (!s || !make_layout(*s, &L)) return 0;
+  return L.ws_bytes;
+}
+
+const char* moe_status_string(moe_status st) {
+  switch (st) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or mode";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "ctx or workspace too small";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_NONFINITE: return "non-finite router logit";
+  }
+  return "unknown status";
+}
+
+static moe_status check_shape(const moe_shape* s, Layout* L) {
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->d <= 0 || s->E <= 0 || s->I <= 0 || s->top_k <= 0 || s->first_local_expert < 0 ||
+      s->num_local_experts < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (s->prec != MOE_BF16 && s->prec != MOE_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (s->prec == MOE_MXFP8) return MOE_ERR_UNSUPPORTED;
+  if (!make_layout(*s, L)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status moe_fwd(const moe_shape* s, const void* X, const void* W_r, const float* bias, const void* W_gate,
+                   const void* W_up, const void* W_down, void* Y, void* ctx, size_t ctx_bytes, void* ws,
+                   size_t ws_bytes, void* stream) {
+  Layout L;
+  const moe_status cs = check_shape(s, &L);
+  if (cs != MOE_OK) return cs;
+  const bool tok = s->T > 0;  // with no tokens, X and Y may be empty (NULL)
+  if ((tok && (!X || !Y)) || !W_r || !W_gate || !W_up || !W_down || !ctx || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W_r) || !aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_down) ||
+      !aligned16(Y) || !aligned16(ctx) || !aligned16(ws) || (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+    return MOE_ERR_INVALID_ARG;
+  if (ctx_bytes < L.ctx_bytes || ws_bytes < L.ws_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ctx c = make_ctx(L, ctx, ws);
+  MOE_TRY(cudaMemsetAsync(c.hdr, 0, HDR_WORDS * 4, st));  // clears the status word
+  if (L.T == 0) return MOE_OK;
+
+  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
+  // 1-2. router GEMM, top-k gating, per-block histograms
+  MOE_TRY(timed(K_ROUTER_LOGITS, st, [&] { return launch_router_logits(L, Xb, static_cast<const __nv_bfloat16*>(W_r), bias, c.logits, st); }));
+  MOE_TRY(timed(K_TOPK, st, [&] { return launch_topk(L, c, st); }));
+  // 3. counts, prefix sums, padded offsets
+  MOE_TRY(timed(K_SCAN, st, [&] { return launch_scan(L, c, st); }));
+  // 4. stable scatter + dispatch
+  MOE_TRY(cudaMemsetAsync(c.row_asg, 0xFF, static_cast<size_t>(L.RP) * 4, st));
+  MOE_TRY(cudaMemsetAsync(c.row_gate, 0, static_cast<size_t>(L.RP) * 4, st));
+  MOE_TRY(timed(K_SCATTER, st, [&] { return launch_scatter(L, c, st); }));
+  MOE_TRY(timed(K_DISPATCH, st, [&] { return launch_gather_rows(L, c, Xb, c.xperm, st); }));
+
+  const int grid = num_sms();
+  int* status = c.hdr + HDR_STATUS;
+  const uint64_t RP = static_cast<uint64_t>(L.RP);
+  // 5. grouped gate/up GEMM with the SwiGLU epilogue
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, c.xperm, L.d, RP, L.d, 64, 128));
+    MOE_TMAP(tmap_2d(&p.tb0, W_gate, L.I, static_cast<uint64_t>(L.El) * L.d, L.I, 64, 64));
+    MOE_TMAP(tmap_2d(&p.tb1, W_up, L.I, static_cast<uint64_t>(L.El) * L.d, L.I, 64, 64));
+    p.ta1 = p.ta0;
+    p.out0 = c.abuf;
+    p.out1 = c.bbuf;
+    p.out2 = c.hbuf;
+    MOE_TRY(timed(K_GEMM_GATEUP, st, [&] { return launch_gemm(G_GATEUP, p, grid, st); }));
+  }
+  // 6. grouped down GEMM with the combine-weight epilogue
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, c.hbuf, L.I, RP, L.I, 64, 128));
+    MOE_TMAP(tmap_2d(&p.tb0, W_down, L.d, static_cast<uint64_t>(L.El) * L.I, L.d, 64, 64));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.out0 = c.obuf;
+    MOE_TRY(timed(K_GEMM_DOWN, st, [&] { return launch_gemm(G_DOWN, p, grid, st); }));
+  }
+  // 7. combine
+  MOE_TRY(timed(K_COMBINE, st, [&] { return launch_combine(L, c, c.obuf, static_cast<__nv_bfloat16*>(Y), st); }));
+  return MOE_OK;
+}
+
+moe_status moe_bwd(const moe_shape* s, const void* X, const void* W_r, const void* W_gate, const void* W_up,
+                   const void* W_down, const void* dY, void* ctx, size_t ctx_bytes, void* dX, void* dW_gate,
+                   void* dW_up, void* dW_down, float* dW_r, void* ws, size_t ws_bytes, void* stream) {
+  Layout L;
+  const moe_status cs = check_shape(s, &L);
+  if (cs != MOE_OK) return cs;
+  const bool tok = s->T > 0;  // with no tokens, X, dY and dX may be empty (NULL)
+  if ((tok && (!X || !dY || !dX)) || !W_r || !W_gate || !W_up || !W_down || !ctx || !dW_gate || !dW_up ||
+      !dW_down || !dW_r || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W_r) || !aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_down) ||
+      !aligned16(dY) || !aligned16(ctx) || !aligned16(dX) || !aligned16(dW_gate) || !aligned16(dW_up) ||
+      !aligned16(dW_down) || !aligned16(dW_r) || !aligned16(ws))
+    return MOE_ERR_INVALID_ARG;
+  if (ctx_bytes < L.ctx_bytes || ws_bytes < L.ws_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ctx c = make_ctx(L, ctx, ws);
+  if (L.T == 0) {  // no tokens: every gradient is zero
+    const size_t wexp = static_cast<size_t>(L.El) * L.d * L.I * 2;
+    MOE_TRY(cudaMemsetAsync(dW_gate, 0, wexp, st));
+    MOE_TRY(cudaMemsetAsync(dW_up, 0, wexp, st));
+    MOE_TRY(cudaMemsetAsync(dW_down, 0, wexp, st));
+    MOE_TRY(cudaMemsetAsync(dW_r, 0, static_cast<size_t>(L.d) * L.E * 4, st));
+    return MOE_OK;
+  }
+  const int grid = num_sms();
+  int* status = c.hdr + HDR_STATUS;
+  const uint64_t RP = static_cast<uint64_t>(L.RP);
+  const uint64_t El = static_cast<uint64_t>(L.El);
+
+  // 8. reverse-combine: dY into the expert-contiguous layout
+  MOE_TRY(timed(K_REV_COMBINE, st, [&] { return launch_gather_rows(L, c, static_cast<const __nv_bfloat16*>(dY), c.dyperm, st); }));
+  // 9. dgrad of the down projection + SwiGLU backward + router-gate gradient partials
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, c.dyperm, L.d, RP, L.d, 64, 128));
+    MOE_TMAP(tmap_2d(&p.tb0, W_down, L.d, El * L.I, L.d, 64, 256));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.in0 = c.abuf;
+    p.in1 = c.bbuf;
+    p.out0 = c.dabuf;
+    p.out1 = c.dbbuf;
+    p.out2 = c.hgbuf;
+    p.outf = c.dgpart;
+    MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm(G_DGRAD_DOWN, p, grid, st); }));
+  }
+  // 10. router backward: dl, then dW_r (sparse X^T dl); W_r^T for the dX router term
+  MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st); }));
+  MOE_TRY(timed(K_DWR, st, [&] { return launch_dwr(L, c, static_cast<const __nv_bfloat16*>(X), dW_r, st); }));
+  MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] { return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st); }));
+  // 11. dgrad of gate/up
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, c.dabuf, L.I, RP, L.I, 64, 128));
+    MOE_TMAP(tmap_2d(&p.ta1, c.dbbuf, L.I, RP, L.I, 64, 128));
+    MOE_TMAP(tmap_2d(&p.tb0, W_gate, L.I, El * L.d, L.I, 64, 256));
+    MOE_TMAP(tmap_2d(&p.tb1, W_up, L.I, El * L.d, L.I, 64, 256));
+    p.out0 = c.dxperm;
+    MOE_TRY(timed(K_GEMM_DGRAD_GATEUP, st, [&] { return launch_gemm(G_DGRAD_GATEUP, p, grid, st); }));
+  }
+  // 12. reverse-dispatch (+ router term dl W_r^T)
+  MOE_TRY(timed(K_REV_DISPATCH, st, [&] { return launch_rev_dispatch(L, c, static_cast<__nv_bfloat16*>(dX), st); }));
+  // 13. wgrad: gate/up then down
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, c.xperm, L.d, RP, L.d, 64, 64));
+    MOE_TMAP(tmap_2d(&p.tb0, c.dabuf, L.I, RP, L.I, 64, 64));
+    MOE_TMAP(tmap_2d(&p.tb1, c.dbbuf, L.I, RP, L.I, 64, 64));
+    p.ta1 = p.ta0;
+    p.out0 = static_cast<__nv_bfloat16*>(dW_gate);
+    p.out1 = static_cast<__nv_bfloat16*>(dW_up);
+    MOE_TRY(timed(K_GEMM_WGRAD_GATEUP, st, [&] { return launch_gemm(G_WGRAD_GATEUP, p, grid, st); }));
+  }
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, c.hgbuf, L.I, RP, L.I, 64, 64));
+    MOE_TMAP(tmap_2d(&p.tb0, c.dyperm, L.d, RP, L.d, 64, 64));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.out0 = static_cast<__nv_bfloat16*>(dW_down);
+    MOE_TRY(timed(K_GEMM_WGRAD_DOWN, st, [&] { return launch_gemm(G_WGRAD_DOWN, p, grid, st); }));
+  }
+  return MOE_OK;
+}
+
+moe_status moe_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_prof_on = on != 0;
+  return MOE_OK;
+}
+
+int moe_profile_read(int max_kernels, double* total_ms, int* launches) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (int i = 0; i < max_kernels && i < K_NUM; ++i) {
+    if (total_ms) total_ms[i] = 0.0;
+    if (launches) launches[i] = 0;
+  }
+  for (const ProfRec& r : g_prof) {
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess && r.kid < max_kernels) {
+      if (total_ms) total_ms[r.kid] += ms;
+      if (launches) launches[r.kid] += 1;
+    }
+    g_pool.push_back(r.a);
+    g_pool.push_back(r.b);
+  }
+  g_prof.clear();
+  return K_NUM;
+}
+
+const char* moe_kernel_name(int kernel_id) {
+  return (kernel_id >= 0 && kernel_id < K_NUM) ? kKernelNames[kernel_id] : "";
+}
+
+unsigned long long moe_kernel_launches(void) { return g_launches.load(); }
+
+moe_status moe_get_error(void* ctx, void* stream) {
+  if (!ctx) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  int code = 0;
+  if (cudaMemcpy(&code, static_cast<char*>(ctx) + HDR_STATUS * 4, 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int zero = 0;
+  if (code != 0 && cudaMemcpy(static_cast<char*>(ctx) + HDR_STATUS * 4, &zero, 4, cudaMemcpyHostToDevice) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return static_cast<moe_status>(code);
+}
+
+moe_status moe_debug_routing(const moe_shape* s, const void* ctx, int32_t* ids, float* gates, int32_t* counts,
+                             int32_t* offsets, int32_t* padded_offsets, int32_t* perm, int32_t* slot_row,
+                             void* stream) {
+  Layout L;
+  const moe_status cs = check_shape(s, &L);
+  if (cs != MOE_OK) return cs;
+  if (!ctx) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ctx c = make_ctx(L, const_cast<void*>(ctx), nullptr);
+  const size_t tk = static_cast<size_t>(L.T) * L.k * 4;
+  if (L.T == 0) return MOE_OK;
+  if (ids) MOE_TRY(cudaMemcpyAsync(ids, c.ids, tk, cudaMemcpyDeviceToDevice, st));
+  if (gates) MOE_TRY(cudaMemcpyAsync(gates, c.gates, tk, cudaMemcpyDeviceToDevice, st));
+  if (slot_row) MOE_TRY(cudaMemcpyAsync(slot_row, c.slot_row, tk, cudaMemcpyDeviceToDevice, st));
+  if (counts || offsets || padded_offsets || perm)
+    MOE_TRY(launch_export_routing(L, c, counts, offsets, padded_offsets, perm, st));
+  return MOE_OK;
+}
+
+moe_status moe_debug_logits(const moe_shape* s, const void* ws, float* logits, void* stream) {
+  Layout L;
+  const moe_status cs = check_shape(s, &L);
+  if (cs != MOE_OK) return cs;
+  if (!ws || !logits) return MOE_ERR_INVALID_ARG;
+  if (L.T == 0) return MOE_OK;
+  MOE_TRY(cudaMemcpyAsync(logits, static_cast<const char*>(ws) + L.logits, static_cast<size_t>(L.T) * L.E * 4,
+                          cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+}  // extern "C"

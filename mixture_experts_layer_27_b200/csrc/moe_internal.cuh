@@ -1,0 +1,107 @@
+// Internal declarations shared by the translation units of libmoe.so:
+// the context / workspace layout, the GEMM parameter block and the kernel
+// launchers.  Nothing here is part of the public ABI.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "moe.h"
+
+namespace moe {
+
+constexpr int kPad = 128;          // rows of an expert segment are padded to a multiple of this
+constexpr int kTokensPerBlock = 16;  // tokens per block of the top-k / scatter kernels
+constexpr int kMaxE = 512;
+constexpr int kMaxK = 16;
+
+// ctx header words (int32)
+enum HdrWord { HDR_STATUS = 0, HDR_ROWS_P = 1, HDR_MTILES = 2, HDR_WORDS = 64 };
+
+// Byte offsets of every region of ctx (saved for backward) and ws (scratch).
+struct Layout {
+  // shape
+  int64_t T;
+  int d, E, I, k, first, El;
+  int64_t RP;     // padded-row capacity: worst case of sum_e ceil(count_e / 128) * 128
+  int nblk;       // blocks of the top-k / scatter kernels
+  // ctx
+  size_t hdr, ids, gates, counts, offsets, poff, perm_tok, perm_asg, slot_row, row_asg, row_gate, xperm, abuf,
+      bbuf, ctx_bytes;
+  // ws
+  size_t hist, logits, hbuf, obuf, dyperm, dabuf, dbbuf, hgbuf, dgpart, dlasg, wrt, dxperm, ws_bytes;
+};
+
+// Returns false for shapes outside the supported limits.
+bool make_layout(const moe_shape& s, Layout* L);
+
+// ---------------------------------------------------------------------------
+// grouped GEMM (tcgen05 + TMA), see gemm.cu
+// ---------------------------------------------------------------------------
+enum GemmKind {
+  G_GATEUP = 0,         // [A|B] = X_perm . [W_gate | W_up], SwiGLU epilogue -> A, B, H
+  G_DOWN = 1,           // O' = g * (H . W_down)
+  G_DGRAD_DOWN = 2,     // dH' = dY_perm . W_down^T, SwiGLU-backward + router-grad epilogue
+  G_DGRAD_GATEUP = 3,   // dX_perm = dA . W_gate^T + dB . W_up^T
+  G_WGRAD_GATEUP = 4,   // dW_gate = X_perm^T dA, dW_up = X_perm^T dB (per expert)
+  G_WGRAD_DOWN = 5,     // dW_down = Hg^T dY_perm (per expert)
+};
+
+struct GemmParams {
+  CUtensorMap ta0, ta1, tb0, tb1;
+  const int* hdr;             // ctx header (rows_p)
+  const int* poff;            // padded offsets [El+1]
+  const float* row_gate;      // [RP]
+  const __nv_bfloat16* in0;   // epilogue inputs
+  const __nv_bfloat16* in1;
+  __nv_bfloat16* out0;        // epilogue outputs
+  __nv_bfloat16* out1;
+  __nv_bfloat16* out2;
+  float* outf;
+  int El, d, I;
+  int* status;
+};
+
+constexpr int GEMM_BM = 128, GEMM_BN = 256, GEMM_BK = 64, GEMM_STAGES = 4;
+constexpr int GEMM_THREADS = 192;
+constexpr size_t GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;
+constexpr size_t GEMM_B_BYTES = GEMM_BN * GEMM_BK * 2;
+constexpr size_t GEMM_STAGE_BYTES = GEMM_A_BYTES + GEMM_B_BYTES;
+constexpr size_t GEMM_SMEM_BYTES = GEMM_STAGES * GEMM_STAGE_BYTES + 1024 + 256;
+
+cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream_t st);
+
+// ---------------------------------------------------------------------------
+// routing / permutation kernels, see routing.cu
+// ---------------------------------------------------------------------------
+struct Ctx {  // typed views of ctx + ws for one shape
+  int* hdr;
+  int *ids, *counts, *offsets, *poff, *perm_tok, *perm_asg, *slot_row, *row_asg;
+  float *gates, *row_gate;
+  __nv_bfloat16 *xperm, *abuf, *bbuf;
+  int* hist;
+  float* logits;
+  __nv_bfloat16 *hbuf, *obuf, *dyperm, *dabuf, *dbbuf, *hgbuf, *wrt, *dxperm;
+  float *dgpart, *dlasg;
+};
+Ctx make_ctx(const Layout& L, void* ctx, void* ws);
+
+cudaError_t launch_router_logits(const Layout& L, const __nv_bfloat16* X, const __nv_bfloat16* W_r,
+                                 const float* bias, float* logits, cudaStream_t st);
+cudaError_t launch_topk(const Layout& L, const Ctx& c, cudaStream_t st);
+cudaError_t launch_scan(const Layout& L, const Ctx& c, cudaStream_t st);
+cudaError_t launch_scatter(const Layout& L, const Ctx& c, cudaStream_t st);
+cudaError_t launch_gather_rows(const Layout& L, const Ctx& c, const __nv_bfloat16* src, __nv_bfloat16* dst,
+                               cudaStream_t st);
+cudaError_t launch_combine(const Layout& L, const Ctx& c, const __nv_bfloat16* Oprime, __nv_bfloat16* Y,
+                           cudaStream_t st);
+cudaError_t launch_router_bwd(const Layout& L, const Ctx& c, cudaStream_t st);
+cudaError_t launch_transpose_wr(const Layout& L, const __nv_bfloat16* W_r, __nv_bfloat16* W_rT, cudaStream_t st);
+cudaError_t launch_rev_dispatch(const Layout& L, const Ctx& c, __nv_bfloat16* dX, cudaStream_t st);
+cudaError_t launch_dwr(const Layout& L, const Ctx& c, const __nv_bfloat16* X, float* dW_r, cudaStream_t st);
+cudaError_t launch_export_routing(const Layout& L, const Ctx& c, int32_t* counts, int32_t* offsets,
+                                  int32_t* poff, int32_t* perm, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,472 @@
+// Routing, dispatch and combine kernels of the MoE layer (and their
+// backward mirrors).  These are the "schedule table" steps of the MoK pages
+// (page 1, "Three design decisions that matter", bullet 1): one routing table
+// (counts, prefix sums, a stable per-expert token order) drives the forward
+// dispatch and combine and the backward reverse-combine and reverse-dispatch.
+// On one GPU the NVLink pull/push becomes an on-device gather.
+//
+// Every reduction has a fixed order; integer atomics are used only where the
+// result does not depend on their order (shared-memory histogram counts).
+#include <cfloat>
+#include <cmath>
+
+#include "moe_internal.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// router GEMM: logits[T, E] = X[T, d] W_r[d, E] (+ bias), fp32 accumulate
+// 64 x 64 output tile per block, 256 threads x (4 x 4) outputs, K step 32.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_router_logits(const __nv_bfloat16* __restrict__ X,
+                                                       const __nv_bfloat16* __restrict__ Wr,
+                                                       const float* __restrict__ bias, float* __restrict__ logits,
+                                                       int T, int d, int E) {
+  __shared__ float sX[32][64 + 4];  // [k][token]
+  __shared__ float sW[32][64 + 4];  // [k][expert]
+  const int t0 = blockIdx.y * 64, e0 = blockIdx.x * 64;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < d; k0 += 32) {
+    for (int i = threadIdx.x; i < 64 * 32; i += 256) {
+      const int r = i >> 5, kk = i & 31;  // X tile: 64 tokens x 32 k
+      const int t = t0 + r;
+      sX[kk][r] = t < T ? __bfloat162float(X[static_cast<size_t>(t) * d + k0 + kk]) : 0.f;
+      const int kr = i >> 6, c = i & 63;  // W tile: 32 k x 64 experts
+      const int e = e0 + c;
+      sW[kr][c] = e < E ? __bfloat162float(Wr[static_cast<size_t>(k0 + kr) * E + e]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < 32; ++kk) {
+      float xv[4], wv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xv[i] = sX[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) wv[j] = sW[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e < E) logits[static_cast<size_t>(t) * E + e] = acc[i][j] + (bias ? bias[e] : 0.f);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// top-k + softmax gating, one warp per token, plus a per-block expert histogram.
+// Order key: value descending, then expert id ascending; -0 == +0; NaN lowest.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ unsigned long long order_key(float v, int e) {
+  uint32_t ord;
+  if (isnan(v)) {
+    ord = 1u;  // below every number, above a removed entry (key 0)
+  } else {
+    if (v == 0.f) v = 0.f;  // -0 -> +0
+    const uint32_t u = __float_as_uint(v);
+    ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  }
+  return (static_cast<unsigned long long>(ord) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(e));
+}
+
+__global__ void __launch_bounds__(kTokensPerBlock * 32) k_topk(const float* __restrict__ logits, int T, int E, int k,
+                                                               int* __restrict__ ids, float* __restrict__ gates,
+                                                               int* __restrict__ hist, int* status) {
+  __shared__ int sh[kMaxE];
+  for (int i = threadIdx.x; i < E; i += blockDim.x) sh[i] = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kTokensPerBlock + warp;
+  if (t < T) {
+    const float* row = logits + static_cast<size_t>(t) * E;
+    unsigned long long key[kMaxE / 32];
+    bool bad = false;
+#pragma unroll
+    for (int q = 0; q < kMaxE / 32; ++q) {
+      const int e = lane + 32 * q;
+      key[q] = 0ull;
+      if (e < E) {
+        const float v = row[e];
+        bad |= !isfinite(v);
+        key[q] = order_key(v, e);
+      }
+    }
+    int my_e = 0;
+    float my_v = 0.f;
+    for (int j = 0; j < k; ++j) {
+      unsigned long long best = 0ull;
+      int bq = -1;
+#pragma unroll
+      for (int q = 0; q < kMaxE / 32; ++q)
+        if (key[q] > best) { best = key[q]; bq = q; }
+      unsigned long long wb = best;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const unsigned long long o = __shfl_xor_sync(0xffffffffu, wb, off);
+        wb = o > wb ? o : wb;
+      }
+      const int e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(wb & 0xFFFFFFFFull));
+      if (bq >= 0 && best == wb) {  // the owning lane removes the winner (ids are unique)
+#pragma unroll
+        for (int q = 0; q < kMaxE / 32; ++q)
+          if (q == bq) key[q] = 0ull;
+      }
+      if (lane == j) { my_e = e; my_v = row[e]; }
+    }
+    // softmax over the selected logits; the first selected is the largest
+    const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
+    const float ex = lane < k ? expf(my_v - vmax) : 0.f;
+    float sum = 0.f;
+    for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, ex, j);  // fixed order
+    if (lane < k) {
+      ids[static_cast<size_t>(t) * k + lane] = my_e;
+      gates[static_cast<size_t>(t) * k + lane] = ex / sum;
+      atomicAdd(&sh[my_e], 1);
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    if (bad && lane == 0) raise_status(status, MOE_ERR_NONFINITE);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < E; i += blockDim.x) hist[static_cast<size_t>(blockIdx.x) * E + i] = sh[i];
+}
+
+// ---------------------------------------------------------------------------
+// histogram -> per-block bases, counts, offsets, padded offsets (one block).
+// hist[b][e] is replaced in place by the exclusive scan over b.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) k_scan(int* __restrict__ hist, int nblk, int E, int first, int El,
+                                               int* __restrict__ counts, int* __restrict__ offsets,
+                                               int* __restrict__ poff, int* __restrict__ hdr) {
+  __shared__ int sc[kMaxE];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int b = 0; b < nblk; ++b) {
+      const int h = hist[static_cast<size_t>(b) * E + e];
+      hist[static_cast<size_t>(b) * E + e] = run;
+      run += h;
+    }
+    counts[e] = run;
+    sc[e] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int e = 0; e < E; ++e) { offsets[e] = run; run += sc[e]; }
+    offsets[E] = run;
+    int prun = 0;
+    for (int el = 0; el < El; ++el) {
+      poff[el] = prun;
+      prun += (sc[first + el] + kPad - 1) / kPad * kPad;
+    }
+    poff[El] = prun;
+    hdr[HDR_ROWS_P] = prun;
+    hdr[HDR_MTILES] = prun / kPad;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// stable scatter: one warp per block of tokens, tokens in ascending order.
+// row position of (t, j) inside expert e = base[b][e] + #{earlier tokens of b with e}.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(32) k_scatter(const int* __restrict__ ids, const float* __restrict__ gates,
+                                                const int* __restrict__ base, const int* __restrict__ offsets,
+                                                const int* __restrict__ poff, int T, int E, int k, int first, int El,
+                                                int* __restrict__ perm_tok, int* __restrict__ perm_asg,
+                                                int* __restrict__ slot_row, int* __restrict__ row_asg,
+                                                float* __restrict__ row_gate) {
+  __shared__ int run[kMaxE];
+  const int b = blockIdx.x, lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) run[e] = base[static_cast<size_t>(b) * E + e];
+  __syncwarp();
+  for (int i = 0; i < kTokensPerBlock; ++i) {
+    const int t = b * kTokensPerBlock + i;
+    if (t >= T) break;
+    if (lane < k) {
+      const int a = t * k + lane;
+      const int e = ids[a];
+      const int pos = run[e];
+      run[e] = pos + 1;  // the k experts of one token are distinct: no two lanes share e
+      const int u = offsets[e] + pos;
+      perm_tok[u] = t;
+      perm_asg[u] = a;
+      const int el = e - first;
+      if (el >= 0 && el < El) {
+        const int R = poff[el] + pos;
+        slot_row[a] = R;
+        row_asg[R] = a;
+        row_gate[R] = gates[a];
+      } else {
+        slot_row[a] = -1;
+      }
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dispatch / reverse-combine: dst[R] = src[token(R)], zero rows for padding.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) k_gather_rows(const __nv_bfloat16* __restrict__ src,
+                                                     const int* __restrict__ row_asg, const int* __restrict__ hdr,
+                                                     int k, int d, int64_t RP, __nv_bfloat16* __restrict__ dst) {
+  const int rows_p = __ldg(hdr + HDR_ROWS_P);
+  const int nv = d / 8;
+  for (int64_t R = blockIdx.x; R < rows_p; R += gridDim.x) {
+    const int a = row_asg[R];
+    uint4* out = reinterpret_cast<uint4*>(dst + R * d);
+    if (a >= 0) {
+      const uint4* in = reinterpret_cast<const uint4*>(src + static_cast<size_t>(a / k) * d);
+      for (int i = threadIdx.x; i < nv; i += blockDim.x) out[i] = __ldg(in + i);
+    } else {
+      const uint4 z = make_uint4(0, 0, 0, 0);
+      for (int i = threadIdx.x; i < nv; i += blockDim.x) out[i] = z;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// combine: Y[t] = sum_j O'[slot_row[t, j]] in slot order, fp32, stored bf16.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) k_combine(const __nv_bfloat16* __restrict__ Op,
+                                                 const int* __restrict__ slot_row, int k, int d,
+                                                 __nv_bfloat16* __restrict__ Y) {
+  const int t = blockIdx.x;
+  __shared__ int rows[kMaxK];
+  if (threadIdx.x < k) rows[threadIdx.x] = slot_row[static_cast<size_t>(t) * k + threadIdx.x];
+  __syncthreads();
+  for (int i = threadIdx.x * 8; i < d; i += blockDim.x * 8) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < k; ++j) {
+      const int R = rows[j];
+      if (R < 0) continue;
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(Op + static_cast<size_t>(R) * d + i));
+      float2 f;
+      f = unpack_bf16(u.x); acc[0] += f.x; acc[1] += f.y;
+      f = unpack_bf16(u.y); acc[2] += f.x; acc[3] += f.y;
+      f = unpack_bf16(u.z); acc[4] += f.x; acc[5] += f.y;
+      f = unpack_bf16(u.w); acc[6] += f.x; acc[7] += f.y;
+    }
+    uint4 o;
+    o.x = pack_bf16(acc[0], acc[1]);
+    o.y = pack_bf16(acc[2], acc[3]);
+    o.z = pack_bf16(acc[4], acc[5]);
+    o.w = pack_bf16(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(Y + static_cast<size_t>(t) * d + i) = o;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// router backward, one warp per token:
+//   dg_j = sum over n-tiles of the dgrad epilogue's partials (fixed order)
+//   dl_j = g_j (dg_j - sum_m g_m dg_m)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_router_bwd(const float* __restrict__ dgpart, const int* __restrict__ slot_row,
+                                                    const float* __restrict__ gates, int T, int k, int ntn,
+                                                    float* __restrict__ dlasg) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= T) return;
+  float dg = 0.f, g = 0.f;
+  if (lane < k) {
+    const size_t a = static_cast<size_t>(t) * k + lane;
+    const int R = slot_row[a];
+    g = gates[a];
+    if (R >= 0)
+      for (int q = 0; q < ntn; ++q) dg += dgpart[static_cast<size_t>(R) * ntn + q];
+  }
+  float s = 0.f;
+  const float gd = g * dg;
+  for (int j = 0; j < k; ++j) s += __shfl_sync(0xffffffffu, gd, j);
+  if (lane < k) dlasg[static_cast<size_t>(t) * k + lane] = g * (dg - s);
+}
+
+// W_r [d, E] -> W_r^T [E, d] (bf16), 32 x 32 tiles
+__global__ void __launch_bounds__(256) k_transpose_wr(const __nv_bfloat16* __restrict__ Wr, int d, int E,
+                                                      __nv_bfloat16* __restrict__ WrT) {
+  __shared__ __nv_bfloat16 tile[32][33];
+  const int i0 = blockIdx.y * 32, e0 = blockIdx.x * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int r = ty; r < 32; r += 8) {
+    const int i = i0 + r, e = e0 + tx;
+    if (i < d && e < E) tile[r][tx] = Wr[static_cast<size_t>(i) * E + e];
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int e = e0 + r, i = i0 + tx;
+    if (i < d && e < E) WrT[static_cast<size_t>(e) * d + i] = tile[tx][r];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// reverse-dispatch: dX[t] = sum_j dX_perm[slot_row[t,j]] + sum_j dl_j W_r[:, e_j]
+// (expert terms first, then router terms, each in slot order; fp32; bf16 out)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) k_rev_dispatch(const __nv_bfloat16* __restrict__ dxperm,
+                                                      const int* __restrict__ slot_row, const int* __restrict__ ids,
+                                                      const float* __restrict__ dlasg,
+                                                      const __nv_bfloat16* __restrict__ WrT, int k, int d,
+                                                      __nv_bfloat16* __restrict__ dX) {
+  const int t = blockIdx.x;
+  __shared__ int rows[kMaxK], eid[kMaxK];
+  __shared__ float dl[kMaxK];
+  if (threadIdx.x < k) {
+    const size_t a = static_cast<size_t>(t) * k + threadIdx.x;
+    rows[threadIdx.x] = slot_row[a];
+    eid[threadIdx.x] = ids[a];
+    dl[threadIdx.x] = dlasg[a];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x * 8; i < d; i += blockDim.x * 8) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < k; ++j) {
+      const int R = rows[j];
+      if (R < 0) continue;
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(dxperm + static_cast<size_t>(R) * d + i));
+      float2 f;
+      f = unpack_bf16(u.x); acc[0] += f.x; acc[1] += f.y;
+      f = unpack_bf16(u.y); acc[2] += f.x; acc[3] += f.y;
+      f = unpack_bf16(u.z); acc[4] += f.x; acc[5] += f.y;
+      f = unpack_bf16(u.w); acc[6] += f.x; acc[7] += f.y;
+    }
+    for (int j = 0; j < k; ++j) {
+      const float w = dl[j];
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(WrT + static_cast<size_t>(eid[j]) * d + i));
+      float2 f;
+      f = unpack_bf16(u.x); acc[0] = fmaf(w, f.x, acc[0]); acc[1] = fmaf(w, f.y, acc[1]);
+      f = unpack_bf16(u.y); acc[2] = fmaf(w, f.x, acc[2]); acc[3] = fmaf(w, f.y, acc[3]);
+      f = unpack_bf16(u.z); acc[4] = fmaf(w, f.x, acc[4]); acc[5] = fmaf(w, f.y, acc[5]);
+      f = unpack_bf16(u.w); acc[6] = fmaf(w, f.x, acc[6]); acc[7] = fmaf(w, f.y, acc[7]);
+    }
+    uint4 o;
+    o.x = pack_bf16(acc[0], acc[1]);
+    o.y = pack_bf16(acc[2], acc[3]);
+    o.z = pack_bf16(acc[4], acc[5]);
+    o.w = pack_bf16(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(dX + static_cast<size_t>(t) * d + i) = o;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dW_r[i, e] = sum over the assignments (t, j) to e, in the table's order, of dl_tj X[t, i].
+// dl has k nonzeros per token, so this is the sparse form of X^T dl.
+// Block: 32 columns of d x all experts; the [32 x E] result is staged in smem.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_dwr(const __nv_bfloat16* __restrict__ X, const int* __restrict__ offsets,
+                                             const int* __restrict__ perm_asg, const float* __restrict__ dlasg,
+                                             int d, int E, int k, float* __restrict__ dWr) {
+  extern __shared__ float sacc[];  // [32][E + 1]
+  const int i0 = blockIdx.x * 32;
+  const int i = threadIdx.x & 31, eg = threadIdx.x >> 5;
+  for (int e = eg; e < E; e += 8) {
+    float acc = 0.f;
+    const int u0 = offsets[e], u1 = offsets[e + 1];
+    for (int u = u0; u < u1; ++u) {
+      const int a = __ldg(perm_asg + u);
+      const float w = __ldg(dlasg + a);
+      acc = fmaf(w, __bfloat162float(X[static_cast<size_t>(a / k) * d + i0 + i]), acc);
+    }
+    sacc[i * (E + 1) + e] = acc;
+  }
+  __syncthreads();
+  for (int r = 0; r < 32; ++r)
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+      dWr[static_cast<size_t>(i0 + r) * E + e] = sacc[r * (E + 1) + e];
+}
+
+// local views of the routing table for the test hook
+__global__ void k_export_routing(const int* __restrict__ counts, const int* __restrict__ offsets,
+                                 const int* __restrict__ poff, const int* __restrict__ perm_tok, int first, int El,
+                                 int32_t* o_counts, int32_t* o_offsets, int32_t* o_poff, int32_t* o_perm) {
+  const int base = offsets[first];
+  const int n = offsets[first + El] - base;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i <= El || i < n; i += gridDim.x * blockDim.x) {
+    if (i < El && o_counts) o_counts[i] = counts[first + i];
+    if (i <= El && o_offsets) o_offsets[i] = offsets[first + i] - base;
+    if (i <= El && o_poff) o_poff[i] = poff[i];
+    if (i < n && o_perm) o_perm[i] = perm_tok[base + i];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+cudaError_t launch_router_logits(const Layout& L, const __nv_bfloat16* X, const __nv_bfloat16* W_r,
+                                 const float* bias, float* logits, cudaStream_t st) {
+  dim3 grid((L.E + 63) / 64, static_cast<unsigned>((L.T + 63) / 64));
+  k_router_logits<<<grid, 256, 0, st>>>(X, W_r, bias, logits, static_cast<int>(L.T), L.d, L.E);
+  return cudaGetLastError();
+}
+cudaError_t launch_topk(const Layout& L, const Ctx& c, cudaStream_t st) {
+  k_topk<<<L.nblk, kTokensPerBlock * 32, 0, st>>>(c.logits, static_cast<int>(L.T), L.E, L.k, c.ids, c.gates, c.hist,
+                                                  c.hdr + HDR_STATUS);
+  return cudaGetLastError();
+}
+cudaError_t launch_scan(const Layout& L, const Ctx& c, cudaStream_t st) {
+  k_scan<<<1, 1024, 0, st>>>(c.hist, L.nblk, L.E, L.first, L.El, c.counts, c.offsets, c.poff, c.hdr);
+  return cudaGetLastError();
+}
+cudaError_t launch_scatter(const Layout& L, const Ctx& c, cudaStream_t st) {
+  k_scatter<<<L.nblk, 32, 0, st>>>(c.ids, c.gates, c.hist, c.offsets, c.poff, static_cast<int>(L.T), L.E, L.k,
+                                   L.first, L.El, c.perm_tok, c.perm_asg, c.slot_row, c.row_asg, c.row_gate);
+  return cudaGetLastError();
+}
+cudaError_t launch_gather_rows(const Layout& L, const Ctx& c, const __nv_bfloat16* src, __nv_bfloat16* dst,
+                               cudaStream_t st) {
+  const int grid = static_cast<int>(L.RP < 148 * 16 ? L.RP : 148 * 16);
+  k_gather_rows<<<grid, 128, 0, st>>>(src, c.row_asg, c.hdr, L.k, L.d, L.RP, dst);
+  return cudaGetLastError();
+}
+cudaError_t launch_combine(const Layout& L, const Ctx& c, const __nv_bfloat16* Oprime, __nv_bfloat16* Y,
+                           cudaStream_t st) {
+  k_combine<<<static_cast<unsigned>(L.T), 128, 0, st>>>(Oprime, c.slot_row, L.k, L.d, Y);
+  return cudaGetLastError();
+}
+cudaError_t launch_router_bwd(const Layout& L, const Ctx& c, cudaStream_t st) {
+  k_router_bwd<<<static_cast<unsigned>((L.T + 7) / 8), 256, 0, st>>>(c.dgpart, c.slot_row, c.gates,
+                                                                       static_cast<int>(L.T), L.k, L.I / 256,
+                                                                       c.dlasg);
+  return cudaGetLastError();
+}
+cudaError_t launch_transpose_wr(const Layout& L, const __nv_bfloat16* W_r, __nv_bfloat16* W_rT, cudaStream_t st) {
+  dim3 grid((L.E + 31) / 32, (L.d + 31) / 32);
+  k_transpose_wr<<<grid, 256, 0, st>>>(W_r, L.d, L.E, W_rT);
+  return cudaGetLastError();
+}
+cudaError_t launch_rev_dispatch(const Layout& L, const Ctx& c, __nv_bfloat16* dX, cudaStream_t st) {
+  k_rev_dispatch<<<static_cast<unsigned>(L.T), 128, 0, st>>>(c.dxperm, c.slot_row, c.ids, c.dlasg, c.wrt, L.k, L.d,
+                                                              dX);
+  return cudaGetLastError();
+}
+cudaError_t launch_dwr(const Layout& L, const Ctx& c, const __nv_bfloat16* X, float* dW_r, cudaStream_t st) {
+  const size_t smem = 32 * static_cast<size_t>(L.E + 1) * sizeof(float);
+  static bool configured = false;
+  if (!configured) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(k_dwr, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * (kMaxE + 1) * 4);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  k_dwr<<<L.d / 32, 256, smem, st>>>(X, c.offsets, c.perm_asg, c.dlasg, L.d, L.E, L.k, dW_r);
+  return cudaGetLastError();
+}
+cudaError_t launch_export_routing(const Layout& L, const Ctx& c, int32_t* counts, int32_t* offsets, int32_t* poff,
+                                  int32_t* perm, cudaStream_t st) {
+  const int64_t n = L.T * L.k + L.El + 1;
+  const int grid = static_cast<int>((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
+  k_export_routing<<<grid, 256, 0, st>>>(c.counts, c.offsets, c.poff, c.perm_tok, L.first, L.El, counts, offsets,
+                                         poff, perm);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,85 @@
+"""The C-ABI library: it loads, exports every declared symbol, sizes buffers
+from shapes alone and rejects bad arguments on the host (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixture_experts_layer_27_b200 import binding as B
+from mixture_experts_layer_27_b200 import build as BUILD
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    BUILD.build()
+    return B.lib()
+
+
+def declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(moe_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert {"moe_fwd", "moe_bwd", "moe_ctx_size", "moe_workspace_size", "moe_get_error"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_sizes_depend_on_shape_only_and_grow_with_it():
+    s1 = B.make_shape(128, 256, 8, 512, 2)
+    s2 = B.make_shape(2048, 7168, 256, 2048, 8)
+    for s in (s1, s2):
+        assert B.moe_ctx_size(s) > 0 and B.moe_workspace_size(s) > 0
+    assert B.moe_workspace_size(s2) > B.moe_workspace_size(s1)
+    # worst-case padded rows for the DeepSeek-V3-like shape: T*k + 127*E rows of X_perm (bf16)
+    rp = -(-(2048 * 8 + 127 * 256) // 128) * 128
+    assert B.moe_ctx_size(s2) >= rp * 7168 * 2 + 2 * rp * 2048 * 2
+
+
+@pytest.mark.parametrize("bad", [
+    dict(T=-1), dict(d=0), dict(d=200), dict(I=100), dict(E=0), dict(E=513), dict(top_k=0), dict(top_k=17),
+    dict(E=4, top_k=5), dict(first_local_expert=-1), dict(first_local_expert=6, num_local_experts=4),
+])
+def test_invalid_shapes_size_zero(bad):
+    kw = dict(T=64, d=256, E=8, I=256, top_k=2)
+    kw.update(bad)
+    s = B.make_shape(**kw)
+    assert B.moe_ctx_size(s) == 0 and B.moe_workspace_size(s) == 0
+
+
+def test_argument_errors_are_synchronous(lib):
+    s = B.make_shape(64, 256, 8, 256, 2)
+    nc, nw = B.moe_ctx_size(s), B.moe_workspace_size(s)
+    fake = 1 << 20  # never dereferenced: validation fails first
+    ok = dict(X=fake, W_r=fake, bias=None, W_gate=fake, W_up=fake, W_down=fake, Y=fake, ctx=fake, ws=fake)
+
+    def fwd(**over):
+        a = dict(ok, **over)
+        return B.moe_fwd(s, a["X"], a["W_r"], a["bias"], a["W_gate"], a["W_up"], a["W_down"], a["Y"], a["ctx"],
+                         a["ws"], stream=0, ctx_bytes=over.get("cb", nc), ws_bytes=over.get("wb", nw))
+
+    assert fwd(X=None) == B.MOE_ERR_INVALID_ARG
+    assert fwd(ctx=None) == B.MOE_ERR_INVALID_ARG
+    assert fwd(X=fake + 2) == B.MOE_ERR_INVALID_ARG  # misaligned
+    assert fwd(cb=nc - 1) == B.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert fwd(wb=nw - 1) == B.MOE_ERR_WORKSPACE_TOO_SMALL
+    bad = B.make_shape(64, 256, 8, 256, 9)
+    assert B.moe_fwd(bad, *[fake] * 2, None, *[fake] * 5, nc, fake, nw, 0) == B.MOE_ERR_UNSUPPORTED
+    mx = B.make_shape(64, 256, 8, 256, 2, prec=B.MOE_MXFP8)
+    assert B.moe_fwd(mx, *[fake] * 2, None, *[fake] * 5, nc, fake, nw, 0) == B.MOE_ERR_UNSUPPORTED
+    r = B.moe_bwd(s, fake, fake, fake, fake, fake, None, fake, fake, fake, fake, fake, fake, fake, stream=0,
+                  ctx_bytes=nc, ws_bytes=nw)
+    assert r == B.MOE_ERR_INVALID_ARG  # dY missing
+    assert B.moe_get_error(None, 0) == B.MOE_ERR_INVALID_ARG
+    for code in range(7):
+        assert B.status_string(code)

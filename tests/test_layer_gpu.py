@@ -1,0 +1,135 @@
+"""GPU parity of the whole layer (forward + backward) against the fp64 oracle.
+
+Floating-point outputs: max |gpu - oracle| / max |oracle| <= 2e-2 per tensor (bf16 mode).
+Routing table: bit-exact against the oracle's selection run on the GPU's own
+fp32 logits (the argmax is decided in the kernel's precision on both sides).
+Results: bit-identical across repeated runs and across workspace placements.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from mixture_experts_layer_27_b200 import binding as B
+
+from _util import TOL_BF16, make_case, relerr, run_gpu, run_oracle, to64
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_routing(layer, x, k, E, first, num):
+    r = layer.routing()
+    lg = to64(layer.logits())
+    ids = O.topk_ids(lg, k)
+    assert np.array_equal(r["ids"].cpu().numpy(), ids)
+    s = O.schedule(ids, E, first, num or None)
+    assert np.array_equal(r["counts"].cpu().numpy(), s["counts"])
+    assert np.array_equal(r["offsets"].cpu().numpy(), s["offsets"])
+    assert np.array_equal(r["padded_offsets"].cpu().numpy(), s["padded_offsets"])
+    assert np.array_equal(r["perm"].cpu().numpy(), s["perm"])
+    assert np.array_equal(r["slot_row"].cpu().numpy(), s["slot_row"])
+    g = O.gates(lg, ids)
+    assert np.max(np.abs(r["gates"].cpu().numpy() - g)) < 1e-6
+    # the fp32 logits themselves against fp64
+    X, Wr = to64(x["X"]), to64(x["W_r"])
+    b = None if x["bias"] is None else to64(x["bias"])
+    assert relerr(lg, O.router_logits(X, Wr, b)) < 1e-5
+    return s
+
+
+def _check_layer(T, d, E, k, I, first=0, num=0, bias=None, seed=0):
+    w, x = make_case(T, d, E, k, I, seed=seed, bias=bias)
+    layer, Y, g, st = run_gpu(x, T, d, E, k, I, first, num)
+    assert st == B.MOE_OK, B.status_string(st)
+    _check_routing(layer, x, k, E, first, num)
+    Yo, ctx, go = run_oracle(x, k, first, num or None)
+    El = num or (E - first)
+    errs = {
+        "Y": relerr(to64(Y), Yo),
+        "dX": relerr(to64(g["dX"]), go["dX"]),
+        "dW_r": relerr(to64(g["dW_r"]), go["dW_r"]),
+        "dW_gate": relerr(to64(g["dW_gate"]), np.stack([go["dW_gate"][first + e] for e in range(El)])),
+        "dW_up": relerr(to64(g["dW_up"]), np.stack([go["dW_up"][first + e] for e in range(El)])),
+        "dW_down": relerr(to64(g["dW_down"]), np.stack([go["dW_down"][first + e] for e in range(El)])),
+    }
+    bad = {kk: v for kk, v in errs.items() if not v <= TOL_BF16}
+    assert not bad, errs
+    return layer, x, Y, g
+
+
+def test_tiny_config_matches_oracle():
+    """T=128, d=256, E=8, top-2, I=512 (the small workload), seed 0."""
+    _check_layer(128, 256, 8, 2, 512)
+
+
+def test_ragged_tokens_and_uneven_experts():
+    _check_layer(77, 256, 6, 3, 256, seed=1)
+
+
+def test_hot_expert_spans_many_tiles_and_empty_expert():
+    bias = np.zeros(4, dtype=np.float32)
+    bias[0] = 8.0    # every token picks expert 0: 600 rows -> 5 padded tiles
+    bias[3] = -40.0  # expert 3 is never picked: zero gradient
+    _check_layer(600, 512, 4, 2, 512, bias=bias, seed=2)
+
+
+def test_k_equals_E():
+    _check_layer(64, 256, 4, 4, 256, seed=3)
+
+
+def test_single_expert():
+    _check_layer(100, 256, 1, 1, 256, seed=4)
+
+
+def test_many_experts_mostly_empty():
+    _check_layer(256, 256, 384, 8, 256, seed=5)
+
+
+def test_local_expert_slice():
+    _check_layer(200, 256, 16, 4, 256, first=4, num=5, seed=6)
+
+
+def test_no_tokens():
+    T, d, E, k, I = 0, 256, 4, 2, 256
+    layer = B.MoELayer(T, d, E, I, k)
+    x = {n: torch.randn(*s, device="cuda").to(torch.bfloat16) for n, s in
+         dict(X=(1, d), W_r=(d, E), W_gate=(E, d, I), W_up=(E, d, I), W_down=(E, I, d), dY=(1, d)).items()}
+    X0, dY0 = x["X"][:0], x["dY"][:0]
+    layer.forward(X0, x["W_r"], None, x["W_gate"], x["W_up"], x["W_down"], Y=torch.empty(0, d, device="cuda",
+                                                                                         dtype=torch.bfloat16))
+    g = layer.backward(X0, x["W_r"], x["W_gate"], x["W_up"], x["W_down"], dY0,
+                       out=dict(dX=torch.empty(0, d, device="cuda", dtype=torch.bfloat16),
+                                dW_gate=torch.full((E, d, I), 7.0, device="cuda", dtype=torch.bfloat16),
+                                dW_up=torch.full((E, d, I), 7.0, device="cuda", dtype=torch.bfloat16),
+                                dW_down=torch.full((E, I, d), 7.0, device="cuda", dtype=torch.bfloat16),
+                                dW_r=torch.full((d, E), 7.0, device="cuda")))
+    torch.cuda.synchronize()
+    for n in ("dW_gate", "dW_up", "dW_down", "dW_r"):
+        assert torch.count_nonzero(g[n]) == 0
+
+
+def test_bit_identical_across_runs_and_workspace_placement():
+    T, d, E, k, I = 300, 512, 8, 2, 512
+    w, x = make_case(T, d, E, k, I, seed=7)
+    _, Y1, g1, st1 = run_gpu(x, T, d, E, k, I)
+    _, Y2, g2, st2 = run_gpu(x, T, d, E, k, I)
+    # a second layer whose ctx / ws start 256 bytes further into larger buffers
+    lay = B.MoELayer(T, d, E, I, k)
+    lay.ctx = torch.empty(lay.ctx.numel() + 4096, dtype=torch.uint8, device="cuda")[256:]
+    lay.ws = torch.empty(lay.ws.numel() + 4096, dtype=torch.uint8, device="cuda")[1024:]
+    _, Y3, g3, st3 = run_gpu(x, T, d, E, k, I, layer=lay)
+    assert st1 == st2 == st3 == B.MOE_OK
+    for Ya, ga in ((Y2, g2), (Y3, g3)):
+        assert torch.equal(Y1.view(torch.int16), Ya.view(torch.int16))
+        for n in g1:
+            assert torch.equal(g1[n].view(torch.int16) if g1[n].dtype == torch.bfloat16 else g1[n].view(torch.int32),
+                               ga[n].view(torch.int16) if ga[n].dtype == torch.bfloat16 else ga[n].view(torch.int32)), n
+
+
+def test_nonfinite_logit_sets_status():
+    T, d, E, k, I = 32, 256, 8, 2, 256
+    w, x = make_case(T, d, E, k, I, seed=8)
+    x["X"][5, 3] = float("inf")
+    layer, Y, g, st = run_gpu(x, T, d, E, k, I)
+    assert st == B.MOE_ERR_NONFINITE
+    assert layer.error() == B.MOE_OK  # reading the status clears it
