@@ -1,19 +1,21 @@
 // Expert-grouped GEMMs of the MoE layer on sm_100a tensor cores.
 //
-// One persistent, warp-specialised kernel template serves all six GEMMs of
+// One persistent, warp-specialised kernel template serves the six GEMMs of
 // the forward and backward ("expert-grouped GEMM", page 1 of the MoK pages,
-// "Three design decisions that matter", bullet 2):
+// "Three design decisions that matter", bullet 2) and the router GEMM:
 //
-//   warp 0      one thread issues TMA tile loads into a 4-stage smem ring
+//   warp 0      one thread issues TMA tile loads into a 3-4 stage smem ring
 //   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
 //   warps 2..5  epilogue: tcgen05.ld from TMEM, fused math, global stores
+//               (the wgrad GEMMs stage their tiles in smem for TMA stores)
 //
 // The output tile is 128 x 256 (fp32 in TMEM), K advances 64 at a time
 // (one 128-byte swizzle atom of bf16).  Two accumulators let the epilogue of
-// tile i overlap the MMAs of tile i+1.  Every output tile is produced by one
-// CTA with one fixed K order, so results are bit-reproducible (no split-K,
-// no atomics).  Tiles are listed on the device from the padded expert
-// offsets, so the host never needs the routing result.
+// tile i overlap the MMAs of tile i+1.  Every output element is produced by
+// one CTA with one fixed K order, so results are bit-reproducible (no
+// atomics; the router GEMM's fixed K splits are summed in split order by the
+// top-k kernel).  Expert tiles are listed on the device from the padded
+// expert offsets, so the host never needs the routing result.
 #include <cstdio>
 
 #include "moe_internal.cuh"
@@ -29,6 +31,19 @@ template <> struct Traits<G_DGRAD_DOWN>   { static constexpr bool A_MN = false, 
 template <> struct Traits<G_DGRAD_GATEUP> { static constexpr bool A_MN = false, B_MN = false; };
 template <> struct Traits<G_WGRAD_GATEUP> { static constexpr bool A_MN = true, B_MN = true; };
 template <> struct Traits<G_WGRAD_DOWN>   { static constexpr bool A_MN = true, B_MN = true; };
+template <> struct Traits<G_ROUTER>       { static constexpr bool A_MN = false, B_MN = false; };
+
+// The wgrad GEMMs have short K loops (one expert's rows) and write a full
+// 128 x 256 output tile per tile: they trade a smem stage for a staging
+// buffer that feeds TMA stores.
+template <int KIND>
+constexpr bool is_wgrad() { return KIND == G_WGRAD_GATEUP || KIND == G_WGRAD_DOWN; }
+template <int KIND>
+constexpr int stages_of() { return is_wgrad<KIND>() ? 3 : GEMM_STAGES; }
+template <int KIND>
+constexpr size_t smem_bytes() {
+  return stages_of<KIND>() * GEMM_STAGE_BYTES + (is_wgrad<KIND>() ? GEMM_STAGE_OUT_BYTES : 0) + 1024 + 256;
+}
 
 struct Tile {
   int el;   // local expert
@@ -63,6 +78,7 @@ __device__ __forceinline__ int expert_of_row(const int* poff, int El, int R) {
 
 template <int KIND>
 __device__ __forceinline__ int num_tiles(const GemmParams& p) {
+  if (KIND == G_ROUTER) return ((p.T + 127) / 128) * ((p.E + 255) / 256) * p.splits;
   if (KIND <= G_DGRAD_GATEUP) return (__ldg(p.hdr + HDR_ROWS_P) / 128) * ntiles_n<KIND>(p);
   return p.El * mtiles_w<KIND>(p) * ntiles_n<KIND>(p);
 }
@@ -70,6 +86,19 @@ __device__ __forceinline__ int num_tiles(const GemmParams& p) {
 template <int KIND>
 __device__ __forceinline__ Tile decode(const GemmParams& p, int t) {
   Tile tl;
+  if constexpr (KIND == G_ROUTER) {
+    // tile = (m-tile, n-tile, K split); the splits of one output tile are adjacent
+    const int S = p.splits, NTr = (p.E + 255) / 256, KB = p.d / 64;
+    const int sp = t % S, rest = t / S;
+    const int nt = rest % NTr, mt = rest / NTr;
+    tl.el = sp;  // the split index rides in the expert slot
+    tl.m0 = mt * 128;
+    tl.nt = nt;
+    tl.n0 = nt * 256;
+    tl.kb0 = sp * KB / S;
+    tl.nk = (sp + 1) * KB / S - tl.kb0;
+    return tl;
+  }
   const int NT = ntiles_n<KIND>(p);
   if constexpr (KIND <= G_DGRAD_GATEUP) {
     // Tiles of expert e are [NT*poff[e]/128, NT*poff[e+1]/128), n-tile major so that
@@ -137,6 +166,10 @@ __device__ __forceinline__ void load_stage(const GemmParams& p, const Tile& tl, 
     const int nb = (tl.nt < NTg ? tl.nt : tl.nt - NTg) * 256;
 #pragma unroll
     for (int j = 0; j < 4; ++j) tma_load_2d(sB + j * 8192, mb, bar, nb + 64 * j, row, pol_act);
+  } else if constexpr (KIND == G_ROUTER) {
+    const int kx = (tl.kb0 + kb) * 64;
+    tma_load_2d(sA, &p.ta0, bar, kx, tl.m0, pol_act);  // X [T, d], rows >= T read as zero
+    tma_load_2d(sB, &p.tb0, bar, kx, tl.n0, pol_act);  // W_r^T [E, d], rows >= E read as zero
   } else {  // G_WGRAD_DOWN
     const int row = (tl.kb0 + kb) * 64;
     tma_load_2d(sA, &p.ta0, bar, tl.m0, row, pol_act);                 // Hg, M = I (contiguous)
@@ -241,29 +274,71 @@ __device__ __forceinline__ void epilogue_row(const GemmParams& p, const Tile& tl
       tmem_ld32(taddr + c * 32, v);
       store_row32(p.out0 + R * p.d + tl.n0 + c * 32, v);
     }
-  } else {
-    __nv_bfloat16* out;
-    size_t base;
-    if constexpr (KIND == G_WGRAD_GATEUP) {
-      const int NTg = p.I / 256;
-      out = tl.nt < NTg ? p.out0 : p.out1;
-      const int nb = (tl.nt < NTg ? tl.nt : tl.nt - NTg) * 256;
-      base = static_cast<size_t>(tl.el) * p.d * p.I + static_cast<size_t>(tl.m0 + row) * p.I + nb;
-    } else {
-      out = p.out0;
-      base = static_cast<size_t>(tl.el) * p.I * p.d + static_cast<size_t>(tl.m0 + row) * p.d + tl.n0;
-    }
+  } else if constexpr (KIND == G_ROUTER) {
+    // fp32 partial logits of K split tl.el; rows >= T and columns >= E are dropped
+    const int t = tl.m0 + row;
+    float* dst = p.outf + (static_cast<size_t>(tl.el) * p.T + t) * p.E;
 #pragma unroll 1
     for (int c = 0; c < 8; ++c) {
       float v[32];
-      if (tl.nk > 0) {
-        tmem_ld32(taddr + c * 32, v);
-      } else {
+      tmem_ld32(taddr + c * 32, v);  // every lane loads (warp-collective), then masks
+      const int e0 = tl.n0 + c * 32;
+      if (t < p.T) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0.f;  // expert without tokens: zero gradient
+        for (int i = 0; i < 32; ++i)
+          if (e0 + i < p.E) dst[e0 + i] = v[i];
       }
-      store_row32(out + base + c * 32, v);
     }
+  }
+}
+
+// wgrad epilogue: the warp's 32 x 256 slice of the output tile goes through a
+// 128B-swizzled staging buffer (four 32 x 64 boxes) and out by TMA stores.
+template <int KIND>
+__device__ __forceinline__ void epilogue_wgrad(const GemmParams& p, const Tile& tl, int quarter, int lane,
+                                               uint32_t taddr, uint8_t* stage_out) {
+  const CUtensorMap* map;
+  int x0, y0;
+  if constexpr (KIND == G_WGRAD_GATEUP) {
+    const int NTg = p.I / 256;
+    map = tl.nt < NTg ? &p.to0 : &p.to1;  // dW_gate or dW_up as [El*d, I]
+    x0 = (tl.nt < NTg ? tl.nt : tl.nt - NTg) * 256;
+    y0 = tl.el * p.d + tl.m0 + quarter * 32;
+  } else {
+    map = &p.to0;  // dW_down as [El*I, d]
+    x0 = tl.n0;
+    y0 = tl.el * p.I + tl.m0 + quarter * 32;
+  }
+  if (lane == 0) bulk_wait_read0();  // the previous tile's stores have left the buffer
+  __syncwarp();
+  uint8_t* rowp = stage_out + lane * 128;
+#pragma unroll 1
+  for (int c = 0; c < 8; ++c) {
+    float v[32];
+    if (tl.nk > 0) {
+      tmem_ld32(taddr + c * 32, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0.f;  // expert without tokens: zero gradient
+    }
+    uint8_t* box = rowp + (c >> 1) * 4096;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int chunk = (c & 1) * 4 + q;  // 16-byte chunk within the 128-byte row
+      uint4 u;
+      u.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
+      u.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+      u.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+      u.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+      *reinterpret_cast<uint4*>(box + ((chunk ^ (lane & 7)) << 4)) = u;
+    }
+  }
+  fence_proxy_async();
+  __syncwarp();
+  if (lane == 0) {
+#pragma unroll
+    for (int b = 0; b < 4; ++b) tma_store_2d(map, stage_out + b * 4096, x0 + b * 64, y0);
+    bulk_commit();
   }
 }
 
@@ -279,16 +354,18 @@ template <int KIND>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + GEMM_STAGES * GEMM_STAGE_BYTES);
-  uint64_t* empty = full + GEMM_STAGES;
-  uint64_t* tfull = empty + GEMM_STAGES;
+  constexpr int STAGES = stages_of<KIND>();
+  uint8_t* stage_out = smem + STAGES * GEMM_STAGE_BYTES;  // wgrad only: 4 x 16 KB
+  uint64_t* full = reinterpret_cast<uint64_t*>(stage_out + (is_wgrad<KIND>() ? GEMM_STAGE_OUT_BYTES : 0));
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < GEMM_STAGES; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -323,8 +400,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
       const uint64_t pol_w = policy_evict_first();
       int stage = 0;
       uint32_t phase = 0;
-      int last_parity[GEMM_STAGES];
-      for (int s = 0; s < GEMM_STAGES; ++s) last_parity[s] = -1;
+      int last_parity[STAGES];
+      for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         const Tile tl = decode<KIND>(p, t);
@@ -335,11 +412,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
           mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(GEMM_STAGE_BYTES));
           load_stage<KIND>(p, tl, kb, sA, sB, &full[stage], pol_act, pol_w);
           last_parity[stage] = static_cast<int>(phase);
-          if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1; }
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
       if (!ok) {  // let copies already in flight land before the CTA's smem goes away
-        for (int s = 0; s < GEMM_STAGES; ++s)
+        for (int s = 0; s < STAGES; ++s)
           if (last_parity[s] >= 0) mbar_wait_drain(&full[s], static_cast<uint32_t>(last_parity[s]));
       }
     }
@@ -371,7 +448,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
             umma_bf16(dtm, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
-          if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1; }
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
         if (tl.nk > 0) umma_commit(&tfull[acc]);
@@ -396,10 +473,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
       __syncwarp();
       tc_fence_after();
       const uint32_t taddr = tbase + (static_cast<uint32_t>(quarter * 32) << 16) + acc * GEMM_BN;
-      epilogue_row<KIND>(p, tl, row, taddr);
+      if constexpr (is_wgrad<KIND>())
+        epilogue_wgrad<KIND>(p, tl, quarter, lane, taddr, stage_out + (warp - 2) * (GEMM_STAGE_OUT_BYTES / 4));
+      else
+        epilogue_row<KIND>(p, tl, row, taddr);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+    if constexpr (is_wgrad<KIND>()) {
+      if (lane == 0) bulk_wait0();  // stores complete before the CTA (and its smem) goes away
+      __syncwarp();
     }
   }
   __syncthreads();
@@ -415,11 +499,11 @@ static cudaError_t launch_kind(const GemmParams& p, int grid, cudaStream_t st) {
   static bool configured = false;
   if (!configured) {
     const cudaError_t e = cudaFuncSetAttribute(k_moe_gemm<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(GEMM_SMEM_BYTES));
+                                               static_cast<int>(smem_bytes<KIND>()));
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  k_moe_gemm<KIND><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(p);
+  k_moe_gemm<KIND><<<grid, GEMM_THREADS, smem_bytes<KIND>(), st>>>(p);
   return cudaGetLastError();
 }
 
@@ -431,6 +515,7 @@ cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream
     case G_DGRAD_GATEUP: return launch_kind<G_DGRAD_GATEUP>(p, grid, st);
     case G_WGRAD_GATEUP: return launch_kind<G_WGRAD_GATEUP>(p, grid, st);
     case G_WGRAD_DOWN: return launch_kind<G_WGRAD_DOWN>(p, grid, st);
+    case G_ROUTER: return launch_kind<G_ROUTER>(p, grid, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -61,6 +61,7 @@ bool make_layout(const moe_shape& s, Layout* L) {
   o = 0;
   L->hist = take(static_cast<size_t>(L->nblk) * s.E * 4);
   L->logits = take(T * s.E * 4);
+  L->rpart = take(static_cast<size_t>(router_splits(s.T, s.E, s.d)) * T * s.E * 4);
   L->hbuf = take(RP * s.I * 2);
   L->obuf = take(RP * s.d * 2);
   L->dyperm = take(RP * s.d * 2);
@@ -96,6 +97,7 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
   if (ws) {
     c.hist = reinterpret_cast<int*>(W(L.hist));
     c.logits = reinterpret_cast<float*>(W(L.logits));
+    c.rpart = reinterpret_cast<float*>(W(L.rpart));
     c.hbuf = reinterpret_cast<__nv_bfloat16*>(W(L.hbuf));
     c.obuf = reinterpret_cast<__nv_bfloat16*>(W(L.obuf));
     c.dyperm = reinterpret_cast<__nv_bfloat16*>(W(L.dyperm));
@@ -295,9 +297,30 @@ moe_status moe_fwd(const moe_shape* s, const void* X, const void* W_r, const flo
   if (L.T == 0) return MOE_OK;
 
   const auto* Xb = static_cast<const __nv_bfloat16*>(X);
-  // 1-2. router GEMM, top-k gating, per-block histograms
-  MOE_TRY(timed(K_ROUTER_LOGITS, st, [&] { return launch_router_logits(L, Xb, static_cast<const __nv_bfloat16*>(W_r), bias, c.logits, st); }));
-  MOE_TRY(timed(K_TOPK, st, [&] { return launch_topk(L, c, st); }));
+  const int grid = num_sms();
+  int* status = c.hdr + HDR_STATUS;
+  const uint64_t RP = static_cast<uint64_t>(L.RP);
+  // 1. router GEMM on the tensor cores: fixed K splits -> fp32 partials
+  MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
+    return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
+  }));
+  const int splits = router_splits(L.T, L.E, L.d);
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, X, L.d, static_cast<uint64_t>(L.T), L.d, 64, 128));
+    MOE_TMAP(tmap_2d(&p.tb0, c.wrt, L.d, static_cast<uint64_t>(L.E), L.d, 64, 256));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.T = static_cast<int>(L.T);
+    p.E = L.E;
+    p.splits = splits;
+    p.outf = c.rpart;
+    const int64_t tiles = ((L.T + 127) / 128) * ((L.E + 255) / 256) * splits;
+    const int g = static_cast<int>(tiles < grid ? tiles : grid);
+    MOE_TRY(timed(K_ROUTER_LOGITS, st, [&] { return launch_gemm(G_ROUTER, p, g, st); }));
+  }
+  // 2. partial sums (fixed order) + bias, top-k gating, per-block histograms
+  MOE_TRY(timed(K_TOPK, st, [&] { return launch_topk(L, c, bias, splits, st); }));
   // 3. counts, prefix sums, padded offsets
   MOE_TRY(timed(K_SCAN, st, [&] { return launch_scan(L, c, st); }));
   // 4. stable scatter + dispatch
@@ -306,9 +329,6 @@ moe_status moe_fwd(const moe_shape* s, const void* X, const void* W_r, const flo
   MOE_TRY(timed(K_SCATTER, st, [&] { return launch_scatter(L, c, st); }));
   MOE_TRY(timed(K_DISPATCH, st, [&] { return launch_gather_rows(L, c, Xb, c.xperm, st); }));
 
-  const int grid = num_sms();
-  int* status = c.hdr + HDR_STATUS;
-  const uint64_t RP = static_cast<uint64_t>(L.RP);
   // 5. grouped gate/up GEMM with the SwiGLU epilogue
   {
     GemmParams p = base_params(L, c, status);
@@ -405,6 +425,8 @@ moe_status moe_bwd(const moe_shape* s, const void* X, const void* W_r, const voi
     MOE_TMAP(tmap_2d(&p.ta0, c.xperm, L.d, RP, L.d, 64, 64));
     MOE_TMAP(tmap_2d(&p.tb0, c.dabuf, L.I, RP, L.I, 64, 64));
     MOE_TMAP(tmap_2d(&p.tb1, c.dbbuf, L.I, RP, L.I, 64, 64));
+    MOE_TMAP(tmap_2d(&p.to0, dW_gate, L.I, El * L.d, L.I, 64, 32));
+    MOE_TMAP(tmap_2d(&p.to1, dW_up, L.I, El * L.d, L.I, 64, 32));
     p.ta1 = p.ta0;
     p.out0 = static_cast<__nv_bfloat16*>(dW_gate);
     p.out1 = static_cast<__nv_bfloat16*>(dW_up);
@@ -414,6 +436,8 @@ moe_status moe_bwd(const moe_shape* s, const void* X, const void* W_r, const voi
     GemmParams p = base_params(L, c, status);
     MOE_TMAP(tmap_2d(&p.ta0, c.hgbuf, L.I, RP, L.I, 64, 64));
     MOE_TMAP(tmap_2d(&p.tb0, c.dyperm, L.d, RP, L.d, 64, 64));
+    MOE_TMAP(tmap_2d(&p.to0, dW_down, L.d, El * L.I, L.d, 64, 32));
+    p.to1 = p.to0;
     p.ta1 = p.ta0;
     p.tb1 = p.tb0;
     p.out0 = static_cast<__nv_bfloat16*>(dW_down);

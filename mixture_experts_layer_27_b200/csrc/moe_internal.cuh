@@ -31,7 +31,7 @@ struct Layout {
   size_t hdr, ids, gates, counts, offsets, poff, perm_tok, perm_asg, slot_row, row_asg, row_gate, xperm, abuf,
       bbuf, ctx_bytes;
   // ws
-  size_t hist, logits, hbuf, obuf, dyperm, dabuf, dbbuf, hgbuf, dgpart, dlasg, wrt, dxperm, ws_bytes;
+  size_t hist, logits, rpart, hbuf, obuf, dyperm, dabuf, dbbuf, hgbuf, dgpart, dlasg, wrt, dxperm, ws_bytes;
 };
 
 // Returns false for shapes outside the supported limits.
@@ -47,10 +47,12 @@ enum GemmKind {
   G_DGRAD_GATEUP = 3,   // dX_perm = dA . W_gate^T + dB . W_up^T
   G_WGRAD_GATEUP = 4,   // dW_gate = X_perm^T dA, dW_up = X_perm^T dB (per expert)
   G_WGRAD_DOWN = 5,     // dW_down = Hg^T dY_perm (per expert)
+  G_ROUTER = 6,         // router logits partials: part[s] = X[:, Ks] . W_r[Ks, :] (fixed K split s)
 };
 
 struct GemmParams {
-  CUtensorMap ta0, ta1, tb0, tb1;
+  CUtensorMap ta0, ta1, tb0, tb1;  // operand maps
+  CUtensorMap to0, to1;            // output maps (TMA stores of the wgrad epilogues)
   const int* hdr;             // ctx header (rows_p)
   const int* poff;            // padded offsets [El+1]
   const float* row_gate;      // [RP]
@@ -61,6 +63,7 @@ struct GemmParams {
   __nv_bfloat16* out2;
   float* outf;
   int El, d, I;
+  int T, E, splits;           // router GEMM: tokens, experts, K splits
   int* status;
 };
 
@@ -69,7 +72,14 @@ constexpr int GEMM_THREADS = 192;
 constexpr size_t GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;
 constexpr size_t GEMM_B_BYTES = GEMM_BN * GEMM_BK * 2;
 constexpr size_t GEMM_STAGE_BYTES = GEMM_A_BYTES + GEMM_B_BYTES;
-constexpr size_t GEMM_SMEM_BYTES = GEMM_STAGES * GEMM_STAGE_BYTES + 1024 + 256;
+constexpr size_t GEMM_STAGE_OUT_BYTES = 4 * 32 * 256 * 2;  // wgrad: one 32 x 256 bf16 slice per epilogue warp
+constexpr int router_splits(int64_t T, int E, int d) {  // K splits of the router GEMM (about one wave)
+  const int64_t tiles = ((T + 127) / 128) * ((E + 255) / 256);
+  int64_t s = tiles > 0 ? 148 / tiles : 1;
+  if (s < 1) s = 1;
+  if (s > d / 64) s = d / 64;
+  return static_cast<int>(s);
+}
 
 cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream_t st);
 
@@ -83,14 +93,13 @@ struct Ctx {  // typed views of ctx + ws for one shape
   __nv_bfloat16 *xperm, *abuf, *bbuf;
   int* hist;
   float* logits;
+  float* rpart;  // router split-K partials [splits, T, E]
   __nv_bfloat16 *hbuf, *obuf, *dyperm, *dabuf, *dbbuf, *hgbuf, *wrt, *dxperm;
   float *dgpart, *dlasg;
 };
 Ctx make_ctx(const Layout& L, void* ctx, void* ws);
 
-cudaError_t launch_router_logits(const Layout& L, const __nv_bfloat16* X, const __nv_bfloat16* W_r,
-                                 const float* bias, float* logits, cudaStream_t st);
-cudaError_t launch_topk(const Layout& L, const Ctx& c, cudaStream_t st);
+cudaError_t launch_topk(const Layout& L, const Ctx& c, const float* bias, int splits, cudaStream_t st);
 cudaError_t launch_scan(const Layout& L, const Ctx& c, cudaStream_t st);
 cudaError_t launch_scatter(const Layout& L, const Ctx& c, cudaStream_t st);
 cudaError_t launch_gather_rows(const Layout& L, const Ctx& c, const __nv_bfloat16* src, __nv_bfloat16* dst,

@@ -16,55 +16,6 @@
 namespace moe {
 
 // ---------------------------------------------------------------------------
-// router GEMM: logits[T, E] = X[T, d] W_r[d, E] (+ bias), fp32 accumulate
-// 64 x 64 output tile per block, 256 threads x (4 x 4) outputs, K step 32.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_router_logits(const __nv_bfloat16* __restrict__ X,
-                                                       const __nv_bfloat16* __restrict__ Wr,
-                                                       const float* __restrict__ bias, float* __restrict__ logits,
-                                                       int T, int d, int E) {
-  __shared__ float sX[32][64 + 4];  // [k][token]
-  __shared__ float sW[32][64 + 4];  // [k][expert]
-  const int t0 = blockIdx.y * 64, e0 = blockIdx.x * 64;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < d; k0 += 32) {
-    for (int i = threadIdx.x; i < 64 * 32; i += 256) {
-      const int r = i >> 5, kk = i & 31;  // X tile: 64 tokens x 32 k
-      const int t = t0 + r;
-      sX[kk][r] = t < T ? __bfloat162float(X[static_cast<size_t>(t) * d + k0 + kk]) : 0.f;
-      const int kr = i >> 6, c = i & 63;  // W tile: 32 k x 64 experts
-      const int e = e0 + c;
-      sW[kr][c] = e < E ? __bfloat162float(Wr[static_cast<size_t>(k0 + kr) * E + e]) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < 32; ++kk) {
-      float xv[4], wv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) xv[i] = sX[kk][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) wv[j] = sW[kk][tx * 4 + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = t0 + ty * 4 + i;
-    if (t >= T) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = e0 + tx * 4 + j;
-      if (e < E) logits[static_cast<size_t>(t) * E + e] = acc[i][j] + (bias ? bias[e] : 0.f);
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
 // top-k + softmax gating, one warp per token, plus a per-block expert histogram.
 // Order key: value descending, then expert id ascending; -0 == +0; NaN lowest.
 // ---------------------------------------------------------------------------
@@ -80,7 +31,11 @@ __device__ __forceinline__ unsigned long long order_key(float v, int e) {
   return (static_cast<unsigned long long>(ord) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(e));
 }
 
-__global__ void __launch_bounds__(kTokensPerBlock * 32) k_topk(const float* __restrict__ logits, int T, int E, int k,
+// The router GEMM leaves `splits` fp32 partial sums per logit (fixed K ranges);
+// they are added here in split order, then the bias, and the logit is stored.
+__global__ void __launch_bounds__(kTokensPerBlock * 32) k_topk(const float* __restrict__ part, int splits,
+                                                               const float* __restrict__ bias,
+                                                               float* __restrict__ logits, int T, int E, int k,
                                                                int* __restrict__ ids, float* __restrict__ gates,
                                                                int* __restrict__ hist, int* status) {
   __shared__ int sh[kMaxE];
@@ -89,7 +44,8 @@ __global__ void __launch_bounds__(kTokensPerBlock * 32) k_topk(const float* __re
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kTokensPerBlock + warp;
   if (t < T) {
-    const float* row = logits + static_cast<size_t>(t) * E;
+    float* row = logits + static_cast<size_t>(t) * E;
+    const size_t plane = static_cast<size_t>(T) * E;
     unsigned long long key[kMaxE / 32];
     bool bad = false;
 #pragma unroll
@@ -97,11 +53,16 @@ __global__ void __launch_bounds__(kTokensPerBlock * 32) k_topk(const float* __re
       const int e = lane + 32 * q;
       key[q] = 0ull;
       if (e < E) {
-        const float v = row[e];
+        const float* pp = part + static_cast<size_t>(t) * E + e;
+        float v = pp[0];
+        for (int s = 1; s < splits; ++s) v += pp[s * plane];
+        if (bias) v += bias[e];
+        row[e] = v;
         bad |= !isfinite(v);
         key[q] = order_key(v, e);
       }
     }
+    __syncwarp();
     int my_e = 0;
     float my_v = 0.f;
     for (int j = 0; j < k; ++j) {
@@ -358,30 +319,31 @@ __global__ void __launch_bounds__(128) k_rev_dispatch(const __nv_bfloat16* __res
 }
 
 // ---------------------------------------------------------------------------
-// dW_r[i, e] = sum over the assignments (t, j) to e, in the table's order, of dl_tj X[t, i].
-// dl has k nonzeros per token, so this is the sparse form of X^T dl.
-// Block: 32 columns of d x all experts; the [32 x E] result is staged in smem.
+// dW_r[:, e] = sum over the assignments (t, j) routed to e, in the table's
+// order (ascending t), of dl_tj X[t, :].  dl has k nonzeros per token, so this
+// is the sparse form of X^T dl.  One block per expert; each thread owns eight
+// consecutive columns of d and reads X rows with 16-byte loads.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_dwr(const __nv_bfloat16* __restrict__ X, const int* __restrict__ offsets,
                                              const int* __restrict__ perm_asg, const float* __restrict__ dlasg,
                                              int d, int E, int k, float* __restrict__ dWr) {
-  extern __shared__ float sacc[];  // [32][E + 1]
-  const int i0 = blockIdx.x * 32;
-  const int i = threadIdx.x & 31, eg = threadIdx.x >> 5;
-  for (int e = eg; e < E; e += 8) {
-    float acc = 0.f;
-    const int u0 = offsets[e], u1 = offsets[e + 1];
+  const int e = blockIdx.x;
+  const int u0 = offsets[e], u1 = offsets[e + 1];
+  for (int i = threadIdx.x * 8; i < d; i += blockDim.x * 8) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int u = u0; u < u1; ++u) {
       const int a = __ldg(perm_asg + u);
       const float w = __ldg(dlasg + a);
-      acc = fmaf(w, __bfloat162float(X[static_cast<size_t>(a / k) * d + i0 + i]), acc);
+      const uint4 x = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(a / k) * d + i));
+      float2 f;
+      f = unpack_bf16(x.x); acc[0] = fmaf(w, f.x, acc[0]); acc[1] = fmaf(w, f.y, acc[1]);
+      f = unpack_bf16(x.y); acc[2] = fmaf(w, f.x, acc[2]); acc[3] = fmaf(w, f.y, acc[3]);
+      f = unpack_bf16(x.z); acc[4] = fmaf(w, f.x, acc[4]); acc[5] = fmaf(w, f.y, acc[5]);
+      f = unpack_bf16(x.w); acc[6] = fmaf(w, f.x, acc[6]); acc[7] = fmaf(w, f.y, acc[7]);
     }
-    sacc[i * (E + 1) + e] = acc;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) dWr[static_cast<size_t>(i + q) * E + e] = acc[q];
   }
-  __syncthreads();
-  for (int r = 0; r < 32; ++r)
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
-      dWr[static_cast<size_t>(i0 + r) * E + e] = sacc[r * (E + 1) + e];
 }
 
 // local views of the routing table for the test hook
@@ -401,15 +363,9 @@ __global__ void k_export_routing(const int* __restrict__ counts, const int* __re
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-cudaError_t launch_router_logits(const Layout& L, const __nv_bfloat16* X, const __nv_bfloat16* W_r,
-                                 const float* bias, float* logits, cudaStream_t st) {
-  dim3 grid((L.E + 63) / 64, static_cast<unsigned>((L.T + 63) / 64));
-  k_router_logits<<<grid, 256, 0, st>>>(X, W_r, bias, logits, static_cast<int>(L.T), L.d, L.E);
-  return cudaGetLastError();
-}
-cudaError_t launch_topk(const Layout& L, const Ctx& c, cudaStream_t st) {
-  k_topk<<<L.nblk, kTokensPerBlock * 32, 0, st>>>(c.logits, static_cast<int>(L.T), L.E, L.k, c.ids, c.gates, c.hist,
-                                                  c.hdr + HDR_STATUS);
+cudaError_t launch_topk(const Layout& L, const Ctx& c, const float* bias, int splits, cudaStream_t st) {
+  k_topk<<<L.nblk, kTokensPerBlock * 32, 0, st>>>(c.rpart, splits, bias, c.logits, static_cast<int>(L.T), L.E, L.k,
+                                                  c.ids, c.gates, c.hist, c.hdr + HDR_STATUS);
   return cudaGetLastError();
 }
 cudaError_t launch_scan(const Layout& L, const Ctx& c, cudaStream_t st) {
@@ -449,15 +405,7 @@ cudaError_t launch_rev_dispatch(const Layout& L, const Ctx& c, __nv_bfloat16* dX
   return cudaGetLastError();
 }
 cudaError_t launch_dwr(const Layout& L, const Ctx& c, const __nv_bfloat16* X, float* dW_r, cudaStream_t st) {
-  const size_t smem = 32 * static_cast<size_t>(L.E + 1) * sizeof(float);
-  static bool configured = false;
-  if (!configured) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(k_dwr, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * (kMaxE + 1) * 4);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  k_dwr<<<L.d / 32, 256, smem, st>>>(X, c.offsets, c.perm_asg, c.dlasg, L.d, L.E, L.k, dW_r);
+  k_dwr<<<L.E, 256, 0, st>>>(X, c.offsets, c.perm_asg, c.dlasg, L.d, L.E, L.k, dW_r);
   return cudaGetLastError();
 }
 cudaError_t launch_export_routing(const Layout& L, const Ctx& c, int32_t* counts, int32_t* offsets, int32_t* poff,

@@ -10,6 +10,7 @@ Workloads (the pages name model families and print no shapes; these stand in):
 * ``kimi``      T=4096, d=7168, E=384, k=8, I=2048   (Kimi-K2-like, Zipf(1.2)-skewed load)
 * ``kimi_mx``   ``kimi`` in MXFP8 mode
 * ``ep64``      6 local experts of 384, 16 minibatches x 2048 tokens, ring buffer
+* ``dsv3_e16``  the dsv3 expert shape with 16 experts and 128 tokens (profiler captures)
 
 Distributions: X, dY ~ N(0, 1); W_gate, W_up ~ N(0, 1/d) (std 1/sqrt(fan_in));
 W_down ~ N(0, 1/I); W_r ~ N(0, 0.02^2); every tensor rounded once to bf16 (RNE).
@@ -54,6 +55,9 @@ WORKLOADS = {
     "dsv3": Workload("dsv3", 2048, 7168, 256, 8, 2048),
     "kimi": Workload("kimi", 4096, 7168, 384, 8, 2048, zipf=True),
     "kimi_mx": Workload("kimi_mx", 4096, 7168, 384, 8, 2048, mxfp8=True, zipf=True),
+    # the dsv3 expert shape and load (64 tokens per expert) with 16 experts: a
+    # ~3 GB case for profiler captures (weights still exceed the 126 MB L2)
+    "dsv3_e16": Workload("dsv3_e16", 128, 7168, 16, 8, 2048),
 }
 
 
