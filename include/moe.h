@@ -144,6 +144,29 @@ int moe_profile_read(int max_kernels, double* total_ms, int* launches);
 const char* moe_kernel_name(int kernel_id);
 unsigned long long moe_kernel_launches(void);
 
+/* Router GEMM + top-k gating that allocates nothing.  The pages have no
+ * counterpart of this call: it exists for callers that must not allocate
+ * device memory while they run -- code executing inside an allocator or
+ * memory-planner callback (where cudaMalloc would re-enter the allocator), or
+ * a service whose device memory was all handed to its own pool at start-up.
+ *   X [T, d] bf16, W_r [d, E] bf16, bias [E] fp32 or NULL     (inputs)
+ *   ids [T, k] int32, gates [T, k] fp32                       (outputs: the same
+ *       values moe_fwd puts in its routing table)
+ *   status: one int32 in device memory, or NULL; cleared, then set to a
+ *       moe_status code by a device-side error (non-finite logit, timeout)
+ * Its scratch (W_r transposed, split-K partial logits, logits, per-block
+ * histograms) is a static device array of MOE_STATIC_SCRATCH_BYTES = 32 MiB
+ * inside the library; every GPU that loads the library holds it until the
+ * process exits.  Shapes needing more (about E*d*2 + (S+1)*T*E*4 +
+ * ceil(T/16)*E*4 bytes, S = K splits of the router GEMM) are refused with
+ * MOE_ERR_WORKSPACE_TOO_SMALL.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  The call allocates
+ * nothing and never synchronises.  All calls share the one array: calls that
+ * overlap on the GPU race on it and must be serialised by the caller. */
+moe_status moe_route_static(const moe_shape* shape, const void* X, const void* W_r, const float* bias,
+                            int32_t* ids, float* gates, int32_t* status, void* stream);
+
 /* Static string naming a status code. */
 const char* moe_status_string(moe_status status);
 

@@ -57,6 +57,7 @@ _SIGS = {
     "moe_profile_read": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
     "moe_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_kernel_launches": (ctypes.c_ulonglong, []),
+    "moe_route_static": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P]),
 }
 
 
@@ -157,6 +158,12 @@ def moe_kernel_name(kernel_id: int) -> str:
 
 def moe_kernel_launches() -> int:
     return int(lib().moe_kernel_launches())
+
+
+def moe_route_static(shape, X, W_r, bias, ids, gates, status=None, stream=None) -> int:
+    """Router + top-k gating with the library's static scratch (no allocation)."""
+    return int(lib().moe_route_static(ctypes.byref(shape), _ptr(X), _ptr(W_r), _ptr(bias), _ptr(ids), _ptr(gates),
+                                      _ptr(status), _stream(stream)))
 
 
 def check(status: int, what: str = "moe"):
