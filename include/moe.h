@@ -130,6 +130,11 @@ moe_status moe_debug_routing(const moe_shape* shape, const void* ctx, int32_t* i
  * moe_fwd computed in `ws` into `logits` (device pointer). */
 moe_status moe_debug_logits(const moe_shape* shape, const void* ws, float* logits, void* stream);
 
+/* Test hook: copies the router-logit gradient of the last moe_bwd that used
+ * `ws` into `dl` [T, k] fp32 (device pointer): dl[t, j] = dL/dl_{t, ids[t, j]},
+ * the only nonzeros of dL/dlogits (dW_r = X^T dl scattered to the ids). */
+moe_status moe_debug_router_grad(const moe_shape* shape, const void* ws, float* dl, void* stream);
+
 /* Benchmark support (no counterpart on the pages).  When enabled, every
  * kernel launch of the library is bracketed by two CUDA events recorded on the
  * launch stream.  moe_profile_read synchronises the device, writes per kernel

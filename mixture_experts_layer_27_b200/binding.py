@@ -52,6 +52,7 @@ _SIGS = {
     "moe_get_error": (ctypes.c_int, [_P, _P]),
     "moe_debug_routing": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_debug_logits": (ctypes.c_int, [_S, _P, _P, _P]),
+    "moe_debug_router_grad": (ctypes.c_int, [_S, _P, _P, _P]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
     "moe_profile_read": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
@@ -136,6 +137,10 @@ def moe_debug_routing(shape, ctx, ids=None, gates=None, counts=None, offsets=Non
 
 def moe_debug_logits(shape, ws, logits, stream=None) -> int:
     return int(lib().moe_debug_logits(ctypes.byref(shape), _ptr(ws), _ptr(logits), _stream(stream)))
+
+
+def moe_debug_router_grad(shape, ws, dl, stream=None) -> int:
+    return int(lib().moe_debug_router_grad(ctypes.byref(shape), _ptr(ws), _ptr(dl), _stream(stream)))
 
 
 def moe_profile_enable(on: bool) -> int:
@@ -227,6 +232,12 @@ class MoELayer:
         import torch
         out = torch.empty(self.T, self.E, dtype=torch.float32, device=self.ws.device)
         check(moe_debug_logits(self.shape, self.ws, out), "moe_debug_logits")
+        return out
+
+    def router_grad(self):
+        import torch
+        out = torch.empty(self.T, self.k, dtype=torch.float32, device=self.ws.device)
+        check(moe_debug_router_grad(self.shape, self.ws, out), "moe_debug_router_grad")
         return out
 
     def error(self, stream=None) -> int:

@@ -496,12 +496,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
 
 template <int KIND>
 static cudaError_t launch_kind(const GemmParams& p, int grid, cudaStream_t st) {
-  static bool configured = false;
-  if (!configured) {
+  static bool configured[64] = {};  // the attribute is set once per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
     const cudaError_t e = cudaFuncSetAttribute(k_moe_gemm<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem_bytes<KIND>()));
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured[dev] = true;
   }
   k_moe_gemm<KIND><<<grid, GEMM_THREADS, smem_bytes<KIND>(), st>>>(p);
   return cudaGetLastError();

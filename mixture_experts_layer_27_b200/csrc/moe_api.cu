@@ -510,6 +510,17 @@ moe_status moe_debug_routing(const moe_shape* s, const void* ctx, int32_t* ids, 
   return MOE_OK;
 }
 
+moe_status moe_debug_router_grad(const moe_shape* s, const void* ws, float* dl, void* stream) {
+  Layout L;
+  const moe_status cs = check_shape(s, &L);
+  if (cs != MOE_OK) return cs;
+  if (!ws || !dl) return MOE_ERR_INVALID_ARG;
+  if (L.T == 0) return MOE_OK;
+  MOE_TRY(cudaMemcpyAsync(dl, static_cast<const char*>(ws) + L.dlasg, static_cast<size_t>(L.T) * L.k * 4,
+                          cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
 moe_status moe_debug_logits(const moe_shape* s, const void* ws, float* logits, void* stream) {
   Layout L;
   const moe_status cs = check_shape(s, &L);

@@ -1,0 +1,125 @@
+"""Full-size parity: the bench workloads, in the launch configuration bench.py times.
+
+The oracle cannot run the whole layer at these sizes in seconds, so it checks
+what it can compute one piece at a time:
+
+* routing table: bit-exact against the oracle's selection on the GPU's fp32
+  logits (all T tokens); against the oracle's own fp64 logits, every token
+  whose ids differ must be a near-tie in fp64;
+* Y, dX and the router gradient dl at sampled tokens (each depends on that
+  token's data alone);
+* dW_gate, dW_up, dW_down of sampled experts (each depends on that expert's
+  tokens alone);
+* dW_r in full against X^T dl computed in fp64 from the GPU's own dl, whose
+  sampled rows were checked against the oracle;
+* a second run is bit-identical.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from mixture_experts_layer_27_b200 import binding as B
+from mixture_experts_layer_27_b200 import inputs as IN
+
+from _util import TOL_BF16, relerr, to64
+
+pytestmark = pytest.mark.gpu
+
+
+class ExpertCache:
+    """fp64 host copies of single experts' weights, fetched on demand (last few kept)."""
+
+    def __init__(self, W, keep=2):
+        self.W, self.keep, self.cache = W, keep, {}
+
+    def __call__(self, e):
+        e = int(e)
+        if e not in self.cache:
+            if len(self.cache) >= self.keep:
+                self.cache.pop(next(iter(self.cache)))
+            self.cache[e] = to64(self.W[e])
+        return self.cache[e]
+
+
+def _run(w, x):
+    layer = B.MoELayer(w.T, w.d, w.E, w.I, w.k)
+    Y = layer.forward(x["X"], x["W_r"], x["bias"], x["W_gate"], x["W_up"], x["W_down"])
+    g = layer.backward(x["X"], x["W_r"], x["W_gate"], x["W_up"], x["W_down"], x["dY"])
+    torch.cuda.synchronize()
+    assert layer.error() == B.MOE_OK
+    return layer, Y, g
+
+
+@pytest.mark.parametrize("name", ["dsv3", "kimi"])
+def test_full_size_workload(name):
+    w = IN.WORKLOADS[name]
+    x = IN.make_inputs(w, device="cuda")
+    layer, Y, g = _run(w, x)
+    r = layer.routing()
+    lg_gpu = to64(layer.logits())
+    X, Wr = to64(x["X"]), to64(x["W_r"])
+    b = None if x["bias"] is None else to64(x["bias"])
+
+    # -- routing table, bit-exact on the GPU's logits
+    ids = O.topk_ids(lg_gpu, w.k)
+    s = O.schedule(ids, w.E)
+    gids = r["ids"].cpu().numpy()
+    assert np.array_equal(gids, ids)
+    for key in ("counts", "offsets", "padded_offsets", "perm", "slot_row"):
+        assert np.array_equal(r[key].cpu().numpy(), s[key]), key
+    assert np.max(np.abs(r["gates"].cpu().numpy() - O.gates(lg_gpu, ids))) < 1e-6
+
+    # -- against fp64 logits: differences only at near-ties
+    lg64 = O.router_logits(X, Wr, b)
+    ids64 = O.topk_ids(lg64, w.k)
+    srt = -np.sort(-lg64, axis=1)
+    gap = srt[:, w.k - 1] - srt[:, w.k]
+    differ = np.nonzero(np.any(np.sort(ids64, 1) != np.sort(gids, 1), axis=1))[0]
+    near = gap < 1e-3
+    assert np.all(near[differ]), (differ, gap[differ])
+    tie_tokens = set(differ.tolist())
+
+    # -- Y, dX at sampled tokens
+    Wg, Wu, Wd = ExpertCache(x["W_gate"]), ExpertCache(x["W_up"]), ExpertCache(x["W_down"])
+    dY = to64(x["dY"])
+    rng = np.random.default_rng(1234)
+    toks = [t for t in rng.choice(w.T, size=12, replace=False).tolist() if t not in tie_tokens][:8]
+    Yg, dXg = to64(Y), to64(g["dX"])
+    dl_gpu = to64(layer.router_grad())  # [T, k], slot order of the GPU's ids
+    ys, yo, dxs, dxo, dls, dlo = [], [], [], [], [], []
+    for t in toks:
+        y, dx, dl, tid, gt = O.token_forward_backward(t, X, Wr, b, Wg, Wu, Wd, w.k, dY)
+        ys.append(Yg[t]); yo.append(y); dxs.append(dXg[t]); dxo.append(dx)
+        dls.append(dl_gpu[t]); dlo.append(dl[gids[t]])
+    assert relerr(np.array(ys), np.array(yo)) <= TOL_BF16
+    assert relerr(np.array(dxs), np.array(dxo)) <= TOL_BF16
+    assert relerr(np.array(dls), np.array(dlo)) <= TOL_BF16
+
+    # -- dW_r in full: X^T dl in fp64 from the GPU's (sampled-checked) dl
+    dl_dense = np.zeros((w.T, w.E))
+    np.put_along_axis(dl_dense, gids.astype(np.int64), dl_gpu, axis=1)
+    assert relerr(to64(g["dW_r"]), X.T @ dl_dense) <= 1e-4
+
+    # -- expert weight gradients for the hottest and the coldest non-empty expert
+    counts = r["counts"].cpu().numpy()
+    nz = np.nonzero(counts)[0]
+    hot, cold = int(nz[np.argmax(counts[nz])]), int(nz[np.argmin(counts[nz])])
+    for e in sorted({hot, cold}):
+        _, ctx = O.forward(X, Wr, b, Wg, Wu, Wd, w.k, first_local=e, num_local=1)
+        ctx_tokens = set(ctx["sched"]["perm"].tolist())
+        if ctx_tokens & tie_tokens:
+            continue  # a near-tie token changes this expert's token set between fp32 and fp64
+        go = O.backward(ctx, dY)
+        assert relerr(to64(g["dW_gate"][e]), go["dW_gate"][e]) <= TOL_BF16, e
+        assert relerr(to64(g["dW_up"][e]), go["dW_up"][e]) <= TOL_BF16, e
+        assert relerr(to64(g["dW_down"][e]), go["dW_down"][e]) <= TOL_BF16, e
+
+    # -- bit-identical second run
+    _, Y2, g2 = _run(w, x)
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+    for n in ("dX", "dW_gate", "dW_up", "dW_down"):
+        assert torch.equal(g[n].view(torch.int16), g2[n].view(torch.int16)), n
+    assert torch.equal(g["dW_r"].view(torch.int32), g2["dW_r"].view(torch.int32))
+    del layer, Y, g, Y2, g2, x
+    torch.cuda.empty_cache()
