@@ -87,6 +87,32 @@ def algorithmic_bytes(w: IN.Workload) -> dict:
     }
 
 
+# DRAM bytes per launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum),
+# scaled to the workload by the units processed; see profiles/ncu_gemm_gateup_wgrad_dsv3_e16.md.
+# A figure is reported only while the GEMM sources still hash to the value they had
+# when the counters were taken.
+NCU_TRAFFIC = {
+    ("gemm_wgrad_gateup", "dsv3"): (925.3e6 * 16, "80ff2ed0ecc526b0"),
+}
+GEMM_SOURCES = ("gemm.cu", "ptx.cuh", "moe_internal.cuh")
+
+
+def gemm_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for n in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "mixture_experts_layer_27_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    t = NCU_TRAFFIC.get((kernel, workload))
+    if t is None or t[1] != gemm_source_hash():
+        return None
+    return t[0]
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples while the timed region runs."""
 
@@ -363,7 +389,7 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     ach = kern[top].get("achieved_GBs")
     roof = {"kernel": top, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
-            "frac": (ach / hbm) if ach else None, "traffic": None,
+            "frac": (ach / hbm) if ach else None, "traffic": ncu_traffic(top, w.name),
             "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
             if peak_kind == "measured" else "fallback 6.65 TB/s"}
     bf16 = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))

@@ -321,29 +321,53 @@ __global__ void __launch_bounds__(128) k_rev_dispatch(const __nv_bfloat16* __res
 // ---------------------------------------------------------------------------
 // dW_r[:, e] = sum over the assignments (t, j) routed to e, in the table's
 // order (ascending t), of dl_tj X[t, :].  dl has k nonzeros per token, so this
-// is the sparse form of X^T dl.  One block per expert; each thread owns eight
-// consecutive columns of d and reads X rows with 16-byte loads.
+// is the sparse form of X^T dl.  Block = (expert, 256 columns of d); its four
+// warps take fixed quarters of the expert's assignment list, each lane eight
+// columns, and the quarters are added in warp order: the result does not
+// depend on scheduling.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_dwr(const __nv_bfloat16* __restrict__ X, const int* __restrict__ offsets,
+__device__ __forceinline__ void axpy8(float w, const uint4& x, float (&acc)[8]) {
+  float2 f;
+  f = unpack_bf16(x.x); acc[0] = fmaf(w, f.x, acc[0]); acc[1] = fmaf(w, f.y, acc[1]);
+  f = unpack_bf16(x.y); acc[2] = fmaf(w, f.x, acc[2]); acc[3] = fmaf(w, f.y, acc[3]);
+  f = unpack_bf16(x.z); acc[4] = fmaf(w, f.x, acc[4]); acc[5] = fmaf(w, f.y, acc[5]);
+  f = unpack_bf16(x.w); acc[6] = fmaf(w, f.x, acc[6]); acc[7] = fmaf(w, f.y, acc[7]);
+}
+
+__global__ void __launch_bounds__(128) k_dwr(const __nv_bfloat16* __restrict__ X, const int* __restrict__ offsets,
                                              const int* __restrict__ perm_asg, const float* __restrict__ dlasg,
                                              int d, int E, int k, float* __restrict__ dWr) {
-  const int e = blockIdx.x;
-  const int u0 = offsets[e], u1 = offsets[e + 1];
-  for (int i = threadIdx.x * 8; i < d; i += blockDim.x * 8) {
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int u = u0; u < u1; ++u) {
-      const int a = __ldg(perm_asg + u);
-      const float w = __ldg(dlasg + a);
-      const uint4 x = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(a / k) * d + i));
-      float2 f;
-      f = unpack_bf16(x.x); acc[0] = fmaf(w, f.x, acc[0]); acc[1] = fmaf(w, f.y, acc[1]);
-      f = unpack_bf16(x.y); acc[2] = fmaf(w, f.x, acc[2]); acc[3] = fmaf(w, f.y, acc[3]);
-      f = unpack_bf16(x.z); acc[4] = fmaf(w, f.x, acc[4]); acc[5] = fmaf(w, f.y, acc[5]);
-      f = unpack_bf16(x.w); acc[6] = fmaf(w, f.x, acc[6]); acc[7] = fmaf(w, f.y, acc[7]);
+  __shared__ float part[4][256];
+  const int e = blockIdx.x, i0 = blockIdx.y * 256;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u0 = offsets[e], n = offsets[e + 1] - u0;
+  const int q0 = u0 + (n * warp) / 4, q1 = u0 + (n * (warp + 1)) / 4;
+  const int col = i0 + lane * 8;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int u = q0;
+  for (; u + 4 <= q1; u += 4) {  // four independent rows in flight
+    int a[4];
+    float w[4];
+    uint4 x[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) a[j] = __ldg(perm_asg + u + j);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      w[j] = __ldg(dlasg + a[j]);
+      x[j] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(a[j] / k) * d + col));
     }
 #pragma unroll
-    for (int q = 0; q < 8; ++q) dWr[static_cast<size_t>(i + q) * E + e] = acc[q];
+    for (int j = 0; j < 4; ++j) axpy8(w[j], x[j], acc);
   }
+  for (; u < q1; ++u) {
+    const int a = __ldg(perm_asg + u);
+    axpy8(__ldg(dlasg + a), __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(a / k) * d + col)), acc);
+  }
+#pragma unroll
+  for (int q = 0; q < 8; ++q) part[warp][lane * 8 + q] = acc[q];
+  __syncthreads();
+  for (int c = threadIdx.x; c < 256; c += blockDim.x)
+    dWr[static_cast<size_t>(i0 + c) * E + e] = ((part[0][c] + part[1][c]) + part[2][c]) + part[3][c];
 }
 
 // local views of the routing table for the test hook
@@ -405,7 +429,7 @@ cudaError_t launch_rev_dispatch(const Layout& L, const Ctx& c, __nv_bfloat16* dX
   return cudaGetLastError();
 }
 cudaError_t launch_dwr(const Layout& L, const Ctx& c, const __nv_bfloat16* X, float* dW_r, cudaStream_t st) {
-  k_dwr<<<L.E, 256, 0, st>>>(X, c.offsets, c.perm_asg, c.dlasg, L.d, L.E, L.k, dW_r);
+  k_dwr<<<dim3(L.E, L.d / 256), 128, 0, st>>>(X, c.offsets, c.perm_asg, c.dlasg, L.d, L.E, L.k, dW_r);
   return cudaGetLastError();
 }
 cudaError_t launch_export_routing(const Layout& L, const Ctx& c, int32_t* counts, int32_t* offsets, int32_t* poff,
