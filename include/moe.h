@@ -149,6 +149,50 @@ int moe_profile_read(int max_kernels, double* total_ms, int* launches);
 const char* moe_kernel_name(int kernel_id);
 unsigned long long moe_kernel_launches(void);
 
+/* ---------------------------------------------------------------------------
+ * Ring-streamed layer (page 1, "Three design decisions that matter", bullet 3:
+ * a fixed ring token buffer cycled at minibatch granularity, dispatch and
+ * combine interleaved at macrobatch boundaries, walked in reverse in the
+ * backward so that little forward activation has to be replayed).
+ *
+ * One call processes M minibatches of shape->T tokens each (X, Y, dY, dX are
+ * [M*T, d]).  The result is the layer of moe_fwd / moe_bwd over all M*T tokens;
+ * only where the dispatched token rows (X_perm) live changes: in the caller's
+ * ring of ring_bytes (ring_bytes / (2 d) rows) instead of ctx.
+ *   - The device groups consecutive minibatches into macrobatches: a macrobatch
+ *     closes once its padded rows give the gate/up grouped GEMM two full waves
+ *     of 128 x 256 tiles ((rows / 128) * (I / 128) >= 2 * SMs), or before a
+ *     minibatch that would not fit in the ring with it.
+ *   - Forward: each macrobatch's rows are dispatched at the ring's write
+ *     pointer (a segment that would run past the end restarts at row 0), then
+ *     its grouped GEMMs and its combine run.
+ *   - Backward: the dgrad path runs over all rows; the gate/up weight gradient
+ *     walks the macrobatches in reverse, reusing those still intact in the ring
+ *     and re-dispatching (replaying) older ones chunk by chunk.
+ * No host synchronisation and no dropped tokens: all sizes are decided on the
+ * device; the host enqueues a fixed number of launches per minibatch.
+ * Requirements: shape->T a multiple of 16; 1 <= M <= 256; ring_bytes at least
+ * moe_stream_min_ring_bytes(shape) (one minibatch's worst case), else
+ * MOE_ERR_WORKSPACE_TOO_SMALL.  bf16 only. */
+size_t moe_stream_ctx_size(const moe_shape* shape, int32_t num_minibatches);
+size_t moe_stream_workspace_size(const moe_shape* shape, int32_t num_minibatches);
+size_t moe_stream_min_ring_bytes(const moe_shape* shape);
+moe_status moe_fwd_stream(const moe_shape* shape, int32_t num_minibatches, const void* X, const void* W_r,
+                          const float* bias, const void* W_gate, const void* W_up, const void* W_down, void* Y,
+                          void* ctx, size_t ctx_bytes, void* ring, size_t ring_bytes, void* ws, size_t ws_bytes,
+                          void* stream);
+moe_status moe_bwd_stream(const moe_shape* shape, int32_t num_minibatches, const void* X, const void* W_r,
+                          const void* W_gate, const void* W_up, const void* W_down, const void* dY, void* ctx,
+                          size_t ctx_bytes, void* dX, void* dW_gate, void* dW_up, void* dW_down, float* dW_r,
+                          void* ring, size_t ring_bytes, void* ws, size_t ws_bytes, void* stream);
+/* Test hook: copies the plan of the last moe_fwd_stream (int32 words, device
+ * pointer): [16 header words: macrobatches, backward chunks, padded rows,
+ * replayed rows, resident rows, ring rows, 0...] then mb_of[M],
+ * seg_poff[M*El+1], cum[M*El], mb_range[2M], shift_fwd[M], shift_bwd[M],
+ * replay[M], chunk[4M] ({m_lo, m_hi, valid, mode}), ring_start[M]. */
+moe_status moe_debug_stream_plan(const moe_shape* shape, int32_t num_minibatches, const void* ctx, int32_t* tables,
+                                 void* stream);
+
 /* Router GEMM + top-k gating that allocates nothing.  The pages have no
  * counterpart of this call: it exists for callers that must not allocate
  * device memory while they run -- code executing inside an allocator or

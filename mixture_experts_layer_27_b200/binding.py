@@ -59,6 +59,14 @@ _SIGS = {
     "moe_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_kernel_launches": (ctypes.c_ulonglong, []),
     "moe_route_static": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_stream_ctx_size": (ctypes.c_size_t, [_S, ctypes.c_int32]),
+    "moe_stream_workspace_size": (ctypes.c_size_t, [_S, ctypes.c_int32]),
+    "moe_stream_min_ring_bytes": (ctypes.c_size_t, [_S]),
+    "moe_fwd_stream": (ctypes.c_int, [_S, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P,
+                                      ctypes.c_size_t, _P, ctypes.c_size_t, _P]),
+    "moe_bwd_stream": (ctypes.c_int, [_S, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, _P,
+                                      _P, _P, _P, ctypes.c_size_t, _P, ctypes.c_size_t, _P]),
+    "moe_debug_stream_plan": (ctypes.c_int, [_S, ctypes.c_int32, _P, _P, _P]),
 }
 
 
@@ -171,9 +179,97 @@ def moe_route_static(shape, X, W_r, bias, ids, gates, status=None, stream=None) 
                                       _ptr(status), _stream(stream)))
 
 
+def moe_stream_ctx_size(shape, M) -> int:
+    return int(lib().moe_stream_ctx_size(ctypes.byref(shape), int(M)))
+
+
+def moe_stream_workspace_size(shape, M) -> int:
+    return int(lib().moe_stream_workspace_size(ctypes.byref(shape), int(M)))
+
+
+def moe_stream_min_ring_bytes(shape) -> int:
+    return int(lib().moe_stream_min_ring_bytes(ctypes.byref(shape)))
+
+
+def moe_fwd_stream(shape, M, X, W_r, bias, W_gate, W_up, W_down, Y, ctx, ring, ws, stream=None):
+    return int(lib().moe_fwd_stream(ctypes.byref(shape), int(M), _ptr(X), _ptr(W_r), _ptr(bias), _ptr(W_gate),
+                                    _ptr(W_up), _ptr(W_down), _ptr(Y), _ptr(ctx), _nbytes(ctx), _ptr(ring),
+                                    _nbytes(ring), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def moe_bwd_stream(shape, M, X, W_r, W_gate, W_up, W_down, dY, ctx, dX, dW_gate, dW_up, dW_down, dW_r, ring, ws,
+                   stream=None):
+    return int(lib().moe_bwd_stream(ctypes.byref(shape), int(M), _ptr(X), _ptr(W_r), _ptr(W_gate), _ptr(W_up),
+                                    _ptr(W_down), _ptr(dY), _ptr(ctx), _nbytes(ctx), _ptr(dX), _ptr(dW_gate),
+                                    _ptr(dW_up), _ptr(dW_down), _ptr(dW_r), _ptr(ring), _nbytes(ring), _ptr(ws),
+                                    _nbytes(ws), _stream(stream)))
+
+
+def moe_debug_stream_plan(shape, M, ctx, tables, stream=None) -> int:
+    return int(lib().moe_debug_stream_plan(ctypes.byref(shape), int(M), _ptr(ctx), _ptr(tables), _stream(stream)))
+
+
 def check(status: int, what: str = "moe"):
     if status != MOE_OK:
         raise MoeError(status, what)
+
+
+class MoEStream:
+    """ctx / ring / workspace owner for the ring-streamed layer (M minibatches of T tokens)."""
+
+    def __init__(self, T, d, E, I, top_k, M, ring_bytes, first_local_expert=0, num_local_experts=0, device="cuda"):
+        import torch
+        self.shape = make_shape(T, d, E, I, top_k, MOE_BF16, first_local_expert, num_local_experts)
+        nc, nw = moe_stream_ctx_size(self.shape, M), moe_stream_workspace_size(self.shape, M)
+        if nc == 0 or nw == 0:
+            raise MoeError(MOE_ERR_UNSUPPORTED, "stream shape")
+        self.ctx = torch.empty(nc, dtype=torch.uint8, device=device)
+        self.ws = torch.empty(nw, dtype=torch.uint8, device=device)
+        self.ring = torch.empty(ring_bytes, dtype=torch.uint8, device=device)
+        self.T, self.d, self.E, self.I, self.k, self.M = T, d, E, I, top_k, M
+        self.El = num_local_experts or (E - first_local_expert)
+
+    def forward(self, X, W_r, bias, W_gate, W_up, W_down, Y=None, stream=None):
+        import torch
+        if Y is None:
+            Y = torch.empty(self.M * self.T, self.d, dtype=torch.bfloat16, device=X.device)
+        check(moe_fwd_stream(self.shape, self.M, X, W_r, bias, W_gate, W_up, W_down, Y, self.ctx, self.ring,
+                             self.ws, stream), "moe_fwd_stream")
+        return Y
+
+    def backward(self, X, W_r, W_gate, W_up, W_down, dY, out=None, stream=None):
+        import torch
+        if out is None:
+            dev = X.device
+            out = dict(dX=torch.empty(self.M * self.T, self.d, dtype=torch.bfloat16, device=dev),
+                       dW_gate=torch.empty(self.El, self.d, self.I, dtype=torch.bfloat16, device=dev),
+                       dW_up=torch.empty(self.El, self.d, self.I, dtype=torch.bfloat16, device=dev),
+                       dW_down=torch.empty(self.El, self.I, self.d, dtype=torch.bfloat16, device=dev),
+                       dW_r=torch.empty(self.d, self.E, dtype=torch.float32, device=dev))
+        check(moe_bwd_stream(self.shape, self.M, X, W_r, W_gate, W_up, W_down, dY, self.ctx, out["dX"],
+                             out["dW_gate"], out["dW_up"], out["dW_down"], out["dW_r"], self.ring, self.ws, stream),
+              "moe_bwd_stream")
+        return out
+
+    def plan(self) -> dict:
+        """The device plan of the last forward, split into named tables (host numpy)."""
+        import torch
+        M, El = self.M, self.El
+        n = 16 + M + (M * El + 1) + M * El + 2 * M + 4 * M + 4 * M
+        t = torch.empty(n, dtype=torch.int32, device=self.ctx.device)
+        check(moe_debug_stream_plan(self.shape, M, self.ctx, t), "moe_debug_stream_plan")
+        torch.cuda.synchronize()
+        a = t.cpu().numpy()
+        out, o = {}, 0
+        for name, size in (("plan", 16), ("mb_of", M), ("seg_poff", M * El + 1), ("cum", M * El),
+                           ("mb_range", 2 * M), ("shift_fwd", M), ("shift_bwd", M), ("replay", M),
+                           ("chunk", 4 * M), ("ring_start", M)):
+            out[name] = a[o:o + size]
+            o += size
+        return out
+
+    def error(self, stream=None) -> int:
+        return moe_get_error(self.ctx, stream)
 
 
 class MoELayer:

@@ -46,6 +46,8 @@ constexpr size_t smem_bytes() {
 }
 
 struct Tile {
+  int m;    // macrobatch (wgrad: first macrobatch of the chunk)
+  int shift;  // row shift of the X_perm operand (ring position) / wgrad: last macrobatch + 1
   int el;   // local expert
   int m0;   // first output row (padded token row, or weight row for wgrad)
   int n0;   // first output column
@@ -66,9 +68,10 @@ __device__ __forceinline__ int mtiles_w(const GemmParams& p) {
   return KIND == G_WGRAD_GATEUP ? p.d / 128 : p.I / 128;
 }
 
-// Local expert whose padded segment [poff[e], poff[e+1]) holds row R.
-__device__ __forceinline__ int expert_of_row(const int* poff, int El, int R) {
-  int lo = 0, hi = El - 1;
+// Segment s with poff[s] <= R < poff[s+1] (the largest s with poff[s] <= R; empty
+// segments before a non-empty one are skipped because they share its start).
+__device__ __forceinline__ int segment_of_row(const int* poff, int nseg, int R) {
+  int lo = 0, hi = nseg - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (__ldg(poff + mid) <= R) lo = mid; else hi = mid - 1;
@@ -79,7 +82,8 @@ __device__ __forceinline__ int expert_of_row(const int* poff, int El, int R) {
 template <int KIND>
 __device__ __forceinline__ int num_tiles(const GemmParams& p) {
   if (KIND == G_ROUTER) return ((p.T + 127) / 128) * ((p.E + 255) / 256) * p.splits;
-  if (KIND <= G_DGRAD_GATEUP) return (__ldg(p.hdr + HDR_ROWS_P) / 128) * ntiles_n<KIND>(p);
+  if (KIND <= G_DGRAD_GATEUP) return ((__ldg(p.poff + p.nseg) - __ldg(p.poff)) / 128) * ntiles_n<KIND>(p);
+  if (p.chunk && __ldg(p.chunk + 2) == 0) return 0;  // chunk not used by this routing
   return p.El * mtiles_w<KIND>(p) * ntiles_n<KIND>(p);
 }
 
@@ -101,13 +105,17 @@ __device__ __forceinline__ Tile decode(const GemmParams& p, int t) {
   }
   const int NT = ntiles_n<KIND>(p);
   if constexpr (KIND <= G_DGRAD_GATEUP) {
-    // Tiles of expert e are [NT*poff[e]/128, NT*poff[e+1]/128), n-tile major so that
-    // the m-tiles of a hot expert sharing one weight tile run back to back.
-    const int el = expert_of_row(p.poff, p.El, (t / NT) * 128);
-    const int p0 = __ldg(p.poff + el), p1 = __ldg(p.poff + el + 1);
+    // Tiles of segment s are [NT*(poff[s]-poff[0])/128, NT*(poff[s+1]-poff[0])/128),
+    // n-tile major so that the m-tiles of a hot expert sharing one weight tile run back to back.
+    const int base = __ldg(p.poff);
+    const int seg = segment_of_row(p.poff, p.nseg, base + (t / NT) * 128);
+    const int p0 = __ldg(p.poff + seg), p1 = __ldg(p.poff + seg + 1);
     const int mte = (p1 - p0) / 128;
-    const int local = t - NT * (p0 / 128);
+    const int local = t - NT * ((p0 - base) / 128);
     const int nt = local / mte, mi = local - nt * mte;
+    const int el = seg % p.El;
+    tl.m = seg / p.El;
+    tl.shift = p.ring_shift ? __ldg(p.ring_shift + tl.m) : 0;
     tl.el = el;
     tl.m0 = p0 + mi * 128;
     tl.nt = nt;
@@ -115,16 +123,25 @@ __device__ __forceinline__ Tile decode(const GemmParams& p, int t) {
     tl.kb0 = 0;
     tl.nk = (KIND == G_GATEUP || KIND == G_DGRAD_DOWN) ? p.d / 64 : (KIND == G_DOWN ? p.I / 64 : 2 * p.I / 64);
   } else {
+    // contraction over the expert's rows in every macrobatch of the chunk, in order
     const int tpe = mtiles_w<KIND>(p) * NT;
     const int el = t / tpe, local = t - el * tpe;
     const int mt = local / NT, nt = local - mt * NT;
-    const int p0 = __ldg(p.poff + el), p1 = __ldg(p.poff + el + 1);
+    const int m_lo = p.chunk ? __ldg(p.chunk) : 0;
+    const int m_hi = p.chunk ? __ldg(p.chunk + 1) : p.nseg / p.El;
+    int nk = 0;
+    for (int m = m_lo; m < m_hi; ++m) {
+      const int s = m * p.El + el;
+      nk += (__ldg(p.poff + s + 1) - __ldg(p.poff + s)) / 64;
+    }
+    tl.m = m_lo;
+    tl.shift = m_hi;
     tl.el = el;
     tl.m0 = mt * 128;
     tl.nt = nt;
     tl.n0 = nt * 256;
-    tl.kb0 = p0 / 64;
-    tl.nk = (p1 - p0) / 64;
+    tl.kb0 = 0;
+    tl.nk = nk;
   }
   return tl;
 }
@@ -135,7 +152,7 @@ __device__ __forceinline__ void load_stage(const GemmParams& p, const Tile& tl, 
                                            uint64_t* bar, uint64_t pol_act, uint64_t pol_w) {
   const int k0 = kb * 64;
   if constexpr (KIND == G_GATEUP) {
-    tma_load_2d(sA, &p.ta0, bar, k0, tl.m0, pol_act);  // X_perm [rows, d] (K-major)
+    tma_load_2d(sA, &p.ta0, bar, k0, tl.m0 + tl.shift, pol_act);  // X_perm [rows, d] (K-major), maybe a ring
     const int krow = tl.el * p.d + k0;                 // W_gate / W_up as [El*d, I] (N contiguous)
     tma_load_2d(sB, &p.tb0, bar, tl.n0, krow, pol_w);
     tma_load_2d(sB + 8192, &p.tb0, bar, tl.n0 + 64, krow, pol_w);
@@ -157,25 +174,32 @@ __device__ __forceinline__ void load_stage(const GemmParams& p, const Tile& tl, 
       tma_load_2d(sA, &p.ta1, bar, k0 - p.I, tl.m0, pol_act);          // dB
       tma_load_2d(sB, &p.tb1, bar, k0 - p.I, tl.el * p.d + tl.n0, pol_w);  // W_up
     }
-  } else if constexpr (KIND == G_WGRAD_GATEUP) {
-    const int row = (tl.kb0 + kb) * 64;                                // contraction over padded rows
-    tma_load_2d(sA, &p.ta0, bar, tl.m0, row, pol_act);                 // X_perm, M = d (contiguous)
-    tma_load_2d(sA + 8192, &p.ta0, bar, tl.m0 + 64, row, pol_act);
-    const int NTg = p.I / 256;
-    const CUtensorMap* mb = tl.nt < NTg ? &p.tb0 : &p.tb1;             // dA for gate, dB for up
-    const int nb = (tl.nt < NTg ? tl.nt : tl.nt - NTg) * 256;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) tma_load_2d(sB + j * 8192, mb, bar, nb + 64 * j, row, pol_act);
   } else if constexpr (KIND == G_ROUTER) {
     const int kx = (tl.kb0 + kb) * 64;
     tma_load_2d(sA, &p.ta0, bar, kx, tl.m0, pol_act);  // X [T, d], rows >= T read as zero
     tma_load_2d(sB, &p.tb0, bar, kx, tl.n0, pol_act);  // W_r^T [E, d], rows >= E read as zero
-  } else {  // G_WGRAD_DOWN
-    const int row = (tl.kb0 + kb) * 64;
-    tma_load_2d(sA, &p.ta0, bar, tl.m0, row, pol_act);                 // Hg, M = I (contiguous)
-    tma_load_2d(sA + 8192, &p.ta0, bar, tl.m0 + 64, row, pol_act);
+  }
+}
+
+// wgrad: the 64-row K block starting at padded row `row`; X_perm rows live at row + xshift
+// (a ring position in the streamed backward).  Contraction over rows, so both operands
+// are MN-major: M = d (or I) and N = I (or d) are the contiguous dimensions.
+template <int KIND>
+__device__ __forceinline__ void load_wgrad(const GemmParams& p, const Tile& tl, int row, int xshift, uint8_t* sA,
+                                           uint8_t* sB, uint64_t* bar, uint64_t pol) {
+  if constexpr (KIND == G_WGRAD_GATEUP) {
+    tma_load_2d(sA, &p.ta0, bar, tl.m0, row + xshift, pol);            // X_perm
+    tma_load_2d(sA + 8192, &p.ta0, bar, tl.m0 + 64, row + xshift, pol);
+    const int NTg = p.I / 256;
+    const CUtensorMap* mb = tl.nt < NTg ? &p.tb0 : &p.tb1;             // dA for gate, dB for up
+    const int nb = (tl.nt < NTg ? tl.nt : tl.nt - NTg) * 256;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) tma_load_2d(sB + j * 8192, &p.tb0, bar, tl.n0 + 64 * j, row, pol_act);  // dY_perm
+    for (int j = 0; j < 4; ++j) tma_load_2d(sB + j * 8192, mb, bar, nb + 64 * j, row, pol);
+  } else {
+    tma_load_2d(sA, &p.ta0, bar, tl.m0, row, pol);                     // Hg, M = I
+    tma_load_2d(sA + 8192, &p.ta0, bar, tl.m0 + 64, row, pol);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tma_load_2d(sB + j * 8192, &p.tb0, bar, tl.n0 + 64 * j, row, pol);  // dY_perm
   }
 }
 
@@ -293,52 +317,111 @@ __device__ __forceinline__ void epilogue_row(const GemmParams& p, const Tile& tl
 }
 
 // wgrad epilogue: the warp's 32 x 256 slice of the output tile goes through a
-// 128B-swizzled staging buffer (four 32 x 64 boxes) and out by TMA stores.
+// 128B-swizzled staging buffer and out by TMA stores.  Mode (from the chunk
+// descriptor of a ring-streamed backward; 0 otherwise):
+//   0  bf16 dW (the whole contraction was in this launch)
+//   1  fp32 partial into the accumulator (first of several chunks)
+//   2  fp32: accumulator + this chunk's partial, back into the accumulator
+// Chunks run in a fixed order, so the sum is reproducible.
+__device__ __forceinline__ void stage_chunk16(uint8_t* box, int lane, int chunk, uint4 u) {
+  *reinterpret_cast<uint4*>(box + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = u;
+}
+
 template <int KIND>
 __device__ __forceinline__ void epilogue_wgrad(const GemmParams& p, const Tile& tl, int quarter, int lane,
                                                uint32_t taddr, uint8_t* stage_out) {
   const CUtensorMap* map;
-  int x0, y0;
+  int x0, y0, yacc = 0;
   if constexpr (KIND == G_WGRAD_GATEUP) {
     const int NTg = p.I / 256;
-    map = tl.nt < NTg ? &p.to0 : &p.to1;  // dW_gate or dW_up as [El*d, I]
-    x0 = (tl.nt < NTg ? tl.nt : tl.nt - NTg) * 256;
+    const int up = tl.nt < NTg ? 0 : 1;
+    map = up ? &p.to1 : &p.to0;  // dW_gate or dW_up as [El*d, I]
+    x0 = (tl.nt - up * NTg) * 256;
     y0 = tl.el * p.d + tl.m0 + quarter * 32;
+    yacc = (up * p.El + tl.el) * p.d + tl.m0 + quarter * 32;  // accumulator as [2*El*d, I] fp32
   } else {
     map = &p.to0;  // dW_down as [El*I, d]
     x0 = tl.n0;
     y0 = tl.el * p.I + tl.m0 + quarter * 32;
   }
-  if (lane == 0) bulk_wait_read0();  // the previous tile's stores have left the buffer
-  __syncwarp();
-  uint8_t* rowp = stage_out + lane * 128;
+  const int mode = (KIND == G_WGRAD_GATEUP && p.chunk) ? __ldg(p.chunk + 3) : 0;
+  if (mode == 0) {
+    if (lane == 0) bulk_wait_read0();  // the previous tile's stores have left the buffer
+    __syncwarp();
 #pragma unroll 1
-  for (int c = 0; c < 8; ++c) {
-    float v[32];
-    if (tl.nk > 0) {
-      tmem_ld32(taddr + c * 32, v);
-    } else {
+    for (int c = 0; c < 8; ++c) {
+      float v[32];
+      if (tl.nk > 0) {
+        tmem_ld32(taddr + c * 32, v);
+      } else {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = 0.f;  // expert without tokens: zero gradient
-    }
-    uint8_t* box = rowp + (c >> 1) * 4096;
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;  // expert without tokens: zero gradient
+      }
+      uint8_t* box = stage_out + (c >> 1) * 4096;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int chunk = (c & 1) * 4 + q;  // 16-byte chunk within the 128-byte row
-      uint4 u;
-      u.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
-      u.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
-      u.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
-      u.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
-      *reinterpret_cast<uint4*>(box + ((chunk ^ (lane & 7)) << 4)) = u;
+      for (int q = 0; q < 4; ++q) {
+        uint4 u;
+        u.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
+        u.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+        u.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+        u.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+        stage_chunk16(box, lane, (c & 1) * 4 + q, u);
+      }
     }
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0) {
+#pragma unroll
+      for (int b = 0; b < 4; ++b) tma_store_2d(map, stage_out + b * 4096, x0 + b * 64, y0);
+      bulk_commit();
+    }
+    return;
   }
-  fence_proxy_async();
-  __syncwarp();
-  if (lane == 0) {
+  // fp32 accumulator: two halves of 128 columns, four 32 x 32 fp32 boxes each
+  const float* prev = p.acc32 + static_cast<size_t>(yacc + lane) * p.I + x0;
+#pragma unroll 1
+  for (int h = 0; h < 2; ++h) {
+    if (lane == 0) bulk_wait_read0();
+    __syncwarp();
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      const int col = h * 128 + c * 32;
+      float v[32];
+      if (tl.nk > 0) {
+        tmem_ld32(taddr + col, v);
+      } else {
 #pragma unroll
-    for (int b = 0; b < 4; ++b) tma_store_2d(map, stage_out + b * 4096, x0 + b * 64, y0);
-    bulk_commit();
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      }
+      if (mode == 2) {
+        const float4* pv = reinterpret_cast<const float4*>(prev + col);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 o = pv[q];
+          v[4 * q + 0] = o.x + v[4 * q + 0];
+          v[4 * q + 1] = o.y + v[4 * q + 1];
+          v[4 * q + 2] = o.z + v[4 * q + 2];
+          v[4 * q + 3] = o.w + v[4 * q + 3];
+        }
+      }
+      uint8_t* box = stage_out + c * 4096;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        uint4 u;
+        u.x = __float_as_uint(v[4 * q + 0]);
+        u.y = __float_as_uint(v[4 * q + 1]);
+        u.z = __float_as_uint(v[4 * q + 2]);
+        u.w = __float_as_uint(v[4 * q + 3]);
+        stage_chunk16(box, lane, q, u);
+      }
+    }
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0) {
+#pragma unroll
+      for (int b = 0; b < 4; ++b) tma_store_2d(&p.tacc, stage_out + b * 4096, x0 + h * 128 + b * 32, yacc);
+      bulk_commit();
+    }
   }
 }
 
@@ -405,14 +488,31 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         const Tile tl = decode<KIND>(p, t);
-        for (int kb = 0; kb < tl.nk; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, p.status)) { ok = false; break; }
-          uint8_t* sA = smem + stage * GEMM_STAGE_BYTES;
-          uint8_t* sB = sA + GEMM_A_BYTES;
-          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(GEMM_STAGE_BYTES));
-          load_stage<KIND>(p, tl, kb, sA, sB, &full[stage], pol_act, pol_w);
-          last_parity[stage] = static_cast<int>(phase);
-          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        if constexpr (is_wgrad<KIND>()) {
+          // K runs over the expert's padded rows in each macrobatch of the chunk, in order
+          for (int m = tl.m; m < tl.shift && ok; ++m) {
+            const int sg = m * p.El + tl.el;
+            const int r0 = __ldg(p.poff + sg), r1 = __ldg(p.poff + sg + 1);
+            const int xs = (KIND == G_WGRAD_GATEUP && p.ring_shift) ? __ldg(p.ring_shift + m) : 0;
+            for (int row = r0; row < r1; row += 64) {
+              if (!mbar_wait(&empty[stage], phase ^ 1, p.status)) { ok = false; break; }
+              uint8_t* sA = smem + stage * GEMM_STAGE_BYTES;
+              mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(GEMM_STAGE_BYTES));
+              load_wgrad<KIND>(p, tl, row, xs, sA, sA + GEMM_A_BYTES, &full[stage], pol_act);
+              last_parity[stage] = static_cast<int>(phase);
+              if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+          }
+        } else {
+          for (int kb = 0; kb < tl.nk; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, p.status)) { ok = false; break; }
+            uint8_t* sA = smem + stage * GEMM_STAGE_BYTES;
+            uint8_t* sB = sA + GEMM_A_BYTES;
+            mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(GEMM_STAGE_BYTES));
+            load_stage<KIND>(p, tl, kb, sA, sB, &full[stage], pol_act, pol_w);
+            last_parity[stage] = static_cast<int>(phase);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
         }
       }
       if (!ok) {  // let copies already in flight land before the CTA's smem goes away

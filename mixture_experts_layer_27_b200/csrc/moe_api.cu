@@ -14,28 +14,35 @@ namespace moe {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-bool make_layout(const moe_shape& s, Layout* L) {
+bool make_layout(const moe_shape& s, Layout* L, int M) {
   if (s.T < 0 || s.d <= 0 || s.E <= 0 || s.I <= 0 || s.top_k <= 0) return false;
   if (s.E > kMaxE || s.top_k > kMaxK || s.top_k > s.E) return false;
   if (s.d % 256 || s.I % 256) return false;
   const int El = s.num_local_experts == 0 ? s.E - s.first_local_expert : s.num_local_experts;
   if (s.first_local_expert < 0 || El <= 0 || s.first_local_expert + El > s.E) return false;
-  if (s.T * static_cast<int64_t>(s.top_k) >= (int64_t(1) << 31)) return false;
-  L->T = s.T;
+  if (M < 0 || M > kMaxMinibatches) return false;
+  if (M > 0 && (s.T % kTokensPerBlock != 0 || s.T == 0)) return false;  // minibatches of whole token blocks
+  const int64_t T_all = M > 0 ? s.T * M : s.T;
+  if (T_all * static_cast<int64_t>(s.top_k) >= (int64_t(1) << 31)) return false;
+  L->T = T_all;
+  L->M = M;
+  L->T_mb = s.T;
   L->d = s.d;
   L->E = s.E;
   L->I = s.I;
   L->k = s.top_k;
   L->first = s.first_local_expert;
   L->El = El;
-  const int64_t A = s.T * s.top_k;
-  L->RP = static_cast<int64_t>(align_up(static_cast<size_t>(A + int64_t(kPad - 1) * El), kPad));
+  // a token has at most min(k, El) local assignments; every (macrobatch, expert) segment pads < 128 rows
+  const int64_t A = T_all * (s.top_k < El ? s.top_k : El);
+  const int64_t nseg = static_cast<int64_t>(El) * (M > 0 ? M : 1);
+  L->RP = static_cast<int64_t>(align_up(static_cast<size_t>(A + int64_t(kPad - 1) * nseg), kPad));
   if (L->RP < kPad) L->RP = kPad;
   if (L->RP * static_cast<int64_t>(s.d > s.I ? s.d : s.I) >= (int64_t(1) << 40)) return false;
-  L->nblk = static_cast<int>((s.T + kTokensPerBlock - 1) / kTokensPerBlock);
+  L->nblk = static_cast<int>((T_all + kTokensPerBlock - 1) / kTokensPerBlock);
   if (L->nblk < 1) L->nblk = 1;
 
-  const size_t RP = static_cast<size_t>(L->RP), T = static_cast<size_t>(s.T), k = s.top_k;
+  const size_t RP = static_cast<size_t>(L->RP), T = static_cast<size_t>(T_all), k = s.top_k;
   size_t o = 0;
   auto take = [&](size_t bytes) {
     const size_t at = o;
@@ -53,15 +60,16 @@ bool make_layout(const moe_shape& s, Layout* L) {
   L->slot_row = take(T * k * 4);
   L->row_asg = take(RP * 4);
   L->row_gate = take(RP * 4);
-  L->xperm = take(RP * s.d * 2);
+  L->xperm = take(M > 0 ? 0 : RP * s.d * 2);  // streamed layer: X_perm lives in the caller's ring
   L->abuf = take(RP * s.I * 2);
   L->bbuf = take(RP * s.I * 2);
+  L->stab = take(M > 0 ? static_cast<size_t>(stream_table_words(M, El)) * 4 : 0);
   L->ctx_bytes = o;
 
   o = 0;
   L->hist = take(static_cast<size_t>(L->nblk) * s.E * 4);
   L->logits = take(T * s.E * 4);
-  L->rpart = take(static_cast<size_t>(router_splits(s.T, s.E, s.d)) * T * s.E * 4);
+  L->rpart = take(static_cast<size_t>(router_splits(T_all, s.E, s.d)) * T * s.E * 4);
   L->hbuf = take(RP * s.I * 2);
   L->obuf = take(RP * s.d * 2);
   L->dyperm = take(RP * s.d * 2);
@@ -72,6 +80,7 @@ bool make_layout(const moe_shape& s, Layout* L) {
   L->dlasg = take(T * k * 4);
   L->wrt = take(static_cast<size_t>(s.E) * s.d * 2);
   L->dxperm = take(RP * s.d * 2);
+  L->acc32 = take(M > 0 ? 2 * static_cast<size_t>(El) * s.d * s.I * 4 : 0);
   L->ws_bytes = o;
   return true;
 }
@@ -94,6 +103,22 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
   c.xperm = reinterpret_cast<__nv_bfloat16*>(C(L.xperm));
   c.abuf = reinterpret_cast<__nv_bfloat16*>(C(L.abuf));
   c.bbuf = reinterpret_cast<__nv_bfloat16*>(C(L.bbuf));
+  c.tab = StreamTables{};
+  if (L.M > 0) {
+    int* t = reinterpret_cast<int*>(C(L.stab));
+    const int M = L.M, El = L.El;
+    c.tab.plan = t;        t += PLAN_WORDS;
+    c.tab.mb_of = t;       t += M;
+    c.tab.seg_poff = t;    t += M * El + 1;
+    c.tab.cum = t;         t += M * El;
+    c.tab.mb_range = t;    t += 2 * M;
+    c.tab.shift_fwd = t;   t += M;
+    c.tab.shift_bwd = t;   t += M;
+    c.tab.replay = t;      t += M;
+    c.tab.chunk = t;       t += 4 * M;
+    c.tab.ring_start = t;
+  }
+  c.acc32 = nullptr;
   if (ws) {
     c.hist = reinterpret_cast<int*>(W(L.hist));
     c.logits = reinterpret_cast<float*>(W(L.logits));
@@ -108,6 +133,7 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
     c.dlasg = reinterpret_cast<float*>(W(L.dlasg));
     c.wrt = reinterpret_cast<__nv_bfloat16*>(W(L.wrt));
     c.dxperm = reinterpret_cast<__nv_bfloat16*>(W(L.dxperm));
+    c.acc32 = L.M > 0 ? reinterpret_cast<float*>(W(L.acc32)) : nullptr;
   }
   return c;
 }
@@ -165,12 +191,13 @@ static int num_sms() {
 enum KernelId {
   K_ROUTER_LOGITS, K_TOPK, K_SCAN, K_SCATTER, K_DISPATCH, K_GEMM_GATEUP, K_GEMM_DOWN, K_COMBINE,
   K_REV_COMBINE, K_GEMM_DGRAD_DOWN, K_ROUTER_BWD, K_DWR, K_TRANSPOSE_WR, K_GEMM_DGRAD_GATEUP, K_REV_DISPATCH,
-  K_GEMM_WGRAD_GATEUP, K_GEMM_WGRAD_DOWN, K_NUM
+  K_GEMM_WGRAD_GATEUP, K_GEMM_WGRAD_DOWN, K_PLAN, K_REPLAY, K_FINISH_ACC, K_NUM
 };
 static const char* kKernelNames[K_NUM] = {
     "router_logits", "topk_gating", "hist_scan", "stable_scatter", "dispatch", "gemm_gateup_swiglu",
     "gemm_down_combw", "combine", "reverse_combine", "gemm_dgrad_down_swiglu_bwd", "router_bwd", "router_wgrad",
-    "transpose_wr", "gemm_dgrad_gateup", "reverse_dispatch", "gemm_wgrad_gateup", "gemm_wgrad_down"};
+    "transpose_wr", "gemm_dgrad_gateup", "reverse_dispatch", "gemm_wgrad_gateup", "gemm_wgrad_down",
+    "stream_plan", "ring_replay", "wgrad_accumulator_finish"};
 
 struct ProfRec {
   int kid;
@@ -224,6 +251,7 @@ static GemmParams base_params(const Layout& L, const Ctx& c, int* status) {
   p.El = L.El;
   p.d = L.d;
   p.I = L.I;
+  p.nseg = L.El;
   p.status = status;
   return p;
 }
@@ -279,6 +307,42 @@ static moe_status check_shape(const moe_shape* s, Layout* L) {
   return MOE_OK;
 }
 
+// Router GEMM, top-k gating, histogram + scan (+ the stream plan) and the stable scatter.
+static moe_status route_tokens(const Layout& L, const Ctx& c, const void* X, const void* W_r, const float* bias,
+                               int ring_rows, cudaStream_t st) {
+  const int grid = num_sms();
+  int* status = c.hdr + HDR_STATUS;
+  MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
+    return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
+  }));
+  const int splits = router_splits(L.T, L.E, L.d);
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, X, L.d, static_cast<uint64_t>(L.T), L.d, 64, 128));
+    MOE_TMAP(tmap_2d(&p.tb0, c.wrt, L.d, static_cast<uint64_t>(L.E), L.d, 64, 256));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.T = static_cast<int>(L.T);
+    p.E = L.E;
+    p.splits = splits;
+    p.outf = c.rpart;
+    const int64_t tiles = ((L.T + 127) / 128) * ((L.E + 255) / 256) * splits;
+    const int g = static_cast<int>(tiles < grid ? tiles : grid);
+    MOE_TRY(timed(K_ROUTER_LOGITS, st, [&] { return launch_gemm(G_ROUTER, p, g, st); }));
+  }
+  MOE_TRY(timed(K_TOPK, st, [&] { return launch_topk(L, c, bias, splits, st); }));
+  MOE_TRY(timed(K_SCAN, st, [&] { return launch_scan(L, c, st); }));
+  if (L.M > 0) {
+    // two full waves of the gate/up GEMM: (rows / 128) * (I / 128) >= 2 * SMs
+    const int min_rows = static_cast<int>((2LL * grid * 128) / (L.I / 128));
+    MOE_TRY(timed(K_PLAN, st, [&] { return launch_plan(L, c, ring_rows, min_rows, st); }));
+  }
+  MOE_TRY(cudaMemsetAsync(c.row_asg, 0xFF, static_cast<size_t>(L.RP) * 4, st));
+  MOE_TRY(cudaMemsetAsync(c.row_gate, 0, static_cast<size_t>(L.RP) * 4, st));
+  MOE_TRY(timed(K_SCATTER, st, [&] { return launch_scatter(L, c, st); }));
+  return MOE_OK;
+}
+
 moe_status moe_fwd(const moe_shape* s, const void* X, const void* W_r, const float* bias, const void* W_gate,
                    const void* W_up, const void* W_down, void* Y, void* ctx, size_t ctx_bytes, void* ws,
                    size_t ws_bytes, void* stream) {
@@ -300,33 +364,12 @@ moe_status moe_fwd(const moe_shape* s, const void* X, const void* W_r, const flo
   const int grid = num_sms();
   int* status = c.hdr + HDR_STATUS;
   const uint64_t RP = static_cast<uint64_t>(L.RP);
-  // 1. router GEMM on the tensor cores: fixed K splits -> fp32 partials
-  MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
-    return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
-  }));
-  const int splits = router_splits(L.T, L.E, L.d);
+  // 1-4. router GEMM (tensor cores, fixed K splits), top-k gating, histogram + scan, stable scatter
   {
-    GemmParams p = base_params(L, c, status);
-    MOE_TMAP(tmap_2d(&p.ta0, X, L.d, static_cast<uint64_t>(L.T), L.d, 64, 128));
-    MOE_TMAP(tmap_2d(&p.tb0, c.wrt, L.d, static_cast<uint64_t>(L.E), L.d, 64, 256));
-    p.ta1 = p.ta0;
-    p.tb1 = p.tb0;
-    p.T = static_cast<int>(L.T);
-    p.E = L.E;
-    p.splits = splits;
-    p.outf = c.rpart;
-    const int64_t tiles = ((L.T + 127) / 128) * ((L.E + 255) / 256) * splits;
-    const int g = static_cast<int>(tiles < grid ? tiles : grid);
-    MOE_TRY(timed(K_ROUTER_LOGITS, st, [&] { return launch_gemm(G_ROUTER, p, g, st); }));
+    const moe_status r = route_tokens(L, c, X, W_r, bias, 0, st);
+    if (r != MOE_OK) return r;
   }
-  // 2. partial sums (fixed order) + bias, top-k gating, per-block histograms
-  MOE_TRY(timed(K_TOPK, st, [&] { return launch_topk(L, c, bias, splits, st); }));
-  // 3. counts, prefix sums, padded offsets
-  MOE_TRY(timed(K_SCAN, st, [&] { return launch_scan(L, c, st); }));
-  // 4. stable scatter + dispatch
-  MOE_TRY(cudaMemsetAsync(c.row_asg, 0xFF, static_cast<size_t>(L.RP) * 4, st));
-  MOE_TRY(cudaMemsetAsync(c.row_gate, 0, static_cast<size_t>(L.RP) * 4, st));
-  MOE_TRY(timed(K_SCATTER, st, [&] { return launch_scatter(L, c, st); }));
+  // 4. dispatch into the expert-contiguous layout
   MOE_TRY(timed(K_DISPATCH, st, [&] { return launch_gather_rows(L, c, Xb, c.xperm, st); }));
 
   // 5. grouped gate/up GEMM with the SwiGLU epilogue
@@ -477,6 +520,235 @@ const char* moe_kernel_name(int kernel_id) {
 }
 
 unsigned long long moe_kernel_launches(void) { return g_launches.load(); }
+
+// ---------------------------------------------------------------------------
+// Ring-streamed layer: M minibatches of shape->T tokens through a fixed ring
+// ---------------------------------------------------------------------------
+static moe_status check_stream(const moe_shape* s, int32_t M, Layout* L) {
+  if (!s || M <= 0) return MOE_ERR_INVALID_ARG;
+  if (s->prec != MOE_BF16) return s->prec == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (!make_layout(*s, L, M)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+// Worst-case padded rows of one minibatch: every macrobatch must fit in the ring.
+static int64_t minibatch_rows(const Layout& L) {
+  const int64_t kl = L.k < L.El ? L.k : L.El;
+  return static_cast<int64_t>(align_up(static_cast<size_t>(L.T_mb * kl + int64_t(kPad - 1) * L.El), kPad));
+}
+
+size_t moe_stream_ctx_size(const moe_shape* s, int32_t M) {
+  Layout L;
+  if (check_stream(s, M, &L) != MOE_OK) return 0;
+  return L.ctx_bytes;
+}
+
+size_t moe_stream_workspace_size(const moe_shape* s, int32_t M) {
+  Layout L;
+  if (check_stream(s, M, &L) != MOE_OK) return 0;
+  return L.ws_bytes;
+}
+
+size_t moe_stream_min_ring_bytes(const moe_shape* s) {
+  Layout L;
+  if (check_stream(s, 1, &L) != MOE_OK) return 0;
+  return static_cast<size_t>(minibatch_rows(L)) * L.d * 2;
+}
+
+moe_status moe_fwd_stream(const moe_shape* s, int32_t M, const void* X, const void* W_r, const float* bias,
+                          const void* W_gate, const void* W_up, const void* W_down, void* Y, void* ctx,
+                          size_t ctx_bytes, void* ring, size_t ring_bytes, void* ws, size_t ws_bytes, void* stream) {
+  Layout L;
+  const moe_status cs = check_stream(s, M, &L);
+  if (cs != MOE_OK) return cs;
+  if (!X || !Y || !W_r || !W_gate || !W_up || !W_down || !ctx || !ring || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W_r) || !aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_down) ||
+      !aligned16(Y) || !aligned16(ctx) || !aligned16(ring) || !aligned16(ws) ||
+      (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+    return MOE_ERR_INVALID_ARG;
+  const int64_t ring_rows = static_cast<int64_t>(ring_bytes / (static_cast<size_t>(L.d) * 2));
+  if (ctx_bytes < L.ctx_bytes || ws_bytes < L.ws_bytes || ring_rows < minibatch_rows(L) ||
+      ring_rows >= (int64_t(1) << 31))
+    return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ctx c = make_ctx(L, ctx, ws);
+  MOE_TRY(cudaMemsetAsync(c.hdr, 0, HDR_WORDS * 4, st));
+  {
+    const moe_status r = route_tokens(L, c, X, W_r, bias, static_cast<int>(ring_rows), st);
+    if (r != MOE_OK) return r;
+  }
+  const int grid = num_sms();
+  int* status = c.hdr + HDR_STATUS;
+  const uint64_t RP = static_cast<uint64_t>(L.RP);
+  const int El = L.El;
+  CUtensorMap ring_map, wg_map, wu_map, h_map, wd_map;
+  MOE_TMAP(tmap_2d(&ring_map, ring, L.d, static_cast<uint64_t>(ring_rows), L.d, 64, 128));
+  MOE_TMAP(tmap_2d(&wg_map, W_gate, L.I, static_cast<uint64_t>(El) * L.d, L.I, 64, 64));
+  MOE_TMAP(tmap_2d(&wu_map, W_up, L.I, static_cast<uint64_t>(El) * L.d, L.I, 64, 64));
+  MOE_TMAP(tmap_2d(&h_map, c.hbuf, L.I, RP, L.I, 64, 128));
+  MOE_TMAP(tmap_2d(&wd_map, W_down, L.d, static_cast<uint64_t>(El) * L.I, L.d, 64, 64));
+  // Macrobatches walk the ring forward.  The host enqueues M of them (the most
+  // the plan can form); launches past the plan's count find empty segments and exit.
+  for (int m = 0; m < M; ++m) {
+    const int* seg = c.tab.seg_poff + m * El;
+    MOE_TRY(timed(K_DISPATCH, st, [&] {
+      return launch_gather_range(L, c, static_cast<const __nv_bfloat16*>(X), seg, seg + El, c.tab.shift_fwd + m,
+                                 ring_rows, static_cast<__nv_bfloat16*>(ring), st);
+    }));
+    GemmParams p = base_params(L, c, status);
+    p.poff = seg;
+    p.nseg = El;
+    p.ta0 = ring_map;
+    p.ta1 = ring_map;
+    p.tb0 = wg_map;
+    p.tb1 = wu_map;
+    p.ring_shift = c.tab.shift_fwd + m;
+    p.out0 = c.abuf;
+    p.out1 = c.bbuf;
+    p.out2 = c.hbuf;
+    MOE_TRY(timed(K_GEMM_GATEUP, st, [&] { return launch_gemm(G_GATEUP, p, grid, st); }));
+    GemmParams q = base_params(L, c, status);
+    q.poff = seg;
+    q.nseg = El;
+    q.ta0 = q.ta1 = h_map;
+    q.tb0 = q.tb1 = wd_map;
+    q.out0 = c.obuf;
+    MOE_TRY(timed(K_GEMM_DOWN, st, [&] { return launch_gemm(G_DOWN, q, grid, st); }));
+    MOE_TRY(timed(K_COMBINE, st, [&] {
+      return launch_combine(L, c, c.obuf, static_cast<__nv_bfloat16*>(Y), st, c.tab.mb_range + 2 * m);
+    }));
+  }
+  return MOE_OK;
+}
+
+moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const void* W_r, const void* W_gate,
+                          const void* W_up, const void* W_down, const void* dY, void* ctx, size_t ctx_bytes, void* dX,
+                          void* dW_gate, void* dW_up, void* dW_down, float* dW_r, void* ring, size_t ring_bytes,
+                          void* ws, size_t ws_bytes, void* stream) {
+  Layout L;
+  const moe_status cs = check_stream(s, M, &L);
+  if (cs != MOE_OK) return cs;
+  if (!X || !dY || !dX || !W_r || !W_gate || !W_up || !W_down || !ctx || !dW_gate || !dW_up || !dW_down || !dW_r ||
+      !ring || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W_r) || !aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_down) ||
+      !aligned16(dY) || !aligned16(ctx) || !aligned16(dX) || !aligned16(dW_gate) || !aligned16(dW_up) ||
+      !aligned16(dW_down) || !aligned16(dW_r) || !aligned16(ring) || !aligned16(ws))
+    return MOE_ERR_INVALID_ARG;
+  const int64_t ring_rows = static_cast<int64_t>(ring_bytes / (static_cast<size_t>(L.d) * 2));
+  if (ctx_bytes < L.ctx_bytes || ws_bytes < L.ws_bytes || ring_rows < minibatch_rows(L) ||
+      ring_rows >= (int64_t(1) << 31))
+    return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ctx c = make_ctx(L, ctx, ws);
+  const int grid = num_sms();
+  int* status = c.hdr + HDR_STATUS;
+  const uint64_t RP = static_cast<uint64_t>(L.RP);
+  const uint64_t El = static_cast<uint64_t>(L.El);
+  const int nseg = L.M * L.El;
+
+  // dgrad path over every row of the stream (no X_perm needed)
+  MOE_TRY(timed(K_REV_COMBINE, st, [&] {
+    return launch_gather_rows(L, c, static_cast<const __nv_bfloat16*>(dY), c.dyperm, st);
+  }));
+  {
+    GemmParams p = base_params(L, c, status);
+    p.poff = c.tab.seg_poff;
+    p.nseg = nseg;
+    MOE_TMAP(tmap_2d(&p.ta0, c.dyperm, L.d, RP, L.d, 64, 128));
+    MOE_TMAP(tmap_2d(&p.tb0, W_down, L.d, El * L.I, L.d, 64, 256));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.in0 = c.abuf;
+    p.in1 = c.bbuf;
+    p.out0 = c.dabuf;
+    p.out1 = c.dbbuf;
+    p.out2 = c.hgbuf;
+    p.outf = c.dgpart;
+    MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm(G_DGRAD_DOWN, p, grid, st); }));
+  }
+  MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st); }));
+  MOE_TRY(timed(K_DWR, st, [&] { return launch_dwr(L, c, static_cast<const __nv_bfloat16*>(X), dW_r, st); }));
+  MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
+    return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
+  }));
+  {
+    GemmParams p = base_params(L, c, status);
+    p.poff = c.tab.seg_poff;
+    p.nseg = nseg;
+    MOE_TMAP(tmap_2d(&p.ta0, c.dabuf, L.I, RP, L.I, 64, 128));
+    MOE_TMAP(tmap_2d(&p.ta1, c.dbbuf, L.I, RP, L.I, 64, 128));
+    MOE_TMAP(tmap_2d(&p.tb0, W_gate, L.I, El * L.d, L.I, 64, 256));
+    MOE_TMAP(tmap_2d(&p.tb1, W_up, L.I, El * L.d, L.I, 64, 256));
+    p.out0 = c.dxperm;
+    MOE_TRY(timed(K_GEMM_DGRAD_GATEUP, st, [&] { return launch_gemm(G_DGRAD_GATEUP, p, grid, st); }));
+  }
+  MOE_TRY(timed(K_REV_DISPATCH, st, [&] { return launch_rev_dispatch(L, c, static_cast<__nv_bfloat16*>(dX), st); }));
+  {  // wgrad of W_down: Hg and dY_perm cover the whole stream
+    GemmParams p = base_params(L, c, status);
+    p.poff = c.tab.seg_poff;
+    p.nseg = nseg;
+    MOE_TMAP(tmap_2d(&p.ta0, c.hgbuf, L.I, RP, L.I, 64, 64));
+    MOE_TMAP(tmap_2d(&p.tb0, c.dyperm, L.d, RP, L.d, 64, 64));
+    MOE_TMAP(tmap_2d(&p.to0, dW_down, L.d, El * L.I, L.d, 64, 32));
+    p.to1 = p.to0;
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.out0 = static_cast<__nv_bfloat16*>(dW_down);
+    MOE_TRY(timed(K_GEMM_WGRAD_DOWN, st, [&] { return launch_gemm(G_WGRAD_DOWN, p, grid, st); }));
+  }
+  // wgrad of W_gate / W_up needs X_perm: walk the ring in reverse, chunk by chunk
+  {
+    GemmParams p = base_params(L, c, status);
+    p.poff = c.tab.seg_poff;
+    p.nseg = nseg;
+    p.ring_shift = c.tab.shift_bwd;
+    p.acc32 = c.acc32;
+    MOE_TMAP(tmap_2d(&p.ta0, ring, L.d, static_cast<uint64_t>(ring_rows), L.d, 64, 64));
+    MOE_TMAP(tmap_2d(&p.tb0, c.dabuf, L.I, RP, L.I, 64, 64));
+    MOE_TMAP(tmap_2d(&p.tb1, c.dbbuf, L.I, RP, L.I, 64, 64));
+    MOE_TMAP(tmap_2d(&p.to0, dW_gate, L.I, El * L.d, L.I, 64, 32));
+    MOE_TMAP(tmap_2d(&p.to1, dW_up, L.I, El * L.d, L.I, 64, 32));
+    {  // fp32 accumulator [2 * El * d, I], 32 x 32 boxes (128-byte rows)
+      EncodeTiledFn enc = get_encode();
+      if (!enc) return MOE_ERR_CUDA;
+      const cuuint64_t dims[2] = {static_cast<cuuint64_t>(L.I), 2 * El * static_cast<cuuint64_t>(L.d)};
+      const cuuint64_t strides[1] = {static_cast<cuuint64_t>(L.I) * 4};
+      const cuuint32_t box[2] = {32, 32};
+      const cuuint32_t estr[2] = {1, 1};
+      if (enc(&p.tacc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, c.acc32, dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return MOE_ERR_CUDA;
+    }
+    p.ta1 = p.ta0;
+    p.out0 = static_cast<__nv_bfloat16*>(dW_gate);
+    p.out1 = static_cast<__nv_bfloat16*>(dW_up);
+    for (int ch = 0; ch < L.M; ++ch) {
+      MOE_TRY(timed(K_REPLAY, st, [&] {
+        return launch_replay(L, c, ch, static_cast<const __nv_bfloat16*>(X), static_cast<__nv_bfloat16*>(ring),
+                             ring_rows, st);
+      }));
+      p.chunk = c.tab.chunk + 4 * ch;
+      MOE_TRY(timed(K_GEMM_WGRAD_GATEUP, st, [&] { return launch_gemm(G_WGRAD_GATEUP, p, grid, st); }));
+    }
+  }
+  MOE_TRY(timed(K_FINISH_ACC, st, [&] {
+    return launch_finish_acc(L, c, static_cast<__nv_bfloat16*>(dW_gate), static_cast<__nv_bfloat16*>(dW_up), st);
+  }));
+  return MOE_OK;
+}
+
+moe_status moe_debug_stream_plan(const moe_shape* s, int32_t M, const void* ctx, int32_t* tables, void* stream) {
+  Layout L;
+  const moe_status cs = check_stream(s, M, &L);
+  if (cs != MOE_OK) return cs;
+  if (!ctx || !tables) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(cudaMemcpyAsync(tables, static_cast<const char*>(ctx) + L.stab,
+                          static_cast<size_t>(stream_table_words(M, L.El)) * 4, cudaMemcpyDeviceToDevice,
+                          static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
 
 moe_status moe_get_error(void* ctx, void* stream) {
   if (!ctx) return MOE_ERR_INVALID_ARG;

@@ -16,9 +16,35 @@ constexpr int kPad = 128;          // rows of an expert segment are padded to a 
 constexpr int kTokensPerBlock = 16;  // tokens per block of the top-k / scatter kernels
 constexpr int kMaxE = 512;
 constexpr int kMaxK = 16;
+constexpr int kMaxMinibatches = 256;  // ring-streamed layer
 
 // ctx header words (int32)
 enum HdrWord { HDR_STATUS = 0, HDR_ROWS_P = 1, HDR_MTILES = 2, HDR_WORDS = 64 };
+
+// Plan of a ring-streamed layer (M minibatches grouped into macrobatches), written on
+// the device by k_plan and read by every per-macrobatch / per-chunk launch.
+enum PlanWord {
+  PLAN_N_MACRO = 0,   // macrobatches formed
+  PLAN_N_CHUNKS = 1,  // backward wgrad chunks
+  PLAN_ROWS = 2,      // padded rows of the whole stream
+  PLAN_REPLAYED = 3,  // padded rows re-dispatched in the backward
+  PLAN_RESIDENT = 4,  // padded rows the backward found still in the ring
+  PLAN_RING_ROWS = 5, // ring capacity in rows
+  PLAN_WORDS = 16
+};
+struct StreamTables {
+  int* plan;       // [PLAN_WORDS]
+  int* mb_of;      // [M]        macrobatch of each minibatch
+  int* seg_poff;   // [M*El+1]   padded row where segment (m, el) starts
+  int* cum;        // [M*El]     assignments to el in macrobatches before m
+  int* mb_range;   // [2M]       minibatches [begin, end) of macrobatch m
+  int* shift_fwd;  // [M]        ring row - padded row, forward placement
+  int* shift_bwd;  // [M]        ring row - padded row, backward placement
+  int* replay;     // [M]        1 if the backward re-dispatches macrobatch m
+  int* chunk;      // [4M]       backward chunk c: {m_lo, m_hi, valid, mode}
+  int* ring_start; // [M]        forward ring row of macrobatch m
+};
+constexpr int stream_table_words(int M, int El) { return PLAN_WORDS + M + (M * El + 1) + M * El + 2 * M + 4 * M + 4 * M; }
 
 // Byte offsets of every region of ctx (saved for backward) and ws (scratch).
 struct Layout {
@@ -27,15 +53,18 @@ struct Layout {
   int d, E, I, k, first, El;
   int64_t RP;     // padded-row capacity: worst case of sum_e ceil(count_e / 128) * 128
   int nblk;       // blocks of the top-k / scatter kernels
+  int M;          // minibatches of a ring-streamed layer (0: one call = one batch)
+  int64_t T_mb;   // tokens per minibatch (streamed layer)
   // ctx
   size_t hdr, ids, gates, counts, offsets, poff, perm_tok, perm_asg, slot_row, row_asg, row_gate, xperm, abuf,
-      bbuf, ctx_bytes;
+      bbuf, stab, ctx_bytes;
   // ws
-  size_t hist, logits, rpart, hbuf, obuf, dyperm, dabuf, dbbuf, hgbuf, dgpart, dlasg, wrt, dxperm, ws_bytes;
+  size_t hist, logits, rpart, hbuf, obuf, dyperm, dabuf, dbbuf, hgbuf, dgpart, dlasg, wrt, dxperm, acc32, ws_bytes;
 };
 
-// Returns false for shapes outside the supported limits.
-bool make_layout(const moe_shape& s, Layout* L);
+// Returns false for shapes outside the supported limits.  M > 0: a ring-streamed
+// layer of M minibatches of s.T tokens (X_perm lives in the caller's ring).
+bool make_layout(const moe_shape& s, Layout* L, int M = 0);
 
 // ---------------------------------------------------------------------------
 // grouped GEMM (tcgen05 + TMA), see gemm.cu
@@ -53,8 +82,15 @@ enum GemmKind {
 struct GemmParams {
   CUtensorMap ta0, ta1, tb0, tb1;  // operand maps
   CUtensorMap to0, to1;            // output maps (TMA stores of the wgrad epilogues)
-  const int* hdr;             // ctx header (rows_p)
-  const int* poff;            // padded offsets [El+1]
+  CUtensorMap tacc;                // fp32 wgrad accumulator map (ring-streamed backward, several chunks)
+  const int* hdr;             // ctx header
+  // Padded row space: nseg segments (macrobatch m, local expert el) = m * El + el,
+  // segment s covers rows [poff[s], poff[s+1]).  One macrobatch: nseg = El.
+  const int* poff;
+  int nseg;
+  const int* ring_shift;      // per macrobatch: ring row - padded row of X_perm (NULL: X_perm not in a ring)
+  const int* chunk;           // wgrad gate/up over a chunk of macrobatches: {m_lo, m_hi, valid, mode}; NULL = all
+  float* acc32;               // fp32 accumulator for dW_gate / dW_up when a backward needs several chunks
   const float* row_gate;      // [RP]
   const __nv_bfloat16* in0;   // epilogue inputs
   const __nv_bfloat16* in1;
@@ -96,6 +132,8 @@ struct Ctx {  // typed views of ctx + ws for one shape
   float* rpart;  // router split-K partials [splits, T, E]
   __nv_bfloat16 *hbuf, *obuf, *dyperm, *dabuf, *dbbuf, *hgbuf, *wrt, *dxperm;
   float *dgpart, *dlasg;
+  float* acc32;
+  StreamTables tab;
 };
 Ctx make_ctx(const Layout& L, void* ctx, void* ws);
 
@@ -104,8 +142,16 @@ cudaError_t launch_scan(const Layout& L, const Ctx& c, cudaStream_t st);
 cudaError_t launch_scatter(const Layout& L, const Ctx& c, cudaStream_t st);
 cudaError_t launch_gather_rows(const Layout& L, const Ctx& c, const __nv_bfloat16* src, __nv_bfloat16* dst,
                                cudaStream_t st);
+// rows [*lo, *hi) to dst row + *shift (streamed layer)
+cudaError_t launch_gather_range(const Layout& L, const Ctx& c, const __nv_bfloat16* src, const int* lo, const int* hi,
+                                const int* shift, int64_t max_rows, __nv_bfloat16* dst, cudaStream_t st);
 cudaError_t launch_combine(const Layout& L, const Ctx& c, const __nv_bfloat16* Oprime, __nv_bfloat16* Y,
-                           cudaStream_t st);
+                           cudaStream_t st, const int* mb_range = nullptr);
+cudaError_t launch_plan(const Layout& L, const Ctx& c, int ring_rows, int min_rows, cudaStream_t st);
+cudaError_t launch_replay(const Layout& L, const Ctx& c, int chunk, const __nv_bfloat16* X, __nv_bfloat16* ring,
+                          int64_t ring_rows, cudaStream_t st);
+cudaError_t launch_finish_acc(const Layout& L, const Ctx& c, __nv_bfloat16* dW_gate, __nv_bfloat16* dW_up,
+                              cudaStream_t st);
 cudaError_t launch_router_bwd(const Layout& L, const Ctx& c, cudaStream_t st);
 cudaError_t launch_transpose_wr(const Layout& L, const __nv_bfloat16* W_r, __nv_bfloat16* W_rT, cudaStream_t st);
 cudaError_t launch_rev_dispatch(const Layout& L, const Ctx& c, __nv_bfloat16* dX, cudaStream_t st);

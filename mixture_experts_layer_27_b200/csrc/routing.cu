@@ -140,9 +140,14 @@ __global__ void __launch_bounds__(1024) k_scan(int* __restrict__ hist, int nblk,
 // stable scatter: one warp per block of tokens, tokens in ascending order.
 // row position of (t, j) inside expert e = base[b][e] + #{earlier tokens of b with e}.
 // ---------------------------------------------------------------------------
+// Ring-streamed layer: the padded rows are grouped by macrobatch, then expert
+// (segment m * El + el starts at seg_poff[...]); `cum` counts the expert's
+// assignments in earlier macrobatches.  Without macrobatches (mb_of == NULL)
+// the segments are the experts' and poff gives their starts.
 __global__ void __launch_bounds__(32) k_scatter(const int* __restrict__ ids, const float* __restrict__ gates,
                                                 const int* __restrict__ base, const int* __restrict__ offsets,
                                                 const int* __restrict__ poff, int T, int E, int k, int first, int El,
+                                                int T_mb, const int* __restrict__ mb_of, const int* __restrict__ cum,
                                                 int* __restrict__ perm_tok, int* __restrict__ perm_asg,
                                                 int* __restrict__ slot_row, int* __restrict__ row_asg,
                                                 float* __restrict__ row_gate) {
@@ -163,7 +168,13 @@ __global__ void __launch_bounds__(32) k_scatter(const int* __restrict__ ids, con
       perm_asg[u] = a;
       const int el = e - first;
       if (el >= 0 && el < El) {
-        const int R = poff[el] + pos;
+        int R;
+        if (mb_of) {
+          const int sg = mb_of[t / T_mb] * El + el;
+          R = poff[sg] + pos - cum[sg];
+        } else {
+          R = poff[el] + pos;
+        }
         slot_row[a] = R;
         row_asg[R] = a;
         row_gate[R] = gates[a];
@@ -178,14 +189,18 @@ __global__ void __launch_bounds__(32) k_scatter(const int* __restrict__ ids, con
 // ---------------------------------------------------------------------------
 // dispatch / reverse-combine: dst[R] = src[token(R)], zero rows for padding.
 // ---------------------------------------------------------------------------
+// Rows [*lo, *hi) of the padded layout, written at row R + *shift of dst (a
+// ring position for the streamed layer; shift NULL = 0).
 __global__ void __launch_bounds__(128) k_gather_rows(const __nv_bfloat16* __restrict__ src,
-                                                     const int* __restrict__ row_asg, const int* __restrict__ hdr,
-                                                     int k, int d, int64_t RP, __nv_bfloat16* __restrict__ dst) {
-  const int rows_p = __ldg(hdr + HDR_ROWS_P);
+                                                     const int* __restrict__ row_asg, const int* __restrict__ lo,
+                                                     const int* __restrict__ hi, const int* __restrict__ shift, int k,
+                                                     int d, __nv_bfloat16* __restrict__ dst) {
+  const int r0 = __ldg(lo), r1 = __ldg(hi);
+  const int sh = shift ? __ldg(shift) : 0;
   const int nv = d / 8;
-  for (int64_t R = blockIdx.x; R < rows_p; R += gridDim.x) {
+  for (int64_t R = r0 + blockIdx.x; R < r1; R += gridDim.x) {
     const int a = row_asg[R];
-    uint4* out = reinterpret_cast<uint4*>(dst + R * d);
+    uint4* out = reinterpret_cast<uint4*>(dst + (R + sh) * d);
     if (a >= 0) {
       const uint4* in = reinterpret_cast<const uint4*>(src + static_cast<size_t>(a / k) * d);
       for (int i = threadIdx.x; i < nv; i += blockDim.x) out[i] = __ldg(in + i);
@@ -199,11 +214,16 @@ __global__ void __launch_bounds__(128) k_gather_rows(const __nv_bfloat16* __rest
 // ---------------------------------------------------------------------------
 // combine: Y[t] = sum_j O'[slot_row[t, j]] in slot order, fp32, stored bf16.
 // ---------------------------------------------------------------------------
+// Tokens [0, T), or the minibatches [range[0], range[1]) of T_mb tokens each.
 __global__ void __launch_bounds__(128) k_combine(const __nv_bfloat16* __restrict__ Op,
-                                                 const int* __restrict__ slot_row, int k, int d,
+                                                 const int* __restrict__ slot_row, int k, int d, int T,
+                                                 const int* __restrict__ range, int T_mb,
                                                  __nv_bfloat16* __restrict__ Y) {
-  const int t = blockIdx.x;
+  const int t0 = range ? __ldg(range) * T_mb : 0;
+  const int t1 = range ? __ldg(range + 1) * T_mb : T;
   __shared__ int rows[kMaxK];
+  for (int t = t0 + blockIdx.x; t < t1; t += gridDim.x) {
+  __syncthreads();
   if (threadIdx.x < k) rows[threadIdx.x] = slot_row[static_cast<size_t>(t) * k + threadIdx.x];
   __syncthreads();
   for (int i = threadIdx.x * 8; i < d; i += blockDim.x * 8) {
@@ -224,6 +244,7 @@ __global__ void __launch_bounds__(128) k_combine(const __nv_bfloat16* __restrict
     o.z = pack_bf16(acc[4], acc[5]);
     o.w = pack_bf16(acc[6], acc[7]);
     *reinterpret_cast<uint4*>(Y + static_cast<size_t>(t) * d + i) = o;
+  }
   }
 }
 
@@ -370,6 +391,187 @@ __global__ void __launch_bounds__(128) k_dwr(const __nv_bfloat16* __restrict__ X
     dWr[static_cast<size_t>(i0 + c) * E + e] = ((part[0][c] + part[1][c]) + part[2][c]) + part[3][c];
 }
 
+// ---------------------------------------------------------------------------
+// Ring-streamed layer planner (one thread; M minibatches, El local experts).
+//
+// Forward: consecutive minibatches are grouped into a macrobatch until its
+// padded rows reach min_rows (the gate/up grouped GEMM then has at least two
+// full waves of tiles, the MoK pages' heuristic), or until the next minibatch
+// would not fit in the ring.  Each macrobatch's padded segment is placed at the
+// ring's write pointer; a segment that would run past the end starts at row 0.
+// Backward: macrobatches are visited in reverse.  The ones whose segment is
+// still intact (no later segment overlapped it) form the first chunk and are
+// reused in place; older ones are re-dispatched (replayed) into the ring in
+// chunks of consecutive macrobatches that fit in it together.
+// ---------------------------------------------------------------------------
+__global__ void k_plan(const int* __restrict__ base, const int* __restrict__ counts, int nblk_per_mb, int nblk, int M,
+                       int E, int first, int El, int ring_rows, int min_rows, StreamTables tb) {
+  __shared__ int open_cnt[kMaxE];  // assignments per expert in the macrobatch being formed
+  __shared__ int tot_cnt[kMaxE];   // assignments per expert in the macrobatches already formed
+  __shared__ int resident[kMaxMinibatches];
+  if (threadIdx.x != 0) return;
+  for (int el = 0; el < El; ++el) open_cnt[el] = tot_cnt[el] = 0;
+  // count of local expert el in minibatch b: difference of the block-level exclusive scans
+  auto mb_count = [&](int b, int el) {
+    const int e = first + el;
+    const int b1 = (b + 1) * nblk_per_mb;
+    const int hi = b1 >= nblk ? counts[e] : base[static_cast<size_t>(b1) * E + e];
+    return hi - base[static_cast<size_t>(b * nblk_per_mb) * E + e];
+  };
+  auto padded = [](int c) { return (c + kPad - 1) / kPad * kPad; };
+  int row = 0, wp = 0, nm = 0, b0 = 0;
+  auto emit = [&](int b_end) {  // close the open macrobatch = minibatches [b0, b_end)
+    const int start = row;
+    for (int el = 0; el < El; ++el) {
+      const int sg = nm * El + el;
+      tb.seg_poff[sg] = row;
+      tb.cum[sg] = tot_cnt[el];
+      row += padded(open_cnt[el]);
+      tot_cnt[el] += open_cnt[el];
+      open_cnt[el] = 0;
+    }
+    const int size = row - start;
+    if (wp + size > ring_rows) wp = 0;  // would straddle the end: restart at row 0
+    tb.ring_start[nm] = wp;
+    tb.shift_fwd[nm] = wp - start;
+    wp += size;
+    tb.mb_range[2 * nm] = b0;
+    tb.mb_range[2 * nm + 1] = b_end;
+    ++nm;
+    b0 = b_end;
+  };
+  for (int b = 0; b < M; ++b) {
+    if (b > b0) {  // does minibatch b still fit in the ring with the open macrobatch?
+      int with_b = 0;
+      for (int el = 0; el < El; ++el) with_b += padded(open_cnt[el] + mb_count(b, el));
+      if (with_b > ring_rows) emit(b);
+    }
+    int rows_now = 0;
+    for (int el = 0; el < El; ++el) {
+      open_cnt[el] += mb_count(b, el);
+      rows_now += padded(open_cnt[el]);
+    }
+    tb.mb_of[b] = nm;
+    if (rows_now >= min_rows) emit(b + 1);  // two full waves of gate/up tiles
+  }
+  if (b0 < M) emit(M);
+  for (int m = nm; m < M; ++m) {  // macrobatches not formed: empty segments at the end
+    for (int el = 0; el < El; ++el) {
+      tb.seg_poff[m * El + el] = row;
+      tb.cum[m * El + el] = tot_cnt[el];
+    }
+    tb.mb_range[2 * m] = tb.mb_range[2 * m + 1] = M;
+    tb.shift_fwd[m] = tb.shift_bwd[m] = tb.ring_start[m] = tb.replay[m] = 0;
+  }
+  tb.seg_poff[M * El] = row;
+
+  // residency after the forward: no later segment overlaps this one in the ring
+  auto seg_rows = [&](int m) { return tb.seg_poff[(m + 1) * El] - tb.seg_poff[m * El]; };
+  for (int m = 0; m < nm; ++m) {
+    const int a0 = tb.ring_start[m], a1 = a0 + seg_rows(m);
+    int ok = 1;
+    for (int q = m + 1; q < nm && ok; ++q) {
+      const int c0 = tb.ring_start[q], c1 = c0 + seg_rows(q);
+      if (a1 > a0 && c1 > c0 && c0 < a1 && a0 < c1) ok = 0;
+    }
+    resident[m] = ok;
+  }
+  // backward chunks, walking the macrobatches in reverse
+  int nc = 0, replayed = 0, resident_rows = 0, m = nm - 1;
+  while (m >= 0 && resident[m]) {
+    tb.shift_bwd[m] = tb.shift_fwd[m];
+    tb.replay[m] = 0;
+    resident_rows += seg_rows(m);
+    --m;
+  }
+  if (m + 1 < nm) {
+    tb.chunk[0] = m + 1;
+    tb.chunk[1] = nm;
+    tb.chunk[2] = 1;
+    nc = 1;
+  }
+  while (m >= 0) {
+    const int hi = m + 1;
+    int rows_c = 0;
+    do {
+      rows_c += seg_rows(m);
+      --m;
+    } while (m >= 0 && rows_c + seg_rows(m) <= ring_rows);
+    int pos = 0;
+    for (int q = m + 1; q < hi; ++q) {
+      tb.replay[q] = 1;
+      tb.shift_bwd[q] = pos - tb.seg_poff[q * El];
+      pos += seg_rows(q);
+    }
+    replayed += rows_c;
+    tb.chunk[4 * nc] = m + 1;
+    tb.chunk[4 * nc + 1] = hi;
+    tb.chunk[4 * nc + 2] = 1;
+    ++nc;
+  }
+  if (nc == 0) {  // no rows at all: one empty chunk still writes the (zero) gradients
+    tb.chunk[0] = tb.chunk[1] = 0;
+    tb.chunk[2] = 1;
+    nc = 1;
+  }
+  for (int c = 0; c < M; ++c) {
+    if (c < nc) {
+      tb.chunk[4 * c + 3] = nc == 1 ? 0 : (c == 0 ? 1 : 2);
+    } else {
+      tb.chunk[4 * c] = tb.chunk[4 * c + 1] = tb.chunk[4 * c + 2] = tb.chunk[4 * c + 3] = 0;
+    }
+  }
+  tb.plan[PLAN_N_MACRO] = nm;
+  tb.plan[PLAN_N_CHUNKS] = nc;
+  tb.plan[PLAN_ROWS] = row;
+  tb.plan[PLAN_REPLAYED] = replayed;
+  tb.plan[PLAN_RESIDENT] = resident_rows;
+  tb.plan[PLAN_RING_ROWS] = ring_rows;
+}
+
+// Backward chunk c: re-dispatch the X rows of every macrobatch marked for replay
+// into the ring at its backward position.  Resident macrobatches are left alone.
+__global__ void __launch_bounds__(128) k_replay(const __nv_bfloat16* __restrict__ X, const int* __restrict__ row_asg,
+                                                StreamTables tb, int El, int c, int k, int d,
+                                                __nv_bfloat16* __restrict__ ring) {
+  if (!tb.chunk[4 * c + 2]) return;
+  const int m_lo = tb.chunk[4 * c], m_hi = tb.chunk[4 * c + 1];
+  const int nv = d / 8;
+  for (int m = m_lo; m < m_hi; ++m) {
+    if (!tb.replay[m]) continue;
+    const int r0 = tb.seg_poff[m * El], r1 = tb.seg_poff[(m + 1) * El];
+    const int sh = tb.shift_bwd[m];
+    for (int64_t R = r0 + blockIdx.x; R < r1; R += gridDim.x) {
+      const int a = row_asg[R];
+      uint4* out = reinterpret_cast<uint4*>(ring + (R + sh) * d);
+      if (a >= 0) {
+        const uint4* in = reinterpret_cast<const uint4*>(X + static_cast<size_t>(a / k) * d);
+        for (int i = threadIdx.x; i < nv; i += blockDim.x) out[i] = __ldg(in + i);
+      } else {
+        const uint4 z = make_uint4(0, 0, 0, 0);
+        for (int i = threadIdx.x; i < nv; i += blockDim.x) out[i] = z;
+      }
+    }
+  }
+}
+
+// dW_gate / dW_up (bf16) from the fp32 accumulator when the backward used several chunks.
+__global__ void __launch_bounds__(256) k_finish_acc(const float* __restrict__ acc, const int* __restrict__ plan,
+                                                    size_t n_each, __nv_bfloat16* __restrict__ dWg,
+                                                    __nv_bfloat16* __restrict__ dWu) {
+  if (plan[PLAN_N_CHUNKS] <= 1) return;  // the wgrad epilogue already wrote bf16
+  const size_t n4 = n_each / 4;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < 2 * n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 v = reinterpret_cast<const float4*>(acc)[i];
+    __nv_bfloat16* dst = i < n4 ? dWg + 4 * i : dWu + 4 * (i - n4);
+    uint2 u;
+    u.x = pack_bf16(v.x, v.y);
+    u.y = pack_bf16(v.z, v.w);
+    *reinterpret_cast<uint2*>(dst) = u;
+  }
+}
+
 // local views of the routing table for the test hook
 __global__ void k_export_routing(const int* __restrict__ counts, const int* __restrict__ offsets,
                                  const int* __restrict__ poff, const int* __restrict__ perm_tok, int first, int El,
@@ -397,19 +599,48 @@ cudaError_t launch_scan(const Layout& L, const Ctx& c, cudaStream_t st) {
   return cudaGetLastError();
 }
 cudaError_t launch_scatter(const Layout& L, const Ctx& c, cudaStream_t st) {
-  k_scatter<<<L.nblk, 32, 0, st>>>(c.ids, c.gates, c.hist, c.offsets, c.poff, static_cast<int>(L.T), L.E, L.k,
-                                   L.first, L.El, c.perm_tok, c.perm_asg, c.slot_row, c.row_asg, c.row_gate);
+  const bool streamed = L.M > 0;
+  k_scatter<<<L.nblk, 32, 0, st>>>(c.ids, c.gates, c.hist, c.offsets, streamed ? c.tab.seg_poff : c.poff,
+                                   static_cast<int>(L.T), L.E, L.k, L.first, L.El, static_cast<int>(L.T_mb),
+                                   streamed ? c.tab.mb_of : nullptr, streamed ? c.tab.cum : nullptr, c.perm_tok,
+                                   c.perm_asg, c.slot_row, c.row_asg, c.row_gate);
+  return cudaGetLastError();
+}
+cudaError_t launch_gather_range(const Layout& L, const Ctx& c, const __nv_bfloat16* src, const int* lo, const int* hi,
+                                const int* shift, int64_t max_rows, __nv_bfloat16* dst, cudaStream_t st) {
+  const int grid = static_cast<int>(max_rows < 148 * 16 ? (max_rows > 0 ? max_rows : 1) : 148 * 16);
+  k_gather_rows<<<grid, 128, 0, st>>>(src, c.row_asg, lo, hi, shift, L.k, L.d, dst);
   return cudaGetLastError();
 }
 cudaError_t launch_gather_rows(const Layout& L, const Ctx& c, const __nv_bfloat16* src, __nv_bfloat16* dst,
                                cudaStream_t st) {
-  const int grid = static_cast<int>(L.RP < 148 * 16 ? L.RP : 148 * 16);
-  k_gather_rows<<<grid, 128, 0, st>>>(src, c.row_asg, c.hdr, L.k, L.d, L.RP, dst);
-  return cudaGetLastError();
+  if (L.M > 0)  // all rows of the stream
+    return launch_gather_range(L, c, src, c.tab.seg_poff, c.tab.seg_poff + L.M * L.El, nullptr, L.RP, dst, st);
+  return launch_gather_range(L, c, src, c.poff, c.poff + L.El, nullptr, L.RP, dst, st);
 }
 cudaError_t launch_combine(const Layout& L, const Ctx& c, const __nv_bfloat16* Oprime, __nv_bfloat16* Y,
-                           cudaStream_t st) {
-  k_combine<<<static_cast<unsigned>(L.T), 128, 0, st>>>(Oprime, c.slot_row, L.k, L.d, Y);
+                           cudaStream_t st, const int* mb_range) {
+  const int64_t n = mb_range ? L.T_mb * L.M : L.T;
+  const int grid = static_cast<int>(n < 148 * 16 ? (n > 0 ? n : 1) : 148 * 16);
+  k_combine<<<grid, 128, 0, st>>>(Oprime, c.slot_row, L.k, L.d, static_cast<int>(L.T), mb_range,
+                                  static_cast<int>(L.T_mb), Y);
+  return cudaGetLastError();
+}
+cudaError_t launch_plan(const Layout& L, const Ctx& c, int ring_rows, int min_rows, cudaStream_t st) {
+  k_plan<<<1, 32, 0, st>>>(c.hist, c.counts, static_cast<int>(L.T_mb / kTokensPerBlock), L.nblk, L.M, L.E, L.first,
+                           L.El, ring_rows, min_rows, c.tab);
+  return cudaGetLastError();
+}
+cudaError_t launch_replay(const Layout& L, const Ctx& c, int chunk, const __nv_bfloat16* X, __nv_bfloat16* ring,
+                          int64_t ring_rows, cudaStream_t st) {
+  const int grid = static_cast<int>(ring_rows < 148 * 16 ? ring_rows : 148 * 16);
+  k_replay<<<grid, 128, 0, st>>>(X, c.row_asg, c.tab, L.El, chunk, L.k, L.d, ring);
+  return cudaGetLastError();
+}
+cudaError_t launch_finish_acc(const Layout& L, const Ctx& c, __nv_bfloat16* dW_gate, __nv_bfloat16* dW_up,
+                              cudaStream_t st) {
+  const size_t n_each = static_cast<size_t>(L.El) * L.d * L.I;
+  k_finish_acc<<<148 * 8, 256, 0, st>>>(c.acc32, c.tab.plan, n_each, dW_gate, dW_up);
   return cudaGetLastError();
 }
 cudaError_t launch_router_bwd(const Layout& L, const Ctx& c, cudaStream_t st) {

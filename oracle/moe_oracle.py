@@ -388,3 +388,75 @@ def mx_dequantize(codes, sbytes, axis: int = -1, block: int = 32) -> np.ndarray:
     vals = e4m3_decode(c).reshape(c.shape[:-1] + (c.shape[-1] // block, block))
     vals = vals * np.ldexp(1.0, s - 127)[..., None]
     return np.moveaxis(vals.reshape(c.shape), -1, axis)
+
+
+# ----------------------------------------------------------------------------
+# Ring-streamed layer ("Three design decisions that matter", bullets 2 and 3):
+# minibatches grouped into macrobatches of at least two full waves of
+# grouped-GEMM tiles, dispatched rows cycled through a fixed ring, the ring
+# walked in reverse in the backward with replay of what was overwritten.
+# Readings: a macrobatch also closes before a minibatch that would not fit in
+# the ring with it; a segment that would run past the ring's end restarts at
+# row 0; the backward reuses the macrobatches still intact (a suffix in time)
+# and replays older ones in groups of consecutive macrobatches that fit in the
+# ring together.  The layer's values do not depend on the plan.
+# ----------------------------------------------------------------------------
+def stream_plan(mb_counts, ring_rows: int, min_rows: int, P: int = P_PAD) -> dict:
+    """mb_counts[b][el]: assignments of local expert el in minibatch b."""
+    mb_counts = np.asarray(mb_counts, dtype=np.int64)
+    M, El = mb_counts.shape
+
+    def padded(c):
+        return int(np.sum((np.asarray(c) + P - 1) // P * P))
+
+    macro, cur, b0 = [], np.zeros(El, dtype=np.int64), 0
+    for b in range(M):
+        if b > b0 and padded(cur + mb_counts[b]) > ring_rows:
+            macro.append((b0, b, cur.copy()))
+            cur[:] = 0
+            b0 = b
+        cur += mb_counts[b]
+        if padded(cur) >= min_rows:
+            macro.append((b0, b + 1, cur.copy()))
+            cur[:] = 0
+            b0 = b + 1
+    if b0 < M:
+        macro.append((b0, M, cur.copy()))
+    seg_poff, rows, ring_start, sizes, wp, row = [], [], [], [], 0, 0
+    for (_, _, cnt) in macro:
+        starts = []
+        for el in range(El):
+            starts.append(row)
+            row += (int(cnt[el]) + P - 1) // P * P
+        seg_poff.append(starts)
+        size = row - starts[0]
+        if wp + size > ring_rows:
+            wp = 0
+        ring_start.append(wp)
+        sizes.append(size)
+        wp += size
+    n = len(macro)
+    resident = []
+    for m in range(n):
+        a0, a1 = ring_start[m], ring_start[m] + sizes[m]
+        resident.append(all(not (sizes[m] > 0 and sizes[q] > 0 and ring_start[q] < a1 and a0 < ring_start[q] + sizes[q])
+                            for q in range(m + 1, n)))
+    chunks, m = [], n - 1
+    while m >= 0 and resident[m]:
+        m -= 1
+    if m + 1 < n:
+        chunks.append((m + 1, n))
+    replayed = 0
+    while m >= 0:
+        hi, rows_c = m + 1, 0
+        while True:
+            rows_c += sizes[m]
+            m -= 1
+            if m < 0 or rows_c + sizes[m] > ring_rows:
+                break
+        chunks.append((m + 1, hi))
+        replayed += rows_c
+    if not chunks:
+        chunks = [(0, 0)]
+    return dict(macro=[(a, b) for a, b, _ in macro], seg_poff=seg_poff, rows=row, ring_start=ring_start,
+                sizes=sizes, resident=resident, chunks=chunks, replayed=replayed)
