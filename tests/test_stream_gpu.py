@@ -74,9 +74,9 @@ def test_streamed_layer(T_mb, M, d, E, k, I, first, num, ring_mult, seed):
     assert plan["seg_poff"][:n * El].reshape(n, El).tolist() == op["seg_poff"]
     assert plan["ring_start"][:n].tolist() == op["ring_start"]
     assert [tuple(plan["chunk"][4 * c:4 * c + 2]) for c in range(len(op["chunks"]))] == op["chunks"]
-    if ring_mult < 2:
+    if ring_mult == 1.0:
         assert op["replayed"] > 0 and len(op["chunks"]) > 1  # the case exercises replay and accumulation
-    else:
+    if ring_mult >= 100:
         assert op["replayed"] == 0
 
     # bit-identical second run
