@@ -55,11 +55,40 @@ def load_peaks():
 
 
 def workload_config(w: IN.Workload) -> dict:
-    routing = "zipf(1.2) bias, hottest ~10x mean" if w.zipf else "near-uniform (W_r ~ N(0, 0.02^2))"
-    return {"workload": f"{w.name}: T={w.T} d={w.d} E={w.E} top_k={w.k} I={w.I} bf16, {routing}",
-            "T": w.T, "d": w.d, "E": w.E, "top_k": w.k, "I": w.I, "precision": "mxfp8" if w.mxfp8 else "bf16",
-            "seed": w.seed, "l2": "no flush: expert weights (%.1f GB) exceed the 126 MB L2 and stream every step"
-            % (3 * w.El * w.d * w.I * 2 / 1e9), "parallelism": "replicas"}
+    if w.stream_M:
+        routing = (f"{w.El} local experts of {w.E}, each receiving {w.local_tokens} tokens over the stream; "
+                   f"{w.stream_M} minibatches x {w.T} tokens through a {w.ring_bytes >> 20} MiB ring")
+        l2 = ("no flush: the step streams %.2f GB of tokens (X, dY, the dispatched rows and their "
+              "activations) through HBM, far beyond the 126 MB L2" % (4 * w.tokens * w.d * 2 / 1e9))
+    else:
+        routing = "zipf(1.2) bias, hottest ~10x mean" if w.zipf else "near-uniform (W_r ~ N(0, 0.02^2))"
+        l2 = ("no flush: expert weights (%.1f GB) exceed the 126 MB L2 and stream every step"
+              % (3 * w.El * w.d * w.I * 2 / 1e9))
+        if needs_flush(w):
+            l2 = "L2 flushed (256 MB write) between timed steps; each step timed on its own"
+    return {"workload": f"{w.name}: T={w.tokens} d={w.d} E={w.E} top_k={w.k} I={w.I} bf16, {routing}",
+            "T": w.tokens, "d": w.d, "E": w.E, "top_k": w.k, "I": w.I, "precision": "mxfp8" if w.mxfp8 else "bf16",
+            "seed": w.seed, "l2": l2, "parallelism": "replicas"}
+
+
+L2_BYTES = 126 << 20
+
+
+def needs_flush(w: IN.Workload) -> bool:
+    """Workloads whose weights and tokens fit in L2 flush it between timed steps."""
+    return 3 * w.El * w.d * w.I * 2 + 2 * w.tokens * w.d * 2 < 2 * L2_BYTES
+
+
+def local_rows(w: IN.Workload) -> int:
+    return w.El * w.local_tokens if w.local_tokens else w.tokens * w.k
+
+
+def algorithmic_flops(w: IN.Workload) -> dict:
+    rows, dI = local_rows(w), w.d * w.I
+    return {"gemm_gateup_swiglu": 4 * dI * rows, "gemm_down_combw": 2 * dI * rows,
+            "gemm_dgrad_down_swiglu_bwd": 2 * dI * rows, "gemm_dgrad_gateup": 4 * dI * rows,
+            "gemm_wgrad_gateup": 4 * dI * rows, "gemm_wgrad_down": 2 * dI * rows,
+            "router_logits": 2 * w.tokens * w.d * w.E}
 
 
 # ----------------------------------------------------------------------------
@@ -67,8 +96,8 @@ def workload_config(w: IN.Workload) -> dict:
 # rows = T*k routed assignments; weights of all local experts; bf16 = 2 bytes
 # ----------------------------------------------------------------------------
 def algorithmic_bytes(w: IN.Workload) -> dict:
-    T, d, E, I, k, El = w.T, w.d, w.E, w.I, w.k, w.El
-    rows = T * k
+    T, d, E, I, k, El = w.tokens, w.d, w.E, w.I, w.k, w.El
+    rows = local_rows(w)
     W1 = El * d * I * 2  # one expert weight matrix family (gate, up or down), bytes
     return {
         "router_logits": T * d * 2 + d * E * 2 + T * E * 4,
@@ -192,19 +221,25 @@ def oracle_sample(w: IN.Workload, x_cpu: dict, m: int) -> float:
     b = None if x_cpu["bias"] is None else f64(x_cpu["bias"])
     Wg, Wu, Wd = (f64(x_cpu[n][:m]) for n in ("W_gate", "W_up", "W_down"))
     t0 = time.perf_counter()
-    _, ctx = O.forward(X, Wr, b, Wg, Wu, Wd, w.k, first_local=0, num_local=m)
+    _, ctx = O.forward(X, Wr, b, lambda e: Wg[e - w.first_local], lambda e: Wu[e - w.first_local],
+                       lambda e: Wd[e - w.first_local], w.k, first_local=w.first_local, num_local=m)
     O.backward(ctx, dY)
     return time.perf_counter() - t0
 
 
 def cpu_inputs(w: IN.Workload, m: int) -> dict:
     """Host copies of the inputs the sample needs (CPU generator; same distributions)."""
-    x = {"X": IN._normal((w.T, w.d), 1.0, IN._seed(w.seed, w.name, "X"), "cpu"),
+    x = {"X": IN._normal((w.tokens, w.d), 1.0, IN._seed(w.seed, w.name, "X"), "cpu"),
          "W_r": IN._normal((w.d, w.E), 0.02, IN._seed(w.seed, w.name, "W_r"), "cpu"),
-         "dY": IN._normal((w.T, w.d), 1.0, IN._seed(w.seed, w.name, "dY"), "cpu")}
+         "dY": IN._normal((w.tokens, w.d), 1.0, IN._seed(w.seed, w.name, "dY"), "cpu")}
     for n in ("W_gate", "W_up", "W_down"):
-        x[n] = torch.stack([IN.expert_weights(w, n, e, "cpu") for e in range(m)])
-    x["bias"] = IN.zipf_bias(w, x["X"], x["W_r"]) if w.zipf else None
+        x[n] = torch.stack([IN.expert_weights(w, n, w.first_local + e, "cpu") for e in range(m)])
+    if w.zipf:
+        x["bias"] = IN.zipf_bias(w, x["X"], x["W_r"])
+    elif w.local_tokens:
+        x["bias"] = IN.local_load_bias(w, x["X"], x["W_r"])
+    else:
+        x["bias"] = None
     return x
 
 
@@ -220,13 +255,15 @@ def blas_threads() -> int:
 
 
 def cpu_baseline(w: IN.Workload, m1: int = 4, m2: int = 8) -> dict:
+    m2 = min(m2, w.El)
+    m1 = min(m1, max(m2 // 2, 1))
     x = cpu_inputs(w, m2)
     t1 = oracle_sample(w, x, m1)
     t2 = oracle_sample(w, x, m2)
     per_expert = max(t2 - t1, 0.0) / (m2 - m1)
     t_full = t1 + per_expert * (w.El - m1)
-    return {"value": w.T / t_full, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": (f"fp64 numpy oracle, all {w.T} tokens routed, fwd+bwd of {m1} and {m2} of {w.El} experts "
+    return {"value": w.tokens / t_full, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"fp64 numpy oracle, all {w.tokens} tokens routed, fwd+bwd of {m1} and {m2} of {w.El} experts "
                        f"({t1:.1f} s, {t2:.1f} s); time extrapolated linearly to {w.El} experts = {t_full:.1f} s "
                        "per full fwd+bwd")}
 
@@ -272,9 +309,9 @@ def run_reference(args, w: IN.Workload, world: int, rank: int):
     t4 = oracle_sample(w, x, 4)
     t2 = statistics.median(ts)
     t_full = t2 + max(t4 - t2, 0.0) / 2 * (w.El - 2)
-    value = w.T / t_full
+    value = w.tokens / t_full
     cores = blas_threads()
-    sample = (f"fp64 numpy oracle per step: all {w.T} tokens routed + fwd/bwd of 2 of {w.El} experts "
+    sample = (f"fp64 numpy oracle per step: all {w.tokens} tokens routed + fwd/bwd of 2 of {w.El} experts "
               f"(median {t2:.2f} s over {args.steps} steps); per-expert cost from a 4-expert run, "
               f"extrapolated to {w.El} experts = {t_full:.1f} s per layer fwd+bwd")
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
@@ -293,9 +330,14 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     torch.cuda.set_device(dev)
     peaks, peak_kind = load_peaks()
     x = IN.make_inputs(w, device=dev)
-    layer = B.MoELayer(w.T, w.d, w.E, w.I, w.k, device=dev)
-    Y = torch.empty(w.T, w.d, dtype=torch.bfloat16, device=dev)
-    grads = dict(dX=torch.empty(w.T, w.d, dtype=torch.bfloat16, device=dev),
+    if w.stream_M:
+        layer = B.MoEStream(w.T, w.d, w.E, w.I, w.k, w.stream_M, w.ring_bytes, w.first_local, w.num_local,
+                            device=dev)
+    else:
+        layer = B.MoELayer(w.T, w.d, w.E, w.I, w.k, device=dev)
+    NT = w.tokens
+    Y = torch.empty(NT, w.d, dtype=torch.bfloat16, device=dev)
+    grads = dict(dX=torch.empty(NT, w.d, dtype=torch.bfloat16, device=dev),
                  dW_gate=torch.empty_like(x["W_gate"]), dW_up=torch.empty_like(x["W_up"]),
                  dW_down=torch.empty_like(x["W_down"]),
                  dW_r=torch.empty(w.d, w.E, dtype=torch.float32, device=dev))
@@ -320,12 +362,25 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step(x["X"], x["dY"], Y, grads)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    if needs_flush(w):
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for a, b in evs:
+            flush.fill_(1)
+            a.record(stream)
+            step(x["X"], x["dY"], Y, grads)
+            b.record(stream)
+        torch.cuda.synchronize()
+        t_local = sum(a.elapsed_time(b) for a, b in evs) / 1e3
+    else:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step(x["X"], x["dY"], Y, grads)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t_local = e0.elapsed_time(e1) / 1e3
     barrier(world)
     clk = clocks.stop()
     launches = B.moe_kernel_launches() - launches0
@@ -334,10 +389,10 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     st = layer.error()
     if st != B.MOE_OK:
         raise RuntimeError("device error in the timed region: " + B.status_string(st))
-    t = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+    t = max_over_ranks(t_local, world)
 
     # ---------------- end to end through host buffers ----------------
-    hX = torch.empty(w.T, w.d, dtype=torch.bfloat16, pin_memory=True)
+    hX = torch.empty(NT, w.d, dtype=torch.bfloat16, pin_memory=True)
     hdY = torch.empty_like(hX, pin_memory=True)
     hY = torch.empty_like(hX, pin_memory=True)
     hdX = torch.empty_like(hX, pin_memory=True)
@@ -371,28 +426,42 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
 
     if rank != 0:
         return
-    tokens = w.T * args.steps * world
+    tokens = NT * args.steps * world
     flops = w.model_flops() * args.steps * world
     value = tokens / t
     tflops = flops / t / 1e12
     per_gpu_tflops = tflops / world
     algo = algorithmic_bytes(w)
+    aflops = algorithmic_flops(w)
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    bf16 = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     kern = {}
     for name, (ms, n) in sorted(prof.items(), key=lambda kv: -kv[1][0]):
-        avg = ms / n
-        e = {"ms_per_launch": avg, "launches": n, "share": ms / (t * 1e3)}
+        steps = args.steps
+        e = {"ms_per_step": ms / steps, "launches_per_step": n / steps, "share": ms / (t * 1e3)}
+        sec = ms / steps / 1e3  # the kernel's time in one step (all its launches)
         if name in algo:
             e["algorithmic_GB"] = algo[name] / 1e9
-            e["achieved_GBs"] = algo[name] / (avg / 1e3) / 1e9
+            e["achieved_GBs"] = algo[name] / sec / 1e9
+        if name in aflops:
+            e["achieved_TFLOPs"] = aflops[name] / sec / 1e12
+            # the binding resource: the larger of the two times at peak
+            e["bound"] = "tensor" if aflops[name] / (bf16 * 1e12) > algo.get(name, 0) / (hbm * 1e9) else "hbm"
+        else:
+            e["bound"] = "hbm"
         kern[name] = e
     top = max(kern.items(), key=lambda kv: kv[1]["share"])[0]
-    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    ach = kern[top].get("achieved_GBs")
-    roof = {"kernel": top, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
-            "frac": (ach / hbm) if ach else None, "traffic": ncu_traffic(top, w.name),
-            "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
-            if peak_kind == "measured" else "fallback 6.65 TB/s"}
-    bf16 = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    if kern[top]["bound"] == "tensor":
+        ach = kern[top]["achieved_TFLOPs"]
+        roof = {"kernel": top, "bound": "tensor", "achieved": ach, "peak": bf16, "unit": "TFLOP/s",
+                "frac": ach / bf16, "traffic": ncu_traffic(top, w.name),
+                "peak_source": f"{peak_kind} sustained bf16 GEMM (MEASURED_PEAKS.json bf16_tflops_sustained)"}
+    else:
+        ach = kern[top].get("achieved_GBs")
+        roof = {"kernel": top, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+                "frac": (ach / hbm) if ach else None, "traffic": ncu_traffic(top, w.name),
+                "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6.65 TB/s"}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -401,14 +470,18 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
         "tflops": tflops, "pct_of_bf16_peak": 100.0 * per_gpu_tflops / bf16,
         "peak_note": f"bf16 sustained {bf16} TFLOP/s ({peak_kind}); model FLOPs 18 d I T k + 6 T d E per step",
         "roofline": roof,
-        "e2e": {"value": tokens / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": 2 * w.T * w.d * 2,
-                "d2h_bytes_per_step": 2 * w.T * w.d * 2,
+        "e2e": {"value": tokens / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": 2 * NT * w.d * 2,
+                "d2h_bytes_per_step": 2 * NT * w.d * 2,
                 "note": "X, dY copied in from pinned host memory; Y, dX copied back; weights and their gradients "
                         "stay in HBM"},
         "gpu_launches": int(launches),
         "clocks": clk,
         "kernels": kern,
     }
+    if w.stream_M:
+        pl = layer.plan()["plan"]
+        line["stream_plan"] = {"macrobatches": int(pl[0]), "backward_chunks": int(pl[1]), "padded_rows": int(pl[2]),
+                               "replayed_rows": int(pl[3]), "resident_rows": int(pl[4]), "ring_rows": int(pl[5])}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)

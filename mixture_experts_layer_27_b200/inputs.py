@@ -40,14 +40,23 @@ class Workload:
     first_local: int = 0
     num_local: int = 0          # 0 = all experts are local
     seed: int = 0
+    stream_M: int = 0           # > 0: M minibatches of T tokens through a ring of ring_bytes
+    ring_bytes: int = 0
+    local_tokens: int = 0       # streamed slice: assignments each local expert receives over the stream
 
     @property
     def El(self) -> int:
         return self.num_local or self.E
 
+    @property
+    def tokens(self) -> int:
+        """Tokens per step (all minibatches of a streamed workload)."""
+        return self.T * max(self.stream_M, 1)
+
     def model_flops(self) -> float:
-        """fwd+bwd model FLOPs: 18 d I per assignment (6 fwd, 12 bwd) + 6 T d E router."""
-        return 18.0 * self.d * self.I * self.T * self.k + 6.0 * self.T * self.d * self.E
+        """fwd+bwd model FLOPs: 18 d I per local assignment (6 fwd, 12 bwd) + 6 T d E router."""
+        assign = self.El * self.local_tokens if self.local_tokens else self.tokens * self.k
+        return 18.0 * self.d * self.I * assign + 6.0 * self.tokens * self.d * self.E
 
 
 WORKLOADS = {
@@ -59,6 +68,11 @@ WORKLOADS = {
     # ~3 GB case for profiler captures (weights still exceed the 126 MB L2)
     "dsv3_e16": Workload("dsv3_e16", 128, 7168, 16, 8, 2048),
 }
+# Per-rank expert slice as at EP64: 6 local experts of 384, 16 minibatches of 2048
+# tokens streamed through a 256 MiB ring; n = tokens each local expert receives.
+for _n in (512, 1024, 2048, 2368, 4096, 8192, 16384):
+    WORKLOADS[f"ep64_n{_n}"] = Workload(f"ep64_n{_n}", 2048, 7168, 384, 8, 2048, first_local=0, num_local=6,
+                                        stream_M=16, ring_bytes=256 << 20, local_tokens=_n)
 
 
 def _seed(base: int, *names) -> int:
@@ -85,8 +99,10 @@ def expert_weights(w: Workload, name: str, e: int, device="cpu") -> torch.Tensor
 
 
 def make_inputs(w: Workload, device="cpu", T: int | None = None) -> dict:
-    """All layer inputs for workload w (T may be overridden to sub-sample tokens)."""
-    T = T or w.T
+    """All layer inputs for workload w (T may be overridden to sub-sample tokens).
+
+    Streamed workloads get all M * T tokens; only the local experts' weights."""
+    T = T or w.tokens
     out = {
         "X": _normal((T, w.d), 1.0, _seed(w.seed, w.name, "X"), device),
         "W_r": _normal((w.d, w.E), 0.02, _seed(w.seed, w.name, "W_r"), device),
@@ -99,8 +115,31 @@ def make_inputs(w: Workload, device="cpu", T: int | None = None) -> dict:
         for el in range(El):
             t[el] = expert_weights(w, name, w.first_local + el, device)
         out[name] = t
-    out["bias"] = zipf_bias(w, out["X"], out["W_r"]) if w.zipf else None
+    if w.zipf:
+        out["bias"] = zipf_bias(w, out["X"], out["W_r"])
+    elif w.local_tokens:
+        out["bias"] = local_load_bias(w, out["X"], out["W_r"])
+    else:
+        out["bias"] = None
     return out
+
+
+def local_load_bias(w: Workload, X: torch.Tensor, W_r: torch.Tensor, iters: int = 60) -> torch.Tensor:
+    """Router bias giving each local expert about w.local_tokens assignments over the
+    stream, the other experts sharing the rest evenly (same fixed-count calibration
+    as zipf_bias; torch.topk only measures the load)."""
+    dev = X.device
+    logits = X.float() @ W_r.float()
+    total = X.shape[0] * w.k
+    target = torch.full((w.E,), (total - w.El * w.local_tokens) / (w.E - w.El), dtype=torch.float64, device=dev)
+    target[w.first_local:w.first_local + w.El] = float(w.local_tokens)
+    b = torch.zeros(w.E, dtype=torch.float64, device=dev)
+    for _ in range(iters):
+        idx = torch.topk(logits + b.float(), w.k, dim=1).indices
+        obs = torch.bincount(idx.flatten(), minlength=w.E).double()
+        b += 0.5 * (torch.log(target) - torch.log(torch.clamp(obs, min=0.5)))
+        b -= b.mean()
+    return b.float()
 
 
 def zipf_target_shares(E: int, s: float = 1.2, hot_over_mean: float = 10.0) -> torch.Tensor:
