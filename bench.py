@@ -108,7 +108,7 @@ def algorithmic_bytes(w: IN.Workload) -> dict:
         "combine": rows * d * 2 + T * d * 2,
         "reverse_combine": T * d * 2 + rows * d * 2,
         "gemm_dgrad_down_swiglu_bwd": W1 + rows * d * 2 + 2 * rows * I * 2 + 3 * rows * I * 2,
-        "router_wgrad": rows * d * 2 + d * E * 4,
+        "router_wgrad": T * d * 2 + T * k * 8 + d * E * 4,  # X once, dl and ids, dW_r
         "gemm_dgrad_gateup": 2 * W1 + 2 * rows * I * 2 + rows * d * 2,
         "reverse_dispatch": rows * d * 2 + T * d * 2 + E * d * 2,
         "gemm_wgrad_gateup": rows * d * 2 + 2 * rows * I * 2 + 2 * W1,
