@@ -330,7 +330,9 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     torch.cuda.set_device(dev)
     peaks, peak_kind = load_peaks()
     x = IN.make_inputs(w, device=dev)
-    if w.stream_M:
+    if w.mxfp8:
+        layer = B.MoELayerMX(w.T, w.d, w.E, w.I, w.k, device=dev)
+    elif w.stream_M:
         layer = B.MoEStream(w.T, w.d, w.E, w.I, w.k, w.stream_M, w.ring_bytes, w.first_local, w.num_local,
                             device=dev)
     else:
@@ -343,9 +345,24 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
                  dW_r=torch.empty(w.d, w.E, dtype=torch.float32, device=dev))
     stream = torch.cuda.current_stream(dev)
 
-    def step(X, dY, Yout, g):
-        layer.forward(X, x["W_r"], x["bias"], x["W_gate"], x["W_up"], x["W_down"], Y=Yout)
-        layer.backward(X, x["W_r"], x["W_gate"], x["W_up"], x["W_down"], dY, out=g)
+    prep_ms = None
+    if w.mxfp8:
+        # quantised weights are prepared once per optimiser step, outside the layer step
+        layer.prepare(x["W_gate"], x["W_up"], x["W_down"])
+        pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        pa.record(stream)
+        layer.prepare(x["W_gate"], x["W_up"], x["W_down"])
+        pb.record(stream)
+        torch.cuda.synchronize()
+        prep_ms = pa.elapsed_time(pb)
+
+        def step(X, dY, Yout, g):
+            layer.forward(X, x["W_r"], x["bias"], Y=Yout)
+            layer.backward(X, x["W_r"], dY, out=g)
+    else:
+        def step(X, dY, Yout, g):
+            layer.forward(X, x["W_r"], x["bias"], x["W_gate"], x["W_up"], x["W_down"], Y=Yout)
+            layer.backward(X, x["W_r"], x["W_gate"], x["W_up"], x["W_down"], dY, out=g)
 
     for _ in range(args.warmup):
         step(x["X"], x["dY"], Y, grads)
@@ -478,6 +495,11 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
         "clocks": clk,
         "kernels": kern,
     }
+    if prep_ms is not None:
+        line["prepare_weights_ms"] = prep_ms
+        line["peak_note"] += ("; MXFP8: gate/up, down and both dgrads on block-scaled fp8 tensor cores, "
+                              "weight gradients bf16; % of bf16 peak shown (fp8 peak not measured)")
+        line["dtype"] = "mxfp8 (e4m3 + e8m0 scales) / bf16 wgrad"
     if w.stream_M:
         pl = layer.plan()["plan"]
         line["stream_plan"] = {"macrobatches": int(pl[0]), "backward_chunks": int(pl[1]), "padded_rows": int(pl[2]),

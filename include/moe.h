@@ -55,7 +55,8 @@ typedef enum moe_status {
 
 typedef enum moe_precision {
   MOE_BF16 = 0,  /* bf16 operands, fp32 accumulation */
-  MOE_MXFP8 = 1  /* E4M3 operands with one E8M0 scale per 32 along each GEMM's contraction dim */
+  MOE_MXFP8 = 1  /* E4M3 operands with one E8M0 scale per 32 along each GEMM's contraction dim:
+                    use moe_prepare_weights + moe_fwd_mx / moe_bwd_mx (moe_fwd / moe_bwd refuse it) */
 } moe_precision;
 
 /* Layer shape.  Experts [first_local_expert, first_local_expert + num_local_experts)
@@ -148,6 +149,40 @@ moe_status moe_profile_enable(int on);
 int moe_profile_read(int max_kernels, double* total_ms, int* launches);
 const char* moe_kernel_name(int kernel_id);
 unsigned long long moe_kernel_launches(void);
+
+/* ---------------------------------------------------------------------------
+ * MXFP8 mode (page 1: "It supports BF16 and MXFP8 precision modes").  Shapes
+ * carry prec = MOE_MXFP8.  E4M3 codes with one E8M0 scale per 32 values along
+ * each GEMM's contraction dimension (OCP MX: scale exponent = floor(log2 amax)
+ * - 8; codes rounded to nearest even, saturating at +-448).  The gate/up and
+ * down GEMMs and both dgrad GEMMs run on kind::mxf8f6f4 block-scaled tensor
+ * cores with both operands quantised; the two weight-gradient GEMMs contract
+ * over tokens and stay bf16.  The router stays bf16, so routing is the same in
+ * both modes; all outputs are bf16 (dW_r fp32).
+ *
+ * moe_prepare_weights quantises the bf16 master weights once (e.g. after each
+ * optimiser step) into `wq` (moe_weights_size bytes), laid out as ten regions,
+ * each starting on a 256-byte boundary:
+ *   [Wgu codes][Wgu scales] [Wd2 ..][..] [Wd3 ..][..] [Wg4 ..][..] [Wu4 ..][..]
+ *   Wgu [El*2I, d]: W_gate / W_up with K = d, rows per expert in blocks of 128 =
+ *        64 W_gate columns then the same 64 W_up columns;
+ *   Wd2 [El*d, I]: W_down transposed (K = I);   Wd3 [El*I, d]: W_down (K = d);
+ *   Wg4 [El*d, I]: W_gate (K = I);              Wu4 [El*d, I]: W_up (K = I).
+ * Codes are row-major bytes; the scales of a [R, K] region sit in 512-byte
+ * chunks, byte (r%32)*16 + ((r%128)/32)*4 + (k%128)/32 of chunk
+ * (r/128)*(K/128) + k/128 (the order the block-scaled MMA reads them in).
+ * moe_fwd_mx / moe_bwd_mx take the same arguments as moe_fwd / moe_bwd with
+ * wq in place of the bf16 expert weights; ctx and ws are sized by
+ * moe_ctx_size / moe_workspace_size of the MXFP8 shape. */
+size_t moe_weights_size(const moe_shape* shape);
+moe_status moe_prepare_weights(const moe_shape* shape, const void* W_gate, const void* W_up, const void* W_down,
+                               void* wq, size_t wq_bytes, void* stream);
+moe_status moe_fwd_mx(const moe_shape* shape, const void* X, const void* W_r, const float* bias, const void* wq,
+                      size_t wq_bytes, void* Y, void* ctx, size_t ctx_bytes, void* ws, size_t ws_bytes,
+                      void* stream);
+moe_status moe_bwd_mx(const moe_shape* shape, const void* X, const void* W_r, const void* wq, size_t wq_bytes,
+                      const void* dY, void* ctx, size_t ctx_bytes, void* dX, void* dW_gate, void* dW_up,
+                      void* dW_down, float* dW_r, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Ring-streamed layer (page 1, "Three design decisions that matter", bullet 3:

@@ -67,6 +67,12 @@ _SIGS = {
     "moe_bwd_stream": (ctypes.c_int, [_S, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, _P,
                                       _P, _P, _P, ctypes.c_size_t, _P, ctypes.c_size_t, _P]),
     "moe_debug_stream_plan": (ctypes.c_int, [_S, ctypes.c_int32, _P, _P, _P]),
+    "moe_weights_size": (ctypes.c_size_t, [_S]),
+    "moe_prepare_weights": (ctypes.c_int, [_S, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_fwd_mx": (ctypes.c_int, [_S, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, ctypes.c_size_t, _P, ctypes.c_size_t,
+                                  _P]),
+    "moe_bwd_mx": (ctypes.c_int, [_S, _P, _P, _P, ctypes.c_size_t, _P, _P, ctypes.c_size_t, _P, _P, _P, _P, _P, _P,
+                                  ctypes.c_size_t, _P]),
 }
 
 
@@ -209,9 +215,102 @@ def moe_debug_stream_plan(shape, M, ctx, tables, stream=None) -> int:
     return int(lib().moe_debug_stream_plan(ctypes.byref(shape), int(M), _ptr(ctx), _ptr(tables), _stream(stream)))
 
 
+def moe_weights_size(shape) -> int:
+    return int(lib().moe_weights_size(ctypes.byref(shape)))
+
+
+def moe_prepare_weights(shape, W_gate, W_up, W_down, wq, stream=None) -> int:
+    return int(lib().moe_prepare_weights(ctypes.byref(shape), _ptr(W_gate), _ptr(W_up), _ptr(W_down), _ptr(wq),
+                                         _nbytes(wq), _stream(stream)))
+
+
+def moe_fwd_mx(shape, X, W_r, bias, wq, Y, ctx, ws, stream=None) -> int:
+    return int(lib().moe_fwd_mx(ctypes.byref(shape), _ptr(X), _ptr(W_r), _ptr(bias), _ptr(wq), _nbytes(wq), _ptr(Y),
+                                _ptr(ctx), _nbytes(ctx), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def moe_bwd_mx(shape, X, W_r, wq, dY, ctx, dX, dW_gate, dW_up, dW_down, dW_r, ws, stream=None) -> int:
+    return int(lib().moe_bwd_mx(ctypes.byref(shape), _ptr(X), _ptr(W_r), _ptr(wq), _nbytes(wq), _ptr(dY), _ptr(ctx),
+                                _nbytes(ctx), _ptr(dX), _ptr(dW_gate), _ptr(dW_up), _ptr(dW_down), _ptr(dW_r),
+                                _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
 def check(status: int, what: str = "moe"):
     if status != MOE_OK:
         raise MoeError(status, what)
+
+
+class MoELayerMX:
+    """MXFP8 layer: prepared (quantised) weights + ctx / workspace owner."""
+
+    def __init__(self, T, d, E, I, top_k, first_local_expert=0, num_local_experts=0, device="cuda"):
+        import torch
+        self.shape = make_shape(T, d, E, I, top_k, MOE_MXFP8, first_local_expert, num_local_experts)
+        self.shape_bf16 = make_shape(T, d, E, I, top_k, MOE_BF16, first_local_expert, num_local_experts)
+        nc, nw, nq = moe_ctx_size(self.shape), moe_workspace_size(self.shape), moe_weights_size(self.shape)
+        if nc == 0 or nw == 0 or nq == 0:
+            raise MoeError(MOE_ERR_UNSUPPORTED, "shape")
+        self.ctx = torch.empty(nc, dtype=torch.uint8, device=device)
+        self.ws = torch.empty(nw, dtype=torch.uint8, device=device)
+        self.wq = torch.empty(nq, dtype=torch.uint8, device=device)
+        self.T, self.d, self.E, self.I, self.k = T, d, E, I, top_k
+        self.El = num_local_experts or (E - first_local_expert)
+
+    def prepare(self, W_gate, W_up, W_down, stream=None):
+        check(moe_prepare_weights(self.shape, W_gate, W_up, W_down, self.wq, stream), "moe_prepare_weights")
+
+    def forward(self, X, W_r, bias, Y=None, stream=None):
+        import torch
+        if Y is None:
+            Y = torch.empty(self.T, self.d, dtype=torch.bfloat16, device=X.device)
+        check(moe_fwd_mx(self.shape, X, W_r, bias, self.wq, Y, self.ctx, self.ws, stream), "moe_fwd_mx")
+        return Y
+
+    def backward(self, X, W_r, dY, out=None, stream=None):
+        import torch
+        if out is None:
+            dev = X.device
+            out = dict(dX=torch.empty(self.T, self.d, dtype=torch.bfloat16, device=dev),
+                       dW_gate=torch.empty(self.El, self.d, self.I, dtype=torch.bfloat16, device=dev),
+                       dW_up=torch.empty(self.El, self.d, self.I, dtype=torch.bfloat16, device=dev),
+                       dW_down=torch.empty(self.El, self.I, self.d, dtype=torch.bfloat16, device=dev),
+                       dW_r=torch.empty(self.d, self.E, dtype=torch.float32, device=dev))
+        check(moe_bwd_mx(self.shape, X, W_r, self.wq, dY, self.ctx, out["dX"], out["dW_gate"], out["dW_up"],
+                         out["dW_down"], out["dW_r"], self.ws, stream), "moe_bwd_mx")
+        return out
+
+    def weight_regions(self):
+        """Host numpy views (codes [R, K], scale chunks) of the five prepared weights."""
+        import numpy as np
+        a = self.wq.cpu().numpy()
+        El, d, I = self.El, self.d, self.I
+        out, o = {}, 0
+        for name, R, K in (("Wgu", El * 2 * I, d), ("Wd2", El * d, I), ("Wd3", El * I, d), ("Wg4", El * d, I),
+                           ("Wu4", El * d, I)):
+            codes = a[o:o + R * K].reshape(R, K)
+            o = (o + R * K + 255) // 256 * 256
+            sc = a[o:o + R * K // 32]
+            o = (o + R * K // 32 + 255) // 256 * 256
+            out[name] = (codes, sc, R, K)
+        return out
+
+    def routing(self):
+        return MoELayer.routing(self)
+
+    def logits(self):
+        return MoELayer.logits(self)
+
+    def error(self, stream=None) -> int:
+        return moe_get_error(self.ctx, stream)
+
+
+def unchunk_scales(chunks, R, K):
+    """[R, K/32] scale bytes from the 512-byte chunk order of a K-major fp8 operand."""
+    import numpy as np
+    r = np.arange(R)[:, None]
+    kb = np.arange(K // 32)[None, :]
+    idx = ((r // 128) * (K // 128) + (kb * 32) // 128) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + kb % 4
+    return chunks[idx]
 
 
 class MoEStream:
@@ -317,7 +416,8 @@ class MoELayer:
                  padded_offsets=torch.empty(El + 1, dtype=torch.int32, device=dev),
                  perm=torch.empty(max(T * k, 1), dtype=torch.int32, device=dev),
                  slot_row=torch.empty(T, k, dtype=torch.int32, device=dev))
-        check(moe_debug_routing(self.shape, self.ctx, r["ids"], r["gates"], r["counts"], r["offsets"],
+        check(moe_debug_routing(getattr(self, "shape_bf16", self.shape), self.ctx, r["ids"], r["gates"], r["counts"],
+                                r["offsets"],
                                 r["padded_offsets"], r["perm"], r["slot_row"]), "moe_debug_routing")
         torch.cuda.synchronize()
         n = int(r["offsets"][-1].item())
@@ -327,7 +427,7 @@ class MoELayer:
     def logits(self):
         import torch
         out = torch.empty(self.T, self.E, dtype=torch.float32, device=self.ws.device)
-        check(moe_debug_logits(self.shape, self.ws, out), "moe_debug_logits")
+        check(moe_debug_logits(getattr(self, "shape_bf16", self.shape), self.ws, out), "moe_debug_logits")
         return out
 
     def router_grad(self):

@@ -64,6 +64,10 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->abuf = take(RP * s.I * 2);
   L->bbuf = take(RP * s.I * 2);
   L->stab = take(M > 0 ? static_cast<size_t>(stream_table_words(M, El)) * 4 : 0);
+  L->mx = s.prec == MOE_MXFP8;
+  const size_t mxd = L->mx ? RP * s.d : 0, mxi = L->mx ? RP * s.I : 0;  // fp8 bytes; scales are 1/32 of that
+  L->xq = take(mxd);
+  L->xqs = take(mxd / 32);
   L->ctx_bytes = o;
 
   o = 0;
@@ -76,12 +80,34 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->dabuf = take(RP * s.I * 2);
   L->dbbuf = take(RP * s.I * 2);
   L->hgbuf = take(RP * s.I * 2);
-  L->dgpart = take(RP * (s.I / 256) * 4);
+  L->dgpart = take(RP * (s.I / 128) * 4);  // dg partials per n-tile (256 wide bf16, 128 wide MXFP8)
   L->dlasg = take(T * k * 4);
   L->wrt = take(static_cast<size_t>(s.E) * s.d * 2);
   L->dxperm = take(RP * s.d * 2);
   L->acc32 = take(M > 0 ? 2 * static_cast<size_t>(El) * s.d * s.I * 4 : 0);
+  L->hq = take(mxi);
+  L->hqs = take(mxi / 32);
+  L->dyq = take(mxd);
+  L->dyqs = take(mxd / 32);
+  L->daq = take(mxi);
+  L->daqs = take(mxi / 32);
+  L->dbq = take(mxi);
+  L->dbqs = take(mxi / 32);
   L->ws_bytes = o;
+  // prepared weights: [W_gate|W_up paired, K = d] [W_down^T, K = I] [W_down, K = d] [W_gate, K = I] [W_up, K = I]
+  o = 0;
+  const size_t w1 = static_cast<size_t>(El) * s.d * s.I;
+  L->wgu1 = take(2 * w1);
+  L->wgu1s = take(2 * w1 / 32);
+  L->wd2 = take(w1);
+  L->wd2s = take(w1 / 32);
+  L->wd3 = take(w1);
+  L->wd3s = take(w1 / 32);
+  L->wg4 = take(w1);
+  L->wg4s = take(w1 / 32);
+  L->wu4 = take(w1);
+  L->wu4s = take(w1 / 32);
+  L->wq_bytes = o;
   return true;
 }
 
@@ -119,6 +145,19 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
     c.tab.ring_start = t;
   }
   c.acc32 = nullptr;
+  c.xq = L.mx ? reinterpret_cast<uint8_t*>(C(L.xq)) : nullptr;
+  c.xqs = L.mx ? reinterpret_cast<uint8_t*>(C(L.xqs)) : nullptr;
+  c.hq = c.hqs = c.dyq = c.dyqs = c.daq = c.daqs = c.dbq = c.dbqs = nullptr;
+  if (ws && L.mx) {
+    c.hq = reinterpret_cast<uint8_t*>(W(L.hq));
+    c.hqs = reinterpret_cast<uint8_t*>(W(L.hqs));
+    c.dyq = reinterpret_cast<uint8_t*>(W(L.dyq));
+    c.dyqs = reinterpret_cast<uint8_t*>(W(L.dyqs));
+    c.daq = reinterpret_cast<uint8_t*>(W(L.daq));
+    c.daqs = reinterpret_cast<uint8_t*>(W(L.daqs));
+    c.dbq = reinterpret_cast<uint8_t*>(W(L.dbq));
+    c.dbqs = reinterpret_cast<uint8_t*>(W(L.dbqs));
+  }
   if (ws) {
     c.hist = reinterpret_cast<int*>(W(L.hist));
     c.logits = reinterpret_cast<float*>(W(L.logits));
@@ -174,6 +213,19 @@ static bool tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t o
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D fp8 (byte) tensor [outer, inner], box {128, 128}, 128-byte swizzle.
+static bool tmap_fp8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static int num_sms() {
   static int n = 0;
   if (n == 0) {
@@ -191,13 +243,13 @@ static int num_sms() {
 enum KernelId {
   K_ROUTER_LOGITS, K_TOPK, K_SCAN, K_SCATTER, K_DISPATCH, K_GEMM_GATEUP, K_GEMM_DOWN, K_COMBINE,
   K_REV_COMBINE, K_GEMM_DGRAD_DOWN, K_ROUTER_BWD, K_DWR, K_TRANSPOSE_WR, K_GEMM_DGRAD_GATEUP, K_REV_DISPATCH,
-  K_GEMM_WGRAD_GATEUP, K_GEMM_WGRAD_DOWN, K_PLAN, K_REPLAY, K_FINISH_ACC, K_NUM
+  K_GEMM_WGRAD_GATEUP, K_GEMM_WGRAD_DOWN, K_PLAN, K_REPLAY, K_FINISH_ACC, K_QUANT_WEIGHTS, K_NUM
 };
 static const char* kKernelNames[K_NUM] = {
     "router_logits", "topk_gating", "hist_scan", "stable_scatter", "dispatch", "gemm_gateup_swiglu",
     "gemm_down_combw", "combine", "reverse_combine", "gemm_dgrad_down_swiglu_bwd", "router_bwd", "router_wgrad",
     "transpose_wr", "gemm_dgrad_gateup", "reverse_dispatch", "gemm_wgrad_gateup", "gemm_wgrad_down",
-    "stream_plan", "ring_replay", "wgrad_accumulator_finish"};
+    "stream_plan", "ring_replay", "wgrad_accumulator_finish", "quantize_weights"};
 
 struct ProfRec {
   int kid;
@@ -294,6 +346,16 @@ const char* moe_status_string(moe_status st) {
     case MOE_ERR_NONFINITE: return "non-finite router logit";
   }
   return "unknown status";
+}
+
+static moe_status check_shape_mx(const moe_shape* s, Layout* L) {
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (s->prec != MOE_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->d <= 0 || s->E <= 0 || s->I <= 0 || s->top_k <= 0 || s->first_local_expert < 0 ||
+      s->num_local_experts < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!make_layout(*s, L)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
 }
 
 static moe_status check_shape(const moe_shape* s, Layout* L) {
@@ -747,6 +809,212 @@ moe_status moe_debug_stream_plan(const moe_shape* s, int32_t M, const void* ctx,
   MOE_TRY(cudaMemcpyAsync(tables, static_cast<const char*>(ctx) + L.stab,
                           static_cast<size_t>(stream_table_words(M, L.El)) * 4, cudaMemcpyDeviceToDevice,
                           static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// MXFP8 mode
+// ---------------------------------------------------------------------------
+size_t moe_weights_size(const moe_shape* s) {
+  Layout L;
+  if (check_shape_mx(s, &L) != MOE_OK) return 0;
+  return L.wq_bytes;
+}
+
+moe_status moe_prepare_weights(const moe_shape* s, const void* W_gate, const void* W_up, const void* W_down, void* wq,
+                               size_t wq_bytes, void* stream) {
+  Layout L;
+  const moe_status cs = check_shape_mx(s, &L);
+  if (cs != MOE_OK) return cs;
+  if (!W_gate || !W_up || !W_down || !wq) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_down) || !aligned16(wq)) return MOE_ERR_INVALID_ARG;
+  if (wq_bytes < L.wq_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto* w = static_cast<uint8_t*>(wq);
+  const auto* g = static_cast<const __nv_bfloat16*>(W_gate);
+  const auto* u = static_cast<const __nv_bfloat16*>(W_up);
+  const auto* dn = static_cast<const __nv_bfloat16*>(W_down);
+  const int64_t El = L.El;
+  MOE_TRY(timed(K_QUANT_WEIGHTS, st, [&] {  // gate/up for the forward: K = d, 64-row gate/up pairs
+    return launch_quant_weight(2, g, u, El * 2 * L.I, L.d, L.I, w + L.wgu1, w + L.wgu1s, st);
+  }));
+  MOE_TRY(timed(K_QUANT_WEIGHTS, st, [&] {  // down for the forward: K = I (transposed)
+    return launch_quant_weight(1, dn, nullptr, El * L.d, L.I, L.d, w + L.wd2, w + L.wd2s, st);
+  }));
+  MOE_TRY(timed(K_QUANT_WEIGHTS, st, [&] {  // down for the backward: K = d (as stored)
+    return launch_quant_weight(0, dn, nullptr, El * L.I, L.d, 0, w + L.wd3, w + L.wd3s, st);
+  }));
+  MOE_TRY(timed(K_QUANT_WEIGHTS, st, [&] {  // gate for the backward: K = I (as stored)
+    return launch_quant_weight(0, g, nullptr, El * L.d, L.I, 0, w + L.wg4, w + L.wg4s, st);
+  }));
+  MOE_TRY(timed(K_QUANT_WEIGHTS, st, [&] {  // up for the backward: K = I (as stored)
+    return launch_quant_weight(0, u, nullptr, El * L.d, L.I, 0, w + L.wu4, w + L.wu4s, st);
+  }));
+  return MOE_OK;
+}
+
+static MxParams mx_params(const Layout& L, const Ctx& c, int* status) {
+  MxParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.poff = c.poff;
+  p.nseg = L.El;
+  p.row_gate = c.row_gate;
+  p.El = L.El;
+  p.d = L.d;
+  p.I = L.I;
+  p.status = status;
+  return p;
+}
+
+moe_status moe_fwd_mx(const moe_shape* s, const void* X, const void* W_r, const float* bias, const void* wq,
+                      size_t wq_bytes, void* Y, void* ctx, size_t ctx_bytes, void* ws, size_t ws_bytes,
+                      void* stream) {
+  Layout L;
+  const moe_status cs = check_shape_mx(s, &L);
+  if (cs != MOE_OK) return cs;
+  const bool tok = s->T > 0;
+  if ((tok && (!X || !Y)) || !W_r || !wq || !ctx || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W_r) || !aligned16(wq) || !aligned16(Y) || !aligned16(ctx) || !aligned16(ws) ||
+      (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+    return MOE_ERR_INVALID_ARG;
+  if (ctx_bytes < L.ctx_bytes || ws_bytes < L.ws_bytes || wq_bytes < L.wq_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ctx c = make_ctx(L, ctx, ws);
+  MOE_TRY(cudaMemsetAsync(c.hdr, 0, HDR_WORDS * 4, st));
+  if (L.T == 0) return MOE_OK;
+  {
+    const moe_status r = route_tokens(L, c, X, W_r, bias, 0, st);
+    if (r != MOE_OK) return r;
+  }
+  MOE_TRY(timed(K_DISPATCH, st, [&] {
+    return launch_gather_rows_mx(L, c, static_cast<const __nv_bfloat16*>(X), c.xperm, c.xq, c.xqs, st);
+  }));
+  const int grid = num_sms();
+  int* status = c.hdr + HDR_STATUS;
+  const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
+  const auto* w = static_cast<const uint8_t*>(wq);
+  {
+    MxParams p = mx_params(L, c, status);
+    MOE_TMAP(tmap_fp8(&p.ta0, c.xq, L.d, RP));
+    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wgu1, L.d, El * 2 * L.I));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.sfa0 = p.sfa1 = c.xqs;
+    p.sfb0 = p.sfb1 = w + L.wgu1s;
+    p.out0 = c.abuf;
+    p.out1 = c.bbuf;
+    p.q0 = c.hq;
+    p.qs0 = c.hqs;
+    MOE_TRY(timed(K_GEMM_GATEUP, st, [&] { return launch_gemm_mx(MX_GATEUP, p, grid, st); }));
+  }
+  {
+    MxParams p = mx_params(L, c, status);
+    MOE_TMAP(tmap_fp8(&p.ta0, c.hq, L.I, RP));
+    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wd2, L.I, El * L.d));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.sfa0 = p.sfa1 = c.hqs;
+    p.sfb0 = p.sfb1 = w + L.wd2s;
+    p.out0 = c.obuf;
+    MOE_TRY(timed(K_GEMM_DOWN, st, [&] { return launch_gemm_mx(MX_DOWN, p, grid, st); }));
+  }
+  MOE_TRY(timed(K_COMBINE, st, [&] { return launch_combine(L, c, c.obuf, static_cast<__nv_bfloat16*>(Y), st); }));
+  return MOE_OK;
+}
+
+moe_status moe_bwd_mx(const moe_shape* s, const void* X, const void* W_r, const void* wq, size_t wq_bytes,
+                      const void* dY, void* ctx, size_t ctx_bytes, void* dX, void* dW_gate, void* dW_up,
+                      void* dW_down, float* dW_r, void* ws, size_t ws_bytes, void* stream) {
+  Layout L;
+  const moe_status cs = check_shape_mx(s, &L);
+  if (cs != MOE_OK) return cs;
+  const bool tok = s->T > 0;
+  if ((tok && (!X || !dY || !dX)) || !W_r || !wq || !ctx || !dW_gate || !dW_up || !dW_down || !dW_r || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W_r) || !aligned16(wq) || !aligned16(dY) || !aligned16(ctx) || !aligned16(dX) ||
+      !aligned16(dW_gate) || !aligned16(dW_up) || !aligned16(dW_down) || !aligned16(dW_r) || !aligned16(ws))
+    return MOE_ERR_INVALID_ARG;
+  if (ctx_bytes < L.ctx_bytes || ws_bytes < L.ws_bytes || wq_bytes < L.wq_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ctx c = make_ctx(L, ctx, ws);
+  if (L.T == 0) {
+    const size_t wexp = static_cast<size_t>(L.El) * L.d * L.I * 2;
+    MOE_TRY(cudaMemsetAsync(dW_gate, 0, wexp, st));
+    MOE_TRY(cudaMemsetAsync(dW_up, 0, wexp, st));
+    MOE_TRY(cudaMemsetAsync(dW_down, 0, wexp, st));
+    MOE_TRY(cudaMemsetAsync(dW_r, 0, static_cast<size_t>(L.d) * L.E * 4, st));
+    return MOE_OK;
+  }
+  const int grid = num_sms();
+  int* status = c.hdr + HDR_STATUS;
+  const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
+  const auto* w = static_cast<const uint8_t*>(wq);
+  MOE_TRY(timed(K_REV_COMBINE, st, [&] {
+    return launch_gather_rows_mx(L, c, static_cast<const __nv_bfloat16*>(dY), c.dyperm, c.dyq, c.dyqs, st);
+  }));
+  {
+    MxParams p = mx_params(L, c, status);
+    MOE_TMAP(tmap_fp8(&p.ta0, c.dyq, L.d, RP));
+    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wd3, L.d, El * L.I));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.sfa0 = p.sfa1 = c.dyqs;
+    p.sfb0 = p.sfb1 = w + L.wd3s;
+    p.in0 = c.abuf;
+    p.in1 = c.bbuf;
+    p.out0 = c.dabuf;
+    p.out1 = c.dbbuf;
+    p.out2 = c.hgbuf;
+    p.q0 = c.daq;
+    p.qs0 = c.daqs;
+    p.q1 = c.dbq;
+    p.qs1 = c.dbqs;
+    p.outf = c.dgpart;
+    MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm_mx(MX_DGRAD_DOWN, p, grid, st); }));
+  }
+  MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st, L.I / 128); }));
+  MOE_TRY(timed(K_DWR, st, [&] { return launch_dwr(L, c, static_cast<const __nv_bfloat16*>(X), dW_r, st); }));
+  MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
+    return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
+  }));
+  {
+    MxParams p = mx_params(L, c, status);
+    MOE_TMAP(tmap_fp8(&p.ta0, c.daq, L.I, RP));
+    MOE_TMAP(tmap_fp8(&p.ta1, c.dbq, L.I, RP));
+    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wg4, L.I, El * L.d));
+    MOE_TMAP(tmap_fp8(&p.tb1, w + L.wu4, L.I, El * L.d));
+    p.sfa0 = c.daqs;
+    p.sfa1 = c.dbqs;
+    p.sfb0 = w + L.wg4s;
+    p.sfb1 = w + L.wu4s;
+    p.out0 = c.dxperm;
+    MOE_TRY(timed(K_GEMM_DGRAD_GATEUP, st, [&] { return launch_gemm_mx(MX_DGRAD_GATEUP, p, grid, st); }));
+  }
+  MOE_TRY(timed(K_REV_DISPATCH, st, [&] { return launch_rev_dispatch(L, c, static_cast<__nv_bfloat16*>(dX), st); }));
+  // weight gradients contract over tokens and are written in bf16: the bf16 engine
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, c.xperm, L.d, RP, L.d, 64, 64));
+    MOE_TMAP(tmap_2d(&p.tb0, c.dabuf, L.I, RP, L.I, 64, 64));
+    MOE_TMAP(tmap_2d(&p.tb1, c.dbbuf, L.I, RP, L.I, 64, 64));
+    MOE_TMAP(tmap_2d(&p.to0, dW_gate, L.I, El * L.d, L.I, 64, 32));
+    MOE_TMAP(tmap_2d(&p.to1, dW_up, L.I, El * L.d, L.I, 64, 32));
+    p.ta1 = p.ta0;
+    p.out0 = static_cast<__nv_bfloat16*>(dW_gate);
+    p.out1 = static_cast<__nv_bfloat16*>(dW_up);
+    MOE_TRY(timed(K_GEMM_WGRAD_GATEUP, st, [&] { return launch_gemm(G_WGRAD_GATEUP, p, grid, st); }));
+  }
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, c.hgbuf, L.I, RP, L.I, 64, 64));
+    MOE_TMAP(tmap_2d(&p.tb0, c.dyperm, L.d, RP, L.d, 64, 64));
+    MOE_TMAP(tmap_2d(&p.to0, dW_down, L.d, El * L.I, L.d, 64, 32));
+    p.to1 = p.to0;
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.out0 = static_cast<__nv_bfloat16*>(dW_down);
+    MOE_TRY(timed(K_GEMM_WGRAD_DOWN, st, [&] { return launch_gemm(G_WGRAD_DOWN, p, grid, st); }));
+  }
   return MOE_OK;
 }
 

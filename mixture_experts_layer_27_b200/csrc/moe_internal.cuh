@@ -57,9 +57,13 @@ struct Layout {
   int64_t T_mb;   // tokens per minibatch (streamed layer)
   // ctx
   size_t hdr, ids, gates, counts, offsets, poff, perm_tok, perm_asg, slot_row, row_asg, row_gate, xperm, abuf,
-      bbuf, stab, ctx_bytes;
+      bbuf, stab, xq, xqs, ctx_bytes;
   // ws
-  size_t hist, logits, rpart, hbuf, obuf, dyperm, dabuf, dbbuf, hgbuf, dgpart, dlasg, wrt, dxperm, acc32, ws_bytes;
+  size_t hist, logits, rpart, hbuf, obuf, dyperm, dabuf, dbbuf, hgbuf, dgpart, dlasg, wrt, dxperm, acc32, hq, hqs, dyq,
+      dyqs, daq, daqs, dbq, dbqs, ws_bytes;
+  bool mx;  // MXFP8 mode
+  // prepared MXFP8 weights (moe_prepare_weights): fp8 codes and scale chunks
+  size_t wgu1, wgu1s, wd2, wd2s, wd3, wd3s, wg4, wg4s, wu4, wu4s, wq_bytes;
 };
 
 // Returns false for shapes outside the supported limits.  M > 0: a ring-streamed
@@ -120,6 +124,42 @@ constexpr int router_splits(int64_t T, int E, int d) {  // K splits of the route
 cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream_t st);
 
 // ---------------------------------------------------------------------------
+// MXFP8 grouped GEMMs (tcgen05 kind::mxf8f6f4 block_scale), see gemm_mx.cu
+// ---------------------------------------------------------------------------
+enum MxKind {
+  MX_GATEUP = 0,        // [A|B] = Xq . [Wg|Wu]q (64 gate + 64 up columns per tile); H quantised in the epilogue
+  MX_DOWN = 1,          // O' = g * (Hq . Wd_q)
+  MX_DGRAD_DOWN = 2,    // dH' = dYq . Wd_q^T; SwiGLU backward; dA, dB quantised in the epilogue
+  MX_DGRAD_GATEUP = 3,  // dX_perm = dAq . Wg_q^T + dBq . Wu_q^T
+};
+struct MxParams {
+  CUtensorMap ta0, ta1, tb0, tb1;  // fp8 K-major operands, box {128 bytes of K, 128 rows}
+  const uint8_t* sfa0;             // scale chunks of the A operands (K = the GEMM's contraction)
+  const uint8_t* sfa1;
+  const uint8_t* sfb0;             // scale chunks of the B operands
+  const uint8_t* sfb1;
+  const int* poff;                 // padded expert offsets [nseg+1]
+  int nseg;
+  const float* row_gate;
+  const __nv_bfloat16* in0;        // dgrad-down epilogue: saved A, B
+  const __nv_bfloat16* in1;
+  __nv_bfloat16* out0;
+  __nv_bfloat16* out1;
+  __nv_bfloat16* out2;
+  uint8_t* q0;                     // fp8 epilogue outputs and their scale chunks
+  uint8_t* q1;
+  uint8_t* qs0;
+  uint8_t* qs1;
+  float* outf;
+  int El, d, I;
+  int* status;
+};
+constexpr int MX_STAGES = 6;
+constexpr size_t MX_STAGE_BYTES = 16384 + 16384 + 1024;  // A tile, B tile, two scale chunks
+constexpr size_t MX_SMEM_BYTES = MX_STAGES * MX_STAGE_BYTES + 1024 + 256;
+cudaError_t launch_gemm_mx(MxKind kind, const MxParams& p, int grid, cudaStream_t st);
+
+// ---------------------------------------------------------------------------
 // routing / permutation kernels, see routing.cu
 // ---------------------------------------------------------------------------
 struct Ctx {  // typed views of ctx + ws for one shape
@@ -134,6 +174,7 @@ struct Ctx {  // typed views of ctx + ws for one shape
   float *dgpart, *dlasg;
   float* acc32;
   StreamTables tab;
+  uint8_t *xq, *xqs, *hq, *hqs, *dyq, *dyqs, *daq, *daqs, *dbq, *dbqs;  // MXFP8 operands and scales
 };
 Ctx make_ctx(const Layout& L, void* ctx, void* ws);
 
@@ -152,7 +193,12 @@ cudaError_t launch_replay(const Layout& L, const Ctx& c, int chunk, const __nv_b
                           int64_t ring_rows, cudaStream_t st);
 cudaError_t launch_finish_acc(const Layout& L, const Ctx& c, __nv_bfloat16* dW_gate, __nv_bfloat16* dW_up,
                               cudaStream_t st);
-cudaError_t launch_router_bwd(const Layout& L, const Ctx& c, cudaStream_t st);
+cudaError_t launch_router_bwd(const Layout& L, const Ctx& c, cudaStream_t st, int n_tiles_i = 0);
+// MXFP8 quantisation, see quant.cu
+cudaError_t launch_quant_weight(int mode, const __nv_bfloat16* src0, const __nv_bfloat16* src1, int64_t R_out, int K,
+                                int N, uint8_t* q, uint8_t* qs, cudaStream_t st);
+cudaError_t launch_gather_rows_mx(const Layout& L, const Ctx& c, const __nv_bfloat16* src, __nv_bfloat16* dst,
+                                  uint8_t* q, uint8_t* qs, cudaStream_t st);
 cudaError_t launch_transpose_wr(const Layout& L, const __nv_bfloat16* W_r, __nv_bfloat16* W_rT, cudaStream_t st);
 cudaError_t launch_rev_dispatch(const Layout& L, const Ctx& c, __nv_bfloat16* dX, cudaStream_t st);
 cudaError_t launch_dwr(const Layout& L, const Ctx& c, const __nv_bfloat16* X, float* dW_r, cudaStream_t st);

@@ -210,4 +210,71 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   return __bfloat1622float2(h);
 }
 
+
+// ---------------------------------------------------------------------------
+// MXFP8 (E4M3 payload, one E8M0 scale per 32 values along K)
+// ---------------------------------------------------------------------------
+// Scale factors of a K-major operand [R, K] are stored in 512-byte chunks, one per
+// (128 rows, 128 K): byte (r % 32) * 16 + ((r % 128) / 32) * 4 + (k % 128) / 32 of
+// chunk (r / 128) * (K / 128) + k / 128.  tcgen05.cp.32x128b.warpx4 moves one chunk
+// into 4 TMEM columns (replicated over the four lane quarters), and the MMA's sf_id
+// picks the 32-wide K block inside it.
+__device__ __forceinline__ size_t sf_index(int r, int k, int K) {
+  return (static_cast<size_t>(r >> 7) * (K >> 7) + (k >> 7)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 +
+         ((k & 127) >> 5);
+}
+
+// Quantise 32 values (one block) to E4M3 with a shared power-of-two scale:
+// exponent = floor(log2(amax)) - 8 (E4M3's largest exponent), scale byte = exponent + 127
+// clamped to [0, 254]; values are scaled exactly and rounded to nearest even with
+// saturation at +-448.  An all-zero block gives byte 0 and +0 codes.
+__device__ __forceinline__ uint8_t mx_quant32(const float (&v)[32], uint32_t (&q)[8]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  int byte = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 8;  // biased exponent - 8
+  byte = byte < 0 ? 0 : (byte > 254 ? 254 : byte);
+  const float inv = __uint_as_float(static_cast<uint32_t>(254 - byte) << 23);  // 2^(127 - byte)
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint16_t lo, hi;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(lo) : "f"(v[4 * j] * inv), "f"(v[4 * j + 1] * inv));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(hi) : "f"(v[4 * j + 2] * inv), "f"(v[4 * j + 3] * inv));
+    q[j] = amax == 0.f ? 0u : (static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16));
+  }
+  return static_cast<uint8_t>(byte);
+}
+
+// tcgen05 pieces of the block-scaled MMA
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint32_t saddr) {
+  // smem descriptor of a 32-row x 16-byte block, no swizzle (8-row core matrices 128 B apart)
+  uint64_t d = static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128 >> 4) << 16;
+  d |= static_cast<uint64_t>(128 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
+}
+__device__ __forceinline__ void umma_mxf8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+// Instruction descriptor, kind::mxf8f6f4 with E4M3 A/B, E8M0 scales, K = 32, both K-major;
+// sf_id selects the scale byte (K block) inside the 32-bit TMEM scale words.
+__host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, uint32_t sf_id) {
+  return (sf_id << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24) |
+         (sf_id << 29);
+}
+// 1-D bulk copy global -> shared, completion on an mbarrier (16-byte aligned, size multiple of 16)
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 }  // namespace moe

@@ -1,0 +1,148 @@
+// MXFP8 quantisation: prepared weights (once per optimiser step) and the
+// dispatched activations (fused into the gather that builds X_perm / dY_perm).
+// Every 32-value block along a GEMM's contraction dimension gets one E8M0 scale
+// (floor(log2 amax) - 8, the OCP MX rule) and E4M3 codes rounded to nearest
+// even with saturation; scales are laid out in the 512-byte chunks the
+// block-scaled MMA copies into tensor memory (see sf_index in ptx.cuh).
+#include "moe_internal.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+// One block = 128 output rows x 128 K of a K-major fp8 weight [R_out, K].
+//   mode 0: source [R_out, K] row-major (K contiguous)
+//   mode 1: source [El][K][N] (N contiguous), output row el*N + n
+//   mode 2: paired gate/up, source gate/up [El][K][N]; output rows per expert come in
+//           blocks of 128 = 64 gate rows then 64 up rows (columns j*64 .. j*64+63)
+__global__ void __launch_bounds__(128) k_quant_weight(const __nv_bfloat16* __restrict__ src0,
+                                                      const __nv_bfloat16* __restrict__ src1, int mode, int K, int N,
+                                                      uint8_t* __restrict__ q, uint8_t* __restrict__ qs) {
+  extern __shared__ float tile[];  // [128][129]
+  const int k0 = blockIdx.x * 128;
+  const int o0 = blockIdx.y * 128;
+  if (mode == 0) {
+    for (int c = threadIdx.x; c < 128 * 16; c += 128) {  // 16-byte chunks along K
+      const int r = c >> 4, kc = (c & 15) * 8;
+      const uint4 u = *reinterpret_cast<const uint4*>(src0 + static_cast<size_t>(o0 + r) * K + k0 + kc);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = unpack_bf16(w[j]);
+        tile[r * 129 + kc + 2 * j] = f.x;
+        tile[r * 129 + kc + 2 * j + 1] = f.y;
+      }
+    }
+  } else {
+    for (int c = threadIdx.x; c < 128 * 16; c += 128) {  // 16-byte chunks along N of source row k
+      const int kk = c >> 4, nc = (c & 15) * 8;
+      const int r = nc;  // tile row of the first of the 8 columns
+      const int o = o0 + r;
+      const __nv_bfloat16* src;
+      size_t off;
+      if (mode == 1) {
+        const int el = o / N, n = o - el * N;
+        src = src0;
+        off = (static_cast<size_t>(el) * K + k0 + kk) * N + n;
+      } else {
+        const int el = o / (2 * N), w = o - el * 2 * N;
+        const int j = w >> 7, h = (w >> 6) & 1, n = j * 64 + (w & 63);
+        src = h ? src1 : src0;
+        off = (static_cast<size_t>(el) * K + k0 + kk) * N + n;
+      }
+      const uint4 u = *reinterpret_cast<const uint4*>(src + off);
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = unpack_bf16(w4[j]);
+        tile[(r + 2 * j) * 129 + kk] = f.x;
+        tile[(r + 2 * j + 1) * 129 + kk] = f.y;
+      }
+    }
+  }
+  __syncthreads();
+  const int r = threadIdx.x;
+  const int o = o0 + r;
+#pragma unroll 1
+  for (int b = 0; b < 4; ++b) {
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = tile[r * 129 + b * 32 + i];
+    uint32_t w[8];
+    const uint8_t sb = mx_quant32(v, w);
+    uint4* d = reinterpret_cast<uint4*>(q + static_cast<size_t>(o) * K + k0 + b * 32);
+    d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    qs[sf_index(o, k0 + b * 32, K)] = sb;
+  }
+}
+
+// Dispatch / reverse-combine in MXFP8 mode: rows [lo, hi) of the padded layout get the
+// bf16 row (kept for the weight gradients) and its fp8 codes + scales along d.
+__global__ void __launch_bounds__(128) k_gather_rows_mx(const __nv_bfloat16* __restrict__ src,
+                                                        const int* __restrict__ row_asg, const int* __restrict__ lo,
+                                                        const int* __restrict__ hi, int k, int d,
+                                                        __nv_bfloat16* __restrict__ dst, uint8_t* __restrict__ q,
+                                                        uint8_t* __restrict__ qs) {
+  const int r0 = __ldg(lo), r1 = __ldg(hi);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nb = d / 32;
+  for (int64_t R = r0 + blockIdx.x * 4 + warp; R < r1; R += gridDim.x * 4) {
+    const int a = row_asg[R];
+    for (int b = lane; b < nb; b += 32) {
+      float v[32];
+      uint4 u[4];
+      if (a >= 0) {
+        const uint4* in = reinterpret_cast<const uint4*>(src + static_cast<size_t>(a / k) * d + b * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) u[j] = __ldg(in + j);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) u[j] = make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t w4[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = unpack_bf16(w4[i]);
+          v[8 * j + 2 * i] = f.x;
+          v[8 * j + 2 * i + 1] = f.y;
+        }
+      }
+      uint4* o = reinterpret_cast<uint4*>(dst + R * d + b * 32);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) o[j] = u[j];
+      uint32_t w[8];
+      const uint8_t sb = mx_quant32(v, w);
+      uint4* qd = reinterpret_cast<uint4*>(q + R * d + b * 32);
+      qd[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      qd[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      qs[sf_index(static_cast<int>(R), b * 32, d)] = sb;
+    }
+  }
+}
+
+cudaError_t launch_quant_weight(int mode, const __nv_bfloat16* src0, const __nv_bfloat16* src1, int64_t R_out, int K,
+                                int N, uint8_t* q, uint8_t* qs, cudaStream_t st) {
+  const int smem = 128 * 129 * 4;
+  static bool configured[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(k_quant_weight, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  k_quant_weight<<<dim3(K / 128, static_cast<unsigned>(R_out / 128)), 128, smem, st>>>(src0, src1, mode, K, N, q, qs);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows_mx(const Layout& L, const Ctx& c, const __nv_bfloat16* src, __nv_bfloat16* dst,
+                                  uint8_t* q, uint8_t* qs, cudaStream_t st) {
+  const int64_t g = (L.RP + 3) / 4;
+  const int grid = static_cast<int>(g < 148 * 8 ? g : 148 * 8);
+  k_gather_rows_mx<<<grid, 128, 0, st>>>(src, c.row_asg, c.poff, c.poff + L.El, L.k, L.d, dst, q, qs);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

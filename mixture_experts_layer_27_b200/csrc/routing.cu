@@ -643,10 +643,11 @@ cudaError_t launch_finish_acc(const Layout& L, const Ctx& c, __nv_bfloat16* dW_g
   k_finish_acc<<<148 * 8, 256, 0, st>>>(c.acc32, c.tab.plan, n_each, dW_gate, dW_up);
   return cudaGetLastError();
 }
-cudaError_t launch_router_bwd(const Layout& L, const Ctx& c, cudaStream_t st) {
+cudaError_t launch_router_bwd(const Layout& L, const Ctx& c, cudaStream_t st, int n_tiles_i) {
+  // n_tiles_i: dg partials per row = n-tiles of the dgrad-down GEMM (I / 256 bf16, I / 128 MXFP8)
   k_router_bwd<<<static_cast<unsigned>((L.T + 7) / 8), 256, 0, st>>>(c.dgpart, c.slot_row, c.gates,
-                                                                       static_cast<int>(L.T), L.k, L.I / 256,
-                                                                       c.dlasg);
+                                                                       static_cast<int>(L.T), L.k,
+                                                                       n_tiles_i ? n_tiles_i : L.I / 256, c.dlasg);
   return cudaGetLastError();
 }
 cudaError_t launch_transpose_wr(const Layout& L, const __nv_bfloat16* W_r, __nv_bfloat16* W_rT, cudaStream_t st) {

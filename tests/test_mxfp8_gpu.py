@@ -1,0 +1,98 @@
+"""MXFP8 mode on the GPU.
+
+* prepared weights: E4M3 codes and E8M0 scale bytes bit-exact against the
+  oracle's MX quantiser (OCP MX rule), for every prepared layout;
+* layer: forward + backward within 6e-2 (max |gpu - ref| / max |ref|) of the
+  unquantised fp64 oracle; routing table bit-exact (the router stays bf16);
+* two runs are bit-identical.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from mixture_experts_layer_27_b200 import binding as B
+
+from _util import make_case, relerr, run_oracle, to64
+
+pytestmark = pytest.mark.gpu
+TOL_MX = 6e-2
+
+
+def _pairs(Wg, Wu):
+    """[El*2I, d]: per expert, blocks of 64 W_gate columns then the same 64 W_up columns (as rows)."""
+    El, d, I = Wg.shape
+    rows = []
+    for e in range(El):
+        for j in range(I // 64):
+            rows.append(Wg[e][:, j * 64:(j + 1) * 64].T)
+            rows.append(Wu[e][:, j * 64:(j + 1) * 64].T)
+    return np.concatenate(rows, axis=0)
+
+
+def test_prepared_weights_match_the_oracle_quantiser_bit_for_bit():
+    T, d, E, k, I = 64, 256, 4, 2, 512
+    w, x = make_case(T, d, E, k, I, seed=41)
+    lay = B.MoELayerMX(T, d, E, I, k)
+    lay.prepare(x["W_gate"], x["W_up"], x["W_down"])
+    torch.cuda.synchronize()
+    reg = lay.weight_regions()
+    Wg, Wu, Wd = to64(x["W_gate"]), to64(x["W_up"]), to64(x["W_down"])
+    src = {"Wgu": _pairs(Wg, Wu), "Wd2": Wd.transpose(0, 2, 1).reshape(E * d, I),
+           "Wd3": Wd.reshape(E * I, d), "Wg4": Wg.reshape(E * d, I), "Wu4": Wu.reshape(E * d, I)}
+    for name, ref in src.items():
+        codes, chunks, R, K = reg[name]
+        qc, qs = O.mx_quantize(ref, axis=1)
+        assert np.array_equal(codes, qc), name
+        assert np.array_equal(B.unchunk_scales(chunks, R, K), qs), name
+
+
+def _check_layer_mx(T, d, E, k, I, bias=None, seed=0):
+    w, x = make_case(T, d, E, k, I, seed=seed, bias=bias)
+    lay = B.MoELayerMX(T, d, E, I, k)
+    lay.prepare(x["W_gate"], x["W_up"], x["W_down"])
+    Y = lay.forward(x["X"], x["W_r"], x["bias"])
+    g = lay.backward(x["X"], x["W_r"], x["dY"])
+    torch.cuda.synchronize()
+    assert lay.error() == B.MOE_OK
+    r = lay.routing()
+    lg = to64(lay.logits())
+    ids = O.topk_ids(lg, k)
+    assert np.array_equal(r["ids"].cpu().numpy(), ids)
+    Yo, ctx, go = run_oracle(x, k)
+    errs = {
+        "Y": relerr(to64(Y), Yo),
+        "dX": relerr(to64(g["dX"]), go["dX"]),
+        "dW_r": relerr(to64(g["dW_r"]), go["dW_r"]),
+        "dW_gate": relerr(to64(g["dW_gate"]), np.stack([go["dW_gate"][e] for e in range(E)])),
+        "dW_up": relerr(to64(g["dW_up"]), np.stack([go["dW_up"][e] for e in range(E)])),
+        "dW_down": relerr(to64(g["dW_down"]), np.stack([go["dW_down"][e] for e in range(E)])),
+    }
+    assert all(v <= TOL_MX for v in errs.values()), errs
+    return lay, x, Y, g
+
+
+def test_mxfp8_tiny_config():
+    _check_layer_mx(128, 256, 8, 2, 512, seed=0)
+
+
+def test_mxfp8_hot_expert_multi_tile_and_empty_expert():
+    bias = np.zeros(4, dtype=np.float32)
+    bias[0] = 8.0
+    bias[3] = -40.0
+    _check_layer_mx(600, 512, 4, 2, 512, bias=bias, seed=42)
+
+
+def test_mxfp8_many_experts_ragged_tokens():
+    _check_layer_mx(333, 768, 48, 6, 768, seed=43)
+
+
+def test_mxfp8_bit_identical_runs():
+    lay, x, Y, g = _check_layer_mx(256, 512, 8, 2, 512, seed=44)
+    Y2 = lay.forward(x["X"], x["W_r"], x["bias"])
+    g2 = lay.backward(x["X"], x["W_r"], x["dY"])
+    torch.cuda.synchronize()
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+    for n in ("dX", "dW_gate", "dW_up", "dW_down"):
+        assert torch.equal(g[n].view(torch.int16), g2[n].view(torch.int16)), n
+    assert torch.equal(g["dW_r"].view(torch.int32), g2["dW_r"].view(torch.int32))
