@@ -460,3 +460,82 @@ def stream_plan(mb_counts, ring_rows: int, min_rows: int, P: int = P_PAD) -> dic
         chunks = [(0, 0)]
     return dict(macro=[(a, b) for a, b, _ in macro], seg_poff=seg_poff, rows=row, ring_start=ring_start,
                 sizes=sizes, resident=resident, chunks=chunks, replayed=replayed)
+
+
+# ----------------------------------------------------------------------------
+# MXFP8 layer: every operand of the gate/up, down and dgrad GEMMs rounded to MX
+# (E4M3 + E8M0 per 32 along that GEMM's contraction dimension) before the
+# product; the weight-gradient GEMMs contract over tokens and are not quantised.
+# fp64 everywhere else.  The router gradient takes dg = <dH', H> with dH' the
+# quantised dgrad of W_down (the fused form; the identity with <dY, O> holds only
+# without quantisation).
+# ----------------------------------------------------------------------------
+def mx_round(v, axis: int):
+    """v rounded to its MXFP8 value along `axis` (fp64)."""
+    c, s = mx_quantize(v, axis=axis)
+    return mx_dequantize(c, s, axis=axis)
+
+
+def forward_mx(X, W_r, bias, W_gate, W_up, W_down, top_k: int):
+    X64 = _f64(X)
+    T, d = X64.shape
+    E = np.asarray(W_r).shape[1]
+    logits = router_logits(X64, W_r, bias)
+    ids = topk_ids(logits, top_k)
+    g = gates(logits, ids)
+    sched = schedule(ids, E)
+    Y = np.zeros((T, d))
+    saved = []
+    for e in range(E):
+        toks, slots = _expert_rows(ids, sched, e)
+        if toks.size == 0:
+            saved.append(None)
+            continue
+        Xq = mx_round(X64[toks], axis=1)  # K = d
+        A = Xq @ mx_round(_expert(W_gate, e), axis=0)
+        B = Xq @ mx_round(_expert(W_up, e), axis=0)
+        H = silu(A) * B
+        O = mx_round(H, axis=1) @ mx_round(_expert(W_down, e), axis=0)  # K = I
+        ge = g[toks, slots]
+        Y[toks] += ge[:, None] * O
+        saved.append((toks, slots, A, B))
+    ctx = dict(X=X64, W_r=_f64(W_r), W_gate=W_gate, W_up=W_up, W_down=W_down, logits=logits, ids=ids, g=g,
+               sched=sched, saved=saved, E=E)
+    return Y, ctx
+
+
+def backward_mx(ctx, dY):
+    dY64 = _f64(dY)
+    X64, ids, g, sched = ctx["X"], ctx["ids"], ctx["g"], ctx["sched"]
+    T, d = X64.shape
+    k = ids.shape[1]
+    E = ctx["E"]
+    dX = np.zeros((T, d))
+    dg = np.zeros((T, k))
+    dW_gate, dW_up, dW_down = {}, {}, {}
+    for e in range(E):
+        Wg, Wu, Wd = _expert(ctx["W_gate"], e), _expert(ctx["W_up"], e), _expert(ctx["W_down"], e)
+        item = ctx["saved"][e]
+        if item is None:
+            I = Wg.shape[1]
+            dW_gate[e] = np.zeros((d, I)); dW_up[e] = np.zeros((d, I)); dW_down[e] = np.zeros((I, d))
+            continue
+        toks, slots, A, B = item
+        Xe = X64[toks]
+        ge = g[toks, slots]
+        dYe = dY64[toks]
+        H = silu(A) * B
+        dHp = mx_round(dYe, axis=1) @ mx_round(Wd, axis=1).T  # K = d
+        dg[toks, slots] = np.sum(dHp * H, axis=1)
+        dH = ge[:, None] * dHp
+        dA = dH * B * silu_grad(A)
+        dB = dH * silu(A)
+        dX[toks] += mx_round(dA, axis=1) @ mx_round(Wg, axis=1).T + mx_round(dB, axis=1) @ mx_round(Wu, axis=1).T
+        dW_gate[e] = Xe.T @ dA
+        dW_up[e] = Xe.T @ dB
+        dW_down[e] = H.T @ (ge[:, None] * dYe)
+    dl = np.zeros((T, E))
+    s = np.sum(g * dg, axis=1, keepdims=True)
+    np.put_along_axis(dl, ids.astype(np.int64), g * (dg - s), axis=1)
+    dX += dl @ ctx["W_r"].T
+    return dict(dX=dX, dW_gate=dW_gate, dW_up=dW_up, dW_down=dW_down, dW_r=X64.T @ dl, dl=dl, dg=dg)

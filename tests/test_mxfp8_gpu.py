@@ -3,7 +3,10 @@
 * prepared weights: E4M3 codes and E8M0 scale bytes bit-exact against the
   oracle's MX quantiser (OCP MX rule), for every prepared layout;
 * layer: forward + backward within 6e-2 (max |gpu - ref| / max |ref|) of the
-  unquantised fp64 oracle; routing table bit-exact (the router stays bf16);
+  MXFP8 oracle (fp64 with every quantised GEMM operand rounded to MX along its
+  contraction dimension); against the unquantised fp64 oracle, within the
+  format's own error (MXFP8 oracle vs unquantised oracle, 5-9% at these shapes)
+  plus 2e-2; routing table bit-exact (the router stays bf16);
 * two runs are bit-identical.
 """
 import numpy as np
@@ -59,16 +62,28 @@ def _check_layer_mx(T, d, E, k, I, bias=None, seed=0):
     lg = to64(lay.logits())
     ids = O.topk_ids(lg, k)
     assert np.array_equal(r["ids"].cpu().numpy(), ids)
+    f64 = {n: (None if x[n] is None else to64(x[n])) for n in ("X", "W_r", "bias", "W_gate", "W_up", "W_down", "dY")}
+    Yq, cq = O.forward_mx(f64["X"], f64["W_r"], f64["bias"], f64["W_gate"], f64["W_up"], f64["W_down"], k)
+    gq = O.backward_mx(cq, f64["dY"])
     Yo, ctx, go = run_oracle(x, k)
-    errs = {
-        "Y": relerr(to64(Y), Yo),
-        "dX": relerr(to64(g["dX"]), go["dX"]),
-        "dW_r": relerr(to64(g["dW_r"]), go["dW_r"]),
-        "dW_gate": relerr(to64(g["dW_gate"]), np.stack([go["dW_gate"][e] for e in range(E)])),
-        "dW_up": relerr(to64(g["dW_up"]), np.stack([go["dW_up"][e] for e in range(E)])),
-        "dW_down": relerr(to64(g["dW_down"]), np.stack([go["dW_down"][e] for e in range(E)])),
-    }
-    assert all(v <= TOL_MX for v in errs.values()), errs
+
+    def errs_vs(Yr, gr):
+        return {
+            "Y": relerr(to64(Y), Yr),
+            "dX": relerr(to64(g["dX"]), gr["dX"]),
+            "dW_r": relerr(to64(g["dW_r"]), gr["dW_r"]),
+            "dW_gate": relerr(to64(g["dW_gate"]), np.stack([gr["dW_gate"][e] for e in range(E)])),
+            "dW_up": relerr(to64(g["dW_up"]), np.stack([gr["dW_up"][e] for e in range(E)])),
+            "dW_down": relerr(to64(g["dW_down"]), np.stack([gr["dW_down"][e] for e in range(E)])),
+        }
+
+    errs_q = errs_vs(Yq, gq)
+    assert all(v <= TOL_MX for v in errs_q.values()), errs_q
+    errs_u = errs_vs(Yo, go)
+    fmt = {"Y": relerr(Yq, Yo), "dX": relerr(gq["dX"], go["dX"]), "dW_r": relerr(gq["dW_r"], go["dW_r"])}
+    for n in ("dW_gate", "dW_up", "dW_down"):
+        fmt[n] = relerr(np.stack([gq[n][e] for e in range(E)]), np.stack([go[n][e] for e in range(E)]))
+    assert all(errs_u[n] <= fmt[n] + 2e-2 for n in fmt), (errs_u, fmt)
     return lay, x, Y, g
 
 

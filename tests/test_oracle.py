@@ -351,3 +351,38 @@ def test_mx_quantize_axis0_equals_transposed_axis1():
     c0, s0 = O.mx_quantize(v, axis=0)
     c1, s1 = O.mx_quantize(v.T, axis=1)
     assert np.array_equal(c0, c1.T) and np.array_equal(s0, s1.T)
+
+
+# --------------------------------------------------------------------------
+# MXFP8 layer of the oracle: with MX rounding replaced by the identity it must
+# be the bf16 layer exactly (operands, axes and the fused router gradient wired
+# as the unquantised definition); the rounding itself is pinned above.
+# --------------------------------------------------------------------------
+def test_mx_layer_reduces_to_the_plain_layer_without_rounding(monkeypatch):
+    import oracle.moe_oracle as M
+    rng = np.random.default_rng(14)
+    T, d, E, I, k = 40, 64, 6, 96, 2
+    X, W_r, Wg, Wu, Wd, dY = _rand_layer(rng, T, d, E, I, k)
+    Y, ctx = O.forward(X, W_r, None, Wg, Wu, Wd, k)
+    g = O.backward(ctx, dY)
+    monkeypatch.setattr(M, "mx_round", lambda v, axis: np.asarray(v, dtype=np.float64))
+    Yq, cq = M.forward_mx(X, W_r, None, Wg, Wu, Wd, k)
+    gq = M.backward_mx(cq, dY)
+    np.testing.assert_allclose(Yq, Y, rtol=1e-13, atol=1e-13)
+    for n in ("dX", "dW_r", "dl", "dg"):
+        np.testing.assert_allclose(gq[n], g[n], rtol=1e-11, atol=1e-12)
+    for n in ("dW_gate", "dW_up", "dW_down"):
+        for e in range(E):
+            np.testing.assert_allclose(gq[n][e], g[n][e], rtol=1e-11, atol=1e-12)
+
+
+def test_mx_round_error_bound_and_idempotence():
+    rng = np.random.default_rng(15)
+    v = rng.standard_normal((16, 256))
+    r = O.mx_round(v, axis=1)
+    assert np.array_equal(O.mx_round(r, axis=1), r)  # MX values are fixed points
+    # per 32-block: |error| <= half an E4M3 ulp of the block's top binade after saturation at 448
+    vb, rb = v.reshape(16, 8, 32), r.reshape(16, 8, 32)
+    amax = np.abs(vb).max(-1, keepdims=True)
+    step = 2.0 ** (np.floor(np.log2(amax)) - 8)  # scale; codes are <= 448 = 1.75 * 2^8
+    assert np.all(np.abs(vb - rb) <= np.maximum(amax - 448 * step, 0) + 16 * step + 1e-300)
