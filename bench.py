@@ -99,6 +99,25 @@ def algorithmic_bytes(w: IN.Workload) -> dict:
     T, d, E, I, k, El = w.tokens, w.d, w.E, w.I, w.k, w.El
     rows = local_rows(w)
     W1 = El * d * I * 2  # one expert weight matrix family (gate, up or down), bytes
+    if w.mxfp8:
+        # fp8 operands carry one scale byte per 32 values; outputs stay bf16 (H, dA, dB also as fp8)
+        Wq = El * d * I * 33 // 32
+        return {
+            "router_logits": T * d * 2 + d * E * 2 + T * E * 4,
+            "topk_gating": T * E * 4 + rows * 8,
+            "dispatch": T * d * 2 + rows * d * 2 + rows * d * 33 // 32,
+            "gemm_gateup_swiglu": 2 * Wq + rows * d * 33 // 32 + 2 * rows * I * 2 + rows * I * 33 // 32,
+            "gemm_down_combw": Wq + rows * I * 33 // 32 + rows * d * 2,
+            "combine": rows * d * 2 + T * d * 2,
+            "reverse_combine": T * d * 2 + rows * d * 2 + rows * d * 33 // 32,
+            "gemm_dgrad_down_swiglu_bwd": Wq + rows * d * 33 // 32 + 2 * rows * I * 2 + 3 * rows * I * 2
+            + 2 * rows * I * 33 // 32,
+            "router_wgrad": T * d * 2 + T * k * 8 + d * E * 4,
+            "gemm_dgrad_gateup": 2 * Wq + 2 * rows * I * 33 // 32 + rows * d * 2,
+            "reverse_dispatch": rows * d * 2 + T * d * 2 + E * d * 2,
+            "gemm_wgrad_gateup": rows * d * 2 + 2 * rows * I * 2 + 2 * W1,
+            "gemm_wgrad_down": rows * I * 2 + rows * d * 2 + W1,
+        }
     return {
         "router_logits": T * d * 2 + d * E * 2 + T * E * 4,
         "topk_gating": T * E * 4 + rows * 8,
