@@ -95,7 +95,7 @@ def algorithmic_flops(w: IN.Workload) -> dict:
 # algorithmic bytes per launch of each kernel (minimum HBM traffic of its job)
 # rows = T*k routed assignments; weights of all local experts; bf16 = 2 bytes
 # ----------------------------------------------------------------------------
-def algorithmic_bytes(w: IN.Workload) -> dict:
+def _algorithmic_bytes(w: IN.Workload) -> dict:
     T, d, E, I, k, El = w.tokens, w.d, w.E, w.I, w.k, w.El
     rows = local_rows(w)
     W1 = El * d * I * 2  # one expert weight matrix family (gate, up or down), bytes
@@ -133,6 +133,10 @@ def algorithmic_bytes(w: IN.Workload) -> dict:
         "gemm_wgrad_gateup": rows * d * 2 + 2 * rows * I * 2 + 2 * W1,
         "gemm_wgrad_down": rows * I * 2 + rows * d * 2 + W1,
     }
+
+
+def algorithmic_bytes(w: IN.Workload) -> dict:
+    return _algorithmic_bytes(w)
 
 
 # DRAM bytes per launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum),

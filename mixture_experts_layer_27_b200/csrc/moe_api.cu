@@ -3,6 +3,7 @@
 // Every step of the layer runs in this library's kernels; the host only
 // enqueues work and never waits on the device (except in moe_get_error).
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <atomic>
 #include <mutex>
@@ -524,7 +525,7 @@ moe_status moe_bwd(const moe_shape* s, const void* X, const void* W_r, const voi
   }
   // 12. reverse-dispatch (+ router term dl W_r^T)
   MOE_TRY(timed(K_REV_DISPATCH, st, [&] { return launch_rev_dispatch(L, c, static_cast<__nv_bfloat16*>(dX), st); }));
-  // 13. wgrad: gate/up then down
+  // 13. wgrad: gate/up then down (write-bound; separate launches keep HBM traffic one-directional)
   {
     GemmParams p = base_params(L, c, status);
     MOE_TMAP(tmap_2d(&p.ta0, c.xperm, L.d, RP, L.d, 64, 64));
