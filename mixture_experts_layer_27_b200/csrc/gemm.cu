@@ -433,150 +433,30 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   }
 }
 
-// Barriers, tensor memory and staging of one CTA.
-struct CtaRes {
-  uint8_t* smem;       // operand stages (1024-aligned)
-  uint8_t* stage_out;  // wgrad staging (4 x 16 KB)
-  uint64_t* full;
-  uint64_t* empty;
-  uint64_t* tfull;
-  uint64_t* tempty;
-  uint64_t* drain;
-  uint32_t tbase;
-};
-// Pipeline position of one role; carried across GEMM kinds run back to back by a CTA.
-struct RoleState {
-  int stage = 0;
-  uint32_t phase = 0;
-  int it = 0;  // tiles processed (accumulator index / parity)
-  bool ok = true;
-  int last_parity[GEMM_STAGES];
-  bool wrote_tma = false;  // epilogue: TMA stores outstanding
-};
-
-template <int KIND, int STAGES>
-__device__ __forceinline__ void producer_loop(const GemmParams& p, const CtaRes& r, RoleState& s, int t0, int dt,
-                                              int t_end = 0x7fffffff) {
-  const uint64_t pol_act = policy_evict_last();
-  const uint64_t pol_w = policy_evict_first();
-  const int ntiles = min(num_tiles<KIND>(p), t_end);
-  for (int t = t0; t < ntiles && s.ok; t += dt) {
-    const Tile tl = decode<KIND>(p, t);
-    if constexpr (is_wgrad<KIND>()) {
-      // K runs over the expert's padded rows in each macrobatch of the chunk, in order
-      for (int m = tl.m; m < tl.shift && s.ok; ++m) {
-        const int sg = m * p.El + tl.el;
-        const int r0 = __ldg(p.poff + sg), r1 = __ldg(p.poff + sg + 1);
-        const int xs = (KIND == G_WGRAD_GATEUP && p.ring_shift) ? __ldg(p.ring_shift + m) : 0;
-        for (int row = r0; row < r1; row += 64) {
-          if (!mbar_wait(&r.empty[s.stage], s.phase ^ 1, p.status)) { s.ok = false; break; }
-          uint8_t* sA = r.smem + s.stage * GEMM_STAGE_BYTES;
-          mbar_arrive_expect_tx(&r.full[s.stage], static_cast<uint32_t>(GEMM_STAGE_BYTES));
-          load_wgrad<KIND>(p, tl, row, xs, sA, sA + GEMM_A_BYTES, &r.full[s.stage], pol_act);
-          s.last_parity[s.stage] = static_cast<int>(s.phase);
-          if (++s.stage == STAGES) { s.stage = 0; s.phase ^= 1; }
-        }
-      }
-    } else {
-      for (int kb = 0; kb < tl.nk; ++kb) {
-        if (!mbar_wait(&r.empty[s.stage], s.phase ^ 1, p.status)) { s.ok = false; break; }
-        uint8_t* sA = r.smem + s.stage * GEMM_STAGE_BYTES;
-        mbar_arrive_expect_tx(&r.full[s.stage], static_cast<uint32_t>(GEMM_STAGE_BYTES));
-        load_stage<KIND>(p, tl, kb, sA, sA + GEMM_A_BYTES, &r.full[s.stage], pol_act, pol_w);
-        s.last_parity[s.stage] = static_cast<int>(s.phase);
-        if (++s.stage == STAGES) { s.stage = 0; s.phase ^= 1; }
-      }
-    }
-  }
-}
-
-template <int KIND, int STAGES>
-__device__ __forceinline__ void mma_loop(const GemmParams& p, const CtaRes& r, RoleState& s, int t0, int dt,
-                                         int t_end = 0x7fffffff) {
-  constexpr uint32_t IDESC = idesc_bf16(GEMM_BM, GEMM_BN, Traits<KIND>::A_MN, Traits<KIND>::B_MN);
-  const int ntiles = min(num_tiles<KIND>(p), t_end);
-  for (int t = t0; t < ntiles && s.ok; t += dt, ++s.it) {
-    const Tile tl = decode<KIND>(p, t);
-    const int acc = s.it & 1;
-    const uint32_t accp = (s.it >> 1) & 1;
-    if (!mbar_wait(&r.tempty[acc], accp ^ 1, p.status)) { s.ok = false; break; }
-    tc_fence_after();
-    const uint32_t dtm = r.tbase + acc * GEMM_BN;
-    for (int kb = 0; kb < tl.nk; ++kb) {
-      if (!mbar_wait(&r.full[s.stage], s.phase, p.status)) { s.ok = false; break; }
-      tc_fence_after();
-      const uint32_t a0 = smem_u32(r.smem + s.stage * GEMM_STAGE_BYTES);
-      const uint32_t b0 = a0 + static_cast<uint32_t>(GEMM_A_BYTES);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {  // 4 x K16 per 64-wide block
-        const uint64_t ad = Traits<KIND>::A_MN ? sdesc_sw128(a0 + kk * 2048, 8192, 1024)
-                                               : sdesc_sw128(a0 + kk * 32, 16, 1024);
-        const uint64_t bd = Traits<KIND>::B_MN ? sdesc_sw128(b0 + kk * 2048, 8192, 1024)
-                                               : sdesc_sw128(b0 + kk * 32, 16, 1024);
-        umma_bf16(dtm, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
-      }
-      umma_commit(&r.empty[s.stage]);  // frees the stage once these MMAs have read it
-      if (++s.stage == STAGES) { s.stage = 0; s.phase ^= 1; }
-    }
-    if (!s.ok) break;
-    if (tl.nk > 0) umma_commit(&r.tfull[acc]);
-    else mbar_arrive(&r.tfull[acc]);
-  }
-}
-
 template <int KIND>
-__device__ __forceinline__ void epilogue_loop(const GemmParams& p, const CtaRes& r, RoleState& s, int t0, int dt,
-                                              int warp, int lane, int t_end = 0x7fffffff) {
-  const int quarter = warp & 3;  // TMEM lanes this warp may access: 32*quarter ..
-  const int row = quarter * 32 + lane;
-  const int ntiles = min(num_tiles<KIND>(p), t_end);
-  for (int t = t0; t < ntiles; t += dt, ++s.it) {
-    const Tile tl = decode<KIND>(p, t);
-    const int acc = s.it & 1;
-    const uint32_t accp = (s.it >> 1) & 1;
-    int ok = 1;
-    if (lane == 0) ok = mbar_wait(&r.tfull[acc], accp, p.status) ? 1 : 0;
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (!ok) { s.ok = false; break; }
-    __syncwarp();
-    tc_fence_after();
-    const uint32_t taddr = r.tbase + (static_cast<uint32_t>(quarter * 32) << 16) + acc * GEMM_BN;
-    if constexpr (is_wgrad<KIND>()) {
-      epilogue_wgrad<KIND>(p, tl, quarter, lane, taddr, r.stage_out + (warp - 2) * (GEMM_STAGE_OUT_BYTES / 4));
-      s.wrote_tma = true;
-    } else {
-      epilogue_row<KIND>(p, tl, row, taddr);
-    }
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&r.tempty[acc]);
-  }
-}
+__global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int STAGES = stages_of<KIND>();
+  uint8_t* stage_out = smem + STAGES * GEMM_STAGE_BYTES;  // wgrad only: 4 x 16 KB
+  uint64_t* full = reinterpret_cast<uint64_t*>(stage_out + (is_wgrad<KIND>() ? GEMM_STAGE_OUT_BYTES : 0));
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
-// Set-up shared by the GEMM kernels: barriers for `stages` stages placed after
-// `data_bytes` of stage / staging memory, and 512 TMEM columns.
-__device__ __forceinline__ CtaRes cta_setup(uint8_t* smem_raw, int stages, size_t stage_region, size_t out_region,
-                                            const GemmParams& p) {
-  CtaRes r;
-  r.smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  r.stage_out = r.smem + stage_region;
-  r.full = reinterpret_cast<uint64_t*>(r.smem + stage_region + out_region);
-  r.empty = r.full + GEMM_STAGES;
-  r.tfull = r.empty + GEMM_STAGES;
-  r.tempty = r.tfull + 2;
-  r.drain = r.tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(r.drain + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < stages; ++s) {
-      mbar_init(&r.full[s], 1);
-      mbar_init(&r.empty[s], 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&r.tfull[a], 1);
-      mbar_init(&r.tempty[a], 4);  // one arrival per epilogue warp
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
     }
-    mbar_init(r.drain, 1);
+    mbar_init(drain, 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -592,50 +472,126 @@ __device__ __forceinline__ CtaRes cta_setup(uint8_t* smem_raw, int stages, size_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  r.tbase = *tmem_slot;
-  return r;
-}
+  const uint32_t tbase = *tmem_slot;
+  const int ntiles = num_tiles<KIND>(p);
+  constexpr uint32_t IDESC = idesc_bf16(GEMM_BM, GEMM_BN, Traits<KIND>::A_MN, Traits<KIND>::B_MN);
 
-// Tear-down after the role loops: drain in-flight copies / MMAs / stores, free TMEM.
-template <int STAGES>
-__device__ __forceinline__ void cta_finish(const CtaRes& r, RoleState& s, int warp, int lane) {
-  if (warp == 0 && lane == 0 && !s.ok) {  // let copies already in flight land before the smem goes away
-    for (int q = 0; q < STAGES; ++q)
-      if (s.last_parity[q] >= 0) mbar_wait_drain(&r.full[q], static_cast<uint32_t>(s.last_parity[q]));
-  }
-  if (warp == 1 && lane == 0) {
-    umma_commit(r.drain);  // all MMAs issued by this thread are complete once this lands
-    mbar_wait_drain(r.drain, 0);
-  }
-  if (warp >= 2 && s.wrote_tma) {
-    if (lane == 0) bulk_wait0();  // stores complete before the CTA (and its smem) goes away
-    __syncwarp();
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      const uint64_t pol_act = policy_evict_last();
+      const uint64_t pol_w = policy_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_parity[STAGES];
+      for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const Tile tl = decode<KIND>(p, t);
+        if constexpr (is_wgrad<KIND>()) {
+          // K runs over the expert's padded rows in each macrobatch of the chunk, in order
+          for (int m = tl.m; m < tl.shift && ok; ++m) {
+            const int sg = m * p.El + tl.el;
+            const int r0 = __ldg(p.poff + sg), r1 = __ldg(p.poff + sg + 1);
+            const int xs = (KIND == G_WGRAD_GATEUP && p.ring_shift) ? __ldg(p.ring_shift + m) : 0;
+            for (int row = r0; row < r1; row += 64) {
+              if (!mbar_wait(&empty[stage], phase ^ 1, p.status)) { ok = false; break; }
+              uint8_t* sA = smem + stage * GEMM_STAGE_BYTES;
+              mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(GEMM_STAGE_BYTES));
+              load_wgrad<KIND>(p, tl, row, xs, sA, sA + GEMM_A_BYTES, &full[stage], pol_act);
+              last_parity[stage] = static_cast<int>(phase);
+              if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+          }
+        } else {
+          for (int kb = 0; kb < tl.nk; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, p.status)) { ok = false; break; }
+            uint8_t* sA = smem + stage * GEMM_STAGE_BYTES;
+            uint8_t* sB = sA + GEMM_A_BYTES;
+            mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(GEMM_STAGE_BYTES));
+            load_stage<KIND>(p, tl, kb, sA, sB, &full[stage], pol_act, pol_w);
+            last_parity[stage] = static_cast<int>(phase);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+        }
+      }
+      if (!ok) {  // let copies already in flight land before the CTA's smem goes away
+        for (int s = 0; s < STAGES; ++s)
+          if (last_parity[s] >= 0) mbar_wait_drain(&full[s], static_cast<uint32_t>(last_parity[s]));
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
+        const Tile tl = decode<KIND>(p, t);
+        const int acc = it & 1;
+        const uint32_t accp = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], accp ^ 1, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dtm = tbase + acc * GEMM_BN;
+        for (int kb = 0; kb < tl.nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * GEMM_STAGE_BYTES);
+          const uint32_t b0 = a0 + static_cast<uint32_t>(GEMM_A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // 4 x K16 per 64-wide block
+            const uint64_t ad = Traits<KIND>::A_MN ? sdesc_sw128(a0 + kk * 2048, 8192, 1024)
+                                                   : sdesc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t bd = Traits<KIND>::B_MN ? sdesc_sw128(b0 + kk * 2048, 8192, 1024)
+                                                   : sdesc_sw128(b0 + kk * 32, 16, 1024);
+            umma_bf16(dtm, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        if (tl.nk > 0) umma_commit(&tfull[acc]);
+        else mbar_arrive(&tfull[acc]);
+      }
+      umma_commit(drain);  // all MMAs issued by this thread are complete once this lands
+      mbar_wait_drain(drain, 0);
+    }
+  } else {
+    // ---------------- epilogue warps 2..5 ----------------
+    const int quarter = warp & 3;  // TMEM lanes this warp may access: 32*quarter ..
+    const int row = quarter * 32 + lane;
+    int it = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+      const Tile tl = decode<KIND>(p, t);
+      const int acc = it & 1;
+      const uint32_t accp = (it >> 1) & 1;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&tfull[acc], accp, p.status) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t taddr = tbase + (static_cast<uint32_t>(quarter * 32) << 16) + acc * GEMM_BN;
+      if constexpr (is_wgrad<KIND>())
+        epilogue_wgrad<KIND>(p, tl, quarter, lane, taddr, stage_out + (warp - 2) * (GEMM_STAGE_OUT_BYTES / 4));
+      else
+        epilogue_row<KIND>(p, tl, row, taddr);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+    if constexpr (is_wgrad<KIND>()) {
+      if (lane == 0) bulk_wait0();  // stores complete before the CTA (and its smem) goes away
+      __syncwarp();
+    }
   }
   __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(r.tbase, 512);
+    tmem_dealloc(tbase, 512);
   }
-}
-
-template <int KIND>
-__global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_constant__ GemmParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  constexpr int STAGES = stages_of<KIND>();
-  const CtaRes r = cta_setup(smem_raw, STAGES, STAGES * GEMM_STAGE_BYTES,
-                             is_wgrad<KIND>() ? GEMM_STAGE_OUT_BYTES : 0, p);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  RoleState s;
-  for (int q = 0; q < GEMM_STAGES; ++q) s.last_parity[q] = -1;
-  if (warp == 0) {
-    if (lane == 0) producer_loop<KIND, STAGES>(p, r, s, blockIdx.x, gridDim.x);
-  } else if (warp == 1) {
-    if (lane == 0) mma_loop<KIND, STAGES>(p, r, s, blockIdx.x, gridDim.x);
-  } else {
-    epilogue_loop<KIND>(p, r, s, blockIdx.x, gridDim.x, warp, lane);
-  }
-  cta_finish<STAGES>(r, s, warp, lane);
 }
 
 template <int KIND>

@@ -122,6 +122,7 @@ constexpr int router_splits(int64_t T, int E, int d) {  // K splits of the route
 }
 
 cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream_t st);
+
 // ---------------------------------------------------------------------------
 // MXFP8 grouped GEMMs (tcgen05 kind::mxf8f6f4 block_scale), see gemm_mx.cu
 // ---------------------------------------------------------------------------
