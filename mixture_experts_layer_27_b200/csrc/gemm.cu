@@ -316,12 +316,12 @@ __device__ __forceinline__ void epilogue_row(const GemmParams& p, const Tile& tl
   }
 }
 
-// wgrad epilogue: the warp's 32 x 256 slice of the output tile goes through a
-// 128B-swizzled staging buffer and out by TMA stores.  Mode (from the chunk
+// wgrad epilogue: the warp's 32 x 256 slice of the output tile.  Mode (from the chunk
 // descriptor of a ring-streamed backward; 0 otherwise):
 //   0  bf16 dW (the whole contraction was in this launch)
 //   1  fp32 partial into the accumulator (first of several chunks)
 //   2  fp32: accumulator + this chunk's partial, back into the accumulator
+// Both go through a 128B-swizzled staging buffer and out by TMA stores.
 // Chunks run in a fixed order, so the sum is reproducible.
 __device__ __forceinline__ void stage_chunk16(uint8_t* box, int lane, int chunk, uint4 u) {
   *reinterpret_cast<uint4*>(box + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = u;
@@ -330,96 +330,92 @@ __device__ __forceinline__ void stage_chunk16(uint8_t* box, int lane, int chunk,
 template <int KIND>
 __device__ __forceinline__ void epilogue_wgrad(const GemmParams& p, const Tile& tl, int quarter, int lane,
                                                uint32_t taddr, uint8_t* stage_out) {
-  const CUtensorMap* map;
-  int x0, y0, yacc = 0;
+  int x0, y0, yacc = 0, up = 0;
   if constexpr (KIND == G_WGRAD_GATEUP) {
     const int NTg = p.I / 256;
-    const int up = tl.nt < NTg ? 0 : 1;
-    map = up ? &p.to1 : &p.to0;  // dW_gate or dW_up as [El*d, I]
+    up = tl.nt < NTg ? 0 : 1;  // dW_gate or dW_up as [El*d, I]
     x0 = (tl.nt - up * NTg) * 256;
     y0 = tl.el * p.d + tl.m0 + quarter * 32;
     yacc = (up * p.El + tl.el) * p.d + tl.m0 + quarter * 32;  // accumulator as [2*El*d, I] fp32
   } else {
-    map = &p.to0;  // dW_down as [El*I, d]
-    x0 = tl.n0;
+    x0 = tl.n0;  // dW_down as [El*I, d]
     y0 = tl.el * p.I + tl.m0 + quarter * 32;
   }
   const int mode = (KIND == G_WGRAD_GATEUP && p.chunk) ? __ldg(p.chunk + 3) : 0;
+  // The warp's 16 KB staging slice holds four boxes.  Each box is staged, stored and committed
+  // as its own bulk group, and a box slot is refilled once the store issued from it one tile
+  // (bf16) or half a tile (fp32) earlier has been read: all but the 3 newest groups.  So the
+  // TMA engine drains box b while the warp converts box b+1.
   if (mode == 0) {
-    if (lane == 0) bulk_wait_read0();  // the previous tile's stores have left the buffer
-    __syncwarp();
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
-      float v[32];
+    for (int b = 0; b < 4; ++b) {  // 64 bf16 columns per box
+      float v[64];
       if (tl.nk > 0) {
-        tmem_ld32(taddr + c * 32, v);
+        tmem_ld64(taddr + b * 64, v);
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0.f;  // expert without tokens: zero gradient
+        for (int i = 0; i < 64; ++i) v[i] = 0.f;  // expert without tokens: zero gradient
       }
-      uint8_t* box = stage_out + (c >> 1) * 4096;
+      if (lane == 0) bulk_wait_read<3>();
+      __syncwarp();
+      uint8_t* box = stage_out + b * 4096;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 8; ++q) {
         uint4 u;
         u.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
         u.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
         u.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
         u.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
-        stage_chunk16(box, lane, (c & 1) * 4 + q, u);
+        stage_chunk16(box, lane, q, u);
       }
-    }
-    fence_proxy_async();
-    __syncwarp();
-    if (lane == 0) {
-#pragma unroll
-      for (int b = 0; b < 4; ++b) tma_store_2d(map, stage_out + b * 4096, x0 + b * 64, y0);
-      bulk_commit();
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(up ? &p.to1 : &p.to0, box, x0 + b * 64, y0);
+        bulk_commit();
+      }
     }
     return;
   }
-  // fp32 accumulator: two halves of 128 columns, four 32 x 32 fp32 boxes each
+  // fp32 accumulator: eight 32 x 32 fp32 boxes
   const float* prev = p.acc32 + static_cast<size_t>(yacc + lane) * p.I + x0;
 #pragma unroll 1
-  for (int h = 0; h < 2; ++h) {
-    if (lane == 0) bulk_wait_read0();
-    __syncwarp();
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      const int col = h * 128 + c * 32;
-      float v[32];
-      if (tl.nk > 0) {
-        tmem_ld32(taddr + col, v);
-      } else {
+  for (int j = 0; j < 8; ++j) {
+    const int col = j * 32;
+    float v[32];
+    if (tl.nk > 0) {
+      tmem_ld32(taddr + col, v);
+    } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0.f;
-      }
-      if (mode == 2) {
-        const float4* pv = reinterpret_cast<const float4*>(prev + col);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 o = pv[q];
-          v[4 * q + 0] = o.x + v[4 * q + 0];
-          v[4 * q + 1] = o.y + v[4 * q + 1];
-          v[4 * q + 2] = o.z + v[4 * q + 2];
-          v[4 * q + 3] = o.w + v[4 * q + 3];
-        }
-      }
-      uint8_t* box = stage_out + c * 4096;
+      for (int i = 0; i < 32; ++i) v[i] = 0.f;
+    }
+    if (mode == 2) {
+      const float4* pv = reinterpret_cast<const float4*>(prev + col);
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        uint4 u;
-        u.x = __float_as_uint(v[4 * q + 0]);
-        u.y = __float_as_uint(v[4 * q + 1]);
-        u.z = __float_as_uint(v[4 * q + 2]);
-        u.w = __float_as_uint(v[4 * q + 3]);
-        stage_chunk16(box, lane, q, u);
+        const float4 o = pv[q];
+        v[4 * q + 0] = o.x + v[4 * q + 0];
+        v[4 * q + 1] = o.y + v[4 * q + 1];
+        v[4 * q + 2] = o.z + v[4 * q + 2];
+        v[4 * q + 3] = o.w + v[4 * q + 3];
       }
+    }
+    if (lane == 0) bulk_wait_read<3>();
+    __syncwarp();
+    uint8_t* box = stage_out + (j & 3) * 4096;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      uint4 u;
+      u.x = __float_as_uint(v[4 * q + 0]);
+      u.y = __float_as_uint(v[4 * q + 1]);
+      u.z = __float_as_uint(v[4 * q + 2]);
+      u.w = __float_as_uint(v[4 * q + 3]);
+      stage_chunk16(box, lane, q, u);
     }
     fence_proxy_async();
     __syncwarp();
     if (lane == 0) {
-#pragma unroll
-      for (int b = 0; b < 4; ++b) tma_store_2d(&p.tacc, stage_out + b * 4096, x0 + h * 128 + b * 32, yacc);
+      tma_store_2d(&p.tacc, box, x0 + col, yacc);
       bulk_commit();
     }
   }
