@@ -87,6 +87,19 @@ __device__ __forceinline__ int num_tiles(const GemmParams& p) {
   return p.El * mtiles_w<KIND>(p) * ntiles_n<KIND>(p);
 }
 
+// K blocks (64 rows) of segment (macrobatch m, local expert el) in a weight-gradient GEMM: its
+// real rows rounded up to 64.  They are a prefix of the segment, and the rows past them up to
+// the next multiple of 64 are zero pad rows, so the 128-row padding adds no K work.
+__device__ __forceinline__ int wgrad_kblocks(const GemmParams& p, int m, int el) {
+  const int tot = __ldg(p.cnt + el);
+  int rows = tot;
+  if (p.cum) {
+    const int nm = p.nseg / p.El;
+    rows = (m + 1 < nm ? __ldg(p.cum + (m + 1) * p.El + el) : tot) - __ldg(p.cum + m * p.El + el);
+  }
+  return (rows + 63) / 64;
+}
+
 template <int KIND>
 __device__ __forceinline__ Tile decode(const GemmParams& p, int t) {
   Tile tl;
@@ -130,10 +143,7 @@ __device__ __forceinline__ Tile decode(const GemmParams& p, int t) {
     const int m_lo = p.chunk ? __ldg(p.chunk) : 0;
     const int m_hi = p.chunk ? __ldg(p.chunk + 1) : p.nseg / p.El;
     int nk = 0;
-    for (int m = m_lo; m < m_hi; ++m) {
-      const int s = m * p.El + el;
-      nk += (__ldg(p.poff + s + 1) - __ldg(p.poff + s)) / 64;
-    }
+    for (int m = m_lo; m < m_hi; ++m) nk += wgrad_kblocks(p, m, el);
     tl.m = m_lo;
     tl.shift = m_hi;
     tl.el = el;
@@ -485,10 +495,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         const Tile tl = decode<KIND>(p, t);
         if constexpr (is_wgrad<KIND>()) {
-          // K runs over the expert's padded rows in each macrobatch of the chunk, in order
+          // K runs over the expert's rows in each macrobatch of the chunk, in order
           for (int m = tl.m; m < tl.shift && ok; ++m) {
             const int sg = m * p.El + tl.el;
-            const int r0 = __ldg(p.poff + sg), r1 = __ldg(p.poff + sg + 1);
+            const int r0 = __ldg(p.poff + sg), r1 = r0 + 64 * wgrad_kblocks(p, m, tl.el);
             const int xs = (KIND == G_WGRAD_GATEUP && p.ring_shift) ? __ldg(p.ring_shift + m) : 0;
             for (int row = r0; row < r1; row += 64) {
               if (!mbar_wait(&empty[stage], phase ^ 1, p.status)) { ok = false; break; }

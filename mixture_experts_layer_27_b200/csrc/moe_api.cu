@@ -300,6 +300,7 @@ static GemmParams base_params(const Layout& L, const Ctx& c, int* status) {
   std::memset(&p, 0, sizeof(p));
   p.hdr = c.hdr;
   p.poff = c.poff;
+  p.cnt = c.counts + L.first;
   p.row_gate = c.row_gate;
   p.El = L.El;
   p.d = L.d;
@@ -717,6 +718,7 @@ moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
   {
     GemmParams p = base_params(L, c, status);
     p.poff = c.tab.seg_poff;
+    p.cum = c.tab.cum;
     p.nseg = nseg;
     MOE_TMAP(tmap_2d(&p.ta0, c.dyperm, L.d, RP, L.d, 64, 128));
     MOE_TMAP(tmap_2d(&p.tb0, W_down, L.d, El * L.I, L.d, 64, 256));
@@ -738,6 +740,7 @@ moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
   {
     GemmParams p = base_params(L, c, status);
     p.poff = c.tab.seg_poff;
+    p.cum = c.tab.cum;
     p.nseg = nseg;
     MOE_TMAP(tmap_2d(&p.ta0, c.dabuf, L.I, RP, L.I, 64, 128));
     MOE_TMAP(tmap_2d(&p.ta1, c.dbbuf, L.I, RP, L.I, 64, 128));
@@ -750,6 +753,7 @@ moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
   {  // wgrad of W_down: Hg and dY_perm cover the whole stream
     GemmParams p = base_params(L, c, status);
     p.poff = c.tab.seg_poff;
+    p.cum = c.tab.cum;
     p.nseg = nseg;
     MOE_TMAP(tmap_2d(&p.ta0, c.hgbuf, L.I, RP, L.I, 64, 64));
     MOE_TMAP(tmap_2d(&p.tb0, c.dyperm, L.d, RP, L.d, 64, 64));
@@ -764,6 +768,7 @@ moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
   {
     GemmParams p = base_params(L, c, status);
     p.poff = c.tab.seg_poff;
+    p.cum = c.tab.cum;
     p.nseg = nseg;
     p.ring_shift = c.tab.shift_bwd;
     p.acc32 = c.acc32;

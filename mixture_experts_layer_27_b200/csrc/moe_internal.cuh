@@ -94,6 +94,10 @@ struct GemmParams {
   int nseg;
   const int* ring_shift;      // per macrobatch: ring row - padded row of X_perm (NULL: X_perm not in a ring)
   const int* chunk;           // wgrad gate/up over a chunk of macrobatches: {m_lo, m_hi, valid, mode}; NULL = all
+  // Real (unpadded) rows of a segment, a prefix of it: cnt[el] for one batch; with a ring
+  // stream cum[m*El+el] counts el's rows in macrobatches before m (cnt[el] = the total).
+  const int* cnt;
+  const int* cum;
   float* acc32;               // fp32 accumulator for dW_gate / dW_up when a backward needs several chunks
   const float* row_gate;      // [RP]
   const __nv_bfloat16* in0;   // epilogue inputs

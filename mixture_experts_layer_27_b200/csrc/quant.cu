@@ -78,46 +78,62 @@ __global__ void __launch_bounds__(128) k_quant_weight(const __nv_bfloat16* __res
 
 // Dispatch / reverse-combine in MXFP8 mode: rows [lo, hi) of the padded layout get the
 // bf16 row (kept for the weight gradients) and its fp8 codes + scales along d.
-__global__ void __launch_bounds__(128) k_gather_rows_mx(const __nv_bfloat16* __restrict__ src,
+__global__ void __launch_bounds__(256) k_gather_rows_mx(const __nv_bfloat16* __restrict__ src,
                                                         const int* __restrict__ row_asg, const int* __restrict__ lo,
                                                         const int* __restrict__ hi, int k, int d,
                                                         __nv_bfloat16* __restrict__ dst, uint8_t* __restrict__ q,
                                                         uint8_t* __restrict__ qs) {
+  // One warp per padded row.  Lane i takes the row's 16-byte chunks i, i + 32, ... (8 values
+  // each), four chunks in flight; the four lanes 4m .. 4m+3 hold one 32-value block and share
+  // its amax through two xor shuffles.  d is a multiple of 256, so every lane runs the same
+  // number of chunks and the shuffles see the whole warp.
   const int r0 = __ldg(lo), r1 = __ldg(hi);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nb = d / 32;
-  for (int64_t R = r0 + blockIdx.x * 4 + warp; R < r1; R += gridDim.x * 4) {
-    const int a = row_asg[R];
-    for (int b = lane; b < nb; b += 32) {
-      float v[32];
+  const int nv = d / 8;
+  for (int64_t R = r0 + blockIdx.x * 8 + warp; R < r1; R += gridDim.x * 8) {
+    const int a = __ldg(row_asg + R);
+    const uint4* in = a >= 0 ? reinterpret_cast<const uint4*>(src + static_cast<size_t>(a / k) * d) : nullptr;
+    uint4* o = reinterpret_cast<uint4*>(dst + R * d);
+    uint2* qd = reinterpret_cast<uint2*>(q + R * d);
+    for (int c0 = lane; c0 < nv; c0 += 128) {
       uint4 u[4];
-      if (a >= 0) {
-        const uint4* in = reinterpret_cast<const uint4*>(src + static_cast<size_t>(a / k) * d + b * 32);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) u[j] = __ldg(in + j);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) u[j] = make_uint4(0, 0, 0, 0);
+      for (int j = 0; j < 4; ++j) {
+        const int c = c0 + 32 * j;
+        u[j] = (in != nullptr && c < nv) ? __ldg(in + c) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
+        const int c = c0 + 32 * j;
+        if (c >= nv) break;  // the same for every lane of the warp
+        o[c] = u[j];
         const uint32_t w4[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+        float v[8];
+        float amax = 0.f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float2 f = unpack_bf16(w4[i]);
-          v[8 * j + 2 * i] = f.x;
-          v[8 * j + 2 * i + 1] = f.y;
+          v[2 * i] = f.x;
+          v[2 * i + 1] = f.y;
+          amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
         }
-      }
-      uint4* o = reinterpret_cast<uint4*>(dst + R * d + b * 32);
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        // the block rule of mx_quant32: exponent floor(log2 amax) - 8, byte clamped to [0, 254]
+        int byte = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 8;
+        byte = byte < 0 ? 0 : (byte > 254 ? 254 : byte);
+        const float inv = __uint_as_float(static_cast<uint32_t>(254 - byte) << 23);
+        uint32_t w[2];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) o[j] = u[j];
-      uint32_t w[8];
-      const uint8_t sb = mx_quant32(v, w);
-      uint4* qd = reinterpret_cast<uint4*>(q + R * d + b * 32);
-      qd[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      qd[1] = make_uint4(w[4], w[5], w[6], w[7]);
-      qs[sf_index(static_cast<int>(R), b * 32, d)] = sb;
+        for (int h = 0; h < 2; ++h) {
+          uint16_t p0, p1;
+          asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(p0) : "f"(v[4 * h] * inv), "f"(v[4 * h + 1] * inv));
+          asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(p1) : "f"(v[4 * h + 2] * inv), "f"(v[4 * h + 3] * inv));
+          w[h] = amax == 0.f ? 0u : (static_cast<uint32_t>(p0) | (static_cast<uint32_t>(p1) << 16));
+        }
+        qd[c] = make_uint2(w[0], w[1]);
+        if ((lane & 3) == 0) qs[sf_index(static_cast<int>(R), c * 8, d)] = static_cast<uint8_t>(byte);
+      }
     }
   }
 }
@@ -139,9 +155,9 @@ cudaError_t launch_quant_weight(int mode, const __nv_bfloat16* src0, const __nv_
 
 cudaError_t launch_gather_rows_mx(const Layout& L, const Ctx& c, const __nv_bfloat16* src, __nv_bfloat16* dst,
                                   uint8_t* q, uint8_t* qs, cudaStream_t st) {
-  const int64_t g = (L.RP + 3) / 4;
-  const int grid = static_cast<int>(g < 148 * 8 ? g : 148 * 8);
-  k_gather_rows_mx<<<grid, 128, 0, st>>>(src, c.row_asg, c.poff, c.poff + L.El, L.k, L.d, dst, q, qs);
+  const int64_t g = (L.RP + 7) / 8;
+  const int grid = static_cast<int>(g < 148 * 8 ? (g > 0 ? g : 1) : 148 * 8);
+  k_gather_rows_mx<<<grid, 256, 0, st>>>(src, c.row_asg, c.poff, c.poff + L.El, L.k, L.d, dst, q, qs);
   return cudaGetLastError();
 }
 

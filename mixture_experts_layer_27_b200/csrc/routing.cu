@@ -197,16 +197,24 @@ __global__ void __launch_bounds__(128) k_gather_rows(const __nv_bfloat16* __rest
                                                      int d, __nv_bfloat16* __restrict__ dst) {
   const int r0 = __ldg(lo), r1 = __ldg(hi);
   const int sh = shift ? __ldg(shift) : 0;
-  const int nv = d / 8;
+  const int nv = d / 8;  // 16-byte chunks per row
   for (int64_t R = r0 + blockIdx.x; R < r1; R += gridDim.x) {
     const int a = row_asg[R];
     uint4* out = reinterpret_cast<uint4*>(dst + (R + sh) * d);
-    if (a >= 0) {
-      const uint4* in = reinterpret_cast<const uint4*>(src + static_cast<size_t>(a / k) * d);
-      for (int i = threadIdx.x; i < nv; i += blockDim.x) out[i] = __ldg(in + i);
-    } else {
-      const uint4 z = make_uint4(0, 0, 0, 0);
-      for (int i = threadIdx.x; i < nv; i += blockDim.x) out[i] = z;
+    const uint4* in = a >= 0 ? reinterpret_cast<const uint4*>(src + static_cast<size_t>(a / k) * d) : nullptr;
+    // four independent loads in flight per thread before their stores
+    for (int i0 = threadIdx.x; i0 < nv; i0 += 4 * blockDim.x) {
+      uint4 u[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = i0 + j * blockDim.x;
+        u[j] = (in != nullptr && i < nv) ? __ldg(in + i) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = i0 + j * blockDim.x;
+        if (i < nv) out[i] = u[j];
+      }
     }
   }
 }
