@@ -11,6 +11,7 @@ Workloads (the pages name model families and print no shapes; these stand in):
 * ``kimi_mx``   ``kimi`` in MXFP8 mode
 * ``ep64``      6 local experts of 384, 16 minibatches x 2048 tokens, ring buffer
 * ``dsv3_e16``  the dsv3 expert shape with 16 experts and 128 tokens (profiler captures)
+* ``kimi_mx_e24`` the kimi expert shape in MXFP8, 24 experts, 256 tokens (profiler captures)
 
 Distributions: X, dY ~ N(0, 1); W_gate, W_up ~ N(0, 1/d) (std 1/sqrt(fan_in));
 W_down ~ N(0, 1/I); W_r ~ N(0, 0.02^2); every tensor rounded once to bf16 (RNE).
@@ -67,6 +68,9 @@ WORKLOADS = {
     # the dsv3 expert shape and load (64 tokens per expert) with 16 experts: a
     # ~3 GB case for profiler captures (weights still exceed the 126 MB L2)
     "dsv3_e16": Workload("dsv3_e16", 128, 7168, 16, 8, 2048),
+    # the kimi expert shape in MXFP8 with 24 experts and 256 tokens (~85 per expert, near-uniform):
+    # a few-GB case for profiler captures of the block-scaled GEMMs
+    "kimi_mx_e24": Workload("kimi_mx_e24", 256, 7168, 24, 8, 2048, mxfp8=True),
 }
 # Per-rank expert slice as at EP64: 6 local experts of 384, 16 minibatches of 2048
 # tokens streamed through a 256 MiB ring; n = tokens each local expert receives.
