@@ -3,11 +3,17 @@
 //
 // Same persistent warp-specialised structure as the bf16 engine (gemm.cu), with
 // tcgen05.mma kind::mxf8f6f4.block_scale: E4M3 operands, one E8M0 scale per 32
-// values along K.  Every stage carries a 128 x 128-byte tile of each operand
-// and one 512-byte scale chunk for each; the MMA thread copies the chunks into
-// a per-stage TMEM slot (tcgen05.cp) and issues four K = 32 MMAs whose sf_id
-// selects the K block.  Output tiles are 128 x 128 (two fp32 accumulators of
-// 128 TMEM columns, double-buffered; scale slots live above them).
+// values along K.  Every stage carries a 128-byte-deep K slice of a 128-row A
+// tile and a 256-row B tile, with their 512-byte scale chunks (one for A, two
+// for B); the MMA thread copies the chunks into a per-stage TMEM slot
+// (tcgen05.cp) and issues four K = 32 MMAs whose sf_id selects the K block.
+// Output tiles are 128 x 256 (gate/up, down, dgrad of gate/up): 32 KB of fp8
+// weights per stage keeps as many weight bytes in flight per SM as the bf16
+// engine; the fp32 accumulator takes 256 TMEM columns and the scale slots sit
+// above it, so there is one accumulator (the producer keeps loading while the
+// epilogue drains it).  The dgrad of W_down, whose epilogue reads A and B and
+// writes five outputs, uses 128 x 128 tiles with two accumulators instead, so
+// its epilogue overlaps the next tile's MMAs.
 #include "moe_internal.cuh"
 #include "ptx.cuh"
 
@@ -19,9 +25,9 @@ struct MxTile {
 
 template <int KIND>
 __device__ __forceinline__ int mx_ntiles_n(const MxParams& p) {
-  if (KIND == MX_GATEUP) return p.I / 64;  // 64 gate + 64 up columns
-  if (KIND == MX_DGRAD_DOWN) return p.I / 128;
-  return p.d / 128;  // MX_DOWN, MX_DGRAD_GATEUP
+  if (KIND == MX_GATEUP) return p.I / (mx_bn(KIND) / 2);  // per tile: [64 gate | 64 up] column pairs
+  if (KIND == MX_DGRAD_DOWN) return p.I / mx_bn(KIND);
+  return p.d / mx_bn(KIND);  // MX_DOWN, MX_DGRAD_GATEUP
 }
 template <int KIND>
 __device__ __forceinline__ int mx_kblocks(const MxParams& p) {
@@ -57,7 +63,7 @@ __device__ __forceinline__ MxTile mx_decode(const MxParams& p, int t) {
   tl.el = seg % p.El;
   tl.m0 = p0 + mi * 128;
   tl.nt = nt;
-  tl.n0 = nt * (KIND == MX_GATEUP ? 64 : 128);
+  tl.n0 = nt * (KIND == MX_GATEUP ? mx_bn(KIND) / 2 : mx_bn(KIND));  // MX_GATEUP: first column of H / A / B
   tl.nk = mx_kblocks<KIND>(p);
   return tl;
 }
@@ -67,15 +73,16 @@ template <int KIND>
 __device__ __forceinline__ void mx_load(const MxParams& p, const MxTile& tl, int kb, uint8_t* st, uint64_t* bar,
                                         uint64_t pol_act, uint64_t pol_w) {
   uint8_t* sA = st;
-  uint8_t* sB = st + 16384;
-  uint8_t* sSF = st + 32768;
+  constexpr int BN = mx_bn(KIND);
+  uint8_t* sB = st + MX_A_BYTES;
+  uint8_t* sSF = sB + BN * 128;  // the A chunk, then a B chunk per 128 rows of the B tile
   const CUtensorMap* ma = &p.ta0;
   const CUtensorMap* mb = &p.tb0;
   const uint8_t* sfa = p.sfa0;
   const uint8_t* sfb = p.sfb0;
   int kl = kb, brow, KA, KB;
   if constexpr (KIND == MX_GATEUP) {
-    brow = tl.el * 2 * p.I + tl.nt * 128;  // paired [64 gate | 64 up] rows of the prepared weight
+    brow = tl.el * 2 * p.I + tl.nt * BN;  // blocks of paired [64 gate | 64 up] rows of the prepared weight
     KA = KB = p.d;
   } else if constexpr (KIND == MX_DOWN) {
     brow = tl.el * p.d + tl.n0;
@@ -99,6 +106,8 @@ __device__ __forceinline__ void mx_load(const MxParams& p, const MxTile& tl, int
   tma_load_2d(sB, mb, bar, kl * 128, brow, pol_w);
   bulk_load(sSF, sfa + (static_cast<size_t>(tl.m0 >> 7) * (KA >> 7) + kl) * 512, 512, bar);
   bulk_load(sSF + 512, sfb + (static_cast<size_t>(brow >> 7) * (KB >> 7) + kl) * 512, 512, bar);
+  if constexpr (BN == 256)
+    bulk_load(sSF + 1024, sfb + (static_cast<size_t>((brow >> 7) + 1) * (KB >> 7) + kl) * 512, 512, bar);
 }
 
 __device__ __forceinline__ float mx_sigmoid(float a) { return 1.0f / (1.0f + expf(-a)); }
@@ -136,15 +145,17 @@ template <int KIND>
 __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl, int row, uint32_t taddr) {
   const int R = tl.m0 + row;
   const size_t Rz = static_cast<size_t>(R);
+  constexpr int BN = mx_bn(KIND);
   if constexpr (KIND == MX_GATEUP) {
 #pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
+    for (int c = 0; c < BN / 64; ++c) {  // accumulator columns: [64 gate | 64 up] per 128
+      const int j = c >> 1, c32 = (c & 1) * 32;
       float a[32], b[32], h[32];
-      tmem_ld32(taddr + c * 32, a);       // gate
-      tmem_ld32(taddr + 64 + c * 32, b);  // up
+      tmem_ld32(taddr + j * 128 + c32, a);       // gate
+      tmem_ld32(taddr + j * 128 + 64 + c32, b);  // up
 #pragma unroll
       for (int i = 0; i < 32; ++i) h[i] = a[i] * mx_sigmoid(a[i]) * b[i];
-      const int col = tl.n0 + c * 32;
+      const int col = tl.n0 + j * 64 + c32;
       mx_store_bf16_32(p.out0 + Rz * p.I + col, a);
       mx_store_bf16_32(p.out1 + Rz * p.I + col, b);
       mx_store_q32(p.q0, p.qs0, R, col, p.I, h);  // H, the down GEMM's A operand (K = I)
@@ -152,7 +163,7 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
   } else if constexpr (KIND == MX_DOWN) {
     const float g = p.row_gate[R];
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < BN / 32; ++c) {
       float o[32];
       tmem_ld32(taddr + c * 32, o);
 #pragma unroll
@@ -163,7 +174,7 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
     const float g = p.row_gate[R];
     float dg = 0.f;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < BN / 32; ++c) {
       float dh[32], a[32], b[32];
       tmem_ld32(taddr + c * 32, dh);
       const int col = tl.n0 + c * 32;
@@ -186,10 +197,10 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
       mx_store_q32(p.q0, p.qs0, R, col, p.I, a);  // dA, dB: the gate/up dgrad's A operands (K = I)
       mx_store_q32(p.q1, p.qs1, R, col, p.I, b);
     }
-    p.outf[Rz * (p.I / 128) + tl.nt] = dg;
+    p.outf[Rz * (p.I / BN) + tl.nt] = dg;
   } else {
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < BN / 32; ++c) {
       float v[32];
       tmem_ld32(taddr + c * 32, v);
       mx_store_bf16_32(p.out0 + Rz * p.d + tl.n0 + c * 32, v);
@@ -206,23 +217,25 @@ __device__ __forceinline__ void mx_wait_drain(uint64_t* bar, uint32_t parity) {
 
 template <int KIND>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm_mx(const __grid_constant__ MxParams p) {
+  constexpr int BN = mx_bn(KIND), ACCS = mx_accs(KIND), STAGES = mx_stages(KIND);
+  constexpr size_t SB = mx_stage_bytes(KIND);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + MX_STAGES * MX_STAGE_BYTES);
-  uint64_t* empty = full + MX_STAGES;
-  uint64_t* tfull = empty + MX_STAGES;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * SB);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;  // per accumulator
+  uint64_t* tempty = tfull + ACCS;
+  uint64_t* drain = tempty + ACCS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < MX_STAGES; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < ACCS; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -249,21 +262,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm_mx(const __grid_co
       const uint64_t pol_w = policy_evict_first();
       int stage = 0;
       uint32_t phase = 0;
-      int last_parity[MX_STAGES];
-      for (int s = 0; s < MX_STAGES; ++s) last_parity[s] = -1;
+      int last_parity[MX_MAX_STAGES];
+      for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         const MxTile tl = mx_decode<KIND>(p, t);
         for (int kb = 0; kb < tl.nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, p.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(MX_STAGE_BYTES));
-          mx_load<KIND>(p, tl, kb, smem + stage * MX_STAGE_BYTES, &full[stage], pol_act, pol_w);
+          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(mx_stage_tx(KIND)));
+          mx_load<KIND>(p, tl, kb, smem + stage * SB, &full[stage], pol_act, pol_w);
           last_parity[stage] = static_cast<int>(phase);
-          if (++stage == MX_STAGES) { stage = 0; phase ^= 1; }
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
       if (!ok)
-        for (int s = 0; s < MX_STAGES; ++s)
+        for (int s = 0; s < STAGES; ++s)
           if (last_parity[s] >= 0) mx_wait_drain(&full[s], static_cast<uint32_t>(last_parity[s]));
     }
   } else if (warp == 1) {
@@ -274,25 +287,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm_mx(const __grid_co
       int it = 0;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
         const MxTile tl = mx_decode<KIND>(p, t);
-        const int acc = it & 1;
-        const uint32_t accp = (it >> 1) & 1;
+        const int acc = it % ACCS;
+        const uint32_t accp = (it / ACCS) & 1;
         if (!mbar_wait(&tempty[acc], accp ^ 1, p.status)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t dtm = tbase + acc * 128;
+        const uint32_t dtm = tbase + acc * BN;  // accumulators in columns [0, 256)
         for (int kb = 0; kb < tl.nk; ++kb) {
           if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + stage * MX_STAGE_BYTES);
-          const uint32_t b0 = a0 + 16384;
-          const uint32_t sfa_t = tbase + 256 + stage * 8, sfb_t = sfa_t + 4;
-          tc_cp_sf(sfa_t, a0 + 32768);
-          tc_cp_sf(sfb_t, a0 + 32768 + 512);
+          const uint32_t a0 = smem_u32(smem + stage * SB);
+          const uint32_t b0 = a0 + static_cast<uint32_t>(MX_A_BYTES);
+          const uint32_t sf0 = b0 + static_cast<uint32_t>(BN * 128);
+          // scale slot of this stage: 16 columns from column 256 on; A in the first 4,
+          // B (rows 0..127, then 128..255) in the columns from 8 on
+          const uint32_t sfa_t = tbase + 256 + stage * 16, sfb_t = sfa_t + 8;
+          tc_cp_sf(sfa_t, sf0);
+          tc_cp_sf(sfb_t, sf0 + 512);
+          if constexpr (BN == 256) tc_cp_sf(sfb_t + 4, sf0 + 1024);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             umma_mxf8(dtm, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024),
-                      idesc_mxf8(128, 128, static_cast<uint32_t>(kk)), sfa_t, sfb_t, (kb | kk) != 0 ? 1u : 0u);
+                      idesc_mxf8(128, BN, static_cast<uint32_t>(kk)), sfa_t, sfb_t, (kb | kk) != 0 ? 1u : 0u);
           umma_commit(&empty[stage]);
-          if (++stage == MX_STAGES) { stage = 0; phase ^= 1; }
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
         umma_commit(&tfull[acc]);
@@ -306,15 +323,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm_mx(const __grid_co
     int it = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
       const MxTile tl = mx_decode<KIND>(p, t);
-      const int acc = it & 1;
-      const uint32_t accp = (it >> 1) & 1;
+      const int acc = it % ACCS;
+      const uint32_t accp = (it / ACCS) & 1;
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&tfull[acc], accp, p.status) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       __syncwarp();
       tc_fence_after();
-      mx_epilogue<KIND>(p, tl, row, tbase + (static_cast<uint32_t>(quarter * 32) << 16) + acc * 128);
+      mx_epilogue<KIND>(p, tl, row, tbase + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -335,11 +352,11 @@ static cudaError_t mx_launch_kind(const MxParams& p, int grid, cudaStream_t st) 
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
     const cudaError_t e = cudaFuncSetAttribute(k_moe_gemm_mx<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(MX_SMEM_BYTES));
+                                               static_cast<int>(mx_smem_bytes(KIND)));
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  k_moe_gemm_mx<KIND><<<grid, GEMM_THREADS, MX_SMEM_BYTES, st>>>(p);
+  k_moe_gemm_mx<KIND><<<grid, GEMM_THREADS, mx_smem_bytes(KIND), st>>>(p);
   return cudaGetLastError();
 }
 

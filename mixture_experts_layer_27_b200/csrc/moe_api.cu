@@ -81,7 +81,7 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->dabuf = take(RP * s.I * 2);
   L->dbbuf = take(RP * s.I * 2);
   L->hgbuf = take(RP * s.I * 2);
-  L->dgpart = take(RP * (s.I / 128) * 4);  // dg partials per n-tile (256 wide bf16, 128 wide MXFP8)
+  L->dgpart = take(RP * (s.I / 128) * 4);  // dg partials per n-tile of the dgrad-down GEMM (256 wide bf16, 128 MXFP8)
   L->dlasg = take(T * k * 4);
   L->wrt = take(static_cast<size_t>(s.E) * s.d * 2);
   L->dxperm = take(RP * s.d * 2);
@@ -215,12 +215,12 @@ static bool tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t o
 }
 
 // 2-D fp8 (byte) tensor [outer, inner], box {128, 128}, 128-byte swizzle.
-static bool tmap_fp8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer) {
+static bool tmap_fp8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_rows) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {inner};
-  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t box[2] = {128, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -901,8 +901,8 @@ moe_status moe_fwd_mx(const moe_shape* s, const void* X, const void* W_r, const 
   const auto* w = static_cast<const uint8_t*>(wq);
   {
     MxParams p = mx_params(L, c, status);
-    MOE_TMAP(tmap_fp8(&p.ta0, c.xq, L.d, RP));
-    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wgu1, L.d, El * 2 * L.I));
+    MOE_TMAP(tmap_fp8(&p.ta0, c.xq, L.d, RP, 128));
+    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wgu1, L.d, El * 2 * L.I, mx_bn(MX_GATEUP)));
     p.ta1 = p.ta0;
     p.tb1 = p.tb0;
     p.sfa0 = p.sfa1 = c.xqs;
@@ -915,8 +915,8 @@ moe_status moe_fwd_mx(const moe_shape* s, const void* X, const void* W_r, const 
   }
   {
     MxParams p = mx_params(L, c, status);
-    MOE_TMAP(tmap_fp8(&p.ta0, c.hq, L.I, RP));
-    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wd2, L.I, El * L.d));
+    MOE_TMAP(tmap_fp8(&p.ta0, c.hq, L.I, RP, 128));
+    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wd2, L.I, El * L.d, mx_bn(MX_DOWN)));
     p.ta1 = p.ta0;
     p.tb1 = p.tb0;
     p.sfa0 = p.sfa1 = c.hqs;
@@ -960,8 +960,8 @@ moe_status moe_bwd_mx(const moe_shape* s, const void* X, const void* W_r, const 
   }));
   {
     MxParams p = mx_params(L, c, status);
-    MOE_TMAP(tmap_fp8(&p.ta0, c.dyq, L.d, RP));
-    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wd3, L.d, El * L.I));
+    MOE_TMAP(tmap_fp8(&p.ta0, c.dyq, L.d, RP, 128));
+    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wd3, L.d, El * L.I, mx_bn(MX_DGRAD_DOWN)));
     p.ta1 = p.ta0;
     p.tb1 = p.tb0;
     p.sfa0 = p.sfa1 = c.dyqs;
@@ -978,17 +978,17 @@ moe_status moe_bwd_mx(const moe_shape* s, const void* X, const void* W_r, const 
     p.outf = c.dgpart;
     MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm_mx(MX_DGRAD_DOWN, p, grid, st); }));
   }
-  MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st, L.I / 128); }));
+  MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st, L.I / mx_bn(MX_DGRAD_DOWN)); }));
   MOE_TRY(timed(K_DWR, st, [&] { return launch_dwr(L, c, static_cast<const __nv_bfloat16*>(X), dW_r, st); }));
   MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
     return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
   }));
   {
     MxParams p = mx_params(L, c, status);
-    MOE_TMAP(tmap_fp8(&p.ta0, c.daq, L.I, RP));
-    MOE_TMAP(tmap_fp8(&p.ta1, c.dbq, L.I, RP));
-    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wg4, L.I, El * L.d));
-    MOE_TMAP(tmap_fp8(&p.tb1, w + L.wu4, L.I, El * L.d));
+    MOE_TMAP(tmap_fp8(&p.ta0, c.daq, L.I, RP, 128));
+    MOE_TMAP(tmap_fp8(&p.ta1, c.dbq, L.I, RP, 128));
+    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wg4, L.I, El * L.d, mx_bn(MX_DGRAD_GATEUP)));
+    MOE_TMAP(tmap_fp8(&p.tb1, w + L.wu4, L.I, El * L.d, mx_bn(MX_DGRAD_GATEUP)));
     p.sfa0 = c.daqs;
     p.sfa1 = c.dbqs;
     p.sfb0 = w + L.wg4s;

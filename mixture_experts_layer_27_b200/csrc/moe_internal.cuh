@@ -131,13 +131,13 @@ cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream
 // MXFP8 grouped GEMMs (tcgen05 kind::mxf8f6f4 block_scale), see gemm_mx.cu
 // ---------------------------------------------------------------------------
 enum MxKind {
-  MX_GATEUP = 0,        // [A|B] = Xq . [Wg|Wu]q (64 gate + 64 up columns per tile); H quantised in the epilogue
+  MX_GATEUP = 0,        // [A|B] = Xq . [Wg|Wu]q (2 x (64 gate + 64 up) columns per tile); H quantised in the epilogue
   MX_DOWN = 1,          // O' = g * (Hq . Wd_q)
   MX_DGRAD_DOWN = 2,    // dH' = dYq . Wd_q^T; SwiGLU backward; dA, dB quantised in the epilogue
   MX_DGRAD_GATEUP = 3,  // dX_perm = dAq . Wg_q^T + dBq . Wu_q^T
 };
 struct MxParams {
-  CUtensorMap ta0, ta1, tb0, tb1;  // fp8 K-major operands, box {128 bytes of K, 128 rows}
+  CUtensorMap ta0, ta1, tb0, tb1;  // fp8 K-major operands, box {128 bytes of K, 128 rows (A) / mx_bn rows (B)}
   const uint8_t* sfa0;             // scale chunks of the A operands (K = the GEMM's contraction)
   const uint8_t* sfa1;
   const uint8_t* sfb0;             // scale chunks of the B operands
@@ -158,9 +158,21 @@ struct MxParams {
   int El, d, I;
   int* status;
 };
-constexpr int MX_STAGES = 6;
-constexpr size_t MX_STAGE_BYTES = 16384 + 16384 + 1024;  // A tile, B tile, two scale chunks
-constexpr size_t MX_SMEM_BYTES = MX_STAGES * MX_STAGE_BYTES + 1024 + 256;
+// Tile width per kind: 128 x 256 tiles (one accumulator, four stages) keep 32 KB of fp8 weights
+// per stage in flight; the dgrad of W_down, whose epilogue reads and writes the most, keeps
+// 128 x 128 tiles with two accumulators (six stages) so that its epilogue overlaps the MMAs.
+// A stage = A tile (128 rows x 128 bytes of K), B tile (BN rows), the A scale chunk and BN/128
+// B scale chunks; stages start on 1 KB boundaries (128-byte swizzle atoms).
+__host__ __device__ constexpr int mx_bn(int kind) { return kind == MX_DGRAD_DOWN ? 128 : 256; }
+__host__ __device__ constexpr int mx_accs(int kind) { return mx_bn(kind) == 128 ? 2 : 1; }
+__host__ __device__ constexpr int mx_stages(int kind) { return mx_bn(kind) == 128 ? 6 : 4; }
+constexpr size_t MX_A_BYTES = 128 * 128;
+__host__ __device__ constexpr size_t mx_stage_tx(int kind) {  // bytes one stage receives
+  return MX_A_BYTES + static_cast<size_t>(mx_bn(kind)) * 128 + 512 * (1 + mx_bn(kind) / 128);
+}
+__host__ __device__ constexpr size_t mx_stage_bytes(int kind) { return (mx_stage_tx(kind) + 1023) / 1024 * 1024; }
+__host__ __device__ constexpr size_t mx_smem_bytes(int kind) { return mx_stages(kind) * mx_stage_bytes(kind) + 1024 + 256; }
+constexpr int MX_MAX_STAGES = 6;
 cudaError_t launch_gemm_mx(MxKind kind, const MxParams& p, int grid, cudaStream_t st);
 
 // ---------------------------------------------------------------------------
