@@ -87,18 +87,18 @@ __device__ __forceinline__ int num_tiles(const GemmParams& p) {
   return p.El * mtiles_w<KIND>(p) * ntiles_n<KIND>(p);
 }
 
-// K blocks (64 rows) of segment (macrobatch m, local expert el) in a weight-gradient GEMM: its
-// real rows rounded up to 64.  They are a prefix of the segment, and the rows past them up to
-// the next multiple of 64 are zero pad rows, so the 128-row padding adds no K work.
-__device__ __forceinline__ int wgrad_kblocks(const GemmParams& p, int m, int el) {
+// Real rows of segment (macrobatch m, local expert el): a prefix of the segment, pad rows after.
+__device__ __forceinline__ int seg_rows(const GemmParams& p, int m, int el) {
   const int tot = __ldg(p.cnt + el);
-  int rows = tot;
-  if (p.cum) {
-    const int nm = p.nseg / p.El;
-    rows = (m + 1 < nm ? __ldg(p.cum + (m + 1) * p.El + el) : tot) - __ldg(p.cum + m * p.El + el);
-  }
-  return (rows + 63) / 64;
+  if (!p.cum) return tot;
+  const int nm = p.nseg / p.El;
+  return (m + 1 < nm ? __ldg(p.cum + (m + 1) * p.El + el) : tot) - __ldg(p.cum + m * p.El + el);
 }
+// K blocks (64 rows) of a segment in a weight-gradient GEMM: its real rows rounded up to 64, so
+// the 128-row padding adds no K work.  In the last block the MMAs skip the K16 steps past the
+// real rows; the pad rows of the last step they issue (up to the next multiple of 16) are the
+// segment's "live" pad rows, which every producer writes as zeros.
+__device__ __forceinline__ int wgrad_kblocks(const GemmParams& p, int m, int el) { return (seg_rows(p, m, el) + 63) / 64; }
 
 template <int KIND>
 __device__ __forceinline__ Tile decode(const GemmParams& p, int t) {
@@ -240,11 +240,14 @@ __device__ __forceinline__ void load_row32(const __nv_bfloat16* src, float (&v)[
   }
 }
 
-// Epilogue for one output row (this thread's TMEM lane) of tile tl.
+// Epilogue for one output row (this thread's TMEM lane) of tile tl.  Rows past a segment's
+// live pad rows (row_asg == ROW_DEAD) store nothing: no later kernel reads them, so their
+// operand rows may hold anything.  Live pad rows come from zero operand rows and store zeros.
 template <int KIND>
 __device__ __forceinline__ void epilogue_row(const GemmParams& p, const Tile& tl, int row, uint32_t taddr) {
   if constexpr (KIND == G_GATEUP) {
     const size_t R = static_cast<size_t>(tl.m0 + row);
+    const bool live = __ldg(p.row_asg + R) != ROW_DEAD;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       float a[32], b[32], h[32];
@@ -252,27 +255,31 @@ __device__ __forceinline__ void epilogue_row(const GemmParams& p, const Tile& tl
       tmem_ld32(taddr + 128 + c * 32, b);  // up columns
 #pragma unroll
       for (int i = 0; i < 32; ++i) h[i] = a[i] * sigmoidf_(a[i]) * b[i];  // SwiGLU
-      const size_t off = R * p.I + tl.n0 + c * 32;
-      store_row32(p.out0 + off, a);
-      store_row32(p.out1 + off, b);
-      store_row32(p.out2 + off, h);
+      if (live) {
+        const size_t off = R * p.I + tl.n0 + c * 32;
+        store_row32(p.out0 + off, a);
+        store_row32(p.out1 + off, b);
+        store_row32(p.out2 + off, h);
+      }
     }
   } else if constexpr (KIND == G_DOWN) {
     const size_t R = static_cast<size_t>(tl.m0 + row);
-    const float g = p.row_gate[R];  // combine weight, 0 on pad rows
+    const bool live = __ldg(p.row_asg + R) != ROW_DEAD;
+    const float g = p.row_gate[R];  // combine weight
 #pragma unroll 1
     for (int c = 0; c < 8; ++c) {
       float o[32];
       tmem_ld32(taddr + c * 32, o);
 #pragma unroll
       for (int i = 0; i < 32; ++i) o[i] *= g;
-      store_row32(p.out0 + R * p.d + tl.n0 + c * 32, o);
+      if (live) store_row32(p.out0 + R * p.d + tl.n0 + c * 32, o);
     }
   } else if constexpr (KIND == G_DGRAD_DOWN) {
     // dH' = dY W_down^T arrives in TMEM.  With H = silu(A) B rebuilt from the saved A, B:
     //   dg partial = sum_i dH'_i H_i          (router-gate gradient, "SonicMoE-style")
     //   dH = g dH',  dA = dH B silu'(A),  dB = dH silu(A),  Hg = g H (wgrad operand)
     const size_t R = static_cast<size_t>(tl.m0 + row);
+    const bool live = __ldg(p.row_asg + R) != ROW_DEAD;
     const float g = p.row_gate[R];
     float dg = 0.f;
 #pragma unroll 1
@@ -280,8 +287,13 @@ __device__ __forceinline__ void epilogue_row(const GemmParams& p, const Tile& tl
       float dh[32], a[32], b[32];
       tmem_ld32(taddr + c * 32, dh);
       const size_t off = R * p.I + tl.n0 + c * 32;
-      load_row32(p.in0 + off, a);
-      load_row32(p.in1 + off, b);
+      if (live) {
+        load_row32(p.in0 + off, a);
+        load_row32(p.in1 + off, b);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) a[i] = b[i] = 0.f;
+      }
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float s = sigmoidf_(a[i]);
@@ -295,18 +307,21 @@ __device__ __forceinline__ void epilogue_row(const GemmParams& p, const Tile& tl
         b[i] = db;
         dh[i] = g * hh;
       }
-      store_row32(p.out0 + off, a);   // dA
-      store_row32(p.out1 + off, b);   // dB
-      store_row32(p.out2 + off, dh);  // Hg
+      if (live) {
+        store_row32(p.out0 + off, a);   // dA
+        store_row32(p.out1 + off, b);   // dB
+        store_row32(p.out2 + off, dh);  // Hg
+      }
     }
-    p.outf[R * (p.I / 256) + tl.nt] = dg;
+    if (live) p.outf[R * (p.I / 256) + tl.nt] = dg;
   } else if constexpr (KIND == G_DGRAD_GATEUP) {
     const size_t R = static_cast<size_t>(tl.m0 + row);
+    const bool live = __ldg(p.row_asg + R) != ROW_DEAD;
 #pragma unroll 1
     for (int c = 0; c < 8; ++c) {
       float v[32];
       tmem_ld32(taddr + c * 32, v);
-      store_row32(p.out0 + R * p.d + tl.n0 + c * 32, v);
+      if (live) store_row32(p.out0 + R * p.d + tl.n0 + c * 32, v);
     }
   } else if constexpr (KIND == G_ROUTER) {
     // fp32 partial logits of K split tl.el; rows >= T and columns >= E are dropped
@@ -525,6 +540,44 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
         for (int s = 0; s < STAGES; ++s)
           if (last_parity[s] >= 0) mbar_wait_drain(&full[s], static_cast<uint32_t>(last_parity[s]));
       }
+    }
+  } else if (warp == 1 && is_wgrad<KIND>()) {
+    if (lane == 0) {
+      // ---------------- MMA issuer, weight gradients: walks the segments of the tile's expert so
+      // that a segment's last block issues only the K16 steps that hold real rows ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
+        const Tile tl = decode<KIND>(p, t);
+        const int acc = it & 1;
+        const uint32_t accp = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], accp ^ 1, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dtm = tbase + acc * GEMM_BN;
+        int kb = 0;
+        for (int m = tl.m; m < tl.shift && ok; ++m) {
+          const int rows = seg_rows(p, m, tl.el);
+          for (int r = 0; r < rows; r += 64, ++kb) {
+            if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(smem + stage * GEMM_STAGE_BYTES);
+            const uint32_t b0 = a0 + static_cast<uint32_t>(GEMM_A_BYTES);
+            const int valid = rows - r < 64 ? rows - r : 64;
+            for (int kk = 0; kk * 16 < valid; ++kk)
+              umma_bf16(dtm, sdesc_sw128(a0 + kk * 2048, 8192, 1024), sdesc_sw128(b0 + kk * 2048, 8192, 1024), IDESC,
+                        (kb | kk) != 0 ? 1u : 0u);
+            umma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+        }
+        if (!ok) break;
+        if (kb > 0) umma_commit(&tfull[acc]);
+        else mbar_arrive(&tfull[acc]);
+      }
+      umma_commit(drain);  // all MMAs issued by this thread are complete once this lands
+      mbar_wait_drain(drain, 0);
     }
   } else if (warp == 1) {
     if (lane == 0) {

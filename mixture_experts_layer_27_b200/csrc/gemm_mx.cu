@@ -141,10 +141,13 @@ __device__ __forceinline__ void mx_store_q32(uint8_t* q, uint8_t* qs, int R, int
   qs[sf_index(R, c0, K)] = sb;
 }
 
+// Rows past a segment's live pad rows (row_asg == ROW_DEAD) store nothing: no later kernel
+// reads them.
 template <int KIND>
 __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl, int row, uint32_t taddr) {
   const int R = tl.m0 + row;
   const size_t Rz = static_cast<size_t>(R);
+  const bool live = __ldg(p.row_asg + R) != ROW_DEAD;
   constexpr int BN = mx_bn(KIND);
   if constexpr (KIND == MX_GATEUP) {
 #pragma unroll 1
@@ -156,9 +159,11 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
 #pragma unroll
       for (int i = 0; i < 32; ++i) h[i] = a[i] * mx_sigmoid(a[i]) * b[i];
       const int col = tl.n0 + j * 64 + c32;
-      mx_store_bf16_32(p.out0 + Rz * p.I + col, a);
-      mx_store_bf16_32(p.out1 + Rz * p.I + col, b);
-      mx_store_q32(p.q0, p.qs0, R, col, p.I, h);  // H, the down GEMM's A operand (K = I)
+      if (live) {
+        mx_store_bf16_32(p.out0 + Rz * p.I + col, a);
+        mx_store_bf16_32(p.out1 + Rz * p.I + col, b);
+        mx_store_q32(p.q0, p.qs0, R, col, p.I, h);  // H, the down GEMM's A operand (K = I)
+      }
     }
   } else if constexpr (KIND == MX_DOWN) {
     const float g = p.row_gate[R];
@@ -168,7 +173,7 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
       tmem_ld32(taddr + c * 32, o);
 #pragma unroll
       for (int i = 0; i < 32; ++i) o[i] *= g;
-      mx_store_bf16_32(p.out0 + Rz * p.d + tl.n0 + c * 32, o);
+      if (live) mx_store_bf16_32(p.out0 + Rz * p.d + tl.n0 + c * 32, o);
     }
   } else if constexpr (KIND == MX_DGRAD_DOWN) {
     const float g = p.row_gate[R];
@@ -178,8 +183,13 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
       float dh[32], a[32], b[32];
       tmem_ld32(taddr + c * 32, dh);
       const int col = tl.n0 + c * 32;
-      mx_load_bf16_32(p.in0 + Rz * p.I + col, a);
-      mx_load_bf16_32(p.in1 + Rz * p.I + col, b);
+      if (live) {
+        mx_load_bf16_32(p.in0 + Rz * p.I + col, a);
+        mx_load_bf16_32(p.in1 + Rz * p.I + col, b);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) a[i] = b[i] = 0.f;
+      }
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float s = mx_sigmoid(a[i]);
@@ -191,19 +201,21 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
         b[i] = dhg * sl;                                       // dB
         dh[i] = g * hh;                                        // Hg
       }
-      mx_store_bf16_32(p.out0 + Rz * p.I + col, a);
-      mx_store_bf16_32(p.out1 + Rz * p.I + col, b);
-      mx_store_bf16_32(p.out2 + Rz * p.I + col, dh);
-      mx_store_q32(p.q0, p.qs0, R, col, p.I, a);  // dA, dB: the gate/up dgrad's A operands (K = I)
-      mx_store_q32(p.q1, p.qs1, R, col, p.I, b);
+      if (live) {
+        mx_store_bf16_32(p.out0 + Rz * p.I + col, a);
+        mx_store_bf16_32(p.out1 + Rz * p.I + col, b);
+        mx_store_bf16_32(p.out2 + Rz * p.I + col, dh);
+        mx_store_q32(p.q0, p.qs0, R, col, p.I, a);  // dA, dB: the gate/up dgrad's A operands (K = I)
+        mx_store_q32(p.q1, p.qs1, R, col, p.I, b);
+      }
     }
-    p.outf[Rz * (p.I / BN) + tl.nt] = dg;
+    if (live) p.outf[Rz * (p.I / BN) + tl.nt] = dg;
   } else {
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
       float v[32];
       tmem_ld32(taddr + c * 32, v);
-      mx_store_bf16_32(p.out0 + Rz * p.d + tl.n0 + c * 32, v);
+      if (live) mx_store_bf16_32(p.out0 + Rz * p.d + tl.n0 + c * 32, v);
     }
   }
 }

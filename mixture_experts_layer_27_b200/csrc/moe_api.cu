@@ -244,13 +244,13 @@ static int num_sms() {
 enum KernelId {
   K_ROUTER_LOGITS, K_TOPK, K_SCAN, K_SCATTER, K_DISPATCH, K_GEMM_GATEUP, K_GEMM_DOWN, K_COMBINE,
   K_REV_COMBINE, K_GEMM_DGRAD_DOWN, K_ROUTER_BWD, K_DWR, K_TRANSPOSE_WR, K_GEMM_DGRAD_GATEUP, K_REV_DISPATCH,
-  K_GEMM_WGRAD_GATEUP, K_GEMM_WGRAD_DOWN, K_PLAN, K_REPLAY, K_FINISH_ACC, K_QUANT_WEIGHTS, K_NUM
+  K_GEMM_WGRAD_GATEUP, K_GEMM_WGRAD_DOWN, K_PLAN, K_REPLAY, K_FINISH_ACC, K_QUANT_WEIGHTS, K_MARK_ROWS, K_NUM
 };
 static const char* kKernelNames[K_NUM] = {
     "router_logits", "topk_gating", "hist_scan", "stable_scatter", "dispatch", "gemm_gateup_swiglu",
     "gemm_down_combw", "combine", "reverse_combine", "gemm_dgrad_down_swiglu_bwd", "router_bwd", "router_wgrad",
     "transpose_wr", "gemm_dgrad_gateup", "reverse_dispatch", "gemm_wgrad_gateup", "gemm_wgrad_down",
-    "stream_plan", "ring_replay", "wgrad_accumulator_finish", "quantize_weights"};
+    "stream_plan", "ring_replay", "wgrad_accumulator_finish", "quantize_weights", "mark_pad_rows"};
 
 struct ProfRec {
   int kid;
@@ -302,6 +302,7 @@ static GemmParams base_params(const Layout& L, const Ctx& c, int* status) {
   p.poff = c.poff;
   p.cnt = c.counts + L.first;
   p.row_gate = c.row_gate;
+  p.row_asg = c.row_asg;
   p.El = L.El;
   p.d = L.d;
   p.I = L.I;
@@ -401,8 +402,7 @@ static moe_status route_tokens(const Layout& L, const Ctx& c, const void* X, con
     const int min_rows = static_cast<int>((2LL * grid * 128) / (L.I / 128));
     MOE_TRY(timed(K_PLAN, st, [&] { return launch_plan(L, c, ring_rows, min_rows, st); }));
   }
-  MOE_TRY(cudaMemsetAsync(c.row_asg, 0xFF, static_cast<size_t>(L.RP) * 4, st));
-  MOE_TRY(cudaMemsetAsync(c.row_gate, 0, static_cast<size_t>(L.RP) * 4, st));
+  MOE_TRY(timed(K_MARK_ROWS, st, [&] { return launch_mark_rows(L, c, st); }));  // pad rows: live / dead
   MOE_TRY(timed(K_SCATTER, st, [&] { return launch_scatter(L, c, st); }));
   return MOE_OK;
 }
@@ -865,6 +865,7 @@ static MxParams mx_params(const Layout& L, const Ctx& c, int* status) {
   p.poff = c.poff;
   p.nseg = L.El;
   p.row_gate = c.row_gate;
+  p.row_asg = c.row_asg;
   p.El = L.El;
   p.d = L.d;
   p.I = L.I;

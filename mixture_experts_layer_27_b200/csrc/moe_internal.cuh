@@ -32,6 +32,12 @@ enum PlanWord {
   PLAN_RING_ROWS = 5, // ring capacity in rows
   PLAN_WORDS = 16
 };
+// Pad rows of an expert segment (its real rows are a prefix): the first ones, up to the next
+// multiple of 16 rows, are ROW_PAD, written as zero rows by every producer because the weight
+// gradients' last K16 step reads them; the rest are ROW_DEAD, never written and never read.
+constexpr int ROW_PAD = -1;
+constexpr int ROW_DEAD = -2;
+
 struct StreamTables {
   int* plan;       // [PLAN_WORDS]
   int* mb_of;      // [M]        macrobatch of each minibatch
@@ -100,6 +106,7 @@ struct GemmParams {
   const int* cum;
   float* acc32;               // fp32 accumulator for dW_gate / dW_up when a backward needs several chunks
   const float* row_gate;      // [RP]
+  const int* row_asg;         // [RP] assignment of each padded row, ROW_PAD / ROW_DEAD for pad rows
   const __nv_bfloat16* in0;   // epilogue inputs
   const __nv_bfloat16* in1;
   __nv_bfloat16* out0;        // epilogue outputs
@@ -145,6 +152,7 @@ struct MxParams {
   const int* poff;                 // padded expert offsets [nseg+1]
   int nseg;
   const float* row_gate;
+  const int* row_asg;              // assignment of each padded row, ROW_PAD / ROW_DEAD for pad rows
   const __nv_bfloat16* in0;        // dgrad-down epilogue: saved A, B
   const __nv_bfloat16* in1;
   __nv_bfloat16* out0;
@@ -197,6 +205,7 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws);
 cudaError_t launch_topk(const Layout& L, const Ctx& c, const float* bias, int splits, cudaStream_t st);
 cudaError_t launch_scan(const Layout& L, const Ctx& c, cudaStream_t st);
 cudaError_t launch_scatter(const Layout& L, const Ctx& c, cudaStream_t st);
+cudaError_t launch_mark_rows(const Layout& L, const Ctx& c, cudaStream_t st);
 cudaError_t launch_gather_rows(const Layout& L, const Ctx& c, const __nv_bfloat16* src, __nv_bfloat16* dst,
                                cudaStream_t st);
 // rows [*lo, *hi) to dst row + *shift (streamed layer)

@@ -76,8 +76,8 @@ __global__ void __launch_bounds__(128) k_quant_weight(const __nv_bfloat16* __res
   }
 }
 
-// Dispatch / reverse-combine in MXFP8 mode: rows [lo, hi) of the padded layout get the
-// bf16 row (kept for the weight gradients) and its fp8 codes + scales along d.
+// Dispatch / reverse-combine in MXFP8 mode: rows [lo, hi) of the padded layout get the bf16 row
+// (kept for the weight gradients) and its fp8 codes + scales along d; dead pad rows are skipped.
 __global__ void __launch_bounds__(256) k_gather_rows_mx(const __nv_bfloat16* __restrict__ src,
                                                         const int* __restrict__ row_asg, const int* __restrict__ lo,
                                                         const int* __restrict__ hi, int k, int d,
@@ -92,6 +92,7 @@ __global__ void __launch_bounds__(256) k_gather_rows_mx(const __nv_bfloat16* __r
   const int nv = d / 8;
   for (int64_t R = r0 + blockIdx.x * 8 + warp; R < r1; R += gridDim.x * 8) {
     const int a = __ldg(row_asg + R);
+    if (a == ROW_DEAD) continue;  // never read; a live pad row gets zero codes and scale 0
     const uint4* in = a >= 0 ? reinterpret_cast<const uint4*>(src + static_cast<size_t>(a / k) * d) : nullptr;
     uint4* o = reinterpret_cast<uint4*>(dst + R * d);
     uint2* qd = reinterpret_cast<uint2*>(q + R * d);

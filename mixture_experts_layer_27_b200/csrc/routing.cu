@@ -137,6 +137,26 @@ __global__ void __launch_bounds__(1024) k_scan(int* __restrict__ hist, int nblk,
 }
 
 // ---------------------------------------------------------------------------
+// pad-row marks of every segment, before the scatter fills its real rows: rows up to the real
+// count rounded up to 16 are ROW_PAD, the rest of the 128-row padding ROW_DEAD; gates 0.
+// One block per segment; with macrobatches, segment m * El + el counts cum's difference.
+__global__ void __launch_bounds__(128) k_mark_rows(const int* __restrict__ poff, int nseg, int El,
+                                                   const int* __restrict__ cnt, const int* __restrict__ cum, int nm,
+                                                   int* __restrict__ row_asg, float* __restrict__ row_gate) {
+  const int s = blockIdx.x;
+  if (s >= nseg) return;
+  const int el = s % El, m = s / El;
+  const int tot = cnt[el];
+  const int rows = cum ? (m + 1 < nm ? cum[(m + 1) * El + el] : tot) - cum[m * El + el] : tot;
+  const int live = (rows + 15) & ~15;
+  const int r0 = poff[s], r1 = poff[s + 1];
+  for (int r = r0 + threadIdx.x; r < r1; r += blockDim.x) {
+    row_asg[r] = r - r0 < live ? ROW_PAD : ROW_DEAD;
+    row_gate[r] = 0.f;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // stable scatter: one warp per block of tokens, tokens in ascending order.
 // row position of (t, j) inside expert e = base[b][e] + #{earlier tokens of b with e}.
 // ---------------------------------------------------------------------------
@@ -187,7 +207,8 @@ __global__ void __launch_bounds__(32) k_scatter(const int* __restrict__ ids, con
 }
 
 // ---------------------------------------------------------------------------
-// dispatch / reverse-combine: dst[R] = src[token(R)], zero rows for padding.
+// dispatch / reverse-combine: dst[R] = src[token(R)], zero rows for live pad rows, dead pad
+// rows left as they are.
 // ---------------------------------------------------------------------------
 // Rows [*lo, *hi) of the padded layout, written at row R + *shift of dst (a
 // ring position for the streamed layer; shift NULL = 0).
@@ -200,6 +221,7 @@ __global__ void __launch_bounds__(128) k_gather_rows(const __nv_bfloat16* __rest
   const int nv = d / 8;  // 16-byte chunks per row
   for (int64_t R = r0 + blockIdx.x; R < r1; R += gridDim.x) {
     const int a = row_asg[R];
+    if (a == ROW_DEAD) continue;  // never read
     uint4* out = reinterpret_cast<uint4*>(dst + (R + sh) * d);
     const uint4* in = a >= 0 ? reinterpret_cast<const uint4*>(src + static_cast<size_t>(a / k) * d) : nullptr;
     // four independent loads in flight per thread before their stores
@@ -551,6 +573,7 @@ __global__ void __launch_bounds__(128) k_replay(const __nv_bfloat16* __restrict_
     const int sh = tb.shift_bwd[m];
     for (int64_t R = r0 + blockIdx.x; R < r1; R += gridDim.x) {
       const int a = row_asg[R];
+      if (a == ROW_DEAD) continue;
       uint4* out = reinterpret_cast<uint4*>(ring + (R + sh) * d);
       if (a >= 0) {
         const uint4* in = reinterpret_cast<const uint4*>(X + static_cast<size_t>(a / k) * d);
@@ -612,6 +635,13 @@ cudaError_t launch_scatter(const Layout& L, const Ctx& c, cudaStream_t st) {
                                    static_cast<int>(L.T), L.E, L.k, L.first, L.El, static_cast<int>(L.T_mb),
                                    streamed ? c.tab.mb_of : nullptr, streamed ? c.tab.cum : nullptr, c.perm_tok,
                                    c.perm_asg, c.slot_row, c.row_asg, c.row_gate);
+  return cudaGetLastError();
+}
+cudaError_t launch_mark_rows(const Layout& L, const Ctx& c, cudaStream_t st) {
+  const bool mb = L.M > 0;
+  const int nseg = mb ? L.M * L.El : L.El;
+  k_mark_rows<<<nseg, 128, 0, st>>>(mb ? c.tab.seg_poff : c.poff, nseg, L.El, c.counts + L.first,
+                                    mb ? c.tab.cum : nullptr, mb ? L.M : 1, c.row_asg, c.row_gate);
   return cudaGetLastError();
 }
 cudaError_t launch_gather_range(const Layout& L, const Ctx& c, const __nv_bfloat16* src, const int* lo, const int* hi,

@@ -111,3 +111,25 @@ def test_mxfp8_bit_identical_runs():
     for n in ("dX", "dW_gate", "dW_up", "dW_down"):
         assert torch.equal(g[n].view(torch.int16), g2[n].view(torch.int16)), n
     assert torch.equal(g["dW_r"].view(torch.int32), g2["dW_r"].view(torch.int32))
+
+
+def test_mxfp8_results_do_not_depend_on_stale_ctx_and_workspace_contents():
+    T, d, E, k, I = 333, 512, 12, 3, 512
+    w, x = make_case(T, d, E, k, I, seed=45)
+    outs = []
+    for fill in (0, 255):
+        lay = B.MoELayerMX(T, d, E, I, k)
+        lay.ctx.fill_(fill)
+        lay.ws.fill_(fill)
+        lay.prepare(x["W_gate"], x["W_up"], x["W_down"])
+        Y = lay.forward(x["X"], x["W_r"], x["bias"])
+        g = lay.backward(x["X"], x["W_r"], x["dY"])
+        torch.cuda.synchronize()
+        assert lay.error() == B.MOE_OK
+        assert torch.isfinite(Y.float()).all()
+        outs.append((Y, g))
+    (Y0, g0), (Y1, g1) = outs
+    assert torch.equal(Y0.view(torch.int16), Y1.view(torch.int16))
+    for n in ("dX", "dW_gate", "dW_up", "dW_down"):
+        assert torch.equal(g0[n].view(torch.int16), g1[n].view(torch.int16)), n
+    assert torch.equal(g0["dW_r"].view(torch.int32), g1["dW_r"].view(torch.int32))

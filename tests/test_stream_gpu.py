@@ -103,3 +103,26 @@ def test_stream_refuses_a_ring_below_one_minibatch():
     st = B.moe_fwd_stream(s.shape, 4, x["X"], x["W_r"], None, x["W_gate"], x["W_up"], x["W_down"],
                           torch.empty_like(x["X"]), s.ctx, s.ring, s.ws)
     assert st == B.MOE_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_stream_results_do_not_depend_on_stale_ring_ctx_and_workspace():
+    T_mb, M, d, E, k, I = 128, 6, 256, 16, 4, 256
+    T = T_mb * M
+    w, x = make_case(T, d, E, k, I, seed=34)
+    shape = B.make_shape(T_mb, d, E, I, k)
+    ring_bytes = int(B.moe_stream_min_ring_bytes(shape) * 1.2) // (2 * d) * (2 * d)
+    outs = []
+    for fill in (0, 255):
+        s = B.MoEStream(T_mb, d, E, I, k, M, ring_bytes)
+        for buf in (s.ctx, s.ws, s.ring):
+            buf.fill_(fill)
+        Y = s.forward(x["X"], x["W_r"], x["bias"], x["W_gate"], x["W_up"], x["W_down"])
+        g = s.backward(x["X"], x["W_r"], x["W_gate"], x["W_up"], x["W_down"], x["dY"])
+        torch.cuda.synchronize()
+        assert s.error() == B.MOE_OK
+        outs.append((Y, g))
+    (Y0, g0), (Y1, g1) = outs
+    assert torch.equal(Y0.view(torch.int16), Y1.view(torch.int16))
+    for n in ("dX", "dW_gate", "dW_up", "dW_down"):
+        assert torch.equal(g0[n].view(torch.int16), g1[n].view(torch.int16)), n
+    assert torch.equal(g0["dW_r"].view(torch.int32), g1["dW_r"].view(torch.int32))
