@@ -32,6 +32,7 @@ template <> struct Traits<G_DGRAD_GATEUP> { static constexpr bool A_MN = false, 
 template <> struct Traits<G_WGRAD_GATEUP> { static constexpr bool A_MN = true, B_MN = true; };
 template <> struct Traits<G_WGRAD_DOWN>   { static constexpr bool A_MN = true, B_MN = true; };
 template <> struct Traits<G_ROUTER>       { static constexpr bool A_MN = false, B_MN = false; };
+template <> struct Traits<G_ROUTER_WGRAD> { static constexpr bool A_MN = true, B_MN = true; };
 
 // The wgrad GEMMs have short K loops (one expert's rows) and write a full
 // 128 x 256 output tile per tile: they trade a smem stage for a staging
@@ -82,6 +83,7 @@ __device__ __forceinline__ int segment_of_row(const int* poff, int nseg, int R) 
 template <int KIND>
 __device__ __forceinline__ int num_tiles(const GemmParams& p) {
   if (KIND == G_ROUTER) return ((p.T + 127) / 128) * ((p.E + 255) / 256) * p.splits;
+  if (KIND == G_ROUTER_WGRAD) return (p.d / 128) * ((p.E + 255) / 256);
   if (KIND <= G_DGRAD_GATEUP) return ((__ldg(p.poff + p.nseg) - __ldg(p.poff)) / 128) * ntiles_n<KIND>(p);
   if (p.chunk && __ldg(p.chunk + 2) == 0) return 0;  // chunk not used by this routing
   return p.El * mtiles_w<KIND>(p) * ntiles_n<KIND>(p);
@@ -114,6 +116,20 @@ __device__ __forceinline__ Tile decode(const GemmParams& p, int t) {
     tl.n0 = nt * 256;
     tl.kb0 = sp * KB / S;
     tl.nk = (sp + 1) * KB / S - tl.kb0;
+    return tl;
+  }
+  if constexpr (KIND == G_ROUTER_WGRAD) {
+    // tile = (128 rows of d, 256 experts); K = all tokens in 64-row blocks
+    const int NTe = (p.E + 255) / 256;
+    const int mt = t / NTe, nt = t - mt * NTe;
+    tl.m = 0;
+    tl.shift = 0;
+    tl.el = 0;
+    tl.m0 = mt * 128;
+    tl.nt = nt;
+    tl.n0 = nt * 256;
+    tl.kb0 = 0;
+    tl.nk = 2 * ((p.T + 63) / 64);  // the hi terms of dl, then the lo terms
     return tl;
   }
   const int NT = ntiles_n<KIND>(p);
@@ -188,6 +204,16 @@ __device__ __forceinline__ void load_stage(const GemmParams& p, const Tile& tl, 
     const int kx = (tl.kb0 + kb) * 64;
     tma_load_2d(sA, &p.ta0, bar, kx, tl.m0, pol_act);  // X [T, d], rows >= T read as zero
     tma_load_2d(sB, &p.tb0, bar, kx, tl.n0, pol_act);  // W_r^T [E, d], rows >= E read as zero
+  } else if constexpr (KIND == G_ROUTER_WGRAD) {
+    // X [T, d] and DL [2 * Tpad, E64] with the contraction over tokens: both MN-major (d and E
+    // contiguous); K block kb of DL pairs with X's block kb mod Tpad/64; tokens >= T read as
+    // zero, experts >= E64 too
+    const int half = (p.T + 63) / 64;
+    const int kx = (kb < half ? kb : kb - half) * 64;
+    tma_load_2d(sA, &p.ta0, bar, tl.m0, kx, pol_act);
+    tma_load_2d(sA + 8192, &p.ta0, bar, tl.m0 + 64, kx, pol_act);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tma_load_2d(sB + j * 8192, &p.tb0, bar, tl.n0 + 64 * j, k0, pol_act);
   }
 }
 
@@ -322,6 +348,18 @@ __device__ __forceinline__ void epilogue_row(const GemmParams& p, const Tile& tl
       float v[32];
       tmem_ld32(taddr + c * 32, v);
       if (live) store_row32(p.out0 + R * p.d + tl.n0 + c * 32, v);
+    }
+  } else if constexpr (KIND == G_ROUTER_WGRAD) {
+    // dW_r row (of d) tl.m0 + row, fp32; columns >= E are dropped
+    float* dst = p.outf + static_cast<size_t>(tl.m0 + row) * p.E;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      float v[32];
+      tmem_ld32(taddr + c * 32, v);
+      const int e0 = tl.n0 + c * 32;
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (e0 + i < p.E) dst[e0 + i] = v[i];
     }
   } else if constexpr (KIND == G_ROUTER) {
     // fp32 partial logits of K split tl.el; rows >= T and columns >= E are dropped
@@ -677,6 +715,7 @@ cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream
     case G_WGRAD_GATEUP: return launch_kind<G_WGRAD_GATEUP>(p, grid, st);
     case G_WGRAD_DOWN: return launch_kind<G_WGRAD_DOWN>(p, grid, st);
     case G_ROUTER: return launch_kind<G_ROUTER>(p, grid, st);
+    case G_ROUTER_WGRAD: return launch_kind<G_ROUTER_WGRAD>(p, grid, st);
   }
   return cudaErrorInvalidValue;
 }

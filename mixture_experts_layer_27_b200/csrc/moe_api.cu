@@ -83,6 +83,7 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->hgbuf = take(RP * s.I * 2);
   L->dgpart = take(RP * (s.I / 128) * 4);  // dg partials per n-tile of the dgrad-down GEMM (256 wide bf16, 128 MXFP8)
   L->dlasg = take(T * k * 4);
+  L->dldense = take(2 * align_up(static_cast<size_t>(T), 64) * align_up(static_cast<size_t>(s.E), 64) * 2);
   L->wrt = take(static_cast<size_t>(s.E) * s.d * 2);
   L->dxperm = take(RP * s.d * 2);
   L->acc32 = take(M > 0 ? 2 * static_cast<size_t>(El) * s.d * s.I * 4 : 0);
@@ -171,6 +172,7 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
     c.hgbuf = reinterpret_cast<__nv_bfloat16*>(W(L.hgbuf));
     c.dgpart = reinterpret_cast<float*>(W(L.dgpart));
     c.dlasg = reinterpret_cast<float*>(W(L.dlasg));
+    c.dldense = reinterpret_cast<__nv_bfloat16*>(W(L.dldense));
     c.wrt = reinterpret_cast<__nv_bfloat16*>(W(L.wrt));
     c.dxperm = reinterpret_cast<__nv_bfloat16*>(W(L.dxperm));
     c.acc32 = L.M > 0 ? reinterpret_cast<float*>(W(L.acc32)) : nullptr;
@@ -309,6 +311,27 @@ static GemmParams base_params(const Layout& L, const Ctx& c, int* status) {
   p.nseg = L.El;
   p.status = status;
   return p;
+}
+
+// dW_r = X^T . DL on the tensor cores (both operands MN-major: d and E are contiguous, the
+// contraction runs over tokens, twice: the hi and the lo bf16 terms of dl); fp32 out, one CTA
+// per 128 x 256 tile, fixed K order.
+static cudaError_t launch_router_wgrad(const Layout& L, const Ctx& c, const void* X, float* dW_r, int* status,
+                                       cudaStream_t st) {
+  GemmParams p = base_params(L, c, status);
+  const uint64_t E64 = align_up(static_cast<size_t>(L.E), 64);
+  if (!tmap_2d(&p.ta0, X, L.d, static_cast<uint64_t>(L.T), L.d, 64, 64)) return cudaErrorInvalidValue;
+  const uint64_t Tpad = align_up(static_cast<size_t>(L.T), 64);
+  if (!tmap_2d(&p.tb0, c.dldense, E64, 2 * Tpad, E64, 64, 64)) return cudaErrorInvalidValue;
+  p.ta1 = p.ta0;
+  p.tb1 = p.tb0;
+  p.outf = dW_r;
+  p.T = static_cast<int>(L.T);
+  p.E = L.E;
+  p.splits = 1;
+  const int tiles = (L.d / 128) * ((L.E + 255) / 256);
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  return launch_gemm(G_ROUTER_WGRAD, p, grid, st);
 }
 
 #define MOE_TRY(x)                                   \
@@ -512,7 +535,7 @@ moe_status moe_bwd(const moe_shape* s, const void* X, const void* W_r, const voi
   }
   // 10. router backward: dl, then dW_r (sparse X^T dl); W_r^T for the dX router term
   MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st); }));
-  MOE_TRY(timed(K_DWR, st, [&] { return launch_dwr(L, c, static_cast<const __nv_bfloat16*>(X), dW_r, st); }));
+  MOE_TRY(timed(K_DWR, st, [&] { return launch_router_wgrad(L, c, X, dW_r, status, st); }));
   MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] { return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st); }));
   // 11. dgrad of gate/up
   {
@@ -733,7 +756,7 @@ moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
     MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm(G_DGRAD_DOWN, p, grid, st); }));
   }
   MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st); }));
-  MOE_TRY(timed(K_DWR, st, [&] { return launch_dwr(L, c, static_cast<const __nv_bfloat16*>(X), dW_r, st); }));
+  MOE_TRY(timed(K_DWR, st, [&] { return launch_router_wgrad(L, c, X, dW_r, status, st); }));
   MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
     return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
   }));
@@ -980,7 +1003,7 @@ moe_status moe_bwd_mx(const moe_shape* s, const void* X, const void* W_r, const 
     MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm_mx(MX_DGRAD_DOWN, p, grid, st); }));
   }
   MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st, L.I / mx_bn(MX_DGRAD_DOWN)); }));
-  MOE_TRY(timed(K_DWR, st, [&] { return launch_dwr(L, c, static_cast<const __nv_bfloat16*>(X), dW_r, st); }));
+  MOE_TRY(timed(K_DWR, st, [&] { return launch_router_wgrad(L, c, X, dW_r, status, st); }));
   MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
     return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
   }));

@@ -65,7 +65,7 @@ struct Layout {
   size_t hdr, ids, gates, counts, offsets, poff, perm_tok, perm_asg, slot_row, row_asg, row_gate, xperm, abuf,
       bbuf, stab, xq, xqs, ctx_bytes;
   // ws
-  size_t hist, logits, rpart, hbuf, obuf, dyperm, dabuf, dbbuf, hgbuf, dgpart, dlasg, wrt, dxperm, acc32, hq, hqs, dyq,
+  size_t hist, logits, rpart, hbuf, obuf, dyperm, dabuf, dbbuf, hgbuf, dgpart, dlasg, dldense, wrt, dxperm, acc32, hq, hqs, dyq,
       dyqs, daq, daqs, dbq, dbqs, ws_bytes;
   bool mx;  // MXFP8 mode
   // prepared MXFP8 weights (moe_prepare_weights): fp8 codes and scale chunks
@@ -87,6 +87,7 @@ enum GemmKind {
   G_WGRAD_GATEUP = 4,   // dW_gate = X_perm^T dA, dW_up = X_perm^T dB (per expert)
   G_WGRAD_DOWN = 5,     // dW_down = Hg^T dY_perm (per expert)
   G_ROUTER = 6,         // router logits partials: part[s] = X[:, Ks] . W_r[Ks, :] (fixed K split s)
+  G_ROUTER_WGRAD = 7,   // dW_r = X^T . DL_hi + X^T . DL_lo, DL = dl as a dense [T, E] matrix in two bf16 terms
 };
 
 struct GemmParams {
@@ -196,6 +197,8 @@ struct Ctx {  // typed views of ctx + ws for one shape
   float* rpart;  // router split-K partials [splits, T, E]
   __nv_bfloat16 *hbuf, *obuf, *dyperm, *dabuf, *dbbuf, *hgbuf, *wrt, *dxperm;
   float *dgpart, *dlasg;
+  __nv_bfloat16* dldense;  // [2, Tpad, E64] bf16 (Tpad, E64: T, E rounded up to 64): dl at (token, expert) as
+                           // hi and lo bf16 terms, zeros elsewhere
   float* acc32;
   StreamTables tab;
   uint8_t *xq, *xqs, *hq, *hqs, *dyq, *dyqs, *daq, *daqs, *dbq, *dbqs;  // MXFP8 operands and scales
@@ -226,7 +229,6 @@ cudaError_t launch_gather_rows_mx(const Layout& L, const Ctx& c, const __nv_bflo
                                   uint8_t* q, uint8_t* qs, cudaStream_t st);
 cudaError_t launch_transpose_wr(const Layout& L, const __nv_bfloat16* W_r, __nv_bfloat16* W_rT, cudaStream_t st);
 cudaError_t launch_rev_dispatch(const Layout& L, const Ctx& c, __nv_bfloat16* dX, cudaStream_t st);
-cudaError_t launch_dwr(const Layout& L, const Ctx& c, const __nv_bfloat16* X, float* dW_r, cudaStream_t st);
 cudaError_t launch_export_routing(const Layout& L, const Ctx& c, int32_t* counts, int32_t* offsets,
                                   int32_t* poff, int32_t* perm, cudaStream_t st);
 

@@ -106,33 +106,72 @@ __global__ void __launch_bounds__(kTokensPerBlock * 32) k_topk(const float* __re
 // histogram -> per-block bases, counts, offsets, padded offsets (one block).
 // hist[b][e] is replaced in place by the exclusive scan over b.
 // ---------------------------------------------------------------------------
+// inclusive scan across the warp
+__device__ __forceinline__ int warp_incl_scan(int x, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  return x;
+}
+// exclusive scan of one value per thread across the block (threads in order); *total gets the sum
+__device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int x = warp_incl_scan(v, lane);
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = warp_incl_scan(lane < nw ? wsum[lane] : 0, lane);
+    if (lane < nw) wsum[lane] = w;
+  }
+  __syncthreads();
+  const int r = (warp > 0 ? wsum[warp - 1] : 0) + x - v;
+  *total = wsum[nw - 1];
+  __syncthreads();  // wsum is reused by the next scan
+  return r;
+}
+
+// Column scan of the per-block histograms: hist[b][e] becomes the exclusive prefix over blocks
+// b' < b (each token block's base inside expert e), counts[e] the total.  One thread per expert
+// (a warp reads 32 consecutive experts of a row), eight rows' loads in flight; then the expert
+// offsets and the padded offsets of the local experts by block-wide scans.
 __global__ void __launch_bounds__(1024) k_scan(int* __restrict__ hist, int nblk, int E, int first, int El,
                                                int* __restrict__ counts, int* __restrict__ offsets,
                                                int* __restrict__ poff, int* __restrict__ hdr) {
   __shared__ int sc[kMaxE];
+  __shared__ int wsum[32];
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int run = 0;
-    for (int b = 0; b < nblk; ++b) {
-      const int h = hist[static_cast<size_t>(b) * E + e];
-      hist[static_cast<size_t>(b) * E + e] = run;
-      run += h;
+    for (int b0 = 0; b0 < nblk; b0 += 8) {
+      int h[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) h[j] = b0 + j < nblk ? hist[static_cast<size_t>(b0 + j) * E + e] : 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (b0 + j < nblk) hist[static_cast<size_t>(b0 + j) * E + e] = run;
+        run += h[j];
+      }
     }
     counts[e] = run;
     sc[e] = run;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int e = 0; e < E; ++e) { offsets[e] = run; run += sc[e]; }
-    offsets[E] = run;
-    int prun = 0;
-    for (int el = 0; el < El; ++el) {
-      poff[el] = prun;
-      prun += (sc[first + el] + kPad - 1) / kPad * kPad;
-    }
-    poff[El] = prun;
-    hdr[HDR_ROWS_P] = prun;
-    hdr[HDR_MTILES] = prun / kPad;
+  // E <= kMaxE <= blockDim: one expert per thread
+  const int e = threadIdx.x;
+  const int c = e < E ? sc[e] : 0;
+  int total = 0;
+  const int off = block_excl_scan(c, wsum, &total);
+  if (e < E) offsets[e] = off;
+  if (e == 0) offsets[E] = total;
+  const bool local = e >= first && e < first + El;
+  const int padded = local ? (c + kPad - 1) / kPad * kPad : 0;
+  const int poffe = block_excl_scan(padded, wsum, &total);  // local experts are contiguous in e
+  if (local) poff[e - first] = poffe;
+  if (e == 0) {
+    poff[El] = total;
+    hdr[HDR_ROWS_P] = total;
+    hdr[HDR_MTILES] = total / kPad;
   }
 }
 
@@ -283,11 +322,20 @@ __global__ void __launch_bounds__(128) k_combine(const __nv_bfloat16* __restrict
 //   dg_j = sum over n-tiles of the dgrad epilogue's partials (fixed order)
 //   dl_j = g_j (dg_j - sum_m g_m dg_m)
 // ---------------------------------------------------------------------------
+// dl of each token's k assignments; also the token's rows of the dense dl matrix, the router
+// weight gradient's B operand, as two bf16 terms: hi = bf16(dl) in row t, lo = bf16(dl - hi) in
+// row Tpad + t (zeros elsewhere), so the tensor cores see dl to about 16 bits.  Warps of tokens
+// in [T, Tpad) write the zero rows that pad K to a multiple of 64.
 __global__ void __launch_bounds__(256) k_router_bwd(const float* __restrict__ dgpart, const int* __restrict__ slot_row,
-                                                    const float* __restrict__ gates, int T, int k, int ntn,
-                                                    float* __restrict__ dlasg) {
+                                                    const float* __restrict__ gates, const int* __restrict__ ids, int T,
+                                                    int Tpad, int k, int ntn, int E64, float* __restrict__ dlasg,
+                                                    __nv_bfloat16* __restrict__ dldense) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
+  if (t >= Tpad) return;
+  uint4* hi_row = reinterpret_cast<uint4*>(dldense + static_cast<size_t>(t) * E64);
+  uint4* lo_row = reinterpret_cast<uint4*>(dldense + (static_cast<size_t>(Tpad) + t) * E64);
+  for (int i = lane; i < E64 / 8; i += 32) hi_row[i] = lo_row[i] = make_uint4(0, 0, 0, 0);
   if (t >= T) return;
   float dg = 0.f, g = 0.f;
   if (lane < k) {
@@ -300,7 +348,16 @@ __global__ void __launch_bounds__(256) k_router_bwd(const float* __restrict__ dg
   float s = 0.f;
   const float gd = g * dg;
   for (int j = 0; j < k; ++j) s += __shfl_sync(0xffffffffu, gd, j);
-  if (lane < k) dlasg[static_cast<size_t>(t) * k + lane] = g * (dg - s);
+  const float dl = g * (dg - s);
+  __syncwarp();  // the zero rows are written before the k entries
+  if (lane < k) {
+    const size_t a = static_cast<size_t>(t) * k + lane;
+    dlasg[a] = dl;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(dl);
+    const int e = ids[a];
+    dldense[static_cast<size_t>(t) * E64 + e] = hi;
+    dldense[(static_cast<size_t>(Tpad) + t) * E64 + e] = __float2bfloat16_rn(dl - __bfloat162float(hi));
+  }
 }
 
 // W_r [d, E] -> W_r^T [E, d] (bf16), 32 x 32 tiles
@@ -369,57 +426,7 @@ __global__ void __launch_bounds__(128) k_rev_dispatch(const __nv_bfloat16* __res
   }
 }
 
-// ---------------------------------------------------------------------------
-// dW_r[:, e] = sum over the assignments (t, j) routed to e, in the table's
-// order (ascending t), of dl_tj X[t, :].  dl has k nonzeros per token, so this
-// is the sparse form of X^T dl.  Block = (expert, 256 columns of d); its four
-// warps take fixed quarters of the expert's assignment list, each lane eight
-// columns, and the quarters are added in warp order: the result does not
-// depend on scheduling.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void axpy8(float w, const uint4& x, float (&acc)[8]) {
-  float2 f;
-  f = unpack_bf16(x.x); acc[0] = fmaf(w, f.x, acc[0]); acc[1] = fmaf(w, f.y, acc[1]);
-  f = unpack_bf16(x.y); acc[2] = fmaf(w, f.x, acc[2]); acc[3] = fmaf(w, f.y, acc[3]);
-  f = unpack_bf16(x.z); acc[4] = fmaf(w, f.x, acc[4]); acc[5] = fmaf(w, f.y, acc[5]);
-  f = unpack_bf16(x.w); acc[6] = fmaf(w, f.x, acc[6]); acc[7] = fmaf(w, f.y, acc[7]);
-}
 
-__global__ void __launch_bounds__(128) k_dwr(const __nv_bfloat16* __restrict__ X, const int* __restrict__ offsets,
-                                             const int* __restrict__ perm_asg, const float* __restrict__ dlasg,
-                                             int d, int E, int k, float* __restrict__ dWr) {
-  __shared__ float part[4][256];
-  const int e = blockIdx.x, i0 = blockIdx.y * 256;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int u0 = offsets[e], n = offsets[e + 1] - u0;
-  const int q0 = u0 + (n * warp) / 4, q1 = u0 + (n * (warp + 1)) / 4;
-  const int col = i0 + lane * 8;
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  int u = q0;
-  for (; u + 4 <= q1; u += 4) {  // four independent rows in flight
-    int a[4];
-    float w[4];
-    uint4 x[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) a[j] = __ldg(perm_asg + u + j);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      w[j] = __ldg(dlasg + a[j]);
-      x[j] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(a[j] / k) * d + col));
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) axpy8(w[j], x[j], acc);
-  }
-  for (; u < q1; ++u) {
-    const int a = __ldg(perm_asg + u);
-    axpy8(__ldg(dlasg + a), __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(a / k) * d + col)), acc);
-  }
-#pragma unroll
-  for (int q = 0; q < 8; ++q) part[warp][lane * 8 + q] = acc[q];
-  __syncthreads();
-  for (int c = threadIdx.x; c < 256; c += blockDim.x)
-    dWr[static_cast<size_t>(i0 + c) * E + e] = ((part[0][c] + part[1][c]) + part[2][c]) + part[3][c];
-}
 
 // ---------------------------------------------------------------------------
 // Ring-streamed layer planner (one thread; M minibatches, El local experts).
@@ -683,9 +690,12 @@ cudaError_t launch_finish_acc(const Layout& L, const Ctx& c, __nv_bfloat16* dW_g
 }
 cudaError_t launch_router_bwd(const Layout& L, const Ctx& c, cudaStream_t st, int n_tiles_i) {
   // n_tiles_i: dg partials per row = n-tiles of the dgrad-down GEMM (I / 256 bf16, I / 128 MXFP8)
-  k_router_bwd<<<static_cast<unsigned>((L.T + 7) / 8), 256, 0, st>>>(c.dgpart, c.slot_row, c.gates,
-                                                                       static_cast<int>(L.T), L.k,
-                                                                       n_tiles_i ? n_tiles_i : L.I / 256, c.dlasg);
+  const int E64 = (L.E + 63) / 64 * 64;
+  const int Tpad = static_cast<int>((L.T + 63) / 64 * 64);
+  k_router_bwd<<<static_cast<unsigned>(Tpad / 8), 256, 0, st>>>(c.dgpart, c.slot_row, c.gates, c.ids,
+                                                                 static_cast<int>(L.T), Tpad, L.k,
+                                                                 n_tiles_i ? n_tiles_i : L.I / 256, E64, c.dlasg,
+                                                                 c.dldense);
   return cudaGetLastError();
 }
 cudaError_t launch_transpose_wr(const Layout& L, const __nv_bfloat16* W_r, __nv_bfloat16* W_rT, cudaStream_t st) {
@@ -696,10 +706,6 @@ cudaError_t launch_transpose_wr(const Layout& L, const __nv_bfloat16* W_r, __nv_
 cudaError_t launch_rev_dispatch(const Layout& L, const Ctx& c, __nv_bfloat16* dX, cudaStream_t st) {
   k_rev_dispatch<<<static_cast<unsigned>(L.T), 128, 0, st>>>(c.dxperm, c.slot_row, c.ids, c.dlasg, c.wrt, L.k, L.d,
                                                               dX);
-  return cudaGetLastError();
-}
-cudaError_t launch_dwr(const Layout& L, const Ctx& c, const __nv_bfloat16* X, float* dW_r, cudaStream_t st) {
-  k_dwr<<<dim3(L.E, L.d / 256), 128, 0, st>>>(X, c.offsets, c.perm_asg, c.dlasg, L.d, L.E, L.k, dW_r);
   return cudaGetLastError();
 }
 cudaError_t launch_export_routing(const Layout& L, const Ctx& c, int32_t* counts, int32_t* offsets, int32_t* poff,
