@@ -148,6 +148,43 @@ def test_results_do_not_depend_on_stale_ctx_and_workspace_contents():
                            b.view(torch.int16) if b.dtype == torch.bfloat16 else b.view(torch.int32)), n
 
 
+def test_cuda_graph_replay_matches_direct_launches():
+    # moe_fwd + moe_bwd only enqueue work (no host synchronisation, no allocation), so one step
+    # can be captured as a CUDA graph; its replays must give the direct launches' bits.
+    T, d, E, k, I = 300, 512, 8, 2, 512
+    w, x = make_case(T, d, E, k, I, seed=10)
+    lay = B.MoELayer(T, d, E, I, k)
+    Y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    g = dict(dX=torch.empty(T, d, dtype=torch.bfloat16, device="cuda"),
+             dW_gate=torch.empty(E, d, I, dtype=torch.bfloat16, device="cuda"),
+             dW_up=torch.empty(E, d, I, dtype=torch.bfloat16, device="cuda"),
+             dW_down=torch.empty(E, I, d, dtype=torch.bfloat16, device="cuda"),
+             dW_r=torch.empty(d, E, dtype=torch.float32, device="cuda"))
+
+    def step():
+        lay.forward(x["X"], x["W_r"], x["bias"], x["W_gate"], x["W_up"], x["W_down"], Y=Y)
+        lay.backward(x["X"], x["W_r"], x["W_gate"], x["W_up"], x["W_down"], x["dY"], out=g)
+
+    step()
+    torch.cuda.synchronize()
+    ref = (Y.clone(), {n: t.clone() for n, t in g.items()})
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for n in g:
+        g[n].zero_()
+    Y.zero_()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert lay.error() == B.MOE_OK
+    assert torch.equal(Y.view(torch.int16), ref[0].view(torch.int16))
+    for n in g:
+        a, b = g[n], ref[1][n]
+        assert torch.equal(a.view(torch.int16) if a.dtype == torch.bfloat16 else a.view(torch.int32),
+                           b.view(torch.int16) if b.dtype == torch.bfloat16 else b.view(torch.int32)), n
+
+
 def test_nonfinite_logit_sets_status():
     T, d, E, k, I = 32, 256, 8, 2, 256
     w, x = make_case(T, d, E, k, I, seed=8)
