@@ -245,7 +245,7 @@ static int num_sms() {
 // ---------------------------------------------------------------------------
 enum KernelId {
   K_ROUTER_LOGITS, K_TOPK, K_SCAN, K_SCATTER, K_DISPATCH, K_GEMM_GATEUP, K_GEMM_DOWN, K_COMBINE,
-  K_REV_COMBINE, K_GEMM_DGRAD_DOWN, K_ROUTER_BWD, K_DWR, K_TRANSPOSE_WR, K_GEMM_DGRAD_GATEUP, K_REV_DISPATCH,
+  K_REV_COMBINE, K_GEMM_DGRAD_DOWN, K_ROUTER_BWD, K_ROUTER_WGRAD, K_TRANSPOSE_WR, K_GEMM_DGRAD_GATEUP, K_REV_DISPATCH,
   K_GEMM_WGRAD_GATEUP, K_GEMM_WGRAD_DOWN, K_PLAN, K_REPLAY, K_FINISH_ACC, K_QUANT_WEIGHTS, K_MARK_ROWS, K_NUM
 };
 static const char* kKernelNames[K_NUM] = {
@@ -533,9 +533,9 @@ moe_status moe_bwd(const moe_shape* s, const void* X, const void* W_r, const voi
     p.outf = c.dgpart;
     MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm(G_DGRAD_DOWN, p, grid, st); }));
   }
-  // 10. router backward: dl, then dW_r (sparse X^T dl); W_r^T for the dX router term
+  // 10. router backward: dl, then dW_r = X^T DL (tensor cores); W_r^T for the dX router term
   MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st); }));
-  MOE_TRY(timed(K_DWR, st, [&] { return launch_router_wgrad(L, c, X, dW_r, status, st); }));
+  MOE_TRY(timed(K_ROUTER_WGRAD, st, [&] { return launch_router_wgrad(L, c, X, dW_r, status, st); }));
   MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] { return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st); }));
   // 11. dgrad of gate/up
   {
@@ -756,7 +756,7 @@ moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
     MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm(G_DGRAD_DOWN, p, grid, st); }));
   }
   MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st); }));
-  MOE_TRY(timed(K_DWR, st, [&] { return launch_router_wgrad(L, c, X, dW_r, status, st); }));
+  MOE_TRY(timed(K_ROUTER_WGRAD, st, [&] { return launch_router_wgrad(L, c, X, dW_r, status, st); }));
   MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
     return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
   }));
@@ -1003,7 +1003,7 @@ moe_status moe_bwd_mx(const moe_shape* s, const void* X, const void* W_r, const 
     MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm_mx(MX_DGRAD_DOWN, p, grid, st); }));
   }
   MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st, L.I / mx_bn(MX_DGRAD_DOWN)); }));
-  MOE_TRY(timed(K_DWR, st, [&] { return launch_router_wgrad(L, c, X, dW_r, status, st); }));
+  MOE_TRY(timed(K_ROUTER_WGRAD, st, [&] { return launch_router_wgrad(L, c, X, dW_r, status, st); }));
   MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
     return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
   }));
