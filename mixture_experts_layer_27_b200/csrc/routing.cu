@@ -33,6 +33,8 @@ __device__ __forceinline__ unsigned long long order_key(float v, int e) {
 
 // The router GEMM leaves `splits` fp32 partial sums per logit (fixed K ranges);
 // they are added here in split order, then the bias, and the logit is stored.
+// NQ = logits per lane (E <= 32 NQ); the loads of one split are all in flight together.
+template <int NQ>
 __global__ void __launch_bounds__(kTokensPerBlock * 32) k_topk(const float* __restrict__ part, int splits,
                                                                const float* __restrict__ bias,
                                                                float* __restrict__ logits, int T, int E, int k,
@@ -46,30 +48,40 @@ __global__ void __launch_bounds__(kTokensPerBlock * 32) k_topk(const float* __re
   if (t < T) {
     float* row = logits + static_cast<size_t>(t) * E;
     const size_t plane = static_cast<size_t>(T) * E;
-    unsigned long long key[kMaxE / 32];
+    const float* pp = part + static_cast<size_t>(t) * E;
+    float v[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      const int e = lane + 32 * q;
+      v[q] = e < E ? pp[e] : 0.f;
+    }
+    for (int sp = 1; sp < splits; ++sp) {
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const int e = lane + 32 * q;
+        if (e < E) v[q] += pp[sp * plane + e];
+      }
+    }
+    unsigned long long key[NQ];
     bool bad = false;
 #pragma unroll
-    for (int q = 0; q < kMaxE / 32; ++q) {
+    for (int q = 0; q < NQ; ++q) {
       const int e = lane + 32 * q;
       key[q] = 0ull;
       if (e < E) {
-        const float* pp = part + static_cast<size_t>(t) * E + e;
-        float v = pp[0];
-        for (int s = 1; s < splits; ++s) v += pp[s * plane];
-        if (bias) v += bias[e];
-        row[e] = v;
-        bad |= !isfinite(v);
-        key[q] = order_key(v, e);
+        if (bias) v[q] += bias[e];
+        row[e] = v[q];
+        bad |= !isfinite(v[q]);
+        key[q] = order_key(v[q], e);
       }
     }
-    __syncwarp();
     int my_e = 0;
     float my_v = 0.f;
     for (int j = 0; j < k; ++j) {
       unsigned long long best = 0ull;
       int bq = -1;
 #pragma unroll
-      for (int q = 0; q < kMaxE / 32; ++q)
+      for (int q = 0; q < NQ; ++q)
         if (key[q] > best) { best = key[q]; bq = q; }
       unsigned long long wb = best;
 #pragma unroll
@@ -80,10 +92,14 @@ __global__ void __launch_bounds__(kTokensPerBlock * 32) k_topk(const float* __re
       const int e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(wb & 0xFFFFFFFFull));
       if (bq >= 0 && best == wb) {  // the owning lane removes the winner (ids are unique)
 #pragma unroll
-        for (int q = 0; q < kMaxE / 32; ++q)
+        for (int q = 0; q < NQ; ++q)
           if (q == bq) key[q] = 0ull;
       }
-      if (lane == j) { my_e = e; my_v = row[e]; }
+      if (lane == j) {  // the winner's logit, back from its key (-0 comes back as +0)
+        const uint32_t ord = static_cast<uint32_t>(wb >> 32);
+        my_e = e;
+        my_v = __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
+      }
     }
     // softmax over the selected logits; the first selected is the largest
     const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
@@ -134,7 +150,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
 
 // Column scan of the per-block histograms: hist[b][e] becomes the exclusive prefix over blocks
 // b' < b (each token block's base inside expert e), counts[e] the total.  One thread per expert
-// (a warp reads 32 consecutive experts of a row), eight rows' loads in flight; then the expert
+// (a warp reads 32 consecutive experts of a row), sixteen rows' loads in flight; then the expert
 // offsets and the padded offsets of the local experts by block-wide scans.
 __global__ void __launch_bounds__(1024) k_scan(int* __restrict__ hist, int nblk, int E, int first, int El,
                                                int* __restrict__ counts, int* __restrict__ offsets,
@@ -143,12 +159,12 @@ __global__ void __launch_bounds__(1024) k_scan(int* __restrict__ hist, int nblk,
   __shared__ int wsum[32];
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int run = 0;
-    for (int b0 = 0; b0 < nblk; b0 += 8) {
-      int h[8];
+    for (int b0 = 0; b0 < nblk; b0 += 16) {
+      int h[16];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) h[j] = b0 + j < nblk ? hist[static_cast<size_t>(b0 + j) * E + e] : 0;
+      for (int j = 0; j < 16; ++j) h[j] = b0 + j < nblk ? hist[static_cast<size_t>(b0 + j) * E + e] : 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < 16; ++j) {
         if (b0 + j < nblk) hist[static_cast<size_t>(b0 + j) * E + e] = run;
         run += h[j];
       }
@@ -374,6 +390,37 @@ __global__ void __launch_bounds__(256) k_transpose_wr(const __nv_bfloat16* __res
   for (int r = ty; r < 32; r += 8) {
     const int e = e0 + r, i = i0 + tx;
     if (i < d && e < E) WrT[static_cast<size_t>(e) * d + i] = tile[tx][r];
+  }
+}
+// The same for E a multiple of 8, with 16-byte global accesses: 64 (d) x 64 (E) tiles; each
+// thread loads two 8-element vectors and stores two, through a tile with an odd row pitch (65
+// elements) so that both the row-wise writes and the column-wise reads spread over the banks.
+__global__ void __launch_bounds__(256) k_transpose_wr_v(const __nv_bfloat16* __restrict__ Wr, int d, int E,
+                                                        __nv_bfloat16* __restrict__ WrT) {
+  __shared__ __nv_bfloat16 tile[64][65];  // [i][e]
+  const int i0 = blockIdx.y * 64, e0 = blockIdx.x * 64;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int c = threadIdx.x + h * 256;  // 512 chunks: row i (64) x chunk (8 elements of e)
+    const int r = c >> 3, ch = c & 7;
+    const int e = e0 + ch * 8;
+    __align__(16) __nv_bfloat16 v[8];
+    *reinterpret_cast<uint4*>(v) = e < E ? __ldg(reinterpret_cast<const uint4*>(Wr + static_cast<size_t>(i0 + r) * E + e))
+                                         : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) tile[r][ch * 8 + j] = v[j];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int c = threadIdx.x + h * 256;  // 512 chunks: row e (64) x chunk (8 elements of i)
+    const int r = c >> 3, ch = c & 7;
+    const int e = e0 + r;
+    if (e >= E) continue;
+    __align__(16) __nv_bfloat16 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = tile[ch * 8 + j][r];
+    *reinterpret_cast<uint4*>(WrT + static_cast<size_t>(e) * d + i0 + ch * 8) = *reinterpret_cast<const uint4*>(v);
   }
 }
 
@@ -628,8 +675,19 @@ __global__ void k_export_routing(const int* __restrict__ counts, const int* __re
 // launchers
 // ---------------------------------------------------------------------------
 cudaError_t launch_topk(const Layout& L, const Ctx& c, const float* bias, int splits, cudaStream_t st) {
-  k_topk<<<L.nblk, kTokensPerBlock * 32, 0, st>>>(c.rpart, splits, bias, c.logits, static_cast<int>(L.T), L.E, L.k,
-                                                  c.ids, c.gates, c.hist, c.hdr + HDR_STATUS);
+  const int T = static_cast<int>(L.T);
+  if (L.E <= 128)
+    k_topk<4><<<L.nblk, kTokensPerBlock * 32, 0, st>>>(c.rpart, splits, bias, c.logits, T, L.E, L.k, c.ids, c.gates,
+                                                       c.hist, c.hdr + HDR_STATUS);
+  else if (L.E <= 256)
+    k_topk<8><<<L.nblk, kTokensPerBlock * 32, 0, st>>>(c.rpart, splits, bias, c.logits, T, L.E, L.k, c.ids, c.gates,
+                                                       c.hist, c.hdr + HDR_STATUS);
+  else if (L.E <= 384)
+    k_topk<12><<<L.nblk, kTokensPerBlock * 32, 0, st>>>(c.rpart, splits, bias, c.logits, T, L.E, L.k, c.ids,
+                                                        c.gates, c.hist, c.hdr + HDR_STATUS);
+  else
+    k_topk<kMaxE / 32><<<L.nblk, kTokensPerBlock * 32, 0, st>>>(c.rpart, splits, bias, c.logits, T, L.E, L.k, c.ids,
+                                                                c.gates, c.hist, c.hdr + HDR_STATUS);
   return cudaGetLastError();
 }
 cudaError_t launch_scan(const Layout& L, const Ctx& c, cudaStream_t st) {
@@ -699,8 +757,12 @@ cudaError_t launch_router_bwd(const Layout& L, const Ctx& c, cudaStream_t st, in
   return cudaGetLastError();
 }
 cudaError_t launch_transpose_wr(const Layout& L, const __nv_bfloat16* W_r, __nv_bfloat16* W_rT, cudaStream_t st) {
-  dim3 grid((L.E + 31) / 32, (L.d + 31) / 32);
-  k_transpose_wr<<<grid, 256, 0, st>>>(W_r, L.d, L.E, W_rT);
+  if (L.E % 8 == 0 && L.d % 64 == 0) {
+    k_transpose_wr_v<<<dim3((L.E + 63) / 64, L.d / 64), 256, 0, st>>>(W_r, L.d, L.E, W_rT);
+  } else {
+    dim3 grid((L.E + 31) / 32, (L.d + 31) / 32);
+    k_transpose_wr<<<grid, 256, 0, st>>>(W_r, L.d, L.E, W_rT);
+  }
   return cudaGetLastError();
 }
 cudaError_t launch_rev_dispatch(const Layout& L, const Ctx& c, __nv_bfloat16* dX, cudaStream_t st) {
