@@ -113,7 +113,7 @@ __device__ __forceinline__ Tile decode(const GemmParams& p, int t) {
     tl.el = sp;  // the split index rides in the expert slot
     tl.m0 = mt * 128;
     tl.nt = nt;
-    tl.n0 = nt * 256;
+    tl.n0 = nt * p.router_bn;
     tl.kb0 = sp * KB / S;
     tl.nk = (sp + 1) * KB / S - tl.kb0;
     return tl;
@@ -366,14 +366,14 @@ __device__ __forceinline__ void epilogue_row(const GemmParams& p, const Tile& tl
     const int t = tl.m0 + row;
     float* dst = p.outf + (static_cast<size_t>(tl.el) * p.T + t) * p.E;
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < p.router_bn / 32 + (p.router_bn % 32 != 0); ++c) {
       float v[32];
       tmem_ld32(taddr + c * 32, v);  // every lane loads (warp-collective), then masks
       const int e0 = tl.n0 + c * 32;
       if (t < p.T) {
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          if (e0 + i < p.E) dst[e0 + i] = v[i];
+          if (c * 32 + i < p.router_bn && e0 + i < p.E) dst[e0 + i] = v[i];  // this tile's columns only
       }
     }
   }
@@ -642,7 +642,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
                                                    : sdesc_sw128(a0 + kk * 32, 16, 1024);
             const uint64_t bd = Traits<KIND>::B_MN ? sdesc_sw128(b0 + kk * 2048, 8192, 1024)
                                                    : sdesc_sw128(b0 + kk * 32, 16, 1024);
-            umma_bf16(dtm, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            umma_bf16(dtm, ad, bd, KIND == G_ROUTER ? idesc_bf16(GEMM_BM, p.router_bn, false, false) : IDESC,
+                      (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
           if (++stage == STAGES) { stage = 0; phase ^= 1; }

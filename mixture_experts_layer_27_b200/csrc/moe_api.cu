@@ -413,6 +413,7 @@ static moe_status route_tokens(const Layout& L, const Ctx& c, const void* X, con
     p.T = static_cast<int>(L.T);
     p.E = L.E;
     p.splits = splits;
+    p.router_bn = router_tile_n(L.E);
     p.outf = c.rpart;
     const int64_t tiles = ((L.T + 127) / 128) * ((L.E + 255) / 256) * splits;
     const int g = static_cast<int>(tiles < grid ? tiles : grid);

@@ -116,6 +116,7 @@ struct GemmParams {
   float* outf;
   int El, d, I;
   int T, E, splits;           // router GEMM: tokens, experts, K splits
+  int router_bn;              // router GEMM: experts per n-tile (E split evenly over ceil(E / 256) tiles)
   int* status;
 };
 
@@ -125,6 +126,9 @@ constexpr size_t GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;
 constexpr size_t GEMM_B_BYTES = GEMM_BN * GEMM_BK * 2;
 constexpr size_t GEMM_STAGE_BYTES = GEMM_A_BYTES + GEMM_B_BYTES;
 constexpr size_t GEMM_STAGE_OUT_BYTES = 4 * 32 * 256 * 2;  // wgrad: one 32 x 256 bf16 slice per epilogue warp
+// experts per n-tile of the router GEMM: E split evenly over ceil(E / 256) tiles, rounded up to
+// the MMA's N granule (16), so that E = 384 runs as two 192-wide tiles instead of 256 + 128
+constexpr int router_tile_n(int E) { return ((E + (E + 255) / 256 - 1) / ((E + 255) / 256) + 15) / 16 * 16; }
 constexpr int router_splits(int64_t T, int E, int d) {  // K splits of the router GEMM (about one wave)
   const int64_t tiles = ((T + 127) / 128) * ((E + 255) / 256);
   int64_t s = tiles > 0 ? 148 / tiles : 1;

@@ -132,6 +132,7 @@ extern "C" moe_status moe_route_static(const moe_shape* shape, const void* X, co
   p.T = static_cast<int>(L.T);
   p.E = L.E;
   p.splits = splits;
+  p.router_bn = router_tile_n(L.E);
   p.outf = c.rpart;
   p.status = status;
   int dev = 0, sms = 148;
