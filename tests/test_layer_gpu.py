@@ -77,6 +77,10 @@ def test_k_equals_E():
     _check_layer(64, 256, 4, 4, 256, seed=3)
 
 
+def test_top_k_16_the_largest_supported():
+    _check_layer(96, 256, 32, 16, 256, seed=11)
+
+
 def test_single_expert():
     _check_layer(100, 256, 1, 1, 256, seed=4)
 
