@@ -133,3 +133,52 @@ def test_mxfp8_results_do_not_depend_on_stale_ctx_and_workspace_contents():
     for n in ("dX", "dW_gate", "dW_up", "dW_down"):
         assert torch.equal(g0[n].view(torch.int16), g1[n].view(torch.int16)), n
     assert torch.equal(g0["dW_r"].view(torch.int32), g1["dW_r"].view(torch.int32))
+
+
+def _run_mx(x, T, d, E, k, I, first=0, num=0):
+    El = num or E - first
+    lay = B.MoELayerMX(T, d, E, I, k, first_local_expert=first, num_local_experts=num)
+    lay.prepare(x["W_gate"][first:first + El].contiguous(), x["W_up"][first:first + El].contiguous(),
+                x["W_down"][first:first + El].contiguous())
+    Y = lay.forward(x["X"], x["W_r"], x["bias"])
+    g = lay.backward(x["X"], x["W_r"], x["dY"])
+    torch.cuda.synchronize()
+    assert lay.error() == B.MOE_OK
+    return Y, g
+
+
+def test_mxfp8_local_expert_slices():
+    # A rank's slice computes its experts exactly as the full layer does (the router is the
+    # full router, so routing and every expert's rows are the same); the slices' outputs add
+    # up to the full layer's.
+    T, d, E, k, I = 200, 256, 16, 4, 256
+    w, x = make_case(T, d, E, k, I, seed=46)
+    Yf, gf = _run_mx(x, T, d, E, k, I)
+    Y0, g0 = _run_mx(x, T, d, E, k, I, first=0, num=7)
+    Y1, g1 = _run_mx(x, T, d, E, k, I, first=7, num=9)
+    for n in ("dW_gate", "dW_up", "dW_down"):
+        assert torch.equal(g0[n].view(torch.int16), gf[n][:7].view(torch.int16)), n
+        assert torch.equal(g1[n].view(torch.int16), gf[n][7:].view(torch.int16)), n
+    assert relerr(to64(Y0) + to64(Y1), to64(Yf)) <= 1e-2
+    assert relerr(to64(g0["dX"]) + to64(g1["dX"]), to64(gf["dX"])) <= 1e-2
+    assert relerr(to64(g0["dW_r"]) + to64(g1["dW_r"]), to64(gf["dW_r"])) <= 1e-2
+
+
+def test_mxfp8_no_tokens():
+    T, d, E, k, I = 0, 256, 4, 2, 256
+    lay = B.MoELayerMX(T, d, E, I, k)
+    W = {n: torch.randn(*s, device="cuda").to(torch.bfloat16) for n, s in
+         dict(W_r=(d, E), W_gate=(E, d, I), W_up=(E, d, I), W_down=(E, I, d)).items()}
+    lay.prepare(W["W_gate"], W["W_up"], W["W_down"])
+    X0 = torch.empty(0, d, device="cuda", dtype=torch.bfloat16)
+    lay.forward(X0, W["W_r"], None, Y=torch.empty(0, d, device="cuda", dtype=torch.bfloat16))
+    g = lay.backward(X0, W["W_r"], X0,
+                     out=dict(dX=torch.empty(0, d, device="cuda", dtype=torch.bfloat16),
+                              dW_gate=torch.full((E, d, I), 7.0, device="cuda", dtype=torch.bfloat16),
+                              dW_up=torch.full((E, d, I), 7.0, device="cuda", dtype=torch.bfloat16),
+                              dW_down=torch.full((E, I, d), 7.0, device="cuda", dtype=torch.bfloat16),
+                              dW_r=torch.full((d, E), 7.0, device="cuda")))
+    torch.cuda.synchronize()
+    assert lay.error() == B.MOE_OK
+    for n in ("dW_gate", "dW_up", "dW_down", "dW_r"):
+        assert torch.count_nonzero(g[n]) == 0, n
