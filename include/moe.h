@@ -136,6 +136,17 @@ moe_status moe_debug_logits(const moe_shape* shape, const void* ws, float* logit
  * the only nonzeros of dL/dlogits (dW_r = X^T dl scattered to the ids). */
 moe_status moe_debug_router_grad(const moe_shape* shape, const void* ws, float* dl, void* stream);
 
+/* Test hook for the device-side failure path (no counterpart on the pages):
+ * clears ctx's status word, then launches one kernel on `stream` whose mbarrier
+ * wait is never satisfied.  The wait is the same bounded wait every GEMM role
+ * uses: it gives up after its spin limit (about 2 s), records
+ * MOE_ERR_DEVICE_TIMEOUT in ctx's status word and the kernel returns, so the
+ * context stays usable; moe_get_error then reports (and clears) the status.
+ * ctx as sized by moe_ctx_size(shape).  Returns MOE_ERR_INVALID_ARG for a NULL
+ * or misaligned ctx, MOE_ERR_WORKSPACE_TOO_SMALL for a short one, MOE_ERR_CUDA
+ * if the launch fails. */
+moe_status moe_debug_bounded_wait(const moe_shape* shape, void* ctx, size_t ctx_bytes, void* stream);
+
 /* Benchmark support (no counterpart on the pages).  When enabled, every
  * kernel launch of the library is bracketed by two CUDA events recorded on the
  * launch stream.  moe_profile_read synchronises the device, writes per kernel

@@ -1092,6 +1092,19 @@ moe_status moe_debug_router_grad(const moe_shape* s, const void* ws, float* dl, 
   return MOE_OK;
 }
 
+moe_status moe_debug_bounded_wait(const moe_shape* s, void* ctx, size_t ctx_bytes, void* stream) {
+  Layout L;
+  const moe_status cs = check_shape(s, &L);
+  if (cs != MOE_OK) return cs;
+  if (!ctx || !aligned16(ctx)) return MOE_ERR_INVALID_ARG;
+  if (ctx_bytes < L.ctx_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  const Ctx c = make_ctx(L, ctx, nullptr);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_TRY(cudaMemsetAsync(c.hdr + HDR_STATUS, 0, 4, st));  // a clear status word: the wait must run out
+  MOE_TRY(launch_wait_probe(c.hdr + HDR_STATUS, st));
+  return MOE_OK;
+}
+
 moe_status moe_debug_logits(const moe_shape* s, const void* ws, float* logits, void* stream) {
   Layout L;
   const moe_status cs = check_shape(s, &L);

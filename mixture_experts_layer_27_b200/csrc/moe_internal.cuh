@@ -213,6 +213,7 @@ cudaError_t launch_topk(const Layout& L, const Ctx& c, const float* bias, int sp
 cudaError_t launch_scan(const Layout& L, const Ctx& c, cudaStream_t st);
 cudaError_t launch_scatter(const Layout& L, const Ctx& c, cudaStream_t st);
 cudaError_t launch_mark_rows(const Layout& L, const Ctx& c, cudaStream_t st);
+cudaError_t launch_wait_probe(int* status, cudaStream_t st);
 cudaError_t launch_gather_rows(const Layout& L, const Ctx& c, const __nv_bfloat16* src, __nv_bfloat16* dst,
                                cudaStream_t st);
 // rows [*lo, *hi) to dst row + *shift (streamed layer)

@@ -702,6 +702,19 @@ cudaError_t launch_scatter(const Layout& L, const Ctx& c, cudaStream_t st) {
                                    c.perm_asg, c.slot_row, c.row_asg, c.row_gate);
   return cudaGetLastError();
 }
+// One thread waits on an mbarrier that nothing arrives at: the bounded wait gives up and
+// records MOE_ERR_DEVICE_TIMEOUT in *status (the failure path of every GEMM role).
+__global__ void k_wait_probe(int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  mbar_wait(&bar, 0, status);
+}
+cudaError_t launch_wait_probe(int* status, cudaStream_t st) {
+  k_wait_probe<<<1, 32, 0, st>>>(status);
+  return cudaGetLastError();
+}
 cudaError_t launch_mark_rows(const Layout& L, const Ctx& c, cudaStream_t st) {
   const bool mb = L.M > 0;
   const int nseg = mb ? L.M * L.El : L.El;

@@ -189,6 +189,22 @@ def test_cuda_graph_replay_matches_direct_launches():
                            b.view(torch.int16) if b.dtype == torch.bfloat16 else b.view(torch.int32)), n
 
 
+def test_bounded_wait_gives_up_records_timeout_and_the_context_stays_usable():
+    # An mbarrier nothing arrives at: the GEMM roles' bounded wait gives up (about 2 s),
+    # records MOE_ERR_DEVICE_TIMEOUT in ctx's status word and the kernel returns.
+    T, d, E, k, I = 64, 256, 4, 2, 256
+    w, x = make_case(T, d, E, k, I, seed=12)
+    lay = B.MoELayer(T, d, E, I, k)
+    assert B.moe_debug_bounded_wait(lay.shape, lay.ctx) == B.MOE_OK
+    torch.cuda.synchronize()
+    assert lay.error() == B.MOE_ERR_DEVICE_TIMEOUT
+    assert lay.error() == B.MOE_OK  # reading the status clears it
+    _, Y, g, st = run_gpu(x, T, d, E, k, I, layer=lay)  # the context still runs the layer
+    assert st == B.MOE_OK
+    Yo, ctx, go = run_oracle(x, k)
+    assert relerr(to64(Y), Yo) <= TOL_BF16 and relerr(to64(g["dX"]), go["dX"]) <= TOL_BF16
+
+
 def test_nonfinite_logit_sets_status():
     T, d, E, k, I = 32, 256, 8, 2, 256
     w, x = make_case(T, d, E, k, I, seed=8)
