@@ -347,13 +347,20 @@ def dist_setup(n_gpus: int):
     return world, rank, local
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def max_over_ranks(v: float, world: int, device="cuda") -> float:
+    """The largest of the ranks' values (the job's time is its slowest rank's)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: float, seconds: float, world: int) -> float:
+    """Whole-job rate: every rank's units over the slowest rank's time (weak scaling: each rank
+    runs the layer on its own tokens, so the per-rank work is fixed as ranks are added)."""
+    return units_per_rank * world / seconds
 
 
 def barrier(world: int):
@@ -565,7 +572,7 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
         return
     tokens = NT * args.steps * world
     flops = w.model_flops() * args.steps * world
-    value = tokens / t
+    value = job_throughput(NT * args.steps, t, world)
     tflops = flops / t / 1e12
     per_gpu_tflops = tflops / world
     algo = algorithmic_bytes(w)
@@ -617,7 +624,7 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
         "tflops": tflops, "pct_of_bf16_peak": 100.0 * per_gpu_tflops / bf16,
         "peak_note": f"bf16 sustained {bf16} TFLOP/s ({peak_kind}); model FLOPs 18 d I T k + 6 T d E per step",
         "roofline": roof,
-        "e2e": {"value": tokens / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": 2 * NT * w.d * 2,
+        "e2e": {"value": job_throughput(NT * args.steps, t_e2e, world), "unit": "tokens/s", "h2d_bytes_per_step": 2 * NT * w.d * 2,
                 "d2h_bytes_per_step": 2 * NT * w.d * 2,
                 "note": "X, dY copied in from pinned host memory; Y, dX copied back; weights and their gradients "
                         "stay in HBM; the step between the copies is the same launch mode as the timed region"},
