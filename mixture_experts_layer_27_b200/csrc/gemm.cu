@@ -410,25 +410,30 @@ __device__ __forceinline__ void epilogue_wgrad(const GemmParams& p, const Tile& 
   // (bf16) or half a tile (fp32) earlier has been read: all but the 3 newest groups.  So the
   // TMA engine drains box b while the warp converts box b+1.
   if (mode == 0) {
-#pragma unroll 1
-    for (int b = 0; b < 4; ++b) {  // 64 bf16 columns per box
-      float v[64];
-      if (tl.nk > 0) {
-        tmem_ld64(taddr + b * 64, v);
-      } else {
+    // TMEM loads pipelined one box ahead: box b+1's load is in flight while box b is converted
+    uint32_t r[2][64];
+    const bool any = tl.nk > 0;  // an expert without tokens has a zero gradient
+    if (any) {
+      tmem_ld64_issue(taddr, r[0]);
+      tmem_ld64_wait(r[0]);
+    } else {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) v[i] = 0.f;  // expert without tokens: zero gradient
-      }
+      for (int i = 0; i < 64; ++i) r[0][i] = r[1][i] = 0u;
+    }
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {  // 64 bf16 columns per box
+      if (any && b < 3) tmem_ld64_issue(taddr + (b + 1) * 64, r[(b + 1) & 1]);
+      const uint32_t (&w)[64] = r[b & 1];
       if (lane == 0) bulk_wait_read<3>();
       __syncwarp();
       uint8_t* box = stage_out + b * 4096;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         uint4 u;
-        u.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
-        u.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
-        u.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
-        u.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+        u.x = pack_bf16(__uint_as_float(w[8 * q + 0]), __uint_as_float(w[8 * q + 1]));
+        u.y = pack_bf16(__uint_as_float(w[8 * q + 2]), __uint_as_float(w[8 * q + 3]));
+        u.z = pack_bf16(__uint_as_float(w[8 * q + 4]), __uint_as_float(w[8 * q + 5]));
+        u.w = pack_bf16(__uint_as_float(w[8 * q + 6]), __uint_as_float(w[8 * q + 7]));
         stage_chunk16(box, lane, q, u);
       }
       fence_proxy_async();
@@ -437,6 +442,7 @@ __device__ __forceinline__ void epilogue_wgrad(const GemmParams& p, const Tile& 
         tma_store_2d(up ? &p.to1 : &p.to0, box, x0 + b * 64, y0);
         bulk_commit();
       }
+      if (any && b < 3) tmem_ld64_wait(r[(b + 1) & 1]);
     }
     return;
   }
