@@ -186,7 +186,7 @@ def algorithmic_bytes(w: IN.Workload) -> dict:
 # A figure is reported only while the GEMM sources still hash to the value they had
 # when the counters were taken.
 NCU_TRAFFIC = {
-    ("gemm_wgrad_gateup", "dsv3"): (914.1e6 * 16, "7aa19e4df7ecf527"),
+    ("gemm_wgrad_gateup", "dsv3"): (913.5e6 * 16, "5bd9e115a8aa58b6"),
 }
 GEMM_SOURCES = ("gemm.cu", "ptx.cuh", "moe_internal.cuh")
 
