@@ -305,6 +305,13 @@ class MoELayerMX:
     def logits(self):
         return MoELayer.logits(self)
 
+    def router_grad(self):
+        # the ws regions before the MXFP8-only ones sit where the bf16 layout puts them
+        import torch
+        out = torch.empty(self.T, self.k, dtype=torch.float32, device=self.ws.device)
+        check(moe_debug_router_grad(self.shape_bf16, self.ws, out), "moe_debug_router_grad")
+        return out
+
     def error(self, stream=None) -> int:
         return moe_get_error(self.ctx, stream)
 
