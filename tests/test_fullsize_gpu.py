@@ -207,3 +207,65 @@ def test_full_size_mxfp8_kimi():
     assert torch.equal(g["dW_r"].view(torch.int32), g2["dW_r"].view(torch.int32))
     del lay2, Y, Y2, g, g2, x
     torch.cuda.empty_cache()
+
+
+def test_full_size_ep64_ring_stream():
+    # Config 5 at n = 4096 tokens per local expert: 16 minibatches of 2048 tokens through the
+    # 256 MiB ring, 6 local experts of 384; the backward replays part of the stream into the
+    # ring and accumulates the gate/up weight gradient over two chunks.
+    w = IN.WORKLOADS["ep64_n4096"]
+    x = IN.make_inputs(w, device="cuda")
+    first, El = w.first_local, w.El
+
+    def run():
+        s = B.MoEStream(w.T, w.d, w.E, w.I, w.k, w.stream_M, w.ring_bytes, first, w.num_local)
+        Y = s.forward(x["X"], x["W_r"], x["bias"], x["W_gate"], x["W_up"], x["W_down"])
+        g = s.backward(x["X"], x["W_r"], x["W_gate"], x["W_up"], x["W_down"], x["dY"])
+        torch.cuda.synchronize()
+        assert s.error() == B.MOE_OK
+        return s, Y, g
+
+    s, Y, g = run()
+    hdr = s.plan()["plan"]
+    assert hdr[1] > 1 and hdr[3] > 0  # several backward chunks, replayed rows
+
+    X, Wr, b, dY = to64(x["X"]), to64(x["W_r"]), to64(x["bias"]), to64(x["dY"])
+    caches = {n: ExpertCache(x[n]) for n in ("W_gate", "W_up", "W_down")}
+    Wg, Wu, Wd = (lambda e, c=caches[n]: c(e - first) for n in ("W_gate", "W_up", "W_down"))
+
+    # Y and dX at sampled tokens, some with local experts and some without; near-ties in the
+    # fp64 logits are skipped (their selection may differ between fp32 and fp64)
+    rng = np.random.default_rng(99)
+    cand = rng.choice(w.tokens, size=64, replace=False)
+    lg = O.router_logits(X[cand], Wr, b)
+    srt = -np.sort(-lg, axis=1)
+    ok = (srt[:, w.k - 1] - srt[:, w.k]) > 1e-3
+    ids = O.topk_ids(lg, w.k)
+    has_local = np.any((ids >= first) & (ids < first + El), axis=1)
+    pick = [int(t) for t, o, h in zip(cand, ok, has_local) if o and h][:5] + \
+           [int(t) for t, o, h in zip(cand, ok, has_local) if o and not h][:2]
+    assert len(pick) >= 5
+    Yg, dXg = to64(Y), to64(g["dX"])
+    ys, yo, dxs, dxo = [], [], [], []
+    for t in pick:
+        y, dx, _, _, _ = O.token_forward_backward(t, X, Wr, b, Wg, Wu, Wd, w.k, dY, first_local=first,
+                                                  num_local=El)
+        ys.append(Yg[t]); yo.append(y); dxs.append(dXg[t]); dxo.append(dx)
+    assert relerr(np.array(ys), np.array(yo)) <= TOL_BF16
+    assert relerr(np.array(dxs), np.array(dxo)) <= TOL_BF16
+
+    # weight gradients of two local experts over the whole stream (the gate/up one accumulated
+    # over the backward chunks in fp32)
+    for el in (0, El - 1):
+        e = first + el
+        _, ctx = O.forward(X, Wr, b, Wg, Wu, Wd, w.k, first_local=e, num_local=1)
+        go = O.backward(ctx, dY)
+        for n in ("dW_gate", "dW_up", "dW_down"):
+            assert relerr(to64(g[n][el]), go[n][e]) <= TOL_BF16, (n, e)
+
+    # a second run is bit-identical
+    _, Y2, g2 = run()
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+    for n in ("dX", "dW_gate", "dW_up", "dW_down"):
+        assert torch.equal(g[n].view(torch.int16), g2[n].view(torch.int16)), n
+    assert torch.equal(g["dW_r"].view(torch.int32), g2["dW_r"].view(torch.int32))
