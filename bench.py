@@ -141,10 +141,11 @@ def algorithmic_flops(w: IN.Workload) -> dict:
 # algorithmic bytes per launch of each kernel (minimum HBM traffic of its job)
 # rows = T*k routed assignments; weights of all local experts; bf16 = 2 bytes
 # ----------------------------------------------------------------------------
-def algorithmic_bytes(w: IN.Workload) -> dict:
+def algorithmic_bytes(w: IN.Workload, wgrad_elem_bytes: int = 2) -> dict:
     T, d, E, I, k, El = w.tokens, w.d, w.E, w.I, w.k, w.El
     rows = local_rows(w)
     W1 = El * d * I * 2  # one expert weight matrix family (gate, up or down), bytes
+    G1 = El * d * I * wgrad_elem_bytes  # its gradient (bf16, or fp32 with --wgrad-fp32)
     if w.mxfp8:
         # fp8 operands carry one scale byte per 32 values; outputs stay bf16 (H, dA, dB also as fp8)
         Wq = El * d * I * 33 // 32
@@ -161,8 +162,8 @@ def algorithmic_bytes(w: IN.Workload) -> dict:
             "router_wgrad": T * d * 2 + T * k * 8 + d * E * 4,
             "gemm_dgrad_gateup": 2 * Wq + 2 * rows * I * 33 // 32 + rows * d * 2,
             "reverse_dispatch": rows * d * 2 + T * d * 2 + E * d * 2,
-            "gemm_wgrad_gateup": rows * d * 2 + 2 * rows * I * 2 + 2 * W1,
-            "gemm_wgrad_down": rows * I * 2 + rows * d * 2 + W1,
+            "gemm_wgrad_gateup": rows * d * 2 + 2 * rows * I * 2 + 2 * G1,
+            "gemm_wgrad_down": rows * I * 2 + rows * d * 2 + G1,
         }
     return {
         "router_logits": T * d * 2 + d * E * 2 + T * E * 4,
@@ -182,11 +183,11 @@ def algorithmic_bytes(w: IN.Workload) -> dict:
 
 
 # DRAM bytes per launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum),
-# scaled to the workload by the units processed; see profiles/ncu_gemm_gateup_wgrad_dsv3_e16.md.
+# scaled to the workload by the units processed; see profiles/ncu_traffic_gemm_wgrad_gateup_dsv3_e16.md.
 # A figure is reported only while the GEMM sources still hash to the value they had
 # when the counters were taken.
 NCU_TRAFFIC = {
-    ("gemm_wgrad_gateup", "dsv3"): (913.5e6 * 16, "5bd9e115a8aa58b6"),
+    ("gemm_wgrad_gateup", "dsv3"): (913.28e6 * 16, "7e6aac1090f2baec"),
 }
 GEMM_SOURCES = ("gemm.cu", "ptx.cuh", "moe_internal.cuh")
 
@@ -402,18 +403,19 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     torch.cuda.set_device(dev)
     peaks, peak_kind = load_peaks()
     x = IN.make_inputs(w, device=dev)
+    wdt = torch.float32 if args.wgrad_fp32 else torch.bfloat16
     if w.mxfp8:
-        layer = B.MoELayerMX(w.T, w.d, w.E, w.I, w.k, device=dev)
+        layer = B.MoELayerMX(w.T, w.d, w.E, w.I, w.k, device=dev, wgrad_dtype=wdt)
     elif w.stream_M:
         layer = B.MoEStream(w.T, w.d, w.E, w.I, w.k, w.stream_M, w.ring_bytes, w.first_local, w.num_local,
-                            device=dev)
+                            device=dev, wgrad_dtype=wdt)
     else:
-        layer = B.MoELayer(w.T, w.d, w.E, w.I, w.k, device=dev)
+        layer = B.MoELayer(w.T, w.d, w.E, w.I, w.k, device=dev, wgrad_dtype=wdt)
     NT = w.tokens
     Y = torch.empty(NT, w.d, dtype=torch.bfloat16, device=dev)
     grads = dict(dX=torch.empty(NT, w.d, dtype=torch.bfloat16, device=dev),
-                 dW_gate=torch.empty_like(x["W_gate"]), dW_up=torch.empty_like(x["W_up"]),
-                 dW_down=torch.empty_like(x["W_down"]),
+                 dW_gate=torch.empty_like(x["W_gate"], dtype=wdt), dW_up=torch.empty_like(x["W_up"], dtype=wdt),
+                 dW_down=torch.empty_like(x["W_down"], dtype=wdt),
                  dW_r=torch.empty(w.d, w.E, dtype=torch.float32, device=dev))
     stream = torch.cuda.current_stream(dev)
 
@@ -605,7 +607,8 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     value = job_throughput(NT * args.steps, t, world)
     tflops = flops / t / 1e12
     per_gpu_tflops = tflops / world
-    algo = algorithmic_bytes(w)
+    algo = algorithmic_bytes(w, 4 if args.wgrad_fp32 else 2)
+    traffic_key = w.name + ("+wgrad_fp32" if args.wgrad_fp32 else "")  # counters were taken with bf16 gradients
     aflops = algorithmic_flops(w)
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     bf16 = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -633,24 +636,24 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     if kern[top]["bound"] == "tensor" and kern[top].get("tensor_peak") == "mxfp8":
         ach = kern[top]["achieved_TFLOPs"]
         roof = {"kernel": top, "bound": "tensor", "achieved": ach, "peak": fp8, "unit": "TFLOP/s",
-                "frac": ach / fp8, "traffic": ncu_traffic(top, w.name),
+                "frac": ach / fp8, "traffic": ncu_traffic(top, traffic_key),
                 "peak_source": "measured sustained MXFP8 cuBLAS GEMM in this run (" + fp8_peak["how"] + ")"}
     elif kern[top]["bound"] == "tensor":
         ach = kern[top]["achieved_TFLOPs"]
         roof = {"kernel": top, "bound": "tensor", "achieved": ach, "peak": bf16, "unit": "TFLOP/s",
-                "frac": ach / bf16, "traffic": ncu_traffic(top, w.name),
+                "frac": ach / bf16, "traffic": ncu_traffic(top, traffic_key),
                 "peak_source": f"{peak_kind} sustained bf16 GEMM (MEASURED_PEAKS.json bf16_tflops_sustained)"}
     else:
         ach = kern[top].get("achieved_GBs")
         roof = {"kernel": top, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
-                "frac": (ach / hbm) if ach else None, "traffic": ncu_traffic(top, w.name),
+                "frac": (ach / hbm) if ach else None, "traffic": ncu_traffic(top, traffic_key),
                 "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s"}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, random-init weights)",
-        "config": workload_config(w),
+        "config": dict(workload_config(w), wgrad_dtype="fp32" if args.wgrad_fp32 else "bf16"),
         "tflops": tflops, "pct_of_bf16_peak": 100.0 * per_gpu_tflops / bf16,
         "peak_note": f"bf16 sustained {bf16} TFLOP/s ({peak_kind}); model FLOPs 18 d I T k + 6 T d E per step",
         "roofline": roof,
@@ -692,6 +695,8 @@ def main():
     ap.add_argument("--impl", default="moe", choices=["moe", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time direct launches instead of a CUDA graph of one step")
+    ap.add_argument("--wgrad-fp32", action="store_true",
+                    help="write the expert weight gradients as fp32 instead of bf16 (the weights' dtype)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -59,9 +59,18 @@ typedef enum moe_precision {
                     use moe_prepare_weights + moe_fwd_mx / moe_bwd_mx (moe_fwd / moe_bwd refuse it) */
 } moe_precision;
 
+typedef enum moe_wgrad_dtype {
+  MOE_WGRAD_BF16 = 0,  /* dW_gate / dW_up / dW_down in bf16, the weights' type (round to nearest even
+                          of the fp32 sum) */
+  MOE_WGRAD_FP32 = 1   /* the same fp32 sums, unrounded: for optimisers that keep fp32 gradients */
+} moe_wgrad_dtype;
+
 /* Layer shape.  Experts [first_local_expert, first_local_expert + num_local_experts)
  * are computed here (num_local_experts = 0 means all E).  Assignments to other
- * experts belong to another rank: they add nothing to Y or to the expert part of dX. */
+ * experts belong to another rank: they add nothing to Y or to the expert part of dX.
+ * wgrad_dtype (moe_wgrad_dtype) is the element type of the expert weight gradients
+ * that moe_bwd, moe_bwd_mx and moe_bwd_stream write; the other entry points ignore it
+ * (buffer sizes do not depend on it), and any value but 0 or 1 makes the shape invalid. */
 typedef struct moe_shape {
   int64_t T;       /* tokens */
   int32_t d;       /* model (hidden) dimension */
@@ -71,6 +80,7 @@ typedef struct moe_shape {
   int32_t prec;    /* moe_precision */
   int32_t first_local_expert;
   int32_t num_local_experts;
+  int32_t wgrad_dtype;
 } moe_shape;
 
 /* Bytes of the saved-for-backward context that moe_fwd writes and moe_bwd reads
@@ -101,7 +111,8 @@ moe_status moe_fwd(const moe_shape* shape, const void* X, const void* W_r, const
 /* Backward of the last moe_fwd that wrote `ctx` (same shape, X, W_r, weights).
  *   dY      [T, d]   bf16   upstream gradient
  *   dX      [T, d]   bf16   written
- *   dW_gate, dW_up [El, d, I] bf16, dW_down [El, I, d] bf16   written (not accumulated)
+ *   dW_gate, dW_up [El, d, I], dW_down [El, I, d]   written (not accumulated); bf16, or
+ *                    fp32 when shape->wgrad_dtype is MOE_WGRAD_FP32
  *   dW_r    [d, E]   fp32   written
  * Implements the mirror of the forward (page 1, "Three design decisions":
  * pull reverse-combine, push reverse-dispatch), grouped dgrad and wgrad with
@@ -169,7 +180,8 @@ unsigned long long moe_kernel_launches(void);
  * down GEMMs and both dgrad GEMMs run on kind::mxf8f6f4 block-scaled tensor
  * cores with both operands quantised; the two weight-gradient GEMMs contract
  * over tokens and stay bf16.  The router stays bf16, so routing is the same in
- * both modes; all outputs are bf16 (dW_r fp32).
+ * both modes; all outputs are bf16 (dW_r fp32; the expert weight gradients
+ * fp32 with wgrad_dtype = MOE_WGRAD_FP32).
  *
  * moe_prepare_weights quantises the bf16 master weights once (e.g. after each
  * optimiser step) into `wq` (moe_weights_size bytes), laid out as ten regions,
@@ -219,7 +231,8 @@ moe_status moe_bwd_mx(const moe_shape* shape, const void* X, const void* W_r, co
  * device; the host enqueues a fixed number of launches per minibatch.
  * Requirements: shape->T a multiple of 16; 1 <= M <= 256; ring_bytes at least
  * moe_stream_min_ring_bytes(shape) (one minibatch's worst case), else
- * MOE_ERR_WORKSPACE_TOO_SMALL.  bf16 only. */
+ * MOE_ERR_WORKSPACE_TOO_SMALL.  bf16 operands only (wgrad_dtype applies as in
+ * moe_bwd). */
 size_t moe_stream_ctx_size(const moe_shape* shape, int32_t num_minibatches);
 size_t moe_stream_workspace_size(const moe_shape* shape, int32_t num_minibatches);
 size_t moe_stream_min_ring_bytes(const moe_shape* shape);

@@ -21,16 +21,38 @@ MOE_ERR_DEVICE_TIMEOUT = 5
 MOE_ERR_NONFINITE = 6
 MOE_BF16 = 0
 MOE_MXFP8 = 1
+MOE_WGRAD_BF16 = 0
+MOE_WGRAD_FP32 = 1
 
 
 class moe_shape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("I", ctypes.c_int32),
                 ("top_k", ctypes.c_int32), ("prec", ctypes.c_int32), ("first_local_expert", ctypes.c_int32),
-                ("num_local_experts", ctypes.c_int32)]
+                ("num_local_experts", ctypes.c_int32), ("wgrad_dtype", ctypes.c_int32)]
 
 
-def make_shape(T, d, E, I, top_k, prec=MOE_BF16, first_local_expert=0, num_local_experts=0) -> moe_shape:
-    return moe_shape(T, d, E, I, top_k, prec, first_local_expert, num_local_experts)
+def make_shape(T, d, E, I, top_k, prec=MOE_BF16, first_local_expert=0, num_local_experts=0,
+               wgrad_dtype=MOE_WGRAD_BF16) -> moe_shape:
+    return moe_shape(T, d, E, I, top_k, prec, first_local_expert, num_local_experts, wgrad_dtype)
+
+
+def _wgrad_code(dtype) -> int:
+    """moe_wgrad_dtype of a torch dtype (bfloat16 or float32)."""
+    import torch
+    if dtype == torch.bfloat16:
+        return MOE_WGRAD_BF16
+    if dtype == torch.float32:
+        return MOE_WGRAD_FP32
+    raise ValueError(f"expert weight gradients are bfloat16 or float32, not {dtype}")
+
+
+def _grad_buffers(T, d, E, I, El, wdt, dev) -> dict:
+    import torch
+    return dict(dX=torch.empty(T, d, dtype=torch.bfloat16, device=dev),
+                dW_gate=torch.empty(El, d, I, dtype=wdt, device=dev),
+                dW_up=torch.empty(El, d, I, dtype=wdt, device=dev),
+                dW_down=torch.empty(El, I, d, dtype=wdt, device=dev),
+                dW_r=torch.empty(d, E, dtype=torch.float32, device=dev))
 
 
 class MoeError(RuntimeError):
@@ -248,9 +270,12 @@ def check(status: int, what: str = "moe"):
 class MoELayerMX:
     """MXFP8 layer: prepared (quantised) weights + ctx / workspace owner."""
 
-    def __init__(self, T, d, E, I, top_k, first_local_expert=0, num_local_experts=0, device="cuda"):
+    def __init__(self, T, d, E, I, top_k, first_local_expert=0, num_local_experts=0, device="cuda",
+                 wgrad_dtype=None):
         import torch
-        self.shape = make_shape(T, d, E, I, top_k, MOE_MXFP8, first_local_expert, num_local_experts)
+        self.wgrad_dtype = wgrad_dtype or torch.bfloat16
+        self.shape = make_shape(T, d, E, I, top_k, MOE_MXFP8, first_local_expert, num_local_experts,
+                                _wgrad_code(self.wgrad_dtype))
         self.shape_bf16 = make_shape(T, d, E, I, top_k, MOE_BF16, first_local_expert, num_local_experts)
         nc, nw, nq = moe_ctx_size(self.shape), moe_workspace_size(self.shape), moe_weights_size(self.shape)
         if nc == 0 or nw == 0 or nq == 0:
@@ -274,12 +299,7 @@ class MoELayerMX:
     def backward(self, X, W_r, dY, out=None, stream=None):
         import torch
         if out is None:
-            dev = X.device
-            out = dict(dX=torch.empty(self.T, self.d, dtype=torch.bfloat16, device=dev),
-                       dW_gate=torch.empty(self.El, self.d, self.I, dtype=torch.bfloat16, device=dev),
-                       dW_up=torch.empty(self.El, self.d, self.I, dtype=torch.bfloat16, device=dev),
-                       dW_down=torch.empty(self.El, self.I, self.d, dtype=torch.bfloat16, device=dev),
-                       dW_r=torch.empty(self.d, self.E, dtype=torch.float32, device=dev))
+            out = _grad_buffers(self.T, self.d, self.E, self.I, self.El, self.wgrad_dtype, X.device)
         check(moe_bwd_mx(self.shape, X, W_r, self.wq, dY, self.ctx, out["dX"], out["dW_gate"], out["dW_up"],
                          out["dW_down"], out["dW_r"], self.ws, stream), "moe_bwd_mx")
         return out
@@ -328,9 +348,12 @@ def unchunk_scales(chunks, R, K):
 class MoEStream:
     """ctx / ring / workspace owner for the ring-streamed layer (M minibatches of T tokens)."""
 
-    def __init__(self, T, d, E, I, top_k, M, ring_bytes, first_local_expert=0, num_local_experts=0, device="cuda"):
+    def __init__(self, T, d, E, I, top_k, M, ring_bytes, first_local_expert=0, num_local_experts=0, device="cuda",
+                 wgrad_dtype=None):
         import torch
-        self.shape = make_shape(T, d, E, I, top_k, MOE_BF16, first_local_expert, num_local_experts)
+        self.wgrad_dtype = wgrad_dtype or torch.bfloat16
+        self.shape = make_shape(T, d, E, I, top_k, MOE_BF16, first_local_expert, num_local_experts,
+                                _wgrad_code(self.wgrad_dtype))
         nc, nw = moe_stream_ctx_size(self.shape, M), moe_stream_workspace_size(self.shape, M)
         if nc == 0 or nw == 0:
             raise MoeError(MOE_ERR_UNSUPPORTED, "stream shape")
@@ -351,12 +374,7 @@ class MoEStream:
     def backward(self, X, W_r, W_gate, W_up, W_down, dY, out=None, stream=None):
         import torch
         if out is None:
-            dev = X.device
-            out = dict(dX=torch.empty(self.M * self.T, self.d, dtype=torch.bfloat16, device=dev),
-                       dW_gate=torch.empty(self.El, self.d, self.I, dtype=torch.bfloat16, device=dev),
-                       dW_up=torch.empty(self.El, self.d, self.I, dtype=torch.bfloat16, device=dev),
-                       dW_down=torch.empty(self.El, self.I, self.d, dtype=torch.bfloat16, device=dev),
-                       dW_r=torch.empty(self.d, self.E, dtype=torch.float32, device=dev))
+            out = _grad_buffers(self.M * self.T, self.d, self.E, self.I, self.El, self.wgrad_dtype, X.device)
         check(moe_bwd_stream(self.shape, self.M, X, W_r, W_gate, W_up, W_down, dY, self.ctx, out["dX"],
                              out["dW_gate"], out["dW_up"], out["dW_down"], out["dW_r"], self.ring, self.ws, stream),
               "moe_bwd_stream")
@@ -387,9 +405,11 @@ class MoELayer:
     """Convenience owner of ctx / workspace buffers (allocated by torch) for one shape."""
 
     def __init__(self, T, d, E, I, top_k, prec=MOE_BF16, first_local_expert=0, num_local_experts=0,
-                 device="cuda"):
+                 device="cuda", wgrad_dtype=None):
         import torch
-        self.shape = make_shape(T, d, E, I, top_k, prec, first_local_expert, num_local_experts)
+        self.wgrad_dtype = wgrad_dtype or torch.bfloat16
+        self.shape = make_shape(T, d, E, I, top_k, prec, first_local_expert, num_local_experts,
+                                _wgrad_code(self.wgrad_dtype))
         nc, nw = moe_ctx_size(self.shape), moe_workspace_size(self.shape)
         if nc == 0 or nw == 0:
             raise MoeError(MOE_ERR_UNSUPPORTED, "shape")
@@ -408,12 +428,7 @@ class MoELayer:
     def backward(self, X, W_r, W_gate, W_up, W_down, dY, out=None, stream=None):
         import torch
         if out is None:
-            dev = X.device
-            out = dict(dX=torch.empty(self.T, self.d, dtype=torch.bfloat16, device=dev),
-                       dW_gate=torch.empty(self.El, self.d, self.I, dtype=torch.bfloat16, device=dev),
-                       dW_up=torch.empty(self.El, self.d, self.I, dtype=torch.bfloat16, device=dev),
-                       dW_down=torch.empty(self.El, self.I, self.d, dtype=torch.bfloat16, device=dev),
-                       dW_r=torch.empty(self.d, self.E, dtype=torch.float32, device=dev))
+            out = _grad_buffers(self.T, self.d, self.E, self.I, self.El, self.wgrad_dtype, X.device)
         check(moe_bwd(self.shape, X, W_r, W_gate, W_up, W_down, dY, self.ctx, out["dX"], out["dW_gate"],
                       out["dW_up"], out["dW_down"], out["dW_r"], self.ws, stream), "moe_bwd")
         return out

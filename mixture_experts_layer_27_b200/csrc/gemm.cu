@@ -381,10 +381,10 @@ __device__ __forceinline__ void epilogue_row(const GemmParams& p, const Tile& tl
 
 // wgrad epilogue: the warp's 32 x 256 slice of the output tile.  Mode (from the chunk
 // descriptor of a ring-streamed backward; 0 otherwise):
-//   0  bf16 dW (the whole contraction was in this launch)
+//   0  dW (the whole contraction was in this launch): bf16, or fp32 when p.wout32
 //   1  fp32 partial into the accumulator (first of several chunks)
 //   2  fp32: accumulator + this chunk's partial, back into the accumulator
-// Both go through a 128B-swizzled staging buffer and out by TMA stores.
+// All go through a 128B-swizzled staging buffer and out by TMA stores.
 // Chunks run in a fixed order, so the sum is reproducible.
 __device__ __forceinline__ void stage_chunk16(uint8_t* box, int lane, int chunk, uint4 u) {
   *reinterpret_cast<uint4*>(box + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = u;
@@ -409,7 +409,7 @@ __device__ __forceinline__ void epilogue_wgrad(const GemmParams& p, const Tile& 
   // as its own bulk group, and a box slot is refilled once the store issued from it one tile
   // (bf16) or half a tile (fp32) earlier has been read: all but the 3 newest groups.  So the
   // TMA engine drains box b while the warp converts box b+1.
-  if (mode == 0) {
+  if (mode == 0 && !p.wout32) {
     // TMEM loads pipelined one box ahead: box b+1's load is in flight while box b is converted
     uint32_t r[2][64];
     const bool any = tl.nk > 0;  // an expert without tokens has a zero gradient
@@ -446,8 +446,10 @@ __device__ __forceinline__ void epilogue_wgrad(const GemmParams& p, const Tile& 
     }
     return;
   }
-  // fp32 accumulator: eight 32 x 32 fp32 boxes
-  const float* prev = p.acc32 + static_cast<size_t>(yacc + lane) * p.I + x0;
+  // fp32: eight 32 x 32 boxes, into the accumulator (modes 1, 2) or the output (mode 0)
+  const CUtensorMap* tm = mode == 0 ? (up ? &p.to1 : &p.to0) : &p.tacc;
+  const int ys = mode == 0 ? y0 : yacc;
+  const float* prev = mode == 2 ? p.acc32 + static_cast<size_t>(yacc + lane) * p.I + x0 : nullptr;
 #pragma unroll 1
   for (int j = 0; j < 8; ++j) {
     const int col = j * 32;
@@ -484,7 +486,7 @@ __device__ __forceinline__ void epilogue_wgrad(const GemmParams& p, const Tile& 
     fence_proxy_async();
     __syncwarp();
     if (lane == 0) {
-      tma_store_2d(&p.tacc, box, x0 + col, yacc);
+      tma_store_2d(tm, box, x0 + col, ys);
       bulk_commit();
     }
   }

@@ -19,6 +19,7 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   if (s.T < 0 || s.d <= 0 || s.E <= 0 || s.I <= 0 || s.top_k <= 0) return false;
   if (s.E > kMaxE || s.top_k > kMaxK || s.top_k > s.E) return false;
   if (s.d % 256 || s.I % 256) return false;
+  if (s.wgrad_dtype != MOE_WGRAD_BF16 && s.wgrad_dtype != MOE_WGRAD_FP32) return false;
   const int El = s.num_local_experts == 0 ? s.E - s.first_local_expert : s.num_local_experts;
   if (s.first_local_expert < 0 || El <= 0 || s.first_local_expert + El > s.E) return false;
   if (M < 0 || M > kMaxMinibatches) return false;
@@ -34,6 +35,7 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->k = s.top_k;
   L->first = s.first_local_expert;
   L->El = El;
+  L->w32 = s.wgrad_dtype == MOE_WGRAD_FP32;
   // a token has at most min(k, El) local assignments; every (macrobatch, expert) segment pads < 128 rows
   const int64_t A = T_all * (s.top_k < El ? s.top_k : El);
   const int64_t nseg = static_cast<int64_t>(El) * (M > 0 ? M : 1);
@@ -229,6 +231,25 @@ static bool tmap_fp8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D fp32 tensor [outer, inner] (dense rows), box {32, 32} (128-byte rows), 128-byte swizzle.
+static bool tmap_f32(CUtensorMap* m, void* base, uint64_t inner, uint64_t outer) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 4};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Output map of an expert weight gradient [outer, inner]: bf16 in 64 x 32 boxes, or fp32 in
+// 32 x 32 boxes when the layer writes the unrounded sums.
+static bool tmap_wgrad_out(const Layout& L, CUtensorMap* m, void* base, uint64_t inner, uint64_t outer) {
+  return L.w32 ? tmap_f32(m, base, inner, outer) : tmap_2d(m, base, inner, outer, inner, 64, 32);
+}
+
 static int num_sms() {
   static int n = 0;
   if (n == 0) {
@@ -309,6 +330,7 @@ static GemmParams base_params(const Layout& L, const Ctx& c, int* status) {
   p.d = L.d;
   p.I = L.I;
   p.nseg = L.El;
+  p.wout32 = L.w32 ? 1 : 0;
   p.status = status;
   return p;
 }
@@ -487,6 +509,46 @@ moe_status moe_fwd(const moe_shape* s, const void* X, const void* W_r, const flo
   return MOE_OK;
 }
 
+// Expert weight gradients from the saved X_perm and the backward's dA, dB, Hg, dY_perm:
+// gate/up, then down (write-bound; separate launches keep the HBM traffic one-directional).
+static moe_status launch_wgrads(const Layout& L, const Ctx& c, int* status, void* dW_gate, void* dW_up,
+                                void* dW_down, cudaStream_t st) {
+  const int grid = num_sms();
+  const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, c.xperm, L.d, RP, L.d, 64, 64));
+    MOE_TMAP(tmap_2d(&p.tb0, c.dabuf, L.I, RP, L.I, 64, 64));
+    MOE_TMAP(tmap_2d(&p.tb1, c.dbbuf, L.I, RP, L.I, 64, 64));
+    MOE_TMAP(tmap_wgrad_out(L, &p.to0, dW_gate, L.I, El * L.d));
+    MOE_TMAP(tmap_wgrad_out(L, &p.to1, dW_up, L.I, El * L.d));
+    p.ta1 = p.ta0;
+    MOE_TRY(timed(K_GEMM_WGRAD_GATEUP, st, [&] { return launch_gemm(G_WGRAD_GATEUP, p, grid, st); }));
+  }
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, c.hgbuf, L.I, RP, L.I, 64, 64));
+    MOE_TMAP(tmap_2d(&p.tb0, c.dyperm, L.d, RP, L.d, 64, 64));
+    MOE_TMAP(tmap_wgrad_out(L, &p.to0, dW_down, L.d, El * L.I));
+    p.to1 = p.to0;
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    MOE_TRY(timed(K_GEMM_WGRAD_DOWN, st, [&] { return launch_gemm(G_WGRAD_DOWN, p, grid, st); }));
+  }
+  return MOE_OK;
+}
+
+// Zero expert and router weight gradients (a backward with no tokens).
+static moe_status zero_wgrads(const Layout& L, void* dW_gate, void* dW_up, void* dW_down, float* dW_r,
+                              cudaStream_t st) {
+  const size_t wexp = static_cast<size_t>(L.El) * L.d * L.I * (L.w32 ? 4 : 2);
+  MOE_TRY(cudaMemsetAsync(dW_gate, 0, wexp, st));
+  MOE_TRY(cudaMemsetAsync(dW_up, 0, wexp, st));
+  MOE_TRY(cudaMemsetAsync(dW_down, 0, wexp, st));
+  MOE_TRY(cudaMemsetAsync(dW_r, 0, static_cast<size_t>(L.d) * L.E * 4, st));
+  return MOE_OK;
+}
+
 moe_status moe_bwd(const moe_shape* s, const void* X, const void* W_r, const void* W_gate, const void* W_up,
                    const void* W_down, const void* dY, void* ctx, size_t ctx_bytes, void* dX, void* dW_gate,
                    void* dW_up, void* dW_down, float* dW_r, void* ws, size_t ws_bytes, void* stream) {
@@ -504,14 +566,7 @@ moe_status moe_bwd(const moe_shape* s, const void* X, const void* W_r, const voi
   if (ctx_bytes < L.ctx_bytes || ws_bytes < L.ws_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Ctx c = make_ctx(L, ctx, ws);
-  if (L.T == 0) {  // no tokens: every gradient is zero
-    const size_t wexp = static_cast<size_t>(L.El) * L.d * L.I * 2;
-    MOE_TRY(cudaMemsetAsync(dW_gate, 0, wexp, st));
-    MOE_TRY(cudaMemsetAsync(dW_up, 0, wexp, st));
-    MOE_TRY(cudaMemsetAsync(dW_down, 0, wexp, st));
-    MOE_TRY(cudaMemsetAsync(dW_r, 0, static_cast<size_t>(L.d) * L.E * 4, st));
-    return MOE_OK;
-  }
+  if (L.T == 0) return zero_wgrads(L, dW_gate, dW_up, dW_down, dW_r, st);  // no tokens: all zero
   const int grid = num_sms();
   int* status = c.hdr + HDR_STATUS;
   const uint64_t RP = static_cast<uint64_t>(L.RP);
@@ -550,31 +605,8 @@ moe_status moe_bwd(const moe_shape* s, const void* X, const void* W_r, const voi
   }
   // 12. reverse-dispatch (+ router term dl W_r^T)
   MOE_TRY(timed(K_REV_DISPATCH, st, [&] { return launch_rev_dispatch(L, c, static_cast<__nv_bfloat16*>(dX), st); }));
-  // 13. wgrad: gate/up then down (write-bound; separate launches keep HBM traffic one-directional)
-  {
-    GemmParams p = base_params(L, c, status);
-    MOE_TMAP(tmap_2d(&p.ta0, c.xperm, L.d, RP, L.d, 64, 64));
-    MOE_TMAP(tmap_2d(&p.tb0, c.dabuf, L.I, RP, L.I, 64, 64));
-    MOE_TMAP(tmap_2d(&p.tb1, c.dbbuf, L.I, RP, L.I, 64, 64));
-    MOE_TMAP(tmap_2d(&p.to0, dW_gate, L.I, El * L.d, L.I, 64, 32));
-    MOE_TMAP(tmap_2d(&p.to1, dW_up, L.I, El * L.d, L.I, 64, 32));
-    p.ta1 = p.ta0;
-    p.out0 = static_cast<__nv_bfloat16*>(dW_gate);
-    p.out1 = static_cast<__nv_bfloat16*>(dW_up);
-    MOE_TRY(timed(K_GEMM_WGRAD_GATEUP, st, [&] { return launch_gemm(G_WGRAD_GATEUP, p, grid, st); }));
-  }
-  {
-    GemmParams p = base_params(L, c, status);
-    MOE_TMAP(tmap_2d(&p.ta0, c.hgbuf, L.I, RP, L.I, 64, 64));
-    MOE_TMAP(tmap_2d(&p.tb0, c.dyperm, L.d, RP, L.d, 64, 64));
-    MOE_TMAP(tmap_2d(&p.to0, dW_down, L.d, El * L.I, L.d, 64, 32));
-    p.to1 = p.to0;
-    p.ta1 = p.ta0;
-    p.tb1 = p.tb0;
-    p.out0 = static_cast<__nv_bfloat16*>(dW_down);
-    MOE_TRY(timed(K_GEMM_WGRAD_DOWN, st, [&] { return launch_gemm(G_WGRAD_DOWN, p, grid, st); }));
-  }
-  return MOE_OK;
+  // 13. wgrad
+  return launch_wgrads(L, c, status, dW_gate, dW_up, dW_down, st);
 }
 
 moe_status moe_profile_enable(int on) {
@@ -781,11 +813,10 @@ moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
     p.nseg = nseg;
     MOE_TMAP(tmap_2d(&p.ta0, c.hgbuf, L.I, RP, L.I, 64, 64));
     MOE_TMAP(tmap_2d(&p.tb0, c.dyperm, L.d, RP, L.d, 64, 64));
-    MOE_TMAP(tmap_2d(&p.to0, dW_down, L.d, El * L.I, L.d, 64, 32));
+    MOE_TMAP(tmap_wgrad_out(L, &p.to0, dW_down, L.d, El * L.I));
     p.to1 = p.to0;
     p.ta1 = p.ta0;
     p.tb1 = p.tb0;
-    p.out0 = static_cast<__nv_bfloat16*>(dW_down);
     MOE_TRY(timed(K_GEMM_WGRAD_DOWN, st, [&] { return launch_gemm(G_WGRAD_DOWN, p, grid, st); }));
   }
   // wgrad of W_gate / W_up needs X_perm: walk the ring in reverse, chunk by chunk
@@ -799,23 +830,10 @@ moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
     MOE_TMAP(tmap_2d(&p.ta0, ring, L.d, static_cast<uint64_t>(ring_rows), L.d, 64, 64));
     MOE_TMAP(tmap_2d(&p.tb0, c.dabuf, L.I, RP, L.I, 64, 64));
     MOE_TMAP(tmap_2d(&p.tb1, c.dbbuf, L.I, RP, L.I, 64, 64));
-    MOE_TMAP(tmap_2d(&p.to0, dW_gate, L.I, El * L.d, L.I, 64, 32));
-    MOE_TMAP(tmap_2d(&p.to1, dW_up, L.I, El * L.d, L.I, 64, 32));
-    {  // fp32 accumulator [2 * El * d, I], 32 x 32 boxes (128-byte rows)
-      EncodeTiledFn enc = get_encode();
-      if (!enc) return MOE_ERR_CUDA;
-      const cuuint64_t dims[2] = {static_cast<cuuint64_t>(L.I), 2 * El * static_cast<cuuint64_t>(L.d)};
-      const cuuint64_t strides[1] = {static_cast<cuuint64_t>(L.I) * 4};
-      const cuuint32_t box[2] = {32, 32};
-      const cuuint32_t estr[2] = {1, 1};
-      if (enc(&p.tacc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, c.acc32, dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return MOE_ERR_CUDA;
-    }
+    MOE_TMAP(tmap_wgrad_out(L, &p.to0, dW_gate, L.I, El * L.d));
+    MOE_TMAP(tmap_wgrad_out(L, &p.to1, dW_up, L.I, El * L.d));
+    MOE_TMAP(tmap_f32(&p.tacc, c.acc32, L.I, 2 * El * L.d));  // fp32 accumulator [2 * El * d, I]
     p.ta1 = p.ta0;
-    p.out0 = static_cast<__nv_bfloat16*>(dW_gate);
-    p.out1 = static_cast<__nv_bfloat16*>(dW_up);
     for (int ch = 0; ch < L.M; ++ch) {
       MOE_TRY(timed(K_REPLAY, st, [&] {
         return launch_replay(L, c, ch, static_cast<const __nv_bfloat16*>(X), static_cast<__nv_bfloat16*>(ring),
@@ -825,9 +843,7 @@ moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
       MOE_TRY(timed(K_GEMM_WGRAD_GATEUP, st, [&] { return launch_gemm(G_WGRAD_GATEUP, p, grid, st); }));
     }
   }
-  MOE_TRY(timed(K_FINISH_ACC, st, [&] {
-    return launch_finish_acc(L, c, static_cast<__nv_bfloat16*>(dW_gate), static_cast<__nv_bfloat16*>(dW_up), st);
-  }));
+  MOE_TRY(timed(K_FINISH_ACC, st, [&] { return launch_finish_acc(L, c, dW_gate, dW_up, st); }));
   return MOE_OK;
 }
 
@@ -968,14 +984,7 @@ moe_status moe_bwd_mx(const moe_shape* s, const void* X, const void* W_r, const 
   if (ctx_bytes < L.ctx_bytes || ws_bytes < L.ws_bytes || wq_bytes < L.wq_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Ctx c = make_ctx(L, ctx, ws);
-  if (L.T == 0) {
-    const size_t wexp = static_cast<size_t>(L.El) * L.d * L.I * 2;
-    MOE_TRY(cudaMemsetAsync(dW_gate, 0, wexp, st));
-    MOE_TRY(cudaMemsetAsync(dW_up, 0, wexp, st));
-    MOE_TRY(cudaMemsetAsync(dW_down, 0, wexp, st));
-    MOE_TRY(cudaMemsetAsync(dW_r, 0, static_cast<size_t>(L.d) * L.E * 4, st));
-    return MOE_OK;
-  }
+  if (L.T == 0) return zero_wgrads(L, dW_gate, dW_up, dW_down, dW_r, st);
   const int grid = num_sms();
   int* status = c.hdr + HDR_STATUS;
   const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
@@ -1022,31 +1031,8 @@ moe_status moe_bwd_mx(const moe_shape* s, const void* X, const void* W_r, const 
     MOE_TRY(timed(K_GEMM_DGRAD_GATEUP, st, [&] { return launch_gemm_mx(MX_DGRAD_GATEUP, p, grid, st); }));
   }
   MOE_TRY(timed(K_REV_DISPATCH, st, [&] { return launch_rev_dispatch(L, c, static_cast<__nv_bfloat16*>(dX), st); }));
-  // weight gradients contract over tokens and are written in bf16: the bf16 engine
-  {
-    GemmParams p = base_params(L, c, status);
-    MOE_TMAP(tmap_2d(&p.ta0, c.xperm, L.d, RP, L.d, 64, 64));
-    MOE_TMAP(tmap_2d(&p.tb0, c.dabuf, L.I, RP, L.I, 64, 64));
-    MOE_TMAP(tmap_2d(&p.tb1, c.dbbuf, L.I, RP, L.I, 64, 64));
-    MOE_TMAP(tmap_2d(&p.to0, dW_gate, L.I, El * L.d, L.I, 64, 32));
-    MOE_TMAP(tmap_2d(&p.to1, dW_up, L.I, El * L.d, L.I, 64, 32));
-    p.ta1 = p.ta0;
-    p.out0 = static_cast<__nv_bfloat16*>(dW_gate);
-    p.out1 = static_cast<__nv_bfloat16*>(dW_up);
-    MOE_TRY(timed(K_GEMM_WGRAD_GATEUP, st, [&] { return launch_gemm(G_WGRAD_GATEUP, p, grid, st); }));
-  }
-  {
-    GemmParams p = base_params(L, c, status);
-    MOE_TMAP(tmap_2d(&p.ta0, c.hgbuf, L.I, RP, L.I, 64, 64));
-    MOE_TMAP(tmap_2d(&p.tb0, c.dyperm, L.d, RP, L.d, 64, 64));
-    MOE_TMAP(tmap_2d(&p.to0, dW_down, L.d, El * L.I, L.d, 64, 32));
-    p.to1 = p.to0;
-    p.ta1 = p.ta0;
-    p.tb1 = p.tb0;
-    p.out0 = static_cast<__nv_bfloat16*>(dW_down);
-    MOE_TRY(timed(K_GEMM_WGRAD_DOWN, st, [&] { return launch_gemm(G_WGRAD_DOWN, p, grid, st); }));
-  }
-  return MOE_OK;
+  // weight gradients contract over tokens from the bf16 operands: the bf16 engine
+  return launch_wgrads(L, c, status, dW_gate, dW_up, dW_down, st);
 }
 
 moe_status moe_get_error(void* ctx, void* stream) {

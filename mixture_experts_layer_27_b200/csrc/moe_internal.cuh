@@ -67,7 +67,8 @@ struct Layout {
   // ws
   size_t hist, logits, rpart, hbuf, obuf, dyperm, dabuf, dbbuf, hgbuf, dgpart, dlasg, dldense, wrt, dxperm, acc32, hq, hqs, dyq,
       dyqs, daq, daqs, dbq, dbqs, ws_bytes;
-  bool mx;  // MXFP8 mode
+  bool mx;   // MXFP8 mode
+  bool w32;  // expert weight gradients written as fp32
   // prepared MXFP8 weights (moe_prepare_weights): fp8 codes and scale chunks
   size_t wgu1, wgu1s, wd2, wd2s, wd3, wd3s, wg4, wg4s, wu4, wu4s, wq_bytes;
 };
@@ -117,6 +118,7 @@ struct GemmParams {
   int El, d, I;
   int T, E, splits;           // router GEMM: tokens, experts, K splits
   int router_bn;              // router GEMM: experts per n-tile (E split evenly over ceil(E / 256) tiles)
+  int wout32;                 // wgrad: to0 / to1 are fp32 maps (32 x 32 boxes) and take the unrounded sums
   int* status;
 };
 
@@ -224,8 +226,8 @@ cudaError_t launch_combine(const Layout& L, const Ctx& c, const __nv_bfloat16* O
 cudaError_t launch_plan(const Layout& L, const Ctx& c, int ring_rows, int min_rows, cudaStream_t st);
 cudaError_t launch_replay(const Layout& L, const Ctx& c, int chunk, const __nv_bfloat16* X, __nv_bfloat16* ring,
                           int64_t ring_rows, cudaStream_t st);
-cudaError_t launch_finish_acc(const Layout& L, const Ctx& c, __nv_bfloat16* dW_gate, __nv_bfloat16* dW_up,
-                              cudaStream_t st);
+// the fp32 gate/up accumulator into dW_gate / dW_up (bf16, or fp32 when L.w32)
+cudaError_t launch_finish_acc(const Layout& L, const Ctx& c, void* dW_gate, void* dW_up, cudaStream_t st);
 cudaError_t launch_router_bwd(const Layout& L, const Ctx& c, cudaStream_t st, int n_tiles_i = 0);
 // MXFP8 quantisation, see quant.cu
 cudaError_t launch_quant_weight(int mode, const __nv_bfloat16* src0, const __nv_bfloat16* src1, int64_t R_out, int K,

@@ -641,19 +641,23 @@ __global__ void __launch_bounds__(128) k_replay(const __nv_bfloat16* __restrict_
 }
 
 // dW_gate / dW_up (bf16) from the fp32 accumulator when the backward used several chunks.
+__device__ __forceinline__ void store4(__nv_bfloat16* dst, float4 v) {
+  uint2 u;
+  u.x = pack_bf16(v.x, v.y);
+  u.y = pack_bf16(v.z, v.w);
+  *reinterpret_cast<uint2*>(dst) = u;
+}
+__device__ __forceinline__ void store4(float* dst, float4 v) { *reinterpret_cast<float4*>(dst) = v; }
+
+template <typename OutT>
 __global__ void __launch_bounds__(256) k_finish_acc(const float* __restrict__ acc, const int* __restrict__ plan,
-                                                    size_t n_each, __nv_bfloat16* __restrict__ dWg,
-                                                    __nv_bfloat16* __restrict__ dWu) {
-  if (plan[PLAN_N_CHUNKS] <= 1) return;  // the wgrad epilogue already wrote bf16
+                                                    size_t n_each, OutT* __restrict__ dWg, OutT* __restrict__ dWu) {
+  if (plan[PLAN_N_CHUNKS] <= 1) return;  // the wgrad epilogue already wrote the gradients
   const size_t n4 = n_each / 4;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < 2 * n4;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const float4 v = reinterpret_cast<const float4*>(acc)[i];
-    __nv_bfloat16* dst = i < n4 ? dWg + 4 * i : dWu + 4 * (i - n4);
-    uint2 u;
-    u.x = pack_bf16(v.x, v.y);
-    u.y = pack_bf16(v.z, v.w);
-    *reinterpret_cast<uint2*>(dst) = u;
+    store4(i < n4 ? dWg + 4 * i : dWu + 4 * (i - n4), v);
   }
 }
 
@@ -753,10 +757,14 @@ cudaError_t launch_replay(const Layout& L, const Ctx& c, int chunk, const __nv_b
   k_replay<<<grid, 128, 0, st>>>(X, c.row_asg, c.tab, L.El, chunk, L.k, L.d, ring);
   return cudaGetLastError();
 }
-cudaError_t launch_finish_acc(const Layout& L, const Ctx& c, __nv_bfloat16* dW_gate, __nv_bfloat16* dW_up,
-                              cudaStream_t st) {
+cudaError_t launch_finish_acc(const Layout& L, const Ctx& c, void* dW_gate, void* dW_up, cudaStream_t st) {
   const size_t n_each = static_cast<size_t>(L.El) * L.d * L.I;
-  k_finish_acc<<<148 * 8, 256, 0, st>>>(c.acc32, c.tab.plan, n_each, dW_gate, dW_up);
+  if (L.w32)
+    k_finish_acc<<<148 * 8, 256, 0, st>>>(c.acc32, c.tab.plan, n_each, static_cast<float*>(dW_gate),
+                                          static_cast<float*>(dW_up));
+  else
+    k_finish_acc<<<148 * 8, 256, 0, st>>>(c.acc32, c.tab.plan, n_each, static_cast<__nv_bfloat16*>(dW_gate),
+                                          static_cast<__nv_bfloat16*>(dW_up));
   return cudaGetLastError();
 }
 cudaError_t launch_router_bwd(const Layout& L, const Ctx& c, cudaStream_t st, int n_tiles_i) {

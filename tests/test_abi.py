@@ -46,9 +46,19 @@ def test_sizes_depend_on_shape_only_and_grow_with_it():
     assert B.moe_ctx_size(s2) >= rp * 7168 * 2 + 2 * rp * 2048 * 2
 
 
+def test_sizes_do_not_depend_on_the_weight_gradient_dtype():
+    for kw in (dict(T=128, d=256, E=8, I=512, top_k=2), dict(T=2048, d=7168, E=256, I=2048, top_k=8)):
+        s16 = B.make_shape(**kw, wgrad_dtype=B.MOE_WGRAD_BF16)
+        s32 = B.make_shape(**kw, wgrad_dtype=B.MOE_WGRAD_FP32)
+        assert B.moe_ctx_size(s16) == B.moe_ctx_size(s32) > 0
+        assert B.moe_workspace_size(s16) == B.moe_workspace_size(s32) > 0
+        assert B.moe_stream_ctx_size(s16, 4) == B.moe_stream_ctx_size(s32, 4) > 0
+
+
 @pytest.mark.parametrize("bad", [
     dict(T=-1), dict(d=0), dict(d=200), dict(I=100), dict(E=0), dict(E=513), dict(top_k=0), dict(top_k=17),
     dict(E=4, top_k=5), dict(first_local_expert=-1), dict(first_local_expert=6, num_local_experts=4),
+    dict(wgrad_dtype=2), dict(wgrad_dtype=-1),
 ])
 def test_invalid_shapes_size_zero(bad):
     kw = dict(T=64, d=256, E=8, I=256, top_k=2)
