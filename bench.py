@@ -134,7 +134,9 @@ def algorithmic_flops(w: IN.Workload) -> dict:
     return {"gemm_gateup_swiglu": 4 * dI * rows, "gemm_down_combw": 2 * dI * rows,
             "gemm_dgrad_down_swiglu_bwd": 2 * dI * rows, "gemm_dgrad_gateup": 4 * dI * rows,
             "gemm_wgrad_gateup": 4 * dI * rows, "gemm_wgrad_down": 2 * dI * rows,
-            "router_logits": 2 * w.tokens * w.d * w.E}
+            "router_logits": 2 * w.tokens * w.d * w.E,
+            # dW_r = X^T dl; the kernel issues it twice (the hi and lo bf16 terms of dl)
+            "router_wgrad": 2 * w.tokens * w.d * w.E}
 
 
 # ----------------------------------------------------------------------------
@@ -177,8 +179,8 @@ def algorithmic_bytes(w: IN.Workload, wgrad_elem_bytes: int = 2) -> dict:
         "router_wgrad": T * d * 2 + T * k * 8 + d * E * 4,  # X once, dl and ids, dW_r
         "gemm_dgrad_gateup": 2 * W1 + 2 * rows * I * 2 + rows * d * 2,
         "reverse_dispatch": rows * d * 2 + T * d * 2 + E * d * 2,
-        "gemm_wgrad_gateup": rows * d * 2 + 2 * rows * I * 2 + 2 * W1,
-        "gemm_wgrad_down": rows * I * 2 + rows * d * 2 + W1,
+        "gemm_wgrad_gateup": rows * d * 2 + 2 * rows * I * 2 + 2 * G1,
+        "gemm_wgrad_down": rows * I * 2 + rows * d * 2 + G1,
     }
 
 

@@ -9,55 +9,87 @@
 
 namespace moe {
 
-// One block = 128 output rows x 128 K of a K-major fp8 weight [R_out, K].
+// One block = 128 output rows x 128 K of a K-major fp8 weight [R_out, K], 128 threads.
 //   mode 0: source [R_out, K] row-major (K contiguous)
 //   mode 1: source [El][K][N] (N contiguous), output row el*N + n
 //   mode 2: paired gate/up, source gate/up [El][K][N]; output rows per expert come in
 //           blocks of 128 = 64 gate rows then 64 up rows (columns j*64 .. j*64+63)
+// Each thread issues all 16 of its 16-byte source loads before it uses any of them.
+// Mode 0 needs no transpose: thread (warp w, lane) owns the 32-value block lane % 4 of rows
+// 32 i + 8 w + lane / 4 (i = 0..3), so the four lanes of a row read its 256 source bytes and
+// write its 128 code bytes contiguously.  Modes 1 and 2 stage the tile transposed in shared
+// memory: a warp loads 4 source rows x 128 bytes, and thread r then quantises output row r.
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 t = unpack_bf16(w[j]);
+    f[2 * j] = t.x;
+    f[2 * j + 1] = t.y;
+  }
+}
+
 __global__ void __launch_bounds__(128) k_quant_weight(const __nv_bfloat16* __restrict__ src0,
                                                       const __nv_bfloat16* __restrict__ src1, int mode, int K, int N,
                                                       uint8_t* __restrict__ q, uint8_t* __restrict__ qs) {
-  extern __shared__ float tile[];  // [128][129]
+  extern __shared__ float tile[];  // [128][129], modes 1 and 2
   const int k0 = blockIdx.x * 128;
   const int o0 = blockIdx.y * 128;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint4 u[16];
   if (mode == 0) {
-    for (int c = threadIdx.x; c < 128 * 16; c += 128) {  // 16-byte chunks along K
-      const int r = c >> 4, kc = (c & 15) * 8;
-      const uint4 u = *reinterpret_cast<const uint4*>(src0 + static_cast<size_t>(o0 + r) * K + k0 + kc);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    const int blk = lane & 3;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = unpack_bf16(w[j]);
-        tile[r * 129 + kc + 2 * j] = f.x;
-        tile[r * 129 + kc + 2 * j + 1] = f.y;
-      }
-    }
-  } else {
-    for (int c = threadIdx.x; c < 128 * 16; c += 128) {  // 16-byte chunks along N of source row k
-      const int kk = c >> 4, nc = (c & 15) * 8;
-      const int r = nc;  // tile row of the first of the 8 columns
-      const int o = o0 + r;
-      const __nv_bfloat16* src;
-      size_t off;
-      if (mode == 1) {
-        const int el = o / N, n = o - el * N;
-        src = src0;
-        off = (static_cast<size_t>(el) * K + k0 + kk) * N + n;
-      } else {
-        const int el = o / (2 * N), w = o - el * 2 * N;
-        const int j = w >> 7, h = (w >> 6) & 1, n = j * 64 + (w & 63);
-        src = h ? src1 : src0;
-        off = (static_cast<size_t>(el) * K + k0 + kk) * N + n;
-      }
-      const uint4 u = *reinterpret_cast<const uint4*>(src + off);
-      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+    for (int i = 0; i < 4; ++i) {
+      const int r = 32 * i + 8 * warp + (lane >> 2);
+      const uint4* s4 = reinterpret_cast<const uint4*>(src0 + static_cast<size_t>(o0 + r) * K + k0 + blk * 32);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = unpack_bf16(w4[j]);
-        tile[(r + 2 * j) * 129 + kk] = f.x;
-        tile[(r + 2 * j + 1) * 129 + kk] = f.y;
-      }
+      for (int j = 0; j < 4; ++j) u[4 * i + j] = __ldg(s4 + j);
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int o = o0 + 32 * i + 8 * warp + (lane >> 2);
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) unpack8(u[4 * i + j], v + 8 * j);
+      uint32_t w[8];
+      const uint8_t sb = mx_quant32(v, w);
+      uint4* d = reinterpret_cast<uint4*>(q + static_cast<size_t>(o) * K + k0 + blk * 32);
+      d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      qs[sf_index(o, k0 + blk * 32, K)] = sb;
+    }
+    return;
+  }
+  // modes 1, 2: load step g = 4 i + warp covers source rows k0 + 4 (g / 2) .. + 3 and the
+  // 64 output rows (g % 2) * 64 .. + 63, eight per lane
+  int kk[16], nc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int g = 4 * i + warp;
+    kk[i] = (g >> 1) * 4 + (lane >> 3);
+    nc[i] = ((g & 1) * 8 + (lane & 7)) * 8;
+    const int o = o0 + nc[i];
+    const __nv_bfloat16* src;
+    size_t off;
+    if (mode == 1) {
+      const int el = o / N, n = o - el * N;
+      src = src0;
+      off = (static_cast<size_t>(el) * K + k0 + kk[i]) * N + n;
+    } else {
+      const int el = o / (2 * N), w = o - el * 2 * N;
+      const int j = w >> 7, h = (w >> 6) & 1, n = j * 64 + (w & 63);
+      src = h ? src1 : src0;
+      off = (static_cast<size_t>(el) * K + k0 + kk[i]) * N + n;
+    }
+    u[i] = __ldg(reinterpret_cast<const uint4*>(src + off));
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float f[8];
+    unpack8(u[i], f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) tile[(nc[i] + e) * 129 + kk[i]] = f[e];
   }
   __syncthreads();
   const int r = threadIdx.x;
@@ -150,7 +182,9 @@ cudaError_t launch_quant_weight(int mode, const __nv_bfloat16* src0, const __nv_
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  k_quant_weight<<<dim3(K / 128, static_cast<unsigned>(R_out / 128)), 128, smem, st>>>(src0, src1, mode, K, N, q, qs);
+  // mode 0 quantises from registers: without the transpose tile more blocks fit on an SM
+  k_quant_weight<<<dim3(K / 128, static_cast<unsigned>(R_out / 128)), 128, mode == 0 ? 0 : smem, st>>>(
+      src0, src1, mode, K, N, q, qs);
   return cudaGetLastError();
 }
 
