@@ -612,6 +612,11 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     algo = algorithmic_bytes(w, 4 if args.wgrad_fp32 else 2)
     traffic_key = w.name + ("+wgrad_fp32" if args.wgrad_fp32 else "")  # counters were taken with bf16 gradients
     aflops = algorithmic_flops(w)
+    if w.El < w.E:
+        # in an expert slice the router weight gradient contracts over the tokens with a local
+        # assignment only; their number depends on the routing, so no figure is claimed for it
+        algo.pop("router_wgrad", None)
+        aflops.pop("router_wgrad", None)
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     bf16 = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     fp8 = fp8_peak.get("sustained_tflops") if fp8_peak else None

@@ -102,6 +102,12 @@ __device__ __forceinline__ int seg_rows(const GemmParams& p, int m, int el) {
 // segment's "live" pad rows, which every producer writes as zeros.
 __device__ __forceinline__ int wgrad_kblocks(const GemmParams& p, int m, int el) { return (seg_rows(p, m, el) + 63) / 64; }
 
+// 64-token K blocks of one dl term in the router weight gradient: all T tokens, or the
+// listed ones (their number is on the device)
+__device__ __forceinline__ int router_wgrad_kblocks(const GemmParams& p) {
+  return ((p.act_n ? __ldg(p.act_n) : p.T) + 63) / 64;
+}
+
 template <int KIND>
 __device__ __forceinline__ Tile decode(const GemmParams& p, int t) {
   Tile tl;
@@ -129,7 +135,7 @@ __device__ __forceinline__ Tile decode(const GemmParams& p, int t) {
     tl.nt = nt;
     tl.n0 = nt * 256;
     tl.kb0 = 0;
-    tl.nk = 2 * ((p.T + 63) / 64);  // the hi terms of dl, then the lo terms
+    tl.nk = 2 * router_wgrad_kblocks(p);  // the hi terms of dl, then the lo terms
     return tl;
   }
   const int NT = ntiles_n<KIND>(p);
@@ -205,15 +211,18 @@ __device__ __forceinline__ void load_stage(const GemmParams& p, const Tile& tl, 
     tma_load_2d(sA, &p.ta0, bar, kx, tl.m0, pol_act);  // X [T, d], rows >= T read as zero
     tma_load_2d(sB, &p.tb0, bar, kx, tl.n0, pol_act);  // W_r^T [E, d], rows >= E read as zero
   } else if constexpr (KIND == G_ROUTER_WGRAD) {
-    // X [T, d] and DL [2 * Tpad, E64] with the contraction over tokens: both MN-major (d and E
-    // contiguous); K block kb of DL pairs with X's block kb mod Tpad/64; tokens >= T read as
-    // zero, experts >= E64 too
-    const int half = (p.T + 63) / 64;
-    const int kx = (kb < half ? kb : kb - half) * 64;
+    // X [T, d] (or the listed tokens' rows) and DL [2 * Tpad, E64] (hi rows from 0, lo rows
+    // from Tpad) with the contraction over tokens: both MN-major (d and E contiguous); the
+    // first `half` K blocks take the hi rows, the rest the lo rows, each paired with the same
+    // X block; tokens >= T read as zero, experts >= E64 too
+    const int half = router_wgrad_kblocks(p);
+    const bool lo = kb >= half;
+    const int kx = (lo ? kb - half : kb) * 64;
+    const int krow = lo ? (p.T + 63) / 64 * 64 + kx : kx;
     tma_load_2d(sA, &p.ta0, bar, tl.m0, kx, pol_act);
     tma_load_2d(sA + 8192, &p.ta0, bar, tl.m0 + 64, kx, pol_act);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) tma_load_2d(sB + j * 8192, &p.tb0, bar, tl.n0 + 64 * j, k0, pol_act);
+    for (int j = 0; j < 4; ++j) tma_load_2d(sB + j * 8192, &p.tb0, bar, tl.n0 + 64 * j, krow, pol_act);
   }
 }
 
@@ -350,12 +359,17 @@ __device__ __forceinline__ void epilogue_row(const GemmParams& p, const Tile& tl
       if (live) store_row32(p.out0 + R * p.d + tl.n0 + c * 32, v);
     }
   } else if constexpr (KIND == G_ROUTER_WGRAD) {
-    // dW_r row (of d) tl.m0 + row, fp32; columns >= E are dropped
+    // dW_r row (of d) tl.m0 + row, fp32; columns >= E are dropped; no listed token: zero
     float* dst = p.outf + static_cast<size_t>(tl.m0 + row) * p.E;
 #pragma unroll 1
     for (int c = 0; c < 8; ++c) {
       float v[32];
-      tmem_ld32(taddr + c * 32, v);
+      if (tl.nk > 0) {
+        tmem_ld32(taddr + c * 32, v);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      }
       const int e0 = tl.n0 + c * 32;
 #pragma unroll
       for (int i = 0; i < 32; ++i)

@@ -44,6 +44,7 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   if (L->RP * static_cast<int64_t>(s.d > s.I ? s.d : s.I) >= (int64_t(1) << 40)) return false;
   L->nblk = static_cast<int>((T_all + kTokensPerBlock - 1) / kTokensPerBlock);
   if (L->nblk < 1) L->nblk = 1;
+  L->scan_groups = L->nblk > kScanOneLevel ? (L->nblk + kScanGroup - 1) / kScanGroup : 0;
 
   const size_t RP = static_cast<size_t>(L->RP), T = static_cast<size_t>(T_all), k = s.top_k;
   size_t o = 0;
@@ -75,6 +76,7 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
 
   o = 0;
   L->hist = take(static_cast<size_t>(L->nblk) * s.E * 4);
+  L->hsum = take(static_cast<size_t>(L->scan_groups) * s.E * 4);
   L->logits = take(T * s.E * 4);
   L->rpart = take(static_cast<size_t>(router_splits(T_all, s.E, s.d)) * T * s.E * 4);
   L->hbuf = take(RP * s.I * 2);
@@ -86,6 +88,10 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->dgpart = take(RP * (s.I / 128) * 4);  // dg partials per n-tile of the dgrad-down GEMM (256 wide bf16, 128 MXFP8)
   L->dlasg = take(T * k * 4);
   L->dldense = take(2 * align_up(static_cast<size_t>(T), 64) * align_up(static_cast<size_t>(s.E), 64) * 2);
+  L->rslice = El < s.E;
+  L->actcnt = take(L->rslice ? ((T + 255) / 256 + 1) * 4 : 0);
+  L->actlist = take(L->rslice ? T * 4 : 0);
+  L->xact = take(L->rslice ? align_up(T, 64) * s.d * 2 : 0);
   L->wrt = take(static_cast<size_t>(s.E) * s.d * 2);
   L->dxperm = take(RP * s.d * 2);
   L->acc32 = take(M > 0 ? 2 * static_cast<size_t>(El) * s.d * s.I * 4 : 0);
@@ -149,6 +155,8 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
     c.tab.ring_start = t;
   }
   c.acc32 = nullptr;
+  c.actcnt = c.actlist = nullptr;
+  c.xact = nullptr;
   c.xq = L.mx ? reinterpret_cast<uint8_t*>(C(L.xq)) : nullptr;
   c.xqs = L.mx ? reinterpret_cast<uint8_t*>(C(L.xqs)) : nullptr;
   c.hq = c.hqs = c.dyq = c.dyqs = c.daq = c.daqs = c.dbq = c.dbqs = nullptr;
@@ -164,6 +172,7 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
   }
   if (ws) {
     c.hist = reinterpret_cast<int*>(W(L.hist));
+    c.hsum = reinterpret_cast<int*>(W(L.hsum));
     c.logits = reinterpret_cast<float*>(W(L.logits));
     c.rpart = reinterpret_cast<float*>(W(L.rpart));
     c.hbuf = reinterpret_cast<__nv_bfloat16*>(W(L.hbuf));
@@ -178,6 +187,11 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
     c.wrt = reinterpret_cast<__nv_bfloat16*>(W(L.wrt));
     c.dxperm = reinterpret_cast<__nv_bfloat16*>(W(L.dxperm));
     c.acc32 = L.M > 0 ? reinterpret_cast<float*>(W(L.acc32)) : nullptr;
+    if (L.rslice) {
+      c.actcnt = reinterpret_cast<int*>(W(L.actcnt));
+      c.actlist = reinterpret_cast<int*>(W(L.actlist));
+      c.xact = reinterpret_cast<__nv_bfloat16*>(W(L.xact));
+    }
   }
   return c;
 }
@@ -267,13 +281,15 @@ static int num_sms() {
 enum KernelId {
   K_ROUTER_LOGITS, K_TOPK, K_SCAN, K_SCATTER, K_DISPATCH, K_GEMM_GATEUP, K_GEMM_DOWN, K_COMBINE,
   K_REV_COMBINE, K_GEMM_DGRAD_DOWN, K_ROUTER_BWD, K_ROUTER_WGRAD, K_TRANSPOSE_WR, K_GEMM_DGRAD_GATEUP, K_REV_DISPATCH,
-  K_GEMM_WGRAD_GATEUP, K_GEMM_WGRAD_DOWN, K_PLAN, K_REPLAY, K_FINISH_ACC, K_QUANT_WEIGHTS, K_MARK_ROWS, K_NUM
+  K_GEMM_WGRAD_GATEUP, K_GEMM_WGRAD_DOWN, K_PLAN, K_REPLAY, K_FINISH_ACC, K_QUANT_WEIGHTS, K_MARK_ROWS,
+  K_ACTIVE_COUNT, K_GATHER_ACTIVE, K_SCAN_GROUPS, K_SCAN_APPLY, K_NUM
 };
 static const char* kKernelNames[K_NUM] = {
     "router_logits", "topk_gating", "hist_scan", "stable_scatter", "dispatch", "gemm_gateup_swiglu",
     "gemm_down_combw", "combine", "reverse_combine", "gemm_dgrad_down_swiglu_bwd", "router_bwd", "router_wgrad",
     "transpose_wr", "gemm_dgrad_gateup", "reverse_dispatch", "gemm_wgrad_gateup", "gemm_wgrad_down",
-    "stream_plan", "ring_replay", "wgrad_accumulator_finish", "quantize_weights", "mark_pad_rows"};
+    "stream_plan", "ring_replay", "wgrad_accumulator_finish", "quantize_weights", "mark_pad_rows",
+    "router_token_count", "router_token_gather", "hist_scan_group_sums", "hist_scan_group_apply"};
 
 struct ProfRec {
   int kid;
@@ -337,13 +353,19 @@ static GemmParams base_params(const Layout& L, const Ctx& c, int* status) {
 
 // dW_r = X^T . DL on the tensor cores (both operands MN-major: d and E are contiguous, the
 // contraction runs over tokens, twice: the hi and the lo bf16 terms of dl); fp32 out, one CTA
-// per 128 x 256 tile, fixed K order.
+// per 128 x 256 tile, fixed K order.  In an expert slice the tokens are the listed ones
+// (c.xact, compacted DL rows, their number on the device).
 static cudaError_t launch_router_wgrad(const Layout& L, const Ctx& c, const void* X, float* dW_r, int* status,
                                        cudaStream_t st) {
   GemmParams p = base_params(L, c, status);
   const uint64_t E64 = align_up(static_cast<size_t>(L.E), 64);
-  if (!tmap_2d(&p.ta0, X, L.d, static_cast<uint64_t>(L.T), L.d, 64, 64)) return cudaErrorInvalidValue;
   const uint64_t Tpad = align_up(static_cast<size_t>(L.T), 64);
+  if (L.rslice) {
+    if (!tmap_2d(&p.ta0, c.xact, L.d, Tpad, L.d, 64, 64)) return cudaErrorInvalidValue;
+    p.act_n = c.actcnt + (L.T + 255) / 256;
+  } else if (!tmap_2d(&p.ta0, X, L.d, static_cast<uint64_t>(L.T), L.d, 64, 64)) {
+    return cudaErrorInvalidValue;
+  }
   if (!tmap_2d(&p.tb0, c.dldense, E64, 2 * Tpad, E64, 64, 64)) return cudaErrorInvalidValue;
   p.ta1 = p.ta0;
   p.tb1 = p.tb0;
@@ -363,6 +385,11 @@ static cudaError_t launch_router_wgrad(const Layout& L, const Ctx& c, const void
 #define MOE_TMAP(x)                                  \
   do {                                               \
     if (!(x)) return MOE_ERR_CUDA;                   \
+  } while (0)
+#define MOE_TRY_STATUS(x)                            \
+  do {                                               \
+    const moe_status s_ = (x);                       \
+    if (s_ != MOE_OK) return s_;                     \
   } while (0)
 
 }  // namespace moe
@@ -442,7 +469,9 @@ static moe_status route_tokens(const Layout& L, const Ctx& c, const void* X, con
     MOE_TRY(timed(K_ROUTER_LOGITS, st, [&] { return launch_gemm(G_ROUTER, p, g, st); }));
   }
   MOE_TRY(timed(K_TOPK, st, [&] { return launch_topk(L, c, bias, splits, st); }));
+  if (L.scan_groups) MOE_TRY(timed(K_SCAN_GROUPS, st, [&] { return launch_scan_groups(L, c, st); }));
   MOE_TRY(timed(K_SCAN, st, [&] { return launch_scan(L, c, st); }));
+  if (L.scan_groups) MOE_TRY(timed(K_SCAN_APPLY, st, [&] { return launch_scan_apply(L, c, st); }));
   if (L.M > 0) {
     // two full waves of the gate/up GEMM: (rows / 128) * (I / 128) >= 2 * SMs
     const int min_rows = static_cast<int>((2LL * grid * 128) / (L.I / 128));
@@ -506,6 +535,20 @@ moe_status moe_fwd(const moe_shape* s, const void* X, const void* W_r, const flo
   }
   // 7. combine
   MOE_TRY(timed(K_COMBINE, st, [&] { return launch_combine(L, c, c.obuf, static_cast<__nv_bfloat16*>(Y), st); }));
+  return MOE_OK;
+}
+
+// 10. router backward: dl (and, in an expert slice, the list of tokens with a local
+// assignment and their X rows), then dW_r = X^T DL on the tensor cores.
+static moe_status router_backward(const Layout& L, const Ctx& c, const void* X, float* dW_r, int* status,
+                                  cudaStream_t st, int n_tiles_i = 0) {
+  if (L.rslice) MOE_TRY(timed(K_ACTIVE_COUNT, st, [&] { return launch_active_count(L, c, st); }));
+  MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st, n_tiles_i); }));
+  if (L.rslice)
+    MOE_TRY(timed(K_GATHER_ACTIVE, st, [&] {
+      return launch_gather_active(L, c, static_cast<const __nv_bfloat16*>(X), st);
+    }));
+  MOE_TRY(timed(K_ROUTER_WGRAD, st, [&] { return launch_router_wgrad(L, c, X, dW_r, status, st); }));
   return MOE_OK;
 }
 
@@ -590,8 +633,7 @@ moe_status moe_bwd(const moe_shape* s, const void* X, const void* W_r, const voi
     MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm(G_DGRAD_DOWN, p, grid, st); }));
   }
   // 10. router backward: dl, then dW_r = X^T DL (tensor cores); W_r^T for the dX router term
-  MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st); }));
-  MOE_TRY(timed(K_ROUTER_WGRAD, st, [&] { return launch_router_wgrad(L, c, X, dW_r, status, st); }));
+  MOE_TRY_STATUS(router_backward(L, c, X, dW_r, status, st));
   MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] { return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st); }));
   // 11. dgrad of gate/up
   {
@@ -788,8 +830,7 @@ moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
     p.outf = c.dgpart;
     MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm(G_DGRAD_DOWN, p, grid, st); }));
   }
-  MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st); }));
-  MOE_TRY(timed(K_ROUTER_WGRAD, st, [&] { return launch_router_wgrad(L, c, X, dW_r, status, st); }));
+  MOE_TRY_STATUS(router_backward(L, c, X, dW_r, status, st));
   MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
     return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
   }));
@@ -1012,8 +1053,7 @@ moe_status moe_bwd_mx(const moe_shape* s, const void* X, const void* W_r, const 
     p.outf = c.dgpart;
     MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm_mx(MX_DGRAD_DOWN, p, grid, st); }));
   }
-  MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st, L.I / mx_bn(MX_DGRAD_DOWN)); }));
-  MOE_TRY(timed(K_ROUTER_WGRAD, st, [&] { return launch_router_wgrad(L, c, X, dW_r, status, st); }));
+  MOE_TRY_STATUS(router_backward(L, c, X, dW_r, status, st, L.I / mx_bn(MX_DGRAD_DOWN)));
   MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
     return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
   }));

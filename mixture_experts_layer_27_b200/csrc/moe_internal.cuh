@@ -14,6 +14,8 @@ namespace moe {
 
 constexpr int kPad = 128;          // rows of an expert segment are padded to a multiple of this
 constexpr int kTokensPerBlock = 16;  // tokens per block of the top-k / scatter kernels
+constexpr int kScanGroup = 32;       // histogram rows per group of the two-level expert scan
+constexpr int kScanOneLevel = 256;   // up to this many token blocks the scan is one block
 constexpr int kMaxE = 512;
 constexpr int kMaxK = 16;
 constexpr int kMaxMinibatches = 256;  // ring-streamed layer
@@ -59,16 +61,18 @@ struct Layout {
   int d, E, I, k, first, El;
   int64_t RP;     // padded-row capacity: worst case of sum_e ceil(count_e / 128) * 128
   int nblk;       // blocks of the top-k / scatter kernels
+  int scan_groups;  // groups of the two-level expert scan (0: one level)
   int M;          // minibatches of a ring-streamed layer (0: one call = one batch)
   int64_t T_mb;   // tokens per minibatch (streamed layer)
   // ctx
   size_t hdr, ids, gates, counts, offsets, poff, perm_tok, perm_asg, slot_row, row_asg, row_gate, xperm, abuf,
       bbuf, stab, xq, xqs, ctx_bytes;
   // ws
-  size_t hist, logits, rpart, hbuf, obuf, dyperm, dabuf, dbbuf, hgbuf, dgpart, dlasg, dldense, wrt, dxperm, acc32, hq, hqs, dyq,
-      dyqs, daq, daqs, dbq, dbqs, ws_bytes;
+  size_t hist, hsum, logits, rpart, hbuf, obuf, dyperm, dabuf, dbbuf, hgbuf, dgpart, dlasg, dldense, wrt, dxperm, acc32, hq, hqs, dyq,
+      dyqs, daq, daqs, dbq, dbqs, actcnt, actlist, xact, ws_bytes;
   bool mx;   // MXFP8 mode
   bool w32;  // expert weight gradients written as fp32
+  bool rslice;  // an expert slice (El < E): the router weight gradient runs over the listed tokens
   // prepared MXFP8 weights (moe_prepare_weights): fp8 codes and scale chunks
   size_t wgu1, wgu1s, wd2, wd2s, wd3, wd3s, wg4, wg4s, wu4, wu4s, wq_bytes;
 };
@@ -119,6 +123,7 @@ struct GemmParams {
   int T, E, splits;           // router GEMM: tokens, experts, K splits
   int router_bn;              // router GEMM: experts per n-tile (E split evenly over ceil(E / 256) tiles)
   int wout32;                 // wgrad: to0 / to1 are fp32 maps (32 x 32 boxes) and take the unrounded sums
+  const int* act_n;           // router wgrad over listed tokens: their number (device); NULL = all T tokens
   int* status;
 };
 
@@ -199,6 +204,7 @@ struct Ctx {  // typed views of ctx + ws for one shape
   float *gates, *row_gate;
   __nv_bfloat16 *xperm, *abuf, *bbuf;
   int* hist;
+  int* hsum;  // two-level scan: per group and expert, the group's sum, then its exclusive prefix
   float* logits;
   float* rpart;  // router split-K partials [splits, T, E]
   __nv_bfloat16 *hbuf, *obuf, *dyperm, *dabuf, *dbbuf, *hgbuf, *wrt, *dxperm;
@@ -206,6 +212,9 @@ struct Ctx {  // typed views of ctx + ws for one shape
   __nv_bfloat16* dldense;  // [2, Tpad, E64] bf16 (Tpad, E64: T, E rounded up to 64): dl at (token, expert) as
                            // hi and lo bf16 terms, zeros elsewhere
   float* acc32;
+  int* actcnt;               // expert slice: token counts per 256-token block, then the list length
+  int* actlist;              // expert slice: the tokens with a local assignment, ascending
+  __nv_bfloat16* xact;       // expert slice: their X rows [Tpad, d] (rows past the list up to a multiple of 64: 0)
   StreamTables tab;
   uint8_t *xq, *xqs, *hq, *hqs, *dyq, *dyqs, *daq, *daqs, *dbq, *dbqs;  // MXFP8 operands and scales
 };
@@ -213,6 +222,8 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws);
 
 cudaError_t launch_topk(const Layout& L, const Ctx& c, const float* bias, int splits, cudaStream_t st);
 cudaError_t launch_scan(const Layout& L, const Ctx& c, cudaStream_t st);
+cudaError_t launch_scan_groups(const Layout& L, const Ctx& c, cudaStream_t st);
+cudaError_t launch_scan_apply(const Layout& L, const Ctx& c, cudaStream_t st);
 cudaError_t launch_scatter(const Layout& L, const Ctx& c, cudaStream_t st);
 cudaError_t launch_mark_rows(const Layout& L, const Ctx& c, cudaStream_t st);
 cudaError_t launch_wait_probe(int* status, cudaStream_t st);
@@ -226,6 +237,10 @@ cudaError_t launch_combine(const Layout& L, const Ctx& c, const __nv_bfloat16* O
 cudaError_t launch_plan(const Layout& L, const Ctx& c, int ring_rows, int min_rows, cudaStream_t st);
 cudaError_t launch_replay(const Layout& L, const Ctx& c, int chunk, const __nv_bfloat16* X, __nv_bfloat16* ring,
                           int64_t ring_rows, cudaStream_t st);
+// expert slice: per-block counts of the tokens with a local assignment (before launch_router_bwd)
+cudaError_t launch_active_count(const Layout& L, const Ctx& c, cudaStream_t st);
+// expert slice: X rows of the listed tokens into c.xact (after launch_router_bwd)
+cudaError_t launch_gather_active(const Layout& L, const Ctx& c, const __nv_bfloat16* X, cudaStream_t st);
 // the fp32 gate/up accumulator into dW_gate / dW_up (bf16, or fp32 when L.w32)
 cudaError_t launch_finish_acc(const Layout& L, const Ctx& c, void* dW_gate, void* dW_up, cudaStream_t st);
 cudaError_t launch_router_bwd(const Layout& L, const Ctx& c, cudaStream_t st, int n_tiles_i = 0);

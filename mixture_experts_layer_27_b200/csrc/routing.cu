@@ -191,6 +191,39 @@ __global__ void __launch_bounds__(1024) k_scan(int* __restrict__ hist, int nblk,
   }
 }
 
+// Two-level form for many token blocks (the single block above walks all nblk rows of every
+// column): one block per group of kScanGroup rows sums its rows, k_scan turns the group sums
+// into exclusive prefixes over groups (and computes counts, offsets, padded offsets), and one
+// block per group writes each row's prefix.  Integer sums: the same result as one pass.
+__global__ void __launch_bounds__(512) k_scan_group_sums(const int* __restrict__ hist, int nblk, int E,
+                                                         int* __restrict__ gsum) {
+  const int b0 = blockIdx.x * kScanGroup;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int h[kScanGroup];
+#pragma unroll
+    for (int j = 0; j < kScanGroup; ++j) h[j] = b0 + j < nblk ? hist[static_cast<size_t>(b0 + j) * E + e] : 0;
+    int sum = 0;
+#pragma unroll
+    for (int j = 0; j < kScanGroup; ++j) sum += h[j];
+    gsum[static_cast<size_t>(blockIdx.x) * E + e] = sum;
+  }
+}
+__global__ void __launch_bounds__(512) k_scan_group_apply(int* __restrict__ hist, int nblk, int E,
+                                                          const int* __restrict__ gsum) {
+  const int b0 = blockIdx.x * kScanGroup;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int h[kScanGroup];
+#pragma unroll
+    for (int j = 0; j < kScanGroup; ++j) h[j] = b0 + j < nblk ? hist[static_cast<size_t>(b0 + j) * E + e] : 0;
+    int run = gsum[static_cast<size_t>(blockIdx.x) * E + e];
+#pragma unroll
+    for (int j = 0; j < kScanGroup; ++j) {
+      if (b0 + j < nblk) hist[static_cast<size_t>(b0 + j) * E + e] = run;
+      run += h[j];
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // pad-row marks of every segment, before the scatter fills its real rows: rows up to the real
 // count rounded up to 16 are ROW_PAD, the rest of the 128-row padding ROW_DEAD; gates 0.
@@ -376,6 +409,140 @@ __global__ void __launch_bounds__(256) k_router_bwd(const float* __restrict__ dg
   }
 }
 
+// ---------------------------------------------------------------------------
+// Router weight gradient of an expert slice.  A token with no local assignment has dg = 0 on
+// every slot, hence dl = 0, so only tokens with a local assignment add to dW_r = X^T DL.  They
+// are listed in ascending token order (a count per 256-token block, a fixed-order sum of the
+// counts before each block and a ballot scan inside it) and the contraction runs over the
+// list alone: row a of the compacted DL and X matrices is the a-th listed token.
+// ---------------------------------------------------------------------------
+constexpr int kActBlock = 256;
+
+__device__ __forceinline__ int has_local_slot(const int* __restrict__ slot_row, int64_t t, int k) {
+  int act = 0;
+  for (int j = 0; j < k; ++j) act |= __ldg(slot_row + t * k + j) >= 0;
+  return act;
+}
+
+__global__ void __launch_bounds__(kActBlock) k_active_count(const int* __restrict__ slot_row, int T, int k,
+                                                            int* __restrict__ cnt) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kActBlock + threadIdx.x;
+  const int n = __syncthreads_count(t < T ? has_local_slot(slot_row, t, k) : 0);
+  if (threadIdx.x == 0) cnt[blockIdx.x] = n;
+}
+
+// dl of every token (dlasg), and the hi / lo DL rows of the listed tokens at their list index
+// a (hi row a, lo row Tpad + a).  cnt[0 .. nb) are the block counts; the last block stores the
+// list length in cnt[nb] and zeroes the rows that pad it to a multiple of 64 in both halves.
+__global__ void __launch_bounds__(kActBlock) k_router_bwd_compact(
+    const float* __restrict__ dgpart, const int* __restrict__ slot_row, const float* __restrict__ gates,
+    const int* __restrict__ ids, int T, int Tpad, int k, int ntn, int E64, int* __restrict__ cnt, int nb,
+    float* __restrict__ dlasg, __nv_bfloat16* __restrict__ dldense, int* __restrict__ act_list) {
+  __shared__ int s_idx[kActBlock];
+  __shared__ int s_warp[kActBlock / 32];
+  __shared__ int s_base, s_total;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0) {
+    int before = 0, total = 0;
+    for (int i = lane; i < nb; i += 32) {
+      const int c = cnt[i];
+      total += c;
+      if (i < static_cast<int>(blockIdx.x)) before += c;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      before += __shfl_xor_sync(0xffffffffu, before, o);
+      total += __shfl_xor_sync(0xffffffffu, total, o);
+    }
+    if (lane == 0) {
+      s_base = before;
+      s_total = total;
+    }
+  }
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kActBlock;
+  const int64_t t = t0 + threadIdx.x;
+  const int act = t < T ? has_local_slot(slot_row, t, k) : 0;
+  const unsigned bal = __ballot_sync(0xffffffffu, act);
+  if (lane == 0) s_warp[warp] = __popc(bal);
+  __syncthreads();
+  int woff = 0;
+  for (int w = 0; w < warp; ++w) woff += s_warp[w];
+  const int a = act ? s_base + woff + __popc(bal & ((1u << lane) - 1u)) : -1;
+  s_idx[threadIdx.x] = a;
+  if (a >= 0) act_list[a] = static_cast<int>(t);
+  __syncthreads();
+  const int n4 = E64 / 8;
+  if (blockIdx.x == gridDim.x - 1) {
+    const int tot = s_total, pad = (tot + 63) / 64 * 64;
+    if (threadIdx.x == 0) cnt[nb] = tot;
+    for (int i = threadIdx.x; i < (pad - tot) * n4; i += kActBlock) {
+      const int r = tot + i / n4, q = i % n4;
+      reinterpret_cast<uint4*>(dldense + static_cast<size_t>(r) * E64)[q] = make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4*>(dldense + (static_cast<size_t>(Tpad) + r) * E64)[q] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  // a warp per token, 32 tokens per warp
+  for (int i = 0; i < 32; ++i) {
+    const int tl = warp * 32 + i;
+    const int64_t tt = t0 + tl;
+    if (tt >= T) break;  // the same for every lane
+    float dg = 0.f, g = 0.f;
+    if (lane < k) {
+      const size_t as = static_cast<size_t>(tt) * k + lane;
+      const int R = slot_row[as];
+      g = gates[as];
+      if (R >= 0)
+        for (int q = 0; q < ntn; ++q) dg += dgpart[static_cast<size_t>(R) * ntn + q];
+    }
+    float sum = 0.f;
+    const float gd = g * dg;
+    for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, gd, j);
+    const float dl = g * (dg - sum);
+    if (lane < k) dlasg[static_cast<size_t>(tt) * k + lane] = dl;
+    const int ar = s_idx[tl];
+    if (ar >= 0) {
+      uint4* hi_row = reinterpret_cast<uint4*>(dldense + static_cast<size_t>(ar) * E64);
+      uint4* lo_row = reinterpret_cast<uint4*>(dldense + (static_cast<size_t>(Tpad) + ar) * E64);
+      for (int q = lane; q < n4; q += 32) hi_row[q] = lo_row[q] = make_uint4(0, 0, 0, 0);
+      __syncwarp();  // the zero rows are written before the k entries
+      if (lane < k) {
+        const int e = ids[static_cast<size_t>(tt) * k + lane];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(dl);
+        dldense[static_cast<size_t>(ar) * E64 + e] = hi;
+        dldense[(static_cast<size_t>(Tpad) + ar) * E64 + e] = __float2bfloat16_rn(dl - __bfloat162float(hi));
+      }
+    }
+  }
+}
+
+// X rows of the listed tokens, then zero rows up to the next multiple of 64 (a warp per row,
+// four 16-byte loads in flight per lane)
+__global__ void __launch_bounds__(256) k_gather_active(const __nv_bfloat16* __restrict__ X, int d,
+                                                       const int* __restrict__ act_list, const int* __restrict__ act_n,
+                                                       int64_t max_rows, __nv_bfloat16* __restrict__ Xa) {
+  const int n = __ldg(act_n);
+  const int64_t pad = (static_cast<int64_t>(n) + 63) / 64 * 64;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nv = d / 8;
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + warp; r < pad && r < max_rows;
+       r += static_cast<int64_t>(gridDim.x) * 8) {
+    uint4* o = reinterpret_cast<uint4*>(Xa + r * d);
+    const uint4* in = r < n ? reinterpret_cast<const uint4*>(X + static_cast<int64_t>(__ldg(act_list + r)) * d)
+                            : nullptr;
+    for (int c0 = lane; c0 < nv; c0 += 128) {
+      uint4 u[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = c0 + 32 * j;
+        u[j] = (in != nullptr && c < nv) ? __ldg(in + c) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (c0 + 32 * j < nv) o[c0 + 32 * j] = u[j];
+    }
+  }
+}
+
 // W_r [d, E] -> W_r^T [E, d] (bf16), 32 x 32 tiles
 __global__ void __launch_bounds__(256) k_transpose_wr(const __nv_bfloat16* __restrict__ Wr, int d, int E,
                                                       __nv_bfloat16* __restrict__ WrT) {
@@ -426,7 +593,9 @@ __global__ void __launch_bounds__(256) k_transpose_wr_v(const __nv_bfloat16* __r
 
 // ---------------------------------------------------------------------------
 // reverse-dispatch: dX[t] = sum_j dX_perm[slot_row[t,j]] + sum_j dl_j W_r[:, e_j]
-// (expert terms first, then router terms, each in slot order; fp32; bf16 out)
+// (expert terms first, then router terms, each in slot order; fp32; bf16 out).  A router term
+// with dl_j = 0 adds nothing and is skipped: in an expert slice that is every slot of a token
+// with no local assignment, whose row is then written without reading W_r.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) k_rev_dispatch(const __nv_bfloat16* __restrict__ dxperm,
                                                       const int* __restrict__ slot_row, const int* __restrict__ ids,
@@ -457,6 +626,7 @@ __global__ void __launch_bounds__(128) k_rev_dispatch(const __nv_bfloat16* __res
     }
     for (int j = 0; j < k; ++j) {
       const float w = dl[j];
+      if (w == 0.f) continue;  // the same for every thread of the block
       const uint4 u = __ldg(reinterpret_cast<const uint4*>(WrT + static_cast<size_t>(eid[j]) * d + i));
       float2 f;
       f = unpack_bf16(u.x); acc[0] = fmaf(w, f.x, acc[0]); acc[1] = fmaf(w, f.y, acc[1]);
@@ -695,7 +865,17 @@ cudaError_t launch_topk(const Layout& L, const Ctx& c, const float* bias, int sp
   return cudaGetLastError();
 }
 cudaError_t launch_scan(const Layout& L, const Ctx& c, cudaStream_t st) {
-  k_scan<<<1, 1024, 0, st>>>(c.hist, L.nblk, L.E, L.first, L.El, c.counts, c.offsets, c.poff, c.hdr);
+  // over the group sums when the scan is two-level (launch_scan_groups before, _apply after)
+  k_scan<<<1, 1024, 0, st>>>(L.scan_groups ? c.hsum : c.hist, L.scan_groups ? L.scan_groups : L.nblk, L.E, L.first,
+                             L.El, c.counts, c.offsets, c.poff, c.hdr);
+  return cudaGetLastError();
+}
+cudaError_t launch_scan_groups(const Layout& L, const Ctx& c, cudaStream_t st) {
+  k_scan_group_sums<<<L.scan_groups, 512, 0, st>>>(c.hist, L.nblk, L.E, c.hsum);
+  return cudaGetLastError();
+}
+cudaError_t launch_scan_apply(const Layout& L, const Ctx& c, cudaStream_t st) {
+  k_scan_group_apply<<<L.scan_groups, 512, 0, st>>>(c.hist, L.nblk, L.E, c.hsum);
   return cudaGetLastError();
 }
 cudaError_t launch_scatter(const Layout& L, const Ctx& c, cudaStream_t st) {
@@ -767,10 +947,30 @@ cudaError_t launch_finish_acc(const Layout& L, const Ctx& c, void* dW_gate, void
                                           static_cast<__nv_bfloat16*>(dW_up));
   return cudaGetLastError();
 }
+cudaError_t launch_active_count(const Layout& L, const Ctx& c, cudaStream_t st) {
+  const int nb = static_cast<int>((L.T + kActBlock - 1) / kActBlock);
+  k_active_count<<<nb, kActBlock, 0, st>>>(c.slot_row, static_cast<int>(L.T), L.k, c.actcnt);
+  return cudaGetLastError();
+}
+cudaError_t launch_gather_active(const Layout& L, const Ctx& c, const __nv_bfloat16* X, cudaStream_t st) {
+  const int nb = static_cast<int>((L.T + kActBlock - 1) / kActBlock);
+  const int64_t Tpad = (L.T + 63) / 64 * 64;
+  const int64_t g = (Tpad + 7) / 8;
+  const int grid = static_cast<int>(g < 148 * 8 ? g : 148 * 8);
+  k_gather_active<<<grid, 256, 0, st>>>(X, L.d, c.actlist, c.actcnt + nb, Tpad, c.xact);
+  return cudaGetLastError();
+}
 cudaError_t launch_router_bwd(const Layout& L, const Ctx& c, cudaStream_t st, int n_tiles_i) {
   // n_tiles_i: dg partials per row = n-tiles of the dgrad-down GEMM (I / 256 bf16, I / 128 MXFP8)
   const int E64 = (L.E + 63) / 64 * 64;
   const int Tpad = static_cast<int>((L.T + 63) / 64 * 64);
+  if (L.rslice) {  // expert slice: DL rows of the listed tokens only (launch_active_count first)
+    const int nb = static_cast<int>((L.T + kActBlock - 1) / kActBlock);
+    k_router_bwd_compact<<<nb, kActBlock, 0, st>>>(c.dgpart, c.slot_row, c.gates, c.ids, static_cast<int>(L.T), Tpad,
+                                                   L.k, n_tiles_i ? n_tiles_i : L.I / 256, E64, c.actcnt, nb,
+                                                   c.dlasg, c.dldense, c.actlist);
+    return cudaGetLastError();
+  }
   k_router_bwd<<<static_cast<unsigned>(Tpad / 8), 256, 0, st>>>(c.dgpart, c.slot_row, c.gates, c.ids,
                                                                  static_cast<int>(L.T), Tpad, L.k,
                                                                  n_tiles_i ? n_tiles_i : L.I / 256, E64, c.dlasg,

@@ -93,6 +93,28 @@ def test_local_expert_slice():
     _check_layer(200, 256, 16, 4, 256, first=4, num=5, seed=6)
 
 
+def test_many_token_blocks_two_level_scan():
+    # 4112 tokens = 257 blocks of 16: the expert scan runs in two levels (groups of 32 rows,
+    # the last group holding one row); routing stays bit-exact against the oracle
+    _check_layer(4112, 256, 16, 2, 256, seed=14)
+
+
+def test_expert_slice_router_gradient_over_listed_tokens():
+    # In a slice only the tokens with a local assignment carry router gradient; the weight
+    # gradient contracts over that list (here about 120 of 700 tokens, spread over three
+    # 256-token blocks and a ragged tail).
+    _check_layer(700, 256, 64, 4, 256, first=10, num=3, seed=12)
+
+
+def test_expert_slice_that_receives_no_tokens():
+    bias = np.zeros(8, dtype=np.float32)
+    bias[6:] = -40.0  # the slice's experts are never picked: no token is listed
+    layer, x, Y, g = _check_layer(300, 256, 8, 2, 256, first=6, num=2, bias=bias, seed=13)
+    for n in ("dW_r", "dW_gate", "dW_up", "dW_down"):
+        assert torch.count_nonzero(g[n]) == 0, n
+    assert torch.count_nonzero(Y) == 0 and torch.count_nonzero(g["dX"]) == 0
+
+
 def test_no_tokens():
     T, d, E, k, I = 0, 256, 4, 2, 256
     layer = B.MoELayer(T, d, E, I, k)
