@@ -189,7 +189,7 @@ def algorithmic_bytes(w: IN.Workload, wgrad_elem_bytes: int = 2) -> dict:
 # A figure is reported only while the GEMM sources still hash to the value they had
 # when the counters were taken.
 NCU_TRAFFIC = {
-    ("gemm_wgrad_gateup", "dsv3"): (913.28e6 * 16, "7e6aac1090f2baec"),
+    ("gemm_wgrad_gateup", "dsv3"): (913.67e6 * 16, "b1939f26a44f1da2"),
 }
 GEMM_SOURCES = ("gemm.cu", "ptx.cuh", "moe_internal.cuh")
 
