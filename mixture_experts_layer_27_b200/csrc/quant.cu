@@ -17,8 +17,11 @@ namespace moe {
 // Each thread issues all 16 of its 16-byte source loads before it uses any of them.
 // Mode 0 needs no transpose: thread (warp w, lane) owns the 32-value block lane % 4 of rows
 // 32 i + 8 w + lane / 4 (i = 0..3), so the four lanes of a row read its 256 source bytes and
-// write its 128 code bytes contiguously.  Modes 1 and 2 stage the tile transposed in shared
-// memory: a warp loads 4 source rows x 128 bytes, and thread r then quantises output row r.
+// write its 128 code bytes contiguously.  Modes 1 and 2 stage the tile in shared memory as it
+// is read (bf16, one row per source row k, 128 output rows wide): a warp loads and stores 4
+// source rows x 128 bytes, and thread r then quantises output row r reading its column.
+constexpr int kQuantPitch = 136;  // bf16 elements per staged row: 272 bytes, 16-byte aligned, rows 4 banks apart
+
 __device__ __forceinline__ void unpack8(const uint4& u, float* f) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -32,7 +35,8 @@ __device__ __forceinline__ void unpack8(const uint4& u, float* f) {
 __global__ void __launch_bounds__(128) k_quant_weight(const __nv_bfloat16* __restrict__ src0,
                                                       const __nv_bfloat16* __restrict__ src1, int mode, int K, int N,
                                                       uint8_t* __restrict__ q, uint8_t* __restrict__ qs) {
-  extern __shared__ float tile[];  // [128][129], modes 1 and 2
+  extern __shared__ __align__(16) uint8_t tile_raw[];  // modes 1, 2: [128 k][kQuantPitch] bf16
+  __nv_bfloat16* tile = reinterpret_cast<__nv_bfloat16*>(tile_raw);
   const int k0 = blockIdx.x * 128;
   const int o0 = blockIdx.y * 128;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -85,12 +89,7 @@ __global__ void __launch_bounds__(128) k_quant_weight(const __nv_bfloat16* __res
     u[i] = __ldg(reinterpret_cast<const uint4*>(src + off));
   }
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    float f[8];
-    unpack8(u[i], f);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) tile[(nc[i] + e) * 129 + kk[i]] = f[e];
-  }
+  for (int i = 0; i < 16; ++i) *reinterpret_cast<uint4*>(tile + kk[i] * kQuantPitch + nc[i]) = u[i];
   __syncthreads();
   const int r = threadIdx.x;
   const int o = o0 + r;
@@ -98,7 +97,7 @@ __global__ void __launch_bounds__(128) k_quant_weight(const __nv_bfloat16* __res
   for (int b = 0; b < 4; ++b) {
     float v[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = tile[r * 129 + b * 32 + i];
+    for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(tile[(b * 32 + i) * kQuantPitch + r]);
     uint32_t w[8];
     const uint8_t sb = mx_quant32(v, w);
     uint4* d = reinterpret_cast<uint4*>(q + static_cast<size_t>(o) * K + k0 + b * 32);
@@ -173,7 +172,7 @@ __global__ void __launch_bounds__(256) k_gather_rows_mx(const __nv_bfloat16* __r
 
 cudaError_t launch_quant_weight(int mode, const __nv_bfloat16* src0, const __nv_bfloat16* src1, int64_t R_out, int K,
                                 int N, uint8_t* q, uint8_t* qs, cudaStream_t st) {
-  const int smem = 128 * 129 * 4;
+  const int smem = 128 * kQuantPitch * 2;
   static bool configured[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
