@@ -603,20 +603,39 @@ __global__ void __launch_bounds__(128) k_rev_dispatch(const __nv_bfloat16* __res
                                                       const __nv_bfloat16* __restrict__ WrT, int k, int d,
                                                       __nv_bfloat16* __restrict__ dX) {
   const int t = blockIdx.x;
+  // the token's contributing slots, compacted in slot order: rows with a local expert, and
+  // router terms with dl != 0 (so a token with nothing to add only writes zeros)
   __shared__ int rows[kMaxK], eid[kMaxK];
   __shared__ float dl[kMaxK];
-  if (threadIdx.x < k) {
-    const size_t a = static_cast<size_t>(t) * k + threadIdx.x;
-    rows[threadIdx.x] = slot_row[a];
-    eid[threadIdx.x] = ids[a];
-    dl[threadIdx.x] = dlasg[a];
+  __shared__ int nr, nd;
+  if (threadIdx.x < 32) {
+    const int j = threadIdx.x;
+    int R = -1, e = 0;
+    float w = 0.f;
+    if (j < k) {
+      const size_t a = static_cast<size_t>(t) * k + j;
+      R = slot_row[a];
+      e = ids[a];
+      w = dlasg[a];
+    }
+    const unsigned mr = __ballot_sync(0xffffffffu, j < k && R >= 0);
+    const unsigned md = __ballot_sync(0xffffffffu, j < k && w != 0.f);
+    const unsigned below = (1u << j) - 1u;
+    if (j < k && R >= 0) rows[__popc(mr & below)] = R;
+    if (j < k && w != 0.f) {
+      eid[__popc(md & below)] = e;
+      dl[__popc(md & below)] = w;
+    }
+    if (j == 0) {
+      nr = __popc(mr);
+      nd = __popc(md);
+    }
   }
   __syncthreads();
   for (int i = threadIdx.x * 8; i < d; i += blockDim.x * 8) {
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < k; ++j) {
+    for (int j = 0; j < nr; ++j) {
       const int R = rows[j];
-      if (R < 0) continue;
       const uint4 u = __ldg(reinterpret_cast<const uint4*>(dxperm + static_cast<size_t>(R) * d + i));
       float2 f;
       f = unpack_bf16(u.x); acc[0] += f.x; acc[1] += f.y;
@@ -624,9 +643,8 @@ __global__ void __launch_bounds__(128) k_rev_dispatch(const __nv_bfloat16* __res
       f = unpack_bf16(u.z); acc[4] += f.x; acc[5] += f.y;
       f = unpack_bf16(u.w); acc[6] += f.x; acc[7] += f.y;
     }
-    for (int j = 0; j < k; ++j) {
+    for (int j = 0; j < nd; ++j) {
       const float w = dl[j];
-      if (w == 0.f) continue;  // the same for every thread of the block
       const uint4 u = __ldg(reinterpret_cast<const uint4*>(WrT + static_cast<size_t>(eid[j]) * d + i));
       float2 f;
       f = unpack_bf16(u.x); acc[0] = fmaf(w, f.x, acc[0]); acc[1] = fmaf(w, f.y, acc[1]);
