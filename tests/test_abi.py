@@ -90,6 +90,10 @@ def test_argument_errors_are_synchronous(lib):
     r = B.moe_bwd(s, fake, fake, fake, fake, fake, None, fake, fake, fake, fake, fake, fake, fake, stream=0,
                   ctx_bytes=nc, ws_bytes=nw)
     assert r == B.MOE_ERR_INVALID_ARG  # dY missing
+    for wd in (2, -1):  # a weight-gradient dtype other than bf16 (0) or fp32 (1): refused before any launch
+        sw = B.make_shape(64, 256, 8, 256, 2, wgrad_dtype=wd)
+        r = B.moe_bwd(sw, *[fake] * 6, fake, fake, fake, fake, fake, fake, fake, stream=0, ctx_bytes=nc, ws_bytes=nw)
+        assert r == B.MOE_ERR_UNSUPPORTED
     assert B.moe_get_error(None, 0) == B.MOE_ERR_INVALID_ARG
     for code in range(7):
         assert B.status_string(code)
