@@ -219,6 +219,25 @@ def test_local_expert_slices_sum_to_full_layer():
     np.testing.assert_allclose(dWrs, gf["dW_r"], rtol=1e-11, atol=1e-12)
 
 
+def test_slice_router_gradient_lives_on_tokens_with_a_local_assignment():
+    """In an expert slice a token with no local assignment has dg = 0 on every slot, so its
+    dl row is exactly zero and dW_r = X^T dl is the same sum over the other tokens alone."""
+    rng = np.random.default_rng(10)
+    T, d, E, I, k = 40, 8, 12, 16, 2
+    X, W_r, Wg, Wu, Wd, dY = _rand_layer(rng, T, d, E, I, k)
+    fl, nl = 3, 2
+    Y, c = O.forward(X, W_r, None, Wg, Wu, Wd, k, first_local=fl, num_local=nl)
+    g = O.backward(c, dY)
+    ids = O.topk_ids(O.router_logits(X, W_r, None), k)
+    listed = np.any((ids >= fl) & (ids < fl + nl), axis=1)
+    assert 0 < listed.sum() < T
+    assert np.all(g["dl"][~listed] == 0.0)
+    assert np.any(g["dl"][listed] != 0.0)
+    np.testing.assert_allclose(X[listed].T @ g["dl"][listed], g["dW_r"], rtol=1e-13, atol=1e-14)
+    assert np.all(Y[~listed] == 0.0)  # nothing of theirs is computed in this slice
+    assert np.all(g["dX"][~listed] == 0.0)
+
+
 # --------------------------------------------------------------------------
 # routing: selection, ties, invariants of the table
 # --------------------------------------------------------------------------
