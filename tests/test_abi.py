@@ -97,3 +97,54 @@ def test_argument_errors_are_synchronous(lib):
     assert B.moe_get_error(None, 0) == B.MOE_ERR_INVALID_ARG
     for code in range(7):
         assert B.status_string(code)
+
+
+def test_stream_shapes_and_sizes():
+    s = B.make_shape(2048, 7168, 384, 2048, 8, first_local_expert=0, num_local_experts=6)
+    assert B.moe_stream_ctx_size(s, 16) > 0 and B.moe_stream_workspace_size(s, 16) > 0
+    # one minibatch's worst case: T*min(k, El) rows + 127 pad rows per local expert, in 128-row tiles
+    rows = -(-(2048 * 6 + 127 * 6) // 128) * 128
+    assert B.moe_stream_min_ring_bytes(s) == rows * 7168 * 2
+    for M in (0, -1, 257):
+        assert B.moe_stream_ctx_size(s, M) == 0 and B.moe_stream_workspace_size(s, M) == 0
+    ragged = B.make_shape(2050, 7168, 384, 2048, 8)  # minibatches are whole 16-token blocks
+    assert B.moe_stream_ctx_size(ragged, 4) == 0 and B.moe_stream_min_ring_bytes(ragged) == 0
+    mx = B.make_shape(2048, 7168, 384, 2048, 8, prec=B.MOE_MXFP8)  # the ring stream is bf16 only
+    assert B.moe_stream_ctx_size(mx, 4) == 0
+
+
+def test_stream_argument_errors_are_synchronous(lib):
+    s = B.make_shape(128, 256, 16, 256, 4)
+    M = 4
+    nc, nw, nr = B.moe_stream_ctx_size(s, M), B.moe_stream_workspace_size(s, M), B.moe_stream_min_ring_bytes(s)
+    f = 1 << 20  # never dereferenced
+
+    def fwd(ring_bytes=nr, X=f, ctx=f, M=M):
+        return lib.moe_fwd_stream(ctypes.byref(s), M, X, f, None, f, f, f, f, ctx, nc, f, ring_bytes, f, nw, None)
+
+    assert fwd(X=None) == B.MOE_ERR_INVALID_ARG
+    assert fwd(X=f + 8) == B.MOE_ERR_INVALID_ARG  # misaligned
+    assert fwd(M=0) == B.MOE_ERR_INVALID_ARG
+    assert fwd(ring_bytes=nr - 512) == B.MOE_ERR_WORKSPACE_TOO_SMALL  # less than one minibatch
+    r = lib.moe_bwd_stream(ctypes.byref(s), M, f, f, f, f, f, None, f, nc, f, f, f, f, f, f, nr, f, nw, None)
+    assert r == B.MOE_ERR_INVALID_ARG  # dY missing
+
+
+def test_mxfp8_sizes_and_argument_errors(lib):
+    mx = B.make_shape(256, 256, 8, 512, 2, prec=B.MOE_MXFP8)
+    bf = B.make_shape(256, 256, 8, 512, 2)
+    nq = B.moe_weights_size(mx)
+    # five prepared regions of E*d*I codes (W_gate and W_up together in the first) and 1/32 of scales
+    assert nq >= 6 * 8 * 256 * 512 * 33 // 32
+    assert B.moe_weights_size(bf) == 0
+    nc, nw = B.moe_ctx_size(mx), B.moe_workspace_size(mx)
+    assert nc > B.moe_ctx_size(bf) and nw > B.moe_workspace_size(bf)  # fp8 copies of the operands
+    f = 1 << 20
+    assert lib.moe_prepare_weights(ctypes.byref(mx), f, f, None, f, nq, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_prepare_weights(ctypes.byref(mx), f, f, f, f, nq - 1, None) == B.MOE_ERR_WORKSPACE_TOO_SMALL
+    # the MXFP8 entry points refuse a bf16 shape, the bf16 ones an MXFP8 shape
+    assert lib.moe_fwd_mx(ctypes.byref(bf), f, f, None, f, nq, f, f, nc, f, nw, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_fwd_mx(ctypes.byref(mx), f, f, None, f, nq - 1, f, f, nc, f, nw, None) == \
+        B.MOE_ERR_WORKSPACE_TOO_SMALL
+    r = lib.moe_bwd_mx(ctypes.byref(mx), f, f, f, nq, None, f, nc, f, f, f, f, f, f, nw, None)
+    assert r == B.MOE_ERR_INVALID_ARG  # dY missing
