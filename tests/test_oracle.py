@@ -405,3 +405,143 @@ def test_mx_round_error_bound_and_idempotence():
     amax = np.abs(vb).max(-1, keepdims=True)
     step = 2.0 ** (np.floor(np.log2(amax)) - 8)  # scale; codes are <= 448 = 1.75 * 2^8
     assert np.all(np.abs(vb - rb) <= np.maximum(amax - 448 * step, 0) + 16 * step + 1e-300)
+
+
+# --------------------------------------------------------------------------
+# MX layer: every operand is rounded in blocks along its own GEMM's contraction
+# dimension (d for X, W_gate, W_up and, in the dgrad of W_down, for dY and W_down;
+# I for H, W_down in the forward, dA, dB and W_gate / W_up in the dgrad of gate/up).
+# Rounding in blocks along one axis commutes with scaling a single line across the
+# other axis by a power of two, so a line scaled that way changes its own results
+# (by that power exactly) and nothing else, bit for bit.  With any operand rounded
+# along the other axis the scaled line would become the amax of its blocks there and
+# change how its neighbours round.  The checks below hold one line of each operand
+# against that, and so fail if any rounding axis of forward_mx / backward_mx flips.
+# --------------------------------------------------------------------------
+_MX_SHAPE = dict(T=96, d=64, E=3, I=64, k=2)
+_P2 = 32.0  # a power of two large enough to become the amax of any block it joins
+
+
+def _mx_case(seed=40):
+    rng = np.random.default_rng(seed)
+    s = _MX_SHAPE
+    X, W_r, Wg, Wu, Wd, dY = _rand_layer(rng, s["T"], s["d"], s["E"], s["I"], s["k"])
+    return X, W_r, Wg, Wu, Wd, dY
+
+
+def _mx_run(X, W_r, Wg, Wu, Wd, dY, k=_MX_SHAPE["k"]):
+    Y, ctx = O.forward_mx(X, W_r, None, Wg, Wu, Wd, k)
+    return Y, ctx, O.backward_mx(ctx, dY)
+
+
+def _same_except(a, b, axis, line):
+    """a and b equal bit for bit outside index `line` of `axis`, and different on it."""
+    a, b = np.moveaxis(a, axis, 0), np.moveaxis(b, axis, 0)
+    keep = np.ones(a.shape[0], dtype=bool)
+    keep[line] = False
+    return np.array_equal(a[keep], b[keep]) and not np.array_equal(a[line], b[line])
+
+
+def test_mx_token_rows_are_independent():
+    # X, H, dY, dA and dB are rounded per token row (along d or I): scaling one token's X and
+    # dY rows leaves every other token's Y, dX and router gradient bit-identical.
+    X, W_r, Wg, Wu, Wd, dY = _mx_case()
+    Y, ctx, g = _mx_run(X, W_r, Wg, Wu, Wd, dY)
+    t = 37
+    X2, dY2 = X.copy(), dY.copy()
+    X2[t] *= _P2
+    dY2[t] *= _P2
+    Y2, ctx2, g2 = _mx_run(X2, W_r, Wg, Wu, Wd, dY2)
+    assert np.array_equal(ctx["ids"], ctx2["ids"])  # a positive scale keeps the selection
+    assert _same_except(Y, Y2, 0, t)
+    assert _same_except(g["dX"], g2["dX"], 0, t)
+    assert _same_except(g["dl"], g2["dl"], 0, t)
+    # the forward alone, with dY unchanged: the other tokens' dX stays put as well
+    _, _, g3 = _mx_run(X2, W_r, Wg, Wu, Wd, dY)
+    assert _same_except(g["dX"], g3["dX"], 0, t)
+    # dY alone: the backward's dY rounding (along d) keeps tokens apart
+    _, _, g4 = _mx_run(X, W_r, Wg, Wu, Wd, dY2)
+    assert _same_except(g["dX"], g4["dX"], 0, t)
+
+
+@pytest.mark.parametrize("name,slot", [("W_gate", 2), ("W_up", 3)])
+def test_mx_forward_gate_up_weight_columns_are_independent(name, slot):
+    # W_gate and W_up are rounded along d (the forward's contraction): scaling column j of one
+    # expert's matrix scales that expert's A (or B) column j exactly and no other column.
+    X, W_r, Wg, Wu, Wd, dY = _mx_case()
+    _, ctx = O.forward_mx(X, W_r, None, Wg, Wu, Wd, _MX_SHAPE["k"])
+    e, j = 1, 21
+    W2 = (Wg if name == "W_gate" else Wu).copy()
+    W2[e][:, j] *= _P2
+    args = (W2, Wu) if name == "W_gate" else (Wg, W2)
+    _, ctx2 = O.forward_mx(X, W_r, None, *args, Wd, _MX_SHAPE["k"])
+    a, a2 = ctx["saved"][e][slot], ctx2["saved"][e][slot]
+    assert _same_except(a, a2, 1, j)
+    assert np.array_equal(a2[:, j], a[:, j] * _P2)
+
+
+def test_mx_forward_down_weight_columns_are_independent():
+    # W_down is rounded along I in the forward: scaling its column c (of d) changes column c of
+    # Y only.
+    X, W_r, Wg, Wu, Wd, dY = _mx_case()
+    Y, _ = O.forward_mx(X, W_r, None, Wg, Wu, Wd, _MX_SHAPE["k"])
+    Wd2 = Wd.copy()
+    Wd2[0][:, 9] *= _P2
+    Y2, _ = O.forward_mx(X, W_r, None, Wg, Wu, Wd2, _MX_SHAPE["k"])
+    assert _same_except(Y, Y2, 1, 9)
+
+
+def test_mx_dgrad_down_weight_rows_are_independent():
+    # In the dgrad of W_down (contraction over d) W_down is rounded along d: scaling its row i
+    # (of I) in the backward alone scales dH'[:, i], hence dA[:, i] and dB[:, i], exactly, so
+    # column i of dW_gate and dW_up scales exactly and no other column moves.
+    X, W_r, Wg, Wu, Wd, dY = _mx_case()
+    _, ctx = O.forward_mx(X, W_r, None, Wg, Wu, Wd, _MX_SHAPE["k"])
+    g = O.backward_mx(ctx, dY)
+    e, i = 2, 45
+    Wd2 = Wd.copy()
+    Wd2[e][i, :] *= _P2
+    g2 = O.backward_mx(dict(ctx, W_down=Wd2), dY)
+    for n in ("dW_gate", "dW_up"):
+        assert _same_except(g[n][e], g2[n][e], 1, i), n
+        assert np.array_equal(g2[n][e][:, i], g[n][e][:, i] * _P2), n
+
+
+@pytest.mark.parametrize("name", ["W_gate", "W_up"])
+def test_mx_dgrad_gate_up_weight_rows_are_independent(name):
+    # In the dgrad of gate/up (contraction over I) W_gate and W_up are rounded along I: scaling
+    # row r (of d) in the backward alone changes column r of dX and no other column.
+    X, W_r, Wg, Wu, Wd, dY = _mx_case()
+    _, ctx = O.forward_mx(X, W_r, None, Wg, Wu, Wd, _MX_SHAPE["k"])
+    g = O.backward_mx(ctx, dY)
+    W2 = ctx[name].copy()
+    W2[0][13, :] *= _P2
+    g2 = O.backward_mx(dict(ctx, **{name: W2}), dY)
+    assert _same_except(g["dX"], g2["dX"], 1, 13)
+
+
+def test_mx_layer_worked_example_by_hand():
+    # tests/golden/mx_layer_worked_example.json: a one-expert MXFP8 layer whose every rounding
+    # is worked out by hand there (the values differ if X, H or dA were rounded along tokens).
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "mx_layer_worked_example.json")) as f:
+        G = json.load(f)
+    s = G["shape"]
+    T, d, E, k, I = s["T"], s["d"], s["E"], s["top_k"], s["I"]
+    arrays = {"X": np.zeros((T, d)), "W_gate[0]": np.zeros((d, I)), "W_up[0]": np.zeros((d, I)),
+              "W_down[0]": np.zeros((I, d)), "dY": np.zeros((T, d)), "W_r": np.zeros((d, E))}
+    for name, entries in G["inputs_nonzero"].items():
+        for r, c, v in entries:
+            arrays[name][r, c] = v
+    Y, ctx = O.forward_mx(arrays["X"], arrays["W_r"], None, arrays["W_gate[0]"][None], arrays["W_up[0]"][None],
+                          arrays["W_down[0]"][None], k)
+    g = O.backward_mx(ctx, arrays["dY"])
+    got = {"Y": Y, "dX": g["dX"], "dg": g["dg"], "dW_gate[0]": g["dW_gate"][0], "dW_up[0]": g["dW_up"][0],
+           "dW_down[0]": g["dW_down"][0]}
+    for name, entries in G["expected"].items():
+        want = np.zeros_like(got[name])
+        for r, c, v in entries:
+            want[r, c] = v
+        np.testing.assert_allclose(got[name], want, rtol=1e-13, atol=0, err_msg=name)
+    assert not np.any(g["dW_r"])
