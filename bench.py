@@ -184,8 +184,8 @@ def algorithmic_bytes(w: IN.Workload, wgrad_elem_bytes: int = 2) -> dict:
     }
 
 
-# DRAM bytes per launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum),
-# scaled to the workload by the units processed; see profiles/ncu_traffic_gemm_wgrad_gateup_dsv3_e16.md.
+# DRAM bytes per launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum) on a
+# 16-expert case of the same expert shape, scaled to the workload by the experts processed.
 # A figure is reported only while the GEMM sources still hash to the value they had
 # when the counters were taken.
 NCU_TRAFFIC = {

@@ -267,11 +267,18 @@ moe_status moe_debug_stream_plan(const moe_shape* shape, int32_t num_minibatches
  * inside the library; every GPU that loads the library holds it until the
  * process exits.  Shapes needing more (about E*d*2 + (S+1)*T*E*4 +
  * ceil(T/16)*E*4 bytes, S = K splits of the router GEMM) are refused with
- * MOE_ERR_WORKSPACE_TOO_SMALL.  The first call on a device looks up the
- * array's device address (cudaGetSymbolAddress) with that device current;
- * make that first call before any stream capture.  The call allocates
- * nothing and never synchronises.  All calls share the one array: calls that
- * overlap on the GPU race on it and must be serialised by the caller. */
+ * MOE_ERR_WORKSPACE_TOO_SMALL.
+ * Set-up: CUDA loads the library's kernels and this array lazily (unless
+ * CUDA_MODULE_LOADING=EAGER), and loading commits device memory.  The first
+ * call on each device (any T, T = 0 included) does the set-up with that device
+ * current: it looks up the array's device address (cudaGetSymbolAddress) and
+ * loads every kernel the call launches.  So make one call on each device
+ * before entering the region that must not allocate, and before any stream
+ * capture; after it, calls allocate nothing.  No call synchronises.  The
+ * address is kept for the life of the process and does not survive
+ * cudaDeviceReset (after a reset, do not call this again in that process).
+ * All calls share the one array: calls that overlap on the GPU race on it and
+ * must be serialised by the caller. */
 moe_status moe_route_static(const moe_shape* shape, const void* X, const void* W_r, const float* bias,
                             int32_t* ids, float* gates, int32_t* status, void* stream);
 

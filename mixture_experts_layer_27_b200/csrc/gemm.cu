@@ -715,7 +715,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
 }
 
 template <int KIND>
-static cudaError_t launch_kind(const GemmParams& p, int grid, cudaStream_t st) {
+static cudaError_t configure_kind() {
   static bool configured[64] = {};  // the attribute is set once per device
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -725,8 +725,36 @@ static cudaError_t launch_kind(const GemmParams& p, int grid, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
+  return cudaSuccess;
+}
+
+template <int KIND>
+static cudaError_t launch_kind(const GemmParams& p, int grid, cudaStream_t st) {
+  const cudaError_t e = configure_kind<KIND>();
+  if (e != cudaSuccess) return e;
   k_moe_gemm<KIND><<<grid, GEMM_THREADS, smem_bytes<KIND>(), st>>>(p);
   return cudaGetLastError();
+}
+
+template <int KIND>
+static cudaError_t preload_kind() {
+  cudaFuncAttributes a;
+  const cudaError_t e = cudaFuncGetAttributes(&a, k_moe_gemm<KIND>);  // loads the kernel's module
+  return e != cudaSuccess ? e : configure_kind<KIND>();
+}
+
+cudaError_t preload_gemm(GemmKind kind) {
+  switch (kind) {
+    case G_GATEUP: return preload_kind<G_GATEUP>();
+    case G_DOWN: return preload_kind<G_DOWN>();
+    case G_DGRAD_DOWN: return preload_kind<G_DGRAD_DOWN>();
+    case G_DGRAD_GATEUP: return preload_kind<G_DGRAD_GATEUP>();
+    case G_WGRAD_GATEUP: return preload_kind<G_WGRAD_GATEUP>();
+    case G_WGRAD_DOWN: return preload_kind<G_WGRAD_DOWN>();
+    case G_ROUTER: return preload_kind<G_ROUTER>();
+    case G_ROUTER_WGRAD: return preload_kind<G_ROUTER_WGRAD>();
+  }
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream_t st) {

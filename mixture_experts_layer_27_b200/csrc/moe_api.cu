@@ -219,7 +219,7 @@ static EncodeTiledFn get_encode() {
 
 // 2-D bf16 tensor [outer, inner] (inner contiguous, row pitch in elements),
 // box {box_inner, box_outer}, 128-byte swizzle, zero fill out of bounds.
-static bool tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch_elems,
+bool tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch_elems,
                     uint32_t box_inner, uint32_t box_outer) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;
@@ -333,6 +333,30 @@ static cudaError_t timed(int kid, cudaStream_t st, F fn) {
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cudaError_t launch_router_logits(const Layout& L, const void* X, const __nv_bfloat16* wrt, float* rpart, int* status,
+                                 cudaStream_t st) {
+  const int splits = router_splits(L.T, L.E, L.d);
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!tmap_2d(&p.ta0, X, L.d, static_cast<uint64_t>(L.T), L.d, 64, 128) ||
+      !tmap_2d(&p.tb0, wrt, L.d, static_cast<uint64_t>(L.E), L.d, 64, 256))
+    return cudaErrorInvalidValue;
+  p.ta1 = p.ta0;
+  p.tb1 = p.tb0;
+  p.El = L.El;
+  p.d = L.d;
+  p.I = L.I;
+  p.T = static_cast<int>(L.T);
+  p.E = L.E;
+  p.splits = splits;
+  p.router_bn = router_tile_n(L.E);
+  p.outf = rpart;
+  p.status = status;
+  const int64_t tiles = ((L.T + 127) / 128) * ((L.E + 255) / 256) * splits;
+  const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
+  return launch_gemm(G_ROUTER, p, grid, st);
+}
 
 static GemmParams base_params(const Layout& L, const Ctx& c, int* status) {
   GemmParams p;
@@ -453,21 +477,7 @@ static moe_status route_tokens(const Layout& L, const Ctx& c, const void* X, con
     return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
   }));
   const int splits = router_splits(L.T, L.E, L.d);
-  {
-    GemmParams p = base_params(L, c, status);
-    MOE_TMAP(tmap_2d(&p.ta0, X, L.d, static_cast<uint64_t>(L.T), L.d, 64, 128));
-    MOE_TMAP(tmap_2d(&p.tb0, c.wrt, L.d, static_cast<uint64_t>(L.E), L.d, 64, 256));
-    p.ta1 = p.ta0;
-    p.tb1 = p.tb0;
-    p.T = static_cast<int>(L.T);
-    p.E = L.E;
-    p.splits = splits;
-    p.router_bn = router_tile_n(L.E);
-    p.outf = c.rpart;
-    const int64_t tiles = ((L.T + 127) / 128) * ((L.E + 255) / 256) * splits;
-    const int g = static_cast<int>(tiles < grid ? tiles : grid);
-    MOE_TRY(timed(K_ROUTER_LOGITS, st, [&] { return launch_gemm(G_ROUTER, p, g, st); }));
-  }
+  MOE_TRY(timed(K_ROUTER_LOGITS, st, [&] { return launch_router_logits(L, X, c.wrt, c.rpart, status, st); }));
   MOE_TRY(timed(K_TOPK, st, [&] { return launch_topk(L, c, bias, splits, st); }));
   if (L.scan_groups) MOE_TRY(timed(K_SCAN_GROUPS, st, [&] { return launch_scan_groups(L, c, st); }));
   MOE_TRY(timed(K_SCAN, st, [&] { return launch_scan(L, c, st); }));

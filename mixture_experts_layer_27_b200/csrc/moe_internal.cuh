@@ -145,6 +145,19 @@ constexpr int router_splits(int64_t T, int E, int d) {  // K splits of the route
 }
 
 cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream_t st);
+// Loads the kernel of one GEMM kind (and sets its shared-memory attribute) without launching it,
+// so that a later launch needs no lazy module loading.
+cudaError_t preload_gemm(GemmKind kind);
+
+// 2-D bf16 tensor map [outer, inner] (inner contiguous, row pitch in elements), box
+// {box_inner, box_outer}, 128-byte swizzle, zero fill out of bounds (moe_api.cu).
+bool tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch_elems,
+             uint32_t box_inner, uint32_t box_outer);
+// Router GEMM: the fp32 partial logits of its router_splits() fixed K splits into rpart
+// [splits, T, E], from X [T, d] and W_r^T [E, d] (moe_api.cu).  Shared by moe_fwd and the
+// allocation-free router entry point, so both run the same tiles in the same order.
+cudaError_t launch_router_logits(const Layout& L, const void* X, const __nv_bfloat16* wrt, float* rpart, int* status,
+                                 cudaStream_t st);
 
 // ---------------------------------------------------------------------------
 // MXFP8 grouped GEMMs (tcgen05 kind::mxf8f6f4 block_scale), see gemm_mx.cu
@@ -221,6 +234,8 @@ struct Ctx {  // typed views of ctx + ws for one shape
 Ctx make_ctx(const Layout& L, void* ctx, void* ws);
 
 cudaError_t launch_topk(const Layout& L, const Ctx& c, const float* bias, int splits, cudaStream_t st);
+// Loads the W_r transpose and top-k kernels without launching them (see preload_gemm).
+cudaError_t preload_router_kernels();
 cudaError_t launch_scan(const Layout& L, const Ctx& c, cudaStream_t st);
 cudaError_t launch_scan_groups(const Layout& L, const Ctx& c, cudaStream_t st);
 cudaError_t launch_scan_apply(const Layout& L, const Ctx& c, cudaStream_t st);

@@ -15,8 +15,18 @@
 // device) race on it, so serialise them.  It keeps the last call's contents;
 // every region a call reads is written earlier in that same call, so nothing
 // needs clearing between calls.
+//
+// Set-up: the library's kernels and this array are loaded lazily by CUDA (on
+// first use, unless CUDA_MODULE_LOADING=EAGER), and loading commits device
+// memory.  So the first call on each device does the set-up, with that device
+// current: it looks up the array's device address and loads every kernel the
+// call launches.  That first call therefore allocates; later calls do not.
+// Make it before entering the region that must not allocate, and before any
+// stream capture.  The device address is kept for the life of the process: it
+// does not survive cudaDeviceReset (or anything else that destroys the
+// device's primary context), after which this entry point must not be called
+// again in that process.
 #include <cstdint>
-#include <cstring>
 #include <mutex>
 
 #include "moe_internal.cuh"
@@ -35,8 +45,8 @@ void* g_scratch_dev[kMaxDevices] = {};  // device address of g_route_scratch, pe
 
 // In host code `g_route_scratch` names a host-side stand-in, not device memory:
 // the device address comes from cudaGetSymbolAddress, once per device, with
-// that device current.
-cudaError_t scratch_address(void** out) {
+// that device current.  The same set-up loads the kernels the call launches.
+cudaError_t setup_device(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -46,35 +56,14 @@ cudaError_t scratch_address(void** out) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_route_scratch);
     if (e != cudaSuccess) return e;
+    e = preload_router_kernels();
+    if (e != cudaSuccess) return e;
+    e = preload_gemm(G_ROUTER);
+    if (e != cudaSuccess) return e;
     g_scratch_dev[dev] = p;
   }
   *out = g_scratch_dev[dev];
   return cudaSuccess;
-}
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-                    uint32_t box_outer) {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {inner * 2};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }
@@ -104,7 +93,7 @@ extern "C" moe_status moe_route_static(const moe_shape* shape, const void* X, co
   if (need > MOE_STATIC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE_TOO_SMALL;
 
   void* base = nullptr;
-  if (scratch_address(&base) != cudaSuccess) return MOE_ERR_CUDA;
+  if (setup_device(&base) != cudaSuccess) return MOE_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (status && cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
   if (!tok) return MOE_OK;
@@ -120,26 +109,7 @@ extern "C" moe_status moe_route_static(const moe_shape* shape, const void* X, co
   c.hist = reinterpret_cast<int*>(s + o_hist);
 
   if (launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), wrt, st) != cudaSuccess) return MOE_ERR_CUDA;
-  GemmParams p;
-  std::memset(&p, 0, sizeof(p));
-  if (!encode_bf16_2d(&p.ta0, X, L.d, T, 64, 128) || !encode_bf16_2d(&p.tb0, wrt, L.d, E, 64, 256))
-    return MOE_ERR_CUDA;
-  p.ta1 = p.ta0;
-  p.tb1 = p.tb0;
-  p.d = L.d;
-  p.I = L.I;
-  p.El = L.El;
-  p.T = static_cast<int>(L.T);
-  p.E = L.E;
-  p.splits = splits;
-  p.router_bn = router_tile_n(L.E);
-  p.outf = c.rpart;
-  p.status = status;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t tiles = ((L.T + 127) / 128) * ((L.E + 255) / 256) * splits;
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  if (launch_gemm(G_ROUTER, p, grid, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_router_logits(L, X, wrt, c.rpart, status, st) != cudaSuccess) return MOE_ERR_CUDA;
   if (launch_topk(L, c, bias, splits, st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }

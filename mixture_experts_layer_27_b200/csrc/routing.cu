@@ -882,6 +882,17 @@ cudaError_t launch_topk(const Layout& L, const Ctx& c, const float* bias, int sp
                                                                 c.gates, c.hist, c.hdr + HDR_STATUS);
   return cudaGetLastError();
 }
+cudaError_t preload_router_kernels() {
+  cudaFuncAttributes a;
+  cudaError_t e = cudaSuccess;
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, k_transpose_wr);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, k_transpose_wr_v);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, k_topk<4>);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, k_topk<8>);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, k_topk<12>);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, k_topk<kMaxE / 32>);
+  return e;
+}
 cudaError_t launch_scan(const Layout& L, const Ctx& c, cudaStream_t st) {
   // over the group sums when the scan is two-level (launch_scan_groups before, _apply after)
   k_scan<<<1, 1024, 0, st>>>(L.scan_groups ? c.hsum : c.hist, L.scan_groups ? L.scan_groups : L.nblk, L.E, L.first,
