@@ -276,32 +276,53 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------
 # CPU oracle on a bounded sample (the baseline and the reference arm)
+#
+# One sample step = the fp64 oracle's forward + backward of the layer restricted to a window of
+# ORACLE_WINDOW consecutive local experts (every token routed, then those experts' assignments
+# through the SwiGLU experts and back, their weight gradients, the router gradient of their
+# tokens).  Its work in token units is the assignments it processed / top_k.  The rate is that
+# work over the measured time: nothing is extrapolated, and both CPU figures (cpu_baseline and
+# the reference arm) use this one sampler.
 # ----------------------------------------------------------------------------
-def oracle_sample(w: IN.Workload, x_cpu: dict, m: int) -> float:
-    """Seconds for the fp64 oracle: routing of all T tokens + fwd/bwd of experts [0, m)."""
+ORACLE_WINDOW = 8
+CPU_BASELINE_STEPS = 8
+
+
+def oracle_window(w: IN.Workload) -> tuple:
+    """(first local expert index, number) of the sampled window: the middle of the local experts."""
+    m = min(ORACLE_WINDOW, w.El)
+    return (w.El - m) // 2, m
+
+
+def oracle_sample(w: IN.Workload, x_cpu: dict) -> tuple:
+    """(seconds, assignments) of one oracle fwd+bwd over the sampled expert window."""
     import numpy as np
     import oracle as O
 
     def f64(t):
         return t.float().numpy().astype(np.float64)
 
+    e0, m = x_cpu["window"]
     X, Wr, dY = f64(x_cpu["X"]), f64(x_cpu["W_r"]), f64(x_cpu["dY"])
     b = None if x_cpu["bias"] is None else f64(x_cpu["bias"])
-    Wg, Wu, Wd = (f64(x_cpu[n][:m]) for n in ("W_gate", "W_up", "W_down"))
+    Wg, Wu, Wd = (f64(x_cpu[n]) for n in ("W_gate", "W_up", "W_down"))
+    first = w.first_local + e0
     t0 = time.perf_counter()
-    _, ctx = O.forward(X, Wr, b, lambda e: Wg[e - w.first_local], lambda e: Wu[e - w.first_local],
-                       lambda e: Wd[e - w.first_local], w.k, first_local=w.first_local, num_local=m)
+    _, ctx = O.forward(X, Wr, b, lambda e: Wg[e - first], lambda e: Wu[e - first], lambda e: Wd[e - first], w.k,
+                       first_local=first, num_local=m)
     O.backward(ctx, dY)
-    return time.perf_counter() - t0
+    dt = time.perf_counter() - t0
+    return dt, int(ctx["sched"]["offsets"][-1])
 
 
-def cpu_inputs(w: IN.Workload, m: int) -> dict:
+def cpu_inputs(w: IN.Workload) -> dict:
     """Host copies of the inputs the sample needs (CPU generator; same distributions)."""
+    e0, m = oracle_window(w)
     x = {"X": IN._normal((w.tokens, w.d), 1.0, IN._seed(w.seed, w.name, "X"), "cpu"),
          "W_r": IN._normal((w.d, w.E), 0.02, IN._seed(w.seed, w.name, "W_r"), "cpu"),
-         "dY": IN._normal((w.tokens, w.d), 1.0, IN._seed(w.seed, w.name, "dY"), "cpu")}
+         "dY": IN._normal((w.tokens, w.d), 1.0, IN._seed(w.seed, w.name, "dY"), "cpu"), "window": (e0, m)}
     for n in ("W_gate", "W_up", "W_down"):
-        x[n] = torch.stack([IN.expert_weights(w, n, w.first_local + e, "cpu") for e in range(m)])
+        x[n] = torch.stack([IN.expert_weights(w, n, w.first_local + e0 + e, "cpu") for e in range(m)])
     if w.zipf:
         x["bias"] = IN.zipf_bias(w, x["X"], x["W_r"])
     elif w.local_tokens:
@@ -322,18 +343,28 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
-def cpu_baseline(w: IN.Workload, m1: int = 4, m2: int = 8) -> dict:
-    m2 = min(m2, w.El)
-    m1 = min(m1, max(m2 // 2, 1))
-    x = cpu_inputs(w, m2)
-    t1 = oracle_sample(w, x, m1)
-    t2 = oracle_sample(w, x, m2)
-    per_expert = max(t2 - t1, 0.0) / (m2 - m1)
-    t_full = t1 + per_expert * (w.El - m1)
-    return {"value": w.tokens / t_full, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": (f"fp64 numpy oracle, all {w.tokens} tokens routed, fwd+bwd of {m1} and {m2} of {w.El} experts "
-                       f"({t1:.1f} s, {t2:.1f} s); time extrapolated linearly to {w.El} experts = {t_full:.1f} s "
-                       "per full fwd+bwd")}
+def oracle_rate(w: IN.Workload, x_cpu: dict, steps: int) -> dict:
+    """Times `steps` sample steps; the rate in tokens/s and the per-step times."""
+    ts, asg = [], []
+    for _ in range(steps):
+        dt, a = oracle_sample(w, x_cpu)
+        ts.append(dt)
+        asg.append(a)
+    tokens = sum(asg) / w.k
+    e0, m = x_cpu["window"]
+    return {"value": tokens / sum(ts), "seconds": ts, "assignments": asg[0],
+            "sample": (f"fp64 numpy oracle, measured (no extrapolation): each step routes all {w.tokens} tokens and "
+                       f"runs forward + backward of local experts {e0}..{e0 + m - 1} ({asg[0]} of the "
+                       f"{w.tokens * w.k if w.El == w.E else 'local'} assignments, weight gradients included); "
+                       f"rate = assignments / top_k / measured time over {steps} steps "
+                       f"({statistics.mean(ts):.2f} s per step)")}
+
+
+def cpu_baseline(w: IN.Workload) -> dict:
+    x = cpu_inputs(w)
+    oracle_sample(w, x)  # first call: imports, BLAS start-up
+    r = oracle_rate(w, x, CPU_BASELINE_STEPS)
+    return {"value": r["value"], "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle", "sample": r["sample"]}
 
 
 # ----------------------------------------------------------------------------
@@ -375,25 +406,18 @@ def barrier(world: int):
 def run_reference(args, w: IN.Workload, world: int, rank: int):
     if rank != 0:
         return
-    x = cpu_inputs(w, 4)
+    x = cpu_inputs(w)
     for _ in range(args.warmup):
-        oracle_sample(w, x, 1)
-    ts = [oracle_sample(w, x, 2) for _ in range(args.steps)]
-    # each step: routing of all tokens + 2 experts' fwd+bwd; the per-expert cost is
-    # measured once more with 4 experts and the step time extrapolated to all experts
-    t4 = oracle_sample(w, x, 4)
-    t2 = statistics.median(ts)
-    t_full = t2 + max(t4 - t2, 0.0) / 2 * (w.El - 2)
-    value = w.tokens / t_full
-    cores = blas_threads()
-    sample = (f"fp64 numpy oracle per step: all {w.tokens} tokens routed + fwd/bwd of 2 of {w.El} experts "
-              f"(median {t2:.2f} s over {args.steps} steps); per-expert cost from a 4-expert run, "
-              f"extrapolated to {w.El} experts = {t_full:.1f} s per layer fwd+bwd")
+        oracle_sample(w, x)
+    r = oracle_rate(w, x, args.steps)
+    value = r["value"]
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": t_full * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(w),
+            "warmup": args.warmup, "ms_per_step": statistics.mean(r["seconds"]) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict(workload_config(w), wgrad_dtype="fp32" if args.wgrad_fp32 else "bf16"),
             "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": r["sample"]},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
