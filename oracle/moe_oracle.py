@@ -476,31 +476,57 @@ def mx_round(v, axis: int):
     return mx_dequantize(c, s, axis=axis)
 
 
-def forward_mx(X, W_r, bias, W_gate, W_up, W_down, top_k: int):
+def mx_weight_layouts(Wg, Wu, Wd) -> dict:
+    """One expert's weights rounded for each GEMM that reads them, along its contraction:
+
+    gate_d, up_d   W_gate, W_up [d, I] along d   (forward gate/up GEMM, K = d)
+    down_i         W_down [I, d] along I         (forward down GEMM, K = I)
+    down_d         W_down [I, d] along d         (dgrad of W_down, K = d)
+    gate_i, up_i   W_gate, W_up [d, I] along I   (dgrad of gate/up, K = I)
+    """
+    Wg, Wu, Wd = _f64(Wg), _f64(Wu), _f64(Wd)
+    return dict(gate_d=mx_round(Wg, axis=0), up_d=mx_round(Wu, axis=0), down_i=mx_round(Wd, axis=0),
+                down_d=mx_round(Wd, axis=1), gate_i=mx_round(Wg, axis=1), up_i=mx_round(Wu, axis=1))
+
+
+def _layouts(rounded, W_gate, W_up, W_down, e: int) -> dict:
+    """Rounded weights of expert e: from the caller's `rounded(e)` (e.g. a cache), else computed."""
+    if rounded is not None:
+        return {k: _f64(v) for k, v in rounded(e).items()}
+    return mx_weight_layouts(_expert(W_gate, e), _expert(W_up, e), _expert(W_down, e))
+
+
+def forward_mx(X, W_r, bias, W_gate, W_up, W_down, top_k: int, first_local: int = 0, num_local: int | None = None,
+               rounded=None):
+    """MXFP8 layer forward (experts [first_local, first_local + num_local) as in forward).
+
+    rounded: optional callable e -> mx_weight_layouts of expert e (the same values, computed
+    once by the caller); without it the weights are rounded here."""
     X64 = _f64(X)
     T, d = X64.shape
     E = np.asarray(W_r).shape[1]
     logits = router_logits(X64, W_r, bias)
     ids = topk_ids(logits, top_k)
     g = gates(logits, ids)
-    sched = schedule(ids, E)
+    sched = schedule(ids, E, first_local, num_local)
     Y = np.zeros((T, d))
     saved = []
-    for e in range(E):
-        toks, slots = _expert_rows(ids, sched, e)
+    for el in range(sched["num_local"]):
+        toks, slots = _expert_rows(ids, sched, el)
         if toks.size == 0:
             saved.append(None)
             continue
+        Wq = _layouts(rounded, W_gate, W_up, W_down, el + sched["first_local"])
         Xq = mx_round(X64[toks], axis=1)  # K = d
-        A = Xq @ mx_round(_expert(W_gate, e), axis=0)
-        B = Xq @ mx_round(_expert(W_up, e), axis=0)
+        A = Xq @ Wq["gate_d"]
+        B = Xq @ Wq["up_d"]
         H = silu(A) * B
-        O = mx_round(H, axis=1) @ mx_round(_expert(W_down, e), axis=0)  # K = I
+        O = mx_round(H, axis=1) @ Wq["down_i"]  # K = I
         ge = g[toks, slots]
         Y[toks] += ge[:, None] * O
         saved.append((toks, slots, A, B))
     ctx = dict(X=X64, W_r=_f64(W_r), W_gate=W_gate, W_up=W_up, W_down=W_down, logits=logits, ids=ids, g=g,
-               sched=sched, saved=saved, E=E)
+               sched=sched, saved=saved, E=E, rounded=rounded)
     return Y, ctx
 
 
@@ -513,24 +539,25 @@ def backward_mx(ctx, dY):
     dX = np.zeros((T, d))
     dg = np.zeros((T, k))
     dW_gate, dW_up, dW_down = {}, {}, {}
-    for e in range(E):
-        Wg, Wu, Wd = _expert(ctx["W_gate"], e), _expert(ctx["W_up"], e), _expert(ctx["W_down"], e)
-        item = ctx["saved"][e]
+    for el in range(sched["num_local"]):
+        e = el + sched["first_local"]
+        item = ctx["saved"][el]
         if item is None:
-            I = Wg.shape[1]
+            I = np.asarray(_expert(ctx["W_gate"], e)).shape[1]
             dW_gate[e] = np.zeros((d, I)); dW_up[e] = np.zeros((d, I)); dW_down[e] = np.zeros((I, d))
             continue
+        Wq = _layouts(ctx.get("rounded"), ctx["W_gate"], ctx["W_up"], ctx["W_down"], e)
         toks, slots, A, B = item
         Xe = X64[toks]
         ge = g[toks, slots]
         dYe = dY64[toks]
         H = silu(A) * B
-        dHp = mx_round(dYe, axis=1) @ mx_round(Wd, axis=1).T  # K = d
+        dHp = mx_round(dYe, axis=1) @ Wq["down_d"].T  # K = d
         dg[toks, slots] = np.sum(dHp * H, axis=1)
         dH = ge[:, None] * dHp
         dA = dH * B * silu_grad(A)
         dB = dH * silu(A)
-        dX[toks] += mx_round(dA, axis=1) @ mx_round(Wg, axis=1).T + mx_round(dB, axis=1) @ mx_round(Wu, axis=1).T
+        dX[toks] += mx_round(dA, axis=1) @ Wq["gate_i"].T + mx_round(dB, axis=1) @ Wq["up_i"].T  # K = I
         dW_gate[e] = Xe.T @ dA
         dW_up[e] = Xe.T @ dB
         dW_down[e] = H.T @ (ge[:, None] * dYe)
@@ -539,3 +566,38 @@ def backward_mx(ctx, dY):
     np.put_along_axis(dl, ids.astype(np.int64), g * (dg - s), axis=1)
     dX += dl @ ctx["W_r"].T
     return dict(dX=dX, dW_gate=dW_gate, dW_up=dW_up, dW_down=dW_down, dW_r=X64.T @ dl, dl=dl, dg=dg)
+
+
+def token_forward_backward_mx(t: int, X, W_r, bias, rounded, top_k: int, dY):
+    """Y_t, dX_t and dl_t of the MXFP8 layer for one token (all experts local).
+
+    The same steps as forward_mx / backward_mx on one row: every activation is rounded
+    along its own row (d or I), so a token's results depend on its data alone.
+    rounded: callable e -> mx_weight_layouts of expert e."""
+    x = _f64(X)[t:t + 1]
+    E = np.asarray(W_r).shape[1]
+    l = router_logits(x, W_r, bias)
+    ids = topk_ids(l, top_k)
+    g = gates(l, ids)[0]
+    dy = _f64(dY)[t:t + 1]
+    y = np.zeros(x.shape[1])
+    dx = np.zeros(x.shape[1])
+    dg = np.zeros(top_k)
+    xq = mx_round(x, axis=1)
+    dyq = mx_round(dy, axis=1)
+    for j, e in enumerate(ids[0]):
+        Wq = {k: _f64(v) for k, v in rounded(int(e)).items()}
+        a = xq @ Wq["gate_d"]
+        b = xq @ Wq["up_d"]
+        h = silu(a) * b
+        y += g[j] * (mx_round(h, axis=1) @ Wq["down_i"])[0]
+        dhp = dyq @ Wq["down_d"].T
+        dg[j] = float(np.sum(dhp * h))
+        dh = g[j] * dhp
+        da = dh * b * silu_grad(a)
+        db = dh * silu(a)
+        dx += (mx_round(da, axis=1) @ Wq["gate_i"].T + mx_round(db, axis=1) @ Wq["up_i"].T)[0]
+    dl = np.zeros(E)
+    dl[ids[0]] = g * (dg - np.sum(g * dg))
+    dx += dl @ _f64(W_r).T
+    return y, dx, dl, ids[0], g

@@ -545,3 +545,29 @@ def test_mx_layer_worked_example_by_hand():
             want[r, c] = v
         np.testing.assert_allclose(got[name], want, rtol=1e-13, atol=0, err_msg=name)
     assert not np.any(g["dW_r"])
+
+
+def test_mx_token_path_and_slices_equal_the_full_mx_layer():
+    # token_forward_backward_mx is the MX layer on one row; forward_mx / backward_mx over expert
+    # slices add up to the full layer; precomputed weight layouts give the same numbers.
+    X, W_r, Wg, Wu, Wd, dY = _mx_case(41)
+    k, E = _MX_SHAPE["k"], _MX_SHAPE["E"]
+    Y, ctx, g = _mx_run(X, W_r, Wg, Wu, Wd, dY)
+    cache = {e: O.mx_weight_layouts(Wg[e], Wu[e], Wd[e]) for e in range(E)}
+    for t in (0, 17, 95):
+        y, dx, dl, ids, gt = O.token_forward_backward_mx(t, X, W_r, None, cache.__getitem__, k, dY)
+        np.testing.assert_allclose(y, Y[t], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(dx, g["dX"][t], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(dl, g["dl"][t], rtol=1e-12, atol=1e-14)
+    Ys, dXs, dls = np.zeros_like(Y), np.zeros_like(X), np.zeros_like(g["dl"])
+    for e in range(E):
+        Ye, ce = O.forward_mx(X, W_r, None, Wg, Wu, Wd, k, first_local=e, num_local=1, rounded=cache.__getitem__)
+        ge = O.backward_mx(ce, dY)
+        Ys += Ye
+        dXs += ge["dX"] - ge["dl"] @ W_r.T  # expert parts; the router term once below
+        dls += ge["dl"]
+        for n in ("dW_gate", "dW_up", "dW_down"):
+            np.testing.assert_allclose(ge[n][e], g[n][e], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(Ys, Y, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(dls, g["dl"], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(dXs + dls @ W_r.T, g["dX"], rtol=1e-10, atol=1e-12)
