@@ -47,3 +47,35 @@ def run_oracle(x, k, first=0, num=None):
     Wg, Wu, Wd = to64(x["W_gate"]), to64(x["W_up"]), to64(x["W_down"])
     Y, ctx = O.forward(X, Wr, b, Wg, Wu, Wd, k, first_local=first, num_local=num)
     return Y, ctx, O.backward(ctx, dY)
+
+
+def mx_layout_job(args):
+    """Worker of a spawned process pool: one MX-rounded weight layout of one expert.
+
+    args = (expert, layout name, float32 weight, axis); returns (expert, name, float32 layout).
+    The rounded values (E4M3 times a power of two) are exact in float32."""
+    e, name, W, axis = args
+    return e, name, O.mx_round(np.asarray(W, dtype=np.float64), axis).astype(np.float32)
+
+
+# the six layouts of oracle.mx_weight_layouts: (name, weight, axis)
+MX_LAYOUTS = (("gate_d", "W_gate", 0), ("up_d", "W_up", 0), ("down_i", "W_down", 0),
+              ("down_d", "W_down", 1), ("gate_i", "W_gate", 1), ("up_i", "W_up", 1))
+
+
+def mx_layout_cache(experts, weights, processes=8) -> dict:
+    """{expert: {layout: float32 array}} for `experts`, rounded in a spawned pool.
+
+    weights: dict name -> callable e -> fp64 weight (host).  The pool is started with
+    'spawn', so it is safe after CUDA has been initialised in this process."""
+    import multiprocessing as mp
+    from concurrent.futures import ProcessPoolExecutor
+    out = {int(e): {} for e in experts}
+    # a worker that dies raises BrokenProcessPool here (no silent respawning)
+    with ProcessPoolExecutor(max_workers=processes, mp_context=mp.get_context("spawn")) as pool:
+        futs = [pool.submit(mx_layout_job, (int(e), ln, weights[wn](e).astype(np.float32), ax))
+                for e in experts for ln, wn, ax in MX_LAYOUTS]
+        for f in futs:
+            e, ln, arr = f.result(timeout=600)
+            out[e][ln] = arr
+    return out
