@@ -41,12 +41,24 @@ template <int KIND>
 constexpr bool is_wgrad() { return KIND == G_WGRAD_GATEUP || KIND == G_WGRAD_DOWN; }
 template <int KIND>
 constexpr int stages_of() { return is_wgrad<KIND>() ? 3 : GEMM_STAGES; }
+// With SCHED, the tiles a CTA works on are decoded once, by a scheduler warp, into a ring of
+// SCHED_DEPTH entries that the producer, the MMA issuer and the epilogue warps read in order
+// (the ring is deeper than the producer runs ahead of the epilogue, so it never throttles it).
+// That takes the decode's global-load latency off the epilogue's path, which is the critical
+// one in a weight-gradient GEMM whose tiles have one or two K blocks (64 tokens per expert:
+// the kernel is bound by its gradient stores).  Where tiles have many K blocks the MMA issuer
+// and the producer are critical, and there every role decodes its own tiles (measured 2-10%
+// faster than the ring for the long-K weight gradients and the other kinds).
+constexpr int SCHED_DEPTH = 8;
+constexpr size_t SCHED_TAIL_BYTES = 1024;  // barriers, TMEM slot and the tile ring
 template <int KIND>
 constexpr size_t smem_bytes() {
-  return stages_of<KIND>() * GEMM_STAGE_BYTES + (is_wgrad<KIND>() ? GEMM_STAGE_OUT_BYTES : 0) + 1024 + 256;
+  return stages_of<KIND>() * GEMM_STAGE_BYTES + (is_wgrad<KIND>() ? GEMM_STAGE_OUT_BYTES : 0) + 1024 +
+         SCHED_TAIL_BYTES;
 }
 
 struct Tile {
+  int t;    // tile index; -1 marks the end of this CTA's tiles
   int m;    // macrobatch (wgrad: first macrobatch of the chunk)
   int shift;  // row shift of the X_perm operand (ring position) / wgrad: last macrobatch + 1
   int el;   // local expert
@@ -111,6 +123,7 @@ __device__ __forceinline__ int router_wgrad_kblocks(const GemmParams& p) {
 template <int KIND>
 __device__ __forceinline__ Tile decode(const GemmParams& p, int t) {
   Tile tl;
+  tl.t = t;
   if constexpr (KIND == G_ROUTER) {
     // tile = (m-tile, n-tile, K split); the splits of one output tile are adjacent
     const int S = p.splits, NTr = (p.E + 255) / 256, KB = p.d / 64;
@@ -422,7 +435,8 @@ __device__ __forceinline__ void epilogue_wgrad(const GemmParams& p, const Tile& 
   // The warp's 16 KB staging slice holds four boxes.  Each box is staged, stored and committed
   // as its own bulk group, and a box slot is refilled once the store issued from it one tile
   // (bf16) or half a tile (fp32) earlier has been read: all but the 3 newest groups.  So the
-  // TMA engine drains box b while the warp converts box b+1.
+  // TMA engine drains box b while the warp converts box b+1.  (Stores of two or four adjacent
+  // boxes at once, through a 3-D map, measured slower: fewer stores, less overlap.)
   if (mode == 0 && !p.wout32) {
     // TMEM loads pipelined one box ahead: box b+1's load is in flight while box b is converted
     uint32_t r[2][64];
@@ -514,8 +528,33 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   }
 }
 
-template <int KIND>
-__global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_constant__ GemmParams p) {
+// The next tile of this CTA from the scheduler's ring (the producer and the MMA issuer: one
+// thread each).  Returns false on a device error; the tile with t = -1 ends the loop.
+__device__ __forceinline__ bool next_tile(const Tile* ring, uint64_t* sfull, uint64_t* sempty, int j, Tile& tl,
+                                          int* status) {
+  const int slot = j % SCHED_DEPTH;
+  if (!mbar_wait(&sfull[slot], (j / SCHED_DEPTH) & 1, status)) return false;
+  tl = ring[slot];
+  mbar_arrive(&sempty[slot]);
+  return true;
+}
+// The j-th tile of this CTA: from the scheduler's ring, or decoded here for kinds without it.
+template <int KIND, bool SCHED>
+__device__ __forceinline__ bool role_tile(const GemmParams& p, const Tile* ring, uint64_t* sfull, uint64_t* sempty,
+                                          int j, int ntiles, Tile& tl) {
+  if constexpr (SCHED) {
+    return next_tile(ring, sfull, sempty, j, tl, p.status);
+  } else {
+    const int t = blockIdx.x + j * gridDim.x;
+    if (t < ntiles) tl = decode<KIND>(p, t);
+    else tl.t = -1;
+    return true;
+  }
+}
+
+template <int KIND, bool SCHED>
+__global__ void __launch_bounds__(SCHED ? GEMM_THREADS_SCHED : GEMM_THREADS, 1)
+    k_moe_gemm(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int STAGES = stages_of<KIND>();
@@ -525,7 +564,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sfull = drain + 1;  // scheduler ring: entry written / entry read by every role
+  uint64_t* sempty = sfull + SCHED_DEPTH;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sempty + SCHED_DEPTH);
+  Tile* ring = reinterpret_cast<Tile*>(sempty + SCHED_DEPTH + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -538,6 +580,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
       mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
+    for (int s = 0; s < SCHED_DEPTH; ++s) {
+      mbar_init(&sfull[s], 1);
+      mbar_init(&sempty[s], 6);  // producer, MMA issuer, four epilogue warps
+    }
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -554,10 +600,26 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const int ntiles = num_tiles<KIND>(p);
   constexpr uint32_t IDESC = idesc_bf16(GEMM_BM, GEMM_BN, Traits<KIND>::A_MN, Traits<KIND>::B_MN);
+  const int ntiles = SCHED ? 0 : num_tiles<KIND>(p);
 
-  if (warp == 0) {
+  if (warp == 6) {
+    if (SCHED && lane == 0) {
+      // ---------------- scheduler: this CTA's tiles, decoded ahead of the roles ----------------
+      const int nt_all = num_tiles<KIND>(p);
+      for (int t = blockIdx.x, j = 0;; t += gridDim.x, ++j) {
+        const int slot = j % SCHED_DEPTH;
+        if (!mbar_wait(&sempty[slot], ((j / SCHED_DEPTH) & 1) ^ 1, p.status)) break;
+        if (t < nt_all) {
+          ring[slot] = decode<KIND>(p, t);
+        } else {
+          ring[slot].t = -1;
+        }
+        mbar_arrive(&sfull[slot]);
+        if (t >= nt_all) break;
+      }
+    }
+  } else if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       const uint64_t pol_act = policy_evict_last();
@@ -567,8 +629,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
       int last_parity[STAGES];
       for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const Tile tl = decode<KIND>(p, t);
+      for (int j = 0; ok; ++j) {
+        Tile tl;
+        if (!role_tile<KIND, SCHED>(p, ring, sfull, sempty, j, ntiles, tl)) { ok = false; break; }
+        if (tl.t < 0) break;
         if constexpr (is_wgrad<KIND>()) {
           // K runs over the expert's rows in each macrobatch of the chunk, in order
           for (int m = tl.m; m < tl.shift && ok; ++m) {
@@ -608,9 +672,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int it = 0;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
-        const Tile tl = decode<KIND>(p, t);
+      for (int it = 0; ok; ++it) {
+        Tile tl;
+        if (!role_tile<KIND, SCHED>(p, ring, sfull, sempty, it, ntiles, tl)) { ok = false; break; }
+        if (tl.t < 0) break;
         const int acc = it & 1;
         const uint32_t accp = (it >> 1) & 1;
         if (!mbar_wait(&tempty[acc], accp ^ 1, p.status)) { ok = false; break; }
@@ -645,9 +710,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int it = 0;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
-        const Tile tl = decode<KIND>(p, t);
+      for (int it = 0; ok; ++it) {
+        Tile tl;
+        if (!role_tile<KIND, SCHED>(p, ring, sfull, sempty, it, ntiles, tl)) { ok = false; break; }
+        if (tl.t < 0) break;
         const int acc = it & 1;
         const uint32_t accp = (it >> 1) & 1;
         if (!mbar_wait(&tempty[acc], accp ^ 1, p.status)) { ok = false; break; }
@@ -677,16 +743,30 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
       umma_commit(drain);  // all MMAs issued by this thread are complete once this lands
       mbar_wait_drain(drain, 0);
     }
-  } else {
+  } else if (warp >= 2 && warp <= 5) {
     // ---------------- epilogue warps 2..5 ----------------
     const int quarter = warp & 3;  // TMEM lanes this warp may access: 32*quarter ..
     const int row = quarter * 32 + lane;
-    int it = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
-      const Tile tl = decode<KIND>(p, t);
+    for (int it = 0;; ++it) {
+      int ok = 1;
+      Tile tl;
+      if constexpr (SCHED) {
+        const int slot = it % SCHED_DEPTH;
+        if (lane == 0) ok = mbar_wait(&sfull[slot], (it / SCHED_DEPTH) & 1, p.status) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        __syncwarp();  // lane 0's acquire of the entry, then every lane reads it
+        tl = ring[slot];
+        __syncwarp();  // every lane has read the entry before lane 0 releases it
+        if (lane == 0) mbar_arrive(&sempty[slot]);
+      } else {
+        const int t = blockIdx.x + it * gridDim.x;
+        if (t >= ntiles) break;
+        tl = decode<KIND>(p, t);
+      }
+      if (tl.t < 0) break;
       const int acc = it & 1;
       const uint32_t accp = (it >> 1) & 1;
-      int ok = 1;
       if (lane == 0) ok = mbar_wait(&tfull[acc], accp, p.status) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
@@ -714,13 +794,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm(const __grid_const
   }
 }
 
-template <int KIND>
+template <int KIND, bool SCHED>
 static cudaError_t configure_kind() {
   static bool configured[64] = {};  // the attribute is set once per device
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(k_moe_gemm<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const cudaError_t e = cudaFuncSetAttribute(k_moe_gemm<KIND, SCHED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem_bytes<KIND>()));
     if (e != cudaSuccess) return e;
     configured[dev] = true;
@@ -728,19 +808,19 @@ static cudaError_t configure_kind() {
   return cudaSuccess;
 }
 
-template <int KIND>
+template <int KIND, bool SCHED = false>
 static cudaError_t launch_kind(const GemmParams& p, int grid, cudaStream_t st) {
-  const cudaError_t e = configure_kind<KIND>();
+  const cudaError_t e = configure_kind<KIND, SCHED>();
   if (e != cudaSuccess) return e;
-  k_moe_gemm<KIND><<<grid, GEMM_THREADS, smem_bytes<KIND>(), st>>>(p);
+  k_moe_gemm<KIND, SCHED><<<grid, SCHED ? GEMM_THREADS_SCHED : GEMM_THREADS, smem_bytes<KIND>(), st>>>(p);
   return cudaGetLastError();
 }
 
 template <int KIND>
 static cudaError_t preload_kind() {
   cudaFuncAttributes a;
-  const cudaError_t e = cudaFuncGetAttributes(&a, k_moe_gemm<KIND>);  // loads the kernel's module
-  return e != cudaSuccess ? e : configure_kind<KIND>();
+  const cudaError_t e = cudaFuncGetAttributes(&a, k_moe_gemm<KIND, false>);  // loads the kernel's module
+  return e != cudaSuccess ? e : configure_kind<KIND, false>();
 }
 
 cudaError_t preload_gemm(GemmKind kind) {
@@ -757,14 +837,16 @@ cudaError_t preload_gemm(GemmKind kind) {
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream_t st) {
+cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream_t st, bool sched) {
   switch (kind) {
     case G_GATEUP: return launch_kind<G_GATEUP>(p, grid, st);
     case G_DOWN: return launch_kind<G_DOWN>(p, grid, st);
     case G_DGRAD_DOWN: return launch_kind<G_DGRAD_DOWN>(p, grid, st);
     case G_DGRAD_GATEUP: return launch_kind<G_DGRAD_GATEUP>(p, grid, st);
-    case G_WGRAD_GATEUP: return launch_kind<G_WGRAD_GATEUP>(p, grid, st);
-    case G_WGRAD_DOWN: return launch_kind<G_WGRAD_DOWN>(p, grid, st);
+    case G_WGRAD_GATEUP:
+      return sched ? launch_kind<G_WGRAD_GATEUP, true>(p, grid, st) : launch_kind<G_WGRAD_GATEUP>(p, grid, st);
+    case G_WGRAD_DOWN:
+      return sched ? launch_kind<G_WGRAD_DOWN, true>(p, grid, st) : launch_kind<G_WGRAD_DOWN>(p, grid, st);
     case G_ROUTER: return launch_kind<G_ROUTER>(p, grid, st);
     case G_ROUTER_WGRAD: return launch_kind<G_ROUTER_WGRAD>(p, grid, st);
   }

@@ -564,9 +564,13 @@ static moe_status router_backward(const Layout& L, const Ctx& c, const void* X, 
 
 // Expert weight gradients from the saved X_perm and the backward's dA, dB, Hg, dY_perm:
 // gate/up, then down (write-bound; separate launches keep the HBM traffic one-directional).
+// With at most 256 rows per expert on average (four 64-row K blocks) a tile's MMAs are short
+// and the gradient stores of the epilogue set the pace: the tiles are then decoded ahead by a
+// scheduler warp (launch_gemm's sched flag).
 static moe_status launch_wgrads(const Layout& L, const Ctx& c, int* status, void* dW_gate, void* dW_up,
                                 void* dW_down, cudaStream_t st) {
   const int grid = num_sms();
+  const bool sched = L.M == 0 && L.T * L.k <= 256LL * L.E;
   const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
   {
     GemmParams p = base_params(L, c, status);
@@ -576,7 +580,7 @@ static moe_status launch_wgrads(const Layout& L, const Ctx& c, int* status, void
     MOE_TMAP(tmap_wgrad_out(L, &p.to0, dW_gate, L.I, El * L.d));
     MOE_TMAP(tmap_wgrad_out(L, &p.to1, dW_up, L.I, El * L.d));
     p.ta1 = p.ta0;
-    MOE_TRY(timed(K_GEMM_WGRAD_GATEUP, st, [&] { return launch_gemm(G_WGRAD_GATEUP, p, grid, st); }));
+    MOE_TRY(timed(K_GEMM_WGRAD_GATEUP, st, [&] { return launch_gemm(G_WGRAD_GATEUP, p, grid, st, sched); }));
   }
   {
     GemmParams p = base_params(L, c, status);
@@ -586,7 +590,7 @@ static moe_status launch_wgrads(const Layout& L, const Ctx& c, int* status, void
     p.to1 = p.to0;
     p.ta1 = p.ta0;
     p.tb1 = p.tb0;
-    MOE_TRY(timed(K_GEMM_WGRAD_DOWN, st, [&] { return launch_gemm(G_WGRAD_DOWN, p, grid, st); }));
+    MOE_TRY(timed(K_GEMM_WGRAD_DOWN, st, [&] { return launch_gemm(G_WGRAD_DOWN, p, grid, st, sched); }));
   }
   return MOE_OK;
 }

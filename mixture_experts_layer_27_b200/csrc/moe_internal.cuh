@@ -128,7 +128,8 @@ struct GemmParams {
 };
 
 constexpr int GEMM_BM = 128, GEMM_BN = 256, GEMM_BK = 64, GEMM_STAGES = 4;
-constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_THREADS = 192;        // six role warps: producer, MMA issuer, four epilogue warps
+constexpr int GEMM_THREADS_SCHED = 224;  // the same plus a tile scheduler warp
 constexpr size_t GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;
 constexpr size_t GEMM_B_BYTES = GEMM_BN * GEMM_BK * 2;
 constexpr size_t GEMM_STAGE_BYTES = GEMM_A_BYTES + GEMM_B_BYTES;
@@ -144,7 +145,10 @@ constexpr int router_splits(int64_t T, int E, int d) {  // K splits of the route
   return static_cast<int>(s);
 }
 
-cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream_t st);
+// sched: the weight-gradient kinds can decode their tiles in a scheduler warp ahead of the
+// roles (worth it when tiles have few K blocks and the epilogue is the critical path); other
+// kinds ignore it.
+cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream_t st, bool sched = false);
 // Loads the kernel of one GEMM kind (and sets its shared-memory attribute) without launching it,
 // so that a later launch needs no lazy module loading.
 cudaError_t preload_gemm(GemmKind kind);
