@@ -111,6 +111,10 @@ __device__ __forceinline__ void mx_load(const MxParams& p, const MxTile& tl, int
 }
 
 __device__ __forceinline__ float mx_sigmoid(float a) { return 1.0f / (1.0f + expf(-a)); }
+// silu(a) = a / (1 + e^-a) with the fast exponential and reciprocal intrinsics: its result only
+// feeds H, which is rounded to E4M3 (3 mantissa bits) for the down GEMM, and the intrinsics'
+// errors are a few ulp of fp32.
+__device__ __forceinline__ float mx_silu_fast(float a) { return a * __frcp_rn(1.0f + __expf(-a)); }
 
 __device__ __forceinline__ void mx_store_bf16_32(__nv_bfloat16* dst, const float (&v)[32]) {
   uint4* d4 = reinterpret_cast<uint4*>(dst);
@@ -143,21 +147,24 @@ __device__ __forceinline__ void mx_store_q32(uint8_t* q, uint8_t* qs, int R, int
 
 // Rows past a segment's live pad rows (row_asg == ROW_DEAD) store nothing: no later kernel
 // reads them.
+// [cbeg, cend): this warp's share of the accumulator's 32-column chunks (all of them, or half
+// when two warps share a TMEM lane quarter).
 template <int KIND>
-__device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl, int row, uint32_t taddr) {
+__device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl, int row, uint32_t taddr, int cbeg,
+                                            int cend) {
   const int R = tl.m0 + row;
   const size_t Rz = static_cast<size_t>(R);
   const bool live = __ldg(p.row_asg + R) != ROW_DEAD;
   constexpr int BN = mx_bn(KIND);
   if constexpr (KIND == MX_GATEUP) {
 #pragma unroll 1
-    for (int c = 0; c < BN / 64; ++c) {  // accumulator columns: [64 gate | 64 up] per 128
+    for (int c = cbeg; c < cend; ++c) {  // 32 H columns each; accumulator: [64 gate | 64 up] per 128
       const int j = c >> 1, c32 = (c & 1) * 32;
       float a[32], b[32], h[32];
       tmem_ld32(taddr + j * 128 + c32, a);       // gate
       tmem_ld32(taddr + j * 128 + 64 + c32, b);  // up
 #pragma unroll
-      for (int i = 0; i < 32; ++i) h[i] = a[i] * mx_sigmoid(a[i]) * b[i];
+      for (int i = 0; i < 32; ++i) h[i] = mx_silu_fast(a[i]) * b[i];
       const int col = tl.n0 + j * 64 + c32;
       if (live) {
         mx_store_bf16_32(p.out0 + Rz * p.I + col, a);
@@ -168,7 +175,7 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
   } else if constexpr (KIND == MX_DOWN) {
     const float g = p.row_gate[R];
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = cbeg; c < cend; ++c) {
       float o[32];
       tmem_ld32(taddr + c * 32, o);
 #pragma unroll
@@ -212,7 +219,7 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
     if (live) p.outf[Rz * (p.I / BN) + tl.nt] = dg;
   } else {
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = cbeg; c < cend; ++c) {
       float v[32];
       tmem_ld32(taddr + c * 32, v);
       if (live) mx_store_bf16_32(p.out0 + Rz * p.d + tl.n0 + c * 32, v);
@@ -228,8 +235,8 @@ __device__ __forceinline__ void mx_wait_drain(uint64_t* bar, uint32_t parity) {
 }
 
 template <int KIND>
-__global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm_mx(const __grid_constant__ MxParams p) {
-  constexpr int BN = mx_bn(KIND), ACCS = mx_accs(KIND), STAGES = mx_stages(KIND);
+__global__ void __launch_bounds__(mx_threads(KIND), 1) k_moe_gemm_mx(const __grid_constant__ MxParams p) {
+  constexpr int BN = mx_bn(KIND), ACCS = mx_accs(KIND), STAGES = mx_stages(KIND), EPI = mx_epi_warps(KIND);
   constexpr size_t SB = mx_stage_bytes(KIND);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -247,7 +254,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm_mx(const __grid_co
     }
     for (int a = 0; a < ACCS; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
+      mbar_init(&tempty[a], EPI);  // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -329,9 +336,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm_mx(const __grid_co
       umma_commit(drain);
       mx_wait_drain(drain, 0);
     }
-  } else {  // epilogue warps 2..5
+  } else {  // epilogue warps 2 .. 2 + EPI - 1
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
+    constexpr int NCH = KIND == MX_GATEUP ? BN / 64 : BN / 32;  // 32-column chunks of the epilogue
+    const int half = EPI == 8 ? (warp - 2) >> 2 : 0;
+    const int cbeg = half * (NCH * 4 / EPI), cend = cbeg + NCH * 4 / EPI;
     int it = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
       const MxTile tl = mx_decode<KIND>(p, t);
@@ -343,7 +353,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_moe_gemm_mx(const __grid_co
       if (!ok) break;
       __syncwarp();
       tc_fence_after();
-      mx_epilogue<KIND>(p, tl, row, tbase + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN);
+      mx_epilogue<KIND>(p, tl, row, tbase + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN, cbeg, cend);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -368,7 +378,7 @@ static cudaError_t mx_launch_kind(const MxParams& p, int grid, cudaStream_t st) 
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  k_moe_gemm_mx<KIND><<<grid, GEMM_THREADS, mx_smem_bytes(KIND), st>>>(p);
+  k_moe_gemm_mx<KIND><<<grid, mx_threads(KIND), mx_smem_bytes(KIND), st>>>(p);
   return cudaGetLastError();
 }
 

@@ -203,6 +203,11 @@ struct MxParams {
 __host__ __device__ constexpr int mx_bn(int kind) { return kind == MX_DGRAD_DOWN ? 128 : 256; }
 __host__ __device__ constexpr int mx_accs(int kind) { return mx_bn(kind) == 128 ? 2 : 1; }
 __host__ __device__ constexpr int mx_stages(int kind) { return mx_bn(kind) == 128 ? 6 : 4; }
+// Epilogue warps: with one accumulator the MMAs of the next tile wait for the epilogue, so it is
+// split over eight warps (two per TMEM lane quarter, each taking half of the columns); the
+// double-buffered 128 x 128 kind keeps four.
+__host__ __device__ constexpr int mx_epi_warps(int kind) { return mx_accs(kind) == 1 ? 8 : 4; }
+__host__ __device__ constexpr int mx_threads(int kind) { return 64 + 32 * mx_epi_warps(kind); }
 constexpr size_t MX_A_BYTES = 128 * 128;
 __host__ __device__ constexpr size_t mx_stage_tx(int kind) {  // bytes one stage receives
   return MX_A_BYTES + static_cast<size_t>(mx_bn(kind)) * 128 + 512 * (1 + mx_bn(kind) / 128);
