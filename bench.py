@@ -189,7 +189,7 @@ def algorithmic_bytes(w: IN.Workload, wgrad_elem_bytes: int = 2) -> dict:
 # A figure is reported only while the GEMM sources still hash to the value they had
 # when the counters were taken.
 NCU_TRAFFIC = {
-    ("gemm_wgrad_gateup", "dsv3"): (913.67e6 * 16, "b1939f26a44f1da2"),
+    ("gemm_wgrad_gateup", "dsv3"): (914.60e6 * 16, "5c3d6c9956e2b2d9"),
 }
 GEMM_SOURCES = ("gemm.cu", "ptx.cuh", "moe_internal.cuh")
 

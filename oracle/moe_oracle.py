@@ -601,3 +601,52 @@ def token_forward_backward_mx(t: int, X, W_r, bias, rounded, top_k: int, dY):
     dl[ids[0]] = g * (dg - np.sum(g * dg))
     dx += dl @ _f64(W_r).T
     return y, dx, dl, ids[0], g
+
+
+# ----------------------------------------------------------------------------
+# Expert parallelism ("Three design decisions that matter", bullet 1: pull-based
+# dispatch and push-based combine, the backward mirrored, one schedule table for
+# all four phases).  Readings: R ranks each hold their own tokens; rank q owns the
+# contiguous experts [q E/R, (q+1) E/R); an owner pulls, for each local expert,
+# the rows of every source rank in source-rank order, each source's tokens in
+# ascending order; it pushes each output row back to the source's slot of that
+# assignment (token t, slot j), where the source combines its k slots in slot order.
+# ----------------------------------------------------------------------------
+def ep_plan(ids_ranks, E: int, P: int = P_PAD) -> dict:
+    """ids_ranks[r]: [T_r, k] expert ids of rank r's tokens.  Returns, per owner q:
+    counts [El] (rows per local expert), padded_offsets [El+1], base [El][R+1] (first row of each
+    source inside the expert's rows), rows: for every real row in order, (source, token, slot);
+    and per source r: dest[r] [T_r, k] = (owner, padded row) of each assignment."""
+    R = len(ids_ranks)
+    if E % R:
+        raise ValueError("E must be a multiple of the number of ranks")
+    El = E // R
+    k = np.asarray(ids_ranks[0]).shape[1]
+    owners = []
+    dest = [np.full(np.asarray(ids).shape + (2,), -1, dtype=np.int64) for ids in ids_ranks]
+    for q in range(R):
+        counts = np.zeros(El, dtype=np.int64)
+        base = np.zeros((El, R + 1), dtype=np.int64)
+        per = [[[] for _ in range(R)] for _ in range(El)]  # per[el][src] = [(token, slot)]
+        for src, ids in enumerate(ids_ranks):
+            ids = np.asarray(ids)
+            for t in range(ids.shape[0]):  # ascending token
+                for j in range(k):
+                    el = int(ids[t, j]) - q * El
+                    if 0 <= el < El:
+                        per[el][src].append((t, j))
+        padded_offsets = np.zeros(El + 1, dtype=np.int64)
+        rows = []
+        for el in range(El):
+            for src in range(R):
+                base[el, src + 1] = base[el, src] + len(per[el][src])
+            counts[el] = base[el, R]
+            padded_offsets[el + 1] = padded_offsets[el] + (counts[el] + P - 1) // P * P
+            i = 0
+            for src in range(R):
+                for (t, j) in per[el][src]:
+                    rows.append((src, t, j))
+                    dest[src][t, j] = (q, padded_offsets[el] + i)
+                    i += 1
+        owners.append(dict(counts=counts, padded_offsets=padded_offsets, base=base, rows=rows))
+    return dict(owners=owners, dest=dest, El=El, R=R)

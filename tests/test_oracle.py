@@ -571,3 +571,36 @@ def test_mx_token_path_and_slices_equal_the_full_mx_layer():
     np.testing.assert_allclose(Ys, Y, rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(dls, g["dl"], rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(dXs + dls @ W_r.T, g["dX"], rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("R,Ts,E,k", [(2, (40, 33), 8, 2), (4, (16, 20, 1, 30), 16, 4), (3, (0, 50, 7), 12, 3)])
+def test_ep_plan_is_the_single_layer_schedule_of_the_rank_major_batch(R, Ts, E, k):
+    # Pull dispatch in source-rank order, each source's tokens ascending, gives every owner the
+    # rows the one-GPU schedule of the concatenated (rank-major) batch gives its expert slice;
+    # every assignment has exactly one destination row, and the rows are a bijection.
+    rng = np.random.default_rng(sum(Ts) + E)
+    ids_ranks = [np.array([rng.choice(E, size=k, replace=False) for _ in range(T)], dtype=np.int32).reshape(T, k)
+                 for T in Ts]
+    plan = O.ep_plan(ids_ranks, E)
+    El = E // R
+    off = np.concatenate([[0], np.cumsum(Ts)])
+    ids_all = np.concatenate(ids_ranks, axis=0)
+    for q, own in enumerate(plan["owners"]):
+        s = O.schedule(ids_all, E, first_local=q * El, num_local=El)
+        assert np.array_equal(own["counts"], s["counts"])
+        assert np.array_equal(own["padded_offsets"], s["padded_offsets"])
+        glob = [off[src] + t for (src, t, j) in own["rows"]]
+        assert np.array_equal(np.array(glob, dtype=np.int64), s["perm"])
+        for el in range(El):
+            assert own["base"][el, R] == own["counts"][el]
+            for src in range(R):
+                n = own["base"][el, src + 1] - own["base"][el, src]
+                assert n == np.sum(ids_ranks[src] == q * El + el)
+    for src in range(R):
+        T = Ts[src]
+        for t in range(T):
+            for j in range(k):
+                q, row = plan["dest"][src][t, j]
+                assert q == ids_ranks[src][t, j] // El
+                sq = O.schedule(ids_all, E, first_local=q * El, num_local=El)
+                assert row == sq["slot_row"][off[src] + t, j]
