@@ -50,7 +50,9 @@ typedef enum moe_status {
   MOE_ERR_WORKSPACE_TOO_SMALL = 3,  /* ctx or workspace smaller than the *_size() call says */
   MOE_ERR_CUDA = 4,                 /* a CUDA runtime call failed (launch, attribute, ...) */
   MOE_ERR_DEVICE_TIMEOUT = 5,       /* a bounded device-side wait ran out */
-  MOE_ERR_NONFINITE = 6             /* a router logit was NaN or +-Inf */
+  MOE_ERR_NONFINITE = 6,            /* a router logit was NaN or +-Inf */
+  MOE_ERR_EXCHANGE = 7              /* expert-parallel exchange buffers held tables that do not fit
+                                       together (routing of another step, or not published) */
 } moe_status;
 
 typedef enum moe_precision {
@@ -281,6 +283,78 @@ moe_status moe_debug_stream_plan(const moe_shape* shape, int32_t num_minibatches
  * must be serialised by the caller. */
 moe_status moe_route_static(const moe_shape* shape, const void* X, const void* W_r, const float* bias,
                             int32_t* ids, float* gates, int32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Expert parallelism across R ranks (page 1, "Three design decisions that
+ * matter", bullet 1: the rank that owns an expert pulls the tokens it needs
+ * from the senders' memory, so senders need not signal arrival; expert outputs
+ * are pushed back to the token's rank; the backward mirrors both; one schedule
+ * table serves all four phases).
+ *
+ * Rank q of R holds shape->T tokens of its own and the experts
+ * [q E/R, (q+1) E/R) (E a multiple of R, 1 <= R <= 64); shape->first_local_expert
+ * and num_local_experts are ignored.  Every rank owns an exchange buffer of
+ * moe_ep_buffer_size bytes (256-byte aligned, zeroed once before the first
+ * step) that all ranks can address: `bufs` lists the R buffers' addresses in this
+ * process (peer mappings across GPUs, or all on one device), bufs[rank] its own.
+ * Peers read a rank's routing table, X and dY from it and write expert outputs,
+ * dX rows and router-gate gradients into it, with plain loads and stores; the
+ * only signals are one ready flag per rank and step phase, and one done flag
+ * per (owner, source) pair, each wait bounded (about 2 s, then
+ * MOE_ERR_DEVICE_TIMEOUT in ctx's status word).  `epoch` numbers the step (a
+ * new value every step, not 0).
+ *
+ * A step is six calls per rank, in this order on its stream; each call of a
+ * phase may wait for the earlier phases of every rank of the same step:
+ *   moe_ep_fwd_route    route this rank's tokens (router GEMM, top-k, the table
+ *                       over all E experts) and publish them with X
+ *   moe_ep_fwd_experts  pull the local experts' rows from every rank (ranks in
+ *                       order, tokens ascending: the one-device layer's order for
+ *                       the rank-major concatenation of the ranks' tokens), run
+ *                       the grouped gate/up + SwiGLU and down GEMMs, push each
+ *                       output row back to its source's slot
+ *   moe_ep_fwd_combine  Y [T, d] = the pushed rows, summed over the k slots in order
+ *   moe_ep_bwd_publish  publish dY [T, d]
+ *   moe_ep_bwd_experts  pull dY rows, dgrad + SwiGLU backward, push each row's
+ *                       router-gate gradient and its dX row back, then the local
+ *                       experts' weight gradients dW_gate, dW_up [E/R, d, I],
+ *                       dW_down [E/R, I, d] (bf16, or fp32 by wgrad_dtype)
+ *   moe_ep_bwd_finish   router backward of this rank's tokens: dX [T, d] and this
+ *                       rank's part of dW_r [d, E] (fp32; the full dW_r is the sum
+ *                       over ranks, as for any replicated weight)
+ * Y, dX and the expert weight gradients equal the one-device layer's on the
+ * rank-major concatenation wherever the router GEMM's fixed K split is the same
+ * for T and R T tokens (bit for bit; see router_splits in the sources).
+ * ctx / ws are this rank's (moe_ep_ctx_size / moe_ep_workspace_size bytes); ctx
+ * leads with the status word moe_get_error reads.  bf16 mode only.  Argument
+ * errors return synchronously; an R, rank or E that does not fit gives
+ * MOE_ERR_INVALID_ARG, an exchange buffer not 256-byte aligned too. */
+size_t moe_ep_buffer_size(const moe_shape* shape, int32_t num_ranks);
+size_t moe_ep_ctx_size(const moe_shape* shape, int32_t num_ranks);
+size_t moe_ep_workspace_size(const moe_shape* shape, int32_t num_ranks);
+moe_status moe_ep_fwd_route(const moe_shape* shape, int32_t num_ranks, int32_t rank, void* const* bufs, const void* X,
+                            const void* W_r, const float* bias, void* ctx, size_t ctx_bytes, void* ws,
+                            size_t ws_bytes, int32_t epoch, void* stream);
+moe_status moe_ep_fwd_experts(const moe_shape* shape, int32_t num_ranks, int32_t rank, void* const* bufs,
+                              const void* W_gate, const void* W_up, const void* W_down, void* ctx, size_t ctx_bytes,
+                              void* ws, size_t ws_bytes, int32_t epoch, void* stream);
+moe_status moe_ep_fwd_combine(const moe_shape* shape, int32_t num_ranks, int32_t rank, void* const* bufs, void* Y,
+                              void* ctx, size_t ctx_bytes, int32_t epoch, void* stream);
+moe_status moe_ep_bwd_publish(const moe_shape* shape, int32_t num_ranks, int32_t rank, void* const* bufs,
+                              const void* dY, void* ctx, size_t ctx_bytes, int32_t epoch, void* stream);
+moe_status moe_ep_bwd_experts(const moe_shape* shape, int32_t num_ranks, int32_t rank, void* const* bufs,
+                              const void* W_gate, const void* W_up, const void* W_down, void* dW_gate, void* dW_up,
+                              void* dW_down, void* ctx, size_t ctx_bytes, void* ws, size_t ws_bytes, int32_t epoch,
+                              void* stream);
+moe_status moe_ep_bwd_finish(const moe_shape* shape, int32_t num_ranks, int32_t rank, void* const* bufs,
+                             const void* X, const void* W_r, void* dX, float* dW_r, void* ctx, size_t ctx_bytes,
+                             void* ws, size_t ws_bytes, int32_t epoch, void* stream);
+/* Test hook: the owner side of the last moe_ep_fwd_experts (device pointers, any may be NULL):
+ * counts [E/R] rows per local expert, padded_offsets [E/R + 1], row_src [rows] for every
+ * padded row: source rank * T * top_k + that rank's assignment index (token * top_k + slot),
+ * or -1 / -2 for pad rows; `rows` = R T min(top_k, E/R) + 127 E/R rounded up to 128. */
+moe_status moe_ep_debug_plan(const moe_shape* shape, int32_t num_ranks, int32_t rank, const void* ctx,
+                             int32_t* counts, int32_t* padded_offsets, int32_t* row_src, void* stream);
 
 /* Static string naming a status code. */
 const char* moe_status_string(moe_status status);

@@ -19,6 +19,7 @@ MOE_ERR_WORKSPACE_TOO_SMALL = 3
 MOE_ERR_CUDA = 4
 MOE_ERR_DEVICE_TIMEOUT = 5
 MOE_ERR_NONFINITE = 6
+MOE_ERR_EXCHANGE = 7
 MOE_BF16 = 0
 MOE_MXFP8 = 1
 MOE_WGRAD_BF16 = 0
@@ -64,6 +65,7 @@ class MoeError(RuntimeError):
 _lib = None
 _P = ctypes.c_void_p
 _S = ctypes.POINTER(moe_shape)
+_PP = ctypes.POINTER(ctypes.c_void_p)
 
 _SIGS = {
     "moe_ctx_size": (ctypes.c_size_t, [_S]),
@@ -96,6 +98,22 @@ _SIGS = {
                                   _P]),
     "moe_bwd_mx": (ctypes.c_int, [_S, _P, _P, _P, ctypes.c_size_t, _P, _P, ctypes.c_size_t, _P, _P, _P, _P, _P, _P,
                                   ctypes.c_size_t, _P]),
+    "moe_ep_buffer_size": (ctypes.c_size_t, [_S, ctypes.c_int32]),
+    "moe_ep_ctx_size": (ctypes.c_size_t, [_S, ctypes.c_int32]),
+    "moe_ep_workspace_size": (ctypes.c_size_t, [_S, ctypes.c_int32]),
+    "moe_ep_fwd_route": (ctypes.c_int, [_S, ctypes.c_int32, ctypes.c_int32, _PP, _P, _P, _P, _P, ctypes.c_size_t, _P,
+                                        ctypes.c_size_t, ctypes.c_int32, _P]),
+    "moe_ep_fwd_experts": (ctypes.c_int, [_S, ctypes.c_int32, ctypes.c_int32, _PP, _P, _P, _P, _P, ctypes.c_size_t,
+                                          _P, ctypes.c_size_t, ctypes.c_int32, _P]),
+    "moe_ep_fwd_combine": (ctypes.c_int, [_S, ctypes.c_int32, ctypes.c_int32, _PP, _P, _P, ctypes.c_size_t,
+                                          ctypes.c_int32, _P]),
+    "moe_ep_bwd_publish": (ctypes.c_int, [_S, ctypes.c_int32, ctypes.c_int32, _PP, _P, _P, ctypes.c_size_t,
+                                          ctypes.c_int32, _P]),
+    "moe_ep_bwd_experts": (ctypes.c_int, [_S, ctypes.c_int32, ctypes.c_int32, _PP, _P, _P, _P, _P, _P, _P, _P,
+                                          ctypes.c_size_t, _P, ctypes.c_size_t, ctypes.c_int32, _P]),
+    "moe_ep_bwd_finish": (ctypes.c_int, [_S, ctypes.c_int32, ctypes.c_int32, _PP, _P, _P, _P, _P, _P,
+                                         ctypes.c_size_t, _P, ctypes.c_size_t, ctypes.c_int32, _P]),
+    "moe_ep_debug_plan": (ctypes.c_int, [_S, ctypes.c_int32, ctypes.c_int32, _P, _P, _P, _P, _P]),
 }
 
 
@@ -343,6 +361,94 @@ def unchunk_scales(chunks, R, K):
     kb = np.arange(K // 32)[None, :]
     idx = ((r // 128) * (K // 128) + (kb * 32) // 128) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + kb % 4
     return chunks[idx]
+
+
+# ---------------------------------------------------------------------------
+# expert parallelism across R ranks (argument marshalling only)
+# ---------------------------------------------------------------------------
+def _ptr_array(bufs):
+    arr = (ctypes.c_void_p * len(bufs))(*[_ptr(b) for b in bufs])
+    return ctypes.cast(arr, _PP), arr
+
+
+def moe_ep_buffer_size(shape, R) -> int:
+    return int(lib().moe_ep_buffer_size(ctypes.byref(shape), int(R)))
+
+
+def moe_ep_ctx_size(shape, R) -> int:
+    return int(lib().moe_ep_ctx_size(ctypes.byref(shape), int(R)))
+
+
+def moe_ep_workspace_size(shape, R) -> int:
+    return int(lib().moe_ep_workspace_size(ctypes.byref(shape), int(R)))
+
+
+class MoEExpertParallel:
+    """One rank of the expert-parallel layer: its ctx / workspace, and the R ranks' exchange
+    buffers (device memory this process can address: peer mappings across GPUs, or all on one
+    device).  Each step runs three forward phases and three backward phases on every rank; a
+    phase's waits are satisfied by the other ranks' earlier phases of the same step (epoch)."""
+
+    def __init__(self, T, d, E, I, top_k, R, rank, bufs, device="cuda", wgrad_dtype=None):
+        import torch
+        self.wgrad_dtype = wgrad_dtype or torch.bfloat16
+        self.shape = make_shape(T, d, E, I, top_k, MOE_BF16, 0, 0, _wgrad_code(self.wgrad_dtype))
+        nc, nw = moe_ep_ctx_size(self.shape, R), moe_ep_workspace_size(self.shape, R)
+        if nc == 0 or nw == 0:
+            raise MoeError(MOE_ERR_UNSUPPORTED, "expert-parallel shape")
+        self.ctx = torch.empty(nc, dtype=torch.uint8, device=device)
+        self.ws = torch.empty(nw, dtype=torch.uint8, device=device)
+        self.T, self.d, self.E, self.I, self.k, self.R, self.rank = T, d, E, I, top_k, R, rank
+        self.El = E // R
+        self._bufs, self._keep = _ptr_array(bufs)
+
+    def _call(self, name, *args, stream=None):
+        check(int(getattr(lib(), name)(ctypes.byref(self.shape), self.R, self.rank, self._bufs, *args,
+                                      _stream(stream))), name)
+
+    def fwd_route(self, X, W_r, bias, epoch, stream=None):
+        self._call("moe_ep_fwd_route", _ptr(X), _ptr(W_r), _ptr(bias), _ptr(self.ctx), _nbytes(self.ctx),
+                   _ptr(self.ws), _nbytes(self.ws), int(epoch), stream=stream)
+
+    def fwd_experts(self, W_gate, W_up, W_down, epoch, stream=None):
+        self._call("moe_ep_fwd_experts", _ptr(W_gate), _ptr(W_up), _ptr(W_down), _ptr(self.ctx), _nbytes(self.ctx),
+                   _ptr(self.ws), _nbytes(self.ws), int(epoch), stream=stream)
+
+    def fwd_combine(self, Y, epoch, stream=None):
+        self._call("moe_ep_fwd_combine", _ptr(Y), _ptr(self.ctx), _nbytes(self.ctx), int(epoch), stream=stream)
+
+    def bwd_publish(self, dY, epoch, stream=None):
+        self._call("moe_ep_bwd_publish", _ptr(dY), _ptr(self.ctx), _nbytes(self.ctx), int(epoch), stream=stream)
+
+    def bwd_experts(self, W_gate, W_up, W_down, dW_gate, dW_up, dW_down, epoch, stream=None):
+        self._call("moe_ep_bwd_experts", _ptr(W_gate), _ptr(W_up), _ptr(W_down), _ptr(dW_gate), _ptr(dW_up),
+                   _ptr(dW_down), _ptr(self.ctx), _nbytes(self.ctx), _ptr(self.ws), _nbytes(self.ws), int(epoch),
+                   stream=stream)
+
+    def bwd_finish(self, X, W_r, dX, dW_r, epoch, stream=None):
+        self._call("moe_ep_bwd_finish", _ptr(X), _ptr(W_r), _ptr(dX), _ptr(dW_r), _ptr(self.ctx), _nbytes(self.ctx),
+                   _ptr(self.ws), _nbytes(self.ws), int(epoch), stream=stream)
+
+    def plan(self):
+        """Owner-side plan of the last forward: rows per local expert [El], padded offsets [El+1],
+        and each padded row's source (source rank * T k + assignment; -1 / -2 for pad rows)."""
+        import torch
+        dev = self.ctx.device
+        counts = torch.empty(self.El, dtype=torch.int32, device=dev)
+        poff = torch.empty(self.El + 1, dtype=torch.int32, device=dev)
+        rows = torch.empty(self._rp(), dtype=torch.int32, device=dev)
+        check(int(lib().moe_ep_debug_plan(ctypes.byref(self.shape), self.R, self.rank, _ptr(self.ctx), _ptr(counts),
+                                          _ptr(poff), _ptr(rows), None)), "moe_ep_debug_plan")
+        torch.cuda.synchronize()
+        return dict(counts=counts, padded_offsets=poff, row_src=rows[:int(poff[-1].item())])
+
+    def _rp(self):
+        # padded-row capacity of the owner role: R T min(k, El) + 127 El, rounded up to 128
+        A = self.R * self.T * min(self.k, self.El) + 127 * self.El
+        return max((A + 127) // 128 * 128, 128)
+
+    def error(self, stream=None):
+        return moe_get_error(self.ctx, stream)
 
 
 class MoEStream:

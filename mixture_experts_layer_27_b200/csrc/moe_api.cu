@@ -9,6 +9,7 @@
 #include <mutex>
 #include <vector>
 
+#include "ep_internal.cuh"
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -443,6 +444,7 @@ const char* moe_status_string(moe_status st) {
     case MOE_ERR_CUDA: return "CUDA runtime error";
     case MOE_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
     case MOE_ERR_NONFINITE: return "non-finite router logit";
+    case MOE_ERR_EXCHANGE: return "expert-parallel exchange tables do not fit together";
   }
   return "unknown status";
 }
@@ -1153,6 +1155,323 @@ moe_status moe_debug_logits(const moe_shape* s, const void* ws, float* logits, v
   if (L.T == 0) return MOE_OK;
   MOE_TRY(cudaMemcpyAsync(logits, static_cast<const char*>(ws) + L.logits, static_cast<size_t>(L.T) * L.E * 4,
                           cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Expert parallelism across R ranks (exchange kernels in ep.cu)
+// ---------------------------------------------------------------------------
+namespace {
+struct EpSetup {
+  Layout Ls;       // the source role: this rank's T tokens, routed over all E experts
+  Layout Lo;       // the owner role: rows from all R ranks for the local experts
+  EpBuf B;         // exchange buffer regions
+  size_t ctx_o;    // owner ctx at ctx + ctx_o, then the per-source row counts table
+  size_t base_off;
+  size_t ws_o;     // owner workspace at ws + ws_o
+  size_t ctx_bytes, ws_bytes;
+  int El, first, R, rank;
+  int64_t TK;
+};
+
+moe_status ep_setup(const moe_shape* s, int32_t R, int32_t rank, EpSetup* S) {
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (s->prec != MOE_BF16) return s->prec == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (R < 1 || R > kEpMaxRanks || rank < 0 || rank >= R || s->E <= 0 || s->E % R) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->T * static_cast<int64_t>(R) * s->top_k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  const int El = s->E / R;
+  moe_shape src = *s, own = *s;
+  // source role: a one-expert "slice" keeps its padded-row buffers small; its router weight
+  // gradient contracts over all of its tokens (every assignment has an owner somewhere)
+  src.first_local_expert = 0;
+  src.num_local_experts = 1;
+  own.T = s->T * R;
+  own.first_local_expert = rank * El;
+  own.num_local_experts = El;
+  if (!make_layout(src, &S->Ls) || !make_layout(own, &S->Lo)) return MOE_ERR_UNSUPPORTED;
+  S->Ls.rslice = false;
+  S->B = ep_buffer_layout(s->T, s->top_k, s->E, s->d, R);
+  S->ctx_o = align_up(S->Ls.ctx_bytes, 256);
+  S->base_off = align_up(S->ctx_o + S->Lo.ctx_bytes, 256);
+  S->ctx_bytes = S->base_off + static_cast<size_t>(El) * (R + 1) * 4;
+  S->ws_o = align_up(S->Ls.ws_bytes, 256);
+  S->ws_bytes = S->ws_o + S->Lo.ws_bytes;
+  S->El = El;
+  S->first = rank * El;
+  S->R = R;
+  S->rank = rank;
+  S->TK = s->T * static_cast<int64_t>(s->top_k);
+  return MOE_OK;
+}
+
+moe_status ep_peers(const EpSetup& S, void* const* bufs, EpPeers* P) {
+  if (!bufs) return MOE_ERR_INVALID_ARG;
+  std::memset(P, 0, sizeof(*P));
+  for (int r = 0; r < S.R; ++r) {
+    if (!bufs[r] || (reinterpret_cast<uintptr_t>(bufs[r]) & 255u)) return MOE_ERR_INVALID_ARG;
+    P->base[r] = static_cast<uint8_t*>(bufs[r]);
+  }
+  return MOE_OK;
+}
+
+// The source role's view: routing table regions in this rank's exchange buffer, slot_row the
+// identity (receive regions are indexed by assignment), the router gradient's dg from recv_dg.
+Ctx ep_source_ctx(const EpSetup& S, void* ctx, void* ws, uint8_t* mine) {
+  Ctx c = make_ctx(S.Ls, ctx, ws);
+  c.counts = reinterpret_cast<int*>(mine + S.B.counts);
+  c.offsets = reinterpret_cast<int*>(mine + S.B.offsets);
+  c.perm_asg = reinterpret_cast<int*>(mine + S.B.perm_asg);
+  c.gates = reinterpret_cast<float*>(mine + S.B.gates);
+  c.dgpart = reinterpret_cast<float*>(mine + S.B.recv_dg);
+  c.dxperm = reinterpret_cast<__nv_bfloat16*>(mine + S.B.recv_dx);
+  return c;
+}
+
+moe_status ep_check(const moe_shape* s, int32_t R, int32_t rank, void* const* bufs, void* ctx, size_t ctx_bytes,
+                    void* ws, size_t ws_bytes, bool need_ws, EpSetup* S, EpPeers* P) {
+  const moe_status e = ep_setup(s, R, rank, S);
+  if (e != MOE_OK) return e;
+  if (!ctx || !aligned16(ctx) || (need_ws && (!ws || !aligned16(ws)))) return MOE_ERR_INVALID_ARG;
+  if (ctx_bytes < S->ctx_bytes || (need_ws && ws_bytes < S->ws_bytes)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  return ep_peers(*S, bufs, P);
+}
+}  // namespace
+
+extern "C" {
+
+size_t moe_ep_buffer_size(const moe_shape* s, int32_t R) {
+  EpSetup S;
+  return ep_setup(s, R, 0, &S) == MOE_OK ? S.B.bytes : 0;
+}
+size_t moe_ep_ctx_size(const moe_shape* s, int32_t R) {
+  EpSetup S;
+  return ep_setup(s, R, 0, &S) == MOE_OK ? S.ctx_bytes : 0;
+}
+size_t moe_ep_workspace_size(const moe_shape* s, int32_t R) {
+  EpSetup S;
+  return ep_setup(s, R, 0, &S) == MOE_OK ? S.ws_bytes : 0;
+}
+
+moe_status moe_ep_fwd_route(const moe_shape* s, int32_t R, int32_t rank, void* const* bufs, const void* X,
+                            const void* W_r, const float* bias, void* ctx, size_t ctx_bytes, void* ws, size_t ws_bytes,
+                            int32_t epoch, void* stream) {
+  EpSetup S;
+  EpPeers P;
+  const moe_status e = ep_check(s, R, rank, bufs, ctx, ctx_bytes, ws, ws_bytes, true, &S, &P);
+  if (e != MOE_OK) return e;
+  if ((s->T > 0 && !X) || !W_r || !aligned16(X) || !aligned16(W_r) || (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* mine = P.base[rank];
+  const Ctx c = ep_source_ctx(S, ctx, ws, mine);
+  MOE_TRY(cudaMemsetAsync(c.hdr, 0, HDR_WORDS * 4, st));  // clears the status word
+  {  // the owner role's row layout starts empty: if this step's plan does not run (a wait gave
+     // up), its GEMMs and exchange kernels see no rows
+    const Ctx co = make_ctx(S.Lo, static_cast<char*>(ctx) + S.ctx_o, nullptr);
+    MOE_TRY(cudaMemsetAsync(co.poff, 0, static_cast<size_t>(S.El + 1) * 4, st));
+    MOE_TRY(cudaMemsetAsync(co.counts, 0, static_cast<size_t>(s->E) * 4, st));
+    MOE_TRY(cudaMemsetAsync(co.hdr, 0, HDR_WORDS * 4, st));
+  }
+  if (S.Ls.T == 0) {
+    MOE_TRY(cudaMemsetAsync(mine + S.B.counts, 0, static_cast<size_t>(s->E) * 4, st));
+    MOE_TRY(cudaMemsetAsync(mine + S.B.offsets, 0, static_cast<size_t>(s->E + 1) * 4, st));
+  } else {
+    MOE_TRY_STATUS(route_tokens(S.Ls, c, X, W_r, bias, 0, st));  // table straight into the exchange buffer
+    MOE_TRY(cudaMemcpyAsync(mine + S.B.x, X, static_cast<size_t>(S.Ls.T) * s->d * 2, cudaMemcpyDeviceToDevice, st));
+    MOE_TRY(launch_ep_identity(c.slot_row, S.TK, st));
+  }
+  MOE_TRY(launch_ep_signal(P, R, rank, false, S.B.flags, EPF_FWD_READY, epoch, st));
+  return MOE_OK;
+}
+
+moe_status moe_ep_fwd_experts(const moe_shape* s, int32_t R, int32_t rank, void* const* bufs, const void* W_gate,
+                              const void* W_up, const void* W_down, void* ctx, size_t ctx_bytes, void* ws,
+                              size_t ws_bytes, int32_t epoch, void* stream) {
+  EpSetup S;
+  EpPeers P;
+  const moe_status e = ep_check(s, R, rank, bufs, ctx, ctx_bytes, ws, ws_bytes, true, &S, &P);
+  if (e != MOE_OK) return e;
+  if (!W_gate || !W_up || !W_down || !aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_down))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Layout& L = S.Lo;
+  int* status = static_cast<int*>(ctx) + HDR_STATUS;  // the source role's status word leads ctx
+  const Ctx c = make_ctx(L, static_cast<char*>(ctx) + S.ctx_o, static_cast<char*>(ws) + S.ws_o);
+  int* base = reinterpret_cast<int*>(static_cast<char*>(ctx) + S.base_off);
+  const int TK = static_cast<int>(S.TK);
+  const uint64_t RP = static_cast<uint64_t>(L.RP);
+  const int grid = num_sms();
+  // every source has published its table and rows: pull them
+  MOE_TRY(launch_ep_wait(P, R, rank, false, S.B.flags, EPF_FWD_READY, epoch, status, st));
+  MOE_TRY(launch_ep_plan(P, R, S.B.counts, S.first, S.El, L.RP, c.counts, c.poff, base, c.hdr, status, st));
+  MOE_TRY(timed(K_MARK_ROWS, st, [&] { return launch_mark_rows(L, c, st); }));
+  MOE_TRY(launch_ep_table(P, R, S.B, S.first, S.El, TK, c.poff, base, c.row_asg, c.row_gate, status, st));
+  MOE_TRY(timed(K_DISPATCH, st, [&] {
+    return launch_ep_gather(P, S.B.x, TK, L.k, L.d, c.poff, L.El, c.row_asg, L.RP, c.xperm, status, st);
+  }));
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, c.xperm, L.d, RP, L.d, 64, 128));
+    MOE_TMAP(tmap_2d(&p.tb0, W_gate, L.I, static_cast<uint64_t>(L.El) * L.d, L.I, 64, 64));
+    MOE_TMAP(tmap_2d(&p.tb1, W_up, L.I, static_cast<uint64_t>(L.El) * L.d, L.I, 64, 64));
+    p.ta1 = p.ta0;
+    p.out0 = c.abuf;
+    p.out1 = c.bbuf;
+    p.out2 = c.hbuf;
+    MOE_TRY(timed(K_GEMM_GATEUP, st, [&] { return launch_gemm(G_GATEUP, p, grid, st); }));
+  }
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, c.hbuf, L.I, RP, L.I, 64, 128));
+    MOE_TMAP(tmap_2d(&p.tb0, W_down, L.d, static_cast<uint64_t>(L.El) * L.I, L.d, 64, 64));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.out0 = c.obuf;
+    MOE_TRY(timed(K_GEMM_DOWN, st, [&] { return launch_gemm(G_DOWN, p, grid, st); }));
+  }
+  // push each output row back to its source's slot, then tell every source
+  MOE_TRY(timed(K_COMBINE, st, [&] {
+    return launch_ep_push_rows(P, S.B.recv_o, TK, L.d, c.poff, L.El, c.row_asg, L.RP, c.obuf, status, st);
+  }));
+  MOE_TRY(launch_ep_signal(P, R, rank, true, S.B.flags, EPF_DONE + rank, epoch, st));
+  return MOE_OK;
+}
+
+moe_status moe_ep_fwd_combine(const moe_shape* s, int32_t R, int32_t rank, void* const* bufs, void* Y, void* ctx,
+                              size_t ctx_bytes, int32_t epoch, void* stream) {
+  EpSetup S;
+  EpPeers P;
+  const moe_status e = ep_check(s, R, rank, bufs, ctx, ctx_bytes, nullptr, 0, false, &S, &P);
+  if (e != MOE_OK) return e;
+  if ((s->T > 0 && !Y) || !aligned16(Y)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* mine = P.base[rank];
+  const Ctx c = ep_source_ctx(S, ctx, nullptr, mine);
+  MOE_TRY(launch_ep_wait(P, R, rank, true, S.B.flags, EPF_DONE, epoch, c.hdr + HDR_STATUS, st));
+  if (S.Ls.T == 0) return MOE_OK;
+  MOE_TRY(timed(K_COMBINE, st, [&] {
+    return launch_combine(S.Ls, c, reinterpret_cast<const __nv_bfloat16*>(mine + S.B.recv_o),
+                          static_cast<__nv_bfloat16*>(Y), st);
+  }));
+  return MOE_OK;
+}
+
+moe_status moe_ep_bwd_publish(const moe_shape* s, int32_t R, int32_t rank, void* const* bufs, const void* dY,
+                              void* ctx, size_t ctx_bytes, int32_t epoch, void* stream) {
+  EpSetup S;
+  EpPeers P;
+  const moe_status e = ep_check(s, R, rank, bufs, ctx, ctx_bytes, nullptr, 0, false, &S, &P);
+  if (e != MOE_OK) return e;
+  if ((s->T > 0 && !dY) || !aligned16(dY)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (S.Ls.T > 0)
+    MOE_TRY(cudaMemcpyAsync(P.base[rank] + S.B.dy, dY, static_cast<size_t>(S.Ls.T) * s->d * 2,
+                            cudaMemcpyDeviceToDevice, st));
+  MOE_TRY(launch_ep_signal(P, R, rank, false, S.B.flags, EPF_BWD_READY, epoch, st));
+  return MOE_OK;
+}
+
+moe_status moe_ep_bwd_experts(const moe_shape* s, int32_t R, int32_t rank, void* const* bufs, const void* W_gate,
+                              const void* W_up, const void* W_down, void* dW_gate, void* dW_up, void* dW_down,
+                              void* ctx, size_t ctx_bytes, void* ws, size_t ws_bytes, int32_t epoch, void* stream) {
+  EpSetup S;
+  EpPeers P;
+  const moe_status e = ep_check(s, R, rank, bufs, ctx, ctx_bytes, ws, ws_bytes, true, &S, &P);
+  if (e != MOE_OK) return e;
+  if (!W_gate || !W_up || !W_down || !dW_gate || !dW_up || !dW_down || !aligned16(W_gate) || !aligned16(W_up) ||
+      !aligned16(W_down) || !aligned16(dW_gate) || !aligned16(dW_up) || !aligned16(dW_down))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Layout& L = S.Lo;
+  int* status = static_cast<int*>(ctx) + HDR_STATUS;
+  const Ctx c = make_ctx(L, static_cast<char*>(ctx) + S.ctx_o, static_cast<char*>(ws) + S.ws_o);
+  const int TK = static_cast<int>(S.TK);
+  const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
+  const int grid = num_sms();
+  MOE_TRY(launch_ep_wait(P, R, rank, false, S.B.flags, EPF_BWD_READY, epoch, status, st));
+  // pull reverse-combine: dY rows from every source
+  MOE_TRY(timed(K_REV_COMBINE, st, [&] {
+    return launch_ep_gather(P, S.B.dy, TK, L.k, L.d, c.poff, L.El, c.row_asg, L.RP, c.dyperm, status, st);
+  }));
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, c.dyperm, L.d, RP, L.d, 64, 128));
+    MOE_TMAP(tmap_2d(&p.tb0, W_down, L.d, El * L.I, L.d, 64, 256));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.in0 = c.abuf;
+    p.in1 = c.bbuf;
+    p.out0 = c.dabuf;
+    p.out1 = c.dbbuf;
+    p.out2 = c.hgbuf;
+    p.outf = c.dgpart;
+    MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm(G_DGRAD_DOWN, p, grid, st); }));
+  }
+  MOE_TRY(timed(K_ROUTER_BWD, st, [&] {
+    return launch_ep_push_dg(P, S.B.recv_dg, TK, c.poff, L.El, c.row_asg, c.dgpart, L.I / 256, L.RP, status, st);
+  }));
+  {
+    GemmParams p = base_params(L, c, status);
+    MOE_TMAP(tmap_2d(&p.ta0, c.dabuf, L.I, RP, L.I, 64, 128));
+    MOE_TMAP(tmap_2d(&p.ta1, c.dbbuf, L.I, RP, L.I, 64, 128));
+    MOE_TMAP(tmap_2d(&p.tb0, W_gate, L.I, El * L.d, L.I, 64, 256));
+    MOE_TMAP(tmap_2d(&p.tb1, W_up, L.I, El * L.d, L.I, 64, 256));
+    p.out0 = c.dxperm;
+    MOE_TRY(timed(K_GEMM_DGRAD_GATEUP, st, [&] { return launch_gemm(G_DGRAD_GATEUP, p, grid, st); }));
+  }
+  // push reverse-dispatch: dX rows to their sources, then tell every source
+  MOE_TRY(timed(K_REV_DISPATCH, st, [&] {
+    return launch_ep_push_rows(P, S.B.recv_dx, TK, L.d, c.poff, L.El, c.row_asg, L.RP, c.dxperm, status, st);
+  }));
+  MOE_TRY(launch_ep_signal(P, R, rank, true, S.B.flags, EPF_DONE + R + rank, epoch, st));
+  return launch_wgrads(L, c, status, dW_gate, dW_up, dW_down, st);
+}
+
+moe_status moe_ep_bwd_finish(const moe_shape* s, int32_t R, int32_t rank, void* const* bufs, const void* X,
+                             const void* W_r, void* dX, float* dW_r, void* ctx, size_t ctx_bytes, void* ws,
+                             size_t ws_bytes, int32_t epoch, void* stream) {
+  EpSetup S;
+  EpPeers P;
+  const moe_status e = ep_check(s, R, rank, bufs, ctx, ctx_bytes, ws, ws_bytes, true, &S, &P);
+  if (e != MOE_OK) return e;
+  if ((s->T > 0 && (!X || !dX)) || !W_r || !dW_r || !aligned16(X) || !aligned16(dX) || !aligned16(W_r) ||
+      !aligned16(dW_r))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Layout& L = S.Ls;
+  const Ctx c = ep_source_ctx(S, ctx, ws, P.base[rank]);
+  int* status = c.hdr + HDR_STATUS;
+  MOE_TRY(launch_ep_wait(P, R, rank, true, S.B.flags, EPF_DONE + R, epoch, status, st));
+  if (L.T == 0) {
+    MOE_TRY(cudaMemsetAsync(dW_r, 0, static_cast<size_t>(L.d) * L.E * 4, st));
+    return MOE_OK;
+  }
+  // router backward over this rank's tokens (dg pushed back by the owners, one value per
+  // assignment), its part of dW_r, and dX = the pushed dX rows in slot order + the router term
+  MOE_TRY(timed(K_ROUTER_BWD, st, [&] { return launch_router_bwd(L, c, st, 1); }));
+  MOE_TRY(timed(K_ROUTER_WGRAD, st, [&] { return launch_router_wgrad(L, c, X, dW_r, status, st); }));
+  MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
+    return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
+  }));
+  MOE_TRY(timed(K_REV_DISPATCH, st, [&] { return launch_rev_dispatch(L, c, static_cast<__nv_bfloat16*>(dX), st); }));
+  return MOE_OK;
+}
+
+moe_status moe_ep_debug_plan(const moe_shape* s, int32_t R, int32_t rank, const void* ctx, int32_t* counts,
+                             int32_t* padded_offsets, int32_t* row_src, void* stream) {
+  EpSetup S;
+  const moe_status e = ep_setup(s, R, rank, &S);
+  if (e != MOE_OK) return e;
+  if (!ctx) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ctx c = make_ctx(S.Lo, const_cast<char*>(static_cast<const char*>(ctx)) + S.ctx_o, nullptr);
+  if (counts) MOE_TRY(cudaMemcpyAsync(counts, c.counts + S.first, S.El * 4, cudaMemcpyDeviceToDevice, st));
+  if (padded_offsets)
+    MOE_TRY(cudaMemcpyAsync(padded_offsets, c.poff, (S.El + 1) * 4, cudaMemcpyDeviceToDevice, st));
+  if (row_src)
+    MOE_TRY(cudaMemcpyAsync(row_src, c.row_asg, static_cast<size_t>(S.Lo.RP) * 4, cudaMemcpyDeviceToDevice, st));
   return MOE_OK;
 }
 

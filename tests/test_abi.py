@@ -148,3 +148,33 @@ def test_mxfp8_sizes_and_argument_errors(lib):
         B.MOE_ERR_WORKSPACE_TOO_SMALL
     r = lib.moe_bwd_mx(ctypes.byref(mx), f, f, f, nq, None, f, nc, f, f, f, f, f, f, nw, None)
     assert r == B.MOE_ERR_INVALID_ARG  # dY missing
+
+
+def test_expert_parallel_sizes_and_argument_errors(lib):
+    s = B.make_shape(64, 256, 8, 256, 2)
+    assert B.moe_ep_buffer_size(s, 3) == 0 and B.moe_ep_ctx_size(s, 3) == 0  # E not a multiple of R
+    assert B.moe_ep_buffer_size(s, 0) == 0 and B.moe_ep_buffer_size(s, 65) == 0
+    nb, nc, nw = B.moe_ep_buffer_size(s, 2), B.moe_ep_ctx_size(s, 2), B.moe_ep_workspace_size(s, 2)
+    assert nb > 0 and nc > 0 and nw > 0
+    assert B.moe_ep_buffer_size(B.make_shape(128, 256, 8, 256, 2), 2) > nb  # more tokens, larger exchange
+    mx = B.make_shape(64, 256, 8, 256, 2, prec=B.MOE_MXFP8)
+    assert B.moe_ep_buffer_size(mx, 2) == 0
+    fake = 1 << 20  # never dereferenced: every check below comes before any launch
+    good, keep1 = B._ptr_array([fake, fake + 4096])
+    misaligned, keep2 = B._ptr_array([fake, fake + 16])
+    by = ctypes.byref
+
+    def route(shape, R, rank, bufs, ctx_bytes=nc, ws_bytes=nw):
+        return lib.moe_ep_fwd_route(by(shape), R, rank, bufs, fake, fake, None, fake, ctx_bytes, fake, ws_bytes, 1,
+                                    None)
+    assert route(s, 2, 2, good) == B.MOE_ERR_INVALID_ARG      # rank out of range
+    assert route(s, 2, -1, good) == B.MOE_ERR_INVALID_ARG
+    assert route(s, 3, 0, good) == B.MOE_ERR_INVALID_ARG      # E = 8 over 3 ranks
+    assert route(s, 2, 0, misaligned) == B.MOE_ERR_INVALID_ARG
+    assert route(s, 2, 0, None) == B.MOE_ERR_INVALID_ARG
+    assert route(s, 2, 0, good, ctx_bytes=nc - 1) == B.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert route(s, 2, 0, good, ws_bytes=nw - 1) == B.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert route(mx, 2, 0, good) == B.MOE_ERR_UNSUPPORTED
+    assert lib.moe_ep_fwd_combine(by(s), 2, 0, good, None, fake, nc, 1, None) == B.MOE_ERR_INVALID_ARG  # no Y
+    assert lib.moe_ep_bwd_finish(by(s), 2, 0, good, fake, fake, fake, None, fake, nc, fake, nw, 1,
+                                 None) == B.MOE_ERR_INVALID_ARG  # no dW_r
