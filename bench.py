@@ -107,12 +107,17 @@ def workload_config(w: IN.Workload) -> dict:
         l2 = ("no flush: the step streams %.2f GB of tokens (X, dY, the dispatched rows and their "
               "activations) through HBM, far beyond the 126 MB L2" % (4 * w.tokens * w.d * 2 / 1e9))
     else:
-        routing = "zipf(1.2) bias, hottest ~10x mean" if w.zipf else "near-uniform (W_r ~ N(0, 0.02^2))"
+        if w.local_tokens:
+            routing = (f"{w.El} local experts of {w.E}, each receiving {w.local_tokens} tokens; one batch, "
+                       "the dispatched rows held whole (no ring)")
+        else:
+            routing = "zipf(1.2) bias, hottest ~10x mean" if w.zipf else "near-uniform (W_r ~ N(0, 0.02^2))"
         l2 = ("no flush: expert weights (%.1f GB) exceed the 126 MB L2 and stream every step"
               % (3 * w.El * w.d * w.I * 2 / 1e9))
         if needs_flush(w):
             l2 = "L2 flushed (256 MB write) between timed steps; each step timed on its own"
-    return {"workload": f"{w.name}: T={w.tokens} d={w.d} E={w.E} top_k={w.k} I={w.I} bf16, {routing}",
+    prec = "mxfp8" if w.mxfp8 else "bf16"
+    return {"workload": f"{w.name}: T={w.tokens} d={w.d} E={w.E} top_k={w.k} I={w.I} {prec}, {routing}",
             "T": w.tokens, "d": w.d, "E": w.E, "top_k": w.k, "I": w.I, "precision": "mxfp8" if w.mxfp8 else "bf16",
             "seed": w.seed, "l2": l2, "parallelism": "replicas"}
 
@@ -431,12 +436,13 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     x = IN.make_inputs(w, device=dev)
     wdt = torch.float32 if args.wgrad_fp32 else torch.bfloat16
     if w.mxfp8:
-        layer = B.MoELayerMX(w.T, w.d, w.E, w.I, w.k, device=dev, wgrad_dtype=wdt)
+        layer = B.MoELayerMX(w.T, w.d, w.E, w.I, w.k, w.first_local, w.num_local, device=dev, wgrad_dtype=wdt)
     elif w.stream_M:
         layer = B.MoEStream(w.T, w.d, w.E, w.I, w.k, w.stream_M, w.ring_bytes, w.first_local, w.num_local,
                             device=dev, wgrad_dtype=wdt)
     else:
-        layer = B.MoELayer(w.T, w.d, w.E, w.I, w.k, device=dev, wgrad_dtype=wdt)
+        layer = B.MoELayer(w.T, w.d, w.E, w.I, w.k, first_local_expert=w.first_local, num_local_experts=w.num_local,
+                           device=dev, wgrad_dtype=wdt)
     NT = w.tokens
     Y = torch.empty(NT, w.d, dtype=torch.bfloat16, device=dev)
     grads = dict(dX=torch.empty(NT, w.d, dtype=torch.bfloat16, device=dev),
