@@ -122,6 +122,12 @@ def workload_config(w: IN.Workload) -> dict:
             "seed": w.seed, "l2": l2, "parallelism": "replicas"}
 
 
+def run_config(w: IN.Workload, args) -> dict:
+    """The `config` of both arms' lines: the workload, the gradient dtype and the forward's launch form."""
+    return dict(workload_config(w), wgrad_dtype="fp32" if args.wgrad_fp32 else "bf16",
+                forward="persistent" if args.persistent else "launches")
+
+
 L2_BYTES = 126 << 20
 
 
@@ -140,6 +146,7 @@ def algorithmic_flops(w: IN.Workload) -> dict:
             "gemm_dgrad_down_swiglu_bwd": 2 * dI * rows, "gemm_dgrad_gateup": 4 * dI * rows,
             "gemm_wgrad_gateup": 4 * dI * rows, "gemm_wgrad_down": 2 * dI * rows,
             "router_logits": 2 * w.tokens * w.d * w.E,
+            "gemm_gateup_down_persistent": 6 * dI * rows,  # gate/up and down in one launch
             # dW_r = X^T dl; the kernel issues it twice (the hi and lo bf16 terms of dl)
             "router_wgrad": 2 * w.tokens * w.d * w.E}
 
@@ -186,6 +193,9 @@ def algorithmic_bytes(w: IN.Workload, wgrad_elem_bytes: int = 2) -> dict:
         "reverse_dispatch": rows * d * 2 + T * d * 2 + E * d * 2,
         "gemm_wgrad_gateup": rows * d * 2 + 2 * rows * I * 2 + 2 * G1,
         "gemm_wgrad_down": rows * I * 2 + rows * d * 2 + G1,
+        # gate/up and down in one launch: the weights, X_perm in, A and B (saved) and O' out;
+        # H passes between two tiles of the launch and is not counted
+        "gemm_gateup_down_persistent": 3 * W1 + rows * d * 2 + 2 * rows * I * 2 + rows * d * 2,
     }
 
 
@@ -419,7 +429,7 @@ def run_reference(args, w: IN.Workload, world: int, rank: int):
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": statistics.mean(r["seconds"]) * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": dict(workload_config(w), wgrad_dtype="fp32" if args.wgrad_fp32 else "bf16"),
+            "config": run_config(w, args),
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                              "sample": r["sample"]},
@@ -467,6 +477,10 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
         def step(X, dY, Yout, g):
             layer.forward(X, x["W_r"], x["bias"], Y=Yout)
             layer.backward(X, x["W_r"], dY, out=g)
+    elif args.persistent:
+        def step(X, dY, Yout, g):
+            layer.forward(X, x["W_r"], x["bias"], x["W_gate"], x["W_up"], x["W_down"], Y=Yout, persistent=True)
+            layer.backward(X, x["W_r"], x["W_gate"], x["W_up"], x["W_down"], dY, out=g)
     else:
         def step(X, dY, Yout, g):
             layer.forward(X, x["W_r"], x["bias"], x["W_gate"], x["W_up"], x["W_down"], Y=Yout)
@@ -691,7 +705,7 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, random-init weights)",
-        "config": dict(workload_config(w), wgrad_dtype="fp32" if args.wgrad_fp32 else "bf16"),
+        "config": run_config(w, args),
         "tflops": tflops, "pct_of_bf16_peak": 100.0 * per_gpu_tflops / bf16,
         "peak_note": f"bf16 sustained {bf16} TFLOP/s ({peak_kind}); model FLOPs 18 d I T k + 6 T d E per step",
         "roofline": roof,
@@ -735,10 +749,14 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="time direct launches instead of a CUDA graph of one step")
     ap.add_argument("--wgrad-fp32", action="store_true",
                     help="write the expert weight gradients as fp32 instead of bf16 (the weights' dtype)")
+    ap.add_argument("--persistent", action="store_true",
+                    help="run the forward's gate/up and down GEMMs as one persistent launch (bf16, one batch)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = IN.WORKLOADS[args.workload]
+    if args.persistent and (w.mxfp8 or w.stream_M):
+        ap.error("--persistent runs the bf16 one-batch layer; %s is %s" % (w.name, "MXFP8" if w.mxfp8 else "streamed"))
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

@@ -110,6 +110,20 @@ moe_status moe_fwd(const moe_shape* shape, const void* X, const void* W_r, const
                    const void* W_gate, const void* W_up, const void* W_down, void* Y,
                    void* ctx, size_t ctx_bytes, void* ws, size_t ws_bytes, void* stream);
 
+/* Forward with its two grouped GEMMs in one persistent launch (page 1, the opening paragraph
+ * and "Three design decisions that matter": one megakernel fusing the MoE steps, its work
+ * scheduled through Cluster Launch Control).  Same arguments, results and ctx as moe_fwd, bit
+ * for bit; bf16 mode, one batch (no ring stream).  The routing and dispatch launches of moe_fwd
+ * run first and the combine launch last; between them one kernel runs every gate/up tile
+ * (SwiGLU epilogue) and then every down tile (gate multiply) as work units that CTAs take in
+ * one global order.  A down tile waits, bounded (about 2 s, then MOE_ERR_DEVICE_TIMEOUT in
+ * ctx's status word), until every gate/up tile of its 128 rows has stored H, so down tiles
+ * start while the last gate/up tiles run.  CTAs of the launch that have not started yet are
+ * cancelled by running CTAs, which take over their work (Cluster Launch Control). */
+moe_status moe_fwd_persistent(const moe_shape* shape, const void* X, const void* W_r, const float* bias,
+                              const void* W_gate, const void* W_up, const void* W_down, void* Y,
+                              void* ctx, size_t ctx_bytes, void* ws, size_t ws_bytes, void* stream);
+
 /* Backward of the last moe_fwd that wrote `ctx` (same shape, X, W_r, weights).
  *   dY      [T, d]   bf16   upstream gradient
  *   dX      [T, d]   bf16   written

@@ -71,6 +71,8 @@ _SIGS = {
     "moe_ctx_size": (ctypes.c_size_t, [_S]),
     "moe_workspace_size": (ctypes.c_size_t, [_S]),
     "moe_fwd": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, ctypes.c_size_t, _P]),
+    "moe_fwd_persistent": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, ctypes.c_size_t,
+                                          _P]),
     "moe_bwd": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, _P, _P, _P, _P,
                                ctypes.c_size_t, _P]),
     "moe_get_error": (ctypes.c_int, [_P, _P]),
@@ -169,6 +171,14 @@ def moe_fwd(shape, X, W_r, bias, W_gate, W_up, W_down, Y, ctx, ws, stream=None, 
     return int(lib().moe_fwd(ctypes.byref(shape), _ptr(X), _ptr(W_r), _ptr(bias), _ptr(W_gate), _ptr(W_up),
                              _ptr(W_down), _ptr(Y), _ptr(ctx), ctx_bytes if ctx_bytes is not None else _nbytes(ctx),
                              _ptr(ws), ws_bytes if ws_bytes is not None else _nbytes(ws), _stream(stream)))
+
+
+def moe_fwd_persistent(shape, X, W_r, bias, W_gate, W_up, W_down, Y, ctx, ws, stream=None, ctx_bytes=None,
+                       ws_bytes=None):
+    return int(lib().moe_fwd_persistent(ctypes.byref(shape), _ptr(X), _ptr(W_r), _ptr(bias), _ptr(W_gate),
+                                        _ptr(W_up), _ptr(W_down), _ptr(Y), _ptr(ctx),
+                                        ctx_bytes if ctx_bytes is not None else _nbytes(ctx), _ptr(ws),
+                                        ws_bytes if ws_bytes is not None else _nbytes(ws), _stream(stream)))
 
 
 def moe_bwd(shape, X, W_r, W_gate, W_up, W_down, dY, ctx, dX, dW_gate, dW_up, dW_down, dW_r, ws, stream=None,
@@ -524,11 +534,13 @@ class MoELayer:
         self.T, self.d, self.E, self.I, self.k = T, d, E, I, top_k
         self.El = num_local_experts or (E - first_local_expert)
 
-    def forward(self, X, W_r, bias, W_gate, W_up, W_down, Y=None, stream=None):
+    def forward(self, X, W_r, bias, W_gate, W_up, W_down, Y=None, stream=None, persistent=False):
+        """persistent: the expert phase as one persistent launch (moe_fwd_persistent); same results."""
         import torch
         if Y is None:
             Y = torch.empty(self.T, self.d, dtype=torch.bfloat16, device=X.device)
-        check(moe_fwd(self.shape, X, W_r, bias, W_gate, W_up, W_down, Y, self.ctx, self.ws, stream), "moe_fwd")
+        fn, name = (moe_fwd_persistent, "moe_fwd_persistent") if persistent else (moe_fwd, "moe_fwd")
+        check(fn(self.shape, X, W_r, bias, W_gate, W_up, W_down, Y, self.ctx, self.ws, stream), name)
         return Y
 
     def backward(self, X, W_r, W_gate, W_up, W_down, dY, out=None, stream=None):

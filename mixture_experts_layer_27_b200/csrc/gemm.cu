@@ -67,6 +67,7 @@ struct Tile {
   int nt;   // n-tile index
   int kb0;  // first 64-wide K block (wgrad: first padded row / 64)
   int nk;   // number of K blocks
+  int u;    // unit kind of the fused forward (FusedUnit); unused elsewhere
 };
 
 template <int KIND>
@@ -851,6 +852,341 @@ cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream
     case G_ROUTER_WGRAD: return launch_kind<G_ROUTER_WGRAD>(p, grid, st);
   }
   return cudaErrorInvalidValue;
+}
+
+// ===========================================================================
+// The forward's grouped GEMMs in one persistent launch
+// ===========================================================================
+// Work units, in ticket order: every gate/up tile, then every down tile.  A CTA takes a ticket
+// when it starts and one for each further unit it claims.  While the grid still has CTAs that
+// have not started, a claim is the cancellation of one of them through Cluster Launch Control
+// (its work moves to the running CTA); once the hardware reports none left, claims come from
+// the ticket counter alone, until the tickets run past the last unit.  So the work spreads
+// over the CTAs that actually run, whatever the grid size, and down tiles fill the SMs that
+// the last round of gate/up tiles leaves idle.  A down tile waits (bounded) until every
+// gate/up tile of its 128 rows has stored its H rows.  Tickets are handed out in one global
+// order and a down tile only waits for gate/up tiles, which have lower tickets and are held
+// by running (or finished) CTAs, so the waits end.  Every wait gives up once the status word
+// is set.
+//
+// A unit computes exactly what the separate GEMM launches compute (the same decode, loads and
+// epilogue functions), so the results are the same bits.
+//
+// Measured and kept out: dispatch and combine as units of this kernel, run by its four
+// epilogue warps.  With one CTA per SM those warps keep too few loads in flight for a copy:
+// traced per unit, the combine ran 12x and the dispatch 2x slower than their own kernels, and
+// gate/up tiles stalled behind the dispatch.
+enum FusedUnit { FU_GATEUP = 1, FU_DOWN = 2 };
+
+// ctl: [0] ticket counter, [1, 1 + cap) gate/up epilogue warps done per m-tile.
+struct FusedCounts {
+  int mt, ngu, ndn;
+  __device__ int total() const { return ngu + ndn; }
+};
+__device__ __forceinline__ FusedCounts fused_counts(const FusedFwdParams& P) {
+  FusedCounts c;
+  c.mt = (__ldg(P.gu.poff + P.gu.nseg) - __ldg(P.gu.poff)) / 128;
+  c.ngu = c.mt * ntiles_n<G_GATEUP>(P.gu);
+  c.ndn = c.mt * ntiles_n<G_DOWN>(P.dn);
+  return c;
+}
+__device__ __forceinline__ Tile fused_decode(const FusedFwdParams& P, const FusedCounts& c, int t) {
+  Tile tl;
+  if (t < c.ngu) {
+    tl = decode<G_GATEUP>(P.gu, t);
+    tl.u = FU_GATEUP;
+    return tl;
+  }
+  t -= c.ngu;
+  if (t < c.ndn) {
+    tl = decode<G_DOWN>(P.dn, t);
+    tl.u = FU_DOWN;
+    return tl;
+  }
+  tl.t = -1;
+  return tl;
+}
+
+// Bounded wait (one thread) until *p >= target, written by other CTAs with release order.
+__device__ __noinline__ bool wait_count(const int* p, int target, int* status) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const long long t0 = clock64();
+  for (uint32_t n = 1;; ++n) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(p) >= target) return true;
+    if ((n & 31u) == 0) {
+      if (status_set(status)) return false;
+      if (clock64() - t0 > MOE_SPIN_CYCLES) {
+        raise_status(status, MOE_ERR_DEVICE_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+// One warp's global stores, then one count: the stores are visible to a CTA that has acquired
+// the count (and, after its proxy fence, to that CTA's TMA loads).
+__device__ __forceinline__ void warp_release_count(int* p, int lane) {
+  __syncwarp();
+  if (lane == 0) {
+    fence_proxy_async_global();
+    __threadfence();
+    atomicAdd(p, 1);
+  }
+}
+
+constexpr size_t FUSED_TAIL_BYTES = 1024;
+constexpr size_t fused_smem_bytes() { return GEMM_STAGES * GEMM_STAGE_BYTES + 1024 + FUSED_TAIL_BYTES; }
+
+__global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_fwd_gemms(const __grid_constant__ FusedFwdParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int STAGES = GEMM_STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * GEMM_STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint64_t* sfull = drain + 1;
+  uint64_t* sempty = sfull + SCHED_DEPTH;
+  uint64_t* staken = sempty + SCHED_DEPTH;  // the producer has read ring entry j
+  uint64_t* clc_bar = staken + SCHED_DEPTH;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(clc_bar + 1);
+  uint4* clc_resp = reinterpret_cast<uint4*>((reinterpret_cast<uintptr_t>(clc_bar + 2) + 15) & ~uintptr_t(15));
+  Tile* ring = reinterpret_cast<Tile*>(clc_resp + 1);
+  int* status = P.gu.status;
+  int* hcnt = P.ctl + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    for (int s = 0; s < SCHED_DEPTH; ++s) {
+      mbar_init(&sfull[s], 1);
+      mbar_init(&sempty[s], 6);  // producer, MMA issuer, four epilogue warps
+      mbar_init(&staken[s], 1);
+    }
+    mbar_init(clc_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&P.gu.ta0);
+    prefetch_tmap(&P.gu.tb0);
+    prefetch_tmap(&P.gu.tb1);
+    prefetch_tmap(&P.dn.ta0);
+    prefetch_tmap(&P.dn.tb0);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  constexpr uint32_t IDESC = idesc_bf16(GEMM_BM, GEMM_BN, false, true);  // both kinds: A K-major, B MN-major
+  static_assert(!Traits<G_GATEUP>::A_MN && Traits<G_GATEUP>::B_MN && !Traits<G_DOWN>::A_MN && Traits<G_DOWN>::B_MN,
+                "the fused forward issues one instruction descriptor for both GEMMs");
+
+  if (warp == 6) {
+    if (lane == 0) {
+      // ---------------- scheduler: tickets in, decoded units into the ring ----------------
+      const FusedCounts cnt = fused_counts(P);
+      const int total = cnt.total();
+      uint32_t clc_phase = 0;
+      bool may_cancel = true;  // false after an answer that cancelled nothing
+      int ticket = status_set(status) ? total : atomicAdd(P.ctl, 1);
+      for (int j = 0;; ++j) {
+        const int slot = j % SCHED_DEPTH;
+        // claim the next unit while this one is queued: cancel a CTA that has not started
+        bool asked = false;
+        if (ticket < total && may_cancel) {
+          fence_proxy_async();  // the last answer was read (generic proxy) before the next is written
+          mbar_arrive_expect_tx(clc_bar, 16);
+          clc_try_cancel(clc_resp, clc_bar);
+          asked = true;
+        }
+        // stay at most two units ahead of the producer, so that unclaimed work stays with CTAs
+        // that reach it first (the tail stays balanced)
+        bool ok = true;
+        if (j >= 2) ok = mbar_wait(&staken[(j - 2) % SCHED_DEPTH], ((j - 2) / SCHED_DEPTH) & 1, status);
+        if (ok) ok = mbar_wait(&sempty[slot], ((j / SCHED_DEPTH) & 1) ^ 1, status);
+        if (ok) {
+          if (ticket < total && !status_set(status)) ring[slot] = fused_decode(P, cnt, ticket);
+          else ring[slot].t = -1;
+          mbar_arrive(&sfull[slot]);
+        }
+        const bool last = !ok || ring[slot].t < 0;
+        if (asked) {
+          // the answer lands in this CTA's shared memory: wait for it (bounded by time only,
+          // also after an error) before the CTA can end
+          mbar_wait_drain(clc_bar, clc_phase);
+          if (!mbar_try_wait(clc_bar, clc_phase)) {
+            raise_status(status, MOE_ERR_DEVICE_TIMEOUT);
+            break;
+          }
+          clc_phase ^= 1;
+          if (!clc_cancelled(clc_resp)) may_cancel = false;  // no CTA left to take over
+        }
+        if (last) break;
+        ticket = atomicAdd(P.ctl, 1);
+      }
+      // Out of units: cancel the CTAs that have not started yet, so that they never launch
+      // only to find no work.  This overlaps with the last units of this CTA's roles.
+      while (may_cancel && !status_set(status)) {
+        fence_proxy_async();
+        mbar_arrive_expect_tx(clc_bar, 16);
+        clc_try_cancel(clc_resp, clc_bar);
+        mbar_wait_drain(clc_bar, clc_phase);
+        if (!mbar_try_wait(clc_bar, clc_phase)) {
+          raise_status(status, MOE_ERR_DEVICE_TIMEOUT);
+          break;
+        }
+        clc_phase ^= 1;
+        may_cancel = clc_cancelled(clc_resp);
+      }
+    }
+  } else if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      const uint64_t pol_act = policy_evict_last();
+      const uint64_t pol_w = policy_evict_first();
+      const int ngu_n = ntiles_n<G_GATEUP>(P.gu);
+      const int poff0 = __ldg(P.gu.poff);
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_parity[STAGES];
+      for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
+      bool ok = true;
+      for (int j = 0; ok; ++j) {
+        Tile tl;
+        const int slot = j % SCHED_DEPTH;
+        if (!mbar_wait(&sfull[slot], (j / SCHED_DEPTH) & 1, status)) break;
+        tl = ring[slot];
+        mbar_arrive(&sempty[slot]);
+        mbar_arrive(&staken[slot]);
+        if (tl.t < 0) break;
+        if (tl.u == FU_DOWN) {
+          // every gate/up tile of these 128 rows has stored its H rows
+          if (!wait_count(hcnt + ((tl.m0 - poff0) >> 7), 4 * ngu_n, status)) { ok = false; break; }
+          fence_proxy_async_global();
+        }
+        for (int kb = 0; kb < tl.nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, status)) { ok = false; break; }
+          uint8_t* sA = smem + stage * GEMM_STAGE_BYTES;
+          uint8_t* sB = sA + GEMM_A_BYTES;
+          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(GEMM_STAGE_BYTES));
+          if (tl.u == FU_GATEUP) load_stage<G_GATEUP>(P.gu, tl, kb, sA, sB, &full[stage], pol_act, pol_w);
+          else load_stage<G_DOWN>(P.dn, tl, kb, sA, sB, &full[stage], pol_act, pol_w);
+          last_parity[stage] = static_cast<int>(phase);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < STAGES; ++s)
+          if (last_parity[s] >= 0) mbar_wait_drain(&full[s], static_cast<uint32_t>(last_parity[s]));
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer: GEMM units only ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int g = 0;  // GEMM units so far: picks the accumulator
+      bool ok = true;
+      for (int j = 0; ok; ++j) {
+        Tile tl;
+        if (!next_tile(ring, sfull, sempty, j, tl, status)) break;
+        if (tl.t < 0) break;
+        const int acc = g & 1;
+        const uint32_t accp = (g >> 1) & 1;
+        ++g;
+        if (!mbar_wait(&tempty[acc], accp ^ 1, status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dtm = tbase + acc * GEMM_BN;
+        for (int kb = 0; kb < tl.nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * GEMM_STAGE_BYTES);
+          const uint32_t b0 = a0 + static_cast<uint32_t>(GEMM_A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(dtm, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 2048, 8192, 1024), IDESC,
+                      (kb | kk) != 0 ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        if (tl.nk > 0) umma_commit(&tfull[acc]);
+        else mbar_arrive(&tfull[acc]);
+      }
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0);
+    }
+  } else if (warp >= 2 && warp <= 5) {
+    // ---------------- epilogue warps ----------------
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int poff0 = __ldg(P.gu.poff);
+    int g = 0;
+    for (int it = 0;; ++it) {
+      int ok = 1;
+      Tile tl;
+      const int slot = it % SCHED_DEPTH;
+      if (lane == 0) ok = mbar_wait(&sfull[slot], (it / SCHED_DEPTH) & 1, status) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      __syncwarp();
+      tl = ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sempty[slot]);
+      if (tl.t < 0) break;
+      const int acc = g & 1;
+      const uint32_t accp = (g >> 1) & 1;
+      ++g;
+      if (lane == 0) ok = mbar_wait(&tfull[acc], accp, status) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t taddr = tbase + (static_cast<uint32_t>(quarter * 32) << 16) + acc * GEMM_BN;
+      if (tl.u == FU_GATEUP) epilogue_row<G_GATEUP>(P.gu, tl, row, taddr);
+      else epilogue_row<G_DOWN>(P.dn, tl, row, taddr);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (tl.u == FU_GATEUP) warp_release_count(hcnt + ((tl.m0 - poff0) >> 7), lane);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+int64_t fused_fwd_units(int64_t RP, int d, int I) { return (RP / 128) * (I / 128 + d / 256); }
+
+cudaError_t launch_fused_fwd(const FusedFwdParams& p, int64_t grid, cudaStream_t st) {
+  static bool configured[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(k_moe_fwd_gemms, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(fused_smem_bytes()));
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  if (grid < 1 || grid > 0x7fffffff) return cudaErrorInvalidValue;
+  k_moe_fwd_gemms<<<static_cast<unsigned>(grid), GEMM_THREADS_SCHED, fused_smem_bytes(), st>>>(p);
+  return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -104,6 +104,7 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->daqs = take(mxi / 32);
   L->dbq = take(mxi);
   L->dbqs = take(mxi / 32);
+  L->fctl = take(M > 0 || L->mx ? 0 : static_cast<size_t>(fused_ctl_words(L->RP)) * 4);
   L->ws_bytes = o;
   // prepared weights: [W_gate|W_up paired, K = d] [W_down^T, K = I] [W_down, K = d] [W_gate, K = I] [W_up, K = I]
   o = 0;
@@ -156,6 +157,7 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
     c.tab.ring_start = t;
   }
   c.acc32 = nullptr;
+  c.fctl = nullptr;
   c.actcnt = c.actlist = nullptr;
   c.xact = nullptr;
   c.xq = L.mx ? reinterpret_cast<uint8_t*>(C(L.xq)) : nullptr;
@@ -188,6 +190,7 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
     c.wrt = reinterpret_cast<__nv_bfloat16*>(W(L.wrt));
     c.dxperm = reinterpret_cast<__nv_bfloat16*>(W(L.dxperm));
     c.acc32 = L.M > 0 ? reinterpret_cast<float*>(W(L.acc32)) : nullptr;
+    c.fctl = L.M == 0 && !L.mx ? reinterpret_cast<int*>(W(L.fctl)) : nullptr;
     if (L.rslice) {
       c.actcnt = reinterpret_cast<int*>(W(L.actcnt));
       c.actlist = reinterpret_cast<int*>(W(L.actlist));
@@ -283,14 +286,15 @@ enum KernelId {
   K_ROUTER_LOGITS, K_TOPK, K_SCAN, K_SCATTER, K_DISPATCH, K_GEMM_GATEUP, K_GEMM_DOWN, K_COMBINE,
   K_REV_COMBINE, K_GEMM_DGRAD_DOWN, K_ROUTER_BWD, K_ROUTER_WGRAD, K_TRANSPOSE_WR, K_GEMM_DGRAD_GATEUP, K_REV_DISPATCH,
   K_GEMM_WGRAD_GATEUP, K_GEMM_WGRAD_DOWN, K_PLAN, K_REPLAY, K_FINISH_ACC, K_QUANT_WEIGHTS, K_MARK_ROWS,
-  K_ACTIVE_COUNT, K_GATHER_ACTIVE, K_SCAN_GROUPS, K_SCAN_APPLY, K_NUM
+  K_ACTIVE_COUNT, K_GATHER_ACTIVE, K_SCAN_GROUPS, K_SCAN_APPLY, K_FUSED_FWD, K_NUM
 };
 static const char* kKernelNames[K_NUM] = {
     "router_logits", "topk_gating", "hist_scan", "stable_scatter", "dispatch", "gemm_gateup_swiglu",
     "gemm_down_combw", "combine", "reverse_combine", "gemm_dgrad_down_swiglu_bwd", "router_bwd", "router_wgrad",
     "transpose_wr", "gemm_dgrad_gateup", "reverse_dispatch", "gemm_wgrad_gateup", "gemm_wgrad_down",
     "stream_plan", "ring_replay", "wgrad_accumulator_finish", "quantize_weights", "mark_pad_rows",
-    "router_token_count", "router_token_gather", "hist_scan_group_sums", "hist_scan_group_apply"};
+    "router_token_count", "router_token_gather", "hist_scan_group_sums", "hist_scan_group_apply",
+    "gemm_gateup_down_persistent"};
 
 struct ProfRec {
   int kid;
@@ -546,6 +550,61 @@ moe_status moe_fwd(const moe_shape* s, const void* X, const void* W_r, const flo
     MOE_TRY(timed(K_GEMM_DOWN, st, [&] { return launch_gemm(G_DOWN, p, grid, st); }));
   }
   // 7. combine
+  MOE_TRY(timed(K_COMBINE, st, [&] { return launch_combine(L, c, c.obuf, static_cast<__nv_bfloat16*>(Y), st); }));
+  return MOE_OK;
+}
+
+// The forward with its two grouped GEMMs in one persistent launch: the same routing, dispatch
+// and combine launches as moe_fwd around k_moe_fwd_gemms.
+moe_status moe_fwd_persistent(const moe_shape* s, const void* X, const void* W_r, const float* bias,
+                              const void* W_gate, const void* W_up, const void* W_down, void* Y, void* ctx,
+                              size_t ctx_bytes, void* ws, size_t ws_bytes, void* stream) {
+  Layout L;
+  const moe_status cs = check_shape(s, &L);
+  if (cs != MOE_OK) return cs;
+  const bool tok = s->T > 0;
+  if ((tok && (!X || !Y)) || !W_r || !W_gate || !W_up || !W_down || !ctx || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W_r) || !aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_down) ||
+      !aligned16(Y) || !aligned16(ctx) || !aligned16(ws) || (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+    return MOE_ERR_INVALID_ARG;
+  if (ctx_bytes < L.ctx_bytes || ws_bytes < L.ws_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ctx c = make_ctx(L, ctx, ws);
+  MOE_TRY(cudaMemsetAsync(c.hdr, 0, HDR_WORDS * 4, st));
+  if (L.T == 0) return MOE_OK;
+
+  int* status = c.hdr + HDR_STATUS;
+  const uint64_t RP = static_cast<uint64_t>(L.RP);
+  {
+    const moe_status r = route_tokens(L, c, X, W_r, bias, 0, st);
+    if (r != MOE_OK) return r;
+  }
+  MOE_TRY(timed(K_DISPATCH, st, [&] {
+    return launch_gather_rows(L, c, static_cast<const __nv_bfloat16*>(X), c.xperm, st);
+  }));
+  FusedFwdParams f;
+  f.gu = base_params(L, c, status);
+  MOE_TMAP(tmap_2d(&f.gu.ta0, c.xperm, L.d, RP, L.d, 64, 128));
+  MOE_TMAP(tmap_2d(&f.gu.tb0, W_gate, L.I, static_cast<uint64_t>(L.El) * L.d, L.I, 64, 64));
+  MOE_TMAP(tmap_2d(&f.gu.tb1, W_up, L.I, static_cast<uint64_t>(L.El) * L.d, L.I, 64, 64));
+  f.gu.ta1 = f.gu.ta0;
+  f.gu.out0 = c.abuf;
+  f.gu.out1 = c.bbuf;
+  f.gu.out2 = c.hbuf;
+  f.dn = base_params(L, c, status);
+  MOE_TMAP(tmap_2d(&f.dn.ta0, c.hbuf, L.I, RP, L.I, 64, 128));
+  MOE_TMAP(tmap_2d(&f.dn.tb0, W_down, L.d, static_cast<uint64_t>(L.El) * L.I, L.d, 64, 64));
+  f.dn.ta1 = f.dn.ta0;
+  f.dn.tb1 = f.dn.tb0;
+  f.dn.out0 = c.obuf;
+  f.ctl = c.fctl;
+  f.mt_cap = static_cast<int>(L.RP / 128);
+  MOE_TRY(cudaMemsetAsync(c.fctl, 0, static_cast<size_t>(fused_ctl_words(L.RP)) * 4, st));
+  // two CTAs per SM at most: the first wave runs, the rest is taken over through Cluster Launch
+  // Control by whichever CTAs claim work first (fewer when there are fewer tiles)
+  const int64_t units = fused_fwd_units(L.RP, L.d, L.I);
+  const int64_t grid = units < 2LL * num_sms() ? units : 2LL * num_sms();
+  MOE_TRY(timed(K_FUSED_FWD, st, [&] { return launch_fused_fwd(f, grid, st); }));
   MOE_TRY(timed(K_COMBINE, st, [&] { return launch_combine(L, c, c.obuf, static_cast<__nv_bfloat16*>(Y), st); }));
   return MOE_OK;
 }

@@ -69,7 +69,7 @@ struct Layout {
       bbuf, stab, xq, xqs, ctx_bytes;
   // ws
   size_t hist, hsum, logits, rpart, hbuf, obuf, dyperm, dabuf, dbbuf, hgbuf, dgpart, dlasg, dldense, wrt, dxperm, acc32, hq, hqs, dyq,
-      dyqs, daq, daqs, dbq, dbqs, actcnt, actlist, xact, ws_bytes;
+      dyqs, daq, daqs, dbq, dbqs, actcnt, actlist, xact, fctl, ws_bytes;
   bool mx;   // MXFP8 mode
   bool w32;  // expert weight gradients written as fp32
   bool rslice;  // an expert slice (El < E): the router weight gradient runs over the listed tokens
@@ -152,6 +152,21 @@ cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream
 // Loads the kernel of one GEMM kind (and sets its shared-memory attribute) without launching it,
 // so that a later launch needs no lazy module loading.
 cudaError_t preload_gemm(GemmKind kind);
+
+// The forward's gate/up and down GEMMs in one persistent launch (gemm.cu): every gate/up
+// tile, then every down tile, as work units that CTAs take from one ticket counter in one
+// global order, CTAs that have not started claimed through Cluster Launch Control.  A down
+// tile waits (bounded) until every gate/up tile of its 128 rows has stored its H rows.
+struct FusedFwdParams {
+  GemmParams gu;  // the gate/up GEMM's parameters (ta0 = X_perm; A, B, H outputs)
+  GemmParams dn;  // the down GEMM's parameters (ta0 = H; O' output)
+  int* ctl;       // fused_ctl_words(RP) ints, zero before the launch
+  int mt_cap;     // m-tile capacity of ctl (RP / 128)
+};
+constexpr int64_t fused_ctl_words(int64_t RP) { return 1 + RP / 128; }
+// Upper bound of the work units (gate/up and down tiles at RP rows).
+int64_t fused_fwd_units(int64_t RP, int d, int I);
+cudaError_t launch_fused_fwd(const FusedFwdParams& p, int64_t grid, cudaStream_t st);
 
 // 2-D bf16 tensor map [outer, inner] (inner contiguous, row pitch in elements), box
 // {box_inner, box_outer}, 128-byte swizzle, zero fill out of bounds (moe_api.cu).
@@ -237,6 +252,7 @@ struct Ctx {  // typed views of ctx + ws for one shape
   int* actcnt;               // expert slice: token counts per 256-token block, then the list length
   int* actlist;              // expert slice: the tokens with a local assignment, ascending
   __nv_bfloat16* xact;       // expert slice: their X rows [Tpad, d] (rows past the list up to a multiple of 64: 0)
+  int* fctl;                 // control block of the one-launch forward expert phase (fused_ctl_words(RP) ints)
   StreamTables tab;
   uint8_t *xq, *xqs, *hq, *hqs, *dyq, *dyqs, *daq, *daqs, *dbq, *dbqs;  // MXFP8 operands and scales
 };

@@ -81,7 +81,7 @@ for _n in (512, 1024, 2048, 2368, 4096, 8192, 16384):
 # The same per-rank slice (6 of 384 experts, 32768 tokens, n per local expert) as one batch, the
 # dispatched rows held whole instead of in a ring: MXFP8 (epmx) and bf16 (epbf), the regime
 # where the grouped GEMMs are bound by the tensor cores rather than by the weight stream.
-for _n in (2368, 4096, 8192):
+for _n in (512, 2368, 4096, 8192):
     WORKLOADS[f"epmx_n{_n}"] = Workload(f"epmx_n{_n}", 32768, 7168, 384, 8, 2048, mxfp8=True, first_local=0,
                                         num_local=6, local_tokens=_n)
     WORKLOADS[f"epbf_n{_n}"] = Workload(f"epbf_n{_n}", 32768, 7168, 384, 8, 2048, first_local=0, num_local=6,

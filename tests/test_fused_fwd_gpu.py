@@ -1,0 +1,92 @@
+"""The forward's two grouped GEMMs in one persistent launch (`moe_fwd_persistent`).
+
+The gate/up GEMM with SwiGLU and the down GEMM with the gate multiply run as work units of one
+kernel, taken by CTAs in one global order and claimed through Cluster Launch Control; a down tile
+waits for the gate/up tiles of its rows.  Each unit computes what the separate launches of
+`moe_fwd` compute, with the same tiles and epilogues, so Y and everything saved in ctx must be the
+same bits, and a
+`moe_bwd` after it must give the same gradients bit for bit.  Y and the gradients must also match
+the fp64 oracle within the bf16 tolerance, and repeated runs must be bit-identical.
+"""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_layer_27_b200 import binding as B
+
+from _util import TOL_BF16, make_case, relerr, run_oracle, to64
+
+pytestmark = pytest.mark.gpu
+
+
+def _step(layer, x, first, El, persistent, poison=False):
+    if poison:  # every byte the step may read before writing it holds a NaN pattern
+        layer.ctx.fill_(0xFF)
+        layer.ws.fill_(0xFF)
+    W = [x[n][first:first + El].contiguous() for n in ("W_gate", "W_up", "W_down")]
+    Y = layer.forward(x["X"], x["W_r"], x["bias"], *W, persistent=persistent)
+    g = layer.backward(x["X"], x["W_r"], *W, x["dY"])
+    torch.cuda.synchronize()
+    assert layer.error() == B.MOE_OK
+    return Y, g
+
+
+def _bits(t):
+    return t.view(torch.int16) if t.dtype == torch.bfloat16 else t.view(torch.int32)
+
+
+def _check(T, d, E, k, I, seed, bias=None, first=0, num=0, oracle=True):
+    w, x = make_case(T, d, E, k, I, seed=seed, bias=bias)
+    El = num or (E - first)
+    ref = B.MoELayer(T, d, E, I, k, first_local_expert=first, num_local_experts=num)
+    fus = B.MoELayer(T, d, E, I, k, first_local_expert=first, num_local_experts=num)
+    Y0, g0 = _step(ref, x, first, El, persistent=False)
+    Y1, g1 = _step(fus, x, first, El, persistent=True, poison=True)
+    assert torch.equal(_bits(Y1), _bits(Y0))
+    for n in g0:
+        assert torch.equal(_bits(g1[n]), _bits(g0[n])), n
+    r0, r1 = ref.routing(), fus.routing()
+    for n in r0:
+        assert torch.equal(r0[n], r1[n]), n
+    # run to run: a second persistent step over the same buffers
+    Y2, g2 = _step(fus, x, first, El, persistent=True)
+    assert torch.equal(_bits(Y2), _bits(Y1))
+    assert torch.equal(_bits(g2["dW_gate"]), _bits(g1["dW_gate"]))
+    if oracle:
+        Yo, _, go = run_oracle(x, k, first=first, num=num or None)
+        assert relerr(to64(Y1), Yo) <= TOL_BF16
+        assert relerr(to64(g1["dX"]), go["dX"]) <= TOL_BF16
+        for n in ("W_gate", "W_up", "W_down"):
+            want = np.stack([go["d" + n][e] for e in range(first, first + El)])
+            assert relerr(to64(g1["d" + n]), want) <= TOL_BF16, n
+    return fus
+
+
+def test_persistent_forward_equals_moe_fwd_several_tiles_per_expert():
+    # 600 tokens x 4 over 16 experts: about 150 rows each, two m-tiles, ragged last tiles
+    _check(600, 512, 16, 4, 512, seed=81)
+
+
+def test_persistent_forward_uneven_load_idle_experts_and_a_slice():
+    E = 16
+    bias = np.zeros(E, dtype=np.float32)
+    bias[3] = 4.0   # one hot expert: many m-tiles
+    bias[8:12] = -40.0  # idle experts: empty segments between full ones
+    _check(500, 256, E, 3, 256, seed=82, bias=bias)
+    _check(500, 256, E, 3, 256, seed=83, bias=bias, first=2, num=9)
+
+
+def test_persistent_forward_one_token_and_many_tiles():
+    _check(1, 256, 8, 2, 256, seed=84)
+    _check(1500, 256, 32, 8, 256, seed=85)  # more tiles than two per SM
+
+
+def test_persistent_forward_full_size_deepseek_v3_like_equals_moe_fwd():
+    # T = 2048, d = 7168, E = 256, top-8, I = 2048: bit for bit against the multi-launch forward
+    # (the oracle comparisons at this size live in test_fullsize_gpu.py)
+    _check(2048, 7168, 256, 8, 2048, seed=0, oracle=False)
+
+
+def test_persistent_forward_ep64_slice_equals_moe_fwd():
+    # 6 of 384 experts, 32,768 tokens (the per-rank slice as one batch)
+    _check(32768, 7168, 384, 8, 2048, seed=86, first=0, num=6, oracle=False)

@@ -65,7 +65,7 @@ def test_reference_arm_runs_on_rank_0_only(capsys):
     from mixture_experts_layer_27_b200 import inputs as IN
 
     class Args:  # the reference arm's arguments; rank 1 must return before doing any work
-        gpus, steps, warmup, wgrad_fp32 = 2, 1, 3, False
+        gpus, steps, warmup, wgrad_fp32, persistent = 2, 1, 3, False, False
     bench.run_reference(Args, IN.WORKLOADS["tiny"], world=2, rank=1)
     assert capsys.readouterr().out == ""
 
@@ -77,7 +77,7 @@ def test_reference_arm_prints_one_line_on_rank_0(capsys):
     from mixture_experts_layer_27_b200 import inputs as IN
 
     class Args:
-        gpus, steps, warmup, wgrad_fp32 = 2, 2, 3, False
+        gpus, steps, warmup, wgrad_fp32, persistent = 2, 2, 3, False, False
     w = IN.WORKLOADS["tiny"]
     bench.run_reference(Args, w, world=2, rank=0)
     lines = capsys.readouterr().out.strip().splitlines()
@@ -86,6 +86,7 @@ def test_reference_arm_prints_one_line_on_rank_0(capsys):
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     # the same config as the GPU arm's line, and a rate that is the timed steps' own
-    assert line["config"] == dict(bench.workload_config(w), wgrad_dtype="bf16")
+    assert line["config"] == bench.run_config(w, Args)
+    assert line["config"]["wgrad_dtype"] == "bf16" and line["config"]["forward"] == "launches"
     tokens = bench.oracle_sample(w, bench.cpu_inputs(w))[1] / w.k  # tokens of work per step
     assert abs(line["value"] * line["ms_per_step"] / 1e3 - tokens) < 1e-6 * tokens
