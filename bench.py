@@ -147,6 +147,7 @@ def algorithmic_flops(w: IN.Workload) -> dict:
             "gemm_wgrad_gateup": 4 * dI * rows, "gemm_wgrad_down": 2 * dI * rows,
             "router_logits": 2 * w.tokens * w.d * w.E,
             "gemm_gateup_down_persistent": 6 * dI * rows,  # gate/up and down in one launch
+            "gemm_dgrads_persistent": 6 * dI * rows,  # both dgrads in one launch
             # dW_r = X^T dl; the kernel issues it twice (the hi and lo bf16 terms of dl)
             "router_wgrad": 2 * w.tokens * w.d * w.E}
 
@@ -196,6 +197,9 @@ def algorithmic_bytes(w: IN.Workload, wgrad_elem_bytes: int = 2) -> dict:
         # gate/up and down in one launch: the weights, X_perm in, A and B (saved) and O' out;
         # H passes between two tiles of the launch and is not counted
         "gemm_gateup_down_persistent": 3 * W1 + rows * d * 2 + 2 * rows * I * 2 + rows * d * 2,
+        # both dgrads in one launch: the weights, dY_perm, A and B in; dA, dB, Hg and dX_perm out
+        # (dA, dB read back by the dgrad of gate/up within the launch are not counted again)
+        "gemm_dgrads_persistent": 3 * W1 + rows * d * 2 + 2 * rows * I * 2 + 3 * rows * I * 2 + rows * d * 2,
     }
 
 
@@ -480,7 +484,7 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     elif args.persistent:
         def step(X, dY, Yout, g):
             layer.forward(X, x["W_r"], x["bias"], x["W_gate"], x["W_up"], x["W_down"], Y=Yout, persistent=True)
-            layer.backward(X, x["W_r"], x["W_gate"], x["W_up"], x["W_down"], dY, out=g)
+            layer.backward(X, x["W_r"], x["W_gate"], x["W_up"], x["W_down"], dY, out=g, persistent=True)
     else:
         def step(X, dY, Yout, g):
             layer.forward(X, x["W_r"], x["bias"], x["W_gate"], x["W_up"], x["W_down"], Y=Yout)
@@ -749,14 +753,20 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="time direct launches instead of a CUDA graph of one step")
     ap.add_argument("--wgrad-fp32", action="store_true",
                     help="write the expert weight gradients as fp32 instead of bf16 (the weights' dtype)")
+    ap.add_argument("--launches", action="store_true",
+                    help="run every grouped GEMM as its own launch instead of the persistent pairs")
     ap.add_argument("--persistent", action="store_true",
-                    help="run the forward's gate/up and down GEMMs as one persistent launch (bf16, one batch)")
+                    help="require the persistent pairs (the default for bf16 one-batch workloads): the forward's "
+                         "gate/up and down GEMMs, and the backward's two dgrads, each pair as one persistent launch")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = IN.WORKLOADS[args.workload]
-    if args.persistent and (w.mxfp8 or w.stream_M):
-        ap.error("--persistent runs the bf16 one-batch layer; %s is %s" % (w.name, "MXFP8" if w.mxfp8 else "streamed"))
+    if args.persistent and (w.mxfp8 or w.stream_M or args.launches):
+        ap.error("--persistent runs the bf16 one-batch layer with persistent GEMM pairs; %s" %
+                 ("--launches was given" if args.launches else "%s is %s" % (w.name, "MXFP8" if w.mxfp8 else "streamed")))
+    # the persistent GEMM pairs (measured 1-3% faster on those GEMMs) wherever the layer has them
+    args.persistent = not (args.launches or w.mxfp8 or w.stream_M)
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

@@ -139,6 +139,17 @@ moe_status moe_bwd(const moe_shape* shape, const void* X, const void* W_r, const
                    void* dX, void* dW_gate, void* dW_up, void* dW_down, float* dW_r,
                    void* ws, size_t ws_bytes, void* stream);
 
+/* Backward with its two dgrad GEMMs in one persistent launch, as moe_fwd_persistent does for the
+ * forward: every tile of the dgrad of W_down (SwiGLU backward and router-gate gradient
+ * epilogue), then every tile of the dgrad of gate/up, which waits (bounded) for the dgrad of
+ * W_down's tiles of its 128 rows.  The router backward runs after that launch instead of
+ * between the two GEMMs.  Same arguments and results as moe_bwd, bit for bit; bf16 mode, one
+ * batch.  Follows either forward. */
+moe_status moe_bwd_persistent(const moe_shape* shape, const void* X, const void* W_r, const void* W_gate,
+                              const void* W_up, const void* W_down, const void* dY, void* ctx,
+                              size_t ctx_bytes, void* dX, void* dW_gate, void* dW_up, void* dW_down,
+                              float* dW_r, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, returns the device status word held in `ctx`
  * (MOE_OK if no device error since the last moe_fwd), and clears it.
  * Returns MOE_ERR_CUDA if the synchronisation itself failed. */

@@ -75,6 +75,8 @@ _SIGS = {
                                           _P]),
     "moe_bwd": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, _P, _P, _P, _P,
                                ctypes.c_size_t, _P]),
+    "moe_bwd_persistent": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, _P, _P, _P, _P,
+                                          ctypes.c_size_t, _P]),
     "moe_get_error": (ctypes.c_int, [_P, _P]),
     "moe_debug_routing": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_debug_logits": (ctypes.c_int, [_S, _P, _P, _P]),
@@ -182,11 +184,12 @@ def moe_fwd_persistent(shape, X, W_r, bias, W_gate, W_up, W_down, Y, ctx, ws, st
 
 
 def moe_bwd(shape, X, W_r, W_gate, W_up, W_down, dY, ctx, dX, dW_gate, dW_up, dW_down, dW_r, ws, stream=None,
-            ctx_bytes=None, ws_bytes=None):
-    return int(lib().moe_bwd(ctypes.byref(shape), _ptr(X), _ptr(W_r), _ptr(W_gate), _ptr(W_up), _ptr(W_down),
-                             _ptr(dY), _ptr(ctx), ctx_bytes if ctx_bytes is not None else _nbytes(ctx), _ptr(dX),
-                             _ptr(dW_gate), _ptr(dW_up), _ptr(dW_down), _ptr(dW_r), _ptr(ws),
-                             ws_bytes if ws_bytes is not None else _nbytes(ws), _stream(stream)))
+            ctx_bytes=None, ws_bytes=None, persistent=False):
+    fn = lib().moe_bwd_persistent if persistent else lib().moe_bwd
+    return int(fn(ctypes.byref(shape), _ptr(X), _ptr(W_r), _ptr(W_gate), _ptr(W_up), _ptr(W_down), _ptr(dY),
+                  _ptr(ctx), ctx_bytes if ctx_bytes is not None else _nbytes(ctx), _ptr(dX), _ptr(dW_gate),
+                  _ptr(dW_up), _ptr(dW_down), _ptr(dW_r), _ptr(ws), ws_bytes if ws_bytes is not None else _nbytes(ws),
+                  _stream(stream)))
 
 
 def moe_get_error(ctx, stream=None) -> int:
@@ -535,7 +538,7 @@ class MoELayer:
         self.El = num_local_experts or (E - first_local_expert)
 
     def forward(self, X, W_r, bias, W_gate, W_up, W_down, Y=None, stream=None, persistent=False):
-        """persistent: the expert phase as one persistent launch (moe_fwd_persistent); same results."""
+        """persistent: the two GEMMs as one persistent launch (moe_fwd_persistent); same results."""
         import torch
         if Y is None:
             Y = torch.empty(self.T, self.d, dtype=torch.bfloat16, device=X.device)
@@ -543,12 +546,14 @@ class MoELayer:
         check(fn(self.shape, X, W_r, bias, W_gate, W_up, W_down, Y, self.ctx, self.ws, stream), name)
         return Y
 
-    def backward(self, X, W_r, W_gate, W_up, W_down, dY, out=None, stream=None):
+    def backward(self, X, W_r, W_gate, W_up, W_down, dY, out=None, stream=None, persistent=False):
+        """persistent: the two dgrad GEMMs as one persistent launch (moe_bwd_persistent); same results."""
         import torch
         if out is None:
             out = _grad_buffers(self.T, self.d, self.E, self.I, self.El, self.wgrad_dtype, X.device)
         check(moe_bwd(self.shape, X, W_r, W_gate, W_up, W_down, dY, self.ctx, out["dX"], out["dW_gate"],
-                      out["dW_up"], out["dW_down"], out["dW_r"], self.ws, stream), "moe_bwd")
+                      out["dW_up"], out["dW_down"], out["dW_r"], self.ws, stream, persistent=persistent),
+              "moe_bwd_persistent" if persistent else "moe_bwd")
         return out
 
     def routing(self):

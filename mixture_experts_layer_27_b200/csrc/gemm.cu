@@ -855,19 +855,22 @@ cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream
 }
 
 // ===========================================================================
-// The forward's grouped GEMMs in one persistent launch
+// Two dependent grouped GEMMs in one persistent launch
 // ===========================================================================
-// Work units, in ticket order: every gate/up tile, then every down tile.  A CTA takes a ticket
+// The forward's gate/up and down GEMMs, or the backward's dgrad of W_down and dgrad of
+// gate/up: the second GEMM of the pair reads, for its 128 rows, what every tile of the first
+// GEMM wrote for those rows (H; or dA and dB).  Work units, in ticket order: every tile of the
+// first GEMM, then every tile of the second.  A CTA takes a ticket
 // when it starts and one for each further unit it claims.  While the grid still has CTAs that
 // have not started, a claim is the cancellation of one of them through Cluster Launch Control
 // (its work moves to the running CTA); once the hardware reports none left, claims come from
 // the ticket counter alone, until the tickets run past the last unit.  So the work spreads
-// over the CTAs that actually run, whatever the grid size, and down tiles fill the SMs that
-// the last round of gate/up tiles leaves idle.  A down tile waits (bounded) until every
-// gate/up tile of its 128 rows has stored its H rows.  Tickets are handed out in one global
-// order and a down tile only waits for gate/up tiles, which have lower tickets and are held
-// by running (or finished) CTAs, so the waits end.  Every wait gives up once the status word
-// is set.
+// over the CTAs that actually run, whatever the grid size, and second-GEMM tiles fill the SMs
+// that the last round of first-GEMM tiles leaves idle.  A second-GEMM tile waits (bounded)
+// until every first-GEMM tile of its 128 rows has stored its rows.  Tickets are handed out in
+// one global order and a second-GEMM tile only waits for first-GEMM tiles, which have lower
+// tickets and are held by running (or finished) CTAs, so the waits end.  Every wait gives up
+// once the status word is set.
 //
 // A unit computes exactly what the separate GEMM launches compute (the same decode, loads and
 // epilogue functions), so the results are the same bits.
@@ -876,31 +879,33 @@ cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream
 // epilogue warps.  With one CTA per SM those warps keep too few loads in flight for a copy:
 // traced per unit, the combine ran 12x and the dispatch 2x slower than their own kernels, and
 // gate/up tiles stalled behind the dispatch.
-enum FusedUnit { FU_GATEUP = 1, FU_DOWN = 2 };
+enum PairUnit { FU_FIRST = 1, FU_SECOND = 2 };
 
-// ctl: [0] ticket counter, [1, 1 + cap) gate/up epilogue warps done per m-tile.
-struct FusedCounts {
-  int mt, ngu, ndn;
-  __device__ int total() const { return ngu + ndn; }
+// ctl: [0] ticket counter, [1, 1 + cap) first-GEMM epilogue warps done per m-tile.
+struct PairCounts {
+  int mt, n1, n2;
+  __device__ int total() const { return n1 + n2; }
 };
-__device__ __forceinline__ FusedCounts fused_counts(const FusedFwdParams& P) {
-  FusedCounts c;
-  c.mt = (__ldg(P.gu.poff + P.gu.nseg) - __ldg(P.gu.poff)) / 128;
-  c.ngu = c.mt * ntiles_n<G_GATEUP>(P.gu);
-  c.ndn = c.mt * ntiles_n<G_DOWN>(P.dn);
+template <int K1, int K2>
+__device__ __forceinline__ PairCounts pair_counts(const GemmPairParams& P) {
+  PairCounts c;
+  c.mt = (__ldg(P.p1.poff + P.p1.nseg) - __ldg(P.p1.poff)) / 128;
+  c.n1 = c.mt * ntiles_n<K1>(P.p1);
+  c.n2 = c.mt * ntiles_n<K2>(P.p2);
   return c;
 }
-__device__ __forceinline__ Tile fused_decode(const FusedFwdParams& P, const FusedCounts& c, int t) {
+template <int K1, int K2>
+__device__ __forceinline__ Tile pair_decode(const GemmPairParams& P, const PairCounts& c, int t) {
   Tile tl;
-  if (t < c.ngu) {
-    tl = decode<G_GATEUP>(P.gu, t);
-    tl.u = FU_GATEUP;
+  if (t < c.n1) {
+    tl = decode<K1>(P.p1, t);
+    tl.u = FU_FIRST;
     return tl;
   }
-  t -= c.ngu;
-  if (t < c.ndn) {
-    tl = decode<G_DOWN>(P.dn, t);
-    tl.u = FU_DOWN;
+  t -= c.n1;
+  if (t < c.n2) {
+    tl = decode<K2>(P.p2, t);
+    tl.u = FU_SECOND;
     return tl;
   }
   tl.t = -1;
@@ -937,7 +942,8 @@ __device__ __forceinline__ void warp_release_count(int* p, int lane) {
 constexpr size_t FUSED_TAIL_BYTES = 1024;
 constexpr size_t fused_smem_bytes() { return GEMM_STAGES * GEMM_STAGE_BYTES + 1024 + FUSED_TAIL_BYTES; }
 
-__global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_fwd_gemms(const __grid_constant__ FusedFwdParams P) {
+template <int K1, int K2>
+__global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_gemm_pair(const __grid_constant__ GemmPairParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int STAGES = GEMM_STAGES;
@@ -953,7 +959,7 @@ __global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_fwd_gemms(const _
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(clc_bar + 1);
   uint4* clc_resp = reinterpret_cast<uint4*>((reinterpret_cast<uintptr_t>(clc_bar + 2) + 15) & ~uintptr_t(15));
   Tile* ring = reinterpret_cast<Tile*>(clc_resp + 1);
-  int* status = P.gu.status;
+  int* status = P.p1.status;
   int* hcnt = P.ctl + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -976,11 +982,14 @@ __global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_fwd_gemms(const _
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&P.gu.ta0);
-    prefetch_tmap(&P.gu.tb0);
-    prefetch_tmap(&P.gu.tb1);
-    prefetch_tmap(&P.dn.ta0);
-    prefetch_tmap(&P.dn.tb0);
+    prefetch_tmap(&P.p1.ta0);
+    prefetch_tmap(&P.p1.ta1);
+    prefetch_tmap(&P.p1.tb0);
+    prefetch_tmap(&P.p1.tb1);
+    prefetch_tmap(&P.p2.ta0);
+    prefetch_tmap(&P.p2.ta1);
+    prefetch_tmap(&P.p2.tb0);
+    prefetch_tmap(&P.p2.tb1);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -990,14 +999,15 @@ __global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_fwd_gemms(const _
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  constexpr uint32_t IDESC = idesc_bf16(GEMM_BM, GEMM_BN, false, true);  // both kinds: A K-major, B MN-major
-  static_assert(!Traits<G_GATEUP>::A_MN && Traits<G_GATEUP>::B_MN && !Traits<G_DOWN>::A_MN && Traits<G_DOWN>::B_MN,
-                "the fused forward issues one instruction descriptor for both GEMMs");
+  static_assert(Traits<K1>::A_MN == Traits<K2>::A_MN && Traits<K1>::B_MN == Traits<K2>::B_MN && !Traits<K1>::A_MN,
+                "one instruction descriptor serves both GEMMs of the pair");
+  constexpr bool B_MN = Traits<K1>::B_MN;
+  constexpr uint32_t IDESC = idesc_bf16(GEMM_BM, GEMM_BN, false, B_MN);
 
   if (warp == 6) {
     if (lane == 0) {
       // ---------------- scheduler: tickets in, decoded units into the ring ----------------
-      const FusedCounts cnt = fused_counts(P);
+      const PairCounts cnt = pair_counts<K1, K2>(P);
       const int total = cnt.total();
       uint32_t clc_phase = 0;
       bool may_cancel = true;  // false after an answer that cancelled nothing
@@ -1018,7 +1028,7 @@ __global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_fwd_gemms(const _
         if (j >= 2) ok = mbar_wait(&staken[(j - 2) % SCHED_DEPTH], ((j - 2) / SCHED_DEPTH) & 1, status);
         if (ok) ok = mbar_wait(&sempty[slot], ((j / SCHED_DEPTH) & 1) ^ 1, status);
         if (ok) {
-          if (ticket < total && !status_set(status)) ring[slot] = fused_decode(P, cnt, ticket);
+          if (ticket < total && !status_set(status)) ring[slot] = pair_decode<K1, K2>(P, cnt, ticket);
           else ring[slot].t = -1;
           mbar_arrive(&sfull[slot]);
         }
@@ -1057,8 +1067,8 @@ __global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_fwd_gemms(const _
       // ---------------- TMA producer ----------------
       const uint64_t pol_act = policy_evict_last();
       const uint64_t pol_w = policy_evict_first();
-      const int ngu_n = ntiles_n<G_GATEUP>(P.gu);
-      const int poff0 = __ldg(P.gu.poff);
+      const int n1_n = ntiles_n<K1>(P.p1);
+      const int poff0 = __ldg(P.p1.poff);
       int stage = 0;
       uint32_t phase = 0;
       int last_parity[STAGES];
@@ -1072,9 +1082,9 @@ __global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_fwd_gemms(const _
         mbar_arrive(&sempty[slot]);
         mbar_arrive(&staken[slot]);
         if (tl.t < 0) break;
-        if (tl.u == FU_DOWN) {
-          // every gate/up tile of these 128 rows has stored its H rows
-          if (!wait_count(hcnt + ((tl.m0 - poff0) >> 7), 4 * ngu_n, status)) { ok = false; break; }
+        if (tl.u == FU_SECOND) {
+          // every first-GEMM tile of these 128 rows has stored its rows
+          if (!wait_count(hcnt + ((tl.m0 - poff0) >> 7), 4 * n1_n, status)) { ok = false; break; }
           fence_proxy_async_global();
         }
         for (int kb = 0; kb < tl.nk; ++kb) {
@@ -1082,8 +1092,8 @@ __global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_fwd_gemms(const _
           uint8_t* sA = smem + stage * GEMM_STAGE_BYTES;
           uint8_t* sB = sA + GEMM_A_BYTES;
           mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(GEMM_STAGE_BYTES));
-          if (tl.u == FU_GATEUP) load_stage<G_GATEUP>(P.gu, tl, kb, sA, sB, &full[stage], pol_act, pol_w);
-          else load_stage<G_DOWN>(P.dn, tl, kb, sA, sB, &full[stage], pol_act, pol_w);
+          if (tl.u == FU_FIRST) load_stage<K1>(P.p1, tl, kb, sA, sB, &full[stage], pol_act, pol_w);
+          else load_stage<K2>(P.p2, tl, kb, sA, sB, &full[stage], pol_act, pol_w);
           last_parity[stage] = static_cast<int>(phase);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -1117,7 +1127,8 @@ __global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_fwd_gemms(const _
           const uint32_t b0 = a0 + static_cast<uint32_t>(GEMM_A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_bf16(dtm, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 2048, 8192, 1024), IDESC,
+            umma_bf16(dtm, sdesc_sw128(a0 + kk * 32, 16, 1024),
+                      B_MN ? sdesc_sw128(b0 + kk * 2048, 8192, 1024) : sdesc_sw128(b0 + kk * 32, 16, 1024), IDESC,
                       (kb | kk) != 0 ? 1u : 0u);
           umma_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -1133,7 +1144,7 @@ __global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_fwd_gemms(const _
     // ---------------- epilogue warps ----------------
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int poff0 = __ldg(P.gu.poff);
+    const int poff0 = __ldg(P.p1.poff);
     int g = 0;
     for (int it = 0;; ++it) {
       int ok = 1;
@@ -1156,12 +1167,12 @@ __global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_fwd_gemms(const _
       __syncwarp();
       tc_fence_after();
       const uint32_t taddr = tbase + (static_cast<uint32_t>(quarter * 32) << 16) + acc * GEMM_BN;
-      if (tl.u == FU_GATEUP) epilogue_row<G_GATEUP>(P.gu, tl, row, taddr);
-      else epilogue_row<G_DOWN>(P.dn, tl, row, taddr);
+      if (tl.u == FU_FIRST) epilogue_row<K1>(P.p1, tl, row, taddr);
+      else epilogue_row<K2>(P.p2, tl, row, taddr);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
-      if (tl.u == FU_GATEUP) warp_release_count(hcnt + ((tl.m0 - poff0) >> 7), lane);
+      if (tl.u == FU_FIRST) warp_release_count(hcnt + ((tl.m0 - poff0) >> 7), lane);
     }
   }
   __syncthreads();
@@ -1172,21 +1183,33 @@ __global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_fwd_gemms(const _
   }
 }
 
-int64_t fused_fwd_units(int64_t RP, int d, int I) { return (RP / 128) * (I / 128 + d / 256); }
-
-cudaError_t launch_fused_fwd(const FusedFwdParams& p, int64_t grid, cudaStream_t st) {
+template <int K1, int K2>
+static cudaError_t launch_pair(const GemmPairParams& p, int64_t grid, cudaStream_t st) {
   static bool configured[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(k_moe_fwd_gemms, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const cudaError_t e = cudaFuncSetAttribute(k_moe_gemm_pair<K1, K2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(fused_smem_bytes()));
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   if (grid < 1 || grid > 0x7fffffff) return cudaErrorInvalidValue;
-  k_moe_fwd_gemms<<<static_cast<unsigned>(grid), GEMM_THREADS_SCHED, fused_smem_bytes(), st>>>(p);
+  k_moe_gemm_pair<K1, K2><<<static_cast<unsigned>(grid), GEMM_THREADS_SCHED, fused_smem_bytes(), st>>>(p);
   return cudaGetLastError();
+}
+
+int64_t gemm_pair_units(GemmPair pair, int64_t RP, int d, int I) {
+  const int64_t mt = RP / 128;
+  return pair == PAIR_FWD ? mt * (I / 128 + d / 256) : mt * (I / 256 + d / 256);
+}
+
+cudaError_t launch_gemm_pair(GemmPair pair, const GemmPairParams& p, int64_t grid, cudaStream_t st) {
+  switch (pair) {
+    case PAIR_FWD: return launch_pair<G_GATEUP, G_DOWN>(p, grid, st);
+    case PAIR_DGRAD: return launch_pair<G_DGRAD_DOWN, G_DGRAD_GATEUP>(p, grid, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace moe

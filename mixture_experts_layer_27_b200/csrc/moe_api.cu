@@ -104,7 +104,7 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->daqs = take(mxi / 32);
   L->dbq = take(mxi);
   L->dbqs = take(mxi / 32);
-  L->fctl = take(M > 0 || L->mx ? 0 : static_cast<size_t>(fused_ctl_words(L->RP)) * 4);
+  L->fctl = take(M > 0 || L->mx ? 0 : static_cast<size_t>(gemm_pair_ctl_words(L->RP)) * 4);
   L->ws_bytes = o;
   // prepared weights: [W_gate|W_up paired, K = d] [W_down^T, K = I] [W_down, K = d] [W_gate, K = I] [W_up, K = I]
   o = 0;
@@ -286,7 +286,7 @@ enum KernelId {
   K_ROUTER_LOGITS, K_TOPK, K_SCAN, K_SCATTER, K_DISPATCH, K_GEMM_GATEUP, K_GEMM_DOWN, K_COMBINE,
   K_REV_COMBINE, K_GEMM_DGRAD_DOWN, K_ROUTER_BWD, K_ROUTER_WGRAD, K_TRANSPOSE_WR, K_GEMM_DGRAD_GATEUP, K_REV_DISPATCH,
   K_GEMM_WGRAD_GATEUP, K_GEMM_WGRAD_DOWN, K_PLAN, K_REPLAY, K_FINISH_ACC, K_QUANT_WEIGHTS, K_MARK_ROWS,
-  K_ACTIVE_COUNT, K_GATHER_ACTIVE, K_SCAN_GROUPS, K_SCAN_APPLY, K_FUSED_FWD, K_NUM
+  K_ACTIVE_COUNT, K_GATHER_ACTIVE, K_SCAN_GROUPS, K_SCAN_APPLY, K_PAIR_FWD, K_PAIR_DGRAD, K_NUM
 };
 static const char* kKernelNames[K_NUM] = {
     "router_logits", "topk_gating", "hist_scan", "stable_scatter", "dispatch", "gemm_gateup_swiglu",
@@ -294,7 +294,7 @@ static const char* kKernelNames[K_NUM] = {
     "transpose_wr", "gemm_dgrad_gateup", "reverse_dispatch", "gemm_wgrad_gateup", "gemm_wgrad_down",
     "stream_plan", "ring_replay", "wgrad_accumulator_finish", "quantize_weights", "mark_pad_rows",
     "router_token_count", "router_token_gather", "hist_scan_group_sums", "hist_scan_group_apply",
-    "gemm_gateup_down_persistent"};
+    "gemm_gateup_down_persistent", "gemm_dgrads_persistent"};
 
 struct ProfRec {
   int kid;
@@ -554,8 +554,24 @@ moe_status moe_fwd(const moe_shape* s, const void* X, const void* W_r, const flo
   return MOE_OK;
 }
 
+// Two dependent grouped GEMMs as one persistent launch (a CTA per SM, a second wave claimed
+// through Cluster Launch Control by the CTAs that run first).
+static cudaError_t run_gemm_pair(const Layout& L, const Ctx& c, GemmPair pair, const GemmParams& p1,
+                                 const GemmParams& p2, cudaStream_t st) {
+  GemmPairParams f;
+  f.p1 = p1;
+  f.p2 = p2;
+  f.ctl = c.fctl;
+  f.mt_cap = static_cast<int>(L.RP / 128);
+  cudaError_t e = cudaMemsetAsync(c.fctl, 0, static_cast<size_t>(gemm_pair_ctl_words(L.RP)) * 4, st);
+  if (e != cudaSuccess) return e;
+  const int64_t units = gemm_pair_units(pair, L.RP, L.d, L.I);
+  const int64_t grid = units < 2LL * num_sms() ? units : 2LL * num_sms();
+  return launch_gemm_pair(pair, f, grid, st);
+}
+
 // The forward with its two grouped GEMMs in one persistent launch: the same routing, dispatch
-// and combine launches as moe_fwd around k_moe_fwd_gemms.
+// and combine launches as moe_fwd around it.
 moe_status moe_fwd_persistent(const moe_shape* s, const void* X, const void* W_r, const float* bias,
                               const void* W_gate, const void* W_up, const void* W_down, void* Y, void* ctx,
                               size_t ctx_bytes, void* ws, size_t ws_bytes, void* stream) {
@@ -582,29 +598,21 @@ moe_status moe_fwd_persistent(const moe_shape* s, const void* X, const void* W_r
   MOE_TRY(timed(K_DISPATCH, st, [&] {
     return launch_gather_rows(L, c, static_cast<const __nv_bfloat16*>(X), c.xperm, st);
   }));
-  FusedFwdParams f;
-  f.gu = base_params(L, c, status);
-  MOE_TMAP(tmap_2d(&f.gu.ta0, c.xperm, L.d, RP, L.d, 64, 128));
-  MOE_TMAP(tmap_2d(&f.gu.tb0, W_gate, L.I, static_cast<uint64_t>(L.El) * L.d, L.I, 64, 64));
-  MOE_TMAP(tmap_2d(&f.gu.tb1, W_up, L.I, static_cast<uint64_t>(L.El) * L.d, L.I, 64, 64));
-  f.gu.ta1 = f.gu.ta0;
-  f.gu.out0 = c.abuf;
-  f.gu.out1 = c.bbuf;
-  f.gu.out2 = c.hbuf;
-  f.dn = base_params(L, c, status);
-  MOE_TMAP(tmap_2d(&f.dn.ta0, c.hbuf, L.I, RP, L.I, 64, 128));
-  MOE_TMAP(tmap_2d(&f.dn.tb0, W_down, L.d, static_cast<uint64_t>(L.El) * L.I, L.d, 64, 64));
-  f.dn.ta1 = f.dn.ta0;
-  f.dn.tb1 = f.dn.tb0;
-  f.dn.out0 = c.obuf;
-  f.ctl = c.fctl;
-  f.mt_cap = static_cast<int>(L.RP / 128);
-  MOE_TRY(cudaMemsetAsync(c.fctl, 0, static_cast<size_t>(fused_ctl_words(L.RP)) * 4, st));
-  // two CTAs per SM at most: the first wave runs, the rest is taken over through Cluster Launch
-  // Control by whichever CTAs claim work first (fewer when there are fewer tiles)
-  const int64_t units = fused_fwd_units(L.RP, L.d, L.I);
-  const int64_t grid = units < 2LL * num_sms() ? units : 2LL * num_sms();
-  MOE_TRY(timed(K_FUSED_FWD, st, [&] { return launch_fused_fwd(f, grid, st); }));
+  GemmParams gu = base_params(L, c, status);
+  MOE_TMAP(tmap_2d(&gu.ta0, c.xperm, L.d, RP, L.d, 64, 128));
+  MOE_TMAP(tmap_2d(&gu.tb0, W_gate, L.I, static_cast<uint64_t>(L.El) * L.d, L.I, 64, 64));
+  MOE_TMAP(tmap_2d(&gu.tb1, W_up, L.I, static_cast<uint64_t>(L.El) * L.d, L.I, 64, 64));
+  gu.ta1 = gu.ta0;
+  gu.out0 = c.abuf;
+  gu.out1 = c.bbuf;
+  gu.out2 = c.hbuf;
+  GemmParams dn = base_params(L, c, status);
+  MOE_TMAP(tmap_2d(&dn.ta0, c.hbuf, L.I, RP, L.I, 64, 128));
+  MOE_TMAP(tmap_2d(&dn.tb0, W_down, L.d, static_cast<uint64_t>(L.El) * L.I, L.d, 64, 64));
+  dn.ta1 = dn.ta0;
+  dn.tb1 = dn.tb0;
+  dn.out0 = c.obuf;
+  MOE_TRY(timed(K_PAIR_FWD, st, [&] { return run_gemm_pair(L, c, PAIR_FWD, gu, dn, st); }));
   MOE_TRY(timed(K_COMBINE, st, [&] { return launch_combine(L, c, c.obuf, static_cast<__nv_bfloat16*>(Y), st); }));
   return MOE_OK;
 }
@@ -667,9 +675,11 @@ static moe_status zero_wgrads(const Layout& L, void* dW_gate, void* dW_up, void*
   return MOE_OK;
 }
 
-moe_status moe_bwd(const moe_shape* s, const void* X, const void* W_r, const void* W_gate, const void* W_up,
-                   const void* W_down, const void* dY, void* ctx, size_t ctx_bytes, void* dX, void* dW_gate,
-                   void* dW_up, void* dW_down, float* dW_r, void* ws, size_t ws_bytes, void* stream) {
+// persistent: both dgrads as one persistent launch (the router backward then runs after them).
+static moe_status bwd_impl(const moe_shape* s, const void* X, const void* W_r, const void* W_gate, const void* W_up,
+                           const void* W_down, const void* dY, void* ctx, size_t ctx_bytes, void* dX, void* dW_gate,
+                           void* dW_up, void* dW_down, float* dW_r, void* ws, size_t ws_bytes, void* stream,
+                           bool persistent) {
   Layout L;
   const moe_status cs = check_shape(s, &L);
   if (cs != MOE_OK) return cs;
@@ -693,37 +703,59 @@ moe_status moe_bwd(const moe_shape* s, const void* X, const void* W_r, const voi
   // 8. reverse-combine: dY into the expert-contiguous layout
   MOE_TRY(timed(K_REV_COMBINE, st, [&] { return launch_gather_rows(L, c, static_cast<const __nv_bfloat16*>(dY), c.dyperm, st); }));
   // 9. dgrad of the down projection + SwiGLU backward + router-gate gradient partials
-  {
-    GemmParams p = base_params(L, c, status);
-    MOE_TMAP(tmap_2d(&p.ta0, c.dyperm, L.d, RP, L.d, 64, 128));
-    MOE_TMAP(tmap_2d(&p.tb0, W_down, L.d, El * L.I, L.d, 64, 256));
-    p.ta1 = p.ta0;
-    p.tb1 = p.tb0;
-    p.in0 = c.abuf;
-    p.in1 = c.bbuf;
-    p.out0 = c.dabuf;
-    p.out1 = c.dbbuf;
-    p.out2 = c.hgbuf;
-    p.outf = c.dgpart;
-    MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm(G_DGRAD_DOWN, p, grid, st); }));
-  }
-  // 10. router backward: dl, then dW_r = X^T DL (tensor cores); W_r^T for the dX router term
-  MOE_TRY_STATUS(router_backward(L, c, X, dW_r, status, st));
-  MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] { return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st); }));
+  GemmParams p9 = base_params(L, c, status);
+  MOE_TMAP(tmap_2d(&p9.ta0, c.dyperm, L.d, RP, L.d, 64, 128));
+  MOE_TMAP(tmap_2d(&p9.tb0, W_down, L.d, El * L.I, L.d, 64, 256));
+  p9.ta1 = p9.ta0;
+  p9.tb1 = p9.tb0;
+  p9.in0 = c.abuf;
+  p9.in1 = c.bbuf;
+  p9.out0 = c.dabuf;
+  p9.out1 = c.dbbuf;
+  p9.out2 = c.hgbuf;
+  p9.outf = c.dgpart;
   // 11. dgrad of gate/up
-  {
-    GemmParams p = base_params(L, c, status);
-    MOE_TMAP(tmap_2d(&p.ta0, c.dabuf, L.I, RP, L.I, 64, 128));
-    MOE_TMAP(tmap_2d(&p.ta1, c.dbbuf, L.I, RP, L.I, 64, 128));
-    MOE_TMAP(tmap_2d(&p.tb0, W_gate, L.I, El * L.d, L.I, 64, 256));
-    MOE_TMAP(tmap_2d(&p.tb1, W_up, L.I, El * L.d, L.I, 64, 256));
-    p.out0 = c.dxperm;
-    MOE_TRY(timed(K_GEMM_DGRAD_GATEUP, st, [&] { return launch_gemm(G_DGRAD_GATEUP, p, grid, st); }));
+  GemmParams p11 = base_params(L, c, status);
+  MOE_TMAP(tmap_2d(&p11.ta0, c.dabuf, L.I, RP, L.I, 64, 128));
+  MOE_TMAP(tmap_2d(&p11.ta1, c.dbbuf, L.I, RP, L.I, 64, 128));
+  MOE_TMAP(tmap_2d(&p11.tb0, W_gate, L.I, El * L.d, L.I, 64, 256));
+  MOE_TMAP(tmap_2d(&p11.tb1, W_up, L.I, El * L.d, L.I, 64, 256));
+  p11.out0 = c.dxperm;
+  if (persistent) {
+    MOE_TRY(timed(K_PAIR_DGRAD, st, [&] { return run_gemm_pair(L, c, PAIR_DGRAD, p9, p11, st); }));
+    // 10. router backward: dl, then dW_r = X^T DL (tensor cores); W_r^T for the dX router term
+    MOE_TRY_STATUS(router_backward(L, c, X, dW_r, status, st));
+    MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
+      return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
+    }));
+  } else {
+    MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm(G_DGRAD_DOWN, p9, grid, st); }));
+    // 10. router backward: dl, then dW_r = X^T DL (tensor cores); W_r^T for the dX router term
+    MOE_TRY_STATUS(router_backward(L, c, X, dW_r, status, st));
+    MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
+      return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
+    }));
+    MOE_TRY(timed(K_GEMM_DGRAD_GATEUP, st, [&] { return launch_gemm(G_DGRAD_GATEUP, p11, grid, st); }));
   }
   // 12. reverse-dispatch (+ router term dl W_r^T)
   MOE_TRY(timed(K_REV_DISPATCH, st, [&] { return launch_rev_dispatch(L, c, static_cast<__nv_bfloat16*>(dX), st); }));
   // 13. wgrad
   return launch_wgrads(L, c, status, dW_gate, dW_up, dW_down, st);
+}
+
+moe_status moe_bwd(const moe_shape* s, const void* X, const void* W_r, const void* W_gate, const void* W_up,
+                   const void* W_down, const void* dY, void* ctx, size_t ctx_bytes, void* dX, void* dW_gate,
+                   void* dW_up, void* dW_down, float* dW_r, void* ws, size_t ws_bytes, void* stream) {
+  return bwd_impl(s, X, W_r, W_gate, W_up, W_down, dY, ctx, ctx_bytes, dX, dW_gate, dW_up, dW_down, dW_r, ws,
+                  ws_bytes, stream, false);
+}
+
+moe_status moe_bwd_persistent(const moe_shape* s, const void* X, const void* W_r, const void* W_gate,
+                              const void* W_up, const void* W_down, const void* dY, void* ctx, size_t ctx_bytes,
+                              void* dX, void* dW_gate, void* dW_up, void* dW_down, float* dW_r, void* ws,
+                              size_t ws_bytes, void* stream) {
+  return bwd_impl(s, X, W_r, W_gate, W_up, W_down, dY, ctx, ctx_bytes, dX, dW_gate, dW_up, dW_down, dW_r, ws,
+                  ws_bytes, stream, true);
 }
 
 moe_status moe_profile_enable(int on) {

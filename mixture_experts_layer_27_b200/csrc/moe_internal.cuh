@@ -153,20 +153,24 @@ cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, int grid, cudaStream
 // so that a later launch needs no lazy module loading.
 cudaError_t preload_gemm(GemmKind kind);
 
-// The forward's gate/up and down GEMMs in one persistent launch (gemm.cu): every gate/up
-// tile, then every down tile, as work units that CTAs take from one ticket counter in one
-// global order, CTAs that have not started claimed through Cluster Launch Control.  A down
-// tile waits (bounded) until every gate/up tile of its 128 rows has stored its H rows.
-struct FusedFwdParams {
-  GemmParams gu;  // the gate/up GEMM's parameters (ta0 = X_perm; A, B, H outputs)
-  GemmParams dn;  // the down GEMM's parameters (ta0 = H; O' output)
-  int* ctl;       // fused_ctl_words(RP) ints, zero before the launch
+// Two dependent grouped GEMMs in one persistent launch (gemm.cu): every tile of the first,
+// then every tile of the second, as work units that CTAs take from one ticket counter in one
+// global order, CTAs that have not started claimed through Cluster Launch Control.  A tile of
+// the second GEMM waits (bounded) until every tile of the first has stored its 128 rows.
+enum GemmPair {
+  PAIR_FWD = 0,    // G_GATEUP then G_DOWN (reads H)
+  PAIR_DGRAD = 1,  // G_DGRAD_DOWN then G_DGRAD_GATEUP (reads dA, dB)
+};
+struct GemmPairParams {
+  GemmParams p1;  // the first GEMM's parameters, as for launch_gemm
+  GemmParams p2;  // the second GEMM's parameters
+  int* ctl;       // gemm_pair_ctl_words(RP) ints, zero before the launch
   int mt_cap;     // m-tile capacity of ctl (RP / 128)
 };
-constexpr int64_t fused_ctl_words(int64_t RP) { return 1 + RP / 128; }
-// Upper bound of the work units (gate/up and down tiles at RP rows).
-int64_t fused_fwd_units(int64_t RP, int d, int I);
-cudaError_t launch_fused_fwd(const FusedFwdParams& p, int64_t grid, cudaStream_t st);
+constexpr int64_t gemm_pair_ctl_words(int64_t RP) { return 1 + RP / 128; }
+// Upper bound of the work units (both GEMMs' tiles at RP rows).
+int64_t gemm_pair_units(GemmPair pair, int64_t RP, int d, int I);
+cudaError_t launch_gemm_pair(GemmPair pair, const GemmPairParams& p, int64_t grid, cudaStream_t st);
 
 // 2-D bf16 tensor map [outer, inner] (inner contiguous, row pitch in elements), box
 // {box_inner, box_outer}, 128-byte swizzle, zero fill out of bounds (moe_api.cu).
@@ -252,7 +256,7 @@ struct Ctx {  // typed views of ctx + ws for one shape
   int* actcnt;               // expert slice: token counts per 256-token block, then the list length
   int* actlist;              // expert slice: the tokens with a local assignment, ascending
   __nv_bfloat16* xact;       // expert slice: their X rows [Tpad, d] (rows past the list up to a multiple of 64: 0)
-  int* fctl;                 // control block of the one-launch forward expert phase (fused_ctl_words(RP) ints)
+  int* fctl;                 // control block of a persistent GEMM pair (gemm_pair_ctl_words(RP) ints)
   StreamTables tab;
   uint8_t *xq, *xqs, *hq, *hqs, *dyq, *dyqs, *daq, *daqs, *dbq, *dbqs;  // MXFP8 operands and scales
 };

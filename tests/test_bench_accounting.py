@@ -40,6 +40,7 @@ def test_router_weight_gradient_flops():
     assert f["gemm_gateup_swiglu"] + f["gemm_down_combw"] == 6 * dI * rows
     # the persistent kernel runs gate/up and down in one launch: an alternative, not an extra GEMM
     assert f["gemm_gateup_down_persistent"] == f["gemm_gateup_swiglu"] + f["gemm_down_combw"]
+    assert f["gemm_dgrads_persistent"] == f["gemm_dgrad_down_swiglu_bwd"] + f["gemm_dgrad_gateup"]
     assert sum(v for k, v in f.items() if k.startswith("gemm_") and "persistent" not in k) == 18 * dI * rows
 
 

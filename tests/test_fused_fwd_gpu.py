@@ -1,12 +1,13 @@
-"""The forward's two grouped GEMMs in one persistent launch (`moe_fwd_persistent`).
+"""Pairs of grouped GEMMs in one persistent launch (`moe_fwd_persistent`, `moe_bwd_persistent`).
 
-The gate/up GEMM with SwiGLU and the down GEMM with the gate multiply run as work units of one
-kernel, taken by CTAs in one global order and claimed through Cluster Launch Control; a down tile
-waits for the gate/up tiles of its rows.  Each unit computes what the separate launches of
-`moe_fwd` compute, with the same tiles and epilogues, so Y and everything saved in ctx must be the
-same bits, and a
-`moe_bwd` after it must give the same gradients bit for bit.  Y and the gradients must also match
-the fp64 oracle within the bf16 tolerance, and repeated runs must be bit-identical.
+The forward's gate/up GEMM (SwiGLU epilogue) and down GEMM (gate multiply), and the backward's
+dgrad of W_down (SwiGLU backward, router-gate gradient) and dgrad of gate/up, each run as work
+units of one kernel, taken by CTAs in one global order and claimed through Cluster Launch Control;
+a tile of the second GEMM waits for the first GEMM's tiles of its rows.  Each unit computes what
+the separate launches compute, with the same tiles and epilogues, so Y, everything saved in ctx
+and every gradient must be the same bits as `moe_fwd` + `moe_bwd`, in either combination.  Y and
+the gradients must also match the fp64 oracle within the bf16 tolerance, and repeated runs must
+be bit-identical.
 """
 import numpy as np
 import pytest
@@ -19,13 +20,14 @@ from _util import TOL_BF16, make_case, relerr, run_oracle, to64
 pytestmark = pytest.mark.gpu
 
 
-def _step(layer, x, first, El, persistent, poison=False):
+def _step(layer, x, first, El, persistent, poison=False, bwd_persistent=None):
     if poison:  # every byte the step may read before writing it holds a NaN pattern
         layer.ctx.fill_(0xFF)
         layer.ws.fill_(0xFF)
     W = [x[n][first:first + El].contiguous() for n in ("W_gate", "W_up", "W_down")]
     Y = layer.forward(x["X"], x["W_r"], x["bias"], *W, persistent=persistent)
-    g = layer.backward(x["X"], x["W_r"], *W, x["dY"])
+    g = layer.backward(x["X"], x["W_r"], *W, x["dY"],
+                       persistent=persistent if bwd_persistent is None else bwd_persistent)
     torch.cuda.synchronize()
     assert layer.error() == B.MOE_OK
     return Y, g
@@ -51,7 +53,14 @@ def _check(T, d, E, k, I, seed, bias=None, first=0, num=0, oracle=True):
     # run to run: a second persistent step over the same buffers
     Y2, g2 = _step(fus, x, first, El, persistent=True)
     assert torch.equal(_bits(Y2), _bits(Y1))
-    assert torch.equal(_bits(g2["dW_gate"]), _bits(g1["dW_gate"]))
+    for n in g1:
+        assert torch.equal(_bits(g2[n]), _bits(g1[n])), n
+    # the mixed combinations: each persistent half pairs with the other's multi-launch half
+    for fp, bp in ((True, False), (False, True)):
+        Y3, g3 = _step(fus, x, first, El, persistent=fp, bwd_persistent=bp)
+        assert torch.equal(_bits(Y3), _bits(Y0))
+        for n in g0:
+            assert torch.equal(_bits(g3[n]), _bits(g0[n])), (fp, bp, n)
     if oracle:
         Yo, _, go = run_oracle(x, k, first=first, num=num or None)
         assert relerr(to64(Y1), Yo) <= TOL_BF16
