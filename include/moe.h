@@ -185,6 +185,16 @@ moe_status moe_debug_router_grad(const moe_shape* shape, const void* ws, float* 
  * if the launch fails. */
 moe_status moe_debug_bounded_wait(const moe_shape* shape, void* ctx, size_t ctx_bytes, void* stream);
 
+/* Test hook for the persistent GEMM pairs' cross-CTA waits (no counterpart on the pages): runs
+ * moe_fwd_persistent with the gate/up tiles left out of the persistent launch, so every down
+ * tile waits for H rows that nobody writes.  The first wait to reach its limit (about 2 s)
+ * records MOE_ERR_DEVICE_TIMEOUT in ctx's status word; every other wait, and every CTA that
+ * starts later, sees the status and stops, and the kernel ends.  Y is not valid afterwards;
+ * the context stays usable.  Same arguments and argument errors as moe_fwd_persistent. */
+moe_status moe_debug_pair_wait(const moe_shape* shape, const void* X, const void* W_r, const float* bias,
+                               const void* W_gate, const void* W_up, const void* W_down, void* Y, void* ctx,
+                               size_t ctx_bytes, void* ws, size_t ws_bytes, void* stream);
+
 /* Benchmark support (no counterpart on the pages).  When enabled, every
  * kernel launch of the library is bracketed by two CUDA events recorded on the
  * launch stream.  moe_profile_read synchronises the device, writes per kernel

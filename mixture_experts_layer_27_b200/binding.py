@@ -82,6 +82,8 @@ _SIGS = {
     "moe_debug_logits": (ctypes.c_int, [_S, _P, _P, _P]),
     "moe_debug_router_grad": (ctypes.c_int, [_S, _P, _P, _P]),
     "moe_debug_bounded_wait": (ctypes.c_int, [_S, _P, ctypes.c_size_t, _P]),
+    "moe_debug_pair_wait": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, ctypes.c_size_t,
+                                           _P]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
     "moe_profile_read": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
@@ -205,6 +207,12 @@ def moe_debug_routing(shape, ctx, ids=None, gates=None, counts=None, offsets=Non
 
 def moe_debug_logits(shape, ws, logits, stream=None) -> int:
     return int(lib().moe_debug_logits(ctypes.byref(shape), _ptr(ws), _ptr(logits), _stream(stream)))
+
+
+def moe_debug_pair_wait(shape, X, W_r, bias, W_gate, W_up, W_down, Y, ctx, ws, stream=None) -> int:
+    return int(lib().moe_debug_pair_wait(ctypes.byref(shape), _ptr(X), _ptr(W_r), _ptr(bias), _ptr(W_gate),
+                                         _ptr(W_up), _ptr(W_down), _ptr(Y), _ptr(ctx), _nbytes(ctx), _ptr(ws),
+                                         _nbytes(ws), _stream(stream)))
 
 
 def moe_debug_bounded_wait(shape, ctx, stream=None) -> int:

@@ -1011,7 +1011,8 @@ __global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_gemm_pair(const _
       const int total = cnt.total();
       uint32_t clc_phase = 0;
       bool may_cancel = true;  // false after an answer that cancelled nothing
-      int ticket = status_set(status) ? total : atomicAdd(P.ctl, 1);
+      const int skip = P.skip_first ? cnt.n1 : 0;
+      int ticket = status_set(status) ? total : skip + atomicAdd(P.ctl, 1);
       for (int j = 0;; ++j) {
         const int slot = j % SCHED_DEPTH;
         // claim the next unit while this one is queued: cancel a CTA that has not started
@@ -1045,7 +1046,7 @@ __global__ void __launch_bounds__(GEMM_THREADS_SCHED, 1) k_moe_gemm_pair(const _
           if (!clc_cancelled(clc_resp)) may_cancel = false;  // no CTA left to take over
         }
         if (last) break;
-        ticket = atomicAdd(P.ctl, 1);
+        ticket = skip + atomicAdd(P.ctl, 1);
       }
       // Out of units: cancel the CTAs that have not started yet, so that they never launch
       // only to find no work.  This overlaps with the last units of this CTA's roles.

@@ -557,12 +557,13 @@ moe_status moe_fwd(const moe_shape* s, const void* X, const void* W_r, const flo
 // Two dependent grouped GEMMs as one persistent launch (a CTA per SM, a second wave claimed
 // through Cluster Launch Control by the CTAs that run first).
 static cudaError_t run_gemm_pair(const Layout& L, const Ctx& c, GemmPair pair, const GemmParams& p1,
-                                 const GemmParams& p2, cudaStream_t st) {
+                                 const GemmParams& p2, cudaStream_t st, bool skip_first = false) {
   GemmPairParams f;
   f.p1 = p1;
   f.p2 = p2;
   f.ctl = c.fctl;
   f.mt_cap = static_cast<int>(L.RP / 128);
+  f.skip_first = skip_first ? 1 : 0;
   cudaError_t e = cudaMemsetAsync(c.fctl, 0, static_cast<size_t>(gemm_pair_ctl_words(L.RP)) * 4, st);
   if (e != cudaSuccess) return e;
   const int64_t units = gemm_pair_units(pair, L.RP, L.d, L.I);
@@ -571,10 +572,10 @@ static cudaError_t run_gemm_pair(const Layout& L, const Ctx& c, GemmPair pair, c
 }
 
 // The forward with its two grouped GEMMs in one persistent launch: the same routing, dispatch
-// and combine launches as moe_fwd around it.
-moe_status moe_fwd_persistent(const moe_shape* s, const void* X, const void* W_r, const float* bias,
-                              const void* W_gate, const void* W_up, const void* W_down, void* Y, void* ctx,
-                              size_t ctx_bytes, void* ws, size_t ws_bytes, void* stream) {
+// and combine launches as moe_fwd around it.  skip_first: the test hook of GemmPairParams.
+static moe_status fwd_persistent_impl(const moe_shape* s, const void* X, const void* W_r, const float* bias,
+                                      const void* W_gate, const void* W_up, const void* W_down, void* Y, void* ctx,
+                                      size_t ctx_bytes, void* ws, size_t ws_bytes, void* stream, bool skip_first) {
   Layout L;
   const moe_status cs = check_shape(s, &L);
   if (cs != MOE_OK) return cs;
@@ -612,9 +613,21 @@ moe_status moe_fwd_persistent(const moe_shape* s, const void* X, const void* W_r
   dn.ta1 = dn.ta0;
   dn.tb1 = dn.tb0;
   dn.out0 = c.obuf;
-  MOE_TRY(timed(K_PAIR_FWD, st, [&] { return run_gemm_pair(L, c, PAIR_FWD, gu, dn, st); }));
+  MOE_TRY(timed(K_PAIR_FWD, st, [&] { return run_gemm_pair(L, c, PAIR_FWD, gu, dn, st, skip_first); }));
   MOE_TRY(timed(K_COMBINE, st, [&] { return launch_combine(L, c, c.obuf, static_cast<__nv_bfloat16*>(Y), st); }));
   return MOE_OK;
+}
+
+moe_status moe_fwd_persistent(const moe_shape* s, const void* X, const void* W_r, const float* bias,
+                              const void* W_gate, const void* W_up, const void* W_down, void* Y, void* ctx,
+                              size_t ctx_bytes, void* ws, size_t ws_bytes, void* stream) {
+  return fwd_persistent_impl(s, X, W_r, bias, W_gate, W_up, W_down, Y, ctx, ctx_bytes, ws, ws_bytes, stream, false);
+}
+
+moe_status moe_debug_pair_wait(const moe_shape* s, const void* X, const void* W_r, const float* bias,
+                               const void* W_gate, const void* W_up, const void* W_down, void* Y, void* ctx,
+                               size_t ctx_bytes, void* ws, size_t ws_bytes, void* stream) {
+  return fwd_persistent_impl(s, X, W_r, bias, W_gate, W_up, W_down, Y, ctx, ctx_bytes, ws, ws_bytes, stream, true);
 }
 
 // 10. router backward: dl (and, in an expert slice, the list of tokens with a local

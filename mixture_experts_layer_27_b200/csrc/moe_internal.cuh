@@ -166,6 +166,8 @@ struct GemmPairParams {
   GemmParams p2;  // the second GEMM's parameters
   int* ctl;       // gemm_pair_ctl_words(RP) ints, zero before the launch
   int mt_cap;     // m-tile capacity of ctl (RP / 128)
+  int skip_first; // test hook: the first GEMM's tiles are not run, so the second GEMM's tiles wait
+                  // for rows that nobody writes until their bounded wait gives up
 };
 constexpr int64_t gemm_pair_ctl_words(int64_t RP) { return 1 + RP / 128; }
 // Upper bound of the work units (both GEMMs' tiles at RP rows).

@@ -99,3 +99,25 @@ def test_persistent_forward_full_size_deepseek_v3_like_equals_moe_fwd():
 def test_persistent_forward_ep64_slice_equals_moe_fwd():
     # 6 of 384 experts, 32,768 tokens (the per-rank slice as one batch)
     _check(32768, 7168, 384, 8, 2048, seed=86, first=0, num=6, oracle=False)
+
+
+def test_persistent_pair_wait_for_rows_nobody_writes_times_out_and_recovers():
+    # The debug hook leaves the gate/up tiles out of the persistent launch: every down tile waits
+    # for H rows that are never counted.  The first bounded wait to run out (about 2 s) records
+    # MOE_ERR_DEVICE_TIMEOUT, every other CTA stops, and the next step on the same buffers is
+    # again bit-identical to moe_fwd + moe_bwd.
+    T, d, E, k, I = 300, 256, 8, 2, 256
+    w, x = make_case(T, d, E, k, I, seed=87)
+    ref = B.MoELayer(T, d, E, I, k)
+    Y0, g0 = _step(ref, x, 0, E, persistent=False)
+    lay = B.MoELayer(T, d, E, I, k)
+    Y = torch.empty_like(Y0)
+    W = [x[n].contiguous() for n in ("W_gate", "W_up", "W_down")]
+    assert B.moe_debug_pair_wait(lay.shape, x["X"], x["W_r"], x["bias"], *W, Y, lay.ctx, lay.ws) == B.MOE_OK
+    torch.cuda.synchronize()
+    assert lay.error() == B.MOE_ERR_DEVICE_TIMEOUT
+    assert lay.error() == B.MOE_OK  # read and cleared
+    Y1, g1 = _step(lay, x, 0, E, persistent=True)
+    assert torch.equal(_bits(Y1), _bits(Y0))
+    for n in g0:
+        assert torch.equal(_bits(g1[n]), _bits(g0[n])), n
