@@ -104,7 +104,7 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->daqs = take(mxi / 32);
   L->dbq = take(mxi);
   L->dbqs = take(mxi / 32);
-  L->fctl = take(M > 0 || L->mx ? 0 : static_cast<size_t>(gemm_pair_ctl_words(L->RP)) * 4);
+  L->fctl = take(L->mx ? 0 : static_cast<size_t>(gemm_pair_ctl_words(L->RP)) * 4);
   L->ws_bytes = o;
   // prepared weights: [W_gate|W_up paired, K = d] [W_down^T, K = I] [W_down, K = d] [W_gate, K = I] [W_up, K = I]
   o = 0;
@@ -190,7 +190,7 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
     c.wrt = reinterpret_cast<__nv_bfloat16*>(W(L.wrt));
     c.dxperm = reinterpret_cast<__nv_bfloat16*>(W(L.dxperm));
     c.acc32 = L.M > 0 ? reinterpret_cast<float*>(W(L.acc32)) : nullptr;
-    c.fctl = L.M == 0 && !L.mx ? reinterpret_cast<int*>(W(L.fctl)) : nullptr;
+    c.fctl = !L.mx ? reinterpret_cast<int*>(W(L.fctl)) : nullptr;
     if (L.rslice) {
       c.actcnt = reinterpret_cast<int*>(W(L.actcnt));
       c.actlist = reinterpret_cast<int*>(W(L.actlist));
@@ -888,14 +888,15 @@ moe_status moe_fwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
     p.out0 = c.abuf;
     p.out1 = c.bbuf;
     p.out2 = c.hbuf;
-    MOE_TRY(timed(K_GEMM_GATEUP, st, [&] { return launch_gemm(G_GATEUP, p, grid, st); }));
     GemmParams q = base_params(L, c, status);
     q.poff = seg;
     q.nseg = El;
     q.ta0 = q.ta1 = h_map;
     q.tb0 = q.tb1 = wd_map;
     q.out0 = c.obuf;
-    MOE_TRY(timed(K_GEMM_DOWN, st, [&] { return launch_gemm(G_DOWN, q, grid, st); }));
+    // gate/up then down as one persistent launch (the down tiles start while the macrobatch's
+    // last gate/up tiles run; measured 2-3% faster per step than two launches at n = 512-2368)
+    MOE_TRY(timed(K_PAIR_FWD, st, [&] { return run_gemm_pair(L, c, PAIR_FWD, p, q, st); }));
     MOE_TRY(timed(K_COMBINE, st, [&] {
       return launch_combine(L, c, c.obuf, static_cast<__nv_bfloat16*>(Y), st, c.tab.mb_range + 2 * m);
     }));
@@ -933,39 +934,36 @@ moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
   MOE_TRY(timed(K_REV_COMBINE, st, [&] {
     return launch_gather_rows(L, c, static_cast<const __nv_bfloat16*>(dY), c.dyperm, st);
   }));
-  {
-    GemmParams p = base_params(L, c, status);
-    p.poff = c.tab.seg_poff;
-    p.cum = c.tab.cum;
-    p.nseg = nseg;
-    MOE_TMAP(tmap_2d(&p.ta0, c.dyperm, L.d, RP, L.d, 64, 128));
-    MOE_TMAP(tmap_2d(&p.tb0, W_down, L.d, El * L.I, L.d, 64, 256));
-    p.ta1 = p.ta0;
-    p.tb1 = p.tb0;
-    p.in0 = c.abuf;
-    p.in1 = c.bbuf;
-    p.out0 = c.dabuf;
-    p.out1 = c.dbbuf;
-    p.out2 = c.hgbuf;
-    p.outf = c.dgpart;
-    MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm(G_DGRAD_DOWN, p, grid, st); }));
-  }
+  // dgrad of W_down (SwiGLU backward, router-gate partials) then dgrad of gate/up, as one
+  // persistent launch over every row of the stream; the router backward follows it
+  GemmParams p9 = base_params(L, c, status);
+  p9.poff = c.tab.seg_poff;
+  p9.cum = c.tab.cum;
+  p9.nseg = nseg;
+  MOE_TMAP(tmap_2d(&p9.ta0, c.dyperm, L.d, RP, L.d, 64, 128));
+  MOE_TMAP(tmap_2d(&p9.tb0, W_down, L.d, El * L.I, L.d, 64, 256));
+  p9.ta1 = p9.ta0;
+  p9.tb1 = p9.tb0;
+  p9.in0 = c.abuf;
+  p9.in1 = c.bbuf;
+  p9.out0 = c.dabuf;
+  p9.out1 = c.dbbuf;
+  p9.out2 = c.hgbuf;
+  p9.outf = c.dgpart;
+  GemmParams p11 = base_params(L, c, status);
+  p11.poff = c.tab.seg_poff;
+  p11.cum = c.tab.cum;
+  p11.nseg = nseg;
+  MOE_TMAP(tmap_2d(&p11.ta0, c.dabuf, L.I, RP, L.I, 64, 128));
+  MOE_TMAP(tmap_2d(&p11.ta1, c.dbbuf, L.I, RP, L.I, 64, 128));
+  MOE_TMAP(tmap_2d(&p11.tb0, W_gate, L.I, El * L.d, L.I, 64, 256));
+  MOE_TMAP(tmap_2d(&p11.tb1, W_up, L.I, El * L.d, L.I, 64, 256));
+  p11.out0 = c.dxperm;
+  MOE_TRY(timed(K_PAIR_DGRAD, st, [&] { return run_gemm_pair(L, c, PAIR_DGRAD, p9, p11, st); }));
   MOE_TRY_STATUS(router_backward(L, c, X, dW_r, status, st));
   MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
     return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
   }));
-  {
-    GemmParams p = base_params(L, c, status);
-    p.poff = c.tab.seg_poff;
-    p.cum = c.tab.cum;
-    p.nseg = nseg;
-    MOE_TMAP(tmap_2d(&p.ta0, c.dabuf, L.I, RP, L.I, 64, 128));
-    MOE_TMAP(tmap_2d(&p.ta1, c.dbbuf, L.I, RP, L.I, 64, 128));
-    MOE_TMAP(tmap_2d(&p.tb0, W_gate, L.I, El * L.d, L.I, 64, 256));
-    MOE_TMAP(tmap_2d(&p.tb1, W_up, L.I, El * L.d, L.I, 64, 256));
-    p.out0 = c.dxperm;
-    MOE_TRY(timed(K_GEMM_DGRAD_GATEUP, st, [&] { return launch_gemm(G_DGRAD_GATEUP, p, grid, st); }));
-  }
   MOE_TRY(timed(K_REV_DISPATCH, st, [&] { return launch_rev_dispatch(L, c, static_cast<__nv_bfloat16*>(dX), st); }));
   {  // wgrad of W_down: Hg and dY_perm cover the whole stream
     GemmParams p = base_params(L, c, status);

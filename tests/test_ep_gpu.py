@@ -132,6 +132,11 @@ def test_expert_parallel_two_ranks_many_experts():
     _check_against_one_device_layer(2, 200, 256, 64, 6, 256, seed=53)
 
 
+def test_expert_parallel_eight_ranks():
+    # eight ranks (one NVL8 node's worth), 4 experts each, top-8 over 32 experts
+    _check_against_one_device_layer(8, 64, 256, 32, 8, 256, seed=55)
+
+
 def test_expert_parallel_wait_for_an_unpublished_step_times_out_and_recovers():
     # After a good step, rank 0's expert phase is asked for an epoch no rank published: its bounded
     # wait gives up (about 2 s), records MOE_ERR_DEVICE_TIMEOUT, and the phase's exchange kernels
