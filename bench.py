@@ -123,9 +123,10 @@ def workload_config(w: IN.Workload) -> dict:
 
 
 def run_config(w: IN.Workload, args) -> dict:
-    """The `config` of both arms' lines: the workload, the gradient dtype and the forward's launch form."""
+    """The `config` of both arms' lines: the workload, the gradient dtype and how the GEMM pairs are
+    launched (the ring-streamed layer always runs them as persistent pairs)."""
     return dict(workload_config(w), wgrad_dtype="fp32" if args.wgrad_fp32 else "bf16",
-                forward="persistent" if args.persistent else "launches")
+                forward="persistent" if args.persistent or w.stream_M else "launches")
 
 
 L2_BYTES = 126 << 20
@@ -762,6 +763,8 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     w = IN.WORKLOADS[args.workload]
+    if args.launches and w.stream_M:
+        ap.error("the ring-streamed layer always runs its GEMM pairs as persistent launches")
     if args.persistent and (w.mxfp8 or w.stream_M or args.launches):
         ap.error("--persistent runs the bf16 one-batch layer with persistent GEMM pairs; %s" %
                  ("--launches was given" if args.launches else "%s is %s" % (w.name, "MXFP8" if w.mxfp8 else "streamed")))
