@@ -859,7 +859,6 @@ moe_status moe_fwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
     const moe_status r = route_tokens(L, c, X, W_r, bias, static_cast<int>(ring_rows), st);
     if (r != MOE_OK) return r;
   }
-  const int grid = num_sms();
   int* status = c.hdr + HDR_STATUS;
   const uint64_t RP = static_cast<uint64_t>(L.RP);
   const int El = L.El;
@@ -1404,7 +1403,6 @@ moe_status moe_ep_fwd_experts(const moe_shape* s, int32_t R, int32_t rank, void*
   int* base = reinterpret_cast<int*>(static_cast<char*>(ctx) + S.base_off);
   const int TK = static_cast<int>(S.TK);
   const uint64_t RP = static_cast<uint64_t>(L.RP);
-  const int grid = num_sms();
   // every source has published its table and rows: pull them
   MOE_TRY(launch_ep_wait(P, R, rank, false, S.B.flags, EPF_FWD_READY, epoch, status, st));
   MOE_TRY(launch_ep_plan(P, R, S.B.counts, S.first, S.El, L.RP, c.counts, c.poff, base, c.hdr, status, st));
@@ -1413,26 +1411,22 @@ moe_status moe_ep_fwd_experts(const moe_shape* s, int32_t R, int32_t rank, void*
   MOE_TRY(timed(K_DISPATCH, st, [&] {
     return launch_ep_gather(P, S.B.x, TK, L.k, L.d, c.poff, L.El, c.row_asg, L.RP, c.xperm, status, st);
   }));
-  {
-    GemmParams p = base_params(L, c, status);
-    MOE_TMAP(tmap_2d(&p.ta0, c.xperm, L.d, RP, L.d, 64, 128));
-    MOE_TMAP(tmap_2d(&p.tb0, W_gate, L.I, static_cast<uint64_t>(L.El) * L.d, L.I, 64, 64));
-    MOE_TMAP(tmap_2d(&p.tb1, W_up, L.I, static_cast<uint64_t>(L.El) * L.d, L.I, 64, 64));
-    p.ta1 = p.ta0;
-    p.out0 = c.abuf;
-    p.out1 = c.bbuf;
-    p.out2 = c.hbuf;
-    MOE_TRY(timed(K_GEMM_GATEUP, st, [&] { return launch_gemm(G_GATEUP, p, grid, st); }));
-  }
-  {
-    GemmParams p = base_params(L, c, status);
-    MOE_TMAP(tmap_2d(&p.ta0, c.hbuf, L.I, RP, L.I, 64, 128));
-    MOE_TMAP(tmap_2d(&p.tb0, W_down, L.d, static_cast<uint64_t>(L.El) * L.I, L.d, 64, 64));
-    p.ta1 = p.ta0;
-    p.tb1 = p.tb0;
-    p.out0 = c.obuf;
-    MOE_TRY(timed(K_GEMM_DOWN, st, [&] { return launch_gemm(G_DOWN, p, grid, st); }));
-  }
+  // the owner's gate/up and down GEMMs as one persistent launch
+  GemmParams gu = base_params(L, c, status);
+  MOE_TMAP(tmap_2d(&gu.ta0, c.xperm, L.d, RP, L.d, 64, 128));
+  MOE_TMAP(tmap_2d(&gu.tb0, W_gate, L.I, static_cast<uint64_t>(L.El) * L.d, L.I, 64, 64));
+  MOE_TMAP(tmap_2d(&gu.tb1, W_up, L.I, static_cast<uint64_t>(L.El) * L.d, L.I, 64, 64));
+  gu.ta1 = gu.ta0;
+  gu.out0 = c.abuf;
+  gu.out1 = c.bbuf;
+  gu.out2 = c.hbuf;
+  GemmParams dn = base_params(L, c, status);
+  MOE_TMAP(tmap_2d(&dn.ta0, c.hbuf, L.I, RP, L.I, 64, 128));
+  MOE_TMAP(tmap_2d(&dn.tb0, W_down, L.d, static_cast<uint64_t>(L.El) * L.I, L.d, 64, 64));
+  dn.ta1 = dn.ta0;
+  dn.tb1 = dn.tb0;
+  dn.out0 = c.obuf;
+  MOE_TRY(timed(K_PAIR_FWD, st, [&] { return run_gemm_pair(L, c, PAIR_FWD, gu, dn, st); }));
   // push each output row back to its source's slot, then tell every source
   MOE_TRY(timed(K_COMBINE, st, [&] {
     return launch_ep_push_rows(P, S.B.recv_o, TK, L.d, c.poff, L.El, c.row_asg, L.RP, c.obuf, status, st);
@@ -1491,38 +1485,35 @@ moe_status moe_ep_bwd_experts(const moe_shape* s, int32_t R, int32_t rank, void*
   const Ctx c = make_ctx(L, static_cast<char*>(ctx) + S.ctx_o, static_cast<char*>(ws) + S.ws_o);
   const int TK = static_cast<int>(S.TK);
   const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
-  const int grid = num_sms();
   MOE_TRY(launch_ep_wait(P, R, rank, false, S.B.flags, EPF_BWD_READY, epoch, status, st));
   // pull reverse-combine: dY rows from every source
   MOE_TRY(timed(K_REV_COMBINE, st, [&] {
     return launch_ep_gather(P, S.B.dy, TK, L.k, L.d, c.poff, L.El, c.row_asg, L.RP, c.dyperm, status, st);
   }));
-  {
-    GemmParams p = base_params(L, c, status);
-    MOE_TMAP(tmap_2d(&p.ta0, c.dyperm, L.d, RP, L.d, 64, 128));
-    MOE_TMAP(tmap_2d(&p.tb0, W_down, L.d, El * L.I, L.d, 64, 256));
-    p.ta1 = p.ta0;
-    p.tb1 = p.tb0;
-    p.in0 = c.abuf;
-    p.in1 = c.bbuf;
-    p.out0 = c.dabuf;
-    p.out1 = c.dbbuf;
-    p.out2 = c.hgbuf;
-    p.outf = c.dgpart;
-    MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm(G_DGRAD_DOWN, p, grid, st); }));
-  }
+  // the owner's dgrad of W_down (SwiGLU backward, router-gate partials) and dgrad of gate/up as
+  // one persistent launch
+  GemmParams p9 = base_params(L, c, status);
+  MOE_TMAP(tmap_2d(&p9.ta0, c.dyperm, L.d, RP, L.d, 64, 128));
+  MOE_TMAP(tmap_2d(&p9.tb0, W_down, L.d, El * L.I, L.d, 64, 256));
+  p9.ta1 = p9.ta0;
+  p9.tb1 = p9.tb0;
+  p9.in0 = c.abuf;
+  p9.in1 = c.bbuf;
+  p9.out0 = c.dabuf;
+  p9.out1 = c.dbbuf;
+  p9.out2 = c.hgbuf;
+  p9.outf = c.dgpart;
+  GemmParams p11 = base_params(L, c, status);
+  MOE_TMAP(tmap_2d(&p11.ta0, c.dabuf, L.I, RP, L.I, 64, 128));
+  MOE_TMAP(tmap_2d(&p11.ta1, c.dbbuf, L.I, RP, L.I, 64, 128));
+  MOE_TMAP(tmap_2d(&p11.tb0, W_gate, L.I, El * L.d, L.I, 64, 256));
+  MOE_TMAP(tmap_2d(&p11.tb1, W_up, L.I, El * L.d, L.I, 64, 256));
+  p11.out0 = c.dxperm;
+  MOE_TRY(timed(K_PAIR_DGRAD, st, [&] { return run_gemm_pair(L, c, PAIR_DGRAD, p9, p11, st); }));
+  // push each row's router-gate gradient back to its source
   MOE_TRY(timed(K_ROUTER_BWD, st, [&] {
     return launch_ep_push_dg(P, S.B.recv_dg, TK, c.poff, L.El, c.row_asg, c.dgpart, L.I / 256, L.RP, status, st);
   }));
-  {
-    GemmParams p = base_params(L, c, status);
-    MOE_TMAP(tmap_2d(&p.ta0, c.dabuf, L.I, RP, L.I, 64, 128));
-    MOE_TMAP(tmap_2d(&p.ta1, c.dbbuf, L.I, RP, L.I, 64, 128));
-    MOE_TMAP(tmap_2d(&p.tb0, W_gate, L.I, El * L.d, L.I, 64, 256));
-    MOE_TMAP(tmap_2d(&p.tb1, W_up, L.I, El * L.d, L.I, 64, 256));
-    p.out0 = c.dxperm;
-    MOE_TRY(timed(K_GEMM_DGRAD_GATEUP, st, [&] { return launch_gemm(G_DGRAD_GATEUP, p, grid, st); }));
-  }
   // push reverse-dispatch: dX rows to their sources, then tell every source
   MOE_TRY(timed(K_REV_DISPATCH, st, [&] {
     return launch_ep_push_rows(P, S.B.recv_dx, TK, L.d, c.poff, L.El, c.row_asg, L.RP, c.dxperm, status, st);
