@@ -121,3 +121,36 @@ def test_persistent_pair_wait_for_rows_nobody_writes_times_out_and_recovers():
     assert torch.equal(_bits(Y1), _bits(Y0))
     for n in g0:
         assert torch.equal(_bits(g1[n]), _bits(g0[n])), n
+
+
+def test_persistent_pairs_with_fp32_weight_gradients():
+    # the dgrad pair feeds the fp32 weight-gradient path exactly as the separate launches do
+    T, d, E, k, I = 400, 256, 8, 2, 256
+    w, x = make_case(T, d, E, k, I, seed=88)
+    W = [x[n].contiguous() for n in ("W_gate", "W_up", "W_down")]
+    out = []
+    for persistent in (False, True):
+        lay = B.MoELayer(T, d, E, I, k, wgrad_dtype=torch.float32)
+        Y = lay.forward(x["X"], x["W_r"], x["bias"], *W, persistent=persistent)
+        g = lay.backward(x["X"], x["W_r"], *W, x["dY"], persistent=persistent)
+        torch.cuda.synchronize()
+        assert lay.error() == B.MOE_OK
+        assert g["dW_gate"].dtype == torch.float32
+        out.append((Y, g))
+    assert torch.equal(_bits(out[1][0]), _bits(out[0][0]))
+    for n in out[0][1]:
+        assert torch.equal(_bits(out[1][1][n]), _bits(out[0][1][n])), n
+
+
+def test_persistent_forward_without_tokens_clears_the_status():
+    T, d, E, k, I = 0, 256, 8, 2, 256
+    lay = B.MoELayer(1, d, E, I, k)  # buffers of a one-token layer; the call below has no tokens
+    shape0 = B.make_shape(T, d, E, I, k)
+    lay.ctx.fill_(0xFF)  # a stale status word
+    W = [torch.zeros(E, d, I, dtype=torch.bfloat16, device="cuda"), torch.zeros(E, d, I, dtype=torch.bfloat16,
+                                                                                     device="cuda"),
+         torch.zeros(E, I, d, dtype=torch.bfloat16, device="cuda")]
+    W_r = torch.zeros(d, E, dtype=torch.bfloat16, device="cuda")
+    assert B.moe_fwd_persistent(shape0, None, W_r, None, *W, None, lay.ctx, lay.ws) == B.MOE_OK
+    torch.cuda.synchronize()
+    assert B.moe_get_error(lay.ctx) == B.MOE_OK
