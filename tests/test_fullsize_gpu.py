@@ -11,7 +11,9 @@ what it can compute one piece at a time:
 * dW_gate, dW_up, dW_down of sampled experts (each depends on that expert's
   tokens alone);
 * dW_r in full against X^T dl computed in fp64 from the GPU's own dl, whose
-  sampled rows were checked against the oracle;
+  sampled rows were checked against the oracle; and, independent of the GPU's dl, the
+  invariant that every row of dW_r sums to zero over the experts (each token's gates sum to
+  one, so its dl sums to zero over its slots);
 * a second run is bit-identical.
 """
 import numpy as np
@@ -84,7 +86,7 @@ def test_full_size_workload(name):
     Wg, Wu, Wd = ExpertCache(x["W_gate"]), ExpertCache(x["W_up"]), ExpertCache(x["W_down"])
     dY = to64(x["dY"])
     rng = np.random.default_rng(1234)
-    toks = [t for t in rng.choice(w.T, size=12, replace=False).tolist() if t not in tie_tokens][:8]
+    toks = [t for t in rng.choice(w.T, size=24, replace=False).tolist() if t not in tie_tokens][:16]
     Yg, dXg = to64(Y), to64(g["dX"])
     dl_gpu = to64(layer.router_grad())  # [T, k], slot order of the GPU's ids
     ys, yo, dxs, dxo, dls, dlo = [], [], [], [], [], []
@@ -100,6 +102,11 @@ def test_full_size_workload(name):
     dl_dense = np.zeros((w.T, w.E))
     np.put_along_axis(dl_dense, gids.astype(np.int64), dl_gpu, axis=1)
     assert relerr(to64(g["dW_r"]), X.T @ dl_dense) <= 1e-4
+    # dl_t = g_t (dg_t - sum_m g_m dg_m) with sum_m g_m = 1 sums to zero over a token's slots,
+    # so dW_r 1_E = X^T DL 1_E = 0 (up to the fp32 rounding of dl and of the GEMM)
+    dWr64 = to64(g["dW_r"])
+    assert np.max(np.abs(dl_gpu.sum(axis=1))) <= 1e-4 * max(np.max(np.abs(dl_gpu)), 1e-30)
+    assert np.max(np.abs(dWr64.sum(axis=1))) <= 3e-3 * np.max(np.abs(dWr64))
 
     # -- expert weight gradients for the hottest and the coldest non-empty expert
     counts = r["counts"].cpu().numpy()
