@@ -312,17 +312,16 @@ __global__ void __launch_bounds__(128) k_gather_rows(const __nv_bfloat16* __rest
     if (a == ROW_DEAD) continue;  // never read
     uint4* out = reinterpret_cast<uint4*>(dst + (R + sh) * d);
     const uint4* in = a >= 0 ? reinterpret_cast<const uint4*>(src + static_cast<size_t>(a / k) * d) : nullptr;
-    // up to eight independent loads in flight per thread before their stores: a row of
-    // d <= 8192 is one round trip
-    for (int i0 = threadIdx.x; i0 < nv; i0 += 8 * blockDim.x) {
-      uint4 u[8];
+    // four independent loads in flight per thread before their stores
+    for (int i0 = threadIdx.x; i0 < nv; i0 += 4 * blockDim.x) {
+      uint4 u[4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < 4; ++j) {
         const int i = i0 + j * blockDim.x;
         u[j] = (in != nullptr && i < nv) ? __ldg(in + i) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < 4; ++j) {
         const int i = i0 + j * blockDim.x;
         if (i < nv) out[i] = u[j];
       }
