@@ -154,3 +154,25 @@ def test_persistent_forward_without_tokens_clears_the_status():
     assert B.moe_fwd_persistent(shape0, None, W_r, None, *W, None, lay.ctx, lay.ws) == B.MOE_OK
     torch.cuda.synchronize()
     assert B.moe_get_error(lay.ctx) == B.MOE_OK
+
+
+def test_persistent_pairs_full_size_kimi_zipf_equals_the_launches():
+    # T = 4096, E = 384, top-8 under the Zipf(1.2) bias (hottest expert about 10x the mean): hot
+    # experts with several m-tiles, so down tiles wait on many gate/up tiles of their rows
+    from mixture_experts_layer_27_b200 import inputs as IN
+    w = IN.WORKLOADS["kimi"]
+    x = IN.make_inputs(w, device="cuda")
+    out = []
+    for persistent in (False, True):
+        lay = B.MoELayer(w.T, w.d, w.E, w.I, w.k)
+        Y = lay.forward(x["X"], x["W_r"], x["bias"], x["W_gate"], x["W_up"], x["W_down"], persistent=persistent)
+        g = lay.backward(x["X"], x["W_r"], x["W_gate"], x["W_up"], x["W_down"], x["dY"], persistent=persistent)
+        torch.cuda.synchronize()
+        assert lay.error() == B.MOE_OK
+        out.append((Y, g))
+        del lay
+    assert torch.equal(_bits(out[1][0]), _bits(out[0][0]))
+    for n in out[0][1]:
+        assert torch.equal(_bits(out[1][1][n]), _bits(out[0][1][n])), n
+    del out, x
+    torch.cuda.empty_cache()
