@@ -303,8 +303,8 @@ class ClockSampler:
 # ORACLE_WINDOW consecutive local experts (every token routed, then those experts' assignments
 # through the SwiGLU experts and back, their weight gradients, the router gradient of their
 # tokens).  Its work in token units is the assignments it processed / top_k.  The rate is that
-# work over the measured time: nothing is extrapolated, and both CPU figures (cpu_baseline and
-# the reference arm) use this one sampler.
+# work over the median measured step time: nothing is extrapolated, and both CPU figures
+# (cpu_baseline and the reference arm) use this one sampler.
 # ----------------------------------------------------------------------------
 ORACLE_WINDOW = 8
 CPU_BASELINE_STEPS = 8
