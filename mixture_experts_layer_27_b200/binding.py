@@ -47,6 +47,37 @@ def _wgrad_code(dtype) -> int:
     raise ValueError(f"expert weight gradients are bfloat16 or float32, not {dtype}")
 
 
+def _expect(t, shape, name):
+    """Refuses a tensor whose shape does not match the layer's: the C ABI takes bare device
+    pointers and cannot see sizes, so a wrong tensor would otherwise be read or written out of
+    bounds on the device.  None passes (optional arguments, empty batches)."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, this layer expects {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous (row-major)")
+
+
+def _expect_layer(lay, T, X=None, W_r=None, bias=None, W_gate=None, W_up=None, W_down=None, Y=None, dY=None,
+                  out=None):
+    d, E, I, El = lay.d, lay.E, lay.I, lay.El
+    _expect(X, (T, d), "X")
+    _expect(W_r, (d, E), "W_r")
+    _expect(bias, (E,), "bias")
+    _expect(W_gate, (El, d, I), "W_gate")
+    _expect(W_up, (El, d, I), "W_up")
+    _expect(W_down, (El, I, d), "W_down")
+    _expect(Y, (T, d), "Y")
+    _expect(dY, (T, d), "dY")
+    if out is not None:
+        _expect(out["dX"], (T, d), "dX")
+        _expect(out["dW_gate"], (El, d, I), "dW_gate")
+        _expect(out["dW_up"], (El, d, I), "dW_up")
+        _expect(out["dW_down"], (El, I, d), "dW_down")
+        _expect(out["dW_r"], (d, E), "dW_r")
+
+
 def _grad_buffers(T, d, E, I, El, wdt, dev) -> dict:
     import torch
     return dict(dX=torch.empty(T, d, dtype=torch.bfloat16, device=dev),
@@ -326,12 +357,14 @@ class MoELayerMX:
         self.El = num_local_experts or (E - first_local_expert)
 
     def prepare(self, W_gate, W_up, W_down, stream=None):
+        _expect_layer(self, self.T, W_gate=W_gate, W_up=W_up, W_down=W_down)
         check(moe_prepare_weights(self.shape, W_gate, W_up, W_down, self.wq, stream), "moe_prepare_weights")
 
     def forward(self, X, W_r, bias, Y=None, stream=None):
         import torch
         if Y is None:
             Y = torch.empty(self.T, self.d, dtype=torch.bfloat16, device=X.device)
+        _expect_layer(self, self.T, X=X, W_r=W_r, bias=bias, Y=Y)
         check(moe_fwd_mx(self.shape, X, W_r, bias, self.wq, Y, self.ctx, self.ws, stream), "moe_fwd_mx")
         return Y
 
@@ -339,6 +372,7 @@ class MoELayerMX:
         import torch
         if out is None:
             out = _grad_buffers(self.T, self.d, self.E, self.I, self.El, self.wgrad_dtype, X.device)
+        _expect_layer(self, self.T, X=X, W_r=W_r, dY=dY, out=out)
         check(moe_bwd_mx(self.shape, X, W_r, self.wq, dY, self.ctx, out["dX"], out["dW_gate"], out["dW_up"],
                          out["dW_down"], out["dW_r"], self.ws, stream), "moe_bwd_mx")
         return out
@@ -494,6 +528,7 @@ class MoEStream:
         import torch
         if Y is None:
             Y = torch.empty(self.M * self.T, self.d, dtype=torch.bfloat16, device=X.device)
+        _expect_layer(self, self.M * self.T, X=X, W_r=W_r, bias=bias, W_gate=W_gate, W_up=W_up, W_down=W_down, Y=Y)
         check(moe_fwd_stream(self.shape, self.M, X, W_r, bias, W_gate, W_up, W_down, Y, self.ctx, self.ring,
                              self.ws, stream), "moe_fwd_stream")
         return Y
@@ -502,6 +537,7 @@ class MoEStream:
         import torch
         if out is None:
             out = _grad_buffers(self.M * self.T, self.d, self.E, self.I, self.El, self.wgrad_dtype, X.device)
+        _expect_layer(self, self.M * self.T, X=X, W_r=W_r, W_gate=W_gate, W_up=W_up, W_down=W_down, dY=dY, out=out)
         check(moe_bwd_stream(self.shape, self.M, X, W_r, W_gate, W_up, W_down, dY, self.ctx, out["dX"],
                              out["dW_gate"], out["dW_up"], out["dW_down"], out["dW_r"], self.ring, self.ws, stream),
               "moe_bwd_stream")
@@ -550,6 +586,7 @@ class MoELayer:
         import torch
         if Y is None:
             Y = torch.empty(self.T, self.d, dtype=torch.bfloat16, device=X.device)
+        _expect_layer(self, self.T, X=X, W_r=W_r, bias=bias, W_gate=W_gate, W_up=W_up, W_down=W_down, Y=Y)
         fn, name = (moe_fwd_persistent, "moe_fwd_persistent") if persistent else (moe_fwd, "moe_fwd")
         check(fn(self.shape, X, W_r, bias, W_gate, W_up, W_down, Y, self.ctx, self.ws, stream), name)
         return Y
@@ -559,6 +596,7 @@ class MoELayer:
         import torch
         if out is None:
             out = _grad_buffers(self.T, self.d, self.E, self.I, self.El, self.wgrad_dtype, X.device)
+        _expect_layer(self, self.T, X=X, W_r=W_r, W_gate=W_gate, W_up=W_up, W_down=W_down, dY=dY, out=out)
         check(moe_bwd(self.shape, X, W_r, W_gate, W_up, W_down, dY, self.ctx, out["dX"], out["dW_gate"],
                       out["dW_up"], out["dW_down"], out["dW_r"], self.ws, stream, persistent=persistent),
               "moe_bwd_persistent" if persistent else "moe_bwd")

@@ -178,3 +178,29 @@ def test_expert_parallel_sizes_and_argument_errors(lib):
     assert lib.moe_ep_fwd_combine(by(s), 2, 0, good, None, fake, nc, 1, None) == B.MOE_ERR_INVALID_ARG  # no Y
     assert lib.moe_ep_bwd_finish(by(s), 2, 0, good, fake, fake, fake, None, fake, nc, fake, nw, 1,
                                  None) == B.MOE_ERR_INVALID_ARG  # no dW_r
+
+
+def test_binding_refuses_tensors_of_the_wrong_shape_before_any_call(lib):
+    # The C ABI takes bare pointers; the binding checks every tensor against the layer's shape
+    # (here a 2-expert slice of 8) and raises before the library sees a pointer.  Host tensors
+    # suffice: nothing reaches the device.
+    import torch
+    T, d, E, I, k = 16, 256, 8, 256, 2
+    lay = B.MoELayer(T, d, E, I, k, first_local_expert=2, num_local_experts=2, device="cpu")
+    bf = torch.bfloat16
+    X, W_r = torch.zeros(T, d, dtype=bf), torch.zeros(d, E, dtype=bf)
+    Wg, Wu, Wd = torch.zeros(2, d, I, dtype=bf), torch.zeros(2, d, I, dtype=bf), torch.zeros(2, I, d, dtype=bf)
+    full = torch.zeros(E, d, I, dtype=bf)  # every expert's weights, not the slice's
+    with pytest.raises(ValueError, match="W_gate"):
+        lay.forward(X, W_r, None, full, Wu, Wd)
+    with pytest.raises(ValueError, match="X"):
+        lay.forward(torch.zeros(T + 1, d, dtype=bf), W_r, None, Wg, Wu, Wd)
+    with pytest.raises(ValueError, match="bias"):
+        lay.forward(X, W_r, torch.zeros(E - 1), Wg, Wu, Wd)
+    with pytest.raises(ValueError, match="contiguous"):
+        lay.forward(X, W_r, None, Wg, Wu, torch.zeros(2, d, I, dtype=bf).transpose(1, 2))
+    with pytest.raises(ValueError, match="dY"):
+        lay.backward(X, W_r, Wg, Wu, Wd, torch.zeros(T, d + 1, dtype=bf))
+    mx = B.MoELayerMX(T, d, E, I, k, 2, 2, device="cpu")
+    with pytest.raises(ValueError, match="W_down"):
+        mx.prepare(Wg, Wu, torch.zeros(E, I, d, dtype=bf))
