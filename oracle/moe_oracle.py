@@ -465,7 +465,10 @@ def stream_plan(mb_counts, ring_rows: int, min_rows: int, P: int = P_PAD) -> dic
 # ----------------------------------------------------------------------------
 # MXFP8 layer: every operand of the gate/up, down and dgrad GEMMs rounded to MX
 # (E4M3 + E8M0 per 32 along that GEMM's contraction dimension) before the
-# product; the weight-gradient GEMMs contract over tokens and are not quantised.
+# product.  The weight-gradient GEMMs contract over tokens: unquantised by
+# default; with mx_wgrad their operands (X, dA, dB, Hg = g H and dY of one
+# expert) are rounded along the expert's rows, in blocks of 32 rows from its
+# first row, the rows zero-padded to a multiple of 32.
 # fp64 everywhere else.  The router gradient takes dg = <dH', H> with dH' the
 # quantised dgrad of W_down (the fused form; the identity with <dY, O> holds only
 # without quantisation).
@@ -474,6 +477,15 @@ def mx_round(v, axis: int):
     """v rounded to its MXFP8 value along `axis` (fp64)."""
     c, s = mx_quantize(v, axis=axis)
     return mx_dequantize(c, s, axis=axis)
+
+
+def mx_round_rows(v):
+    """v [rows, n] (one expert's rows in order) rounded to MXFP8 along the rows, in blocks
+    of 32 rows from the first; rows past the last multiple of 32 are padded with zeros."""
+    v = _f64(v)
+    pad = (-v.shape[0]) % 32
+    vp = np.concatenate([v, np.zeros((pad,) + v.shape[1:])], axis=0) if pad else v
+    return mx_round(vp, axis=0)[:v.shape[0]]
 
 
 def mx_weight_layouts(Wg, Wu, Wd) -> dict:
@@ -530,7 +542,10 @@ def forward_mx(X, W_r, bias, W_gate, W_up, W_down, top_k: int, first_local: int 
     return Y, ctx
 
 
-def backward_mx(ctx, dY):
+def backward_mx(ctx, dY, mx_wgrad: bool = False):
+    """MXFP8 layer backward.  mx_wgrad: the weight-gradient GEMMs on MXFP8 as well, each
+    operand rounded along the expert's rows (mx_round_rows); otherwise they take the
+    unrounded operands."""
     dY64 = _f64(dY)
     X64, ids, g, sched = ctx["X"], ctx["ids"], ctx["g"], ctx["sched"]
     T, d = X64.shape
@@ -558,9 +573,15 @@ def backward_mx(ctx, dY):
         dA = dH * B * silu_grad(A)
         dB = dH * silu(A)
         dX[toks] += mx_round(dA, axis=1) @ Wq["gate_i"].T + mx_round(dB, axis=1) @ Wq["up_i"].T  # K = I
-        dW_gate[e] = Xe.T @ dA
-        dW_up[e] = Xe.T @ dB
-        dW_down[e] = H.T @ (ge[:, None] * dYe)
+        if mx_wgrad:  # K = the expert's rows
+            Xr = mx_round_rows(Xe)
+            dW_gate[e] = Xr.T @ mx_round_rows(dA)
+            dW_up[e] = Xr.T @ mx_round_rows(dB)
+            dW_down[e] = mx_round_rows(ge[:, None] * H).T @ mx_round_rows(dYe)
+        else:
+            dW_gate[e] = Xe.T @ dA
+            dW_up[e] = Xe.T @ dB
+            dW_down[e] = H.T @ (ge[:, None] * dYe)
     dl = np.zeros((T, E))
     s = np.sum(g * dg, axis=1, keepdims=True)
     np.put_along_axis(dl, ids.astype(np.int64), g * (dg - s), axis=1)

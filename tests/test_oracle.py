@@ -377,7 +377,8 @@ def test_mx_quantize_axis0_equals_transposed_axis1():
 # be the bf16 layer exactly (operands, axes and the fused router gradient wired
 # as the unquantised definition); the rounding itself is pinned above.
 # --------------------------------------------------------------------------
-def test_mx_layer_reduces_to_the_plain_layer_without_rounding(monkeypatch):
+@pytest.mark.parametrize("mx_wgrad", [False, True])
+def test_mx_layer_reduces_to_the_plain_layer_without_rounding(monkeypatch, mx_wgrad):
     import oracle.moe_oracle as M
     rng = np.random.default_rng(14)
     T, d, E, I, k = 40, 64, 6, 96, 2
@@ -386,7 +387,7 @@ def test_mx_layer_reduces_to_the_plain_layer_without_rounding(monkeypatch):
     g = O.backward(ctx, dY)
     monkeypatch.setattr(M, "mx_round", lambda v, axis: np.asarray(v, dtype=np.float64))
     Yq, cq = M.forward_mx(X, W_r, None, Wg, Wu, Wd, k)
-    gq = M.backward_mx(cq, dY)
+    gq = M.backward_mx(cq, dY, mx_wgrad=mx_wgrad)
     np.testing.assert_allclose(Yq, Y, rtol=1e-13, atol=1e-13)
     for n in ("dX", "dW_r", "dl", "dg"):
         np.testing.assert_allclose(gq[n], g[n], rtol=1e-11, atol=1e-12)
@@ -491,17 +492,20 @@ def test_mx_forward_down_weight_columns_are_independent():
     assert _same_except(Y, Y2, 1, 9)
 
 
-def test_mx_dgrad_down_weight_rows_are_independent():
+@pytest.mark.parametrize("mx_wgrad", [False, True])
+def test_mx_dgrad_down_weight_rows_are_independent(mx_wgrad):
     # In the dgrad of W_down (contraction over d) W_down is rounded along d: scaling its row i
     # (of I) in the backward alone scales dH'[:, i], hence dA[:, i] and dB[:, i], exactly, so
-    # column i of dW_gate and dW_up scales exactly and no other column moves.
+    # column i of dW_gate and dW_up scales exactly and no other column moves.  With mx_wgrad
+    # the same holds only if dA and dB are rounded along the rows (tokens): rounded along I,
+    # the scaled column would become the amax of its blocks and move its neighbours.
     X, W_r, Wg, Wu, Wd, dY = _mx_case()
     _, ctx = O.forward_mx(X, W_r, None, Wg, Wu, Wd, _MX_SHAPE["k"])
-    g = O.backward_mx(ctx, dY)
+    g = O.backward_mx(ctx, dY, mx_wgrad=mx_wgrad)
     e, i = 2, 45
     Wd2 = Wd.copy()
     Wd2[e][i, :] *= _P2
-    g2 = O.backward_mx(dict(ctx, W_down=Wd2), dY)
+    g2 = O.backward_mx(dict(ctx, W_down=Wd2), dY, mx_wgrad=mx_wgrad)
     for n in ("dW_gate", "dW_up"):
         assert _same_except(g[n][e], g2[n][e], 1, i), n
         assert np.array_equal(g2[n][e][:, i], g[n][e][:, i] * _P2), n
@@ -545,6 +549,93 @@ def test_mx_layer_worked_example_by_hand():
             want[r, c] = v
         np.testing.assert_allclose(got[name], want, rtol=1e-13, atol=0, err_msg=name)
     assert not np.any(g["dW_r"])
+
+
+# --------------------------------------------------------------------------
+# MX weight gradients (mx_wgrad): X, dA, dB, Hg = g H and dY rounded along the expert's
+# rows in blocks of 32.  Blocks along the rows commute with scaling one column by a power
+# of two, so a column scaled that way moves its own row (or column) of the gradient, by
+# that power exactly, and nothing else; rounded along d or I instead, the scaled column
+# would become the amax of its blocks and move its neighbours.
+# --------------------------------------------------------------------------
+def test_mx_wgrad_x_columns_are_independent():
+    # X scaled in the backward alone (its weight gradients): column j of X moves row j of
+    # every expert's dW_gate and dW_up
+    X, W_r, Wg, Wu, Wd, dY = _mx_case()
+    _, ctx = O.forward_mx(X, W_r, None, Wg, Wu, Wd, _MX_SHAPE["k"])
+    g = O.backward_mx(ctx, dY, mx_wgrad=True)
+    j = 29
+    X2 = X.copy()
+    X2[:, j] *= _P2
+    g2 = O.backward_mx(dict(ctx, X=X2), dY, mx_wgrad=True)
+    for e in range(_MX_SHAPE["E"]):
+        for n in ("dW_gate", "dW_up"):
+            assert _same_except(g[n][e], g2[n][e], 0, j), (n, e)
+            assert np.array_equal(g2[n][e][j], g[n][e][j] * _P2), (n, e)
+
+
+def test_mx_wgrad_dy_columns_are_independent():
+    # dY column j moves column j of every expert's dW_down and no other (its dgrad changes
+    # too, but dW_down reads only Hg, from the forward, and dY itself)
+    X, W_r, Wg, Wu, Wd, dY = _mx_case()
+    _, ctx = O.forward_mx(X, W_r, None, Wg, Wu, Wd, _MX_SHAPE["k"])
+    g = O.backward_mx(ctx, dY, mx_wgrad=True)
+    j = 50
+    dY2 = dY.copy()
+    dY2[:, j] *= _P2
+    g2 = O.backward_mx(ctx, dY2, mx_wgrad=True)
+    for e in range(_MX_SHAPE["E"]):
+        assert _same_except(g["dW_down"][e], g2["dW_down"][e], 1, j), e
+        assert np.array_equal(g2["dW_down"][e][:, j], g["dW_down"][e][:, j] * _P2), e
+
+
+def test_mx_wgrad_hg_columns_are_independent():
+    # W_up column i of one expert (rounded along d in the forward) scales B[:, i], hence
+    # H[:, i], Hg[:, i] and dA[:, i], exactly: row i of dW_down and column i of dW_gate move,
+    # by that power, and nothing else of the expert's weight gradients
+    X, W_r, Wg, Wu, Wd, dY = _mx_case()
+    k = _MX_SHAPE["k"]
+    _, ctx = O.forward_mx(X, W_r, None, Wg, Wu, Wd, k)
+    g = O.backward_mx(ctx, dY, mx_wgrad=True)
+    e, i = 1, 7
+    Wu2 = Wu.copy()
+    Wu2[e][:, i] *= _P2
+    _, ctx2 = O.forward_mx(X, W_r, None, Wg, Wu2, Wd, k)
+    g2 = O.backward_mx(ctx2, dY, mx_wgrad=True)
+    assert _same_except(g["dW_down"][e], g2["dW_down"][e], 0, i)
+    assert np.array_equal(g2["dW_down"][e][i], g["dW_down"][e][i] * _P2)
+    assert _same_except(g["dW_gate"][e], g2["dW_gate"][e], 1, i)
+    assert np.array_equal(g2["dW_gate"][e][:, i], g["dW_gate"][e][:, i] * _P2)
+    assert np.array_equal(g2["dW_up"][e], g["dW_up"][e])
+
+
+def test_mx_wgrad_worked_example_by_hand():
+    # tests/golden/mx_wgrad_worked_example.json: the weight gradients of a two-expert MXFP8
+    # layer with MX weight-gradient GEMMs, every rounding worked out by hand there (row blocks
+    # of 32 from the expert's first row; Hg = g H and dY as the W_down operands)
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "mx_wgrad_worked_example.json")) as f:
+        G = json.load(f)
+    s = G["shape"]
+    T, d, E, k, I = s["T"], s["d"], s["E"], s["top_k"], s["I"]
+    arrays = {"X": np.zeros((T, d)), "dY": np.zeros((T, d)), "W_r": np.zeros((d, E))}
+    W = {n: np.zeros((E,) + shp) for n, shp in (("W_gate", (d, I)), ("W_up", (d, I)), ("W_down", (I, d)))}
+    for name, entries in G["inputs_nonzero"].items():
+        for r, c, v in entries:
+            if "[" in name:
+                W[name.split("[")[0]][int(name.split("[")[1][:-1])][r, c] = v
+            else:
+                arrays[name][r, c] = v
+    bias = np.array(G["bias"], dtype=np.float32)
+    Y, ctx = O.forward_mx(arrays["X"], arrays["W_r"], bias, W["W_gate"], W["W_up"], W["W_down"], k)
+    g = O.backward_mx(ctx, arrays["dY"], mx_wgrad=True)
+    for name, entries in G["expected"].items():
+        n, e = name.split("[")[0], int(name.split("[")[1][:-1])
+        want = np.zeros_like(g[n][e])
+        for r, c, v in entries:
+            want[r, c] = v
+        np.testing.assert_allclose(g[n][e], want, rtol=1e-15, atol=0, err_msg=name)
 
 
 def test_mx_token_path_and_slices_equal_the_full_mx_layer():
