@@ -479,6 +479,14 @@ def mx_round(v, axis: int):
     return mx_dequantize(c, s, axis=axis)
 
 
+def bf16_round(v):
+    """v rounded to bfloat16 through float32 (round to nearest even at each step), as fp64."""
+    x = np.asarray(v, dtype=np.float64).astype(np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
 def mx_round_rows(v):
     """v [rows, n] (one expert's rows in order) rounded to MXFP8 along the rows, in blocks
     of 32 rows from the first; rows past the last multiple of 32 are padded with zeros."""
@@ -545,7 +553,12 @@ def forward_mx(X, W_r, bias, W_gate, W_up, W_down, top_k: int, first_local: int 
 def backward_mx(ctx, dY, mx_wgrad: bool = False):
     """MXFP8 layer backward.  mx_wgrad: the weight-gradient GEMMs on MXFP8 as well, each
     operand rounded along the expert's rows (mx_round_rows); otherwise they take the
-    unrounded operands."""
+    unrounded operands.
+
+    The forward's saved pre-activations A and B are read as bf16 (bf16_round), the type the
+    layer keeps them in: every operand quantised here (dA, dB along I; with mx_wgrad dA, dB and
+    Hg along the rows) is computed from the values a kernel has, so both sides take each
+    rounding decision from the same inputs up to the order of fp32 sums."""
     dY64 = _f64(dY)
     X64, ids, g, sched = ctx["X"], ctx["ids"], ctx["g"], ctx["sched"]
     T, d = X64.shape
@@ -563,6 +576,7 @@ def backward_mx(ctx, dY, mx_wgrad: bool = False):
             continue
         Wq = _layouts(ctx.get("rounded"), ctx["W_gate"], ctx["W_up"], ctx["W_down"], e)
         toks, slots, A, B = item
+        A, B = bf16_round(A), bf16_round(B)
         Xe = X64[toks]
         ge = g[toks, slots]
         dYe = dY64[toks]
@@ -612,6 +626,8 @@ def token_forward_backward_mx(t: int, X, W_r, bias, rounded, top_k: int, dY):
         b = xq @ Wq["up_d"]
         h = silu(a) * b
         y += g[j] * (mx_round(h, axis=1) @ Wq["down_i"])[0]
+        a, b = bf16_round(a), bf16_round(b)  # the backward reads the saved bf16 A, B
+        h = silu(a) * b
         dhp = dyq @ Wq["down_d"].T
         dg[j] = float(np.sum(dhp * h))
         dh = g[j] * dhp

@@ -386,6 +386,7 @@ def test_mx_layer_reduces_to_the_plain_layer_without_rounding(monkeypatch, mx_wg
     Y, ctx = O.forward(X, W_r, None, Wg, Wu, Wd, k)
     g = O.backward(ctx, dY)
     monkeypatch.setattr(M, "mx_round", lambda v, axis: np.asarray(v, dtype=np.float64))
+    monkeypatch.setattr(M, "bf16_round", lambda v: np.asarray(v, dtype=np.float64))
     Yq, cq = M.forward_mx(X, W_r, None, Wg, Wu, Wd, k)
     gq = M.backward_mx(cq, dY, mx_wgrad=mx_wgrad)
     np.testing.assert_allclose(Yq, Y, rtol=1e-13, atol=1e-13)
@@ -394,6 +395,38 @@ def test_mx_layer_reduces_to_the_plain_layer_without_rounding(monkeypatch, mx_wg
     for n in ("dW_gate", "dW_up", "dW_down"):
         for e in range(E):
             np.testing.assert_allclose(gq[n][e], g[n][e], rtol=1e-11, atol=1e-12)
+
+
+def test_bf16_round_equals_torch_bfloat16_conversion():
+    # the saved-activation rounding of the MX backward: fp64 -> fp32 -> bf16, nearest even each
+    # time, against torch's conversions (halfway cases, signs, subnormals, large values)
+    import torch
+    rng = np.random.default_rng(16)
+    v = np.concatenate([rng.standard_normal(4000) * 10.0 ** rng.integers(-40, 38, 4000),
+                        [0.0, -0.0, 1.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8), 2.0 ** -130,
+                         3.0e38, 1.0 + 2.0 ** -8 + 2.0 ** -30]])
+    want = torch.from_numpy(v).to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+    got = O.bf16_round(v)
+    assert np.array_equal(np.signbit(got), np.signbit(want))
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("mx_wgrad", [False, True])
+def test_mx_backward_reads_the_saved_activations_as_bf16(mx_wgrad):
+    # Moving each saved A, B entry halfway towards its bf16 value keeps that value: the MX
+    # backward, which reads them as bf16, returns the same bits; the unrounded values differ.
+    X, W_r, Wg, Wu, Wd, dY = _mx_case()
+    _, ctx = O.forward_mx(X, W_r, None, Wg, Wu, Wd, _MX_SHAPE["k"])
+    g = O.backward_mx(ctx, dY, mx_wgrad=mx_wgrad)
+    saved = [None if it is None else (it[0], it[1], (it[2] + O.bf16_round(it[2])) / 2, (it[3] + O.bf16_round(it[3])) / 2)
+             for it in ctx["saved"]]
+    assert any(it is not None and not np.array_equal(it[2], ctx["saved"][e][2]) for e, it in enumerate(saved))
+    g2 = O.backward_mx(dict(ctx, saved=saved), dY, mx_wgrad=mx_wgrad)
+    for n in ("dX", "dg", "dl", "dW_r"):
+        assert np.array_equal(g[n], g2[n]), n
+    for n in ("dW_gate", "dW_up", "dW_down"):
+        for e in g[n]:
+            assert np.array_equal(g[n][e], g2[n][e]), (n, e)
 
 
 def test_mx_round_error_bound_and_idempotence():
