@@ -125,8 +125,11 @@ def workload_config(w: IN.Workload) -> dict:
 def run_config(w: IN.Workload, args) -> dict:
     """The `config` of both arms' lines: the workload, the gradient dtype and how the GEMM pairs are
     launched (the ring-streamed layer always runs them as persistent pairs)."""
-    return dict(workload_config(w), wgrad_dtype="fp32" if args.wgrad_fp32 else "bf16",
-                forward="persistent" if args.persistent or w.stream_M else "launches")
+    cfg = dict(workload_config(w), wgrad_dtype="fp32" if args.wgrad_fp32 else "bf16",
+               forward="persistent" if args.persistent or w.stream_M else "launches")
+    if w.mxfp8:  # the weight-gradient GEMMs: MXFP8 operands along the rows, or the bf16 operands
+        cfg["wgrad_gemms"] = "mxfp8" if getattr(args, "mx_wgrad", False) else "bf16"
+    return cfg
 
 
 L2_BYTES = 126 << 20
@@ -146,6 +149,7 @@ def algorithmic_flops(w: IN.Workload) -> dict:
     return {"gemm_gateup_swiglu": 4 * dI * rows, "gemm_down_combw": 2 * dI * rows,
             "gemm_dgrad_down_swiglu_bwd": 2 * dI * rows, "gemm_dgrad_gateup": 4 * dI * rows,
             "gemm_wgrad_gateup": 4 * dI * rows, "gemm_wgrad_down": 2 * dI * rows,
+            "gemm_wgrad_gateup_mx": 4 * dI * rows, "gemm_wgrad_down_mx": 2 * dI * rows,
             "router_logits": 2 * w.tokens * w.d * w.E,
             "gemm_gateup_down_persistent": 6 * dI * rows,  # gate/up and down in one launch
             "gemm_dgrads_persistent": 6 * dI * rows,  # both dgrads in one launch
@@ -157,7 +161,7 @@ def algorithmic_flops(w: IN.Workload) -> dict:
 # algorithmic bytes per launch of each kernel (minimum HBM traffic of its job)
 # rows = T*k routed assignments; weights of all local experts; bf16 = 2 bytes
 # ----------------------------------------------------------------------------
-def algorithmic_bytes(w: IN.Workload, wgrad_elem_bytes: int = 2) -> dict:
+def algorithmic_bytes(w: IN.Workload, wgrad_elem_bytes: int = 2, mx_wgrad: bool = False) -> dict:
     T, d, E, I, k, El = w.tokens, w.d, w.E, w.I, w.k, w.El
     rows = local_rows(w)
     W1 = El * d * I * 2  # one expert weight matrix family (gate, up or down), bytes
@@ -168,18 +172,24 @@ def algorithmic_bytes(w: IN.Workload, wgrad_elem_bytes: int = 2) -> dict:
         return {
             "router_logits": T * d * 2 + d * E * 2 + T * E * 4,
             "topk_gating": T * E * 4 + rows * 8,
-            "dispatch": T * d * 2 + rows * d * 2 + rows * d * 33 // 32,
+            # X once, then bf16 rows and fp8 along d; or (mx_wgrad) fp8 along d and along the rows
+            "dispatch": T * d * 2 + (2 * rows * d * 33 // 32 if mx_wgrad else rows * d * 2 + rows * d * 33 // 32),
             "gemm_gateup_swiglu": 2 * Wq + rows * d * 33 // 32 + 2 * rows * I * 2 + rows * I * 33 // 32,
             "gemm_down_combw": Wq + rows * I * 33 // 32 + rows * d * 2,
             "combine": rows * d * 2 + T * d * 2,
-            "reverse_combine": T * d * 2 + rows * d * 2 + rows * d * 33 // 32,
-            "gemm_dgrad_down_swiglu_bwd": Wq + rows * d * 33 // 32 + 2 * rows * I * 2 + 3 * rows * I * 2
-            + 2 * rows * I * 33 // 32,
+            "reverse_combine": T * d * 2 + (2 * rows * d * 33 // 32 if mx_wgrad else rows * d * 2 + rows * d * 33 // 32),
+            # dA, dB, Hg out in bf16 for the bf16 weight gradients, or (mx_wgrad) as fp8 along the rows
+            "gemm_dgrad_down_swiglu_bwd": Wq + rows * d * 33 // 32 + 2 * rows * I * 2
+            + (3 * rows * I * 33 // 32 if mx_wgrad else 3 * rows * I * 2) + 2 * rows * I * 33 // 32,
             "router_wgrad": T * d * 2 + T * k * 8 + d * E * 4,
             "gemm_dgrad_gateup": 2 * Wq + 2 * rows * I * 33 // 32 + rows * d * 2,
             "reverse_dispatch": rows * d * 2 + T * d * 2 + E * d * 2,
             "gemm_wgrad_gateup": rows * d * 2 + 2 * rows * I * 2 + 2 * G1,
             "gemm_wgrad_down": rows * I * 2 + rows * d * 2 + G1,
+            # MXFP8 weight gradients: the two GEMMs on the operands quantised along the rows (by the
+            # dispatch, the reverse-combine and the dgrad of W_down)
+            "gemm_wgrad_gateup_mx": (rows * d + 2 * rows * I) * 33 // 32 + 2 * G1,
+            "gemm_wgrad_down_mx": (rows * I + rows * d) * 33 // 32 + G1,
         }
     return {
         "router_logits": T * d * 2 + d * E * 2 + T * E * 4,
@@ -453,7 +463,8 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     x = IN.make_inputs(w, device=dev)
     wdt = torch.float32 if args.wgrad_fp32 else torch.bfloat16
     if w.mxfp8:
-        layer = B.MoELayerMX(w.T, w.d, w.E, w.I, w.k, w.first_local, w.num_local, device=dev, wgrad_dtype=wdt)
+        layer = B.MoELayerMX(w.T, w.d, w.E, w.I, w.k, w.first_local, w.num_local, device=dev, wgrad_dtype=wdt,
+                             mx_wgrad=args.mx_wgrad)
     elif w.stream_M:
         layer = B.MoEStream(w.T, w.d, w.E, w.I, w.k, w.stream_M, w.ring_bytes, w.first_local, w.num_local,
                             device=dev, wgrad_dtype=wdt)
@@ -660,7 +671,7 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     value = job_throughput(NT * args.steps, t, world)
     tflops = flops / t / 1e12
     per_gpu_tflops = tflops / world
-    algo = algorithmic_bytes(w, 4 if args.wgrad_fp32 else 2)
+    algo = algorithmic_bytes(w, 4 if args.wgrad_fp32 else 2, args.mx_wgrad)
     traffic_key = w.name + ("+wgrad_fp32" if args.wgrad_fp32 else "")  # counters were taken with bf16 gradients
     aflops = algorithmic_flops(w)
     if w.El < w.E:
@@ -758,6 +769,9 @@ def main():
                     help="write the expert weight gradients as fp32 instead of bf16 (the weights' dtype)")
     ap.add_argument("--launches", action="store_true",
                     help="run every grouped GEMM as its own launch instead of the persistent pairs")
+    ap.add_argument("--mx-wgrad", action="store_true",
+                    help="MXFP8 workloads: run the weight-gradient GEMMs on MXFP8 as well (operands quantised "
+                         "along each expert's rows) instead of on the bf16 operands")
     ap.add_argument("--persistent", action="store_true",
                     help="require the persistent pairs (the default for bf16 one-batch workloads): the forward's "
                          "gate/up and down GEMMs, and the backward's two dgrads, each pair as one persistent launch")
@@ -765,6 +779,8 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     w = IN.WORKLOADS[args.workload]
+    if args.mx_wgrad and not w.mxfp8:
+        ap.error("--mx-wgrad applies to the MXFP8 workloads; %s is bf16" % w.name)
     if args.launches and w.stream_M:
         ap.error("the ring-streamed layer always runs its GEMM pairs as persistent launches")
     if args.persistent and (w.mxfp8 or w.stream_M or args.launches):

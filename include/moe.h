@@ -57,8 +57,14 @@ typedef enum moe_status {
 
 typedef enum moe_precision {
   MOE_BF16 = 0,  /* bf16 operands, fp32 accumulation */
-  MOE_MXFP8 = 1  /* E4M3 operands with one E8M0 scale per 32 along each GEMM's contraction dim:
-                    use moe_prepare_weights + moe_fwd_mx / moe_bwd_mx (moe_fwd / moe_bwd refuse it) */
+  MOE_MXFP8 = 1,  /* E4M3 operands with one E8M0 scale per 32 along each GEMM's contraction dim:
+                     use moe_prepare_weights + moe_fwd_mx / moe_bwd_mx (moe_fwd / moe_bwd refuse it).
+                     The gate/up, down and both dgrad GEMMs are MXFP8; the weight-gradient GEMMs
+                     contract over tokens from the bf16 operands */
+  MOE_MXFP8_ALL = 2  /* MOE_MXFP8 with the two weight-gradient GEMMs on MXFP8 as well: their
+                        operands (X, dA, dB, Hg = g H and dY of each expert) quantised along the
+                        expert's rows, one scale per 32 rows from its first row, pad rows zero.
+                        Same entry points; a larger workspace (moe_workspace_size of this shape) */
 } moe_precision;
 
 typedef enum moe_wgrad_dtype {
@@ -216,9 +222,11 @@ unsigned long long moe_kernel_launches(void);
  * - 8; codes rounded to nearest even, saturating at +-448).  The gate/up and
  * down GEMMs and both dgrad GEMMs run on kind::mxf8f6f4 block-scaled tensor
  * cores with both operands quantised; the two weight-gradient GEMMs contract
- * over tokens and stay bf16.  The router stays bf16, so routing is the same in
- * both modes; all outputs are bf16 (dW_r fp32; the expert weight gradients
- * fp32 with wgrad_dtype = MOE_WGRAD_FP32).
+ * over tokens and stay bf16 (MOE_MXFP8), or (MOE_MXFP8_ALL) run on the same
+ * tensor cores with X, dA, dB, Hg and dY quantised along each expert's rows in
+ * blocks of 32 rows from its first row.  The router stays bf16, so routing is
+ * the same in every mode; all outputs are bf16 (dW_r fp32; the expert weight
+ * gradients fp32 with wgrad_dtype = MOE_WGRAD_FP32).
  *
  * moe_prepare_weights quantises the bf16 master weights once (e.g. after each
  * optimiser step) into `wq` (moe_weights_size bytes), laid out as ten regions,
@@ -233,8 +241,23 @@ unsigned long long moe_kernel_launches(void);
  * (r/128)*(K/128) + k/128 (the order the block-scaled MMA reads them in).
  * moe_fwd_mx / moe_bwd_mx take the same arguments as moe_fwd / moe_bwd with
  * wq in place of the bf16 expert weights; ctx and ws are sized by
- * moe_ctx_size / moe_workspace_size of the MXFP8 shape. */
+ * moe_ctx_size / moe_workspace_size of the MXFP8 shape (MOE_MXFP8 and
+ * MOE_MXFP8_ALL share ctx and prepared weights; the workspace differs). */
 size_t moe_weights_size(const moe_shape* shape);
+
+/* Test hook (MOE_MXFP8_ALL): copies one weight-gradient operand quantised along the
+ * rows by the last moe_fwd_mx (X_perm, saved in ctx) or moe_bwd_mx (in ws): which = 0
+ * X_perm, 1 dY_perm (C = d),
+ * 2 dA, 3 dB, 4 Hg (C = I).  RP = the padded-row capacity (moe_padded_rows).  codes
+ * (RP*C bytes) are K-major in 128-row tiles: byte ((R/128)*C + c)*128 + R%128 is the
+ * code of padded row R, column c; scales (RP*C/32 bytes) sit in 512-byte chunks,
+ * byte (c%32)*16 + ((c%128)/32)*4 + (R%128)/32 of chunk (R/128)*(C/128) + c/128.
+ * Tiles past an expert's real rows hold whatever the buffer held.  Device pointers;
+ * MOE_ERR_INVALID_ARG for another precision or `which`. */
+moe_status moe_debug_mx_wgrad_operand(const moe_shape* shape, const void* ctx, const void* ws, int32_t which,
+                                      void* codes, void* scales, void* stream);
+/* Padded-row capacity RP of a shape (rows of X_perm and the other row buffers); 0 if invalid. */
+int64_t moe_padded_rows(const moe_shape* shape);
 moe_status moe_prepare_weights(const moe_shape* shape, const void* W_gate, const void* W_up, const void* W_down,
                                void* wq, size_t wq_bytes, void* stream);
 moe_status moe_fwd_mx(const moe_shape* shape, const void* X, const void* W_r, const float* bias, const void* wq,

@@ -22,6 +22,7 @@ MOE_ERR_NONFINITE = 6
 MOE_ERR_EXCHANGE = 7
 MOE_BF16 = 0
 MOE_MXFP8 = 1
+MOE_MXFP8_ALL = 2  # MOE_MXFP8 with the weight-gradient GEMMs on MXFP8 too (operands along tokens)
 MOE_WGRAD_BF16 = 0
 MOE_WGRAD_FP32 = 1
 
@@ -112,6 +113,8 @@ _SIGS = {
     "moe_debug_routing": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_debug_logits": (ctypes.c_int, [_S, _P, _P, _P]),
     "moe_debug_router_grad": (ctypes.c_int, [_S, _P, _P, _P]),
+    "moe_debug_mx_wgrad_operand": (ctypes.c_int, [_S, _P, _P, ctypes.c_int32, _P, _P, _P]),
+    "moe_padded_rows": (ctypes.c_int64, [_S]),
     "moe_debug_bounded_wait": (ctypes.c_int, [_S, _P, ctypes.c_size_t, _P]),
     "moe_debug_pair_wait": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, ctypes.c_size_t,
                                            _P]),
@@ -250,6 +253,15 @@ def moe_debug_bounded_wait(shape, ctx, stream=None) -> int:
     return int(lib().moe_debug_bounded_wait(ctypes.byref(shape), _ptr(ctx), _nbytes(ctx), _stream(stream)))
 
 
+def moe_debug_mx_wgrad_operand(shape, ctx, ws, which, codes, scales, stream=None) -> int:
+    return int(lib().moe_debug_mx_wgrad_operand(ctypes.byref(shape), _ptr(ctx), _ptr(ws), int(which), _ptr(codes),
+                                                _ptr(scales), _stream(stream)))
+
+
+def moe_padded_rows(shape) -> int:
+    return int(lib().moe_padded_rows(ctypes.byref(shape)))
+
+
 def moe_debug_router_grad(shape, ws, dl, stream=None) -> int:
     return int(lib().moe_debug_router_grad(ctypes.byref(shape), _ptr(ws), _ptr(dl), _stream(stream)))
 
@@ -338,14 +350,18 @@ def check(status: int, what: str = "moe"):
 
 
 class MoELayerMX:
-    """MXFP8 layer: prepared (quantised) weights + ctx / workspace owner."""
+    """MXFP8 layer: prepared (quantised) weights + ctx / workspace owner.
+
+    mx_wgrad: the weight-gradient GEMMs on MXFP8 as well (MOE_MXFP8_ALL), their operands
+    quantised along each expert's rows; otherwise they contract the bf16 operands."""
 
     def __init__(self, T, d, E, I, top_k, first_local_expert=0, num_local_experts=0, device="cuda",
-                 wgrad_dtype=None):
+                 wgrad_dtype=None, mx_wgrad=False):
         import torch
         self.wgrad_dtype = wgrad_dtype or torch.bfloat16
-        self.shape = make_shape(T, d, E, I, top_k, MOE_MXFP8, first_local_expert, num_local_experts,
-                                _wgrad_code(self.wgrad_dtype))
+        self.mx_wgrad = bool(mx_wgrad)
+        self.shape = make_shape(T, d, E, I, top_k, MOE_MXFP8_ALL if mx_wgrad else MOE_MXFP8, first_local_expert,
+                                num_local_experts, _wgrad_code(self.wgrad_dtype))
         self.shape_bf16 = make_shape(T, d, E, I, top_k, MOE_BF16, first_local_expert, num_local_experts)
         nc, nw, nq = moe_ctx_size(self.shape), moe_workspace_size(self.shape), moe_weights_size(self.shape)
         if nc == 0 or nw == 0 or nq == 0:
@@ -376,6 +392,27 @@ class MoELayerMX:
         check(moe_bwd_mx(self.shape, X, W_r, self.wq, dY, self.ctx, out["dX"], out["dW_gate"], out["dW_up"],
                          out["dW_down"], out["dW_r"], self.ws, stream), "moe_bwd_mx")
         return out
+
+    def wgrad_operand(self, which):
+        """(codes [C, RP], scale bytes [C, RP / 32]) of weight-gradient operand `which` (0 X_perm,
+        1 dY_perm, 2 dA, 3 dB, 4 Hg) from the last backward, as host numpy arrays, column c's codes
+        and scales along the padded rows (MOE_MXFP8_ALL only; reordered here from the device's
+        128-row-tile layout)."""
+        import numpy as np
+        import torch
+        RP = moe_padded_rows(self.shape)
+        C = self.d if which < 2 else self.I
+        codes = torch.empty(C * RP, dtype=torch.uint8, device=self.ws.device)
+        scales = torch.empty(C * RP // 32, dtype=torch.uint8, device=self.ws.device)
+        check(moe_debug_mx_wgrad_operand(self.shape, self.ctx, self.ws, which, codes, scales),
+              "moe_debug_mx_wgrad_operand")
+        torch.cuda.synchronize()
+        q = codes.cpu().numpy().reshape(RP // 128, C, 128).transpose(1, 0, 2).reshape(C, RP)
+        ch = scales.cpu().numpy()
+        c = np.arange(C)[:, None]
+        kb = np.arange(RP // 32)[None, :]
+        idx = ((kb // 4) * (C // 128) + c // 128) * 512 + (c % 32) * 16 + ((c % 128) // 32) * 4 + kb % 4
+        return q, ch[idx]
 
     def weight_regions(self):
         """Host numpy views (codes [R, K], scale chunks) of the five prepared weights."""

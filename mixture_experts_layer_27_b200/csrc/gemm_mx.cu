@@ -14,6 +14,14 @@
 // epilogue drains it).  The dgrad of W_down, whose epilogue reads A and B and
 // writes five outputs, uses 128 x 128 tiles with two accumulators instead, so
 // its epilogue overlaps the next tile's MMAs.
+//
+// The weight-gradient GEMMs contract over an expert's rows: their operands are
+// quantised along the rows (k_quant_rows) and stored transposed, so they too are
+// K-major; a tile is 128 weight rows x 256 weight columns of one expert, K the
+// expert's real rows in 128-row stages (the last stage issues only the K = 32
+// steps that hold real rows).  Their epilogue moves the accumulator to registers,
+// releases it at once, and writes the gradient through shared memory with TMA
+// box stores.
 #include "moe_internal.cuh"
 #include "ptx.cuh"
 
@@ -21,13 +29,20 @@ namespace moe {
 
 struct MxTile {
   int el, m0, n0, nt, nk;
+  int r0, rows;  // weight-gradient kinds: the expert's first padded row and its real rows
 };
 
 template <int KIND>
 __device__ __forceinline__ int mx_ntiles_n(const MxParams& p) {
   if (KIND == MX_GATEUP) return p.I / (mx_bn(KIND) / 2);  // per tile: [64 gate | 64 up] column pairs
   if (KIND == MX_DGRAD_DOWN) return p.I / mx_bn(KIND);
-  return p.d / mx_bn(KIND);  // MX_DOWN, MX_DGRAD_GATEUP
+  if (KIND == MX_WGRAD_GATEUP) return 2 * p.I / 256;  // gate n-tiles, then up n-tiles
+  return p.d / mx_bn(KIND);  // MX_DOWN, MX_DGRAD_GATEUP, MX_WGRAD_DOWN
+}
+// weight-gradient kinds: 128-row tiles of the gradient (rows of d for gate/up, of I for down)
+template <int KIND>
+__device__ __forceinline__ int mx_mtiles_w(const MxParams& p) {
+  return KIND == MX_WGRAD_GATEUP ? p.d / 128 : p.I / 128;
 }
 template <int KIND>
 __device__ __forceinline__ int mx_kblocks(const MxParams& p) {
@@ -47,12 +62,29 @@ __device__ __forceinline__ int mx_segment_of_row(const int* poff, int nseg, int 
 
 template <int KIND>
 __device__ __forceinline__ int mx_num_tiles(const MxParams& p) {
+  if constexpr (mx_is_wgrad(KIND)) return p.El * mx_mtiles_w<KIND>(p) * mx_ntiles_n<KIND>(p);
   return ((__ldg(p.poff + p.nseg) - __ldg(p.poff)) / 128) * mx_ntiles_n<KIND>(p);
 }
 
 template <int KIND>
 __device__ __forceinline__ MxTile mx_decode(const MxParams& p, int t) {
   const int NT = mx_ntiles_n<KIND>(p);
+  if constexpr (mx_is_wgrad(KIND)) {
+    // per expert, m-tile major and n-tile minor: CTAs that run at the same time write adjacent
+    // column blocks of the same gradient rows
+    const int tpe = mx_mtiles_w<KIND>(p) * NT;
+    const int el = t / tpe, local = t - el * tpe;
+    const int mt = local / NT;
+    MxTile tl;
+    tl.el = el;
+    tl.m0 = mt * 128;
+    tl.nt = local - mt * NT;
+    tl.n0 = tl.nt * 256;
+    tl.r0 = __ldg(p.poff + el);
+    tl.rows = __ldg(p.cnt + el);
+    tl.nk = (tl.rows + 127) / 128;
+    return tl;
+  }
   const int base = __ldg(p.poff);
   const int seg = mx_segment_of_row(p.poff, p.nseg, base + (t / NT) * 128);
   const int p0 = __ldg(p.poff + seg), p1 = __ldg(p.poff + seg + 1);
@@ -80,6 +112,28 @@ __device__ __forceinline__ void mx_load(const MxParams& p, const MxTile& tl, int
   const CUtensorMap* mb = &p.tb0;
   const uint8_t* sfa = p.sfa0;
   const uint8_t* sfb = p.sfb0;
+  if constexpr (mx_is_wgrad(KIND)) {
+    // K block kb = row tile kt = (r0 + 128 kb) / 128 of both operands (rowq layout): A = lines
+    // kt CA + m0 .., B = lines kt CB + nb .. of 128 codes, and the tile's scale chunks
+    const size_t kt = static_cast<size_t>((tl.r0 >> 7) + kb);
+    const int CA = KIND == MX_WGRAD_GATEUP ? p.d : p.I, CB = KIND == MX_WGRAD_GATEUP ? p.I : p.d;
+    int nb = tl.n0;
+    if constexpr (KIND == MX_WGRAD_GATEUP) {
+      const int NTg = p.I / 256;
+      if (tl.nt >= NTg) {  // dW_up: Xq with dBq
+        nb = (tl.nt - NTg) * 256;
+        mb = &p.tb1;
+        sfb = p.sfb1;
+      }
+    }
+    tma_load_2d(sA, ma, bar, 0, static_cast<int>(kt * CA) + tl.m0, pol_act);
+    tma_load_2d(sB, mb, bar, 0, static_cast<int>(kt * CB) + nb, pol_act);
+    bulk_load(sSF, sfa + (kt * (CA >> 7) + (tl.m0 >> 7)) * 512, 512, bar);
+    bulk_load(sSF + 512, sfb + (kt * (CB >> 7) + (nb >> 7)) * 512, 512, bar);
+    bulk_load(sSF + 1024, sfb + (kt * (CB >> 7) + (nb >> 7) + 1) * 512, 512, bar);
+    (void)pol_w;
+    return;
+  }
   int kl = kb, brow, KA, KB;
   if constexpr (KIND == MX_GATEUP) {
     brow = tl.el * 2 * p.I + tl.nt * BN;  // blocks of paired [64 gate | 64 up] rows of the prepared weight
@@ -145,13 +199,37 @@ __device__ __forceinline__ void mx_store_q32(uint8_t* q, uint8_t* qs, int R, int
   qs[sf_index(R, c0, K)] = sb;
 }
 
+// The warp's 32 rows (one 32-row block of one expert: tiles start on multiples of 128) x 32
+// columns quantised along the rows for the MXFP8 weight gradients: the fp32 values go through
+// the warp's shared-memory slice (32 x 33 words: row writes and column reads both hit 32
+// distinct banks), lane i reads column col + i's 32 values, quantises them as one block
+// (mx_quant32) and stores their 32 codes in the K-major, 128-row-tile-major operand q
+// (rowq_index; C = I columns) and the scale byte.  v holds 0 for pad rows.
+constexpr int MX_TPITCH = 33;
+__device__ __forceinline__ void mx_store_rows_q32(uint8_t* q, uint8_t* qs, int R0, int col, int C,
+                                                  const float (&v)[32], int lane, float* scratch) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) scratch[lane * MX_TPITCH + i] = v[i];
+  __syncwarp();
+  float c[32];
+#pragma unroll
+  for (int r = 0; r < 32; ++r) c[r] = scratch[r * MX_TPITCH + lane];
+  __syncwarp();  // every lane has read the block before the next one is written
+  uint32_t w[8];
+  const uint8_t sb = mx_quant32(c, w);
+  uint4* d = reinterpret_cast<uint4*>(q + rowq_index(col + lane, R0, C));
+  d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  qs[rowq_sf_index(col + lane, R0, C)] = sb;
+}
+
 // Rows past a segment's live pad rows (row_asg == ROW_DEAD) store nothing: no later kernel
 // reads them.
 // [cbeg, cend): this warp's share of the accumulator's 32-column chunks (all of them, or half
 // when two warps share a TMEM lane quarter).
 template <int KIND>
 __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl, int row, uint32_t taddr, int cbeg,
-                                            int cend) {
+                                            int cend, float* scratch) {
   const int R = tl.m0 + row;
   const size_t Rz = static_cast<size_t>(R);
   const bool live = __ldg(p.row_asg + R) != ROW_DEAD;
@@ -209,11 +287,27 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
         dh[i] = g * hh;                                        // Hg
       }
       if (live) {
-        mx_store_bf16_32(p.out0 + Rz * p.I + col, a);
-        mx_store_bf16_32(p.out1 + Rz * p.I + col, b);
-        mx_store_bf16_32(p.out2 + Rz * p.I + col, dh);
+        if (p.out0) {  // bf16 operands of the bf16 weight gradients
+          mx_store_bf16_32(p.out0 + Rz * p.I + col, a);
+          mx_store_bf16_32(p.out1 + Rz * p.I + col, b);
+          mx_store_bf16_32(p.out2 + Rz * p.I + col, dh);
+        }
         mx_store_q32(p.q0, p.qs0, R, col, p.I, a);  // dA, dB: the gate/up dgrad's A operands (K = I)
         mx_store_q32(p.q1, p.qs1, R, col, p.I, b);
+      }
+      const int R0 = tl.m0 + (row & ~31);
+      // MXFP8 weight gradients: dA, dB, Hg along the rows (warp-collective); a 32-row block that
+      // starts past the expert's real rows is never read by the GEMM
+      if (p.tq[0] && __ldg(p.row_asg + R0) >= 0) {
+        const bool real = __ldg(p.row_asg + R) >= 0;
+        const int lane = row & 31;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (!real) a[i] = b[i] = dh[i] = 0.f;
+        }
+        mx_store_rows_q32(p.tq[0], p.tqs[0], R0, col, p.I, a, lane, scratch);
+        mx_store_rows_q32(p.tq[1], p.tqs[1], R0, col, p.I, b, lane, scratch);
+        mx_store_rows_q32(p.tq[2], p.tqs[2], R0, col, p.I, dh, lane, scratch);
       }
     }
     if (live) p.outf[Rz * (p.I / BN) + tl.nt] = dg;
@@ -223,6 +317,89 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
       float v[32];
       tmem_ld32(taddr + c * 32, v);
       if (live) mx_store_bf16_32(p.out0 + Rz * p.d + tl.n0 + c * 32, v);
+    }
+  }
+}
+
+// Weight-gradient epilogue of one warp: its 32 gradient rows (TMEM lane quarter) x 128 columns
+// (half of the 256-wide tile).  The accumulator slice goes to registers first and the warp
+// releases it (acc_empty) before any store, so the next tile's MMAs run while the gradient is
+// written: bf16 as two 64 x 32 boxes, or fp32 (wout32) as four 32 x 32 boxes, each staged in
+// one of the warp's two 4 KB slots (128-byte swizzle, as the output maps expect) and written by
+// a TMA store; a slot is refilled once the store issued from it has read it.  An expert without
+// rows has a zero gradient.
+__device__ __forceinline__ void mx_stage16(uint8_t* box, int lane, int chunk, uint4 u) {
+  *reinterpret_cast<uint4*>(box + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = u;
+}
+
+template <int KIND>
+__device__ __forceinline__ void mx_epilogue_wgrad(const MxParams& p, const MxTile& tl, int quarter, int half,
+                                                  int lane, uint32_t taddr, uint8_t* stage_out,
+                                                  uint64_t* acc_empty) {
+  int x0, y0;
+  const CUtensorMap* map = &p.to0;
+  if constexpr (KIND == MX_WGRAD_GATEUP) {
+    const int NTg = p.I / 256;
+    const bool up = tl.nt >= NTg;  // dW_gate or dW_up as [El*d, I]
+    if (up) map = &p.to1;
+    x0 = (up ? tl.nt - NTg : tl.nt) * 256 + half * 128;
+    y0 = tl.el * p.d + tl.m0 + quarter * 32;
+  } else {
+    x0 = tl.n0 + half * 128;  // dW_down as [El*I, d]
+    y0 = tl.el * p.I + tl.m0 + quarter * 32;
+  }
+  uint32_t r[2][64];
+  if (tl.nk > 0) {
+    tmem_ld64_issue(taddr, r[0]);
+    tmem_ld64_issue(taddr + 64, r[1]);
+    tmem_ld64_wait(r[0]);
+    tmem_ld64_wait(r[1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) r[0][i] = r[1][i] = 0u;
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(acc_empty);
+  if (!p.wout32) {
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      if (lane == 0) bulk_wait_read<1>();
+      __syncwarp();
+      uint8_t* box = stage_out + b * 4096;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t* w = r[b] + 8 * q;
+        mx_stage16(box, lane, q,
+                   make_uint4(pack_bf16(__uint_as_float(w[0]), __uint_as_float(w[1])),
+                              pack_bf16(__uint_as_float(w[2]), __uint_as_float(w[3])),
+                              pack_bf16(__uint_as_float(w[4]), __uint_as_float(w[5])),
+                              pack_bf16(__uint_as_float(w[6]), __uint_as_float(w[7]))));
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(map, box, x0 + b * 64, y0);
+        bulk_commit();
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (lane == 0) bulk_wait_read<1>();
+      __syncwarp();
+      uint8_t* box = stage_out + (j & 1) * 4096;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t* w = r[j >> 1] + (j & 1) * 32 + 4 * q;
+        mx_stage16(box, lane, q, make_uint4(w[0], w[1], w[2], w[3]));
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(map, box, x0 + j * 32, y0);
+        bulk_commit();
+      }
     }
   }
 }
@@ -240,7 +417,8 @@ __global__ void __launch_bounds__(mx_threads(KIND), 1) k_moe_gemm_mx(const __gri
   constexpr size_t SB = mx_stage_bytes(KIND);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * SB);
+  uint8_t* stage_out = smem + STAGES * SB;  // weight-gradient kinds: 8 KB per epilogue warp; dgrad of W_down: 1 KB
+  uint64_t* full = reinterpret_cast<uint64_t*>(stage_out + mx_out_bytes(KIND));
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;  // per accumulator
   uint64_t* tempty = tfull + ACCS;
@@ -323,15 +501,24 @@ __global__ void __launch_bounds__(mx_threads(KIND), 1) k_moe_gemm_mx(const __gri
           tc_cp_sf(sfa_t, sf0);
           tc_cp_sf(sfb_t, sf0 + 512);
           if constexpr (BN == 256) tc_cp_sf(sfb_t + 4, sf0 + 1024);
+          // weight gradients: the last 128-row block issues only the K = 32 steps with real rows
+          // (its rows past them up to the next multiple of 32 are zero codes)
+          int nkk = 4;
+          if constexpr (mx_is_wgrad(KIND)) {
+            const int valid = tl.rows - kb * 128;
+            if (valid < 128) nkk = (valid + 31) / 32;
+          }
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_mxf8(dtm, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024),
-                      idesc_mxf8(128, BN, static_cast<uint32_t>(kk)), sfa_t, sfb_t, (kb | kk) != 0 ? 1u : 0u);
+            if (kk < nkk)
+              umma_mxf8(dtm, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024),
+                        idesc_mxf8(128, BN, static_cast<uint32_t>(kk)), sfa_t, sfb_t, (kb | kk) != 0 ? 1u : 0u);
           umma_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        if (tl.nk > 0) umma_commit(&tfull[acc]);
+        else mbar_arrive(&tfull[acc]);  // an expert without rows: nothing to wait for
       }
       umma_commit(drain);
       mx_wait_drain(drain, 0);
@@ -353,10 +540,21 @@ __global__ void __launch_bounds__(mx_threads(KIND), 1) k_moe_gemm_mx(const __gri
       if (!ok) break;
       __syncwarp();
       tc_fence_after();
-      mx_epilogue<KIND>(p, tl, row, tbase + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN, cbeg, cend);
+      const uint32_t taddr = tbase + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
+      if constexpr (mx_is_wgrad(KIND)) {  // releases the accumulator itself, before its stores
+        mx_epilogue_wgrad<KIND>(p, tl, quarter, half, lane, taddr + half * 128, stage_out + (warp - 2) * 8192,
+                                &tempty[acc]);
+        continue;
+      }
+      mx_epilogue<KIND>(p, tl, row, taddr, cbeg, cend,
+                        reinterpret_cast<float*>(stage_out) + (KIND == MX_DGRAD_DOWN ? (warp - 2) * 32 * MX_TPITCH : 0));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+    if constexpr (mx_is_wgrad(KIND)) {
+      if (lane == 0) bulk_wait0();  // stores complete before the CTA (and its smem) goes away
+      __syncwarp();
     }
   }
   __syncthreads();
@@ -388,6 +586,8 @@ cudaError_t launch_gemm_mx(MxKind kind, const MxParams& p, int grid, cudaStream_
     case MX_DOWN: return mx_launch_kind<MX_DOWN>(p, grid, st);
     case MX_DGRAD_DOWN: return mx_launch_kind<MX_DGRAD_DOWN>(p, grid, st);
     case MX_DGRAD_GATEUP: return mx_launch_kind<MX_DGRAD_GATEUP>(p, grid, st);
+    case MX_WGRAD_GATEUP: return mx_launch_kind<MX_WGRAD_GATEUP>(p, grid, st);
+    case MX_WGRAD_DOWN: return mx_launch_kind<MX_WGRAD_DOWN>(p, grid, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -54,6 +54,10 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
     o = align_up(o + bytes, 256);
     return at;
   };
+  L->mx = s.prec == MOE_MXFP8 || s.prec == MOE_MXFP8_ALL;
+  L->mxw = s.prec == MOE_MXFP8_ALL;
+  // row-quantised operands are addressed by TMA as RP / 128 * C lines (a signed 32-bit coordinate)
+  if (L->mxw && (L->RP / 128) * static_cast<int64_t>(s.d > s.I ? s.d : s.I) >= (int64_t(1) << 31)) return false;
   L->hdr = take(HDR_WORDS * 4);
   L->ids = take(T * k * 4);
   L->gates = take(T * k * 4);
@@ -65,14 +69,17 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->slot_row = take(T * k * 4);
   L->row_asg = take(RP * 4);
   L->row_gate = take(RP * 4);
-  L->xperm = take(M > 0 ? 0 : RP * s.d * 2);  // streamed layer: X_perm lives in the caller's ring
+  // streamed layer: X_perm lives in the caller's ring; MXFP8 weight gradients keep X quantised instead
+  L->xperm = take(M > 0 || s.prec == MOE_MXFP8_ALL ? 0 : RP * s.d * 2);
   L->abuf = take(RP * s.I * 2);
   L->bbuf = take(RP * s.I * 2);
   L->stab = take(M > 0 ? static_cast<size_t>(stream_table_words(M, El)) * 4 : 0);
-  L->mx = s.prec == MOE_MXFP8;
   const size_t mxd = L->mx ? RP * s.d : 0, mxi = L->mx ? RP * s.I : 0;  // fp8 bytes; scales are 1/32 of that
   L->xq = take(mxd);
   L->xqs = take(mxd / 32);
+  const size_t wxd = L->mxw ? RP * s.d : 0, wxi = L->mxw ? RP * s.I : 0;
+  L->xqt = take(wxd);  // X along the rows, from the forward's dispatch for the weight gradients
+  L->xqts = take(wxd / 32);
   L->ctx_bytes = o;
 
   o = 0;
@@ -105,6 +112,14 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->dbq = take(mxi);
   L->dbqs = take(mxi / 32);
   L->fctl = take(L->mx ? 0 : static_cast<size_t>(gemm_pair_ctl_words(L->RP)) * 4);
+  L->dyqt = take(wxd);
+  L->dyqts = take(wxd / 32);
+  L->daqt = take(wxi);
+  L->daqts = take(wxi / 32);
+  L->dbqt = take(wxi);
+  L->dbqts = take(wxi / 32);
+  L->hgqt = take(wxi);
+  L->hgqts = take(wxi / 32);
   L->ws_bytes = o;
   // prepared weights: [W_gate|W_up paired, K = d] [W_down^T, K = I] [W_down, K = d] [W_gate, K = I] [W_up, K = I]
   o = 0;
@@ -163,6 +178,21 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
   c.xq = L.mx ? reinterpret_cast<uint8_t*>(C(L.xq)) : nullptr;
   c.xqs = L.mx ? reinterpret_cast<uint8_t*>(C(L.xqs)) : nullptr;
   c.hq = c.hqs = c.dyq = c.dyqs = c.daq = c.daqs = c.dbq = c.dbqs = nullptr;
+  c.xqt = c.xqts = c.dyqt = c.dyqts = c.daqt = c.daqts = c.dbqt = c.dbqts = c.hgqt = c.hgqts = nullptr;
+  if (L.mxw) {
+    c.xqt = reinterpret_cast<uint8_t*>(C(L.xqt));
+    c.xqts = reinterpret_cast<uint8_t*>(C(L.xqts));
+  }
+  if (ws && L.mxw) {
+    c.dyqt = reinterpret_cast<uint8_t*>(W(L.dyqt));
+    c.dyqts = reinterpret_cast<uint8_t*>(W(L.dyqts));
+    c.daqt = reinterpret_cast<uint8_t*>(W(L.daqt));
+    c.daqts = reinterpret_cast<uint8_t*>(W(L.daqts));
+    c.dbqt = reinterpret_cast<uint8_t*>(W(L.dbqt));
+    c.dbqts = reinterpret_cast<uint8_t*>(W(L.dbqts));
+    c.hgqt = reinterpret_cast<uint8_t*>(W(L.hgqt));
+    c.hgqts = reinterpret_cast<uint8_t*>(W(L.hgqts));
+  }
   if (ws && L.mx) {
     c.hq = reinterpret_cast<uint8_t*>(W(L.hq));
     c.hqs = reinterpret_cast<uint8_t*>(W(L.hqs));
@@ -286,7 +316,7 @@ enum KernelId {
   K_ROUTER_LOGITS, K_TOPK, K_SCAN, K_SCATTER, K_DISPATCH, K_GEMM_GATEUP, K_GEMM_DOWN, K_COMBINE,
   K_REV_COMBINE, K_GEMM_DGRAD_DOWN, K_ROUTER_BWD, K_ROUTER_WGRAD, K_TRANSPOSE_WR, K_GEMM_DGRAD_GATEUP, K_REV_DISPATCH,
   K_GEMM_WGRAD_GATEUP, K_GEMM_WGRAD_DOWN, K_PLAN, K_REPLAY, K_FINISH_ACC, K_QUANT_WEIGHTS, K_MARK_ROWS,
-  K_ACTIVE_COUNT, K_GATHER_ACTIVE, K_SCAN_GROUPS, K_SCAN_APPLY, K_PAIR_FWD, K_PAIR_DGRAD, K_NUM
+  K_ACTIVE_COUNT, K_GATHER_ACTIVE, K_SCAN_GROUPS, K_SCAN_APPLY, K_PAIR_FWD, K_PAIR_DGRAD, K_MX_WGRAD_GATEUP, K_MX_WGRAD_DOWN, K_NUM
 };
 static const char* kKernelNames[K_NUM] = {
     "router_logits", "topk_gating", "hist_scan", "stable_scatter", "dispatch", "gemm_gateup_swiglu",
@@ -294,7 +324,7 @@ static const char* kKernelNames[K_NUM] = {
     "transpose_wr", "gemm_dgrad_gateup", "reverse_dispatch", "gemm_wgrad_gateup", "gemm_wgrad_down",
     "stream_plan", "ring_replay", "wgrad_accumulator_finish", "quantize_weights", "mark_pad_rows",
     "router_token_count", "router_token_gather", "hist_scan_group_sums", "hist_scan_group_apply",
-    "gemm_gateup_down_persistent", "gemm_dgrads_persistent"};
+    "gemm_gateup_down_persistent", "gemm_dgrads_persistent", "gemm_wgrad_gateup_mx", "gemm_wgrad_down_mx"};
 
 struct ProfRec {
   int kid;
@@ -453,9 +483,11 @@ const char* moe_status_string(moe_status st) {
   return "unknown status";
 }
 
+static bool is_mx_prec(int32_t prec) { return prec == MOE_MXFP8 || prec == MOE_MXFP8_ALL; }
+
 static moe_status check_shape_mx(const moe_shape* s, Layout* L) {
   if (!s) return MOE_ERR_INVALID_ARG;
-  if (s->prec != MOE_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (!is_mx_prec(s->prec)) return MOE_ERR_INVALID_ARG;
   if (s->T < 0 || s->d <= 0 || s->E <= 0 || s->I <= 0 || s->top_k <= 0 || s->first_local_expert < 0 ||
       s->num_local_experts < 0)
     return MOE_ERR_INVALID_ARG;
@@ -468,8 +500,8 @@ static moe_status check_shape(const moe_shape* s, Layout* L) {
   if (s->T < 0 || s->d <= 0 || s->E <= 0 || s->I <= 0 || s->top_k <= 0 || s->first_local_expert < 0 ||
       s->num_local_experts < 0)
     return MOE_ERR_INVALID_ARG;
-  if (s->prec != MOE_BF16 && s->prec != MOE_MXFP8) return MOE_ERR_INVALID_ARG;
-  if (s->prec == MOE_MXFP8) return MOE_ERR_UNSUPPORTED;
+  if (s->prec != MOE_BF16 && !is_mx_prec(s->prec)) return MOE_ERR_INVALID_ARG;
+  if (is_mx_prec(s->prec)) return MOE_ERR_UNSUPPORTED;
   if (!make_layout(*s, L)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -808,7 +840,7 @@ unsigned long long moe_kernel_launches(void) { return g_launches.load(); }
 // ---------------------------------------------------------------------------
 static moe_status check_stream(const moe_shape* s, int32_t M, Layout* L) {
   if (!s || M <= 0) return MOE_ERR_INVALID_ARG;
-  if (s->prec != MOE_BF16) return s->prec == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (s->prec != MOE_BF16) return is_mx_prec(s->prec) ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
   if (!make_layout(*s, L, M)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -1071,6 +1103,69 @@ static MxParams mx_params(const Layout& L, const Ctx& c, int* status) {
   return p;
 }
 
+// MXFP8 weight gradients from operands quantised along the rows (blocks of 32 rows of one expert,
+// K-major in 128-row tiles): X by the forward's dispatch, dY by the reverse-combine, dA, dB and Hg
+// by the dgrad of W_down from its fp32 values.  One grouped GEMM for gate/up and one for down;
+// gradients leave through TMA box stores (bf16, or fp32 with MOE_WGRAD_FP32).
+static moe_status launch_wgrads_mx(const Layout& L, const Ctx& c, int* status, void* dW_gate, void* dW_up,
+                                   void* dW_down, cudaStream_t st) {
+  const int grid = num_sms();
+  const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
+  {
+    MxParams p = mx_params(L, c, status);
+    // row-quantised operands, 128-row-tile-major: lines of 128 codes, RP / 128 tiles of d (or I) lines
+    MOE_TMAP(tmap_fp8(&p.ta0, c.xqt, 128, RP / 128 * L.d, 128));
+    MOE_TMAP(tmap_fp8(&p.tb0, c.daqt, 128, RP / 128 * L.I, 256));
+    MOE_TMAP(tmap_fp8(&p.tb1, c.dbqt, 128, RP / 128 * L.I, 256));
+    MOE_TMAP(tmap_wgrad_out(L, &p.to0, dW_gate, L.I, El * L.d));
+    MOE_TMAP(tmap_wgrad_out(L, &p.to1, dW_up, L.I, El * L.d));
+    p.ta1 = p.ta0;
+    p.sfa0 = p.sfa1 = c.xqts;
+    p.sfb0 = c.daqts;
+    p.sfb1 = c.dbqts;
+    p.cnt = c.counts + L.first;
+    p.wout32 = L.w32 ? 1 : 0;
+    MOE_TRY(timed(K_MX_WGRAD_GATEUP, st, [&] { return launch_gemm_mx(MX_WGRAD_GATEUP, p, grid, st); }));
+  }
+  {
+    MxParams p = mx_params(L, c, status);
+    MOE_TMAP(tmap_fp8(&p.ta0, c.hgqt, 128, RP / 128 * L.I, 128));
+    MOE_TMAP(tmap_fp8(&p.tb0, c.dyqt, 128, RP / 128 * L.d, 256));
+    MOE_TMAP(tmap_wgrad_out(L, &p.to0, dW_down, L.d, El * L.I));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.to1 = p.to0;
+    p.sfa0 = p.sfa1 = c.hgqts;
+    p.sfb0 = p.sfb1 = c.dyqts;
+    p.cnt = c.counts + L.first;
+    p.wout32 = L.w32 ? 1 : 0;
+    MOE_TRY(timed(K_MX_WGRAD_DOWN, st, [&] { return launch_gemm_mx(MX_WGRAD_DOWN, p, grid, st); }));
+  }
+  return MOE_OK;
+}
+
+moe_status moe_debug_mx_wgrad_operand(const moe_shape* s, const void* ctx, const void* ws, int32_t which,
+                                      void* codes, void* scales, void* stream) {
+  Layout L;
+  const moe_status cs = check_shape_mx(s, &L);
+  if (cs != MOE_OK) return cs;
+  if (!L.mxw || !ctx || !ws || !codes || !scales || which < 0 || which > 4) return MOE_ERR_INVALID_ARG;
+  const size_t off[5][2] = {{L.xqt, L.xqts}, {L.dyqt, L.dyqts}, {L.daqt, L.daqts}, {L.dbqt, L.dbqts},
+                            {L.hgqt, L.hgqts}};
+  const size_t n = static_cast<size_t>(L.RP) * (which < 2 ? L.d : L.I);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const char* w = static_cast<const char*>(which == 0 ? ctx : ws);  // X's codes are saved in ctx
+  MOE_TRY(cudaMemcpyAsync(codes, w + off[which][0], n, cudaMemcpyDeviceToDevice, st));
+  MOE_TRY(cudaMemcpyAsync(scales, w + off[which][1], n / 32, cudaMemcpyDeviceToDevice, st));
+  return MOE_OK;
+}
+
+int64_t moe_padded_rows(const moe_shape* s) {
+  Layout L;
+  if (!s || !make_layout(*s, &L)) return 0;
+  return L.RP;
+}
+
 moe_status moe_fwd_mx(const moe_shape* s, const void* X, const void* W_r, const float* bias, const void* wq,
                       size_t wq_bytes, void* Y, void* ctx, size_t ctx_bytes, void* ws, size_t ws_bytes,
                       void* stream) {
@@ -1092,6 +1187,8 @@ moe_status moe_fwd_mx(const moe_shape* s, const void* X, const void* W_r, const 
     if (r != MOE_OK) return r;
   }
   MOE_TRY(timed(K_DISPATCH, st, [&] {
+    if (L.mxw)  // along d for the gate/up GEMM and along the rows for the weight gradients
+      return launch_gather_quant2(L, c, static_cast<const __nv_bfloat16*>(X), c.xq, c.xqs, c.xqt, c.xqts, st);
     return launch_gather_rows_mx(L, c, static_cast<const __nv_bfloat16*>(X), c.xperm, c.xq, c.xqs, st);
   }));
   const int grid = num_sms();
@@ -1148,6 +1245,8 @@ moe_status moe_bwd_mx(const moe_shape* s, const void* X, const void* W_r, const 
   const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
   const auto* w = static_cast<const uint8_t*>(wq);
   MOE_TRY(timed(K_REV_COMBINE, st, [&] {
+    if (L.mxw)  // along d for the dgrad of W_down and along the rows for the weight gradients
+      return launch_gather_quant2(L, c, static_cast<const __nv_bfloat16*>(dY), c.dyq, c.dyqs, c.dyqt, c.dyqts, st);
     return launch_gather_rows_mx(L, c, static_cast<const __nv_bfloat16*>(dY), c.dyperm, c.dyq, c.dyqs, st);
   }));
   {
@@ -1160,9 +1259,18 @@ moe_status moe_bwd_mx(const moe_shape* s, const void* X, const void* W_r, const 
     p.sfb0 = p.sfb1 = w + L.wd3s;
     p.in0 = c.abuf;
     p.in1 = c.bbuf;
-    p.out0 = c.dabuf;
-    p.out1 = c.dbbuf;
-    p.out2 = c.hgbuf;
+    if (L.mxw) {  // dA, dB, Hg quantised along the rows here, from fp32, for the MXFP8 weight gradients
+      p.tq[0] = c.daqt;
+      p.tq[1] = c.dbqt;
+      p.tq[2] = c.hgqt;
+      p.tqs[0] = c.daqts;
+      p.tqs[1] = c.dbqts;
+      p.tqs[2] = c.hgqts;
+      } else {  // bf16 operands of the bf16 weight gradients
+      p.out0 = c.dabuf;
+      p.out1 = c.dbbuf;
+      p.out2 = c.hgbuf;
+    }
     p.q0 = c.daq;
     p.qs0 = c.daqs;
     p.q1 = c.dbq;
@@ -1188,8 +1296,10 @@ moe_status moe_bwd_mx(const moe_shape* s, const void* X, const void* W_r, const 
     MOE_TRY(timed(K_GEMM_DGRAD_GATEUP, st, [&] { return launch_gemm_mx(MX_DGRAD_GATEUP, p, grid, st); }));
   }
   MOE_TRY(timed(K_REV_DISPATCH, st, [&] { return launch_rev_dispatch(L, c, static_cast<__nv_bfloat16*>(dX), st); }));
-  // weight gradients contract over tokens from the bf16 operands: the bf16 engine
-  return launch_wgrads(L, c, status, dW_gate, dW_up, dW_down, st);
+  // weight gradients contract over tokens: from the bf16 operands on the bf16 engine, or
+  // (MOE_MXFP8_ALL) on MXFP8 from the operands quantised along the rows
+  if (!L.mxw) return launch_wgrads(L, c, status, dW_gate, dW_up, dW_down, st);
+  return launch_wgrads_mx(L, c, status, dW_gate, dW_up, dW_down, st);
 }
 
 moe_status moe_get_error(void* ctx, void* stream) {
@@ -1279,7 +1389,7 @@ struct EpSetup {
 
 moe_status ep_setup(const moe_shape* s, int32_t R, int32_t rank, EpSetup* S) {
   if (!s) return MOE_ERR_INVALID_ARG;
-  if (s->prec != MOE_BF16) return s->prec == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (s->prec != MOE_BF16) return is_mx_prec(s->prec) ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
   if (R < 1 || R > kEpMaxRanks || rank < 0 || rank >= R || s->E <= 0 || s->E % R) return MOE_ERR_INVALID_ARG;
   if (s->T < 0 || s->T * static_cast<int64_t>(R) * s->top_k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
   const int El = s->E / R;

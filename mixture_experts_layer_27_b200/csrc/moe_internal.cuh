@@ -70,7 +70,11 @@ struct Layout {
   // ws
   size_t hist, hsum, logits, rpart, hbuf, obuf, dyperm, dabuf, dbbuf, hgbuf, dgpart, dlasg, dldense, wrt, dxperm, acc32, hq, hqs, dyq,
       dyqs, daq, daqs, dbq, dbqs, actcnt, actlist, xact, fctl, ws_bytes;
+  // MXFP8 weight gradients: X, dY, dA, dB, Hg quantised along the rows, K-major in 128-row tiles
+  // (rowq_index in ptx.cuh) with their scale chunks
+  size_t xqt, xqts, dyqt, dyqts, daqt, daqts, dbqt, dbqts, hgqt, hgqts;
   bool mx;   // MXFP8 mode
+  bool mxw;  // MXFP8 mode with the weight-gradient GEMMs on MXFP8 as well
   bool w32;  // expert weight gradients written as fp32
   bool rslice;  // an expert slice (El < E): the router weight gradient runs over the listed tokens
   // prepared MXFP8 weights (moe_prepare_weights): fp8 codes and scale chunks
@@ -192,6 +196,8 @@ enum MxKind {
   MX_DOWN = 1,          // O' = g * (Hq . Wd_q)
   MX_DGRAD_DOWN = 2,    // dH' = dYq . Wd_q^T; SwiGLU backward; dA, dB quantised in the epilogue
   MX_DGRAD_GATEUP = 3,  // dX_perm = dAq . Wg_q^T + dBq . Wu_q^T
+  MX_WGRAD_GATEUP = 4,  // dW_gate = Xq^T dAq, dW_up = Xq^T dBq per expert, all quantised along its rows
+  MX_WGRAD_DOWN = 5,    // dW_down = Hgq^T dYq per expert
 };
 struct MxParams {
   CUtensorMap ta0, ta1, tb0, tb1;  // fp8 K-major operands, box {128 bytes of K, 128 rows (A) / mx_bn rows (B)}
@@ -215,7 +221,19 @@ struct MxParams {
   float* outf;
   int El, d, I;
   int* status;
+  // weight-gradient kinds: operands quantised along the rows (K = rows; rowq layout), the
+  // real row count of each local expert, and the gradient outputs as TMA store maps (bf16
+  // 64 x 32 boxes, or fp32 32 x 32 boxes with wout32)
+  CUtensorMap to0, to1;
+  const int* cnt;
+  int wout32;
+  // dgrad of W_down with MXFP8 weight gradients: dA, dB and Hg also quantised along the rows,
+  // from the fp32 epilogue values, into the rowq layout (C = I) and its scale chunks (the
+  // bf16 dA, dB, Hg are then not written: out0..out2 NULL)
+  uint8_t* tq[3];
+  uint8_t* tqs[3];
 };
+__host__ __device__ constexpr bool mx_is_wgrad(int kind) { return kind == MX_WGRAD_GATEUP || kind == MX_WGRAD_DOWN; }
 // Tile width per kind: 128 x 256 tiles (one accumulator, four stages) keep 32 KB of fp8 weights
 // per stage in flight; the dgrad of W_down, whose epilogue reads and writes the most, keeps
 // 128 x 128 tiles with two accumulators (six stages) so that its epilogue overlaps the MMAs.
@@ -223,7 +241,7 @@ struct MxParams {
 // B scale chunks; stages start on 1 KB boundaries (128-byte swizzle atoms).
 __host__ __device__ constexpr int mx_bn(int kind) { return kind == MX_DGRAD_DOWN ? 128 : 256; }
 __host__ __device__ constexpr int mx_accs(int kind) { return mx_bn(kind) == 128 ? 2 : 1; }
-__host__ __device__ constexpr int mx_stages(int kind) { return mx_bn(kind) == 128 ? 6 : 4; }
+__host__ __device__ constexpr int mx_stages(int kind) { return mx_bn(kind) == 128 ? 6 : (mx_is_wgrad(kind) ? 3 : 4); }
 // Epilogue warps: with one accumulator the MMAs of the next tile wait for the epilogue, so it is
 // split over eight warps (two per TMEM lane quarter, each taking half of the columns); the
 // double-buffered 128 x 128 kind keeps four.
@@ -234,7 +252,15 @@ __host__ __device__ constexpr size_t mx_stage_tx(int kind) {  // bytes one stage
   return MX_A_BYTES + static_cast<size_t>(mx_bn(kind)) * 128 + 512 * (1 + mx_bn(kind) / 128);
 }
 __host__ __device__ constexpr size_t mx_stage_bytes(int kind) { return (mx_stage_tx(kind) + 1023) / 1024 * 1024; }
-__host__ __device__ constexpr size_t mx_smem_bytes(int kind) { return mx_stages(kind) * mx_stage_bytes(kind) + 1024 + 256; }
+// weight-gradient kinds: 8 KB per epilogue warp stages its two gradient boxes for the TMA stores;
+// the dgrad of W_down: 32 x 33 fp32 words per epilogue warp transpose its 32 x 32 value blocks
+constexpr size_t MX_STAGE_OUT_BYTES = 8 * 8192;
+__host__ __device__ constexpr size_t mx_out_bytes(int kind) {
+  return mx_is_wgrad(kind) ? MX_STAGE_OUT_BYTES : (kind == MX_DGRAD_DOWN ? 4 * 32 * 33 * 4 : 0);
+}
+__host__ __device__ constexpr size_t mx_smem_bytes(int kind) {
+  return mx_stages(kind) * mx_stage_bytes(kind) + mx_out_bytes(kind) + 1024 + 256;
+}
 constexpr int MX_MAX_STAGES = 6;
 cudaError_t launch_gemm_mx(MxKind kind, const MxParams& p, int grid, cudaStream_t st);
 
@@ -261,6 +287,7 @@ struct Ctx {  // typed views of ctx + ws for one shape
   int* fctl;                 // control block of a persistent GEMM pair (gemm_pair_ctl_words(RP) ints)
   StreamTables tab;
   uint8_t *xq, *xqs, *hq, *hqs, *dyq, *dyqs, *daq, *daqs, *dbq, *dbqs;  // MXFP8 operands and scales
+  uint8_t *xqt, *xqts, *dyqt, *dyqts, *daqt, *daqts, *dbqt, *dbqts, *hgqt, *hgqts;  // MXFP8 weight-gradient operands
 };
 Ctx make_ctx(const Layout& L, void* ctx, void* ws);
 
@@ -295,6 +322,11 @@ cudaError_t launch_quant_weight(int mode, const __nv_bfloat16* src0, const __nv_
                                 int N, uint8_t* q, uint8_t* qs, cudaStream_t st);
 cudaError_t launch_gather_rows_mx(const Layout& L, const Ctx& c, const __nv_bfloat16* src, __nv_bfloat16* dst,
                                   uint8_t* q, uint8_t* qs, cudaStream_t st);
+// Dispatch / reverse-combine with MXFP8 weight gradients: the padded rows gathered from src and
+// quantised along d (qd, qds as launch_gather_rows_mx writes them) and along the rows in blocks of
+// 32 (qr, qrs: rowq layout), no bf16 copy.
+cudaError_t launch_gather_quant2(const Layout& L, const Ctx& c, const __nv_bfloat16* src, uint8_t* qd, uint8_t* qds,
+                                 uint8_t* qr, uint8_t* qrs, cudaStream_t st);
 cudaError_t launch_transpose_wr(const Layout& L, const __nv_bfloat16* W_r, __nv_bfloat16* W_rT, cudaStream_t st);
 cudaError_t launch_rev_dispatch(const Layout& L, const Ctx& c, __nv_bfloat16* dX, cudaStream_t st);
 cudaError_t launch_export_routing(const Layout& L, const Ctx& c, int32_t* counts, int32_t* offsets,

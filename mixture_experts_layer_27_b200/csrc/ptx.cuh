@@ -319,6 +319,20 @@ __device__ __forceinline__ size_t sf_index(int r, int k, int K) {
          ((k & 127) >> 5);
 }
 
+// Operands quantised along the rows (the MXFP8 weight gradients' K = an expert's rows) are K-major
+// and stored 128-row-tile-major: tile t = R / 128 holds C lines of 128 codes (line c = the codes
+// of column c for the tile's rows), and the tile's scale chunks (512 bytes per 128 columns, the
+// sf_index byte order inside) follow one another.  A tile's codes for consecutive columns are
+// contiguous, so the writers' stores and the GEMM's TMA boxes (128 lines of one tile) both stay in
+// one region.
+__device__ __forceinline__ size_t rowq_index(int c, int64_t R, int C) {
+  return (static_cast<size_t>(R >> 7) * C + c) * 128 + (R & 127);
+}
+__device__ __forceinline__ size_t rowq_sf_index(int c, int64_t R, int C) {
+  return (static_cast<size_t>(R >> 7) * (C >> 7) + (c >> 7)) * 512 + (c & 31) * 16 + ((c & 127) >> 5) * 4 +
+         ((R & 127) >> 5);
+}
+
 // Quantise 32 values (one block) to E4M3 with a shared power-of-two scale:
 // exponent = floor(log2(amax)) - 8 (E4M3's largest exponent), scale byte = exponent + 127
 // clamped to [0, 254]; values are scaled exactly and rounded to nearest even with

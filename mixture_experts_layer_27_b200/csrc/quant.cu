@@ -170,6 +170,155 @@ __global__ void __launch_bounds__(256) k_gather_rows_mx(const __nv_bfloat16* __r
   }
 }
 
+// Dispatch / reverse-combine with MXFP8 weight gradients: rows [lo, hi) of the padded layout
+// gathered from src (row R takes token row_asg[R] / k; pad rows are zero) and quantised twice,
+// with no bf16 copy kept: along d (q_d, the dgrad and gate/up GEMMs' K) in the row-major layout
+// of k_gather_rows_mx, and along the rows in blocks of 32 (q_r, the weight-gradient GEMMs' K) in
+// the 128-row-tile-major layout (rowq_index, rowq_sf_index).  Every expert segment starts on a
+// multiple of 128 and is its real rows rounded up to 128, so a tile lies in one expert and starts
+// with a real row.
+// A CTA walks 128-row x 64-column tiles through a ring of GQ_STAGES shared-memory stages: each
+// thread copies four 16-byte pieces of a tile with cp.async (zero-filled for pad rows), so the
+// copies of the next GQ_STAGES - 1 tiles are in flight (the row assignments they need are loaded
+// one tile earlier still) while one tile is quantised: thread t takes the 32-value d-block t % 2
+// of row t / 2 (dead pad rows are skipped: nothing reads them), and thread (column t % 64, block
+// t / 64) the column's 32 rows (a block that starts past the expert's real rows is skipped: the
+// GEMM never reads it).
+constexpr int kQRowsPitch = 72;  // bf16 per staged row: 144 bytes (16-byte aligned; rows 4 banks apart)
+constexpr int GQ_STAGES = 4;
+constexpr size_t GQ_STAGE_BYTES = 128 * kQRowsPitch * 2 + 128 * 4;  // rows, then their row_asg
+constexpr size_t GQ_SMEM = GQ_STAGES * GQ_STAGE_BYTES;
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool fill) {
+  // src-size 0 writes 16 zero bytes and reads nothing
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(fill ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void gq_load_asg(const int* __restrict__ row_asg, int64_t r0, int64_t r_hi, int t,
+                                            int (&a)[4]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) a[j] = r0 < r_hi ? __ldg(row_asg + r0 + ((t + 256 * j) >> 3)) : ROW_DEAD;
+}
+// Copies of one tile into a stage (rows of tokens a / k; zeros for pad rows) and its row flags.
+__device__ __forceinline__ void gq_issue(const __nv_bfloat16* __restrict__ src, const int (&a)[4], int k, int d,
+                                         int c0, int t, uint8_t* stage) {
+  __nv_bfloat16* tile = reinterpret_cast<__nv_bfloat16*>(stage);
+  int* flag = reinterpret_cast<int*>(stage + 128 * kQRowsPitch * 2);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int i = t + 256 * j;
+    const bool real = a[j] >= 0;
+    const __nv_bfloat16* g = src + (real ? static_cast<size_t>(a[j] / k) * d : 0) + c0 + (i & 7) * 8;
+    cp_async16(tile + (i >> 3) * kQRowsPitch + (i & 7) * 8, g, real);
+    if ((i & 7) == 0) flag[i >> 3] = a[j];
+  }
+}
+
+__global__ void __launch_bounds__(256, 3) k_gather_quant2(const __nv_bfloat16* __restrict__ src,
+                                                          const int* __restrict__ row_asg, const int* __restrict__ lo,
+                                                          const int* __restrict__ hi, int k, int d,
+                                                          uint8_t* __restrict__ qd, uint8_t* __restrict__ qds,
+                                                          uint8_t* __restrict__ qr, uint8_t* __restrict__ qrs) {
+  extern __shared__ __align__(16) uint8_t gq_smem[];
+  const int64_t r_hi = __ldg(hi);
+  const int c0 = blockIdx.x * 64;
+  const int t = threadIdx.x;
+  const int64_t step = static_cast<int64_t>(gridDim.y) * 128;
+  const int64_t first = __ldg(lo) + static_cast<int64_t>(blockIdx.y) * 128;
+  int a[4];
+  // prologue: tiles 0 .. GQ_STAGES - 2 in flight, the row assignments of the next one loaded
+#pragma unroll
+  for (int s = 0; s < GQ_STAGES - 1; ++s) {
+    const int64_t r = first + s * step;
+    gq_load_asg(row_asg, r, r_hi, t, a);
+    if (r < r_hi) gq_issue(src, a, k, d, c0, t, gq_smem + s * GQ_STAGE_BYTES);
+    cp_async_commit();
+  }
+  gq_load_asg(row_asg, first + (GQ_STAGES - 1) * step, r_hi, t, a);
+  int n = 0;
+  for (int64_t r0 = first; r0 < r_hi; r0 += step, ++n) {
+    cp_async_wait<GQ_STAGES - 2>();  // this thread's copies of tile n have landed
+    __syncthreads();                 // everyone's; and tile n - 1's stage is no longer read
+    {
+      const int64_t rn = r0 + (GQ_STAGES - 1) * step;  // into the stage tile n - 1 used
+      if (rn < r_hi) gq_issue(src, a, k, d, c0, t, gq_smem + ((n + GQ_STAGES - 1) % GQ_STAGES) * GQ_STAGE_BYTES);
+      cp_async_commit();
+      gq_load_asg(row_asg, rn + step, r_hi, t, a);
+    }
+    const uint8_t* stage = gq_smem + (n % GQ_STAGES) * GQ_STAGE_BYTES;
+    const __nv_bfloat16* tile = reinterpret_cast<const __nv_bfloat16*>(stage);
+    const int* flag = reinterpret_cast<const int*>(stage + 128 * kQRowsPitch * 2);
+    {  // along d: block t % 2 (32 columns) of row t / 2
+      const int rr = t >> 1, blk = t & 1;
+      if (flag[rr] != ROW_DEAD) {
+        float v[32];
+        const uint4* s4 = reinterpret_cast<const uint4*>(tile + rr * kQRowsPitch + blk * 32);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint4 w4 = s4[q4];
+          const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const float2 f = unpack_bf16(ww[h]);
+            v[8 * q4 + 2 * h] = f.x;
+            v[8 * q4 + 2 * h + 1] = f.y;
+          }
+        }
+        uint32_t w[8];
+        const uint8_t sb = mx_quant32(v, w);
+        const int64_t R = r0 + rr;
+        uint4* dst = reinterpret_cast<uint4*>(qd + R * d + c0 + blk * 32);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        qds[sf_index(static_cast<int>(R), c0 + blk * 32, d)] = sb;
+      }
+    }
+    {  // along the rows: rows 32 b .. 32 b + 31 of column c
+      const int c = t & 63, b = t >> 6;
+      if (flag[b * 32] >= 0) {
+        float v[32];
+#pragma unroll
+        for (int r = 0; r < 32; ++r) v[r] = __bfloat162float(tile[(b * 32 + r) * kQRowsPitch + c]);
+        uint32_t w[8];
+        const uint8_t sb = mx_quant32(v, w);
+        uint4* dst = reinterpret_cast<uint4*>(qr + rowq_index(c0 + c, r0 + b * 32, d));
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        qrs[rowq_sf_index(c0 + c, r0 + b * 32, d)] = sb;
+      }
+    }
+  }
+  cp_async_wait<0>();  // no copy outlives the CTA's shared memory
+}
+
+cudaError_t launch_gather_quant2(const Layout& L, const Ctx& c, const __nv_bfloat16* src, uint8_t* qd, uint8_t* qds,
+                                 uint8_t* qr, uint8_t* qrs, cudaStream_t st) {
+  static bool configured[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(k_gather_quant2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(GQ_SMEM));
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  // The padded-row capacity RP is a worst case (every token's k assignments local): the routed
+  // rows are often far fewer, so the grid is one wave (three CTAs of 256 threads fit an SM) that
+  // walks the row tiles, instead of one CTA per possible tile.
+  const int64_t tiles = L.RP / 128;
+  const int gx = L.d / 64;
+  int64_t gy = (148 * 3) / gx;
+  if (gy > tiles) gy = tiles;
+  if (gy < 1) gy = 1;
+  k_gather_quant2<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), 256, GQ_SMEM, st>>>(
+      src, c.row_asg, c.poff, c.poff + L.El, L.k, L.d, qd, qds, qr, qrs);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quant_weight(int mode, const __nv_bfloat16* src0, const __nv_bfloat16* src1, int64_t R_out, int K,
                                 int N, uint8_t* q, uint8_t* qs, cudaStream_t st) {
   const int smem = 128 * kQuantPitch * 2;

@@ -41,7 +41,10 @@ def test_router_weight_gradient_flops():
     # the persistent kernel runs gate/up and down in one launch: an alternative, not an extra GEMM
     assert f["gemm_gateup_down_persistent"] == f["gemm_gateup_swiglu"] + f["gemm_down_combw"]
     assert f["gemm_dgrads_persistent"] == f["gemm_dgrad_down_swiglu_bwd"] + f["gemm_dgrad_gateup"]
-    assert sum(v for k, v in f.items() if k.startswith("gemm_") and "persistent" not in k) == 18 * dI * rows
+    # the MXFP8 weight-gradient GEMMs replace the bf16 ones (MOE_MXFP8_ALL): alternatives as well
+    assert f["gemm_wgrad_gateup_mx"] == f["gemm_wgrad_gateup"] and f["gemm_wgrad_down_mx"] == f["gemm_wgrad_down"]
+    assert sum(v for k, v in f.items()
+               if k.startswith("gemm_") and "persistent" not in k and not k.endswith("_mx")) == 18 * dI * rows
 
 
 def test_traffic_figure_only_for_the_captured_sources():
