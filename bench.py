@@ -769,9 +769,9 @@ def main():
                     help="write the expert weight gradients as fp32 instead of bf16 (the weights' dtype)")
     ap.add_argument("--launches", action="store_true",
                     help="run every grouped GEMM as its own launch instead of the persistent pairs")
-    ap.add_argument("--mx-wgrad", action="store_true",
-                    help="MXFP8 workloads: run the weight-gradient GEMMs on MXFP8 as well (operands quantised "
-                         "along each expert's rows) instead of on the bf16 operands")
+    ap.add_argument("--wgrad-gemms", choices=["mxfp8", "bf16"], default=None,
+                    help="MXFP8 workloads: the weight-gradient GEMMs on MXFP8 (operands quantised along each "
+                         "expert's rows; the default) or on the bf16 operands")
     ap.add_argument("--persistent", action="store_true",
                     help="require the persistent pairs (the default for bf16 one-batch workloads): the forward's "
                          "gate/up and down GEMMs, and the backward's two dgrads, each pair as one persistent launch")
@@ -779,8 +779,9 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     w = IN.WORKLOADS[args.workload]
-    if args.mx_wgrad and not w.mxfp8:
-        ap.error("--mx-wgrad applies to the MXFP8 workloads; %s is bf16" % w.name)
+    if args.wgrad_gemms and not w.mxfp8:
+        ap.error("--wgrad-gemms applies to the MXFP8 workloads; %s is bf16" % w.name)
+    args.mx_wgrad = w.mxfp8 and args.wgrad_gemms != "bf16"
     if args.launches and w.stream_M:
         ap.error("the ring-streamed layer always runs its GEMM pairs as persistent launches")
     if args.persistent and (w.mxfp8 or w.stream_M or args.launches):

@@ -256,6 +256,83 @@ def test_full_size_mxfp8_kimi():
     torch.cuda.empty_cache()
 
 
+def test_full_size_mxfp8_weight_gradients_kimi():
+    # kimi_mx with the weight-gradient GEMMs on MXFP8 too (MOE_MXFP8_ALL): Y, dX and dW_r are the
+    # plain MXFP8 mode's bits; the hottest and coldest experts' weight gradients equal the product
+    # of the operands the device quantised, and are within 6e-2 of the MXFP8 oracle with MX
+    # weight gradients; a rerun is bit-identical.
+    w = IN.WORKLOADS["kimi_mx"]
+    x = IN.make_inputs(w, device="cuda")
+
+    def run(mx_wgrad):
+        lay = B.MoELayerMX(w.T, w.d, w.E, w.I, w.k, mx_wgrad=mx_wgrad)
+        lay.prepare(x["W_gate"], x["W_up"], x["W_down"])
+        Y = lay.forward(x["X"], x["W_r"], x["bias"])
+        g = lay.backward(x["X"], x["W_r"], x["dY"])
+        torch.cuda.synchronize()
+        assert lay.error() == B.MOE_OK
+        return lay, Y, g
+
+    lay0, Y0, g0 = run(False)
+    del lay0
+    keep = {"Y": Y0, "dX": g0["dX"], "dW_r": g0["dW_r"]}
+    del g0
+    torch.cuda.empty_cache()
+    lay, Y, g = run(True)
+    assert torch.equal(Y.view(torch.int16), keep["Y"].view(torch.int16))
+    assert torch.equal(g["dX"].view(torch.int16), keep["dX"].view(torch.int16))
+    assert torch.equal(g["dW_r"].view(torch.int32), keep["dW_r"].view(torch.int32))
+    del keep, Y0
+
+    r = lay.routing()
+    counts = r["counts"].cpu().numpy()
+    poff = r["padded_offsets"].cpu().numpy()
+    gids = r["ids"].cpu().numpy()
+    nz = np.nonzero(counts)[0]
+    hot, cold = int(nz[np.argmax(counts[nz])]), int(nz[np.argmin(counts[nz])])
+    # the GEMMs on the device's own operands (dequantised here)
+    vals = {}
+    for which, name in enumerate(("X", "dY", "dA", "dB", "Hg")):
+        codes, sc = lay.wgrad_operand(which)
+        vals[name] = {e: O.mx_dequantize(codes[:, poff[e]:poff[e] + (int(counts[e]) + 31) // 32 * 32],
+                                         sc[:, poff[e] // 32:(poff[e] + (int(counts[e]) + 31) // 32 * 32) // 32],
+                                         axis=1)[:, :int(counts[e])] for e in (hot, cold)}
+        del codes, sc
+    for e in (hot, cold):
+        want = {"dW_gate": vals["X"][e] @ vals["dA"][e].T, "dW_up": vals["X"][e] @ vals["dB"][e].T,
+                "dW_down": vals["Hg"][e] @ vals["dY"][e].T}
+        for n in want:
+            assert relerr(to64(g[n][e]), want[n]) <= 8e-3, (n, e)
+    # against the MXFP8 oracle with MX weight gradients (tokens whose selection is a near tie in
+    # fp64 are left out, as above)
+    X, Wr, dY = to64(x["X"]), to64(x["W_r"]), to64(x["dY"])
+    b = None if x["bias"] is None else to64(x["bias"])
+    lg64 = O.router_logits(X, Wr, b)
+    differ = np.nonzero(np.any(np.sort(O.topk_ids(lg64, w.k), 1) != np.sort(gids, 1), axis=1))[0]
+    tie_tokens = set(differ.tolist())
+    Wg, Wu, Wd = ExpertCache(x["W_gate"]), ExpertCache(x["W_up"]), ExpertCache(x["W_down"])
+    weights = {n: ExpertCache(x[n], keep=1) for n in ("W_gate", "W_up", "W_down")}
+    cache = mx_layout_cache(sorted({hot, cold}), weights)
+    for e in sorted({hot, cold}):
+        _, ctx = O.forward_mx(X, Wr, b, Wg, Wu, Wd, w.k, first_local=e, num_local=1, rounded=cache.__getitem__)
+        if set(ctx["sched"]["perm"].tolist()) & tie_tokens:
+            continue
+        go = O.backward_mx(ctx, dY, mx_wgrad=True)
+        for n in ("dW_gate", "dW_up", "dW_down"):
+            assert relerr(to64(g[n][e]), go[n][e]) <= TOL_MX, (n, e)
+    del cache
+    # a second run over fresh buffers is bit-identical
+    del lay
+    torch.cuda.empty_cache()
+    lay2, Y2, g2 = run(True)
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+    for n in ("dW_gate", "dW_up", "dW_down"):
+        for e0 in range(0, w.E, 32):
+            assert torch.equal(g[n][e0:e0 + 32].view(torch.int16), g2[n][e0:e0 + 32].view(torch.int16)), (n, e0)
+    del lay2, Y, Y2, g, g2, x
+    torch.cuda.empty_cache()
+
+
 def test_full_size_ep64_ring_stream():
     # Config 5 at n = 4096 tokens per local expert: 16 minibatches of 2048 tokens through the
     # 256 MiB ring, 6 local experts of 384; the backward replays part of the stream into the
