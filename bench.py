@@ -219,9 +219,9 @@ def algorithmic_bytes(w: IN.Workload, wgrad_elem_bytes: int = 2, mx_wgrad: bool 
 # A figure is reported only while the GEMM sources still hash to the value they had
 # when the counters were taken.
 NCU_TRAFFIC = {
-    ("gemm_dgrads_persistent", "dsv3"): ((1457.617152e6 + 0.860672e6) * 16, "7f8b1d31de8047ca"),
-    ("gemm_gateup_down_persistent", "dsv3"): ((1442.467840e6 + 4.975872e6) * 16, "7f8b1d31de8047ca"),
-    ("gemm_wgrad_gateup", "dsv3"): ((34.669056e6 + 875.510784e6) * 16, "7f8b1d31de8047ca"),
+    ("gemm_dgrads_persistent", "dsv3"): ((1457.315072e6 + 0.631040e6) * 16, "a795909224e39209"),
+    ("gemm_gateup_down_persistent", "dsv3"): ((1442.505728e6 + 4.907264e6) * 16, "a795909224e39209"),
+    ("gemm_wgrad_gateup", "dsv3"): ((34.690816e6 + 875.523328e6) * 16, "a795909224e39209"),
 }
 GEMM_SOURCES = ("gemm.cu", "ptx.cuh", "moe_internal.cuh")
 
@@ -743,10 +743,11 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
         line["mxfp8_peak"] = fp8_peak
         if fp8:
             line["pct_of_mxfp8_peak"] = 100.0 * per_gpu_tflops / fp8
-        line["peak_note"] += ("; MXFP8: gate/up, down and both dgrads on block-scaled fp8 tensor cores, "
-                              "weight gradients bf16; pct_of_mxfp8_peak against the sustained MXFP8 GEMM "
-                              "measured in this run")
-        line["dtype"] = "mxfp8 (e4m3 + e8m0 scales) / bf16 wgrad"
+        wg = ("weight gradients on block-scaled fp8 too (operands quantised along each expert's rows)"
+              if args.mx_wgrad else "weight gradients bf16")
+        line["peak_note"] += ("; MXFP8: gate/up, down and both dgrads on block-scaled fp8 tensor cores, %s; "
+                              "pct_of_mxfp8_peak against the sustained MXFP8 GEMM measured in this run" % wg)
+        line["dtype"] = "mxfp8 (e4m3 + e8m0 scales)" + ("" if args.mx_wgrad else " / bf16 wgrad")
     if w.stream_M:
         pl = layer.plan()["plan"]
         line["stream_plan"] = {"macrobatches": int(pl[0]), "backward_chunks": int(pl[1]), "padded_rows": int(pl[2]),
