@@ -164,6 +164,8 @@ def algorithmic_flops(w: IN.Workload) -> dict:
 def algorithmic_bytes(w: IN.Workload, wgrad_elem_bytes: int = 2, mx_wgrad: bool = False) -> dict:
     T, d, E, I, k, El = w.tokens, w.d, w.E, w.I, w.k, w.El
     rows = local_rows(w)
+    # token rows a gather reads: every token once, or in an expert slice at most one per local row
+    Tg = min(T, rows)
     W1 = El * d * I * 2  # one expert weight matrix family (gate, up or down), bytes
     G1 = El * d * I * wgrad_elem_bytes  # its gradient (bf16, or fp32 with --wgrad-fp32)
     if w.mxfp8:
@@ -173,11 +175,11 @@ def algorithmic_bytes(w: IN.Workload, wgrad_elem_bytes: int = 2, mx_wgrad: bool 
             "router_logits": T * d * 2 + d * E * 2 + T * E * 4,
             "topk_gating": T * E * 4 + rows * 8,
             # X once, then bf16 rows and fp8 along d; or (mx_wgrad) fp8 along d and along the rows
-            "dispatch": T * d * 2 + (2 * rows * d * 33 // 32 if mx_wgrad else rows * d * 2 + rows * d * 33 // 32),
+            "dispatch": Tg * d * 2 + (2 * rows * d * 33 // 32 if mx_wgrad else rows * d * 2 + rows * d * 33 // 32),
             "gemm_gateup_swiglu": 2 * Wq + rows * d * 33 // 32 + 2 * rows * I * 2 + rows * I * 33 // 32,
             "gemm_down_combw": Wq + rows * I * 33 // 32 + rows * d * 2,
             "combine": rows * d * 2 + T * d * 2,
-            "reverse_combine": T * d * 2 + (2 * rows * d * 33 // 32 if mx_wgrad else rows * d * 2 + rows * d * 33 // 32),
+            "reverse_combine": Tg * d * 2 + (2 * rows * d * 33 // 32 if mx_wgrad else rows * d * 2 + rows * d * 33 // 32),
             # dA, dB, Hg out in bf16 for the bf16 weight gradients, or (mx_wgrad) as fp8 along the rows
             "gemm_dgrad_down_swiglu_bwd": Wq + rows * d * 33 // 32 + 2 * rows * I * 2
             + (3 * rows * I * 33 // 32 if mx_wgrad else 3 * rows * I * 2) + 2 * rows * I * 33 // 32,
@@ -194,11 +196,11 @@ def algorithmic_bytes(w: IN.Workload, wgrad_elem_bytes: int = 2, mx_wgrad: bool 
     return {
         "router_logits": T * d * 2 + d * E * 2 + T * E * 4,
         "topk_gating": T * E * 4 + rows * 8,
-        "dispatch": T * d * 2 + rows * d * 2,
+        "dispatch": Tg * d * 2 + rows * d * 2,
         "gemm_gateup_swiglu": 2 * W1 + rows * d * 2 + 3 * rows * I * 2,
         "gemm_down_combw": W1 + rows * I * 2 + rows * d * 2,
         "combine": rows * d * 2 + T * d * 2,
-        "reverse_combine": T * d * 2 + rows * d * 2,
+        "reverse_combine": Tg * d * 2 + rows * d * 2,
         "gemm_dgrad_down_swiglu_bwd": W1 + rows * d * 2 + 2 * rows * I * 2 + 3 * rows * I * 2,
         "router_wgrad": T * d * 2 + T * k * 8 + d * E * 4,  # X once, dl and ids, dW_r
         "gemm_dgrad_gateup": 2 * W1 + 2 * rows * I * 2 + rows * d * 2,
