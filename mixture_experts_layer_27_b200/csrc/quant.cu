@@ -177,7 +177,10 @@ __global__ void __launch_bounds__(256) k_gather_rows_mx(const __nv_bfloat16* __r
 // the 128-row-tile-major layout (rowq_index, rowq_sf_index).  Every expert segment starts on a
 // multiple of 128 and is its real rows rounded up to 128, so a tile lies in one expert and starts
 // with a real row.
-// A CTA walks 128-row x 64-column tiles through a ring of GQ_STAGES shared-memory stages: each
+// Work items are (128-row tile, 64-column group) pairs, column groups fastest, dealt round-robin
+// to a grid of resident CTAs (so CTAs running together share a tile's rows and every CTA gets the
+// same number of items, give or take one).  A CTA walks its items through a ring of GQ_STAGES
+// shared-memory stages: each
 // thread copies four 16-byte pieces of a tile with cp.async (zero-filled for pad rows), so the
 // copies of the next GQ_STAGES - 1 tiles are in flight (the row assignments they need are loaded
 // one tile earlier still) while one tile is quantised: thread t takes the 32-value d-block t % 2
@@ -198,10 +201,10 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-__device__ __forceinline__ void gq_load_asg(const int* __restrict__ row_asg, int64_t r0, int64_t r_hi, int t,
+__device__ __forceinline__ void gq_load_asg(const int* __restrict__ row_asg, int64_t r0, bool valid, int t,
                                             int (&a)[4]) {
 #pragma unroll
-  for (int j = 0; j < 4; ++j) a[j] = r0 < r_hi ? __ldg(row_asg + r0 + ((t + 256 * j) >> 3)) : ROW_DEAD;
+  for (int j = 0; j < 4; ++j) a[j] = valid ? __ldg(row_asg + r0 + ((t + 256 * j) >> 3)) : ROW_DEAD;
 }
 // Copies of one tile into a stage (rows of tokens a / k; zeros for pad rows) and its row flags.
 __device__ __forceinline__ void gq_issue(const __nv_bfloat16* __restrict__ src, const int (&a)[4], int k, int d,
@@ -224,30 +227,37 @@ __global__ void __launch_bounds__(256, 3) k_gather_quant2(const __nv_bfloat16* _
                                                           uint8_t* __restrict__ qd, uint8_t* __restrict__ qds,
                                                           uint8_t* __restrict__ qr, uint8_t* __restrict__ qrs) {
   extern __shared__ __align__(16) uint8_t gq_smem[];
-  const int64_t r_hi = __ldg(hi);
-  const int c0 = blockIdx.x * 64;
+  const int64_t r_lo = __ldg(lo);
+  const int ng = d / 64;                              // column groups
+  const int64_t items = (__ldg(hi) - r_lo) / 128 * ng;  // (tile, column group) pairs
   const int t = threadIdx.x;
-  const int64_t step = static_cast<int64_t>(gridDim.y) * 128;
-  const int64_t first = __ldg(lo) + static_cast<int64_t>(blockIdx.y) * 128;
+  auto row0 = [&](int64_t it) { return r_lo + (it / ng) * 128; };
+  auto col0 = [&](int64_t it) { return static_cast<int>(it % ng) * 64; };
   int a[4];
-  // prologue: tiles 0 .. GQ_STAGES - 2 in flight, the row assignments of the next one loaded
+  // prologue: items 0 .. GQ_STAGES - 2 of this CTA in flight, the row assignments of the next one loaded
 #pragma unroll
   for (int s = 0; s < GQ_STAGES - 1; ++s) {
-    const int64_t r = first + s * step;
-    gq_load_asg(row_asg, r, r_hi, t, a);
-    if (r < r_hi) gq_issue(src, a, k, d, c0, t, gq_smem + s * GQ_STAGE_BYTES);
+    const int64_t it = blockIdx.x + static_cast<int64_t>(s) * gridDim.x;
+    gq_load_asg(row_asg, row0(it), it < items, t, a);
+    if (it < items) gq_issue(src, a, k, d, col0(it), t, gq_smem + s * GQ_STAGE_BYTES);
     cp_async_commit();
   }
-  gq_load_asg(row_asg, first + (GQ_STAGES - 1) * step, r_hi, t, a);
+  {
+    const int64_t it = blockIdx.x + static_cast<int64_t>(GQ_STAGES - 1) * gridDim.x;
+    gq_load_asg(row_asg, row0(it), it < items, t, a);
+  }
   int n = 0;
-  for (int64_t r0 = first; r0 < r_hi; r0 += step, ++n) {
-    cp_async_wait<GQ_STAGES - 2>();  // this thread's copies of tile n have landed
-    __syncthreads();                 // everyone's; and tile n - 1's stage is no longer read
+  for (int64_t it = blockIdx.x; it < items; it += gridDim.x, ++n) {
+    const int64_t r0 = row0(it);
+    const int c0 = col0(it);
+    cp_async_wait<GQ_STAGES - 2>();  // this thread's copies of item n have landed
+    __syncthreads();                 // everyone's; and item n - 1's stage is no longer read
     {
-      const int64_t rn = r0 + (GQ_STAGES - 1) * step;  // into the stage tile n - 1 used
-      if (rn < r_hi) gq_issue(src, a, k, d, c0, t, gq_smem + ((n + GQ_STAGES - 1) % GQ_STAGES) * GQ_STAGE_BYTES);
+      const int64_t in = it + static_cast<int64_t>(GQ_STAGES - 1) * gridDim.x;  // into the stage item n - 1 used
+      if (in < items) gq_issue(src, a, k, d, col0(in), t, gq_smem + ((n + GQ_STAGES - 1) % GQ_STAGES) * GQ_STAGE_BYTES);
       cp_async_commit();
-      gq_load_asg(row_asg, rn + step, r_hi, t, a);
+      const int64_t in2 = in + gridDim.x;
+      gq_load_asg(row_asg, row0(in2), in2 < items, t, a);
     }
     const uint8_t* stage = gq_smem + (n % GQ_STAGES) * GQ_STAGE_BYTES;
     const __nv_bfloat16* tile = reinterpret_cast<const __nv_bfloat16*>(stage);
@@ -307,15 +317,16 @@ cudaError_t launch_gather_quant2(const Layout& L, const Ctx& c, const __nv_bfloa
     configured[dev] = true;
   }
   // The padded-row capacity RP is a worst case (every token's k assignments local): the routed
-  // rows are often far fewer, so the grid is one wave (three CTAs of 256 threads fit an SM) that
-  // walks the row tiles, instead of one CTA per possible tile.
-  const int64_t tiles = L.RP / 128;
-  const int gx = L.d / 64;
-  int64_t gy = (148 * 3) / gx;
-  if (gy > tiles) gy = tiles;
-  if (gy < 1) gy = 1;
-  k_gather_quant2<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), 256, GQ_SMEM, st>>>(
-      src, c.row_asg, c.poff, c.poff + L.El, L.k, L.d, qd, qds, qr, qrs);
+  // rows are often far fewer, so the grid is one wave of resident CTAs (three of 256 threads fit
+  // an SM) that deals the items among themselves, instead of one CTA per possible item.
+  int sms = 148;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 148;
+  const int64_t max_items = L.RP / 128 * (L.d / 64);
+  int64_t grid = static_cast<int64_t>(sms) * 3;
+  if (grid > max_items) grid = max_items;
+  if (grid < 1) grid = 1;
+  k_gather_quant2<<<static_cast<unsigned>(grid), 256, GQ_SMEM, st>>>(src, c.row_asg, c.poff, c.poff + L.El, L.k,
+                                                                      L.d, qd, qds, qr, qrs);
   return cudaGetLastError();
 }
 

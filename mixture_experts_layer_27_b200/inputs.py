@@ -13,6 +13,7 @@ Workloads (the pages name model families and print no shapes; these stand in):
 * ``epmx``, ``epbf``  the same slice as one batch of 32768 tokens (MXFP8 / bf16), no ring
 * ``dsv3_e16``  the dsv3 expert shape with 16 experts and 128 tokens (profiler captures)
 * ``kimi_mx_e24`` the kimi expert shape in MXFP8, 24 experts, 256 tokens (profiler captures)
+* ``epmx_t8192_n2368`` epmx_n2368's dispatched rows over 8192 tokens, 96 experts (profiler captures)
 
 Distributions: X, dY ~ N(0, 1); W_gate, W_up ~ N(0, 1/d) (std 1/sqrt(fan_in));
 W_down ~ N(0, 1/I); W_r ~ N(0, 0.02^2); every tensor rounded once to bf16 (RNE).
@@ -86,6 +87,11 @@ for _n in (512, 2368, 4096, 8192):
                                         num_local=6, local_tokens=_n)
     WORKLOADS[f"epbf_n{_n}"] = Workload(f"epbf_n{_n}", 32768, 7168, 384, 8, 2048, first_local=0, num_local=6,
                                         local_tokens=_n)
+# epmx_n2368's expert work (6 local experts x 2368 rows, MXFP8) over 8192 tokens and 96 experts: the
+# same dispatched rows and GEMM tiles with a padded-row capacity (and workspace) a quarter of the
+# size, for profiler captures (a few GB on the device)
+WORKLOADS["epmx_t8192_n2368"] = Workload("epmx_t8192_n2368", 8192, 7168, 96, 8, 2048, mxfp8=True, first_local=0,
+                                         num_local=6, local_tokens=2368)
 
 
 def _seed(base: int, *names) -> int:
