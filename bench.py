@@ -126,7 +126,7 @@ def run_config(w: IN.Workload, args) -> dict:
     """The `config` of both arms' lines: the workload, the gradient dtype and how the GEMM pairs are
     launched (the ring-streamed layer always runs them as persistent pairs)."""
     cfg = dict(workload_config(w), wgrad_dtype="fp32" if args.wgrad_fp32 else "bf16",
-               forward="persistent" if args.persistent or w.stream_M else "launches")
+               forward="persistent" if args.persistent or (w.stream_M and not w.mxfp8) else "launches")
     if w.mxfp8:  # the weight-gradient GEMMs: MXFP8 operands along the rows, or the bf16 operands
         cfg["wgrad_gemms"] = "mxfp8" if getattr(args, "mx_wgrad", False) else "bf16"
     return cfg
@@ -464,7 +464,10 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     peaks, peak_kind = load_peaks()
     x = IN.make_inputs(w, device=dev)
     wdt = torch.float32 if args.wgrad_fp32 else torch.bfloat16
-    if w.mxfp8:
+    if w.mxfp8 and w.stream_M:
+        layer = B.MoEStreamMX(w.T, w.d, w.E, w.I, w.k, w.stream_M, w.ring_bytes, w.first_local, w.num_local,
+                              device=dev, wgrad_dtype=wdt)
+    elif w.mxfp8:
         layer = B.MoELayerMX(w.T, w.d, w.E, w.I, w.k, w.first_local, w.num_local, device=dev, wgrad_dtype=wdt,
                              mx_wgrad=args.mx_wgrad)
     elif w.stream_M:
@@ -784,7 +787,10 @@ def main():
     w = IN.WORKLOADS[args.workload]
     if args.wgrad_gemms and not w.mxfp8:
         ap.error("--wgrad-gemms applies to the MXFP8 workloads; %s is bf16" % w.name)
-    args.mx_wgrad = w.mxfp8 and args.wgrad_gemms != "bf16"
+    if args.wgrad_gemms == "mxfp8" and w.stream_M:
+        ap.error("the ring-streamed MXFP8 layer keeps bf16 weight gradients")
+    # MXFP8 weight gradients for the one-batch MXFP8 workloads (the ring stream keeps bf16 ones)
+    args.mx_wgrad = w.mxfp8 and not w.stream_M and args.wgrad_gemms != "bf16"
     if args.launches and w.stream_M:
         ap.error("the ring-streamed layer always runs its GEMM pairs as persistent launches")
     if args.persistent and (w.mxfp8 or w.stream_M or args.launches):

@@ -291,8 +291,9 @@ moe_status moe_bwd_mx(const moe_shape* shape, const void* X, const void* W_r, co
  * device; the host enqueues a fixed number of launches per minibatch.
  * Requirements: shape->T a multiple of 16; 1 <= M <= 256; ring_bytes at least
  * moe_stream_min_ring_bytes(shape) (one minibatch's worst case), else
- * MOE_ERR_WORKSPACE_TOO_SMALL.  bf16 operands only (wgrad_dtype applies as in
- * moe_bwd). */
+ * MOE_ERR_WORKSPACE_TOO_SMALL.  moe_fwd_stream / moe_bwd_stream take bf16 weights
+ * (MOE_BF16 shapes); moe_fwd_stream_mx / moe_bwd_stream_mx below run MOE_MXFP8 shapes
+ * (wgrad_dtype applies as in moe_bwd).  The size calls accept either. */
 size_t moe_stream_ctx_size(const moe_shape* shape, int32_t num_minibatches);
 size_t moe_stream_workspace_size(const moe_shape* shape, int32_t num_minibatches);
 size_t moe_stream_min_ring_bytes(const moe_shape* shape);
@@ -309,6 +310,19 @@ moe_status moe_bwd_stream(const moe_shape* shape, int32_t num_minibatches, const
  * replayed rows, resident rows, ring rows, 0...] then mb_of[M],
  * seg_poff[M*El+1], cum[M*El], mb_range[2M], shift_fwd[M], shift_bwd[M],
  * replay[M], chunk[4M] ({m_lo, m_hi, valid, mode}), ring_start[M]. */
+/* MXFP8 ring-streamed layer (shape->prec = MOE_MXFP8): the same plan, ring and backward chunks as
+ * moe_fwd_stream / moe_bwd_stream, with the gate/up, down and both dgrad GEMMs on MXFP8 from the
+ * prepared weights `wq` (moe_prepare_weights of this shape); the forward's dispatch writes each
+ * macrobatch's rows to the ring in bf16 and quantises them along d.  The weight gradients stay bf16
+ * (MOE_MXFP8_ALL shapes are refused: MOE_ERR_UNSUPPORTED).  ctx / ws / ring sizes: the
+ * moe_stream_* size calls of this shape.  Same errors as the bf16 stream. */
+moe_status moe_fwd_stream_mx(const moe_shape* shape, int32_t num_minibatches, const void* X, const void* W_r,
+                             const float* bias, const void* wq, size_t wq_bytes, void* Y, void* ctx, size_t ctx_bytes,
+                             void* ring, size_t ring_bytes, void* ws, size_t ws_bytes, void* stream);
+moe_status moe_bwd_stream_mx(const moe_shape* shape, int32_t num_minibatches, const void* X, const void* W_r,
+                             const void* wq, size_t wq_bytes, const void* dY, void* ctx, size_t ctx_bytes, void* dX,
+                             void* dW_gate, void* dW_up, void* dW_down, float* dW_r, void* ring, size_t ring_bytes,
+                             void* ws, size_t ws_bytes, void* stream);
 moe_status moe_debug_stream_plan(const moe_shape* shape, int32_t num_minibatches, const void* ctx, int32_t* tables,
                                  void* stream);
 

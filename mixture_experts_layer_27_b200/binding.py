@@ -134,6 +134,10 @@ _SIGS = {
     "moe_debug_stream_plan": (ctypes.c_int, [_S, ctypes.c_int32, _P, _P, _P]),
     "moe_weights_size": (ctypes.c_size_t, [_S]),
     "moe_prepare_weights": (ctypes.c_int, [_S, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_fwd_stream_mx": (ctypes.c_int, [_S, ctypes.c_int32, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, ctypes.c_size_t,
+                                         _P, ctypes.c_size_t, _P, ctypes.c_size_t, _P]),
+    "moe_bwd_stream_mx": (ctypes.c_int, [_S, ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P, _P, ctypes.c_size_t,
+                                         _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, ctypes.c_size_t, _P]),
     "moe_fwd_mx": (ctypes.c_int, [_S, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, ctypes.c_size_t, _P, ctypes.c_size_t,
                                   _P]),
     "moe_bwd_mx": (ctypes.c_int, [_S, _P, _P, _P, ctypes.c_size_t, _P, _P, ctypes.c_size_t, _P, _P, _P, _P, _P, _P,
@@ -331,6 +335,20 @@ def moe_weights_size(shape) -> int:
 def moe_prepare_weights(shape, W_gate, W_up, W_down, wq, stream=None) -> int:
     return int(lib().moe_prepare_weights(ctypes.byref(shape), _ptr(W_gate), _ptr(W_up), _ptr(W_down), _ptr(wq),
                                          _nbytes(wq), _stream(stream)))
+
+
+def moe_fwd_stream_mx(shape, M, X, W_r, bias, wq, Y, ctx, ring, ws, stream=None) -> int:
+    return int(lib().moe_fwd_stream_mx(ctypes.byref(shape), int(M), _ptr(X), _ptr(W_r), _ptr(bias), _ptr(wq),
+                                       _nbytes(wq), _ptr(Y), _ptr(ctx), _nbytes(ctx), _ptr(ring), _nbytes(ring),
+                                       _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def moe_bwd_stream_mx(shape, M, X, W_r, wq, dY, ctx, dX, dW_gate, dW_up, dW_down, dW_r, ring, ws,
+                      stream=None) -> int:
+    return int(lib().moe_bwd_stream_mx(ctypes.byref(shape), int(M), _ptr(X), _ptr(W_r), _ptr(wq), _nbytes(wq),
+                                       _ptr(dY), _ptr(ctx), _nbytes(ctx), _ptr(dX), _ptr(dW_gate), _ptr(dW_up),
+                                       _ptr(dW_down), _ptr(dW_r), _ptr(ring), _nbytes(ring), _ptr(ws), _nbytes(ws),
+                                       _stream(stream)))
 
 
 def moe_fwd_mx(shape, X, W_r, bias, wq, Y, ctx, ws, stream=None) -> int:
@@ -582,23 +600,72 @@ class MoEStream:
 
     def plan(self) -> dict:
         """The device plan of the last forward, split into named tables (host numpy)."""
-        import torch
-        M, El = self.M, self.El
-        n = 16 + M + (M * El + 1) + M * El + 2 * M + 4 * M + 4 * M
-        t = torch.empty(n, dtype=torch.int32, device=self.ctx.device)
-        check(moe_debug_stream_plan(self.shape, M, self.ctx, t), "moe_debug_stream_plan")
-        torch.cuda.synchronize()
-        a = t.cpu().numpy()
-        out, o = {}, 0
-        for name, size in (("plan", 16), ("mb_of", M), ("seg_poff", M * El + 1), ("cum", M * El),
-                           ("mb_range", 2 * M), ("shift_fwd", M), ("shift_bwd", M), ("replay", M),
-                           ("chunk", 4 * M), ("ring_start", M)):
-            out[name] = a[o:o + size]
-            o += size
-        return out
+        return _stream_plan(self)
 
     def error(self, stream=None) -> int:
         return moe_get_error(self.ctx, stream)
+
+
+class MoEStreamMX(MoEStream):
+    """The ring-streamed layer in MXFP8 (MOE_MXFP8: gate/up, down and both dgrads on MXFP8 tensor
+    cores, bf16 weight gradients): ctx / ring / workspace owner plus the prepared weights."""
+
+    def __init__(self, T, d, E, I, top_k, M, ring_bytes, first_local_expert=0, num_local_experts=0, device="cuda",
+                 wgrad_dtype=None):
+        import torch
+        self.wgrad_dtype = wgrad_dtype or torch.bfloat16
+        self.shape = make_shape(T, d, E, I, top_k, MOE_MXFP8, first_local_expert, num_local_experts,
+                                _wgrad_code(self.wgrad_dtype))
+        nc, nw = moe_stream_ctx_size(self.shape, M), moe_stream_workspace_size(self.shape, M)
+        nq = moe_weights_size(self.shape)
+        if nc == 0 or nw == 0 or nq == 0:
+            raise MoeError(MOE_ERR_UNSUPPORTED, "stream shape")
+        self.ctx = torch.empty(nc, dtype=torch.uint8, device=device)
+        self.ws = torch.empty(nw, dtype=torch.uint8, device=device)
+        self.wq = torch.empty(nq, dtype=torch.uint8, device=device)
+        self.ring = torch.empty(ring_bytes, dtype=torch.uint8, device=device)
+        self.T, self.d, self.E, self.I, self.k, self.M = T, d, E, I, top_k, M
+        self.El = num_local_experts or (E - first_local_expert)
+
+    def prepare(self, W_gate, W_up, W_down, stream=None):
+        _expect_layer(self, self.M * self.T, W_gate=W_gate, W_up=W_up, W_down=W_down)
+        check(moe_prepare_weights(self.shape, W_gate, W_up, W_down, self.wq, stream), "moe_prepare_weights")
+
+    def forward(self, X, W_r, bias, Y=None, stream=None):
+        import torch
+        if Y is None:
+            Y = torch.empty(self.M * self.T, self.d, dtype=torch.bfloat16, device=X.device)
+        _expect_layer(self, self.M * self.T, X=X, W_r=W_r, bias=bias, Y=Y)
+        check(moe_fwd_stream_mx(self.shape, self.M, X, W_r, bias, self.wq, Y, self.ctx, self.ring, self.ws, stream),
+              "moe_fwd_stream_mx")
+        return Y
+
+    def backward(self, X, W_r, dY, out=None, stream=None):
+        if out is None:
+            out = _grad_buffers(self.M * self.T, self.d, self.E, self.I, self.El, self.wgrad_dtype, X.device)
+        _expect_layer(self, self.M * self.T, X=X, W_r=W_r, dY=dY, out=out)
+        check(moe_bwd_stream_mx(self.shape, self.M, X, W_r, self.wq, dY, self.ctx, out["dX"], out["dW_gate"],
+                                out["dW_up"], out["dW_down"], out["dW_r"], self.ring, self.ws, stream),
+              "moe_bwd_stream_mx")
+        return out
+
+
+def _stream_plan(layer) -> dict:
+    """The device plan of a stream layer's last forward, split into named tables (host numpy)."""
+    import torch
+    M, El = layer.M, layer.El
+    n = 16 + M + (M * El + 1) + M * El + 2 * M + 4 * M + 4 * M
+    t = torch.empty(n, dtype=torch.int32, device=layer.ctx.device)
+    check(moe_debug_stream_plan(layer.shape, M, layer.ctx, t), "moe_debug_stream_plan")
+    torch.cuda.synchronize()
+    a = t.cpu().numpy()
+    out, o = {}, 0
+    for name, size in (("plan", 16), ("mb_of", M), ("seg_poff", M * El + 1), ("cum", M * El),
+                       ("mb_range", 2 * M), ("shift_fwd", M), ("shift_bwd", M), ("replay", M),
+                       ("chunk", 4 * M), ("ring_start", M)):
+        out[name] = a[o:o + size]
+        o += size
+    return out
 
 
 class MoELayer:

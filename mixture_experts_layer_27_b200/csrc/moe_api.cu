@@ -410,6 +410,20 @@ static GemmParams base_params(const Layout& L, const Ctx& c, int* status) {
   return p;
 }
 
+static MxParams mx_params(const Layout& L, const Ctx& c, int* status) {
+  MxParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.poff = c.poff;
+  p.nseg = L.El;
+  p.row_gate = c.row_gate;
+  p.row_asg = c.row_asg;
+  p.El = L.El;
+  p.d = L.d;
+  p.I = L.I;
+  p.status = status;
+  return p;
+}
+
 // dW_r = X^T . DL on the tensor cores (both operands MN-major: d and E are contiguous, the
 // contraction runs over tokens, twice: the hi and the lo bf16 terms of dl); fp32 out, one CTA
 // per 128 x 256 tile, fixed K order.  In an expert slice the tokens are the listed ones
@@ -838,9 +852,12 @@ unsigned long long moe_kernel_launches(void) { return g_launches.load(); }
 // ---------------------------------------------------------------------------
 // Ring-streamed layer: M minibatches of shape->T tokens through a fixed ring
 // ---------------------------------------------------------------------------
-static moe_status check_stream(const moe_shape* s, int32_t M, Layout* L) {
+// prec: MOE_BF16 for the bf16 entry points, MOE_MXFP8 for the MXFP8 ones, -1 for either (sizes,
+// debug).  The ring-streamed layer keeps bf16 weight gradients: MOE_MXFP8_ALL is refused.
+static moe_status check_stream(const moe_shape* s, int32_t M, Layout* L, int32_t prec = MOE_BF16) {
   if (!s || M <= 0) return MOE_ERR_INVALID_ARG;
-  if (s->prec != MOE_BF16) return is_mx_prec(s->prec) ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (s->prec != MOE_BF16 && !is_mx_prec(s->prec)) return MOE_ERR_INVALID_ARG;
+  if (s->prec == MOE_MXFP8_ALL || (prec >= 0 && s->prec != prec)) return MOE_ERR_UNSUPPORTED;
   if (!make_layout(*s, L, M)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -853,19 +870,19 @@ static int64_t minibatch_rows(const Layout& L) {
 
 size_t moe_stream_ctx_size(const moe_shape* s, int32_t M) {
   Layout L;
-  if (check_stream(s, M, &L) != MOE_OK) return 0;
+  if (check_stream(s, M, &L, -1) != MOE_OK) return 0;
   return L.ctx_bytes;
 }
 
 size_t moe_stream_workspace_size(const moe_shape* s, int32_t M) {
   Layout L;
-  if (check_stream(s, M, &L) != MOE_OK) return 0;
+  if (check_stream(s, M, &L, -1) != MOE_OK) return 0;
   return L.ws_bytes;
 }
 
 size_t moe_stream_min_ring_bytes(const moe_shape* s) {
   Layout L;
-  if (check_stream(s, 1, &L) != MOE_OK) return 0;
+  if (check_stream(s, 1, &L, -1) != MOE_OK) return 0;
   return static_cast<size_t>(minibatch_rows(L)) * L.d * 2;
 }
 
@@ -935,6 +952,9 @@ moe_status moe_fwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
   return MOE_OK;
 }
 
+static moe_status stream_wgrads(const Layout& L, const Ctx& c, int* status, const void* X, void* ring,
+                                int64_t ring_rows, void* dW_gate, void* dW_up, void* dW_down, cudaStream_t st);
+
 moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const void* W_r, const void* W_gate,
                           const void* W_up, const void* W_down, const void* dY, void* ctx, size_t ctx_bytes, void* dX,
                           void* dW_gate, void* dW_up, void* dW_down, float* dW_r, void* ring, size_t ring_bytes,
@@ -955,7 +975,6 @@ moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
     return MOE_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Ctx c = make_ctx(L, ctx, ws);
-  const int grid = num_sms();
   int* status = c.hdr + HDR_STATUS;
   const uint64_t RP = static_cast<uint64_t>(L.RP);
   const uint64_t El = static_cast<uint64_t>(L.El);
@@ -996,6 +1015,17 @@ moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
     return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
   }));
   MOE_TRY(timed(K_REV_DISPATCH, st, [&] { return launch_rev_dispatch(L, c, static_cast<__nv_bfloat16*>(dX), st); }));
+  return stream_wgrads(L, c, status, X, ring, ring_rows, dW_gate, dW_up, dW_down, st);
+}
+
+// Weight gradients of a ring-streamed backward: W_down's over every row of the stream (Hg and
+// dY_perm), W_gate / W_up's walking the ring in reverse, chunk by chunk (replaying the macrobatches
+// the forward overwrote), into the fp32 accumulator, then rounded once.
+static moe_status stream_wgrads(const Layout& L, const Ctx& c, int* status, const void* X, void* ring,
+                                int64_t ring_rows, void* dW_gate, void* dW_up, void* dW_down, cudaStream_t st) {
+  const int grid = num_sms();
+  const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
+  const int nseg = L.M * L.El;
   {  // wgrad of W_down: Hg and dY_perm cover the whole stream
     GemmParams p = base_params(L, c, status);
     p.poff = c.tab.seg_poff;
@@ -1037,9 +1067,165 @@ moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
   return MOE_OK;
 }
 
+// MXFP8 ring-streamed layer: the bf16 stream's macrobatches, ring and backward chunks, with the
+// gate/up, down and both dgrad GEMMs on the MX engine.  The forward's dispatch writes each
+// macrobatch's rows to the ring in bf16 (the weight gradients' operand, replayed as in the bf16
+// stream) and their codes along d at their padded rows (the gate/up GEMM's operand).
+static moe_status check_stream_mx_args(const moe_shape* s, int32_t M, Layout* L, const void* wq, size_t wq_bytes,
+                                       size_t ctx_bytes, size_t ws_bytes, size_t ring_bytes, int64_t* ring_rows) {
+  const moe_status cs = check_stream(s, M, L, MOE_MXFP8);
+  if (cs != MOE_OK) return cs;
+  if (!wq || !aligned16(wq)) return MOE_ERR_INVALID_ARG;
+  *ring_rows = static_cast<int64_t>(ring_bytes / (static_cast<size_t>(L->d) * 2));
+  if (ctx_bytes < L->ctx_bytes || ws_bytes < L->ws_bytes || wq_bytes < L->wq_bytes ||
+      *ring_rows < minibatch_rows(*L) || *ring_rows >= (int64_t(1) << 31))
+    return MOE_ERR_WORKSPACE_TOO_SMALL;
+  return MOE_OK;
+}
+
+moe_status moe_fwd_stream_mx(const moe_shape* s, int32_t M, const void* X, const void* W_r, const float* bias,
+                             const void* wq, size_t wq_bytes, void* Y, void* ctx, size_t ctx_bytes, void* ring,
+                             size_t ring_bytes, void* ws, size_t ws_bytes, void* stream) {
+  Layout L;
+  int64_t ring_rows = 0;
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (!X || !Y || !W_r || !ctx || !ring || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W_r) || !aligned16(Y) || !aligned16(ctx) || !aligned16(ring) || !aligned16(ws) ||
+      (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+    return MOE_ERR_INVALID_ARG;
+  const moe_status cs = check_stream_mx_args(s, M, &L, wq, wq_bytes, ctx_bytes, ws_bytes, ring_bytes, &ring_rows);
+  if (cs != MOE_OK) return cs;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ctx c = make_ctx(L, ctx, ws);
+  MOE_TRY(cudaMemsetAsync(c.hdr, 0, HDR_WORDS * 4, st));
+  {
+    const moe_status r = route_tokens(L, c, X, W_r, bias, static_cast<int>(ring_rows), st);
+    if (r != MOE_OK) return r;
+  }
+  const int grid = num_sms();
+  int* status = c.hdr + HDR_STATUS;
+  const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
+  const auto* w = static_cast<const uint8_t*>(wq);
+  CUtensorMap xq_map, wgu_map, hq_map, wd_map;
+  MOE_TMAP(tmap_fp8(&xq_map, c.xq, L.d, RP, 128));
+  MOE_TMAP(tmap_fp8(&wgu_map, w + L.wgu1, L.d, El * 2 * L.I, mx_bn(MX_GATEUP)));
+  MOE_TMAP(tmap_fp8(&hq_map, c.hq, L.I, RP, 128));
+  MOE_TMAP(tmap_fp8(&wd_map, w + L.wd2, L.I, El * L.d, mx_bn(MX_DOWN)));
+  // Macrobatches walk the ring forward; launches past the plan's count find empty segments and exit.
+  for (int m = 0; m < M; ++m) {
+    const int* seg = c.tab.seg_poff + m * L.El;
+    MOE_TRY(timed(K_DISPATCH, st, [&] {
+      return launch_gather_range_mx(L, c, static_cast<const __nv_bfloat16*>(X), seg, seg + L.El,
+                                    c.tab.shift_fwd + m, ring_rows, static_cast<__nv_bfloat16*>(ring), c.xq, c.xqs,
+                                    st);
+    }));
+    {
+      MxParams p = mx_params(L, c, status);
+      p.poff = seg;
+      p.ta0 = p.ta1 = xq_map;
+      p.tb0 = p.tb1 = wgu_map;
+      p.sfa0 = p.sfa1 = c.xqs;
+      p.sfb0 = p.sfb1 = w + L.wgu1s;
+      p.out0 = c.abuf;
+      p.out1 = c.bbuf;
+      p.q0 = c.hq;
+      p.qs0 = c.hqs;
+      MOE_TRY(timed(K_GEMM_GATEUP, st, [&] { return launch_gemm_mx(MX_GATEUP, p, grid, st); }));
+    }
+    {
+      MxParams p = mx_params(L, c, status);
+      p.poff = seg;
+      p.ta0 = p.ta1 = hq_map;
+      p.tb0 = p.tb1 = wd_map;
+      p.sfa0 = p.sfa1 = c.hqs;
+      p.sfb0 = p.sfb1 = w + L.wd2s;
+      p.out0 = c.obuf;
+      MOE_TRY(timed(K_GEMM_DOWN, st, [&] { return launch_gemm_mx(MX_DOWN, p, grid, st); }));
+    }
+    MOE_TRY(timed(K_COMBINE, st, [&] {
+      return launch_combine(L, c, c.obuf, static_cast<__nv_bfloat16*>(Y), st, c.tab.mb_range + 2 * m);
+    }));
+  }
+  return MOE_OK;
+}
+
+moe_status moe_bwd_stream_mx(const moe_shape* s, int32_t M, const void* X, const void* W_r, const void* wq,
+                             size_t wq_bytes, const void* dY, void* ctx, size_t ctx_bytes, void* dX, void* dW_gate,
+                             void* dW_up, void* dW_down, float* dW_r, void* ring, size_t ring_bytes, void* ws,
+                             size_t ws_bytes, void* stream) {
+  Layout L;
+  int64_t ring_rows = 0;
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (!X || !dY || !dX || !W_r || !ctx || !dW_gate || !dW_up || !dW_down || !dW_r || !ring || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W_r) || !aligned16(dY) || !aligned16(ctx) || !aligned16(dX) ||
+      !aligned16(dW_gate) || !aligned16(dW_up) || !aligned16(dW_down) || !aligned16(dW_r) || !aligned16(ring) ||
+      !aligned16(ws))
+    return MOE_ERR_INVALID_ARG;
+  const moe_status cs = check_stream_mx_args(s, M, &L, wq, wq_bytes, ctx_bytes, ws_bytes, ring_bytes, &ring_rows);
+  if (cs != MOE_OK) return cs;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ctx c = make_ctx(L, ctx, ws);
+  const int grid = num_sms();
+  int* status = c.hdr + HDR_STATUS;
+  const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
+  const int nseg = L.M * L.El;
+  const auto* w = static_cast<const uint8_t*>(wq);
+  // reverse-combine over every row of the stream: bf16 (the W_down weight gradient's operand) and
+  // codes along d (the dgrad of W_down's operand)
+  MOE_TRY(timed(K_REV_COMBINE, st, [&] {
+    return launch_gather_rows_mx(L, c, static_cast<const __nv_bfloat16*>(dY), c.dyperm, c.dyq, c.dyqs, st);
+  }));
+  {
+    MxParams p = mx_params(L, c, status);
+    p.poff = c.tab.seg_poff;
+    p.nseg = nseg;
+    MOE_TMAP(tmap_fp8(&p.ta0, c.dyq, L.d, RP, 128));
+    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wd3, L.d, El * L.I, mx_bn(MX_DGRAD_DOWN)));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.sfa0 = p.sfa1 = c.dyqs;
+    p.sfb0 = p.sfb1 = w + L.wd3s;
+    p.in0 = c.abuf;
+    p.in1 = c.bbuf;
+    p.out0 = c.dabuf;
+    p.out1 = c.dbbuf;
+    p.out2 = c.hgbuf;
+    p.q0 = c.daq;
+    p.qs0 = c.daqs;
+    p.q1 = c.dbq;
+    p.qs1 = c.dbqs;
+    p.outf = c.dgpart;
+    MOE_TRY(timed(K_GEMM_DGRAD_DOWN, st, [&] { return launch_gemm_mx(MX_DGRAD_DOWN, p, grid, st); }));
+  }
+  MOE_TRY_STATUS(router_backward(L, c, X, dW_r, status, st, L.I / mx_bn(MX_DGRAD_DOWN)));
+  MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
+    return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
+  }));
+  {
+    MxParams p = mx_params(L, c, status);
+    p.poff = c.tab.seg_poff;
+    p.nseg = nseg;
+    MOE_TMAP(tmap_fp8(&p.ta0, c.daq, L.I, RP, 128));
+    MOE_TMAP(tmap_fp8(&p.ta1, c.dbq, L.I, RP, 128));
+    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wg4, L.I, El * L.d, mx_bn(MX_DGRAD_GATEUP)));
+    MOE_TMAP(tmap_fp8(&p.tb1, w + L.wu4, L.I, El * L.d, mx_bn(MX_DGRAD_GATEUP)));
+    p.sfa0 = c.daqs;
+    p.sfa1 = c.dbqs;
+    p.sfb0 = w + L.wg4s;
+    p.sfb1 = w + L.wu4s;
+    p.out0 = c.dxperm;
+    MOE_TRY(timed(K_GEMM_DGRAD_GATEUP, st, [&] { return launch_gemm_mx(MX_DGRAD_GATEUP, p, grid, st); }));
+  }
+  MOE_TRY(timed(K_REV_DISPATCH, st, [&] { return launch_rev_dispatch(L, c, static_cast<__nv_bfloat16*>(dX), st); }));
+  // bf16 weight gradients exactly as the bf16 stream: W_down's over every row, gate/up's walking
+  // the ring in reverse, chunk by chunk, into the fp32 accumulator
+  return stream_wgrads(L, c, status, X, ring, ring_rows, dW_gate, dW_up, dW_down, st);
+}
+
 moe_status moe_debug_stream_plan(const moe_shape* s, int32_t M, const void* ctx, int32_t* tables, void* stream) {
   Layout L;
-  const moe_status cs = check_stream(s, M, &L);
+  const moe_status cs = check_stream(s, M, &L, -1);
   if (cs != MOE_OK) return cs;
   if (!ctx || !tables) return MOE_ERR_INVALID_ARG;
   MOE_TRY(cudaMemcpyAsync(tables, static_cast<const char*>(ctx) + L.stab,
@@ -1089,19 +1275,6 @@ moe_status moe_prepare_weights(const moe_shape* s, const void* W_gate, const voi
   return MOE_OK;
 }
 
-static MxParams mx_params(const Layout& L, const Ctx& c, int* status) {
-  MxParams p;
-  std::memset(&p, 0, sizeof(p));
-  p.poff = c.poff;
-  p.nseg = L.El;
-  p.row_gate = c.row_gate;
-  p.row_asg = c.row_asg;
-  p.El = L.El;
-  p.d = L.d;
-  p.I = L.I;
-  p.status = status;
-  return p;
-}
 
 // MXFP8 weight gradients from operands quantised along the rows (blocks of 32 rows of one expert,
 // K-major in 128-row tiles): X by the forward's dispatch, dY by the reverse-combine, dA, dB and Hg

@@ -322,6 +322,10 @@ cudaError_t launch_quant_weight(int mode, const __nv_bfloat16* src0, const __nv_
                                 int N, uint8_t* q, uint8_t* qs, cudaStream_t st);
 cudaError_t launch_gather_rows_mx(const Layout& L, const Ctx& c, const __nv_bfloat16* src, __nv_bfloat16* dst,
                                   uint8_t* q, uint8_t* qs, cudaStream_t st);
+// rows [*lo, *hi): bf16 to dst row + *shift (a ring position; shift may be NULL), codes at the row
+cudaError_t launch_gather_range_mx(const Layout& L, const Ctx& c, const __nv_bfloat16* src, const int* lo,
+                                   const int* hi, const int* shift, int64_t max_rows, __nv_bfloat16* dst, uint8_t* q,
+                                   uint8_t* qs, cudaStream_t st);
 // Dispatch / reverse-combine with MXFP8 weight gradients: the padded rows gathered from src and
 // quantised along d (qd, qds as launch_gather_rows_mx writes them) and along the rows in blocks of
 // 32 (qr, qrs: rowq layout), no bf16 copy.

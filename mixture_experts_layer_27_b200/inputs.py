@@ -10,6 +10,7 @@ Workloads (the pages name model families and print no shapes; these stand in):
 * ``kimi``      T=4096, d=7168, E=384, k=8, I=2048   (Kimi-K2-like, Zipf(1.2)-skewed load)
 * ``kimi_mx``   ``kimi`` in MXFP8 mode
 * ``ep64``      6 local experts of 384, 16 minibatches x 2048 tokens, ring buffer
+* ``ep64mx``  the ring-streamed slice in MXFP8
 * ``epmx``, ``epbf``  the same slice as one batch of 32768 tokens (MXFP8 / bf16), no ring
 * ``dsv3_e16``  the dsv3 expert shape with 16 experts and 128 tokens (profiler captures)
 * ``kimi_mx_e24`` the kimi expert shape in MXFP8, 24 experts, 256 tokens (profiler captures)
@@ -79,6 +80,10 @@ WORKLOADS = {
 for _n in (512, 1024, 2048, 2368, 4096, 8192, 16384):
     WORKLOADS[f"ep64_n{_n}"] = Workload(f"ep64_n{_n}", 2048, 7168, 384, 8, 2048, first_local=0, num_local=6,
                                         stream_M=16, ring_bytes=256 << 20, local_tokens=_n)
+# The same ring-streamed slice in MXFP8 (gate/up, down and both dgrads on MXFP8, bf16 weight gradients)
+for _n in (512, 2368, 4096):
+    WORKLOADS[f"ep64mx_n{_n}"] = Workload(f"ep64mx_n{_n}", 2048, 7168, 384, 8, 2048, mxfp8=True, first_local=0,
+                                          num_local=6, stream_M=16, ring_bytes=256 << 20, local_tokens=_n)
 # The same per-rank slice (6 of 384 experts, 32768 tokens, n per local expert) as one batch, the
 # dispatched rows held whole instead of in a ring: MXFP8 (epmx) and bf16 (epbf), the regime
 # where the grouped GEMMs are bound by the tensor cores rather than by the weight stream.

@@ -109,8 +109,44 @@ def test_stream_shapes_and_sizes():
         assert B.moe_stream_ctx_size(s, M) == 0 and B.moe_stream_workspace_size(s, M) == 0
     ragged = B.make_shape(2050, 7168, 384, 2048, 8)  # minibatches are whole 16-token blocks
     assert B.moe_stream_ctx_size(ragged, 4) == 0 and B.moe_stream_min_ring_bytes(ragged) == 0
-    mx = B.make_shape(2048, 7168, 384, 2048, 8, prec=B.MOE_MXFP8)  # the ring stream is bf16 only
-    assert B.moe_stream_ctx_size(mx, 4) == 0
+    # MXFP8 streams (bf16 weight gradients) are sized like the bf16 ones plus their fp8 operands;
+    # MXFP8 weight gradients are one-batch only
+    mx = B.make_shape(2048, 7168, 384, 2048, 8, prec=B.MOE_MXFP8)
+    bf = B.make_shape(2048, 7168, 384, 2048, 8)
+    assert B.moe_stream_ctx_size(mx, 4) > B.moe_stream_ctx_size(bf, 4) > 0
+    assert B.moe_stream_workspace_size(mx, 4) > B.moe_stream_workspace_size(bf, 4) > 0
+    assert B.moe_stream_min_ring_bytes(mx) == B.moe_stream_min_ring_bytes(bf)
+    mxa = B.make_shape(2048, 7168, 384, 2048, 8, prec=B.MOE_MXFP8_ALL)
+    assert B.moe_stream_ctx_size(mxa, 4) == 0 and B.moe_stream_workspace_size(mxa, 4) == 0
+
+
+def test_stream_mx_argument_errors_are_synchronous(lib):
+    s = B.make_shape(128, 256, 16, 256, 4, prec=B.MOE_MXFP8)
+    M = 4
+    nc, nw, nr = B.moe_stream_ctx_size(s, M), B.moe_stream_workspace_size(s, M), B.moe_stream_min_ring_bytes(s)
+    nq = B.moe_weights_size(s)
+    f = 1 << 20  # never dereferenced
+
+    def fwd(shape=s, wq_bytes=nq, ring_bytes=nr, X=f, wq=f):
+        return lib.moe_fwd_stream_mx(ctypes.byref(shape), M, X, f, None, wq, wq_bytes, f, f, nc, f, ring_bytes, f, nw,
+                                     None)
+
+    def bwd(shape=s, wq_bytes=nq):
+        return lib.moe_bwd_stream_mx(ctypes.byref(shape), M, f, f, f, wq_bytes, f, f, nc, f, f, f, f, f, f, nr, f, nw,
+                                     None)
+
+    assert fwd(X=None) == B.MOE_ERR_INVALID_ARG
+    assert fwd(wq=None) == B.MOE_ERR_INVALID_ARG
+    assert fwd(wq_bytes=nq - 1) == B.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert fwd(ring_bytes=nr - 2 * 256) == B.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert bwd(wq_bytes=nq - 1) == B.MOE_ERR_WORKSPACE_TOO_SMALL
+    bf = B.make_shape(128, 256, 16, 256, 4)  # the MX entry points take MXFP8 shapes only
+    assert fwd(shape=bf) == B.MOE_ERR_UNSUPPORTED and bwd(shape=bf) == B.MOE_ERR_UNSUPPORTED
+    mxa = B.make_shape(128, 256, 16, 256, 4, prec=B.MOE_MXFP8_ALL)
+    assert fwd(shape=mxa) == B.MOE_ERR_UNSUPPORTED
+    # and the bf16 entry points refuse MXFP8 shapes
+    assert lib.moe_fwd_stream(ctypes.byref(s), M, f, f, None, f, f, f, f, f, nc, f, nr, f, nw, None) == \
+        B.MOE_ERR_UNSUPPORTED
 
 
 def test_stream_argument_errors_are_synchronous(lib):

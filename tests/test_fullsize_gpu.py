@@ -333,6 +333,51 @@ def test_full_size_mxfp8_weight_gradients_kimi():
     torch.cuda.empty_cache()
 
 
+def test_full_size_ep64_ring_stream_mx():
+    # Config 5 at n = 4096 in MXFP8: the ring replays part of the stream and the gate/up weight
+    # gradient accumulates over two chunks.  Y, dX and dW_r equal the one-batch MXFP8 layer's over
+    # the same 32768 tokens bit for bit; the weight gradients equal them to fp32 summation order.
+    w = IN.WORKLOADS["ep64mx_n4096"]
+    x = IN.make_inputs(w, device="cuda")
+    first, El = w.first_local, w.El
+
+    def run():
+        s = B.MoEStreamMX(w.T, w.d, w.E, w.I, w.k, w.stream_M, w.ring_bytes, first, w.num_local)
+        s.prepare(x["W_gate"], x["W_up"], x["W_down"])
+        Y = s.forward(x["X"], x["W_r"], x["bias"])
+        g = s.backward(x["X"], x["W_r"], x["dY"])
+        torch.cuda.synchronize()
+        assert s.error() == B.MOE_OK
+        return s, Y, g
+
+    s, Y, g = run()
+    hdr = s.plan()["plan"]
+    assert hdr[1] > 1 and hdr[3] > 0  # several backward chunks, replayed rows
+    del s
+    torch.cuda.empty_cache()
+    lay = B.MoELayerMX(w.tokens, w.d, w.E, w.I, w.k, first, w.num_local)
+    lay.prepare(x["W_gate"], x["W_up"], x["W_down"])
+    Y1 = lay.forward(x["X"], x["W_r"], x["bias"])
+    g1 = lay.backward(x["X"], x["W_r"], x["dY"])
+    torch.cuda.synchronize()
+    assert lay.error() == B.MOE_OK
+    del lay
+    torch.cuda.empty_cache()
+    assert torch.equal(Y.view(torch.int16), Y1.view(torch.int16))
+    assert torch.equal(g["dX"].view(torch.int16), g1["dX"].view(torch.int16))
+    assert torch.equal(g["dW_r"].view(torch.int32), g1["dW_r"].view(torch.int32))
+    for n in ("dW_gate", "dW_up", "dW_down"):
+        assert relerr(to64(g[n]), to64(g1[n])) <= 1e-2, n
+    del Y1, g1
+    # a second run is bit-identical
+    _, Y2, g2 = run()
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+    for n in ("dX", "dW_gate", "dW_up", "dW_down"):
+        assert torch.equal(g[n].view(torch.int16), g2[n].view(torch.int16)), n
+    del Y, Y2, g, g2, x
+    torch.cuda.empty_cache()
+
+
 def test_full_size_ep64_ring_stream():
     # Config 5 at n = 4096 tokens per local expert: 16 minibatches of 2048 tokens through the
     # 256 MiB ring, 6 local experts of 384; the backward replays part of the stream into the

@@ -1,0 +1,85 @@
+"""The ring-streamed layer in MXFP8 (moe_fwd_stream_mx / moe_bwd_stream_mx) on the GPU.
+
+The stream changes where rows live and when each macrobatch runs, not the arithmetic of a row:
+every GEMM output row, its quantisation along d or I, the combine and the reverse dispatch are
+row-local, so Y, dX and dW_r must equal the one-batch MXFP8 layer's over the same M*T tokens bit
+for bit.  The weight gradients contract over rows in chunks with an fp32 accumulator, so they
+differ from the one-batch layer's by fp32 summation order only (checked at 1e-2), and they are
+checked against the MXFP8 oracle at 6e-2.  Small rings force replay and several backward
+chunks; a large ring keeps everything resident; a local expert slice; reruns are bit-identical.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from mixture_experts_layer_27_b200 import binding as B
+
+from _util import make_case, relerr, to64
+
+pytestmark = pytest.mark.gpu
+TOL_MX = 6e-2
+
+
+def _bits(t):
+    return t.view(torch.int16) if t.dtype == torch.bfloat16 else t.view(torch.int32)
+
+
+def _one_batch(x, T, d, E, I, k, first, num, El):
+    lay = B.MoELayerMX(T, d, E, I, k, first_local_expert=first, num_local_experts=num)
+    lay.prepare(*(x[n][first:first + El].contiguous() for n in ("W_gate", "W_up", "W_down")))
+    Y = lay.forward(x["X"], x["W_r"], x["bias"])
+    g = lay.backward(x["X"], x["W_r"], x["dY"])
+    torch.cuda.synchronize()
+    assert lay.error() == B.MOE_OK
+    return Y, g
+
+
+@pytest.mark.parametrize("T_mb,M,d,E,k,I,first,num,ring_mult,seed", [
+    (128, 8, 256, 16, 4, 256, 0, 0, 1.0, 71),    # smallest legal ring: replay, several chunks
+    (128, 8, 256, 16, 4, 256, 0, 0, 100.0, 72),  # everything stays resident
+    (64, 10, 512, 24, 6, 512, 3, 6, 1.5, 73),    # a local expert slice (6 of 24)
+])
+def test_mx_streamed_layer(T_mb, M, d, E, k, I, first, num, ring_mult, seed):
+    T = T_mb * M
+    w, x = make_case(T, d, E, k, I, seed=seed)
+    El = num or E - first
+    shape = B.make_shape(T_mb, d, E, I, k, prec=B.MOE_MXFP8, first_local_expert=first, num_local_experts=num)
+    ring_bytes = int(B.moe_stream_min_ring_bytes(shape) * ring_mult) // (2 * d) * (2 * d)
+    s = B.MoEStreamMX(T_mb, d, E, I, k, M, ring_bytes, first, num)
+    s.ctx.fill_(0xFF)  # NaN patterns wherever the step reads before it writes
+    s.ws.fill_(0xFF)
+    s.ring.fill_(0xFF)
+    s.prepare(*(x[n][first:first + El].contiguous() for n in ("W_gate", "W_up", "W_down")))
+
+    def run():
+        Y = s.forward(x["X"], x["W_r"], x["bias"])
+        g = s.backward(x["X"], x["W_r"], x["dY"])
+        torch.cuda.synchronize()
+        assert s.error() == B.MOE_OK
+        return Y, g
+
+    Y, g = run()
+    Y1, g1 = _one_batch(x, T, d, E, I, k, first, num, El)
+    assert torch.equal(_bits(Y), _bits(Y1))
+    for n in ("dX", "dW_r"):
+        assert torch.equal(_bits(g[n]), _bits(g1[n])), n
+    for n in ("dW_gate", "dW_up", "dW_down"):
+        assert relerr(to64(g[n]), to64(g1[n])) <= 1e-2, n
+    # against the MXFP8 oracle (bf16 weight gradients)
+    f64 = {n: (None if x[n] is None else to64(x[n])) for n in ("X", "W_r", "bias", "W_gate", "W_up", "W_down", "dY")}
+    Yq, cq = O.forward_mx(f64["X"], f64["W_r"], f64["bias"], f64["W_gate"], f64["W_up"], f64["W_down"], k,
+                          first_local=first, num_local=num or None)
+    gq = O.backward_mx(cq, f64["dY"])
+    errs = {"Y": relerr(to64(Y), Yq), "dX": relerr(to64(g["dX"]), gq["dX"])}
+    for n in ("dW_gate", "dW_up", "dW_down"):
+        errs[n] = relerr(to64(g[n]), np.stack([gq[n][first + e] for e in range(El)]))
+    assert all(v <= TOL_MX for v in errs.values()), errs
+    plan = s.plan()["plan"]
+    if ring_mult == 1.0:
+        assert plan[1] > 1  # several backward chunks: the ring was overwritten and replayed
+    # a second run over the same buffers: the same bits
+    Y2, g2 = run()
+    assert torch.equal(_bits(Y2), _bits(Y))
+    for n in g:
+        assert torch.equal(_bits(g2[n]), _bits(g[n])), n
