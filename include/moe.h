@@ -312,10 +312,12 @@ moe_status moe_bwd_stream(const moe_shape* shape, int32_t num_minibatches, const
  * replay[M], chunk[4M] ({m_lo, m_hi, valid, mode}), ring_start[M]. */
 /* MXFP8 ring-streamed layer (shape->prec = MOE_MXFP8): the same plan, ring and backward chunks as
  * moe_fwd_stream / moe_bwd_stream, with the gate/up, down and both dgrad GEMMs on MXFP8 from the
- * prepared weights `wq` (moe_prepare_weights of this shape); the forward's dispatch writes each
- * macrobatch's rows to the ring in bf16 and quantises them along d.  The weight gradients stay bf16
- * (MOE_MXFP8_ALL shapes are refused: MOE_ERR_UNSUPPORTED).  ctx / ws / ring sizes: the
- * moe_stream_* size calls of this shape.  Same errors as the bf16 stream. */
+ * prepared weights `wq` (moe_prepare_weights of this shape); the weight gradients stay bf16
+ * (MOE_MXFP8_ALL shapes are refused: MOE_ERR_UNSUPPORTED).  A ring row holds the bf16 row, its E4M3
+ * codes along d and their scales (2d + d + d/32 bytes): the ring holds R = ring_bytes / (3d + d/32)
+ * rows rounded down to a multiple of 128, laid out as R bf16 rows, R code rows, then the codes' scale
+ * chunks.  ctx / ws / minimum ring sizes: the moe_stream_* size calls of this shape.  Same errors as
+ * the bf16 stream. */
 moe_status moe_fwd_stream_mx(const moe_shape* shape, int32_t num_minibatches, const void* X, const void* W_r,
                              const float* bias, const void* wq, size_t wq_bytes, void* Y, void* ctx, size_t ctx_bytes,
                              void* ring, size_t ring_bytes, void* ws, size_t ws_bytes, void* stream);

@@ -156,9 +156,10 @@ __device__ __forceinline__ void mx_load(const MxParams& p, const MxTile& tl, int
     brow = tl.el * p.d + tl.n0;
     KA = KB = p.I;
   }
-  tma_load_2d(sA, ma, bar, kl * 128, tl.m0, pol_act);
+  const int arow = tl.m0 + (p.ring_shift ? __ldg(p.ring_shift) : 0);  // the A operand's row (ring position)
+  tma_load_2d(sA, ma, bar, kl * 128, arow, pol_act);
   tma_load_2d(sB, mb, bar, kl * 128, brow, pol_w);
-  bulk_load(sSF, sfa + (static_cast<size_t>(tl.m0 >> 7) * (KA >> 7) + kl) * 512, 512, bar);
+  bulk_load(sSF, sfa + (static_cast<size_t>(arow >> 7) * (KA >> 7) + kl) * 512, 512, bar);
   bulk_load(sSF + 512, sfb + (static_cast<size_t>(brow >> 7) * (KB >> 7) + kl) * 512, 512, bar);
   if constexpr (BN == 256)
     bulk_load(sSF + 1024, sfb + (static_cast<size_t>((brow >> 7) + 1) * (KB >> 7) + kl) * 512, 512, bar);

@@ -75,8 +75,9 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->bbuf = take(RP * s.I * 2);
   L->stab = take(M > 0 ? static_cast<size_t>(stream_table_words(M, El)) * 4 : 0);
   const size_t mxd = L->mx ? RP * s.d : 0, mxi = L->mx ? RP * s.I : 0;  // fp8 bytes; scales are 1/32 of that
-  L->xq = take(mxd);
-  L->xqs = take(mxd / 32);
+  // the one-batch MXFP8 forward's X codes (a ring-streamed layer keeps them in the caller's ring)
+  L->xq = take(M > 0 ? 0 : mxd);
+  L->xqs = take(M > 0 ? 0 : mxd / 32);
   const size_t wxd = L->mxw ? RP * s.d : 0, wxi = L->mxw ? RP * s.I : 0;
   L->xqt = take(wxd);  // X along the rows, from the forward's dispatch for the weight gradients
   L->xqts = take(wxd / 32);
@@ -880,10 +881,21 @@ size_t moe_stream_workspace_size(const moe_shape* s, int32_t M) {
   return L.ws_bytes;
 }
 
+// Bytes of the caller's ring per row: the bf16 row, and in MXFP8 its codes along d and their
+// scales (the ring holds ring_rows bf16 rows, then ring_rows code rows, then their scale chunks).
+static size_t ring_row_bytes(const Layout& L) {
+  return static_cast<size_t>(L.d) * 2 + (L.mx ? static_cast<size_t>(L.d) + L.d / 32 : 0);
+}
+// Rows of a ring of ring_bytes; in MXFP8 a multiple of 128 (the scale chunks cover 128-row tiles).
+static int64_t ring_rows_of(const Layout& L, size_t ring_bytes) {
+  const int64_t r = static_cast<int64_t>(ring_bytes / ring_row_bytes(L));
+  return L.mx ? r / 128 * 128 : r;
+}
+
 size_t moe_stream_min_ring_bytes(const moe_shape* s) {
   Layout L;
   if (check_stream(s, 1, &L, -1) != MOE_OK) return 0;
-  return static_cast<size_t>(minibatch_rows(L)) * L.d * 2;
+  return static_cast<size_t>(minibatch_rows(L)) * ring_row_bytes(L);
 }
 
 moe_status moe_fwd_stream(const moe_shape* s, int32_t M, const void* X, const void* W_r, const float* bias,
@@ -1070,13 +1082,14 @@ static moe_status stream_wgrads(const Layout& L, const Ctx& c, int* status, cons
 // MXFP8 ring-streamed layer: the bf16 stream's macrobatches, ring and backward chunks, with the
 // gate/up, down and both dgrad GEMMs on the MX engine.  The forward's dispatch writes each
 // macrobatch's rows to the ring in bf16 (the weight gradients' operand, replayed as in the bf16
-// stream) and their codes along d at their padded rows (the gate/up GEMM's operand).
+// stream) and their codes along d to the same ring rows of the ring's code region (the gate/up
+// GEMM's operand; ring positions are multiples of 128 rows, so the scale chunks stay whole).
 static moe_status check_stream_mx_args(const moe_shape* s, int32_t M, Layout* L, const void* wq, size_t wq_bytes,
                                        size_t ctx_bytes, size_t ws_bytes, size_t ring_bytes, int64_t* ring_rows) {
   const moe_status cs = check_stream(s, M, L, MOE_MXFP8);
   if (cs != MOE_OK) return cs;
   if (!wq || !aligned16(wq)) return MOE_ERR_INVALID_ARG;
-  *ring_rows = static_cast<int64_t>(ring_bytes / (static_cast<size_t>(L->d) * 2));
+  *ring_rows = ring_rows_of(*L, ring_bytes);
   if (ctx_bytes < L->ctx_bytes || ws_bytes < L->ws_bytes || wq_bytes < L->wq_bytes ||
       *ring_rows < minibatch_rows(*L) || *ring_rows >= (int64_t(1) << 31))
     return MOE_ERR_WORKSPACE_TOO_SMALL;
@@ -1106,8 +1119,11 @@ moe_status moe_fwd_stream_mx(const moe_shape* s, int32_t M, const void* X, const
   int* status = c.hdr + HDR_STATUS;
   const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
   const auto* w = static_cast<const uint8_t*>(wq);
+  // the ring: ring_rows bf16 rows, then their codes, then the codes' scale chunks
+  uint8_t* ring_q = static_cast<uint8_t*>(ring) + static_cast<size_t>(ring_rows) * L.d * 2;
+  uint8_t* ring_qs = ring_q + static_cast<size_t>(ring_rows) * L.d;
   CUtensorMap xq_map, wgu_map, hq_map, wd_map;
-  MOE_TMAP(tmap_fp8(&xq_map, c.xq, L.d, RP, 128));
+  MOE_TMAP(tmap_fp8(&xq_map, ring_q, L.d, static_cast<uint64_t>(ring_rows), 128));
   MOE_TMAP(tmap_fp8(&wgu_map, w + L.wgu1, L.d, El * 2 * L.I, mx_bn(MX_GATEUP)));
   MOE_TMAP(tmap_fp8(&hq_map, c.hq, L.I, RP, 128));
   MOE_TMAP(tmap_fp8(&wd_map, w + L.wd2, L.I, El * L.d, mx_bn(MX_DOWN)));
@@ -1116,15 +1132,16 @@ moe_status moe_fwd_stream_mx(const moe_shape* s, int32_t M, const void* X, const
     const int* seg = c.tab.seg_poff + m * L.El;
     MOE_TRY(timed(K_DISPATCH, st, [&] {
       return launch_gather_range_mx(L, c, static_cast<const __nv_bfloat16*>(X), seg, seg + L.El,
-                                    c.tab.shift_fwd + m, ring_rows, static_cast<__nv_bfloat16*>(ring), c.xq, c.xqs,
-                                    st);
+                                    c.tab.shift_fwd + m, true, ring_rows, static_cast<__nv_bfloat16*>(ring), ring_q,
+                                    ring_qs, st);
     }));
     {
       MxParams p = mx_params(L, c, status);
       p.poff = seg;
+      p.ring_shift = c.tab.shift_fwd + m;
       p.ta0 = p.ta1 = xq_map;
       p.tb0 = p.tb1 = wgu_map;
-      p.sfa0 = p.sfa1 = c.xqs;
+      p.sfa0 = p.sfa1 = ring_qs;
       p.sfb0 = p.sfb1 = w + L.wgu1s;
       p.out0 = c.abuf;
       p.out1 = c.bbuf;

@@ -232,6 +232,9 @@ struct MxParams {
   // bf16 dA, dB, Hg are then not written: out0..out2 NULL)
   uint8_t* tq[3];
   uint8_t* tqs[3];
+  // gate/up GEMM of a ring-streamed macrobatch: the A operand's codes and scale chunks sit at ring
+  // row = padded row + *ring_shift (a multiple of 128); NULL: at the padded row
+  const int* ring_shift;
 };
 __host__ __device__ constexpr bool mx_is_wgrad(int kind) { return kind == MX_WGRAD_GATEUP || kind == MX_WGRAD_DOWN; }
 // Tile width per kind: 128 x 256 tiles (one accumulator, four stages) keep 32 KB of fp8 weights
@@ -322,10 +325,11 @@ cudaError_t launch_quant_weight(int mode, const __nv_bfloat16* src0, const __nv_
                                 int N, uint8_t* q, uint8_t* qs, cudaStream_t st);
 cudaError_t launch_gather_rows_mx(const Layout& L, const Ctx& c, const __nv_bfloat16* src, __nv_bfloat16* dst,
                                   uint8_t* q, uint8_t* qs, cudaStream_t st);
-// rows [*lo, *hi): bf16 to dst row + *shift (a ring position; shift may be NULL), codes at the row
+// rows [*lo, *hi): bf16 to dst row + *shift (a ring position; shift may be NULL), codes at the row,
+// or at the ring position too with shift_codes
 cudaError_t launch_gather_range_mx(const Layout& L, const Ctx& c, const __nv_bfloat16* src, const int* lo,
-                                   const int* hi, const int* shift, int64_t max_rows, __nv_bfloat16* dst, uint8_t* q,
-                                   uint8_t* qs, cudaStream_t st);
+                                   const int* hi, const int* shift, bool shift_codes, int64_t max_rows,
+                                   __nv_bfloat16* dst, uint8_t* q, uint8_t* qs, cudaStream_t st);
 // Dispatch / reverse-combine with MXFP8 weight gradients: the padded rows gathered from src and
 // quantised along d (qd, qds as launch_gather_rows_mx writes them) and along the rows in blocks of
 // 32 (qr, qrs: rowq layout), no bf16 copy.

@@ -108,12 +108,13 @@ __global__ void __launch_bounds__(128) k_quant_weight(const __nv_bfloat16* __res
 }
 
 // Dispatch / reverse-combine in MXFP8 mode: rows [lo, hi) of the padded layout get the bf16 row
-// (kept for the weight gradients; at row R + *shift when a ring position is given) and its fp8
-// codes + scales along d (at row R); dead pad rows are skipped.
+// (kept for the weight gradients) and its fp8 codes + scales along d; dead pad rows are skipped.
+// With a ring position (*shift), the bf16 row goes to row R + *shift, and so do the codes when
+// shift_codes is set (a ring of codes beside the bf16 ring); otherwise the codes stay at row R.
 __global__ void __launch_bounds__(256) k_gather_rows_mx(const __nv_bfloat16* __restrict__ src,
                                                         const int* __restrict__ row_asg, const int* __restrict__ lo,
                                                         const int* __restrict__ hi, const int* __restrict__ shift,
-                                                        int k, int d, __nv_bfloat16* __restrict__ dst,
+                                                        int shift_codes, int k, int d, __nv_bfloat16* __restrict__ dst,
                                                         uint8_t* __restrict__ q, uint8_t* __restrict__ qs) {
   // One warp per padded row.  Lane i takes the row's 16-byte chunks i, i + 32, ... (8 values
   // each), four chunks in flight; the four lanes 4m .. 4m+3 hold one 32-value block and share
@@ -121,6 +122,7 @@ __global__ void __launch_bounds__(256) k_gather_rows_mx(const __nv_bfloat16* __r
   // number of chunks and the shuffles see the whole warp.
   const int r0 = __ldg(lo), r1 = __ldg(hi);
   const int64_t sh = shift ? __ldg(shift) : 0;
+  const int64_t shq = shift_codes ? sh : 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nv = d / 8;
   for (int64_t R = r0 + blockIdx.x * 8 + warp; R < r1; R += gridDim.x * 8) {
@@ -128,7 +130,7 @@ __global__ void __launch_bounds__(256) k_gather_rows_mx(const __nv_bfloat16* __r
     if (a == ROW_DEAD) continue;  // never read; a live pad row gets zero codes and scale 0
     const uint4* in = a >= 0 ? reinterpret_cast<const uint4*>(src + static_cast<size_t>(a / k) * d) : nullptr;
     uint4* o = reinterpret_cast<uint4*>(dst + (R + sh) * d);
-    uint2* qd = reinterpret_cast<uint2*>(q + R * d);
+    uint2* qd = reinterpret_cast<uint2*>(q + (R + shq) * d);
     for (int c0 = lane; c0 < nv; c0 += 128) {
       uint4 u[4];
 #pragma unroll
@@ -166,7 +168,7 @@ __global__ void __launch_bounds__(256) k_gather_rows_mx(const __nv_bfloat16* __r
           w[h] = amax == 0.f ? 0u : (static_cast<uint32_t>(p0) | (static_cast<uint32_t>(p1) << 16));
         }
         qd[c] = make_uint2(w[0], w[1]);
-        if ((lane & 3) == 0) qs[sf_index(static_cast<int>(R), c * 8, d)] = static_cast<uint8_t>(byte);
+        if ((lane & 3) == 0) qs[sf_index(static_cast<int>(R + shq), c * 8, d)] = static_cast<uint8_t>(byte);
       }
     }
   }
@@ -350,20 +352,20 @@ cudaError_t launch_quant_weight(int mode, const __nv_bfloat16* src0, const __nv_
 }
 
 cudaError_t launch_gather_range_mx(const Layout& L, const Ctx& c, const __nv_bfloat16* src, const int* lo,
-                                   const int* hi, const int* shift, int64_t max_rows, __nv_bfloat16* dst, uint8_t* q,
-                                   uint8_t* qs, cudaStream_t st) {
+                                   const int* hi, const int* shift, bool shift_codes, int64_t max_rows,
+                                   __nv_bfloat16* dst, uint8_t* q, uint8_t* qs, cudaStream_t st) {
   const int64_t g = (max_rows + 7) / 8;
   const int grid = static_cast<int>(g < 148 * 8 ? (g > 0 ? g : 1) : 148 * 8);
-  k_gather_rows_mx<<<grid, 256, 0, st>>>(src, c.row_asg, lo, hi, shift, L.k, L.d, dst, q, qs);
+  k_gather_rows_mx<<<grid, 256, 0, st>>>(src, c.row_asg, lo, hi, shift, shift_codes ? 1 : 0, L.k, L.d, dst, q, qs);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gather_rows_mx(const Layout& L, const Ctx& c, const __nv_bfloat16* src, __nv_bfloat16* dst,
                                   uint8_t* q, uint8_t* qs, cudaStream_t st) {
   if (L.M > 0)  // all rows of the stream
-    return launch_gather_range_mx(L, c, src, c.tab.seg_poff, c.tab.seg_poff + L.M * L.El, nullptr, L.RP, dst, q, qs,
-                                  st);
-  return launch_gather_range_mx(L, c, src, c.poff, c.poff + L.El, nullptr, L.RP, dst, q, qs, st);
+    return launch_gather_range_mx(L, c, src, c.tab.seg_poff, c.tab.seg_poff + L.M * L.El, nullptr, false, L.RP, dst,
+                                  q, qs, st);
+  return launch_gather_range_mx(L, c, src, c.poff, c.poff + L.El, nullptr, false, L.RP, dst, q, qs, st);
 }
 
 }  // namespace moe

@@ -80,10 +80,12 @@ WORKLOADS = {
 for _n in (512, 1024, 2048, 2368, 4096, 8192, 16384):
     WORKLOADS[f"ep64_n{_n}"] = Workload(f"ep64_n{_n}", 2048, 7168, 384, 8, 2048, first_local=0, num_local=6,
                                         stream_M=16, ring_bytes=256 << 20, local_tokens=_n)
-# The same ring-streamed slice in MXFP8 (gate/up, down and both dgrads on MXFP8, bf16 weight gradients)
+# The same ring-streamed slice in MXFP8 (gate/up, down and both dgrads on MXFP8, bf16 weight gradients).
+# A ring row holds the bf16 row and its fp8 codes (1.52x the bytes): 384 MiB hold 18,432 rows, about
+# the 18,724 of the bf16 stream's 256 MiB ring.
 for _n in (512, 2368, 4096):
     WORKLOADS[f"ep64mx_n{_n}"] = Workload(f"ep64mx_n{_n}", 2048, 7168, 384, 8, 2048, mxfp8=True, first_local=0,
-                                          num_local=6, stream_M=16, ring_bytes=256 << 20, local_tokens=_n)
+                                          num_local=6, stream_M=16, ring_bytes=384 << 20, local_tokens=_n)
 # The same per-rank slice (6 of 384 experts, 32768 tokens, n per local expert) as one batch, the
 # dispatched rows held whole instead of in a ring: MXFP8 (epmx) and bf16 (epbf), the regime
 # where the grouped GEMMs are bound by the tensor cores rather than by the weight stream.

@@ -45,7 +45,7 @@ def test_mx_streamed_layer(T_mb, M, d, E, k, I, first, num, ring_mult, seed):
     w, x = make_case(T, d, E, k, I, seed=seed)
     El = num or E - first
     shape = B.make_shape(T_mb, d, E, I, k, prec=B.MOE_MXFP8, first_local_expert=first, num_local_experts=num)
-    ring_bytes = int(B.moe_stream_min_ring_bytes(shape) * ring_mult) // (2 * d) * (2 * d)
+    ring_bytes = int(B.moe_stream_min_ring_bytes(shape) * ring_mult)  # bf16 rows, their codes and scales
     s = B.MoEStreamMX(T_mb, d, E, I, k, M, ring_bytes, first, num)
     s.ctx.fill_(0xFF)  # NaN patterns wherever the step reads before it writes
     s.ws.fill_(0xFF)
