@@ -83,3 +83,24 @@ def test_mx_streamed_layer(T_mb, M, d, E, k, I, first, num, ring_mult, seed):
     assert torch.equal(_bits(Y2), _bits(Y))
     for n in g:
         assert torch.equal(_bits(g2[n]), _bits(g[n])), n
+
+
+def test_mx_stream_fp32_weight_gradients_round_to_the_bf16_mode():
+    # fp32 weight gradients are the same sums unrounded: bf16 of them is the bf16 mode's dW
+    T_mb, M, d, E, k, I = 128, 6, 256, 16, 4, 256
+    w, x = make_case(T_mb * M, d, E, k, I, seed=74)
+    shape = B.make_shape(T_mb, d, E, I, k, prec=B.MOE_MXFP8)
+    ring_bytes = B.moe_stream_min_ring_bytes(shape)  # the smallest ring: replay and several chunks
+    out = []
+    for wdt in (torch.bfloat16, torch.float32):
+        s = B.MoEStreamMX(T_mb, d, E, I, k, M, ring_bytes, wgrad_dtype=wdt)
+        s.prepare(x["W_gate"], x["W_up"], x["W_down"])
+        s.forward(x["X"], x["W_r"], x["bias"])
+        g = s.backward(x["X"], x["W_r"], x["dY"])
+        torch.cuda.synchronize()
+        assert s.error() == B.MOE_OK
+        out.append(g)
+    for n in ("dW_gate", "dW_up", "dW_down"):
+        assert out[1][n].dtype == torch.float32
+        assert torch.equal(_bits(out[1][n].to(torch.bfloat16)), _bits(out[0][n])), n
+    assert torch.equal(_bits(out[1]["dX"]), _bits(out[0]["dX"]))
