@@ -68,12 +68,16 @@ WORKLOADS = {
     "dsv3": Workload("dsv3", 2048, 7168, 256, 8, 2048),
     "kimi": Workload("kimi", 4096, 7168, 384, 8, 2048, zipf=True),
     "kimi_mx": Workload("kimi_mx", 4096, 7168, 384, 8, 2048, mxfp8=True, zipf=True),
+    # the 256-expert top-8 configuration in MXFP8 (the precision north of the bf16 dsv3 line)
+    "dsv3_mx": Workload("dsv3_mx", 2048, 7168, 256, 8, 2048, mxfp8=True),
     # the dsv3 expert shape and load (64 tokens per expert) with 16 experts: a
     # ~3 GB case for profiler captures (weights still exceed the 126 MB L2)
     "dsv3_e16": Workload("dsv3_e16", 128, 7168, 16, 8, 2048),
     # the kimi expert shape in MXFP8 with 24 experts and 256 tokens (~85 per expert, near-uniform):
     # a few-GB case for profiler captures of the block-scaled GEMMs
     "kimi_mx_e24": Workload("kimi_mx_e24", 256, 7168, 24, 8, 2048, mxfp8=True),
+    # dsv3_e16 in MXFP8 (64 tokens per expert): profiler captures of the MXFP8 weight gradients
+    "dsv3_mx_e16": Workload("dsv3_mx_e16", 128, 7168, 16, 8, 2048, mxfp8=True),
 }
 # Per-rank expert slice as at EP64: 6 local experts of 384, 16 minibatches of 2048
 # tokens streamed through a 256 MiB ring; n = tokens each local expert receives.
