@@ -487,10 +487,21 @@ def bf16_round(v):
     return u.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
-def mx_round_rows(v):
+def mx_round_rows(v, groups=None):
     """v [rows, n] (one expert's rows in order) rounded to MXFP8 along the rows, in blocks
-    of 32 rows from the first; rows past the last multiple of 32 are padded with zeros."""
+    of 32 rows from the first; rows past the last multiple of 32 are padded with zeros.
+    groups: lengths of consecutive runs of rows (summing to rows), each rounded on its own in
+    blocks of 32 from its first row (a ring-streamed layer's (macrobatch, expert) segments);
+    None: one run."""
     v = _f64(v)
+    if groups is not None:
+        out, r = [], 0
+        for n in groups:
+            out.append(mx_round_rows(v[r:r + n]))
+            r += n
+        if r != v.shape[0]:
+            raise ValueError("row groups must cover the rows")
+        return np.concatenate(out, axis=0) if out else v
     pad = (-v.shape[0]) % 32
     vp = np.concatenate([v, np.zeros((pad,) + v.shape[1:])], axis=0) if pad else v
     return mx_round(vp, axis=0)[:v.shape[0]]
@@ -550,10 +561,11 @@ def forward_mx(X, W_r, bias, W_gate, W_up, W_down, top_k: int, first_local: int 
     return Y, ctx
 
 
-def backward_mx(ctx, dY, mx_wgrad: bool = False):
+def backward_mx(ctx, dY, mx_wgrad: bool = False, row_groups=None):
     """MXFP8 layer backward.  mx_wgrad: the weight-gradient GEMMs on MXFP8 as well, each
     operand rounded along the expert's rows (mx_round_rows); otherwise they take the
-    unrounded operands.
+    unrounded operands.  row_groups: optional callable e_local -> run lengths of the expert's
+    rows (the segments of a ring-streamed layer), each run rounded on its own.
 
     The forward's saved pre-activations A and B are read as bf16 (bf16_round), the type the
     layer keeps them in: every operand quantised here (dA, dB along I; with mx_wgrad dA, dB and
@@ -588,10 +600,11 @@ def backward_mx(ctx, dY, mx_wgrad: bool = False):
         dB = dH * silu(A)
         dX[toks] += mx_round(dA, axis=1) @ Wq["gate_i"].T + mx_round(dB, axis=1) @ Wq["up_i"].T  # K = I
         if mx_wgrad:  # K = the expert's rows
-            Xr = mx_round_rows(Xe)
-            dW_gate[e] = Xr.T @ mx_round_rows(dA)
-            dW_up[e] = Xr.T @ mx_round_rows(dB)
-            dW_down[e] = mx_round_rows(ge[:, None] * H).T @ mx_round_rows(dYe)
+            grp = None if row_groups is None else row_groups(el)
+            Xr = mx_round_rows(Xe, grp)
+            dW_gate[e] = Xr.T @ mx_round_rows(dA, grp)
+            dW_up[e] = Xr.T @ mx_round_rows(dB, grp)
+            dW_down[e] = mx_round_rows(ge[:, None] * H, grp).T @ mx_round_rows(dYe, grp)
         else:
             dW_gate[e] = Xe.T @ dA
             dW_up[e] = Xe.T @ dB

@@ -642,6 +642,46 @@ def test_mx_wgrad_hg_columns_are_independent():
     assert np.array_equal(g2["dW_up"][e], g["dW_up"][e])
 
 
+def test_mx_round_rows_in_groups():
+    # Runs of rows rounded on their own (a ring-streamed layer's segments): 20 rows holding 0.005
+    # and then 20 rows whose first is 256.  As one run, the block of rows 0-31 has amax 256 and
+    # 0.005 falls below E4M3's normal range: 2.56 steps of 2^-9 -> 3 -> 0.005859375.  In runs of
+    # 20 + 20, rows 0-19 are their own block (amax 0.005, scale 2^-16): 0.005 * 65536 = 327.68,
+    # step 32 -> 320 -> 0.0048828125, and 256 stays 256.
+    v = np.zeros((40, 32))
+    v[:20, 3] = 0.005
+    v[20, 3] = 256.0
+    one = O.mx_round_rows(v)
+    two = O.mx_round_rows(v, [20, 20])
+    assert np.all(one[:20, 3] == 0.005859375) and one[20, 3] == 256.0
+    assert np.all(two[:20, 3] == 0.0048828125) and two[20, 3] == 256.0
+    # runs that are whole multiples of 32 rows give the blocks of one run; empty runs add nothing
+    rng = np.random.default_rng(17)
+    w = rng.standard_normal((96, 64)) * np.exp(rng.standard_normal((96, 1)))
+    assert np.array_equal(O.mx_round_rows(w, [32, 0, 64]), O.mx_round_rows(w))
+    assert np.array_equal(O.mx_round_rows(w, [96]), O.mx_round_rows(w))
+    with pytest.raises(ValueError):
+        O.mx_round_rows(w, [32, 32])
+
+
+def test_mx_wgrad_row_groups_reach_every_operand():
+    # backward_mx with row groups rounds all five weight-gradient operands by run: runs that
+    # split at multiples of 32 reproduce the one-run gradients bit for bit, runs that do not move
+    # every gradient
+    X, W_r, Wg, Wu, Wd, dY = _mx_case()
+    _, ctx = O.forward_mx(X, W_r, None, Wg, Wu, Wd, _MX_SHAPE["k"])
+    g = O.backward_mx(ctx, dY, mx_wgrad=True)
+    rows = {el: len(ctx["saved"][el][0]) for el in range(_MX_SHAPE["E"]) if ctx["saved"][el] is not None}
+    aligned = O.backward_mx(ctx, dY, mx_wgrad=True, row_groups=lambda el: [32, rows[el] - 32])
+    split = O.backward_mx(ctx, dY, mx_wgrad=True, row_groups=lambda el: [13, rows[el] - 13])
+    for n in ("dW_gate", "dW_up", "dW_down"):
+        for e in rows:
+            assert np.array_equal(aligned[n][e], g[n][e]), (n, e)
+            assert not np.array_equal(split[n][e], g[n][e]), (n, e)
+    for n in ("dX", "dg", "dW_r"):
+        assert np.array_equal(split[n], g[n]), n
+
+
 def test_mx_wgrad_worked_example_by_hand():
     # tests/golden/mx_wgrad_worked_example.json: the weight gradients of a two-expert MXFP8
     # layer with MX weight-gradient GEMMs, every rounding worked out by hand there (row blocks
