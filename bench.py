@@ -466,7 +466,7 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     wdt = torch.float32 if args.wgrad_fp32 else torch.bfloat16
     if w.mxfp8 and w.stream_M:
         layer = B.MoEStreamMX(w.T, w.d, w.E, w.I, w.k, w.stream_M, w.ring_bytes, w.first_local, w.num_local,
-                              device=dev, wgrad_dtype=wdt)
+                              device=dev, wgrad_dtype=wdt, mx_wgrad=args.mx_wgrad)
     elif w.mxfp8:
         layer = B.MoELayerMX(w.T, w.d, w.E, w.I, w.k, w.first_local, w.num_local, device=dev, wgrad_dtype=wdt,
                              mx_wgrad=args.mx_wgrad)
@@ -787,10 +787,7 @@ def main():
     w = IN.WORKLOADS[args.workload]
     if args.wgrad_gemms and not w.mxfp8:
         ap.error("--wgrad-gemms applies to the MXFP8 workloads; %s is bf16" % w.name)
-    if args.wgrad_gemms == "mxfp8" and w.stream_M:
-        ap.error("the ring-streamed MXFP8 layer keeps bf16 weight gradients")
-    # MXFP8 weight gradients for the one-batch MXFP8 workloads (the ring stream keeps bf16 ones)
-    args.mx_wgrad = w.mxfp8 and not w.stream_M and args.wgrad_gemms != "bf16"
+    args.mx_wgrad = w.mxfp8 and args.wgrad_gemms != "bf16"
     if args.launches and w.stream_M:
         ap.error("the ring-streamed layer always runs its GEMM pairs as persistent launches")
     if args.persistent and (w.mxfp8 or w.stream_M or args.launches):

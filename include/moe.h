@@ -310,14 +310,17 @@ moe_status moe_bwd_stream(const moe_shape* shape, int32_t num_minibatches, const
  * replayed rows, resident rows, ring rows, 0...] then mb_of[M],
  * seg_poff[M*El+1], cum[M*El], mb_range[2M], shift_fwd[M], shift_bwd[M],
  * replay[M], chunk[4M] ({m_lo, m_hi, valid, mode}), ring_start[M]. */
-/* MXFP8 ring-streamed layer (shape->prec = MOE_MXFP8): the same plan, ring and backward chunks as
+/* MXFP8 ring-streamed layer (shape->prec = MOE_MXFP8 or MOE_MXFP8_ALL): the same plan and ring as
  * moe_fwd_stream / moe_bwd_stream, with the gate/up, down and both dgrad GEMMs on MXFP8 from the
- * prepared weights `wq` (moe_prepare_weights of this shape); the weight gradients stay bf16
- * (MOE_MXFP8_ALL shapes are refused: MOE_ERR_UNSUPPORTED).  A ring row holds the bf16 row, its E4M3
- * codes along d and their scales (2d + d + d/32 bytes): the ring holds R = ring_bytes / (3d + d/32)
- * rows rounded down to a multiple of 128, laid out as R bf16 rows, R code rows, then the codes' scale
- * chunks.  ctx / ws / minimum ring sizes: the moe_stream_* size calls of this shape.  Same errors as
- * the bf16 stream. */
+ * prepared weights `wq` (moe_prepare_weights of this shape).  MOE_MXFP8: bf16 weight gradients as in
+ * the bf16 stream (ring replay, backward chunks); a ring row holds the bf16 row, its E4M3 codes along
+ * d and their scales (2d + d + d/32 bytes).  MOE_MXFP8_ALL: MXFP8 weight gradients over every
+ * segment of the stream, the operands quantised along the rows in blocks of 32 rows of each
+ * (macrobatch, expert) segment, X's codes along the rows kept at the padded rows of the stream (ctx),
+ * so nothing is replayed; a ring row holds the codes along d and their scales (d + d/32 bytes).  The
+ * ring holds R = ring_bytes / (row bytes) rows rounded down to a multiple of 128, laid out as R bf16
+ * rows (MOE_MXFP8 only), R code rows, then the codes' scale chunks.  ctx / ws / minimum ring sizes:
+ * the moe_stream_* size calls of this shape.  Same errors as the bf16 stream. */
 moe_status moe_fwd_stream_mx(const moe_shape* shape, int32_t num_minibatches, const void* X, const void* W_r,
                              const float* bias, const void* wq, size_t wq_bytes, void* Y, void* ctx, size_t ctx_bytes,
                              void* ring, size_t ring_bytes, void* ws, size_t ws_bytes, void* stream);

@@ -607,15 +607,17 @@ class MoEStream:
 
 
 class MoEStreamMX(MoEStream):
-    """The ring-streamed layer in MXFP8 (MOE_MXFP8: gate/up, down and both dgrads on MXFP8 tensor
-    cores, bf16 weight gradients): ctx / ring / workspace owner plus the prepared weights."""
+    """The ring-streamed layer in MXFP8 (gate/up, down and both dgrads on MXFP8 tensor cores):
+    ctx / ring / workspace owner plus the prepared weights.  mx_wgrad: the weight-gradient GEMMs on
+    MXFP8 too (MOE_MXFP8_ALL); otherwise bf16 (MOE_MXFP8)."""
 
     def __init__(self, T, d, E, I, top_k, M, ring_bytes, first_local_expert=0, num_local_experts=0, device="cuda",
-                 wgrad_dtype=None):
+                 wgrad_dtype=None, mx_wgrad=False):
         import torch
         self.wgrad_dtype = wgrad_dtype or torch.bfloat16
-        self.shape = make_shape(T, d, E, I, top_k, MOE_MXFP8, first_local_expert, num_local_experts,
-                                _wgrad_code(self.wgrad_dtype))
+        self.mx_wgrad = bool(mx_wgrad)
+        self.shape = make_shape(T, d, E, I, top_k, MOE_MXFP8_ALL if mx_wgrad else MOE_MXFP8, first_local_expert,
+                                num_local_experts, _wgrad_code(self.wgrad_dtype))
         nc, nw = moe_stream_ctx_size(self.shape, M), moe_stream_workspace_size(self.shape, M)
         nq = moe_weights_size(self.shape)
         if nc == 0 or nw == 0 or nq == 0:

@@ -29,8 +29,20 @@ namespace moe {
 
 struct MxTile {
   int el, m0, n0, nt, nk;
-  int r0, rows;  // weight-gradient kinds: the expert's first padded row and its real rows
 };
+
+// Weight-gradient kinds: segment m (of nseg / El) of local expert el: its first padded row and its
+// real rows (one segment per expert, or one per macrobatch of a ring-streamed layer).
+__device__ __forceinline__ void mx_wseg(const MxParams& p, int m, int el, int& r0, int& rows) {
+  const int sg = m * p.El + el;
+  r0 = __ldg(p.poff + sg);
+  if (!p.cum) {
+    rows = __ldg(p.cnt + el);
+  } else {
+    const int nm = p.nseg / p.El;
+    rows = (m + 1 < nm ? __ldg(p.cum + sg + p.El) : __ldg(p.cnt + el)) - __ldg(p.cum + sg);
+  }
+}
 
 template <int KIND>
 __device__ __forceinline__ int mx_ntiles_n(const MxParams& p) {
@@ -80,9 +92,12 @@ __device__ __forceinline__ MxTile mx_decode(const MxParams& p, int t) {
     tl.m0 = mt * 128;
     tl.nt = local - mt * NT;
     tl.n0 = tl.nt * 256;
-    tl.r0 = __ldg(p.poff + el);
-    tl.rows = __ldg(p.cnt + el);
-    tl.nk = (tl.rows + 127) / 128;
+    tl.nk = 0;  // 128-row K blocks over the expert's segments
+    for (int m = 0, nm = p.nseg / p.El; m < nm; ++m) {
+      int r0, rows;
+      mx_wseg(p, m, el, r0, rows);
+      tl.nk += (rows + 127) / 128;
+    }
     return tl;
   }
   const int base = __ldg(p.poff);
@@ -100,10 +115,11 @@ __device__ __forceinline__ MxTile mx_decode(const MxParams& p, int t) {
   return tl;
 }
 
-// TMA + bulk loads of K block kb (128 elements) of tile tl into one stage.
+// TMA + bulk loads of K block kb (128 elements) of tile tl into one stage; the weight-gradient
+// kinds take the block's first padded row (krow) instead.
 template <int KIND>
-__device__ __forceinline__ void mx_load(const MxParams& p, const MxTile& tl, int kb, uint8_t* st, uint64_t* bar,
-                                        uint64_t pol_act, uint64_t pol_w) {
+__device__ __forceinline__ void mx_load(const MxParams& p, const MxTile& tl, int kb, int krow, uint8_t* st,
+                                        uint64_t* bar, uint64_t pol_act, uint64_t pol_w) {
   uint8_t* sA = st;
   constexpr int BN = mx_bn(KIND);
   uint8_t* sB = st + MX_A_BYTES;
@@ -113,9 +129,10 @@ __device__ __forceinline__ void mx_load(const MxParams& p, const MxTile& tl, int
   const uint8_t* sfa = p.sfa0;
   const uint8_t* sfb = p.sfb0;
   if constexpr (mx_is_wgrad(KIND)) {
-    // K block kb = row tile kt = (r0 + 128 kb) / 128 of both operands (rowq layout): A = lines
+    // the K block = row tile kt = krow / 128 of both operands (rowq layout): A = lines
     // kt CA + m0 .., B = lines kt CB + nb .. of 128 codes, and the tile's scale chunks
-    const size_t kt = static_cast<size_t>((tl.r0 >> 7) + kb);
+    const size_t kt = static_cast<size_t>(krow >> 7);
+    (void)kb;
     const int CA = KIND == MX_WGRAD_GATEUP ? p.d : p.I, CB = KIND == MX_WGRAD_GATEUP ? p.I : p.d;
     int nb = tl.n0;
     if constexpr (KIND == MX_WGRAD_GATEUP) {
@@ -465,12 +482,26 @@ __global__ void __launch_bounds__(mx_threads(KIND), 1) k_moe_gemm_mx(const __gri
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         const MxTile tl = mx_decode<KIND>(p, t);
-        for (int kb = 0; kb < tl.nk; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, p.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(mx_stage_tx(KIND)));
-          mx_load<KIND>(p, tl, kb, smem + stage * SB, &full[stage], pol_act, pol_w);
-          last_parity[stage] = static_cast<int>(phase);
-          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        if constexpr (mx_is_wgrad(KIND)) {  // K: the 128-row blocks of each of the expert's segments
+          for (int m = 0, nm = p.nseg / p.El; m < nm && ok; ++m) {
+            int r0, rows;
+            mx_wseg(p, m, tl.el, r0, rows);
+            for (int j = 0; j * 128 < rows; ++j) {
+              if (!mbar_wait(&empty[stage], phase ^ 1, p.status)) { ok = false; break; }
+              mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(mx_stage_tx(KIND)));
+              mx_load<KIND>(p, tl, 0, r0 + j * 128, smem + stage * SB, &full[stage], pol_act, pol_w);
+              last_parity[stage] = static_cast<int>(phase);
+              if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+          }
+        } else {
+          for (int kb = 0; kb < tl.nk; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, p.status)) { ok = false; break; }
+            mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(mx_stage_tx(KIND)));
+            mx_load<KIND>(p, tl, kb, 0, smem + stage * SB, &full[stage], pol_act, pol_w);
+            last_parity[stage] = static_cast<int>(phase);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
         }
       }
       if (!ok)
@@ -490,7 +521,21 @@ __global__ void __launch_bounds__(mx_threads(KIND), 1) k_moe_gemm_mx(const __gri
         if (!mbar_wait(&tempty[acc], accp ^ 1, p.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t dtm = tbase + acc * BN;  // accumulators in columns [0, 256)
+        // weight gradients: K walks the expert's segments; (m, j, rows) track the current block
+        int m = 0, j = 0, rows = 0;
+        if constexpr (mx_is_wgrad(KIND)) {
+          int r0;
+          mx_wseg(p, 0, tl.el, r0, rows);
+        }
         for (int kb = 0; kb < tl.nk; ++kb) {
+          if constexpr (mx_is_wgrad(KIND)) {
+            while (j * 128 >= rows) {  // past this segment: the next one with rows (nk counts them)
+              int r0;
+              ++m;
+              j = 0;
+              mx_wseg(p, m, tl.el, r0, rows);
+            }
+          }
           if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + stage * SB);
@@ -506,8 +551,9 @@ __global__ void __launch_bounds__(mx_threads(KIND), 1) k_moe_gemm_mx(const __gri
           // (its rows past them up to the next multiple of 32 are zero codes)
           int nkk = 4;
           if constexpr (mx_is_wgrad(KIND)) {
-            const int valid = tl.rows - kb * 128;
+            const int valid = rows - j * 128;
             if (valid < 128) nkk = (valid + 31) / 32;
+            ++j;
           }
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)

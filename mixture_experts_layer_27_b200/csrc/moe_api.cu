@@ -853,12 +853,13 @@ unsigned long long moe_kernel_launches(void) { return g_launches.load(); }
 // ---------------------------------------------------------------------------
 // Ring-streamed layer: M minibatches of shape->T tokens through a fixed ring
 // ---------------------------------------------------------------------------
-// prec: MOE_BF16 for the bf16 entry points, MOE_MXFP8 for the MXFP8 ones, -1 for either (sizes,
-// debug).  The ring-streamed layer keeps bf16 weight gradients: MOE_MXFP8_ALL is refused.
+// prec: MOE_BF16 for the bf16 entry points, MOE_MXFP8 for the MXFP8 ones (MOE_MXFP8 or
+// MOE_MXFP8_ALL shapes), -1 for any (sizes, debug).
 static moe_status check_stream(const moe_shape* s, int32_t M, Layout* L, int32_t prec = MOE_BF16) {
   if (!s || M <= 0) return MOE_ERR_INVALID_ARG;
   if (s->prec != MOE_BF16 && !is_mx_prec(s->prec)) return MOE_ERR_INVALID_ARG;
-  if (s->prec == MOE_MXFP8_ALL || (prec >= 0 && s->prec != prec)) return MOE_ERR_UNSUPPORTED;
+  if (prec == MOE_BF16 && s->prec != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (prec == MOE_MXFP8 && !is_mx_prec(s->prec)) return MOE_ERR_UNSUPPORTED;
   if (!make_layout(*s, L, M)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -881,10 +882,13 @@ size_t moe_stream_workspace_size(const moe_shape* s, int32_t M) {
   return L.ws_bytes;
 }
 
-// Bytes of the caller's ring per row: the bf16 row, and in MXFP8 its codes along d and their
-// scales (the ring holds ring_rows bf16 rows, then ring_rows code rows, then their scale chunks).
+// Bytes of the caller's ring per row: the bf16 row (the bf16 weight gradients' operand, replayed),
+// and in MXFP8 its codes along d and their scales (ring_rows bf16 rows, then ring_rows code rows,
+// then their scale chunks); with MXFP8 weight gradients the codes only (X's codes along the rows
+// are kept at their padded rows, so nothing is replayed).
 static size_t ring_row_bytes(const Layout& L) {
-  return static_cast<size_t>(L.d) * 2 + (L.mx ? static_cast<size_t>(L.d) + L.d / 32 : 0);
+  const size_t codes = L.mx ? static_cast<size_t>(L.d) + L.d / 32 : 0;
+  return (L.mxw ? 0 : static_cast<size_t>(L.d) * 2) + codes;
 }
 // Rows of a ring of ring_bytes; in MXFP8 a multiple of 128 (the scale chunks cover 128-row tiles).
 static int64_t ring_rows_of(const Layout& L, size_t ring_bytes) {
@@ -966,6 +970,8 @@ moe_status moe_fwd_stream(const moe_shape* s, int32_t M, const void* X, const vo
 
 static moe_status stream_wgrads(const Layout& L, const Ctx& c, int* status, const void* X, void* ring,
                                 int64_t ring_rows, void* dW_gate, void* dW_up, void* dW_down, cudaStream_t st);
+static moe_status launch_wgrads_mx(const Layout& L, const Ctx& c, int* status, void* dW_gate, void* dW_up,
+                                   void* dW_down, cudaStream_t st);
 
 moe_status moe_bwd_stream(const moe_shape* s, int32_t M, const void* X, const void* W_r, const void* W_gate,
                           const void* W_up, const void* W_down, const void* dY, void* ctx, size_t ctx_bytes, void* dX,
@@ -1119,8 +1125,8 @@ moe_status moe_fwd_stream_mx(const moe_shape* s, int32_t M, const void* X, const
   int* status = c.hdr + HDR_STATUS;
   const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
   const auto* w = static_cast<const uint8_t*>(wq);
-  // the ring: ring_rows bf16 rows, then their codes, then the codes' scale chunks
-  uint8_t* ring_q = static_cast<uint8_t*>(ring) + static_cast<size_t>(ring_rows) * L.d * 2;
+  // the ring: ring_rows bf16 rows (not with MXFP8 weight gradients), their codes, the codes' scale chunks
+  uint8_t* ring_q = static_cast<uint8_t*>(ring) + (L.mxw ? 0 : static_cast<size_t>(ring_rows) * L.d * 2);
   uint8_t* ring_qs = ring_q + static_cast<size_t>(ring_rows) * L.d;
   CUtensorMap xq_map, wgu_map, hq_map, wd_map;
   MOE_TMAP(tmap_fp8(&xq_map, ring_q, L.d, static_cast<uint64_t>(ring_rows), 128));
@@ -1131,6 +1137,9 @@ moe_status moe_fwd_stream_mx(const moe_shape* s, int32_t M, const void* X, const
   for (int m = 0; m < M; ++m) {
     const int* seg = c.tab.seg_poff + m * L.El;
     MOE_TRY(timed(K_DISPATCH, st, [&] {
+      if (L.mxw)  // codes along d to the ring, codes along the rows (weight gradients) at the padded rows
+        return launch_gather_quant2_range(L, c, static_cast<const __nv_bfloat16*>(X), seg, seg + L.El,
+                                          c.tab.shift_fwd + m, ring_q, ring_qs, c.xqt, c.xqts, st);
       return launch_gather_range_mx(L, c, static_cast<const __nv_bfloat16*>(X), seg, seg + L.El,
                                     c.tab.shift_fwd + m, true, ring_rows, static_cast<__nv_bfloat16*>(ring), ring_q,
                                     ring_qs, st);
@@ -1188,9 +1197,11 @@ moe_status moe_bwd_stream_mx(const moe_shape* s, int32_t M, const void* X, const
   const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
   const int nseg = L.M * L.El;
   const auto* w = static_cast<const uint8_t*>(wq);
-  // reverse-combine over every row of the stream: bf16 (the W_down weight gradient's operand) and
-  // codes along d (the dgrad of W_down's operand)
+  // reverse-combine over every row of the stream: codes along d (the dgrad of W_down's operand) and
+  // bf16 (the W_down weight gradient's operand), or codes along the rows with MXFP8 weight gradients
   MOE_TRY(timed(K_REV_COMBINE, st, [&] {
+    if (L.mxw)
+      return launch_gather_quant2(L, c, static_cast<const __nv_bfloat16*>(dY), c.dyq, c.dyqs, c.dyqt, c.dyqts, st);
     return launch_gather_rows_mx(L, c, static_cast<const __nv_bfloat16*>(dY), c.dyperm, c.dyq, c.dyqs, st);
   }));
   {
@@ -1205,9 +1216,18 @@ moe_status moe_bwd_stream_mx(const moe_shape* s, int32_t M, const void* X, const
     p.sfb0 = p.sfb1 = w + L.wd3s;
     p.in0 = c.abuf;
     p.in1 = c.bbuf;
-    p.out0 = c.dabuf;
-    p.out1 = c.dbbuf;
-    p.out2 = c.hgbuf;
+    if (L.mxw) {  // dA, dB, Hg along the rows, from fp32, for the MXFP8 weight gradients
+      p.tq[0] = c.daqt;
+      p.tq[1] = c.dbqt;
+      p.tq[2] = c.hgqt;
+      p.tqs[0] = c.daqts;
+      p.tqs[1] = c.dbqts;
+      p.tqs[2] = c.hgqts;
+    } else {
+      p.out0 = c.dabuf;
+      p.out1 = c.dbbuf;
+      p.out2 = c.hgbuf;
+    }
     p.q0 = c.daq;
     p.qs0 = c.daqs;
     p.q1 = c.dbq;
@@ -1235,8 +1255,10 @@ moe_status moe_bwd_stream_mx(const moe_shape* s, int32_t M, const void* X, const
     MOE_TRY(timed(K_GEMM_DGRAD_GATEUP, st, [&] { return launch_gemm_mx(MX_DGRAD_GATEUP, p, grid, st); }));
   }
   MOE_TRY(timed(K_REV_DISPATCH, st, [&] { return launch_rev_dispatch(L, c, static_cast<__nv_bfloat16*>(dX), st); }));
-  // bf16 weight gradients exactly as the bf16 stream: W_down's over every row, gate/up's walking
-  // the ring in reverse, chunk by chunk, into the fp32 accumulator
+  // MXFP8 weight gradients over every segment of the stream (no replay: X's codes along the rows
+  // are kept at the padded rows), or bf16 ones exactly as the bf16 stream: W_down's over every row,
+  // gate/up's walking the ring in reverse, chunk by chunk, into the fp32 accumulator
+  if (L.mxw) return launch_wgrads_mx(L, c, status, dW_gate, dW_up, dW_down, st);
   return stream_wgrads(L, c, status, X, ring, ring_rows, dW_gate, dW_up, dW_down, st);
 }
 
@@ -1293,6 +1315,16 @@ moe_status moe_prepare_weights(const moe_shape* s, const void* W_gate, const voi
 }
 
 
+// The row segments an MXFP8 weight gradient contracts over: one per local expert, or in a
+// ring-streamed layer one per (macrobatch, expert) with the real rows counted by the stream plan.
+static void wgrad_segments(const Layout& L, const Ctx& c, MxParams& p) {
+  if (L.M > 0) {
+    p.poff = c.tab.seg_poff;
+    p.nseg = L.M * L.El;
+    p.cum = c.tab.cum;
+  }
+}
+
 // MXFP8 weight gradients from operands quantised along the rows (blocks of 32 rows of one expert,
 // K-major in 128-row tiles): X by the forward's dispatch, dY by the reverse-combine, dA, dB and Hg
 // by the dgrad of W_down from its fp32 values.  One grouped GEMM for gate/up and one for down;
@@ -1309,6 +1341,7 @@ static moe_status launch_wgrads_mx(const Layout& L, const Ctx& c, int* status, v
     MOE_TMAP(tmap_fp8(&p.tb1, c.dbqt, 128, RP / 128 * L.I, 256));
     MOE_TMAP(tmap_wgrad_out(L, &p.to0, dW_gate, L.I, El * L.d));
     MOE_TMAP(tmap_wgrad_out(L, &p.to1, dW_up, L.I, El * L.d));
+    wgrad_segments(L, c, p);
     p.ta1 = p.ta0;
     p.sfa0 = p.sfa1 = c.xqts;
     p.sfb0 = c.daqts;
@@ -1322,6 +1355,7 @@ static moe_status launch_wgrads_mx(const Layout& L, const Ctx& c, int* status, v
     MOE_TMAP(tmap_fp8(&p.ta0, c.hgqt, 128, RP / 128 * L.I, 128));
     MOE_TMAP(tmap_fp8(&p.tb0, c.dyqt, 128, RP / 128 * L.d, 256));
     MOE_TMAP(tmap_wgrad_out(L, &p.to0, dW_down, L.d, El * L.I));
+    wgrad_segments(L, c, p);
     p.ta1 = p.ta0;
     p.tb1 = p.tb0;
     p.to1 = p.to0;

@@ -226,6 +226,8 @@ struct MxParams {
   // 64 x 32 boxes, or fp32 32 x 32 boxes with wout32)
   CUtensorMap to0, to1;
   const int* cnt;
+  const int* cum;  // ring-streamed layer: real rows of local expert el before segment (m, el), [nseg];
+                   // NULL: one segment per expert (nseg = El)
   int wout32;
   // dgrad of W_down with MXFP8 weight gradients: dA, dB and Hg also quantised along the rows,
   // from the fp32 epilogue values, into the rowq layout (C = I) and its scale chunks (the
@@ -335,6 +337,10 @@ cudaError_t launch_gather_range_mx(const Layout& L, const Ctx& c, const __nv_bfl
 // 32 (qr, qrs: rowq layout), no bf16 copy.
 cudaError_t launch_gather_quant2(const Layout& L, const Ctx& c, const __nv_bfloat16* src, uint8_t* qd, uint8_t* qds,
                                  uint8_t* qr, uint8_t* qrs, cudaStream_t st);
+// rows [*lo, *hi) only, the codes along d at row + *dshift (a ring position; dshift may be NULL)
+cudaError_t launch_gather_quant2_range(const Layout& L, const Ctx& c, const __nv_bfloat16* src, const int* lo,
+                                       const int* hi, const int* dshift, uint8_t* qd, uint8_t* qds, uint8_t* qr,
+                                       uint8_t* qrs, cudaStream_t st);
 cudaError_t launch_transpose_wr(const Layout& L, const __nv_bfloat16* W_r, __nv_bfloat16* W_rT, cudaStream_t st);
 cudaError_t launch_rev_dispatch(const Layout& L, const Ctx& c, __nv_bfloat16* dX, cudaStream_t st);
 cudaError_t launch_export_routing(const Layout& L, const Ctx& c, int32_t* counts, int32_t* offsets,

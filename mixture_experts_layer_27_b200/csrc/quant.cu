@@ -227,11 +227,13 @@ __device__ __forceinline__ void gq_issue(const __nv_bfloat16* __restrict__ src, 
 
 __global__ void __launch_bounds__(256, 3) k_gather_quant2(const __nv_bfloat16* __restrict__ src,
                                                           const int* __restrict__ row_asg, const int* __restrict__ lo,
-                                                          const int* __restrict__ hi, int k, int d,
-                                                          uint8_t* __restrict__ qd, uint8_t* __restrict__ qds,
-                                                          uint8_t* __restrict__ qr, uint8_t* __restrict__ qrs) {
+                                                          const int* __restrict__ hi, const int* __restrict__ dshift,
+                                                          int k, int d, uint8_t* __restrict__ qd,
+                                                          uint8_t* __restrict__ qds, uint8_t* __restrict__ qr,
+                                                          uint8_t* __restrict__ qrs) {
   extern __shared__ __align__(16) uint8_t gq_smem[];
   const int64_t r_lo = __ldg(lo);
+  const int64_t dsh = dshift ? __ldg(dshift) : 0;  // the codes along d at a ring position
   const int ng = d / 64;                              // column groups
   const int64_t items = (__ldg(hi) - r_lo) / 128 * ng;  // (tile, column group) pairs
   const int t = threadIdx.x;
@@ -284,7 +286,7 @@ __global__ void __launch_bounds__(256, 3) k_gather_quant2(const __nv_bfloat16* _
         }
         uint32_t w[8];
         const uint8_t sb = mx_quant32(v, w);
-        const int64_t R = r0 + rr;
+        const int64_t R = r0 + rr + dsh;
         uint4* dst = reinterpret_cast<uint4*>(qd + R * d + c0 + blk * 32);
         dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
         dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
@@ -309,8 +311,9 @@ __global__ void __launch_bounds__(256, 3) k_gather_quant2(const __nv_bfloat16* _
   cp_async_wait<0>();  // no copy outlives the CTA's shared memory
 }
 
-cudaError_t launch_gather_quant2(const Layout& L, const Ctx& c, const __nv_bfloat16* src, uint8_t* qd, uint8_t* qds,
-                                 uint8_t* qr, uint8_t* qrs, cudaStream_t st) {
+cudaError_t launch_gather_quant2_range(const Layout& L, const Ctx& c, const __nv_bfloat16* src, const int* lo,
+                                       const int* hi, const int* dshift, uint8_t* qd, uint8_t* qds, uint8_t* qr,
+                                       uint8_t* qrs, cudaStream_t st) {
   static bool configured[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -329,9 +332,17 @@ cudaError_t launch_gather_quant2(const Layout& L, const Ctx& c, const __nv_bfloa
   int64_t grid = static_cast<int64_t>(sms) * 3;
   if (grid > max_items) grid = max_items;
   if (grid < 1) grid = 1;
-  k_gather_quant2<<<static_cast<unsigned>(grid), 256, GQ_SMEM, st>>>(src, c.row_asg, c.poff, c.poff + L.El, L.k,
-                                                                      L.d, qd, qds, qr, qrs);
+  k_gather_quant2<<<static_cast<unsigned>(grid), 256, GQ_SMEM, st>>>(src, c.row_asg, lo, hi, dshift, L.k, L.d, qd,
+                                                                      qds, qr, qrs);
   return cudaGetLastError();
+}
+
+cudaError_t launch_gather_quant2(const Layout& L, const Ctx& c, const __nv_bfloat16* src, uint8_t* qd, uint8_t* qds,
+                                 uint8_t* qr, uint8_t* qrs, cudaStream_t st) {
+  if (L.M > 0)  // all rows of the stream
+    return launch_gather_quant2_range(L, c, src, c.tab.seg_poff, c.tab.seg_poff + L.M * L.El, nullptr, qd, qds, qr,
+                                      qrs, st);
+  return launch_gather_quant2_range(L, c, src, c.poff, c.poff + L.El, nullptr, qd, qds, qr, qrs, st);
 }
 
 cudaError_t launch_quant_weight(int mode, const __nv_bfloat16* src0, const __nv_bfloat16* src1, int64_t R_out, int K,

@@ -109,16 +109,18 @@ def test_stream_shapes_and_sizes():
         assert B.moe_stream_ctx_size(s, M) == 0 and B.moe_stream_workspace_size(s, M) == 0
     ragged = B.make_shape(2050, 7168, 384, 2048, 8)  # minibatches are whole 16-token blocks
     assert B.moe_stream_ctx_size(ragged, 4) == 0 and B.moe_stream_min_ring_bytes(ragged) == 0
-    # MXFP8 streams (bf16 weight gradients): the same ctx (X's codes live in the ring), a workspace
-    # larger by the backward's fp8 operands; MXFP8 weight gradients are one-batch only
+    # MXFP8 streams with bf16 weight gradients: the same ctx (X's codes live in the ring), a workspace
+    # larger by the backward's fp8 operands; with MXFP8 weight gradients ctx also keeps X's codes
+    # along the rows, and the ring holds codes only
     mx = B.make_shape(2048, 7168, 384, 2048, 8, prec=B.MOE_MXFP8)
     bf = B.make_shape(2048, 7168, 384, 2048, 8)
     assert B.moe_stream_ctx_size(mx, 4) == B.moe_stream_ctx_size(bf, 4) > 0
     assert B.moe_stream_workspace_size(mx, 4) > B.moe_stream_workspace_size(bf, 4) > 0
-    # an MXFP8 ring row holds the bf16 row, its codes along d and their scales
-    assert B.moe_stream_min_ring_bytes(mx) == B.moe_stream_min_ring_bytes(bf) // (2 * 7168) * (3 * 7168 + 7168 // 32)
+    rows = B.moe_stream_min_ring_bytes(bf) // (2 * 7168)
+    assert B.moe_stream_min_ring_bytes(mx) == rows * (3 * 7168 + 7168 // 32)
     mxa = B.make_shape(2048, 7168, 384, 2048, 8, prec=B.MOE_MXFP8_ALL)
-    assert B.moe_stream_ctx_size(mxa, 4) == 0 and B.moe_stream_workspace_size(mxa, 4) == 0
+    assert B.moe_stream_ctx_size(mxa, 4) > B.moe_stream_ctx_size(mx, 4)
+    assert B.moe_stream_min_ring_bytes(mxa) == rows * (7168 + 7168 // 32)
 
 
 def test_stream_mx_argument_errors_are_synchronous(lib):
@@ -143,8 +145,6 @@ def test_stream_mx_argument_errors_are_synchronous(lib):
     assert bwd(wq_bytes=nq - 1) == B.MOE_ERR_WORKSPACE_TOO_SMALL
     bf = B.make_shape(128, 256, 16, 256, 4)  # the MX entry points take MXFP8 shapes only
     assert fwd(shape=bf) == B.MOE_ERR_UNSUPPORTED and bwd(shape=bf) == B.MOE_ERR_UNSUPPORTED
-    mxa = B.make_shape(128, 256, 16, 256, 4, prec=B.MOE_MXFP8_ALL)
-    assert fwd(shape=mxa) == B.MOE_ERR_UNSUPPORTED
     # and the bf16 entry points refuse MXFP8 shapes
     assert lib.moe_fwd_stream(ctypes.byref(s), M, f, f, None, f, f, f, f, f, nc, f, nr, f, nw, None) == \
         B.MOE_ERR_UNSUPPORTED

@@ -378,6 +378,77 @@ def test_full_size_ep64_ring_stream_mx():
     torch.cuda.empty_cache()
 
 
+def test_full_size_ep64_ring_stream_mx_weight_gradients():
+    # Config 5 at n = 4096 in MXFP8 with MXFP8 weight gradients: eight macrobatches, each
+    # (macrobatch, expert) segment quantised along its rows on its own.  Y, dX and dW_r equal the
+    # one-batch layer's bits; two local experts' weight gradients are within 6e-2 of the MX oracle
+    # with the device plan's segments as row groups; a rerun is bit-identical.
+    w = IN.WORKLOADS["ep64mx_n4096"]
+    x = IN.make_inputs(w, device="cuda")
+    first, El = w.first_local, w.El
+
+    def run():
+        s = B.MoEStreamMX(w.T, w.d, w.E, w.I, w.k, w.stream_M, w.ring_bytes, first, w.num_local, mx_wgrad=True)
+        s.prepare(x["W_gate"], x["W_up"], x["W_down"])
+        Y = s.forward(x["X"], x["W_r"], x["bias"])
+        g = s.backward(x["X"], x["W_r"], x["dY"])
+        torch.cuda.synchronize()
+        assert s.error() == B.MOE_OK
+        return s, Y, g
+
+    s, Y, g = run()
+    plan = s.plan()
+    nm = int(plan["plan"][0])
+    assert nm > 1
+    cum = plan["cum"].copy()
+    del s
+    torch.cuda.empty_cache()
+    lay = B.MoELayerMX(w.tokens, w.d, w.E, w.I, w.k, first, w.num_local, mx_wgrad=True)
+    lay.prepare(x["W_gate"], x["W_up"], x["W_down"])
+    Y1 = lay.forward(x["X"], x["W_r"], x["bias"])
+    g1 = lay.backward(x["X"], x["W_r"], x["dY"])
+    torch.cuda.synchronize()
+    assert lay.error() == B.MOE_OK
+    counts = lay.routing()["counts"].cpu().numpy()
+    gids = lay.routing()["ids"].cpu().numpy()
+    del lay
+    torch.cuda.empty_cache()
+    assert torch.equal(Y.view(torch.int16), Y1.view(torch.int16))
+    assert torch.equal(g["dX"].view(torch.int16), g1["dX"].view(torch.int16))
+    assert torch.equal(g["dW_r"].view(torch.int32), g1["dW_r"].view(torch.int32))
+    del Y1, g1
+
+    def groups(el):
+        return [(int(cum[(m + 1) * El + el]) if m + 1 < nm else int(counts[el])) - int(cum[m * El + el])
+                for m in range(nm)]
+
+    X, Wr, dY = to64(x["X"]), to64(x["W_r"]), to64(x["dY"])
+    b = None if x["bias"] is None else to64(x["bias"])
+    lg64 = O.router_logits(X, Wr, b)
+    differ = np.nonzero(np.any(np.sort(O.topk_ids(lg64, w.k), 1) != np.sort(gids, 1), axis=1))[0]
+    tie_tokens = set(differ.tolist())
+    caches = {n: ExpertCache(x[n]) for n in ("W_gate", "W_up", "W_down")}
+    Wg, Wu, Wd = (lambda e, c=caches[n]: c(e - first) for n in ("W_gate", "W_up", "W_down"))
+    weights = {n: ExpertCache(x[n], keep=1) for n in ("W_gate", "W_up", "W_down")}
+    cache = mx_layout_cache([0, El - 1], weights)
+    for el in (0, El - 1):
+        e = first + el
+        _, ctx = O.forward_mx(X, Wr, b, Wg, Wu, Wd, w.k, first_local=e, num_local=1,
+                              rounded=lambda q: cache[q - first])
+        if set(ctx["sched"]["perm"].tolist()) & tie_tokens:
+            continue
+        go = O.backward_mx(ctx, dY, mx_wgrad=True, row_groups=lambda _l, el=el: groups(el))
+        for n in ("dW_gate", "dW_up", "dW_down"):
+            assert relerr(to64(g[n][el]), go[n][e]) <= TOL_MX, (n, e)
+    del cache
+    _, Y2, g2 = run()
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+    for n in ("dX", "dW_gate", "dW_up", "dW_down"):
+        assert torch.equal(g[n].view(torch.int16), g2[n].view(torch.int16)), n
+    del Y, Y2, g, g2, x
+    torch.cuda.empty_cache()
+
+
 def test_full_size_ep64_ring_stream():
     # Config 5 at n = 4096 tokens per local expert: 16 minibatches of 2048 tokens through the
     # 256 MiB ring, 6 local experts of 384; the backward replays part of the stream into the
