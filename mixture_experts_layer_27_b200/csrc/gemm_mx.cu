@@ -16,12 +16,13 @@
 // its epilogue overlaps the next tile's MMAs.
 //
 // The weight-gradient GEMMs contract over an expert's rows: their operands are
-// quantised along the rows (k_quant_rows) and stored transposed, so they too are
-// K-major; a tile is 128 weight rows x 256 weight columns of one expert, K the
-// expert's real rows in 128-row stages (the last stage issues only the K = 32
-// steps that hold real rows).  Their epilogue moves the accumulator to registers,
-// releases it at once, and writes the gradient through shared memory with TMA
-// box stores.
+// quantised along the rows by their producers (the dispatch, the reverse-combine
+// and the dgrad of W_down) and stored K-major in 128-row tiles (rowq_index), so a
+// 128-row K stage of either operand is one TMA box; a tile is 128 weight rows x 256
+// weight columns of one expert, K the real rows of each of the expert's segments in
+// 128-row stages (the last stage of a segment issues only the K = 32 steps that hold
+// real rows).  Their epilogue moves the accumulator to registers, releases it at
+// once, and writes the gradient through shared memory with TMA box stores.
 #include "moe_internal.cuh"
 #include "ptx.cuh"
 
