@@ -329,7 +329,9 @@ def oracle_window(w: IN.Workload) -> tuple:
 
 
 def oracle_sample(w: IN.Workload, x_cpu: dict) -> tuple:
-    """(seconds, assignments) of one oracle fwd+bwd over the sampled expert window."""
+    """(seconds, assignments) of one oracle fwd+bwd over the sampled expert window: the fp64
+    layer, or for MXFP8 workloads the MXFP8 layer (weights rounded once, as the GPU path prepares
+    them once per optimiser step, outside the timed step; weight gradients as the run has them)."""
     import numpy as np
     import oracle as O
 
@@ -341,18 +343,27 @@ def oracle_sample(w: IN.Workload, x_cpu: dict) -> tuple:
     b = None if x_cpu["bias"] is None else f64(x_cpu["bias"])
     Wg, Wu, Wd = (f64(x_cpu[n]) for n in ("W_gate", "W_up", "W_down"))
     first = w.first_local + e0
+    if w.mxfp8 and "mx_layouts" not in x_cpu:
+        x_cpu["mx_layouts"] = {first + e: O.mx_weight_layouts(Wg[e], Wu[e], Wd[e]) for e in range(m)}
     t0 = time.perf_counter()
-    _, ctx = O.forward(X, Wr, b, lambda e: Wg[e - first], lambda e: Wu[e - first], lambda e: Wd[e - first], w.k,
-                       first_local=first, num_local=m)
-    O.backward(ctx, dY)
+    if w.mxfp8:
+        lay = x_cpu["mx_layouts"]
+        _, ctx = O.forward_mx(X, Wr, b, lambda e: Wg[e - first], lambda e: Wu[e - first], lambda e: Wd[e - first], w.k,
+                              first_local=first, num_local=m, rounded=lay.__getitem__)
+        O.backward_mx(ctx, dY, mx_wgrad=x_cpu.get("mx_wgrad", False))
+    else:
+        _, ctx = O.forward(X, Wr, b, lambda e: Wg[e - first], lambda e: Wu[e - first], lambda e: Wd[e - first], w.k,
+                           first_local=first, num_local=m)
+        O.backward(ctx, dY)
     dt = time.perf_counter() - t0
     return dt, int(ctx["sched"]["offsets"][-1])
 
 
-def cpu_inputs(w: IN.Workload) -> dict:
+def cpu_inputs(w: IN.Workload, mx_wgrad: bool = False) -> dict:
     """Host copies of the inputs the sample needs (CPU generator; same distributions)."""
     e0, m = oracle_window(w)
-    x = {"X": IN._normal((w.tokens, w.d), 1.0, IN._seed(w.seed, w.name, "X"), "cpu"),
+    x = {"mx_wgrad": mx_wgrad,
+         "X": IN._normal((w.tokens, w.d), 1.0, IN._seed(w.seed, w.name, "X"), "cpu"),
          "W_r": IN._normal((w.d, w.E), 0.02, IN._seed(w.seed, w.name, "W_r"), "cpu"),
          "dY": IN._normal((w.tokens, w.d), 1.0, IN._seed(w.seed, w.name, "dY"), "cpu"), "window": (e0, m)}
     for n in ("W_gate", "W_up", "W_down"):
@@ -387,15 +398,16 @@ def oracle_rate(w: IN.Workload, x_cpu: dict, steps: int) -> dict:
     e0, m = x_cpu["window"]
     med = statistics.median(ts)  # the median step: robust to a step disturbed by other host work
     return {"value": asg[0] / w.k / med, "seconds": ts, "assignments": asg[0],
-            "sample": (f"fp64 numpy oracle, measured (no extrapolation): each step routes all {w.tokens} tokens and "
+            "sample": (f"fp64 numpy oracle{' (MXFP8 layer' + (', MX weight gradients' if x_cpu.get('mx_wgrad') else '') + ')' if w.mxfp8 else ''}, "
+                       f"measured (no extrapolation): each step routes all {w.tokens} tokens and "
                        f"runs forward + backward of local experts {e0}..{e0 + m - 1} ({asg[0]} of the "
                        f"{w.tokens * w.k if w.El == w.E else 'local'} assignments, weight gradients included); "
                        f"rate = assignments / top_k / the median of {steps} measured steps "
                        f"({med:.2f} s; {min(ts):.2f}-{max(ts):.2f} s)")}
 
 
-def cpu_baseline(w: IN.Workload) -> dict:
-    x = cpu_inputs(w)
+def cpu_baseline(w: IN.Workload, mx_wgrad: bool = False) -> dict:
+    x = cpu_inputs(w, mx_wgrad)
     oracle_sample(w, x)  # first call: imports, BLAS start-up
     r = oracle_rate(w, x, CPU_BASELINE_STEPS)
     return {"value": r["value"], "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle", "sample": r["sample"]}
@@ -440,7 +452,7 @@ def barrier(world: int):
 def run_reference(args, w: IN.Workload, world: int, rank: int):
     if rank != 0:
         return
-    x = cpu_inputs(w)
+    x = cpu_inputs(w, args.mx_wgrad)
     for _ in range(args.warmup):
         oracle_sample(w, x)
     r = oracle_rate(w, x, args.steps)
@@ -758,7 +770,7 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
         line["stream_plan"] = {"macrobatches": int(pl[0]), "backward_chunks": int(pl[1]), "padded_rows": int(pl[2]),
                                "replayed_rows": int(pl[3]), "resident_rows": int(pl[4]), "ring_rows": int(pl[5])}
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w)
+        line["cpu_baseline"] = cpu_baseline(w, args.mx_wgrad)
     print(json.dumps(line), flush=True)
 
 
