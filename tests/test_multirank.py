@@ -65,7 +65,7 @@ def test_reference_arm_runs_on_rank_0_only(capsys):
     from mixture_experts_layer_27_b200 import inputs as IN
 
     class Args:  # the reference arm's arguments; rank 1 must return before doing any work
-        gpus, steps, warmup, wgrad_fp32, persistent = 2, 1, 3, False, False
+        gpus, steps, warmup, wgrad_fp32, persistent, mx_wgrad = 2, 1, 3, False, False, False
     bench.run_reference(Args, IN.WORKLOADS["tiny"], world=2, rank=1)
     assert capsys.readouterr().out == ""
 
@@ -77,7 +77,7 @@ def test_reference_arm_prints_one_line_on_rank_0(capsys):
     from mixture_experts_layer_27_b200 import inputs as IN
 
     class Args:
-        gpus, steps, warmup, wgrad_fp32, persistent = 2, 2, 3, False, False
+        gpus, steps, warmup, wgrad_fp32, persistent, mx_wgrad = 2, 2, 3, False, False, False
     w = IN.WORKLOADS["tiny"]
     bench.run_reference(Args, w, world=2, rank=0)
     lines = capsys.readouterr().out.strip().splitlines()
