@@ -253,7 +253,8 @@ size_t moe_weights_size(const moe_shape* shape);
  * code of padded row R, column c; scales (RP*C/32 bytes) sit in 512-byte chunks,
  * byte (c%32)*16 + ((c%128)/32)*4 + (R%128)/32 of chunk (R/128)*(C/128) + c/128.
  * Tiles past an expert's real rows hold whatever the buffer held.  Device pointers;
- * MOE_ERR_INVALID_ARG for another precision or `which`. */
+ * MOE_ERR_INVALID_ARG for another precision or `which`.  One-batch buffers (moe_fwd_mx /
+ * moe_bwd_mx) only: a ring-streamed layer's ctx and ws are laid out for its minibatches. */
 moe_status moe_debug_mx_wgrad_operand(const moe_shape* shape, const void* ctx, const void* ws, int32_t which,
                                       void* codes, void* scales, void* stream);
 /* Padded-row capacity RP of a shape (rows of X_perm and the other row buffers); 0 if invalid. */
