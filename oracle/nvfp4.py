@@ -1,0 +1,180 @@
+"""Oracle of the NVFP4 layer forward (test infrastructure only).
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg
+use it.  It shares no code, table or helper with the CUDA path.
+
+What it follows
+---------------
+Page 1 ("Cursor open-sources Mixture-of-Kittens (MoK)...", section "MoE layer as
+the bottleneck") names NVFP4 training kernels as earlier work and says nothing
+of the format.  NVFP4 is taken here as NVIDIA publishes it:
+
+* element: E2M1 (1 sign, 2 exponent bits with bias 1, 1 mantissa bit), the
+  magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6;
+* first level: one positive E4M3 scale per 16 consecutive values along the
+  contraction dimension of the GEMM that reads them;
+* second level: one fp32 scale per tensor, chosen so that the tensor's largest
+  magnitude maps to the largest product of the two formats (6 x 448 = 2688).
+
+Readings (the pages are silent, so each is the plainest one; all are listed in
+the design notes):
+
+* global scale  gs = 2688 / amax(tensor) in fp32 (amax = 0 gives gs = 1; an
+  overflow is clamped to the largest fp32);
+* block scale   s  = e4m3_rn_satfinite((amax_block / 6) * gs), fp32 steps;
+* codes         q  = e2m1_rn_satfinite(v * (gs / s)), fp32 steps; a block whose
+  scale rounds to 0 holds zeros;
+* value         q * s / gs;
+* every quantisation decision (scale byte, code) is taken in fp32, the
+  kernels' precision, on the fp32 value of the input;
+* "tensor" is the operand as the layer holds it: X [T, d] (one scale for all
+  tokens), each of W_gate, W_up, W_down over the local experts, and H over all
+  assigned rows of the layer; a GEMM's output is multiplied back by
+  1 / (gs_A gs_B);
+* H = silu(A) * B from the unrounded A, B (as in the MXFP8 oracle).
+
+Only the forward is defined in this mode.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .moe_oracle import (_expert, _expert_rows, _f64, e4m3_decode, e4m3_encode, gates, router_logits,
+                         schedule, silu, topk_ids)
+
+NV_BLOCK = 16
+E2M1_MAX = 6.0
+NV_GS_NUM = 2688.0  # 6 * 448: the largest E2M1 magnitude times the largest E4M3 one
+
+# E2M1 magnitudes by code (bits e1 e0 m): subnormal 0.5 at e = 0, then 1, 1.5, 2, 3, 4, 6
+E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    """4-bit E2M1 codes (sign in bit 3) -> fp64."""
+    c = np.asarray(codes, dtype=np.int64)
+    return np.where(c & 8, -1.0, 1.0) * E2M1_GRID[c & 7]
+
+
+def e2m1_encode(x) -> np.ndarray:
+    """fp64 -> E2M1 code: nearest magnitude, halfway cases to the even code (mantissa bit 0),
+    magnitudes above 6 saturate to 6.  The sign of a value that rounds to zero is kept."""
+    x = _f64(x)
+    a = np.minimum(np.abs(x), E2M1_MAX)
+    dist = np.abs(a[..., None] - E2M1_GRID)
+    dmin = dist.min(axis=-1, keepdims=True)
+    near = dist == dmin
+    # among the (at most two) nearest magnitudes, prefer the even code
+    even = near & ((np.arange(8) & 1) == 0)
+    pick = np.where(even.any(axis=-1), np.argmax(even, axis=-1), np.argmax(near, axis=-1))
+    return (pick | (np.signbit(x).astype(np.int64) << 3)).astype(np.uint8)
+
+
+def nv_global_scale(v) -> np.float32:
+    """fp32 second-level scale of a whole tensor: 2688 / amax (1 for an all-zero tensor)."""
+    amax = np.float32(np.max(np.abs(np.asarray(v, dtype=np.float64).astype(np.float32)))) if np.size(v) else 0
+    if amax == 0:
+        return np.float32(1.0)
+    with np.errstate(over="ignore"):
+        gs = np.float32(NV_GS_NUM) / np.float32(amax)
+    return np.float32(min(gs, np.finfo(np.float32).max))
+
+
+def nv_quantize(v, gs, axis: int = -1):
+    """NVFP4 block quantisation of v along `axis` (blocks of 16) under global scale gs.
+
+    Returns (codes uint8 with one 4-bit code per value, same shape as v;
+    scale bytes uint8 (E4M3) with the block axis shortened 16 times)."""
+    v32 = np.moveaxis(np.asarray(v, dtype=np.float64).astype(np.float32), axis, -1)
+    n = v32.shape[-1]
+    if n % NV_BLOCK:
+        raise ValueError("length along the block axis must be a multiple of 16")
+    vb = v32.reshape(v32.shape[:-1] + (n // NV_BLOCK, NV_BLOCK))
+    gs = np.float32(gs)
+    amax = np.max(np.abs(vb), axis=-1)
+    s = (amax / np.float32(6.0)).astype(np.float32) * gs  # fp32 divide, then fp32 multiply
+    sbytes = e4m3_encode(s.astype(np.float32).astype(np.float64))
+    sdec = e4m3_decode(sbytes).astype(np.float32)
+    zero = sdec == 0
+    with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
+        inv = np.where(zero, np.float32(0.0), gs / np.where(zero, np.float32(1.0), sdec)).astype(np.float32)
+        x = (vb * inv[..., None]).astype(np.float32)
+    codes = e2m1_encode(x.astype(np.float64))
+    codes[zero] = 0
+    codes = np.moveaxis(codes.reshape(v32.shape), -1, axis)
+    return codes, np.moveaxis(sbytes, -1, axis)
+
+
+def nv_dequantize(codes, sbytes, gs, axis: int = -1) -> np.ndarray:
+    c = np.moveaxis(np.asarray(codes), axis, -1)
+    s = e4m3_decode(np.moveaxis(np.asarray(sbytes), axis, -1))
+    vals = e2m1_decode(c).reshape(c.shape[:-1] + (c.shape[-1] // NV_BLOCK, NV_BLOCK)) * s[..., None]
+    return np.moveaxis(vals.reshape(c.shape) / np.float64(np.float32(gs)), -1, axis)
+
+
+def nv_round(v, gs, axis: int) -> np.ndarray:
+    """v rounded to its NVFP4 value along `axis` under global scale gs (fp64)."""
+    c, s = nv_quantize(v, gs, axis=axis)
+    return nv_dequantize(c, s, gs, axis=axis)
+
+
+def nv_weight_scales(W_gate, W_up, W_down, first_local: int = 0, num_local: int | None = None):
+    """Global scales of the three weight tensors over the local experts."""
+    if num_local is None and callable(W_gate):
+        raise ValueError("num_local is needed when the weights come from a callable")
+    n = num_local if num_local is not None else len(W_gate) - first_local
+    out = []
+    for W in (W_gate, W_up, W_down):
+        amax = np.float32(0.0)
+        for e in range(first_local, first_local + n):
+            amax = max(amax, np.float32(np.max(np.abs(_f64(_expert(W, e)).astype(np.float32)))))
+        with np.errstate(over="ignore"):
+            out.append(np.float32(NV_GS_NUM) / amax if amax > 0 else np.float32(1.0))
+    return tuple(np.float32(min(g, np.finfo(np.float32).max)) for g in out)
+
+
+def forward_nv(X, W_r, bias, W_gate, W_up, W_down, top_k: int, first_local: int = 0,
+               num_local: int | None = None, gs_w=None):
+    """NVFP4 layer forward: the routing of `forward`, then per local expert
+    A = Xq Wgq, B = Xq Wuq (K = d), H = silu(A) B, O = Hq Wdq (K = I), Y = sum_j g O.
+
+    gs_w: optional (gs_gate, gs_up, gs_down) computed once by the caller
+    (nv_weight_scales); without it they are computed here.
+    Returns (Y, info) with the routing, the five global scales and, per local expert,
+    (tokens, slots, H, A, B) or None."""
+    X64 = _f64(X)
+    T, d = X64.shape
+    E = np.asarray(W_r).shape[1]
+    logits = router_logits(X64, W_r, bias)
+    ids = topk_ids(logits, top_k)
+    g = gates(logits, ids)
+    sched = schedule(ids, E, first_local, num_local)
+    nl = sched["num_local"]
+    if gs_w is None:
+        gs_w = nv_weight_scales(W_gate, W_up, W_down, first_local, nl)
+    gs_g, gs_u, gs_d = gs_w
+    gs_x = nv_global_scale(X64)
+    Hs = []
+    for el in range(nl):
+        toks, slots = _expert_rows(ids, sched, el)
+        if toks.size == 0:
+            Hs.append(None)
+            continue
+        e = el + first_local
+        Xq = nv_round(X64[toks], gs_x, axis=1)  # K = d
+        A = Xq @ nv_round(_expert(W_gate, e), gs_g, axis=0)
+        B = Xq @ nv_round(_expert(W_up, e), gs_u, axis=0)
+        Hs.append((toks, slots, silu(A) * B, A, B))
+    live = [h[2] for h in Hs if h is not None]
+    gs_h = nv_global_scale(np.concatenate(live, axis=0)) if live else np.float32(1.0)
+    Y = np.zeros((T, d))
+    for el, h in enumerate(Hs):
+        if h is None:
+            continue
+        toks, slots, H = h[:3]
+        O = nv_round(H, gs_h, axis=1) @ nv_round(_expert(W_down, el + first_local), gs_d, axis=0)  # K = I
+        Y[toks] += g[toks, slots][:, None] * O
+    info = dict(ids=ids, g=g, sched=sched, gs_x=gs_x, gs_h=gs_h, gs_w=(gs_g, gs_u, gs_d), experts=Hs)
+    return Y, info
