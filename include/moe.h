@@ -64,7 +64,9 @@ typedef enum moe_precision {
   MOE_MXFP8_ALL = 2  /* MOE_MXFP8 with the two weight-gradient GEMMs on MXFP8 as well: their
                         operands (X, dA, dB, Hg = g H and dY of each expert) quantised along the
                         expert's rows, one scale per 32 rows from its first row, pad rows zero.
-                        Same entry points; a larger workspace (moe_workspace_size of this shape) */
+                        Same entry points; a larger workspace (moe_workspace_size of this shape) */,
+  MOE_NVFP4 = 3  /* forward only (moe_fwd_nvfp4): E2M1 operands with one E4M3 scale per 16 values
+                    along each GEMM's contraction dim and one fp32 scale per tensor */
 } moe_precision;
 
 typedef enum moe_wgrad_dtype {
@@ -267,6 +269,45 @@ moe_status moe_fwd_mx(const moe_shape* shape, const void* X, const void* W_r, co
 moe_status moe_bwd_mx(const moe_shape* shape, const void* X, const void* W_r, const void* wq, size_t wq_bytes,
                       const void* dY, void* ctx, size_t ctx_bytes, void* dX, void* dW_gate, void* dW_up,
                       void* dW_down, float* dW_r, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * NVFP4 forward (page 1, "MoE layer as the bottleneck": NVFP4 training kernels
+ * named as earlier work; the format is NVIDIA's published NVFP4).  Shapes carry
+ * prec = MOE_NVFP4.  Each GEMM operand is E2M1 (values 0, 0.5, 1, 1.5, 2, 3, 4,
+ * 6 and their negatives) with one E4M3 scale per 16 values along the GEMM's
+ * contraction dimension and one fp32 global scale per tensor:
+ *   gs = 2688 / amax(tensor)  (1 for an all-zero tensor),
+ *   block scale s = e4m3((amax_block / 6) * gs), codes q = e2m1(v * (gs / s)),
+ *   value = q * s / gs,
+ * every step in fp32 with round-to-nearest-even and saturation (6, 448); a block
+ * whose scale rounds to 0 holds zeros.  The tensors are X [T, d] (along d), the
+ * local experts' W_gate, W_up (along d) and W_down (along I), and H [rows, I]
+ * over every assigned row (along I); the gate/up and down GEMMs run on
+ * kind::mxf4nvf4 block-scaled tensor cores (K = 64 per MMA) and multiply their
+ * fp32 accumulators by 1 / (gs_A gs_B).  H = silu(A) B is formed in fp32 by the
+ * gate/up GEMM, its amax sets its global scale, then it is quantised.  Routing
+ * is the bf16 router's, Y is bf16.  Forward only: there is no NVFP4 backward.
+ *
+ * moe_prepare_weights with an MOE_NVFP4 shape quantises W_gate, W_up, W_down
+ * (the local experts' [El, d, I], [El, d, I], [El, I, d] bf16) into wq
+ * (moe_weights_size of that shape): [Wgu codes][Wgu scales][Wd2 codes][Wd2 scales]
+ * [global scales], each region on a 256-byte boundary; Wgu [El*2I, d/2 bytes]
+ * has the MXFP8 Wgu row order, Wd2 [El*d, I/2 bytes] is W_down transposed; two
+ * codes per byte, value 2i in the low nibble of byte i; scale byte
+ * (r%32)*16 + ((r%128)/32)*4 + (k%64)/16 of 512-byte chunk (r/128)*(K/64) + k/64;
+ * the global scales are three fp32 (gate, up, down).  moe_fwd_nvfp4 takes
+ * moe_fwd_mx's arguments; ctx and ws are sized by moe_ctx_size /
+ * moe_workspace_size of the MOE_NVFP4 shape; d and I multiples of 256 as
+ * everywhere.  Errors as for moe_fwd_mx; moe_get_error reads the device status. */
+moe_status moe_fwd_nvfp4(const moe_shape* shape, const void* X, const void* W_r, const float* bias, const void* wq,
+                         size_t wq_bytes, void* Y, void* ctx, size_t ctx_bytes, void* ws, size_t ws_bytes,
+                         void* stream);
+/* Test hook: byte offsets of the NVFP4 forward's buffers.  out[0..1]: X codes and scales in
+ * ctx; out[2..5]: H codes, H scales, fp32 H [RP, I] and four scale words (amax X, amax H as
+ * fp32 bits, then gs_X, gs_H) in ws; out[6..10]: Wgu codes, Wgu scales, Wd2 codes, Wd2
+ * scales and the three weight global scales in wq.  Host only; MOE_ERR_INVALID_ARG for
+ * another precision or a NULL out. */
+moe_status moe_debug_nv_offsets(const moe_shape* shape, int64_t* out);
 
 /* ---------------------------------------------------------------------------
  * Ring-streamed layer (page 1, "Three design decisions that matter", bullet 3:

@@ -23,6 +23,7 @@ MOE_ERR_EXCHANGE = 7
 MOE_BF16 = 0
 MOE_MXFP8 = 1
 MOE_MXFP8_ALL = 2  # MOE_MXFP8 with the weight-gradient GEMMs on MXFP8 too (operands along tokens)
+MOE_NVFP4 = 3  # forward only: E2M1 operands, E4M3 scale per 16 along K, fp32 scale per tensor
 MOE_WGRAD_BF16 = 0
 MOE_WGRAD_FP32 = 1
 
@@ -142,6 +143,9 @@ _SIGS = {
                                   _P]),
     "moe_bwd_mx": (ctypes.c_int, [_S, _P, _P, _P, ctypes.c_size_t, _P, _P, ctypes.c_size_t, _P, _P, _P, _P, _P, _P,
                                   ctypes.c_size_t, _P]),
+    "moe_fwd_nvfp4": (ctypes.c_int, [_S, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, ctypes.c_size_t, _P,
+                                     ctypes.c_size_t, _P]),
+    "moe_debug_nv_offsets": (ctypes.c_int, [_S, ctypes.POINTER(ctypes.c_int64)]),
     "moe_ep_buffer_size": (ctypes.c_size_t, [_S, ctypes.c_int32]),
     "moe_ep_ctx_size": (ctypes.c_size_t, [_S, ctypes.c_int32]),
     "moe_ep_workspace_size": (ctypes.c_size_t, [_S, ctypes.c_int32]),
@@ -362,6 +366,17 @@ def moe_bwd_mx(shape, X, W_r, wq, dY, ctx, dX, dW_gate, dW_up, dW_down, dW_r, ws
                                 _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
+def moe_fwd_nvfp4(shape, X, W_r, bias, wq, Y, ctx, ws, stream=None) -> int:
+    return int(lib().moe_fwd_nvfp4(ctypes.byref(shape), _ptr(X), _ptr(W_r), _ptr(bias), _ptr(wq), _nbytes(wq),
+                                   _ptr(Y), _ptr(ctx), _nbytes(ctx), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def moe_debug_nv_offsets(shape) -> list:
+    out = (ctypes.c_int64 * 11)()
+    check(int(lib().moe_debug_nv_offsets(ctypes.byref(shape), out)), "moe_debug_nv_offsets")
+    return [int(v) for v in out]
+
+
 def check(status: int, what: str = "moe"):
     if status != MOE_OK:
         raise MoeError(status, what)
@@ -462,6 +477,102 @@ class MoELayerMX:
 
     def error(self, stream=None) -> int:
         return moe_get_error(self.ctx, stream)
+
+
+class MoELayerNVFP4:
+    """NVFP4 layer forward: prepared (quantised) weights + ctx / workspace owner."""
+
+    def __init__(self, T, d, E, I, top_k, first_local_expert=0, num_local_experts=0, device="cuda"):
+        import torch
+        self.shape = make_shape(T, d, E, I, top_k, MOE_NVFP4, first_local_expert, num_local_experts)
+        self.shape_bf16 = make_shape(T, d, E, I, top_k, MOE_BF16, first_local_expert, num_local_experts)
+        nc, nw, nq = moe_ctx_size(self.shape), moe_workspace_size(self.shape), moe_weights_size(self.shape)
+        if nc == 0 or nw == 0 or nq == 0:
+            raise MoeError(MOE_ERR_UNSUPPORTED, "shape")
+        self.ctx = torch.empty(nc, dtype=torch.uint8, device=device)
+        self.ws = torch.empty(nw, dtype=torch.uint8, device=device)
+        self.wq = torch.empty(nq, dtype=torch.uint8, device=device)
+        self.T, self.d, self.E, self.I, self.k = T, d, E, I, top_k
+        self.El = num_local_experts or (E - first_local_expert)
+        self.off = moe_debug_nv_offsets(self.shape)
+
+    def prepare(self, W_gate, W_up, W_down, stream=None):
+        _expect_layer(self, self.T, W_gate=W_gate, W_up=W_up, W_down=W_down)
+        check(moe_prepare_weights(self.shape, W_gate, W_up, W_down, self.wq, stream), "moe_prepare_weights")
+
+    def forward(self, X, W_r, bias, Y=None, stream=None):
+        import torch
+        if Y is None:
+            Y = torch.empty(self.T, self.d, dtype=torch.bfloat16, device=X.device)
+        _expect_layer(self, self.T, X=X, W_r=W_r, bias=bias, Y=Y)
+        check(moe_fwd_nvfp4(self.shape, X, W_r, bias, self.wq, Y, self.ctx, self.ws, stream), "moe_fwd_nvfp4")
+        return Y
+
+    # --- test accessors (host numpy copies; unpacked codes: one 4-bit code per byte) ---
+    @staticmethod
+    def _unpack(packed, R, K):
+        import numpy as np
+        b = np.asarray(packed, dtype=np.uint8).reshape(R, K // 2)
+        out = np.empty((R, K), dtype=np.uint8)
+        out[:, 0::2] = b & 0xF
+        out[:, 1::2] = b >> 4
+        return out
+
+    def _operand(self, buf, o_codes, o_scales, R, K):
+        a = buf.cpu().numpy()
+        codes = self._unpack(a[o_codes:o_codes + R * K // 2], R, K)
+        return codes, unchunk_scales_nv(a[o_scales:o_scales + R * K // 16], R, K)
+
+    def x_operand(self):
+        """(codes [RP, d], scale bytes [RP, d/16]) of the dispatched X of the last forward."""
+        torch_sync()
+        return self._operand(self.ctx, self.off[0], self.off[1], moe_padded_rows(self.shape_bf16), self.d)
+
+    def h_operand(self):
+        """(codes [RP, I], scale bytes [RP, I/16]) of the quantised H of the last forward."""
+        torch_sync()
+        return self._operand(self.ws, self.off[2], self.off[3], moe_padded_rows(self.shape_bf16), self.I)
+
+    def h_fp32(self):
+        import numpy as np
+        torch_sync()
+        RP = moe_padded_rows(self.shape_bf16)
+        a = self.ws.cpu().numpy()
+        return a[self.off[4]:self.off[4] + RP * self.I * 4].view(np.float32).reshape(RP, self.I)
+
+    def scales(self):
+        """(gs_X, gs_H) of the last forward and (gs_gate, gs_up, gs_down) of the prepared weights."""
+        import numpy as np
+        torch_sync()
+        w = self.ws.cpu().numpy()[self.off[5]:self.off[5] + 16].view(np.float32)
+        q = self.wq.cpu().numpy()[self.off[10]:self.off[10] + 12].view(np.float32)
+        return (w[2], w[3]), tuple(q)
+
+    def weight_regions(self):
+        """{"Wgu": (codes [El*2I, d], scales [El*2I, d/16]), "Wd2": (codes [El*d, I], scales [El*d, I/16])}."""
+        El, d, I = self.El, self.d, self.I
+        return {"Wgu": self._operand(self.wq, self.off[6], self.off[7], El * 2 * I, d),
+                "Wd2": self._operand(self.wq, self.off[8], self.off[9], El * d, I)}
+
+    def routing(self):
+        return MoELayer.routing(self)
+
+    def error(self, stream=None) -> int:
+        return moe_get_error(self.ctx, stream)
+
+
+def torch_sync():
+    import torch
+    torch.cuda.synchronize()
+
+
+def unchunk_scales_nv(chunks, R, K):
+    """[R, K/16] scale bytes from the 512-byte chunk order of a K-major NVFP4 operand."""
+    import numpy as np
+    r = np.arange(R)[:, None]
+    kb = np.arange(K // 16)[None, :]
+    idx = ((r // 128) * (K // 64) + kb // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + kb % 4
+    return np.asarray(chunks)[idx]
 
 
 def unchunk_scales(chunks, R, K):

@@ -47,7 +47,7 @@ __device__ __forceinline__ void mx_wseg(const MxParams& p, int m, int el, int& r
 
 template <int KIND>
 __device__ __forceinline__ int mx_ntiles_n(const MxParams& p) {
-  if (KIND == MX_GATEUP) return p.I / (mx_bn(KIND) / 2);  // per tile: [64 gate | 64 up] column pairs
+  if (KIND == MX_GATEUP || KIND == NV_GATEUP) return p.I / (mx_bn(KIND) / 2);  // per tile: [64 gate | 64 up] column pairs
   if (KIND == MX_DGRAD_DOWN) return p.I / mx_bn(KIND);
   if (KIND == MX_WGRAD_GATEUP) return 2 * p.I / 256;  // gate n-tiles, then up n-tiles
   return p.d / mx_bn(KIND);  // MX_DOWN, MX_DGRAD_GATEUP, MX_WGRAD_DOWN
@@ -59,6 +59,8 @@ __device__ __forceinline__ int mx_mtiles_w(const MxParams& p) {
 }
 template <int KIND>
 __device__ __forceinline__ int mx_kblocks(const MxParams& p) {
+  if (KIND == NV_GATEUP) return p.d / 256;  // 128-byte K stages of 256 E2M1 codes
+  if (KIND == NV_DOWN) return p.I / 256;
   if (KIND == MX_GATEUP || KIND == MX_DGRAD_DOWN) return p.d / 128;
   if (KIND == MX_DOWN) return p.I / 128;
   return 2 * p.I / 128;
@@ -111,7 +113,7 @@ __device__ __forceinline__ MxTile mx_decode(const MxParams& p, int t) {
   tl.el = seg % p.El;
   tl.m0 = p0 + mi * 128;
   tl.nt = nt;
-  tl.n0 = nt * (KIND == MX_GATEUP ? mx_bn(KIND) / 2 : mx_bn(KIND));  // MX_GATEUP: first column of H / A / B
+  tl.n0 = nt * (KIND == MX_GATEUP || KIND == NV_GATEUP ? mx_bn(KIND) / 2 : mx_bn(KIND));  // gate/up: first H column
   tl.nk = mx_kblocks<KIND>(p);
   return tl;
 }
@@ -129,6 +131,20 @@ __device__ __forceinline__ void mx_load(const MxParams& p, const MxTile& tl, int
   const CUtensorMap* mb = &p.tb0;
   const uint8_t* sfa = p.sfa0;
   const uint8_t* sfb = p.sfb0;
+  if constexpr (mx_is_nv(KIND)) {
+    // NVFP4: 128 bytes of K = 256 codes; per 128 rows the stage's four 64-deep scale chunks are
+    // contiguous (2 KB): A's, then those of B's two 128-row halves
+    const int brow = KIND == NV_GATEUP ? tl.el * 2 * p.I + tl.nt * BN : tl.el * p.d + tl.n0;
+    const int K = KIND == NV_GATEUP ? p.d : p.I;
+    const int arow = tl.m0;
+    tma_load_2d(sA, ma, bar, kb * 128, arow, pol_act);
+    tma_load_2d(sB, mb, bar, kb * 128, brow, pol_w);
+    bulk_load(sSF, sfa + (static_cast<size_t>(arow >> 7) * (K >> 6) + 4 * kb) * 512, 2048, bar);
+    bulk_load(sSF + 2048, sfb + (static_cast<size_t>(brow >> 7) * (K >> 6) + 4 * kb) * 512, 2048, bar);
+    bulk_load(sSF + 4096, sfb + (static_cast<size_t>((brow >> 7) + 1) * (K >> 6) + 4 * kb) * 512, 2048, bar);
+    (void)krow;
+    return;
+  }
   if constexpr (mx_is_wgrad(KIND)) {
     // the K block = row tile kt = krow / 128 of both operands (rowq layout): A = lines
     // kt CA + m0 .., B = lines kt CB + nb .. of 128 codes, and the tile's scale chunks
@@ -268,6 +284,45 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
         mx_store_bf16_32(p.out1 + Rz * p.I + col, b);
         mx_store_q32(p.q0, p.qs0, R, col, p.I, h);  // H, the down GEMM's A operand (K = I)
       }
+    }
+  } else if constexpr (KIND == NV_GATEUP) {
+    // A = acc / (gs_X gs_gate), B = acc / (gs_X gs_up); H = silu(A) B in fp32 for the second pass
+    // (its amax sets H's global scale), the warp's largest |H| into *amax
+    const float ag = __frcp_rn(__fmul_rn(__ldg(p.gsa), __ldg(p.gsb)));
+    const float au = __frcp_rn(__fmul_rn(__ldg(p.gsa), __ldg(p.gsb + 1)));
+    float hmax = 0.f;
+#pragma unroll 1
+    for (int c = cbeg; c < cend; ++c) {
+      const int j = c >> 1, c32 = (c & 1) * 32;
+      float a[32], b[32];
+      tmem_ld32(taddr + j * 128 + c32, a);       // gate
+      tmem_ld32(taddr + j * 128 + 64 + c32, b);  // up
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float av = a[i] * ag;
+        a[i] = av / (1.0f + expf(-av)) * (b[i] * au);
+        hmax = fmaxf(hmax, fabsf(a[i]));
+      }
+      if (live) {
+        float4* dst = reinterpret_cast<float4*>(p.hout + Rz * p.I + tl.n0 + j * 64 + c32);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) dst[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+      }
+    }
+    if (!live) hmax = 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
+    if ((row & 31) == 0 && hmax > 0.f) atomicMax(p.amax, __float_as_uint(hmax));
+  } else if constexpr (KIND == NV_DOWN) {
+    const float al = __frcp_rn(__fmul_rn(__ldg(p.gsa), __ldg(p.gsb)));
+    const float g = p.row_gate[R];
+#pragma unroll 1
+    for (int c = cbeg; c < cend; ++c) {
+      float o[32];
+      tmem_ld32(taddr + c * 32, o);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = o[i] * al * g;
+      if (live) mx_store_bf16_32(p.out0 + Rz * p.d + tl.n0 + c * 32, o);
     }
   } else if constexpr (KIND == MX_DOWN) {
     const float g = p.row_gate[R];
@@ -544,6 +599,24 @@ __global__ void __launch_bounds__(mx_threads(KIND), 1) k_moe_gemm_mx(const __gri
           const uint32_t sf0 = b0 + static_cast<uint32_t>(BN * 128);
           // scale slot of this stage: 16 columns from column 256 on; A in the first 4,
           // B (rows 0..127, then 128..255) in the columns from 8 on
+          if constexpr (mx_is_nv(KIND)) {
+            // per stage 48 TMEM columns above the accumulator: A's four chunks (4 columns each),
+            // then per K = 64 step the two 128-row halves of B (8 columns)
+            const uint32_t nfa = tbase + 256 + stage * 48, nfb = nfa + 16;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              tc_cp_sf(nfa + 4 * kk, sf0 + 512 * kk);
+              tc_cp_sf(nfb + 8 * kk, sf0 + 2048 + 512 * kk);
+              tc_cp_sf(nfb + 8 * kk + 4, sf0 + 4096 + 512 * kk);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_nvf4(dtm, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024),
+                        idesc_nvf4(128, BN), nfa + 4 * kk, nfb + 8 * kk, (kb | kk) != 0 ? 1u : 0u);
+            umma_commit(&empty[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            continue;
+          }
           const uint32_t sfa_t = tbase + 256 + stage * 16, sfb_t = sfa_t + 8;
           tc_cp_sf(sfa_t, sf0);
           tc_cp_sf(sfb_t, sf0 + 512);
@@ -574,7 +647,7 @@ __global__ void __launch_bounds__(mx_threads(KIND), 1) k_moe_gemm_mx(const __gri
   } else {  // epilogue warps 2 .. 2 + EPI - 1
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    constexpr int NCH = KIND == MX_GATEUP ? BN / 64 : BN / 32;  // 32-column chunks of the epilogue
+    constexpr int NCH = KIND == MX_GATEUP || KIND == NV_GATEUP ? BN / 64 : BN / 32;  // 32-column chunks of the epilogue
     const int half = EPI == 8 ? (warp - 2) >> 2 : 0;
     const int cbeg = half * (NCH * 4 / EPI), cend = cbeg + NCH * 4 / EPI;
     int it = 0;
@@ -636,6 +709,8 @@ cudaError_t launch_gemm_mx(MxKind kind, const MxParams& p, int grid, cudaStream_
     case MX_DGRAD_GATEUP: return mx_launch_kind<MX_DGRAD_GATEUP>(p, grid, st);
     case MX_WGRAD_GATEUP: return mx_launch_kind<MX_WGRAD_GATEUP>(p, grid, st);
     case MX_WGRAD_DOWN: return mx_launch_kind<MX_WGRAD_DOWN>(p, grid, st);
+    case NV_GATEUP: return mx_launch_kind<NV_GATEUP>(p, grid, st);
+    case NV_DOWN: return mx_launch_kind<NV_DOWN>(p, grid, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -56,6 +56,7 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   };
   L->mx = s.prec == MOE_MXFP8 || s.prec == MOE_MXFP8_ALL;
   L->mxw = s.prec == MOE_MXFP8_ALL;
+  L->nv = s.prec == MOE_NVFP4;
   // row-quantised operands are addressed by TMA as RP / 128 * C lines (a signed 32-bit coordinate)
   if (L->mxw && (L->RP / 128) * static_cast<int64_t>(s.d > s.I ? s.d : s.I) >= (int64_t(1) << 31)) return false;
   L->hdr = take(HDR_WORDS * 4);
@@ -70,14 +71,15 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->row_asg = take(RP * 4);
   L->row_gate = take(RP * 4);
   // streamed layer: X_perm lives in the caller's ring; MXFP8 weight gradients keep X quantised instead
-  L->xperm = take(M > 0 || s.prec == MOE_MXFP8_ALL ? 0 : RP * s.d * 2);
+  L->xperm = take(M > 0 || s.prec == MOE_MXFP8_ALL || L->nv ? 0 : RP * s.d * 2);
   L->abuf = take(RP * s.I * 2);
   L->bbuf = take(RP * s.I * 2);
   L->stab = take(M > 0 ? static_cast<size_t>(stream_table_words(M, El)) * 4 : 0);
   const size_t mxd = L->mx ? RP * s.d : 0, mxi = L->mx ? RP * s.I : 0;  // fp8 bytes; scales are 1/32 of that
   // the one-batch MXFP8 forward's X codes (a ring-streamed layer keeps them in the caller's ring)
-  L->xq = take(M > 0 ? 0 : mxd);
-  L->xqs = take(M > 0 ? 0 : mxd / 32);
+  // (NVFP4: two codes per byte and one scale byte per 16 values)
+  L->xq = take(M > 0 ? 0 : (L->nv ? RP * s.d / 2 : mxd));
+  L->xqs = take(M > 0 ? 0 : (L->nv ? RP * s.d / 16 : mxd / 32));
   const size_t wxd = L->mxw ? RP * s.d : 0, wxi = L->mxw ? RP * s.I : 0;
   L->xqt = take(wxd);  // X along the rows, from the forward's dispatch for the weight gradients
   L->xqts = take(wxd / 32);
@@ -104,8 +106,10 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->wrt = take(static_cast<size_t>(s.E) * s.d * 2);
   L->dxperm = take(RP * s.d * 2);
   L->acc32 = take(M > 0 ? 2 * static_cast<size_t>(El) * s.d * s.I * 4 : 0);
-  L->hq = take(mxi);
-  L->hqs = take(mxi / 32);
+  L->hq = take(L->nv ? RP * s.I / 2 : mxi);
+  L->hqs = take(L->nv ? RP * s.I / 16 : mxi / 32);
+  L->nvh = take(L->nv ? RP * s.I * 4 : 0);
+  L->nvsc = take(L->nv ? 256 : 0);
   L->dyq = take(mxd);
   L->dyqs = take(mxd / 32);
   L->daq = take(mxi);
@@ -124,17 +128,21 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->ws_bytes = o;
   // prepared weights: [W_gate|W_up paired, K = d] [W_down^T, K = I] [W_down, K = d] [W_gate, K = I] [W_up, K = I]
   o = 0;
+  // NVFP4: the two forward layouts only (half a byte per value, a scale byte per 16), then the
+  // three global scales (and their amax words)
   const size_t w1 = static_cast<size_t>(El) * s.d * s.I;
-  L->wgu1 = take(2 * w1);
-  L->wgu1s = take(2 * w1 / 32);
-  L->wd2 = take(w1);
-  L->wd2s = take(w1 / 32);
-  L->wd3 = take(w1);
-  L->wd3s = take(w1 / 32);
-  L->wg4 = take(w1);
-  L->wg4s = take(w1 / 32);
-  L->wu4 = take(w1);
-  L->wu4s = take(w1 / 32);
+  const size_t wb = L->nv ? w1 / 2 : w1, wsb = L->nv ? w1 / 16 : w1 / 32, wbwd = L->nv ? 0 : 1;
+  L->wgu1 = take(2 * wb);
+  L->wgu1s = take(2 * wsb);
+  L->wd2 = take(wb);
+  L->wd2s = take(wsb);
+  L->wd3 = take(wbwd * wb);
+  L->wd3s = take(wbwd * wsb);
+  L->wg4 = take(wbwd * wb);
+  L->wg4s = take(wbwd * wsb);
+  L->wu4 = take(wbwd * wb);
+  L->wu4s = take(wbwd * wsb);
+  L->wnvgs = take(L->nv ? 256 : 0);
   L->wq_bytes = o;
   return true;
 }
@@ -176,8 +184,10 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
   c.fctl = nullptr;
   c.actcnt = c.actlist = nullptr;
   c.xact = nullptr;
-  c.xq = L.mx ? reinterpret_cast<uint8_t*>(C(L.xq)) : nullptr;
-  c.xqs = L.mx ? reinterpret_cast<uint8_t*>(C(L.xqs)) : nullptr;
+  c.xq = L.mx || L.nv ? reinterpret_cast<uint8_t*>(C(L.xq)) : nullptr;
+  c.xqs = L.mx || L.nv ? reinterpret_cast<uint8_t*>(C(L.xqs)) : nullptr;
+  c.nvh = (ws && L.nv) ? reinterpret_cast<float*>(W(L.nvh)) : nullptr;
+  c.nvsc = (ws && L.nv) ? reinterpret_cast<unsigned*>(W(L.nvsc)) : nullptr;
   c.hq = c.hqs = c.dyq = c.dyqs = c.daq = c.daqs = c.dbq = c.dbqs = nullptr;
   c.xqt = c.xqts = c.dyqt = c.dyqts = c.daqt = c.daqts = c.dbqt = c.dbqts = c.hgqt = c.hgqts = nullptr;
   if (L.mxw) {
@@ -194,7 +204,7 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
     c.hgqt = reinterpret_cast<uint8_t*>(W(L.hgqt));
     c.hgqts = reinterpret_cast<uint8_t*>(W(L.hgqts));
   }
-  if (ws && L.mx) {
+  if (ws && (L.mx || L.nv)) {
     c.hq = reinterpret_cast<uint8_t*>(W(L.hq));
     c.hqs = reinterpret_cast<uint8_t*>(W(L.hqs));
     c.dyq = reinterpret_cast<uint8_t*>(W(L.dyq));
@@ -317,7 +327,8 @@ enum KernelId {
   K_ROUTER_LOGITS, K_TOPK, K_SCAN, K_SCATTER, K_DISPATCH, K_GEMM_GATEUP, K_GEMM_DOWN, K_COMBINE,
   K_REV_COMBINE, K_GEMM_DGRAD_DOWN, K_ROUTER_BWD, K_ROUTER_WGRAD, K_TRANSPOSE_WR, K_GEMM_DGRAD_GATEUP, K_REV_DISPATCH,
   K_GEMM_WGRAD_GATEUP, K_GEMM_WGRAD_DOWN, K_PLAN, K_REPLAY, K_FINISH_ACC, K_QUANT_WEIGHTS, K_MARK_ROWS,
-  K_ACTIVE_COUNT, K_GATHER_ACTIVE, K_SCAN_GROUPS, K_SCAN_APPLY, K_PAIR_FWD, K_PAIR_DGRAD, K_MX_WGRAD_GATEUP, K_MX_WGRAD_DOWN, K_NUM
+  K_ACTIVE_COUNT, K_GATHER_ACTIVE, K_SCAN_GROUPS, K_SCAN_APPLY, K_PAIR_FWD, K_PAIR_DGRAD, K_MX_WGRAD_GATEUP, K_MX_WGRAD_DOWN,
+  K_NV_SCALE, K_NV_GATEUP, K_NV_QUANT_H, K_NV_DOWN, K_NUM
 };
 static const char* kKernelNames[K_NUM] = {
     "router_logits", "topk_gating", "hist_scan", "stable_scatter", "dispatch", "gemm_gateup_swiglu",
@@ -325,7 +336,8 @@ static const char* kKernelNames[K_NUM] = {
     "transpose_wr", "gemm_dgrad_gateup", "reverse_dispatch", "gemm_wgrad_gateup", "gemm_wgrad_down",
     "stream_plan", "ring_replay", "wgrad_accumulator_finish", "quantize_weights", "mark_pad_rows",
     "router_token_count", "router_token_gather", "hist_scan_group_sums", "hist_scan_group_apply",
-    "gemm_gateup_down_persistent", "gemm_dgrads_persistent", "gemm_wgrad_gateup_mx", "gemm_wgrad_down_mx"};
+    "gemm_gateup_down_persistent", "gemm_dgrads_persistent", "gemm_wgrad_gateup_mx", "gemm_wgrad_down_mx",
+    "nvfp4_amax_scale", "gemm_gateup_swiglu_nvfp4", "nvfp4_quantize_h", "gemm_down_combw_nvfp4"};
 
 struct ProfRec {
   int kid;
@@ -1276,14 +1288,61 @@ moe_status moe_debug_stream_plan(const moe_shape* s, int32_t M, const void* ctx,
 // ---------------------------------------------------------------------------
 // MXFP8 mode
 // ---------------------------------------------------------------------------
+static moe_status check_shape_nv(const moe_shape* s, Layout* L) {
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (s->prec != MOE_NVFP4) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->d <= 0 || s->E <= 0 || s->I <= 0 || s->top_k <= 0 || s->first_local_expert < 0 ||
+      s->num_local_experts < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!make_layout(*s, L)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
 size_t moe_weights_size(const moe_shape* s) {
   Layout L;
+  if (s && s->prec == MOE_NVFP4) return check_shape_nv(s, &L) == MOE_OK ? L.wq_bytes : 0;
   if (check_shape_mx(s, &L) != MOE_OK) return 0;
   return L.wq_bytes;
 }
 
+// NVFP4 weights: amax of each tensor (the local experts' W_gate, W_up, W_down), their global
+// scales, then the gate/up B operand (K = d, 64-row gate / up blocks) and W_down^T (K = I).
+static moe_status prepare_weights_nv(const moe_shape* s, const void* W_gate, const void* W_up, const void* W_down,
+                                     void* wq, size_t wq_bytes, cudaStream_t st) {
+  Layout L;
+  const moe_status cs = check_shape_nv(s, &L);
+  if (cs != MOE_OK) return cs;
+  if (!W_gate || !W_up || !W_down || !wq) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_down) || !aligned16(wq)) return MOE_ERR_INVALID_ARG;
+  if (wq_bytes < L.wq_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  auto* w = static_cast<uint8_t*>(wq);
+  float* gs = reinterpret_cast<float*>(w + L.wnvgs);
+  unsigned* amx = reinterpret_cast<unsigned*>(w + L.wnvgs + 64);
+  const auto* g = static_cast<const __nv_bfloat16*>(W_gate);
+  const auto* u = static_cast<const __nv_bfloat16*>(W_up);
+  const auto* dn = static_cast<const __nv_bfloat16*>(W_down);
+  const int64_t n = static_cast<int64_t>(L.El) * L.d * L.I;
+  MOE_TRY(cudaMemsetAsync(amx, 0, 3 * sizeof(unsigned), st));
+  MOE_TRY(timed(K_QUANT_WEIGHTS, st, [&] {
+    cudaError_t e = launch_nv_amax(g, n, amx, st);
+    if (e == cudaSuccess) e = launch_nv_amax(u, n, amx + 1, st);
+    if (e == cudaSuccess) e = launch_nv_amax(dn, n, amx + 2, st);
+    if (e == cudaSuccess) e = launch_nv_scale(amx, gs, 3, st);
+    return e;
+  }));
+  MOE_TRY(timed(K_QUANT_WEIGHTS, st, [&] {
+    return launch_nv_quant_weight(true, g, u, L.El, L.d, L.I, gs, w + L.wgu1, w + L.wgu1s, st);
+  }));
+  MOE_TRY(timed(K_QUANT_WEIGHTS, st, [&] {
+    return launch_nv_quant_weight(false, dn, nullptr, L.El, L.I, L.d, gs + 2, w + L.wd2, w + L.wd2s, st);
+  }));
+  return MOE_OK;
+}
+
 moe_status moe_prepare_weights(const moe_shape* s, const void* W_gate, const void* W_up, const void* W_down, void* wq,
                                size_t wq_bytes, void* stream) {
+  if (s && s->prec == MOE_NVFP4)
+    return prepare_weights_nv(s, W_gate, W_up, W_down, wq, wq_bytes, static_cast<cudaStream_t>(stream));
   Layout L;
   const moe_status cs = check_shape_mx(s, &L);
   if (cs != MOE_OK) return cs;
@@ -1445,6 +1504,92 @@ moe_status moe_fwd_mx(const moe_shape* s, const void* X, const void* W_r, const 
     MOE_TRY(timed(K_GEMM_DOWN, st, [&] { return launch_gemm_mx(MX_DOWN, p, grid, st); }));
   }
   MOE_TRY(timed(K_COMBINE, st, [&] { return launch_combine(L, c, c.obuf, static_cast<__nv_bfloat16*>(Y), st); }));
+  return MOE_OK;
+}
+
+// NVFP4 forward: routing as in moe_fwd; X's global scale from its amax; the dispatch quantises
+// X along d; the gate/up GEMM writes H in fp32 and its amax; H's global scale; H quantised along
+// I; the down GEMM (combine weight in its epilogue); the combine.
+moe_status moe_fwd_nvfp4(const moe_shape* s, const void* X, const void* W_r, const float* bias, const void* wq,
+                         size_t wq_bytes, void* Y, void* ctx, size_t ctx_bytes, void* ws, size_t ws_bytes,
+                         void* stream) {
+  Layout L;
+  const moe_status cs = check_shape_nv(s, &L);
+  if (cs != MOE_OK) return cs;
+  const bool tok = s->T > 0;
+  if ((tok && (!X || !Y)) || !W_r || !wq || !ctx || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W_r) || !aligned16(wq) || !aligned16(Y) || !aligned16(ctx) || !aligned16(ws) ||
+      (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+    return MOE_ERR_INVALID_ARG;
+  if (ctx_bytes < L.ctx_bytes || ws_bytes < L.ws_bytes || wq_bytes < L.wq_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ctx c = make_ctx(L, ctx, ws);
+  MOE_TRY(cudaMemsetAsync(c.hdr, 0, HDR_WORDS * 4, st));
+  if (L.T == 0) return MOE_OK;
+  MOE_TRY(cudaMemsetAsync(c.nvsc, 0, 4 * sizeof(unsigned), st));
+  {
+    const moe_status r = route_tokens(L, c, X, W_r, bias, 0, st);
+    if (r != MOE_OK) return r;
+  }
+  unsigned* amx = c.nvsc;                               // [amax X, amax H]
+  float* gsv = reinterpret_cast<float*>(c.nvsc + 2);    // [gs X, gs H]
+  const auto* w = static_cast<const uint8_t*>(wq);
+  const float* gsw = reinterpret_cast<const float*>(w + L.wnvgs);  // [gate, up, down]
+  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
+  MOE_TRY(timed(K_NV_SCALE, st, [&] {
+    const cudaError_t e = launch_nv_amax(Xb, L.T * static_cast<int64_t>(L.d), amx, st);
+    return e != cudaSuccess ? e : launch_nv_scale(amx, gsv, 1, st);
+  }));
+  MOE_TRY(timed(K_DISPATCH, st, [&] { return launch_nv_gather_x(L, c, Xb, gsv, c.xq, c.xqs, st); }));
+  const int grid = num_sms();
+  int* status = c.hdr + HDR_STATUS;
+  const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
+  {
+    MxParams p = mx_params(L, c, status);
+    MOE_TMAP(tmap_fp8(&p.ta0, c.xq, L.d / 2, RP, 128));
+    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wgu1, L.d / 2, El * 2 * L.I, mx_bn(NV_GATEUP)));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.sfa0 = p.sfa1 = c.xqs;
+    p.sfb0 = p.sfb1 = w + L.wgu1s;
+    p.gsa = gsv;
+    p.gsb = gsw;
+    p.hout = c.nvh;
+    p.amax = amx + 1;
+    MOE_TRY(timed(K_NV_GATEUP, st, [&] { return launch_gemm_mx(NV_GATEUP, p, grid, st); }));
+  }
+  MOE_TRY(timed(K_NV_QUANT_H, st, [&] {
+    const cudaError_t e = launch_nv_scale(amx + 1, gsv + 1, 1, st);
+    return e != cudaSuccess ? e : launch_nv_quant_h(L, c, c.nvh, gsv + 1, c.hq, c.hqs, st);
+  }));
+  {
+    MxParams p = mx_params(L, c, status);
+    MOE_TMAP(tmap_fp8(&p.ta0, c.hq, L.I / 2, RP, 128));
+    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wd2, L.I / 2, El * L.d, mx_bn(NV_DOWN)));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.sfa0 = p.sfa1 = c.hqs;
+    p.sfb0 = p.sfb1 = w + L.wd2s;
+    p.gsa = gsv + 1;
+    p.gsb = gsw + 2;
+    p.out0 = c.obuf;
+    MOE_TRY(timed(K_NV_DOWN, st, [&] { return launch_gemm_mx(NV_DOWN, p, grid, st); }));
+  }
+  MOE_TRY(timed(K_COMBINE, st, [&] { return launch_combine(L, c, c.obuf, static_cast<__nv_bfloat16*>(Y), st); }));
+  return MOE_OK;
+}
+
+// Byte offsets of the NVFP4 forward's buffers, for tests: out[0..1] X codes and scales (ctx),
+// out[2..4] H codes, scales, fp32 H (workspace), out[5] the workspace's scale words, out[6..9]
+// gate/up codes and scales, W_down codes and scales, out[10] the weights' global scales
+// (prepared weights).
+moe_status moe_debug_nv_offsets(const moe_shape* s, int64_t* out) {
+  Layout L;
+  const moe_status cs = check_shape_nv(s, &L);
+  if (cs != MOE_OK) return cs;
+  if (!out) return MOE_ERR_INVALID_ARG;
+  const size_t v[11] = {L.xq, L.xqs, L.hq, L.hqs, L.nvh, L.nvsc, L.wgu1, L.wgu1s, L.wd2, L.wd2s, L.wnvgs};
+  for (int i = 0; i < 11; ++i) out[i] = static_cast<int64_t>(v[i]);
   return MOE_OK;
 }
 

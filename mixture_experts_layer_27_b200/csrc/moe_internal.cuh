@@ -77,6 +77,11 @@ struct Layout {
   bool mxw;  // MXFP8 mode with the weight-gradient GEMMs on MXFP8 as well
   bool w32;  // expert weight gradients written as fp32
   bool rslice;  // an expert slice (El < E): the router weight gradient runs over the listed tokens
+  bool nv;      // NVFP4 forward (moe_fwd_nvfp4): xq / xqs and hq / hqs hold E2M1 codes (two per byte)
+                // and E4M3 scale chunks (nv_sf_index), nvh the gate/up GEMM's fp32 H [RP, I], nvsc four
+                // words: amax(X), amax(H) (fp32 bits), then their global scales; the prepared weights
+                // are the two forward layouts and three global scales (wnvgs: gate, up, down)
+  size_t nvh, nvsc, wnvgs;
   // prepared MXFP8 weights (moe_prepare_weights): fp8 codes and scale chunks
   size_t wgu1, wgu1s, wd2, wd2s, wd3, wd3s, wg4, wg4s, wu4, wu4s, wq_bytes;
 };
@@ -198,6 +203,8 @@ enum MxKind {
   MX_DGRAD_GATEUP = 3,  // dX_perm = dAq . Wg_q^T + dBq . Wu_q^T
   MX_WGRAD_GATEUP = 4,  // dW_gate = Xq^T dAq, dW_up = Xq^T dBq per expert, all quantised along its rows
   MX_WGRAD_DOWN = 5,    // dW_down = Hgq^T dYq per expert
+  NV_GATEUP = 6,        // NVFP4 (kind::mxf4nvf4): H = silu(A) B from Xq . [Wg|Wu]q, fp32 H and its amax out
+  NV_DOWN = 7,          // NVFP4: O' = g * (Hq . Wd_q)
 };
 struct MxParams {
   CUtensorMap ta0, ta1, tb0, tb1;  // fp8 K-major operands, box {128 bytes of K, 128 rows (A) / mx_bn rows (B)}
@@ -237,8 +244,15 @@ struct MxParams {
   // gate/up GEMM of a ring-streamed macrobatch: the A operand's codes and scale chunks sit at ring
   // row = padded row + *ring_shift (a multiple of 128); NULL: at the padded row
   const int* ring_shift;
+  // NVFP4 kinds: global scales of the A operand and of the B operand(s) (gate, up), and the gate/up
+  // GEMM's fp32 H with the running amax of |H| (fp32 bits, atomicMax)
+  const float* gsa;
+  const float* gsb;
+  float* hout;
+  unsigned* amax;
 };
 __host__ __device__ constexpr bool mx_is_wgrad(int kind) { return kind == MX_WGRAD_GATEUP || kind == MX_WGRAD_DOWN; }
+__host__ __device__ constexpr bool mx_is_nv(int kind) { return kind == NV_GATEUP || kind == NV_DOWN; }
 // Tile width per kind: 128 x 256 tiles (one accumulator, four stages) keep 32 KB of fp8 weights
 // per stage in flight; the dgrad of W_down, whose epilogue reads and writes the most, keeps
 // 128 x 128 tiles with two accumulators (six stages) so that its epilogue overlaps the MMAs.
@@ -254,7 +268,8 @@ __host__ __device__ constexpr int mx_epi_warps(int kind) { return mx_accs(kind) 
 __host__ __device__ constexpr int mx_threads(int kind) { return 64 + 32 * mx_epi_warps(kind); }
 constexpr size_t MX_A_BYTES = 128 * 128;
 __host__ __device__ constexpr size_t mx_stage_tx(int kind) {  // bytes one stage receives
-  return MX_A_BYTES + static_cast<size_t>(mx_bn(kind)) * 128 + 512 * (1 + mx_bn(kind) / 128);
+  // NVFP4: a 128-byte K slice is 256 values, four 64-deep scale chunks per 128 rows
+  return MX_A_BYTES + static_cast<size_t>(mx_bn(kind)) * 128 + 512 * (1 + mx_bn(kind) / 128) * (mx_is_nv(kind) ? 4 : 1);
 }
 __host__ __device__ constexpr size_t mx_stage_bytes(int kind) { return (mx_stage_tx(kind) + 1023) / 1024 * 1024; }
 // weight-gradient kinds: 8 KB per epilogue warp stages its two gradient boxes for the TMA stores;
@@ -293,6 +308,8 @@ struct Ctx {  // typed views of ctx + ws for one shape
   StreamTables tab;
   uint8_t *xq, *xqs, *hq, *hqs, *dyq, *dyqs, *daq, *daqs, *dbq, *dbqs;  // MXFP8 operands and scales
   uint8_t *xqt, *xqts, *dyqt, *dyqts, *daqt, *daqts, *dbqt, *dbqts, *hgqt, *hgqts;  // MXFP8 weight-gradient operands
+  float* nvh;       // NVFP4 forward: fp32 H [RP, I]
+  unsigned* nvsc;   // NVFP4 forward: amax(X), amax(H) (fp32 bits), gs_X, gs_H (fp32)
 };
 Ctx make_ctx(const Layout& L, void* ctx, void* ws);
 
@@ -341,6 +358,19 @@ cudaError_t launch_gather_quant2(const Layout& L, const Ctx& c, const __nv_bfloa
 cudaError_t launch_gather_quant2_range(const Layout& L, const Ctx& c, const __nv_bfloat16* src, const int* lo,
                                        const int* hi, const int* dshift, uint8_t* qd, uint8_t* qds, uint8_t* qr,
                                        uint8_t* qrs, cudaStream_t st);
+// NVFP4 forward (nvfp4.cu): amax of |x| over n bf16 values (n a multiple of 8) into *amax (fp32 bits,
+// atomicMax: the caller zeroes it); global scales gs[i] = 2688 / amax[i] (1 for 0) for i < n;
+// the dispatch of X quantised along d; H (fp32 [RP, I]) quantised along I; weights quantised
+// along K into the forward layouts (paired: the gate/up B operand, 64-row gate / up blocks;
+// otherwise W [El][K][N] to rows el * N + n), gs the device scale(s) of src0 (and src1)
+cudaError_t launch_nv_amax(const __nv_bfloat16* x, int64_t n, unsigned* amax, cudaStream_t st);
+cudaError_t launch_nv_scale(const unsigned* amax, float* gs, int n, cudaStream_t st);
+cudaError_t launch_nv_gather_x(const Layout& L, const Ctx& c, const __nv_bfloat16* X, const float* gs, uint8_t* q,
+                               uint8_t* qs, cudaStream_t st);
+cudaError_t launch_nv_quant_h(const Layout& L, const Ctx& c, const float* h, const float* gs, uint8_t* q, uint8_t* qs,
+                              cudaStream_t st);
+cudaError_t launch_nv_quant_weight(bool paired, const __nv_bfloat16* src0, const __nv_bfloat16* src1, int El, int K,
+                                   int N, const float* gs, uint8_t* q, uint8_t* qs, cudaStream_t st);
 cudaError_t launch_transpose_wr(const Layout& L, const __nv_bfloat16* W_r, __nv_bfloat16* W_rT, cudaStream_t st);
 cudaError_t launch_rev_dispatch(const Layout& L, const Ctx& c, __nv_bfloat16* dX, cudaStream_t st);
 cudaError_t launch_export_routing(const Layout& L, const Ctx& c, int32_t* counts, int32_t* offsets,

@@ -378,6 +378,77 @@ __host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, uint32_t sf_id) 
   return (sf_id << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24) |
          (sf_id << 29);
 }
+// ---------------------------------------------------------------------------
+// NVFP4 (E2M1 payload, one E4M3 scale per 16 values along K, one fp32 scale per tensor)
+// ---------------------------------------------------------------------------
+// Codes are packed two per byte, value 2i in the low nibble of byte i, K-major.  Scale bytes
+// use the 512-byte chunk of the MXFP8 operands with 64-value K slices: a chunk covers
+// (128 rows, 64 K), byte (r % 32) * 16 + ((r % 128) / 32) * 4 + (k % 64) / 16 of chunk
+// (r / 128) * (K / 64) + k / 64, so one chunk holds the four scales per row that one K = 64
+// MMA reads (tcgen05.cp.32x128b.warpx4 moves it into 4 TMEM columns).
+__device__ __forceinline__ size_t nv_sf_index(int r, int k, int K) {
+  return (static_cast<size_t>(r >> 7) * (K >> 6) + (k >> 6)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 +
+         ((k & 63) >> 4);
+}
+// Exact value of an E4M3 byte with the sign bit clear (bias 7; exponent field 0 = subnormal
+// m * 2^-9), built from its fields.
+__device__ __forceinline__ float e4m3_pos_value(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  if (e == 0) return static_cast<float>(m) * 0x1p-9f;
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));  // (1 + m/8) 2^(e - 7)
+}
+// NVFP4 quantisation of 16 values under the tensor's global scale gs: block scale
+// s = e4m3((amax / 6) * gs) (fp32 divide and multiply, round to nearest even, saturating at
+// 448), codes e2m1(v * (gs / s)) (fp32, round to nearest even, saturating at 6); a block whose
+// scale rounds to 0 gets zero codes.  Returns the scale byte; q holds the 16 codes.
+__device__ __forceinline__ uint8_t nv_quant16(const float (&v)[16], float gs, uint32_t (&q)[2]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const float s = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
+  uint16_t sb2;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(sb2) : "f"(0.0f), "f"(s));
+  const uint32_t sb = sb2 & 0xFFu;
+  const float sdec = e4m3_pos_value(sb);
+  if (sdec == 0.f) {
+    q[0] = q[1] = 0u;
+    return static_cast<uint8_t>(sb);
+  }
+  const float inv = __fdiv_rn(gs, sdec);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t w;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(w)
+        : "f"(__fmul_rn(v[8 * h + 0], inv)), "f"(__fmul_rn(v[8 * h + 1], inv)), "f"(__fmul_rn(v[8 * h + 2], inv)),
+          "f"(__fmul_rn(v[8 * h + 3], inv)), "f"(__fmul_rn(v[8 * h + 4], inv)), "f"(__fmul_rn(v[8 * h + 5], inv)),
+          "f"(__fmul_rn(v[8 * h + 6], inv)), "f"(__fmul_rn(v[8 * h + 7], inv)));
+    q[h] = w;
+  }
+  return static_cast<uint8_t>(sb);
+}
+__device__ __forceinline__ void umma_nvf4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+// Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (format 1 in this kind), UE4M3 scales
+// (bit 23 clear), K = 64 dense (bit 31 clear), both K-major, scale ids 0 (the four scales of a
+// row fill its 32-bit TMEM word).
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // 1-D bulk copy global -> shared, completion on an mbarrier (16-byte aligned, size multiple of 16)
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(

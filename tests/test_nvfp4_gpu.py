@@ -1,0 +1,169 @@
+"""NVFP4 layer forward on the GPU, against the NVFP4 oracle (oracle/nvfp4.py).
+
+* global scales: the three weight scales and X's equal the oracle's bit for bit (both
+  compute 2688 / amax in fp32 on the same bf16 values);
+* prepared weights and the dispatched X: E2M1 codes and E4M3 scale bytes bit-exact against
+  the oracle's quantiser, in every prepared layout and every padded row (pad rows zero);
+* H: the device's H codes equal the oracle's quantiser applied to the device's own fp32 H
+  under the device's H scale, which equals the oracle's scale of that H;
+* Y within 2e-2 (max |gpu - ref| / max |ref|) of forward_nv: both sides take the same
+  quantisation decisions except where the fp32 accumulation order moves an H value across
+  a rounding boundary, so the bf16 tolerance holds; against the exact fp64 layer the error
+  is the format's own (reported, bounded loosely);
+* two runs are bit-identical; an expert slice, a hot expert spanning tiles, an empty
+  expert and T = 0 run.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import oracle.nvfp4 as N
+from mixture_experts_layer_27_b200 import binding as B
+
+from _util import TOL_BF16, make_case, relerr, to64
+
+pytestmark = pytest.mark.gpu
+
+
+def _gate_up_rows(Wg_codes, Wu_codes):
+    """Rows of the prepared gate/up operand for one expert: blocks of 64 gate columns, then the
+    same 64 up columns (each column one row, K = d)."""
+    I = Wg_codes.shape[1]
+    rows = []
+    for j in range(I // 64):
+        rows.append(Wg_codes[:, j * 64:(j + 1) * 64].T)
+        rows.append(Wu_codes[:, j * 64:(j + 1) * 64].T)
+    return np.concatenate(rows, axis=0)
+
+
+def test_nvfp4_prepared_weights_only():
+    # the weight quantiser alone (no forward), so a failure here is the quantiser's
+    T, d, E, k, I = 64, 256, 4, 2, 512
+    w, x = make_case(T, d, E, k, I, seed=41)
+    lay = B.MoELayerNVFP4(T, d, E, I, k)
+    lay.prepare(x["W_gate"], x["W_up"], x["W_down"])
+    torch.cuda.synchronize()
+    Wg64, Wu64, Wd64 = to64(x["W_gate"]), to64(x["W_up"]), to64(x["W_down"])
+    gsw = N.nv_weight_scales(Wg64, Wu64, Wd64)
+    assert [np.float32(v) for v in lay.scales()[1]] == list(gsw)
+    reg = lay.weight_regions()
+    cg, sg = zip(*[N.nv_quantize(Wg64[e], gsw[0], axis=0) for e in range(E)])
+    cu, su = zip(*[N.nv_quantize(Wu64[e], gsw[1], axis=0) for e in range(E)])
+    cd, sd = zip(*[N.nv_quantize(Wd64[e], gsw[2], axis=0) for e in range(E)])
+    assert np.array_equal(reg["Wgu"][0], np.concatenate([_gate_up_rows(cg[e], cu[e]) for e in range(E)]))
+    assert np.array_equal(reg["Wgu"][1], np.concatenate([_gate_up_rows(sg[e], su[e]) for e in range(E)]))
+    assert np.array_equal(reg["Wd2"][0], np.concatenate([c.T for c in cd]))
+    assert np.array_equal(reg["Wd2"][1], np.concatenate([c.T for c in sd]))
+
+
+def _run(T, d, E, k, I, seed=0, bias=None, first=0, num=0):
+    w, x = make_case(T, d, E, k, I, seed=seed, bias=bias)
+    El = num or (E - first)
+    lay = B.MoELayerNVFP4(T, d, E, I, k, first_local_expert=first, num_local_experts=num)
+    Wg = x["W_gate"][first:first + El].contiguous()
+    Wu = x["W_up"][first:first + El].contiguous()
+    Wd = x["W_down"][first:first + El].contiguous()
+    lay.prepare(Wg, Wu, Wd)
+    Y = lay.forward(x["X"], x["W_r"], x["bias"])
+    torch.cuda.synchronize()
+    assert lay.error() == B.MOE_OK
+    return lay, x, Y, (Wg, Wu, Wd)
+
+
+def _check(T, d, E, k, I, seed=0, bias=None, first=0, num=0):
+    lay, x, Y, (Wg, Wu, Wd) = _run(T, d, E, k, I, seed, bias, first, num)
+    El = lay.El
+    f = {n: (None if x[n] is None else to64(x[n])) for n in ("X", "W_r", "bias")}
+    Wg64, Wu64, Wd64 = to64(Wg), to64(Wu), to64(Wd)
+
+    # global scales, bit for bit
+    (gsx, gsh), gsw = lay.scales()
+    want_w = N.nv_weight_scales(Wg64, Wu64, Wd64)
+    assert [np.float32(v) for v in gsw] == list(want_w)
+    assert np.float32(gsx) == N.nv_global_scale(f["X"])
+
+    # prepared weights, bit for bit
+    reg = lay.weight_regions()
+    gu_c, gu_s, d2_c, d2_s = [], [], [], []
+    for e in range(El):
+        cg, sg = N.nv_quantize(Wg64[e], want_w[0], axis=0)  # [d, I], [d/16, I]
+        cu, su = N.nv_quantize(Wu64[e], want_w[1], axis=0)
+        cd, sd = N.nv_quantize(Wd64[e], want_w[2], axis=0)  # [I, d], [I/16, d]
+        gu_c.append(_gate_up_rows(cg, cu))
+        gu_s.append(_gate_up_rows(sg, su))
+        d2_c.append(cd.T)
+        d2_s.append(sd.T)
+    assert np.array_equal(reg["Wgu"][0], np.concatenate(gu_c)), "Wgu codes"
+    assert np.array_equal(reg["Wgu"][1], np.concatenate(gu_s)), "Wgu scales"
+    assert np.array_equal(reg["Wd2"][0], np.concatenate(d2_c)), "Wd2 codes"
+    assert np.array_equal(reg["Wd2"][1], np.concatenate(d2_s)), "Wd2 scales"
+
+    # dispatched X, bit for bit, row by row (pad rows up to the next multiple of 16: zero)
+    r = lay.routing()
+    counts = r["counts"].cpu().numpy()
+    offs = r["offsets"].cpu().numpy()
+    poff = r["padded_offsets"].cpu().numpy()
+    perm = r["perm"].cpu().numpy()
+    xc, xs = lay.x_operand()
+    cx, sx = N.nv_quantize(f["X"], gsx, axis=1)
+    live = []
+    for e in range(El):
+        toks = perm[offs[e]:offs[e + 1]]
+        rows = poff[e] + np.arange(counts[e])
+        assert np.array_equal(xc[rows], cx[toks]) and np.array_equal(xs[rows], sx[toks]), e
+        pad = poff[e] + np.arange(counts[e], (counts[e] + 15) // 16 * 16)
+        assert not xc[pad].any() and not xs[pad].any(), e
+        live.append(rows)
+    live = np.concatenate(live) if live else np.zeros(0, dtype=np.int64)
+
+    # H: the device's codes are the oracle's quantiser on the device's fp32 H and scale
+    if live.size:
+        H = lay.h_fp32().astype(np.float64)[live]
+        assert np.float32(gsh) == N.nv_global_scale(H)
+        hc, hs = lay.h_operand()
+        qc, qs = N.nv_quantize(H, gsh, axis=1)
+        assert np.array_equal(hc[live], qc) and np.array_equal(hs[live], qs)
+
+    # Y against the NVFP4 oracle
+    Yq, info = N.forward_nv(f["X"], f["W_r"], f["bias"], to64(x["W_gate"]), to64(x["W_up"]), to64(x["W_down"]),
+                            k, first_local=first, num_local=El, gs_w=want_w)
+    assert np.array_equal(r["ids"].cpu().numpy(), info["ids"])
+    err = relerr(to64(Y), Yq)
+    assert err <= TOL_BF16, err
+    Yo, _ = O.forward(f["X"], f["W_r"], f["bias"], to64(x["W_gate"]), to64(x["W_up"]), to64(x["W_down"]), k,
+                      first_local=first, num_local=El)
+    assert relerr(to64(Y), Yo) < 0.5
+    return lay, x, Y
+
+
+def test_nvfp4_tiny_config():
+    _check(128, 256, 8, 2, 512, seed=0)
+
+
+def test_nvfp4_hot_expert_multi_tile_and_empty_expert():
+    bias = np.zeros(4, dtype=np.float32)
+    bias[0] = 8.0
+    bias[3] = -40.0
+    _check(600, 512, 4, 2, 512, bias=bias, seed=42)
+
+
+def test_nvfp4_expert_slice_ragged_tokens():
+    _check(328, 768, 8, 3, 512, seed=7, first=2, num=4)
+
+
+def test_nvfp4_runs_are_bit_identical():
+    lay, x, Y = _check(256, 512, 8, 2, 768, seed=3)
+    Y2 = lay.forward(x["X"], x["W_r"], x["bias"])
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y2)
+
+
+def test_nvfp4_empty_batch():
+    lay = B.MoELayerNVFP4(0, 256, 4, 512, 2)
+    w, x = make_case(8, 256, 4, 2, 512, seed=1)
+    lay.prepare(x["W_gate"], x["W_up"], x["W_down"])
+    Y = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    B.check(B.moe_fwd_nvfp4(lay.shape, x["X"][:0], x["W_r"], x["bias"], lay.wq, Y, lay.ctx, lay.ws), "empty")
+    torch.cuda.synchronize()
+    assert lay.error() == B.MOE_OK
