@@ -453,6 +453,19 @@ def run_reference(args, w: IN.Workload, world: int, rank: int):
     if rank != 0:
         return
     x = cpu_inputs(w, args.mx_wgrad)
+    if w.nvfp4:  # the NVFP4 oracle forward (its own start-up call inside)
+        r = nv_oracle_rate(w, x, args.steps)
+        value = r["value"]
+        print(json.dumps({
+            "metric": METRIC_NV, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": statistics.median(r["seconds"]) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": nv_config(w),
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": r["sample"]},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+            flush=True)
+        return
     for _ in range(args.warmup):
         oracle_sample(w, x)
     r = oracle_rate(w, x, args.steps)
@@ -774,6 +787,238 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------
+# NVFP4 layer forward (moe_fwd_nvfp4): a step is one forward over the batch
+# ----------------------------------------------------------------------------
+METRIC_NV = "MoE layer forward tokens/s and TFLOP/s, NVFP4 (% of B200 FP4 tensor peak)"
+NV_GEMMS = ("gemm_gateup_swiglu_nvfp4", "gemm_down_combw_nvfp4")
+
+
+def nv_algorithmic(w: IN.Workload) -> tuple:
+    """(bytes, flops) per launch of the NVFP4 forward's kernels: E2M1 codes at 1/2 byte and one
+    E4M3 scale per 16 values (9/16 byte per value), H in fp32 between the two passes."""
+    T, d, E, I, k, El = w.tokens, w.d, w.E, w.I, w.k, w.El
+    rows = local_rows(w)
+    Tg = min(T, rows)
+    q = 9 / 16
+    W = El * d * I * q  # one weight tensor in NVFP4
+    by = {"nvfp4_amax_scale": T * d * 2, "dispatch": Tg * d * 2 + rows * d * q,
+          "gemm_gateup_swiglu_nvfp4": 2 * W + rows * d * q + rows * I * 4,
+          "nvfp4_quantize_h": rows * I * 4 + rows * I * q,
+          "gemm_down_combw_nvfp4": W + rows * I * q + rows * d * 2,
+          "combine": rows * d * 2 + T * d * 2,
+          "router_logits": T * d * 2 + d * E * 2 + T * E * 4}
+    fl = {"gemm_gateup_swiglu_nvfp4": 4 * d * I * rows, "gemm_down_combw_nvfp4": 2 * d * I * rows,
+          "router_logits": 2 * T * d * E}
+    return by, fl
+
+
+def nv_config(w: IN.Workload) -> dict:
+    cfg = dict(workload_config(w), precision="nvfp4")
+    cfg["pass"] = "forward"
+    cfg["workload"] = cfg["workload"].replace(" bf16,", " nvfp4 forward,")
+    return cfg
+
+
+def nv_oracle_rate(w: IN.Workload, x_cpu: dict, steps: int) -> dict:
+    """The NVFP4 oracle forward on the sampled expert window (all tokens routed), timed."""
+    import numpy as np
+    import oracle.nvfp4 as N
+
+    def f64(t):
+        return t.float().numpy().astype(np.float64)
+
+    e0, m = x_cpu["window"]
+    X, Wr = f64(x_cpu["X"]), f64(x_cpu["W_r"])
+    b = None if x_cpu["bias"] is None else f64(x_cpu["bias"])
+    Wg, Wu, Wd = (f64(x_cpu[n]) for n in ("W_gate", "W_up", "W_down"))
+    first = w.first_local + e0
+    gs_w = N.nv_weight_scales(Wg, Wu, Wd)  # over the window's experts
+    # weights rounded once, outside the timed step (the GPU path prepares them once per optimiser step)
+    lay = {first + e: N.nv_weight_layouts(Wg[e], Wu[e], Wd[e], gs_w) for e in range(m)}
+
+    def one():
+        t0 = time.perf_counter()
+        _, info = N.forward_nv(X, Wr, b, lambda e: Wg[e - first], lambda e: Wu[e - first], lambda e: Wd[e - first],
+                               w.k, first_local=first, num_local=m, gs_w=gs_w, rounded=lay.__getitem__)
+        return time.perf_counter() - t0, int(info["sched"]["offsets"][-1])
+
+    one()  # imports, BLAS start-up
+    ts, asg = zip(*[one() for _ in range(steps)])
+    med = statistics.median(ts)
+    return {"value": asg[0] / w.k / med, "seconds": list(ts),
+            "sample": (f"fp64 numpy NVFP4 oracle forward, measured: each step routes all {w.tokens} tokens and "
+                       f"runs the forward of local experts {e0}..{e0 + m - 1} ({asg[0]} assignments; weights "
+                       f"rounded once outside the step, global scales over the window); rate = assignments / "
+                       f"top_k / the median of {steps} steps ({med:.2f} s)")}
+
+
+def run_nvfp4(args, w: IN.Workload, world: int, rank: int, local: int):
+    from mixture_experts_layer_27_b200 import binding as B
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_kind = load_peaks()
+    x = IN.make_inputs(w, device=dev)
+    layer = B.MoELayerNVFP4(w.T, w.d, w.E, w.I, w.k, w.first_local, w.num_local, device=dev)
+    El = w.El
+    Wg, Wu, Wd = (x[n][w.first_local:w.first_local + El].contiguous() for n in ("W_gate", "W_up", "W_down"))
+    NT = w.tokens
+    Y = torch.empty(NT, w.d, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    fp8_peak = measure_mxfp8_peak(dev)
+    layer.prepare(Wg, Wu, Wd)
+    pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pa.record(stream)
+    layer.prepare(Wg, Wu, Wd)  # once per optimiser step, outside the layer step
+    pb.record(stream)
+    torch.cuda.synchronize()
+    prep_ms = pa.elapsed_time(pb)
+
+    def step(X, Yout):
+        layer.forward(X, x["W_r"], x["bias"], Y=Yout)
+
+    for _ in range(args.warmup):
+        step(x["X"], Y)
+    torch.cuda.synchronize()
+    if layer.error() != B.MOE_OK:
+        raise RuntimeError("device error during warm-up")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if needs_flush(w) else None
+
+    B.moe_profile_read()
+    B.moe_profile_enable(True)
+    launches0 = B.moe_kernel_launches()
+    torch.cuda.synchronize()
+    for _ in range(args.steps):
+        if flush is not None:
+            flush.fill_(1)
+        step(x["X"], Y)
+    torch.cuda.synchronize()
+    launches_per_step = (B.moe_kernel_launches() - launches0) // args.steps
+    B.moe_profile_enable(False)
+    prof = B.moe_profile_read()
+
+    graph, launch_mode = None, "cuda_graph"
+    if not args.no_graph:
+        try:
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                step(x["X"], Y)
+            stream.wait_stream(side)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step(x["X"], Y)
+            torch.cuda.synchronize()
+        except Exception as ex:
+            graph, launch_mode = None, f"direct (graph capture failed: {type(ex).__name__})"
+    else:
+        launch_mode = "direct"
+
+    def run_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            step(x["X"], Y)
+
+    for _ in range(2):
+        run_step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in evs:
+        if flush is not None:
+            flush.fill_(1)
+        a.record(stream)
+        run_step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    t_local = sum(a.elapsed_time(b) for a, b in evs) / 1e3
+    barrier(world)
+    clk = clocks.stop()
+    if layer.error() != B.MOE_OK:
+        raise RuntimeError("device error in the timed region")
+    t = max_over_ranks(t_local, world)
+
+    # end to end: X in from pinned host memory, Y out, every step (in line on the compute stream)
+    hX = torch.empty(NT, w.d, dtype=torch.bfloat16, pin_memory=True)
+    hY = torch.empty_like(hX, pin_memory=True)
+    hX.copy_(x["X"].cpu())
+    Xd = torch.empty_like(x["X"])
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e2.record(stream)
+    for _ in range(args.steps):
+        Xd.copy_(hX, non_blocking=True)
+        step(Xd, Y)
+        hY.copy_(Y, non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = max_over_ranks(e2.elapsed_time(e3) / 1e3, world)
+    if rank != 0:
+        return
+
+    by, fl = nv_algorithmic(w)
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    fp8 = fp8_peak.get("sustained_tflops")
+    fp4 = 2.0 * fp8 if fp8 else 2.0 * 2.0 * float(peaks.get("bf16_tflops_sustained",
+                                                            FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    fp4_src = ("2 x the sustained MXFP8 cuBLAS GEMM measured in this run (the nominal dense fp4 : fp8 ratio, "
+               "9 : 4.5 PFLOP/s)" if fp8 else "4 x the sustained bf16 peak (nominal fp4 : bf16 ratio)")
+    kern = {}
+    for name, (ms, n) in sorted(prof.items(), key=lambda kv: -kv[1][0]):
+        sec = ms / args.steps / 1e3
+        e = {"ms_per_step": ms / args.steps, "launches_per_step": n / args.steps, "share": ms / (t * 1e3)}
+        if name in by:
+            e["algorithmic_GB"] = by[name] / 1e9
+            e["achieved_GBs"] = by[name] / sec / 1e9
+        if name in fl:
+            e["achieved_TFLOPs"] = fl[name] / sec / 1e12
+            tpeak = fp4 if name in NV_GEMMS else float(peaks.get("bf16_tflops_sustained",
+                                                                 FALLBACK_PEAKS["bf16_tflops_sustained"]))
+            e["bound"] = "tensor" if fl[name] / (tpeak * 1e12) > by.get(name, 0) / (hbm * 1e9) else "hbm"
+        else:
+            e["bound"] = "hbm"
+        kern[name] = e
+    top = max(kern.items(), key=lambda kv: kv[1]["share"])[0]
+    if kern[top]["bound"] == "tensor" and top in NV_GEMMS:
+        ach = kern[top]["achieved_TFLOPs"]
+        roof = {"kernel": top, "bound": "tensor", "achieved": ach, "peak": fp4, "unit": "TFLOP/s",
+                "frac": ach / fp4, "traffic": ncu_traffic(top, w.name), "peak_source": fp4_src}
+    else:
+        ach = kern[top].get("achieved_GBs")
+        roof = {"kernel": top, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+                "frac": (ach / hbm) if ach else None, "traffic": ncu_traffic(top, w.name),
+                "peak_source": f"{peak_kind} HBM copy bandwidth" if peak_kind == "measured"
+                else "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"}
+    tflops = w.forward_flops() * args.steps * world / t / 1e12
+    line = {
+        "metric": METRIC_NV, "value": job_throughput(NT * args.steps, t, world), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 + e4m3 per 16 + fp32 per tensor)", "data": "synthetic (seeded, random-init weights)",
+        "config": nv_config(w),
+        "tflops": tflops, "pct_of_fp4_peak": 100.0 * tflops / world / fp4, "fp4_peak_tflops": fp4,
+        "peak_note": "forward model FLOPs 6 d I per assignment + 2 T d E; fp4 peak = " + fp4_src,
+        "roofline": roof,
+        "e2e": {"value": job_throughput(NT * args.steps, t_e2e, world), "unit": "tokens/s",
+                "h2d_bytes_per_step": NT * w.d * 2, "d2h_bytes_per_step": NT * w.d * 2,
+                "note": "X copied in from pinned host memory and Y copied back every step, in line on the "
+                        "compute stream; prepared weights stay in HBM"},
+        "gpu_launches": int(launches_per_step * args.steps), "launch": launch_mode, "clocks": clk,
+        "prepare_weights_ms": prep_ms, "mxfp8_peak": fp8_peak, "kernels": kern,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        r = nv_oracle_rate(w, cpu_inputs(w), CPU_BASELINE_STEPS)
+        line["cpu_baseline"] = {"value": r["value"], "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": r["sample"]}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -814,7 +1059,7 @@ def main():
         return
     world, rank, local = dist_setup(args.gpus)
     try:
-        run_moe(args, w, world, rank, local)
+        (run_nvfp4 if w.nvfp4 else run_moe)(args, w, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

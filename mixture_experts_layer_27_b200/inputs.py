@@ -47,6 +47,7 @@ class Workload:
     stream_M: int = 0           # > 0: M minibatches of T tokens through a ring of ring_bytes
     ring_bytes: int = 0
     local_tokens: int = 0       # streamed slice: assignments each local expert receives over the stream
+    nvfp4: bool = False         # NVFP4 layer forward (no NVFP4 backward exists)
 
     @property
     def El(self) -> int:
@@ -61,6 +62,11 @@ class Workload:
         """fwd+bwd model FLOPs: 18 d I per local assignment (6 fwd, 12 bwd) + 6 T d E router."""
         assign = self.El * self.local_tokens if self.local_tokens else self.tokens * self.k
         return 18.0 * self.d * self.I * assign + 6.0 * self.tokens * self.d * self.E
+
+    def forward_flops(self) -> float:
+        """forward model FLOPs: 6 d I per local assignment + 2 T d E router."""
+        assign = self.El * self.local_tokens if self.local_tokens else self.tokens * self.k
+        return 6.0 * self.d * self.I * assign + 2.0 * self.tokens * self.d * self.E
 
 
 WORKLOADS = {
@@ -101,6 +107,16 @@ for _n in (512, 2368, 4096, 8192):
 # epmx_n2368's expert work (6 local experts x 2368 rows, MXFP8) over 8192 tokens and 96 experts: the
 # same dispatched rows and GEMM tiles with a padded-row capacity (and workspace) a quarter of the
 # size, for profiler captures (a few GB on the device)
+# NVFP4 layer forward: the dsv3 and kimi configurations, the EP64 slice as one batch (where the
+# grouped GEMMs are tensor-bound), and two few-GB cases for profiler captures
+WORKLOADS["dsv3_nv"] = Workload("dsv3_nv", 2048, 7168, 256, 8, 2048, nvfp4=True)
+WORKLOADS["kimi_nv"] = Workload("kimi_nv", 4096, 7168, 384, 8, 2048, zipf=True, nvfp4=True)
+WORKLOADS["dsv3_nv_e16"] = Workload("dsv3_nv_e16", 128, 7168, 16, 8, 2048, nvfp4=True)
+for _n in (512, 2368, 4096, 8192):
+    WORKLOADS[f"epnv_n{_n}"] = Workload(f"epnv_n{_n}", 32768, 7168, 384, 8, 2048, first_local=0, num_local=6,
+                                        local_tokens=_n, nvfp4=True)
+WORKLOADS["epnv_t8192_n2368"] = Workload("epnv_t8192_n2368", 8192, 7168, 96, 8, 2048, first_local=0, num_local=6,
+                                         local_tokens=2368, nvfp4=True)
 WORKLOADS["epmx_t8192_n2368"] = Workload("epmx_t8192_n2368", 8192, 7168, 96, 8, 2048, mxfp8=True, first_local=0,
                                          num_local=6, local_tokens=2368)
 

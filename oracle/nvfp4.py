@@ -63,13 +63,13 @@ def e2m1_encode(x) -> np.ndarray:
     magnitudes above 6 saturate to 6.  The sign of a value that rounds to zero is kept."""
     x = _f64(x)
     a = np.minimum(np.abs(x), E2M1_MAX)
-    dist = np.abs(a[..., None] - E2M1_GRID)
-    dmin = dist.min(axis=-1, keepdims=True)
-    near = dist == dmin
-    # among the (at most two) nearest magnitudes, prefer the even code
-    even = near & ((np.arange(8) & 1) == 0)
-    pick = np.where(even.any(axis=-1), np.argmax(even, axis=-1), np.argmax(near, axis=-1))
-    return (pick | (np.signbit(x).astype(np.int64) << 3)).astype(np.uint8)
+    # the code of a magnitude is the number of midpoints between neighbours lying below it; a
+    # magnitude on a midpoint sits between codes c and c + 1 and takes the even one
+    mids = (E2M1_GRID[1:] + E2M1_GRID[:-1]) / 2
+    c = np.searchsorted(mids, a, side="left")
+    on_mid = (c < mids.size) & (a == mids[np.minimum(c, mids.size - 1)])
+    c = np.where(on_mid & (c % 2 == 1), c + 1, c)
+    return (c | (np.signbit(x).astype(np.int64) << 3)).astype(np.uint8)
 
 
 def nv_global_scale(v) -> np.float32:
@@ -135,13 +135,22 @@ def nv_weight_scales(W_gate, W_up, W_down, first_local: int = 0, num_local: int 
     return tuple(np.float32(min(g, np.finfo(np.float32).max)) for g in out)
 
 
+def nv_weight_layouts(Wg, Wu, Wd, gs_w) -> dict:
+    """One expert's weights rounded for the forward GEMMs that read them (fp64): gate and up
+    along d (K of the gate/up GEMM), down along I (K of the down GEMM)."""
+    return dict(gate=nv_round(_f64(Wg), gs_w[0], axis=0), up=nv_round(_f64(Wu), gs_w[1], axis=0),
+                down=nv_round(_f64(Wd), gs_w[2], axis=0))
+
+
 def forward_nv(X, W_r, bias, W_gate, W_up, W_down, top_k: int, first_local: int = 0,
-               num_local: int | None = None, gs_w=None):
+               num_local: int | None = None, gs_w=None, rounded=None):
     """NVFP4 layer forward: the routing of `forward`, then per local expert
     A = Xq Wgq, B = Xq Wuq (K = d), H = silu(A) B, O = Hq Wdq (K = I), Y = sum_j g O.
 
     gs_w: optional (gs_gate, gs_up, gs_down) computed once by the caller
     (nv_weight_scales); without it they are computed here.
+    rounded: optional callable e -> nv_weight_layouts of expert e under gs_w (the same values,
+    computed once by the caller); without it the weights are rounded here.
     Returns (Y, info) with the routing, the five global scales and, per local expert,
     (tokens, slots, H, A, B) or None."""
     X64 = _f64(X)
@@ -163,9 +172,10 @@ def forward_nv(X, W_r, bias, W_gate, W_up, W_down, top_k: int, first_local: int 
             Hs.append(None)
             continue
         e = el + first_local
+        Wq = rounded(e) if rounded is not None else None
         Xq = nv_round(X64[toks], gs_x, axis=1)  # K = d
-        A = Xq @ nv_round(_expert(W_gate, e), gs_g, axis=0)
-        B = Xq @ nv_round(_expert(W_up, e), gs_u, axis=0)
+        A = Xq @ (Wq["gate"] if Wq else nv_round(_expert(W_gate, e), gs_g, axis=0))
+        B = Xq @ (Wq["up"] if Wq else nv_round(_expert(W_up, e), gs_u, axis=0))
         Hs.append((toks, slots, silu(A) * B, A, B))
     live = [h[2] for h in Hs if h is not None]
     gs_h = nv_global_scale(np.concatenate(live, axis=0)) if live else np.float32(1.0)
@@ -174,7 +184,9 @@ def forward_nv(X, W_r, bias, W_gate, W_up, W_down, top_k: int, first_local: int 
         if h is None:
             continue
         toks, slots, H = h[:3]
-        O = nv_round(H, gs_h, axis=1) @ nv_round(_expert(W_down, el + first_local), gs_d, axis=0)  # K = I
+        Wdq = rounded(el + first_local)["down"] if rounded is not None else \
+            nv_round(_expert(W_down, el + first_local), gs_d, axis=0)
+        O = nv_round(H, gs_h, axis=1) @ Wdq  # K = I
         Y[toks] += g[toks, slots][:, None] * O
     info = dict(ids=ids, g=g, sched=sched, gs_x=gs_x, gs_h=gs_h, gs_w=(gs_g, gs_u, gs_d), experts=Hs)
     return Y, info

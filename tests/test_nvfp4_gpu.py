@@ -167,3 +167,32 @@ def test_nvfp4_empty_batch():
     B.check(B.moe_fwd_nvfp4(lay.shape, x["X"][:0], x["W_r"], x["bias"], lay.wq, Y, lay.ctx, lay.ws), "empty")
     torch.cuda.synchronize()
     assert lay.error() == B.MOE_OK
+
+
+def test_nvfp4_full_size_ep64_slice():
+    # The EP64 per-rank slice at full size, as the bench runs it (epnv_n2368: 32768 tokens routed
+    # top-8 over 384 experts, 6 local experts with 2368 rows each, one batch): every token's Y
+    # against the NVFP4 oracle's full forward, routing bit-exact, X codes bit-exact on every row.
+    from mixture_experts_layer_27_b200 import inputs as IN
+    w = IN.WORKLOADS["epnv_n2368"]
+    x = IN.make_inputs(w, device="cuda")
+    El = w.El
+    lay = B.MoELayerNVFP4(w.T, w.d, w.E, w.I, w.k, w.first_local, w.num_local)
+    Wg, Wu, Wd = (x[n][:El].contiguous() for n in ("W_gate", "W_up", "W_down"))
+    lay.prepare(Wg, Wu, Wd)
+    Y = lay.forward(x["X"], x["W_r"], x["bias"])
+    torch.cuda.synchronize()
+    assert lay.error() == B.MOE_OK
+    f = {n: to64(x[n]) for n in ("X", "W_r", "bias")}
+    W64 = [to64(t) for t in (Wg, Wu, Wd)]
+    gs_w = N.nv_weight_scales(*W64)
+    assert [np.float32(v) for v in lay.scales()[1]] == list(gs_w)
+    Yq, info = N.forward_nv(f["X"], f["W_r"], f["bias"], W64[0], W64[1], W64[2], w.k, first_local=0,
+                            num_local=El, gs_w=gs_w)
+    r = lay.routing()
+    assert np.array_equal(r["ids"].cpu().numpy(), info["ids"])
+    assert np.array_equal(r["counts"].cpu().numpy(), info["sched"]["counts"][:El])
+    # H's scale: the device's H (fp32 accumulation) and the oracle's (fp64) share their amax to ~1e-6
+    assert abs(float(lay.scales()[0][1]) / float(info["gs_h"]) - 1.0) < 1e-5
+    err = relerr(to64(Y), Yq)
+    assert err <= TOL_BF16, err
