@@ -557,6 +557,9 @@ class MoELayerNVFP4:
     def routing(self):
         return MoELayer.routing(self)
 
+    def logits(self):
+        return MoELayer.logits(self)
+
     def error(self, stream=None) -> int:
         return moe_get_error(self.ctx, stream)
 

@@ -172,7 +172,8 @@ def test_nvfp4_empty_batch():
 def test_nvfp4_full_size_ep64_slice():
     # The EP64 per-rank slice at full size, as the bench runs it (epnv_n2368: 32768 tokens routed
     # top-8 over 384 experts, 6 local experts with 2368 rows each, one batch): every token's Y
-    # against the NVFP4 oracle's full forward, routing bit-exact, X codes bit-exact on every row.
+    # (but the few near-tie tokens, whose fp64 routing differs) against the NVFP4 oracle's full
+    # forward, routing bit-exact on the GPU's logits, the global scales.
     from mixture_experts_layer_27_b200 import inputs as IN
     w = IN.WORKLOADS["epnv_n2368"]
     x = IN.make_inputs(w, device="cuda")
@@ -190,9 +191,18 @@ def test_nvfp4_full_size_ep64_slice():
     Yq, info = N.forward_nv(f["X"], f["W_r"], f["bias"], W64[0], W64[1], W64[2], w.k, first_local=0,
                             num_local=El, gs_w=gs_w)
     r = lay.routing()
-    assert np.array_equal(r["ids"].cpu().numpy(), info["ids"])
-    assert np.array_equal(r["counts"].cpu().numpy(), info["sched"]["counts"][:El])
+    gids = r["ids"].cpu().numpy()
+    # routing bit-exact on the GPU's fp32 logits; against the fp64 logits the ids may differ only
+    # at near-ties (fp32 vs fp64 logits of 7168-term dot products), and those tokens are left out
+    lg = to64(lay.logits())
+    assert np.array_equal(gids, O.topk_ids(lg, w.k))
+    lg64 = O.router_logits(f["X"], f["W_r"], f["bias"])
+    differ = np.nonzero(np.any(gids != info["ids"], axis=1))[0]
+    srt = -np.sort(-lg64[differ], axis=1)
+    assert np.all(srt[:, w.k - 1] - srt[:, w.k] < 1e-3), differ
+    keep = np.setdiff1d(np.arange(w.T), differ)
+    assert differ.size < 64
     # H's scale: the device's H (fp32 accumulation) and the oracle's (fp64) share their amax to ~1e-6
     assert abs(float(lay.scales()[0][1]) / float(info["gs_h"]) - 1.0) < 1e-5
-    err = relerr(to64(Y), Yq)
+    err = relerr(to64(Y)[keep], Yq[keep])
     assert err <= TOL_BF16, err
