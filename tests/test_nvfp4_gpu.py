@@ -197,7 +197,8 @@ def test_nvfp4_full_size_ep64_slice():
     lg = to64(lay.logits())
     assert np.array_equal(gids, O.topk_ids(lg, w.k))
     lg64 = O.router_logits(f["X"], f["W_r"], f["bias"])
-    differ = np.nonzero(np.any(gids != info["ids"], axis=1))[0]
+    # selection differences (the order inside a token's top k only orders the combine's sum)
+    differ = np.nonzero(np.any(np.sort(gids, 1) != np.sort(info["ids"], 1), axis=1))[0]
     srt = -np.sort(-lg64[differ], axis=1)
     assert np.all(srt[:, w.k - 1] - srt[:, w.k] < 1e-3), differ
     keep = np.setdiff1d(np.arange(w.T), differ)
