@@ -34,7 +34,9 @@ the design notes):
   1 / (gs_A gs_B);
 * H = silu(A) * B from the unrounded A, B (as in the MXFP8 oracle).
 
-Only the forward is defined in this mode.
+The backward (backward_nv) quantises the two dgrad GEMMs' operands the same way; the
+dgrad of gate/up contracts over K = 2I, so its operands [dA | dB] and [W_gate | W_up] are each
+one tensor with one global scale; the weight gradients take the unrounded operands.
 """
 
 from __future__ import annotations
@@ -190,3 +192,68 @@ def forward_nv(X, W_r, bias, W_gate, W_up, W_down, top_k: int, first_local: int 
         Y[toks] += g[toks, slots][:, None] * O
     info = dict(ids=ids, g=g, sched=sched, gs_x=gs_x, gs_h=gs_h, gs_w=(gs_g, gs_u, gs_d), experts=Hs)
     return Y, info
+
+
+def nv_weight_scales_bwd(W_gate, W_up, W_down, first_local: int = 0, num_local: int | None = None):
+    """Global scales of the backward's weight operands: [W_gate | W_up] along I as one tensor (the
+    dgrad of gate/up contracts over both halves into one sum), W_down as in the forward."""
+    g, u, d = nv_weight_scales(W_gate, W_up, W_down, first_local, num_local)
+    return np.float32(min(g, u)), d
+
+
+def backward_nv(info, X, W_r, W_gate, W_up, W_down, dY, gs_bwd=None):
+    """NVFP4 layer backward after forward_nv (its info): the dgrad GEMMs on NVFP4 operands,
+    the weight gradients from the unrounded operands (as the MXFP8 layer with bf16 weight
+    gradients does).
+
+    dgrad of W_down (K = d): dY rows along d under gs(dY [T, d]), W_down along d;
+    dgrad of gate/up (K = 2I): [dA | dB] rows along I under one scale over every assigned row's
+    dA and dB, [W_gate | W_up] along I under one scale (nv_weight_scales_bwd).
+    A and B are read as bf16 (the layer keeps them in bf16), H = silu(A) B recomputed from them.
+    gs_bwd: optional (gs_gate_up, gs_down) computed once by the caller."""
+    from .moe_oracle import bf16_round, silu_grad
+    X64, dY64 = _f64(X), _f64(dY)
+    ids, g, sched = info["ids"], info["g"], info["sched"]
+    T, d = X64.shape
+    k = ids.shape[1]
+    E = np.asarray(W_r).shape[1]
+    first, nl = sched["first_local"], sched["num_local"]
+    if gs_bwd is None:
+        gs_bwd = nv_weight_scales_bwd(W_gate, W_up, W_down, first, nl)
+    gs_gu, gs_d = gs_bwd
+    gs_dy = nv_global_scale(dY64)
+    dX = np.zeros((T, d))
+    dg = np.zeros((T, k))
+    dW_gate, dW_up, dW_down, parts = {}, {}, {}, []
+    for el, item in enumerate(info["experts"]):
+        e = el + first
+        if item is None:
+            I = np.asarray(_expert(W_gate, e)).shape[1]
+            dW_gate[e] = np.zeros((d, I)); dW_up[e] = np.zeros((d, I)); dW_down[e] = np.zeros((I, d))
+            continue
+        toks, slots, _, A, B = item
+        A, B = bf16_round(A), bf16_round(B)
+        ge = g[toks, slots]
+        dYe = dY64[toks]
+        H = silu(A) * B
+        dHp = nv_round(dYe, gs_dy, axis=1) @ nv_round(_expert(W_down, e), gs_d, axis=1).T  # K = d
+        dg[toks, slots] = np.sum(dHp * H, axis=1)
+        dH = ge[:, None] * dHp
+        dA = dH * B * silu_grad(A)
+        dB = dH * silu(A)
+        Xe = X64[toks]
+        dW_gate[e] = Xe.T @ dA
+        dW_up[e] = Xe.T @ dB
+        dW_down[e] = H.T @ (ge[:, None] * dYe)
+        parts.append((e, toks, dA, dB))
+    live = [np.abs(p[2]).max() for p in parts] + [np.abs(p[3]).max() for p in parts]
+    gs_ab = nv_global_scale(np.array(live)) if live else np.float32(1.0)
+    for e, toks, dA, dB in parts:  # K = I
+        dX[toks] += (nv_round(dA, gs_ab, axis=1) @ nv_round(_expert(W_gate, e), gs_gu, axis=1).T
+                     + nv_round(dB, gs_ab, axis=1) @ nv_round(_expert(W_up, e), gs_gu, axis=1).T)
+    dl = np.zeros((T, E))
+    s = np.sum(g * dg, axis=1, keepdims=True)
+    np.put_along_axis(dl, ids.astype(np.int64), g * (dg - s), axis=1)
+    dX += dl @ _f64(W_r).T
+    return dict(dX=dX, dW_gate=dW_gate, dW_up=dW_up, dW_down=dW_down, dW_r=X64.T @ dl, dl=dl, dg=dg,
+                gs_dy=gs_dy, gs_ab=gs_ab)

@@ -229,3 +229,74 @@ def test_nvfp4_layer_error_against_exact_layer():
     Yp, _ = O.forward(X, W_r, bias, Wg, Wu, Wd, k)
     err = np.max(np.abs(Y - Yp)) / np.max(np.abs(Yp))
     assert 0.01 < err < 0.5
+
+
+# ---------------------------------------------------------------- backward
+def _bwd_case(seed, T=32, d=64, E=4, I=64, k=2):
+    X, W_r, bias, Wg, Wu, Wd, k = _layer(seed, T, d, E, I, k)
+    dY = np.random.default_rng(seed + 100).standard_normal((T, d))
+    dY[0, 0] = 40.0  # amax(dY) held by token 0
+    return X, W_r, bias, Wg, Wu, Wd, k, dY
+
+
+def test_backward_without_rounding_is_the_plain_backward(monkeypatch):
+    X, W_r, bias, Wg, Wu, Wd, k, dY = _bwd_case(21)
+    W_r = np.random.default_rng(1).standard_normal(W_r.shape) * 0.5
+    import oracle.moe_oracle as M
+    monkeypatch.setattr(N, "nv_round", lambda v, gs, axis: np.asarray(v, dtype=np.float64))
+    monkeypatch.setattr(M, "bf16_round", lambda v: np.asarray(v, dtype=np.float64))
+    _, info = N.forward_nv(X, W_r, bias, Wg, Wu, Wd, k)
+    g = N.backward_nv(info, X, W_r, Wg, Wu, Wd, dY)
+    _, ctx = O.forward(X, W_r, bias, Wg, Wu, Wd, k)
+    gp = O.backward(ctx, dY)
+    for n in ("dX", "dW_r"):
+        np.testing.assert_allclose(g[n], gp[n], rtol=1e-12, atol=1e-12)
+    for n in ("dW_gate", "dW_up", "dW_down"):
+        for e in range(4):
+            np.testing.assert_allclose(g[n][e], gp[n][e], rtol=1e-12, atol=1e-12)
+
+
+def test_backward_dy_and_da_db_rounded_along_the_features():
+    # halving token 7's dY halves its dH' exactly (dY rows rounded along d), hence its dA, dB, its
+    # router-gate gradient, and (dA, dB rounded along I) its dX row; every other token's dX stays
+    X, W_r, bias, Wg, Wu, Wd, k, dY = _bwd_case(22)
+    _, info = N.forward_nv(X, W_r, bias, Wg, Wu, Wd, k)
+    g0 = N.backward_nv(info, X, W_r, Wg, Wu, Wd, dY)
+    dY2 = dY.copy()
+    dY2[7] *= 0.5
+    g1 = N.backward_nv(info, X, W_r, Wg, Wu, Wd, dY2)
+    assert g1["gs_ab"] == g0["gs_ab"]
+    np.testing.assert_array_equal(g1["dg"][7], g0["dg"][7] * 0.5)
+    np.testing.assert_array_equal(np.delete(g1["dg"], 7, axis=0), np.delete(g0["dg"], 7, axis=0))
+    np.testing.assert_array_equal(g1["dX"][7], g0["dX"][7] * 0.5)
+    np.testing.assert_array_equal(np.delete(g1["dX"], 7, axis=0), np.delete(g0["dX"], 7, axis=0))
+
+
+def test_backward_w_down_rounded_along_d():
+    # halving row i of every W_down (one I index) halves column i of dH', dA, dB and so of dW_gate
+    X, W_r, bias, Wg, Wu, Wd, k, dY = _bwd_case(23)
+    Wd[0, 0, 0] = 6.0  # amax(W_down) in row 0
+    _, info = N.forward_nv(X, W_r, bias, Wg, Wu, Wd, k)
+    g0 = N.backward_nv(info, X, W_r, Wg, Wu, Wd, dY)
+    Wd2 = Wd.copy()
+    Wd2[:, 11, :] *= 0.5
+    g1 = N.backward_nv(info, X, W_r, Wg, Wu, Wd2, dY)
+    for e in g0["dW_gate"]:
+        np.testing.assert_array_equal(g1["dW_gate"][e][:, 11], g0["dW_gate"][e][:, 11] * 0.5)
+        np.testing.assert_array_equal(np.delete(g1["dW_gate"][e], 11, axis=1), np.delete(g0["dW_gate"][e], 11, axis=1))
+
+
+@pytest.mark.parametrize("which", ["gate", "up"])
+def test_backward_w_gate_up_rounded_along_i(which):
+    # the dgrad of gate/up reads W_gate, W_up along I: halving row j (one d index) of every expert's
+    # W_gate (or W_up) moves only column j of dX
+    X, W_r, bias, Wg, Wu, Wd, k, dY = _bwd_case(24)
+    Wg[0, 0, 0] = 6.0
+    Wu[0, 0, 0] = 6.0  # the joint amax of [W_gate | W_up] in row 0
+    _, info = N.forward_nv(X, W_r, bias, Wg, Wu, Wd, k)
+    g0 = N.backward_nv(info, X, W_r, Wg, Wu, Wd, dY)
+    W2 = (Wg if which == "gate" else Wu).copy()
+    W2[:, 19, :] *= 0.5
+    g1 = N.backward_nv(info, X, W_r, W2 if which == "gate" else Wg, W2 if which == "up" else Wu, Wd, dY)
+    assert not np.array_equal(g1["dX"][:, 19], g0["dX"][:, 19])
+    np.testing.assert_array_equal(np.delete(g1["dX"], 19, axis=1), np.delete(g0["dX"], 19, axis=1))
