@@ -65,7 +65,7 @@ typedef enum moe_precision {
                         operands (X, dA, dB, Hg = g H and dY of each expert) quantised along the
                         expert's rows, one scale per 32 rows from its first row, pad rows zero.
                         Same entry points; a larger workspace (moe_workspace_size of this shape) */,
-  MOE_NVFP4 = 3  /* forward only (moe_fwd_nvfp4): E2M1 operands with one E4M3 scale per 16 values
+  MOE_NVFP4 = 3  /* moe_fwd_nvfp4 / moe_bwd_nvfp4: E2M1 operands with one E4M3 scale per 16 values
                     along each GEMM's contraction dim and one fp32 scale per tensor */
 } moe_precision;
 
@@ -271,7 +271,7 @@ moe_status moe_bwd_mx(const moe_shape* shape, const void* X, const void* W_r, co
                       void* dW_down, float* dW_r, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
- * NVFP4 forward (page 1, "MoE layer as the bottleneck": NVFP4 training kernels
+ * NVFP4 mode (page 1, "MoE layer as the bottleneck": NVFP4 training kernels
  * named as earlier work; the format is NVIDIA's published NVFP4).  Shapes carry
  * prec = MOE_NVFP4.  Each GEMM operand is E2M1 (values 0, 0.5, 1, 1.5, 2, 3, 4,
  * 6 and their negatives) with one E4M3 scale per 16 values along the GEMM's
@@ -286,27 +286,39 @@ moe_status moe_bwd_mx(const moe_shape* shape, const void* X, const void* W_r, co
  * kind::mxf4nvf4 block-scaled tensor cores (K = 64 per MMA) and multiply their
  * fp32 accumulators by 1 / (gs_A gs_B).  H = silu(A) B is formed in fp32 by the
  * gate/up GEMM, its amax sets its global scale, then it is quantised.  Routing
- * is the bf16 router's, Y is bf16.  Forward only: there is no NVFP4 backward.
+ * is the bf16 router's, Y is bf16.  The forward keeps A, B (bf16) and X_perm (bf16) in ctx.
+ *
+ * moe_bwd_nvfp4 runs both dgrad GEMMs on NVFP4 operands: dY [T, d] along d (its own global
+ * scale) with W_down along d; [dA | dB] along I with [W_gate | W_up] along I, each pair one
+ * tensor with one global scale (the GEMM sums over both halves, K = 2I).  dA and dB are formed
+ * in fp32 by the dgrad of W_down's epilogue (SwiGLU backward from the saved bf16 A, B), their
+ * joint amax sets their scale, then they are quantised.  The weight gradients contract the bf16
+ * operands (X_perm, dA, dB, g H, dY_perm) on the bf16 engine, as in MOE_MXFP8; dW_r fp32.
  *
  * moe_prepare_weights with an MOE_NVFP4 shape quantises W_gate, W_up, W_down
  * (the local experts' [El, d, I], [El, d, I], [El, I, d] bf16) into wq
- * (moe_weights_size of that shape): [Wgu codes][Wgu scales][Wd2 codes][Wd2 scales]
- * [global scales], each region on a 256-byte boundary; Wgu [El*2I, d/2 bytes]
- * has the MXFP8 Wgu row order, Wd2 [El*d, I/2 bytes] is W_down transposed; two
- * codes per byte, value 2i in the low nibble of byte i; scale byte
- * (r%32)*16 + ((r%128)/32)*4 + (k%64)/16 of 512-byte chunk (r/128)*(K/64) + k/64;
- * the global scales are three fp32 (gate, up, down).  moe_fwd_nvfp4 takes
- * moe_fwd_mx's arguments; ctx and ws are sized by moe_ctx_size /
- * moe_workspace_size of the MOE_NVFP4 shape; d and I multiples of 256 as
- * everywhere.  Errors as for moe_fwd_mx; moe_get_error reads the device status. */
+ * (moe_weights_size of that shape): the five MXFP8 regions (Wgu, Wd2, Wd3, Wg4,
+ * Wu4, each codes then scales) at half a byte per value, then the global
+ * scales, each region on a 256-byte boundary; two codes per byte, value 2i in
+ * the low nibble of byte i; scale byte (r%32)*16 + ((r%128)/32)*4 + (k%64)/16 of
+ * 512-byte chunk (r/128)*(K/64) + k/64; the global scales are four fp32: gate,
+ * up, down, and [gate | up] (the backward's Wg4 / Wu4 share it).
+ * moe_fwd_nvfp4 / moe_bwd_nvfp4 take moe_fwd_mx's / moe_bwd_mx's arguments; ctx
+ * and ws are sized by moe_ctx_size / moe_workspace_size of the MOE_NVFP4 shape;
+ * d and I multiples of 256 as everywhere.  Errors as for moe_fwd_mx /
+ * moe_bwd_mx; moe_get_error reads the device status. */
 moe_status moe_fwd_nvfp4(const moe_shape* shape, const void* X, const void* W_r, const float* bias, const void* wq,
                          size_t wq_bytes, void* Y, void* ctx, size_t ctx_bytes, void* ws, size_t ws_bytes,
                          void* stream);
-/* Test hook: byte offsets of the NVFP4 forward's buffers.  out[0..1]: X codes and scales in
- * ctx; out[2..5]: H codes, H scales, fp32 H [RP, I] and four scale words (amax X, amax H as
- * fp32 bits, then gs_X, gs_H) in ws; out[6..10]: Wgu codes, Wgu scales, Wd2 codes, Wd2
- * scales and the three weight global scales in wq.  Host only; MOE_ERR_INVALID_ARG for
- * another precision or a NULL out. */
+moe_status moe_bwd_nvfp4(const moe_shape* shape, const void* X, const void* W_r, const void* wq, size_t wq_bytes,
+                         const void* dY, void* ctx, size_t ctx_bytes, void* dX, void* dW_gate, void* dW_up,
+                         void* dW_down, float* dW_r, void* ws, size_t ws_bytes, void* stream);
+/* Test hook: byte offsets of the NVFP4 buffers (out has room for 23).  out[0..1]: X codes and
+ * scales in ctx; out[2..5]: H codes, H scales, fp32 H [RP, I] and eight scale words (amax X,
+ * amax H as fp32 bits, gs_X, gs_H, amax dY, amax [dA | dB], gs_dY, gs_[dA | dB]) in ws;
+ * out[6..10]: Wgu codes, Wgu scales, Wd2 codes, Wd2 scales and the four weight global scales
+ * in wq; out[11..16]: dY, dA, dB codes and scales in ws; out[17..22]: Wd3, Wg4, Wu4 codes and
+ * scales in wq.  Host only; MOE_ERR_INVALID_ARG for another precision or a NULL out. */
 moe_status moe_debug_nv_offsets(const moe_shape* shape, int64_t* out);
 
 /* ---------------------------------------------------------------------------

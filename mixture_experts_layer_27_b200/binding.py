@@ -145,6 +145,8 @@ _SIGS = {
                                   ctypes.c_size_t, _P]),
     "moe_fwd_nvfp4": (ctypes.c_int, [_S, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, ctypes.c_size_t, _P,
                                      ctypes.c_size_t, _P]),
+    "moe_bwd_nvfp4": (ctypes.c_int, [_S, _P, _P, _P, ctypes.c_size_t, _P, _P, ctypes.c_size_t, _P, _P, _P, _P, _P,
+                                     _P, ctypes.c_size_t, _P]),
     "moe_debug_nv_offsets": (ctypes.c_int, [_S, ctypes.POINTER(ctypes.c_int64)]),
     "moe_ep_buffer_size": (ctypes.c_size_t, [_S, ctypes.c_int32]),
     "moe_ep_ctx_size": (ctypes.c_size_t, [_S, ctypes.c_int32]),
@@ -371,8 +373,14 @@ def moe_fwd_nvfp4(shape, X, W_r, bias, wq, Y, ctx, ws, stream=None) -> int:
                                    _ptr(Y), _ptr(ctx), _nbytes(ctx), _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
+def moe_bwd_nvfp4(shape, X, W_r, wq, dY, ctx, dX, dW_gate, dW_up, dW_down, dW_r, ws, stream=None) -> int:
+    return int(lib().moe_bwd_nvfp4(ctypes.byref(shape), _ptr(X), _ptr(W_r), _ptr(wq), _nbytes(wq), _ptr(dY),
+                                   _ptr(ctx), _nbytes(ctx), _ptr(dX), _ptr(dW_gate), _ptr(dW_up), _ptr(dW_down),
+                                   _ptr(dW_r), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
 def moe_debug_nv_offsets(shape) -> list:
-    out = (ctypes.c_int64 * 11)()
+    out = (ctypes.c_int64 * 23)()
     check(int(lib().moe_debug_nv_offsets(ctypes.byref(shape), out)), "moe_debug_nv_offsets")
     return [int(v) for v in out]
 
@@ -480,7 +488,7 @@ class MoELayerMX:
 
 
 class MoELayerNVFP4:
-    """NVFP4 layer forward: prepared (quantised) weights + ctx / workspace owner."""
+    """NVFP4 layer: prepared (quantised) weights + ctx / workspace owner."""
 
     def __init__(self, T, d, E, I, top_k, first_local_expert=0, num_local_experts=0, device="cuda"):
         import torch
@@ -507,6 +515,15 @@ class MoELayerNVFP4:
         _expect_layer(self, self.T, X=X, W_r=W_r, bias=bias, Y=Y)
         check(moe_fwd_nvfp4(self.shape, X, W_r, bias, self.wq, Y, self.ctx, self.ws, stream), "moe_fwd_nvfp4")
         return Y
+
+    def backward(self, X, W_r, dY, out=None, stream=None):
+        import torch
+        if out is None:
+            out = _grad_buffers(self.T, self.d, self.E, self.I, self.El, torch.bfloat16, X.device)
+        _expect_layer(self, self.T, X=X, W_r=W_r, dY=dY, out=out)
+        check(moe_bwd_nvfp4(self.shape, X, W_r, self.wq, dY, self.ctx, out["dX"], out["dW_gate"], out["dW_up"],
+                            out["dW_down"], out["dW_r"], self.ws, stream), "moe_bwd_nvfp4")
+        return out
 
     # --- test accessors (host numpy copies; unpacked codes: one 4-bit code per byte) ---
     @staticmethod
@@ -541,12 +558,32 @@ class MoELayerNVFP4:
         return a[self.off[4]:self.off[4] + RP * self.I * 4].view(np.float32).reshape(RP, self.I)
 
     def scales(self):
-        """(gs_X, gs_H) of the last forward and (gs_gate, gs_up, gs_down) of the prepared weights."""
+        """(gs_X, gs_H) of the last forward and (gs_gate, gs_up, gs_down, gs_gate_up) of the
+        prepared weights."""
         import numpy as np
         torch_sync()
-        w = self.ws.cpu().numpy()[self.off[5]:self.off[5] + 16].view(np.float32)
-        q = self.wq.cpu().numpy()[self.off[10]:self.off[10] + 12].view(np.float32)
+        w = self.ws.cpu().numpy()[self.off[5]:self.off[5] + 32].view(np.float32)
+        q = self.wq.cpu().numpy()[self.off[10]:self.off[10] + 16].view(np.float32)
         return (w[2], w[3]), tuple(q)
+
+    def bwd_scales(self):
+        """(gs_dY, gs_[dA | dB]) of the last backward."""
+        import numpy as np
+        torch_sync()
+        w = self.ws.cpu().numpy()[self.off[5]:self.off[5] + 32].view(np.float32)
+        return w[6], w[7]
+
+    def dy_operand(self):
+        """(codes [RP, d], scale bytes [RP, d/16]) of the quantised dY_perm of the last backward."""
+        torch_sync()
+        return self._operand(self.ws, self.off[11], self.off[12], moe_padded_rows(self.shape_bf16), self.d)
+
+    def bwd_weight_regions(self):
+        """{"Wd3": W_down [El*I, d], "Wg4": W_gate [El*d, I], "Wu4": W_up [El*d, I]}: (codes, scales)."""
+        El, d, I = self.El, self.d, self.I
+        return {"Wd3": self._operand(self.wq, self.off[17], self.off[18], El * I, d),
+                "Wg4": self._operand(self.wq, self.off[19], self.off[20], El * d, I),
+                "Wu4": self._operand(self.wq, self.off[21], self.off[22], El * d, I)}
 
     def weight_regions(self):
         """{"Wgu": (codes [El*2I, d], scales [El*2I, d/16]), "Wd2": (codes [El*d, I], scales [El*d, I/16])}."""

@@ -48,7 +48,7 @@ __device__ __forceinline__ void mx_wseg(const MxParams& p, int m, int el, int& r
 template <int KIND>
 __device__ __forceinline__ int mx_ntiles_n(const MxParams& p) {
   if (KIND == MX_GATEUP || KIND == NV_GATEUP) return p.I / (mx_bn(KIND) / 2);  // per tile: [64 gate | 64 up] column pairs
-  if (KIND == MX_DGRAD_DOWN) return p.I / mx_bn(KIND);
+  if (KIND == MX_DGRAD_DOWN || KIND == NV_DGRAD_DOWN) return p.I / mx_bn(KIND);
   if (KIND == MX_WGRAD_GATEUP) return 2 * p.I / 256;  // gate n-tiles, then up n-tiles
   return p.d / mx_bn(KIND);  // MX_DOWN, MX_DGRAD_GATEUP, MX_WGRAD_DOWN
 }
@@ -59,8 +59,9 @@ __device__ __forceinline__ int mx_mtiles_w(const MxParams& p) {
 }
 template <int KIND>
 __device__ __forceinline__ int mx_kblocks(const MxParams& p) {
-  if (KIND == NV_GATEUP) return p.d / 256;  // 128-byte K stages of 256 E2M1 codes
+  if (KIND == NV_GATEUP || KIND == NV_DGRAD_DOWN) return p.d / 256;  // 128-byte K stages of 256 E2M1 codes
   if (KIND == NV_DOWN) return p.I / 256;
+  if (KIND == NV_DGRAD_GATEUP) return 2 * p.I / 256;
   if (KIND == MX_GATEUP || KIND == MX_DGRAD_DOWN) return p.d / 128;
   if (KIND == MX_DOWN) return p.I / 128;
   return 2 * p.I / 128;
@@ -133,15 +134,36 @@ __device__ __forceinline__ void mx_load(const MxParams& p, const MxTile& tl, int
   const uint8_t* sfb = p.sfb0;
   if constexpr (mx_is_nv(KIND)) {
     // NVFP4: 128 bytes of K = 256 codes; per 128 rows the stage's four 64-deep scale chunks are
-    // contiguous (2 KB): A's, then those of B's two 128-row halves
-    const int brow = KIND == NV_GATEUP ? tl.el * 2 * p.I + tl.nt * BN : tl.el * p.d + tl.n0;
-    const int K = KIND == NV_GATEUP ? p.d : p.I;
+    // contiguous (2 KB): A's, then those of B's 128-row halves
+    int brow, K, kl = kb;
+    if constexpr (KIND == NV_GATEUP) {
+      brow = tl.el * 2 * p.I + tl.nt * BN;
+      K = p.d;
+    } else if constexpr (KIND == NV_DOWN) {
+      brow = tl.el * p.d + tl.n0;
+      K = p.I;
+    } else if constexpr (KIND == NV_DGRAD_DOWN) {
+      brow = tl.el * p.I + tl.n0;
+      K = p.d;
+    } else {  // NV_DGRAD_GATEUP: K = 2I, the dA / W_gate half, then the dB / W_up half
+      const int half = p.I / 256;
+      if (kb >= half) {
+        kl = kb - half;
+        ma = &p.ta1;
+        mb = &p.tb1;
+        sfa = p.sfa1;
+        sfb = p.sfb1;
+      }
+      brow = tl.el * p.d + tl.n0;
+      K = p.I;
+    }
     const int arow = tl.m0;
-    tma_load_2d(sA, ma, bar, kb * 128, arow, pol_act);
-    tma_load_2d(sB, mb, bar, kb * 128, brow, pol_w);
-    bulk_load(sSF, sfa + (static_cast<size_t>(arow >> 7) * (K >> 6) + 4 * kb) * 512, 2048, bar);
-    bulk_load(sSF + 2048, sfb + (static_cast<size_t>(brow >> 7) * (K >> 6) + 4 * kb) * 512, 2048, bar);
-    bulk_load(sSF + 4096, sfb + (static_cast<size_t>((brow >> 7) + 1) * (K >> 6) + 4 * kb) * 512, 2048, bar);
+    tma_load_2d(sA, ma, bar, kl * 128, arow, pol_act);
+    tma_load_2d(sB, mb, bar, kl * 128, brow, pol_w);
+    bulk_load(sSF, sfa + (static_cast<size_t>(arow >> 7) * (K >> 6) + 4 * kl) * 512, 2048, bar);
+    bulk_load(sSF + 2048, sfb + (static_cast<size_t>(brow >> 7) * (K >> 6) + 4 * kl) * 512, 2048, bar);
+    if constexpr (BN == 256)
+      bulk_load(sSF + 4096, sfb + (static_cast<size_t>((brow >> 7) + 1) * (K >> 6) + 4 * kl) * 512, 2048, bar);
     (void)krow;
     return;
   }
@@ -299,8 +321,16 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
       tmem_ld32(taddr + j * 128 + 64 + c32, b);  // up
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float av = a[i] * ag;
-        a[i] = av / (1.0f + expf(-av)) * (b[i] * au);
+        a[i] *= ag;
+        b[i] *= au;
+      }
+      if (live && p.out0) {  // A, B saved (bf16) for the backward
+        mx_store_bf16_32(p.out0 + Rz * p.I + tl.n0 + j * 64 + c32, a);
+        mx_store_bf16_32(p.out1 + Rz * p.I + tl.n0 + j * 64 + c32, b);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        a[i] = a[i] / (1.0f + expf(-a[i])) * b[i];
         hmax = fmaxf(hmax, fabsf(a[i]));
       }
       if (live) {
@@ -323,6 +353,66 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
 #pragma unroll
       for (int i = 0; i < 32; ++i) o[i] = o[i] * al * g;
       if (live) mx_store_bf16_32(p.out0 + Rz * p.d + tl.n0 + c * 32, o);
+    }
+  } else if constexpr (KIND == NV_DGRAD_DOWN) {
+    // dH' = acc / (gs_dY gs_down); the SwiGLU backward from the saved bf16 A, B as in
+    // MX_DGRAD_DOWN; bf16 dA, dB, Hg for the bf16 weight gradients, fp32 dA, dB for their NVFP4
+    // quantisation and the largest |dA|, |dB| of the warp's live rows into *amax
+    const float al = __frcp_rn(__fmul_rn(__ldg(p.gsa), __ldg(p.gsb)));
+    const float g = p.row_gate[R];
+    float dg = 0.f, amx = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      float dh[32], a[32], b[32];
+      tmem_ld32(taddr + c * 32, dh);
+      const int col = tl.n0 + c * 32;
+      if (live) {
+        mx_load_bf16_32(p.in0 + Rz * p.I + col, a);
+        mx_load_bf16_32(p.in1 + Rz * p.I + col, b);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) a[i] = b[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float d1 = dh[i] * al;
+        const float s = mx_sigmoid(a[i]);
+        const float sl = a[i] * s;
+        const float hh = sl * b[i];
+        dg = fmaf(d1, hh, dg);
+        const float dhg = g * d1;
+        a[i] = dhg * b[i] * (s * (1.0f + a[i] * (1.0f - s)));  // dA
+        b[i] = dhg * sl;                                       // dB
+        dh[i] = g * hh;                                        // Hg
+        amx = fmaxf(amx, fmaxf(fabsf(a[i]), fabsf(b[i])));
+      }
+      if (live) {
+        mx_store_bf16_32(p.out0 + Rz * p.I + col, a);
+        mx_store_bf16_32(p.out1 + Rz * p.I + col, b);
+        mx_store_bf16_32(p.out2 + Rz * p.I + col, dh);
+        float4* fa = reinterpret_cast<float4*>(p.hout + Rz * p.I + col);
+        float4* fb = reinterpret_cast<float4*>(p.hout2 + Rz * p.I + col);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          fa[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+          fb[q] = make_float4(b[4 * q], b[4 * q + 1], b[4 * q + 2], b[4 * q + 3]);
+        }
+      }
+    }
+    if (live) p.outf[Rz * (p.I / BN) + tl.nt] = dg;
+    if (!live) amx = 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amx = fmaxf(amx, __shfl_xor_sync(0xffffffffu, amx, o));
+    if ((row & 31) == 0 && amx > 0.f) atomicMax(p.amax, __float_as_uint(amx));
+  } else if constexpr (KIND == NV_DGRAD_GATEUP) {
+    const float al = __frcp_rn(__fmul_rn(__ldg(p.gsa), __ldg(p.gsb)));
+#pragma unroll 1
+    for (int c = cbeg; c < cend; ++c) {
+      float v[32];
+      tmem_ld32(taddr + c * 32, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= al;
+      if (live) mx_store_bf16_32(p.out0 + Rz * p.d + tl.n0 + c * 32, v);
     }
   } else if constexpr (KIND == MX_DOWN) {
     const float g = p.row_gate[R];
@@ -600,19 +690,20 @@ __global__ void __launch_bounds__(mx_threads(KIND), 1) k_moe_gemm_mx(const __gri
           // scale slot of this stage: 16 columns from column 256 on; A in the first 4,
           // B (rows 0..127, then 128..255) in the columns from 8 on
           if constexpr (mx_is_nv(KIND)) {
-            // per stage 48 TMEM columns above the accumulator: A's four chunks (4 columns each),
-            // then per K = 64 step the two 128-row halves of B (8 columns)
-            const uint32_t nfa = tbase + 256 + stage * 48, nfb = nfa + 16;
+            // per stage TMEM columns above the accumulators: A's four chunks (4 columns each),
+            // then per K = 64 step B's 128-row halves (4 columns each)
+            constexpr uint32_t BW = 4 * (BN / 128);  // B columns per K = 64 step
+            const uint32_t nfa = tbase + 256 + stage * (16 + 4 * BW), nfb = nfa + 16;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               tc_cp_sf(nfa + 4 * kk, sf0 + 512 * kk);
-              tc_cp_sf(nfb + 8 * kk, sf0 + 2048 + 512 * kk);
-              tc_cp_sf(nfb + 8 * kk + 4, sf0 + 4096 + 512 * kk);
+              tc_cp_sf(nfb + BW * kk, sf0 + 2048 + 512 * kk);
+              if constexpr (BN == 256) tc_cp_sf(nfb + BW * kk + 4, sf0 + 4096 + 512 * kk);
             }
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               umma_nvf4(dtm, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024),
-                        idesc_nvf4(128, BN), nfa + 4 * kk, nfb + 8 * kk, (kb | kk) != 0 ? 1u : 0u);
+                        idesc_nvf4(128, BN), nfa + 4 * kk, nfb + BW * kk, (kb | kk) != 0 ? 1u : 0u);
             umma_commit(&empty[stage]);
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
             continue;
@@ -711,6 +802,8 @@ cudaError_t launch_gemm_mx(MxKind kind, const MxParams& p, int grid, cudaStream_
     case MX_WGRAD_DOWN: return mx_launch_kind<MX_WGRAD_DOWN>(p, grid, st);
     case NV_GATEUP: return mx_launch_kind<NV_GATEUP>(p, grid, st);
     case NV_DOWN: return mx_launch_kind<NV_DOWN>(p, grid, st);
+    case NV_DGRAD_DOWN: return mx_launch_kind<NV_DGRAD_DOWN>(p, grid, st);
+    case NV_DGRAD_GATEUP: return mx_launch_kind<NV_DGRAD_GATEUP>(p, grid, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -71,7 +71,7 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->row_asg = take(RP * 4);
   L->row_gate = take(RP * 4);
   // streamed layer: X_perm lives in the caller's ring; MXFP8 weight gradients keep X quantised instead
-  L->xperm = take(M > 0 || s.prec == MOE_MXFP8_ALL || L->nv ? 0 : RP * s.d * 2);
+  L->xperm = take(M > 0 || s.prec == MOE_MXFP8_ALL ? 0 : RP * s.d * 2);
   L->abuf = take(RP * s.I * 2);
   L->bbuf = take(RP * s.I * 2);
   L->stab = take(M > 0 ? static_cast<size_t>(stream_table_words(M, El)) * 4 : 0);
@@ -110,12 +110,13 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->hqs = take(L->nv ? RP * s.I / 16 : mxi / 32);
   L->nvh = take(L->nv ? RP * s.I * 4 : 0);
   L->nvsc = take(L->nv ? 256 : 0);
-  L->dyq = take(mxd);
-  L->dyqs = take(mxd / 32);
-  L->daq = take(mxi);
-  L->daqs = take(mxi / 32);
-  L->dbq = take(mxi);
-  L->dbqs = take(mxi / 32);
+  L->dyq = take(L->nv ? RP * s.d / 2 : mxd);
+  L->dyqs = take(L->nv ? RP * s.d / 16 : mxd / 32);
+  L->daq = take(L->nv ? RP * s.I / 2 : mxi);
+  L->daqs = take(L->nv ? RP * s.I / 16 : mxi / 32);
+  L->dbq = take(L->nv ? RP * s.I / 2 : mxi);
+  L->dbqs = take(L->nv ? RP * s.I / 16 : mxi / 32);
+  L->nvdab = take(L->nv ? 2 * RP * s.I * 4 : 0);
   L->fctl = take(L->mx ? 0 : static_cast<size_t>(gemm_pair_ctl_words(L->RP)) * 4);
   L->dyqt = take(wxd);
   L->dyqts = take(wxd / 32);
@@ -128,10 +129,10 @@ bool make_layout(const moe_shape& s, Layout* L, int M) {
   L->ws_bytes = o;
   // prepared weights: [W_gate|W_up paired, K = d] [W_down^T, K = I] [W_down, K = d] [W_gate, K = I] [W_up, K = I]
   o = 0;
-  // NVFP4: the two forward layouts only (half a byte per value, a scale byte per 16), then the
-  // three global scales (and their amax words)
+  // NVFP4: the same five layouts at half a byte per value and a scale byte per 16, then the four
+  // global scales (and their amax words)
   const size_t w1 = static_cast<size_t>(El) * s.d * s.I;
-  const size_t wb = L->nv ? w1 / 2 : w1, wsb = L->nv ? w1 / 16 : w1 / 32, wbwd = L->nv ? 0 : 1;
+  const size_t wb = L->nv ? w1 / 2 : w1, wsb = L->nv ? w1 / 16 : w1 / 32, wbwd = 1;
   L->wgu1 = take(2 * wb);
   L->wgu1s = take(2 * wsb);
   L->wd2 = take(wb);
@@ -188,6 +189,7 @@ Ctx make_ctx(const Layout& L, void* ctx, void* ws) {
   c.xqs = L.mx || L.nv ? reinterpret_cast<uint8_t*>(C(L.xqs)) : nullptr;
   c.nvh = (ws && L.nv) ? reinterpret_cast<float*>(W(L.nvh)) : nullptr;
   c.nvsc = (ws && L.nv) ? reinterpret_cast<unsigned*>(W(L.nvsc)) : nullptr;
+  c.nvdab = (ws && L.nv) ? reinterpret_cast<float*>(W(L.nvdab)) : nullptr;
   c.hq = c.hqs = c.dyq = c.dyqs = c.daq = c.daqs = c.dbq = c.dbqs = nullptr;
   c.xqt = c.xqts = c.dyqt = c.dyqts = c.daqt = c.daqts = c.dbqt = c.dbqts = c.hgqt = c.hgqts = nullptr;
   if (L.mxw) {
@@ -328,7 +330,7 @@ enum KernelId {
   K_REV_COMBINE, K_GEMM_DGRAD_DOWN, K_ROUTER_BWD, K_ROUTER_WGRAD, K_TRANSPOSE_WR, K_GEMM_DGRAD_GATEUP, K_REV_DISPATCH,
   K_GEMM_WGRAD_GATEUP, K_GEMM_WGRAD_DOWN, K_PLAN, K_REPLAY, K_FINISH_ACC, K_QUANT_WEIGHTS, K_MARK_ROWS,
   K_ACTIVE_COUNT, K_GATHER_ACTIVE, K_SCAN_GROUPS, K_SCAN_APPLY, K_PAIR_FWD, K_PAIR_DGRAD, K_MX_WGRAD_GATEUP, K_MX_WGRAD_DOWN,
-  K_NV_SCALE, K_NV_GATEUP, K_NV_QUANT_H, K_NV_DOWN, K_NUM
+  K_NV_SCALE, K_NV_GATEUP, K_NV_QUANT_H, K_NV_DOWN, K_NV_DGRAD_DOWN, K_NV_QUANT_DAB, K_NV_DGRAD_GATEUP, K_NUM
 };
 static const char* kKernelNames[K_NUM] = {
     "router_logits", "topk_gating", "hist_scan", "stable_scatter", "dispatch", "gemm_gateup_swiglu",
@@ -337,7 +339,8 @@ static const char* kKernelNames[K_NUM] = {
     "stream_plan", "ring_replay", "wgrad_accumulator_finish", "quantize_weights", "mark_pad_rows",
     "router_token_count", "router_token_gather", "hist_scan_group_sums", "hist_scan_group_apply",
     "gemm_gateup_down_persistent", "gemm_dgrads_persistent", "gemm_wgrad_gateup_mx", "gemm_wgrad_down_mx",
-    "nvfp4_amax_scale", "gemm_gateup_swiglu_nvfp4", "nvfp4_quantize_h", "gemm_down_combw_nvfp4"};
+    "nvfp4_amax_scale", "gemm_gateup_swiglu_nvfp4", "nvfp4_quantize_h", "gemm_down_combw_nvfp4",
+    "gemm_dgrad_down_swiglu_bwd_nvfp4", "nvfp4_quantize_da_db", "gemm_dgrad_gateup_nvfp4"};
 
 struct ProfRec {
   int kid;
@@ -1322,12 +1325,14 @@ static moe_status prepare_weights_nv(const moe_shape* s, const void* W_gate, con
   const auto* u = static_cast<const __nv_bfloat16*>(W_up);
   const auto* dn = static_cast<const __nv_bfloat16*>(W_down);
   const int64_t n = static_cast<int64_t>(L.El) * L.d * L.I;
-  MOE_TRY(cudaMemsetAsync(amx, 0, 3 * sizeof(unsigned), st));
-  MOE_TRY(timed(K_QUANT_WEIGHTS, st, [&] {
+  MOE_TRY(cudaMemsetAsync(amx, 0, 4 * sizeof(unsigned), st));
+  MOE_TRY(timed(K_QUANT_WEIGHTS, st, [&] {  // gate, up, down, and [gate | up] for the dgrad of gate/up
     cudaError_t e = launch_nv_amax(g, n, amx, st);
     if (e == cudaSuccess) e = launch_nv_amax(u, n, amx + 1, st);
     if (e == cudaSuccess) e = launch_nv_amax(dn, n, amx + 2, st);
-    if (e == cudaSuccess) e = launch_nv_scale(amx, gs, 3, st);
+    if (e == cudaSuccess) e = launch_nv_amax(g, n, amx + 3, st);
+    if (e == cudaSuccess) e = launch_nv_amax(u, n, amx + 3, st);
+    if (e == cudaSuccess) e = launch_nv_scale(amx, gs, 4, st);
     return e;
   }));
   MOE_TRY(timed(K_QUANT_WEIGHTS, st, [&] {
@@ -1335,6 +1340,15 @@ static moe_status prepare_weights_nv(const moe_shape* s, const void* W_gate, con
   }));
   MOE_TRY(timed(K_QUANT_WEIGHTS, st, [&] {
     return launch_nv_quant_weight(false, dn, nullptr, L.El, L.I, L.d, gs + 2, w + L.wd2, w + L.wd2s, st);
+  }));
+  // the backward's layouts, as stored: W_down [El*I, d] (K = d), W_gate, W_up [El*d, I] (K = I)
+  MOE_TRY(timed(K_QUANT_WEIGHTS, st, [&] {
+    cudaError_t e = launch_nv_quant_rows(dn, static_cast<int64_t>(L.El) * L.I, L.d, gs + 2, w + L.wd3, w + L.wd3s, st);
+    if (e == cudaSuccess)
+      e = launch_nv_quant_rows(g, static_cast<int64_t>(L.El) * L.d, L.I, gs + 3, w + L.wg4, w + L.wg4s, st);
+    if (e == cudaSuccess)
+      e = launch_nv_quant_rows(u, static_cast<int64_t>(L.El) * L.d, L.I, gs + 3, w + L.wu4, w + L.wu4s, st);
+    return e;
   }));
   return MOE_OK;
 }
@@ -1526,7 +1540,7 @@ moe_status moe_fwd_nvfp4(const moe_shape* s, const void* X, const void* W_r, con
   const Ctx c = make_ctx(L, ctx, ws);
   MOE_TRY(cudaMemsetAsync(c.hdr, 0, HDR_WORDS * 4, st));
   if (L.T == 0) return MOE_OK;
-  MOE_TRY(cudaMemsetAsync(c.nvsc, 0, 4 * sizeof(unsigned), st));
+  MOE_TRY(cudaMemsetAsync(c.nvsc, 0, 4 * sizeof(unsigned), st));  // amax X, amax H, gs X, gs H
   {
     const moe_status r = route_tokens(L, c, X, W_r, bias, 0, st);
     if (r != MOE_OK) return r;
@@ -1540,7 +1554,8 @@ moe_status moe_fwd_nvfp4(const moe_shape* s, const void* X, const void* W_r, con
     const cudaError_t e = launch_nv_amax(Xb, L.T * static_cast<int64_t>(L.d), amx, st);
     return e != cudaSuccess ? e : launch_nv_scale(amx, gsv, 1, st);
   }));
-  MOE_TRY(timed(K_DISPATCH, st, [&] { return launch_nv_gather_x(L, c, Xb, gsv, c.xq, c.xqs, st); }));
+  // X's codes for the gate/up GEMM, and X_perm in bf16 for the weight gradients
+  MOE_TRY(timed(K_DISPATCH, st, [&] { return launch_nv_gather_x(L, c, Xb, gsv, c.xq, c.xqs, c.xperm, st); }));
   const int grid = num_sms();
   int* status = c.hdr + HDR_STATUS;
   const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
@@ -1556,6 +1571,8 @@ moe_status moe_fwd_nvfp4(const moe_shape* s, const void* X, const void* W_r, con
     p.gsb = gsw;
     p.hout = c.nvh;
     p.amax = amx + 1;
+    p.out0 = c.abuf;  // A, B (bf16) saved for the backward
+    p.out1 = c.bbuf;
     MOE_TRY(timed(K_NV_GATEUP, st, [&] { return launch_gemm_mx(NV_GATEUP, p, grid, st); }));
   }
   MOE_TRY(timed(K_NV_QUANT_H, st, [&] {
@@ -1579,17 +1596,105 @@ moe_status moe_fwd_nvfp4(const moe_shape* s, const void* X, const void* W_r, con
   return MOE_OK;
 }
 
-// Byte offsets of the NVFP4 forward's buffers, for tests: out[0..1] X codes and scales (ctx),
-// out[2..4] H codes, scales, fp32 H (workspace), out[5] the workspace's scale words, out[6..9]
-// gate/up codes and scales, W_down codes and scales, out[10] the weights' global scales
+// NVFP4 backward: the reverse-combine quantises dY along d (its global scale from an amax pass)
+// and keeps its bf16 rows; the dgrad of W_down (SwiGLU backward and router-gate gradient in its
+// epilogue) writes bf16 dA, dB, Hg and fp32 dA, dB with their joint amax; the router backward;
+// [dA | dB] quantised along I under one scale; the dgrad of gate/up over K = 2I; the reverse
+// dispatch; the weight gradients from the bf16 operands.
+moe_status moe_bwd_nvfp4(const moe_shape* s, const void* X, const void* W_r, const void* wq, size_t wq_bytes,
+                         const void* dY, void* ctx, size_t ctx_bytes, void* dX, void* dW_gate, void* dW_up,
+                         void* dW_down, float* dW_r, void* ws, size_t ws_bytes, void* stream) {
+  Layout L;
+  const moe_status cs = check_shape_nv(s, &L);
+  if (cs != MOE_OK) return cs;
+  const bool tok = s->T > 0;
+  if ((tok && (!X || !dY || !dX)) || !W_r || !wq || !ctx || !dW_gate || !dW_up || !dW_down || !dW_r || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W_r) || !aligned16(wq) || !aligned16(dY) || !aligned16(ctx) || !aligned16(dX) ||
+      !aligned16(dW_gate) || !aligned16(dW_up) || !aligned16(dW_down) || !aligned16(dW_r) || !aligned16(ws))
+    return MOE_ERR_INVALID_ARG;
+  if (ctx_bytes < L.ctx_bytes || ws_bytes < L.ws_bytes || wq_bytes < L.wq_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ctx c = make_ctx(L, ctx, ws);
+  if (L.T == 0) return zero_wgrads(L, dW_gate, dW_up, dW_down, dW_r, st);
+  const int grid = num_sms();
+  int* status = c.hdr + HDR_STATUS;
+  const uint64_t RP = static_cast<uint64_t>(L.RP), El = static_cast<uint64_t>(L.El);
+  const auto* w = static_cast<const uint8_t*>(wq);
+  const float* gsw = reinterpret_cast<const float*>(w + L.wnvgs);  // [gate, up, down, gate | up]
+  unsigned* amx = c.nvsc + 4;                                      // [amax dY, amax dA | dB]
+  float* gsv = reinterpret_cast<float*>(c.nvsc + 6);               // [gs dY, gs dA | dB]
+  const auto* dYb = static_cast<const __nv_bfloat16*>(dY);
+  MOE_TRY(cudaMemsetAsync(amx, 0, 2 * sizeof(unsigned), st));
+  MOE_TRY(timed(K_NV_SCALE, st, [&] {
+    const cudaError_t e = launch_nv_amax(dYb, L.T * static_cast<int64_t>(L.d), amx, st);
+    return e != cudaSuccess ? e : launch_nv_scale(amx, gsv, 1, st);
+  }));
+  MOE_TRY(timed(K_REV_COMBINE, st, [&] { return launch_nv_gather_x(L, c, dYb, gsv, c.dyq, c.dyqs, c.dyperm, st); }));
+  {
+    MxParams p = mx_params(L, c, status);
+    MOE_TMAP(tmap_fp8(&p.ta0, c.dyq, L.d / 2, RP, 128));
+    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wd3, L.d / 2, El * L.I, mx_bn(NV_DGRAD_DOWN)));
+    p.ta1 = p.ta0;
+    p.tb1 = p.tb0;
+    p.sfa0 = p.sfa1 = c.dyqs;
+    p.sfb0 = p.sfb1 = w + L.wd3s;
+    p.in0 = c.abuf;
+    p.in1 = c.bbuf;
+    p.out0 = c.dabuf;
+    p.out1 = c.dbbuf;
+    p.out2 = c.hgbuf;
+    p.hout = c.nvdab;
+    p.hout2 = c.nvdab + RP * L.I;
+    p.amax = amx + 1;
+    p.gsa = gsv;
+    p.gsb = gsw + 2;
+    p.outf = c.dgpart;
+    MOE_TRY(timed(K_NV_DGRAD_DOWN, st, [&] { return launch_gemm_mx(NV_DGRAD_DOWN, p, grid, st); }));
+  }
+  MOE_TRY_STATUS(router_backward(L, c, X, dW_r, status, st, L.I / mx_bn(NV_DGRAD_DOWN)));
+  MOE_TRY(timed(K_TRANSPOSE_WR, st, [&] {
+    return launch_transpose_wr(L, static_cast<const __nv_bfloat16*>(W_r), c.wrt, st);
+  }));
+  MOE_TRY(timed(K_NV_QUANT_DAB, st, [&] {
+    cudaError_t e = launch_nv_scale(amx + 1, gsv + 1, 1, st);
+    if (e == cudaSuccess) e = launch_nv_quant_h(L, c, c.nvdab, gsv + 1, c.daq, c.daqs, st);
+    if (e == cudaSuccess) e = launch_nv_quant_h(L, c, c.nvdab + RP * L.I, gsv + 1, c.dbq, c.dbqs, st);
+    return e;
+  }));
+  {
+    MxParams p = mx_params(L, c, status);
+    MOE_TMAP(tmap_fp8(&p.ta0, c.daq, L.I / 2, RP, 128));
+    MOE_TMAP(tmap_fp8(&p.ta1, c.dbq, L.I / 2, RP, 128));
+    MOE_TMAP(tmap_fp8(&p.tb0, w + L.wg4, L.I / 2, El * L.d, mx_bn(NV_DGRAD_GATEUP)));
+    MOE_TMAP(tmap_fp8(&p.tb1, w + L.wu4, L.I / 2, El * L.d, mx_bn(NV_DGRAD_GATEUP)));
+    p.sfa0 = c.daqs;
+    p.sfa1 = c.dbqs;
+    p.sfb0 = w + L.wg4s;
+    p.sfb1 = w + L.wu4s;
+    p.gsa = gsv + 1;
+    p.gsb = gsw + 3;
+    p.out0 = c.dxperm;
+    MOE_TRY(timed(K_NV_DGRAD_GATEUP, st, [&] { return launch_gemm_mx(NV_DGRAD_GATEUP, p, grid, st); }));
+  }
+  MOE_TRY(timed(K_REV_DISPATCH, st, [&] { return launch_rev_dispatch(L, c, static_cast<__nv_bfloat16*>(dX), st); }));
+  return launch_wgrads(L, c, status, dW_gate, dW_up, dW_down, st);
+}
+
+// Byte offsets of the NVFP4 buffers, for tests: out[0..1] X codes and scales (ctx), out[2..4] H
+// codes, scales, fp32 H (workspace), out[5] the workspace's scale words, out[6..9] gate/up codes
+// and scales, W_down^T codes and scales, out[10] the weights' global scales (prepared weights),
+// out[11..14] dY codes and scales, dA codes and scales (workspace), out[15..16] dB codes and
+// scales (workspace), out[17..22] W_down (K = d), W_gate (K = I), W_up (K = I) codes and scales
 // (prepared weights).
 moe_status moe_debug_nv_offsets(const moe_shape* s, int64_t* out) {
   Layout L;
   const moe_status cs = check_shape_nv(s, &L);
   if (cs != MOE_OK) return cs;
   if (!out) return MOE_ERR_INVALID_ARG;
-  const size_t v[11] = {L.xq, L.xqs, L.hq, L.hqs, L.nvh, L.nvsc, L.wgu1, L.wgu1s, L.wd2, L.wd2s, L.wnvgs};
-  for (int i = 0; i < 11; ++i) out[i] = static_cast<int64_t>(v[i]);
+  const size_t v[23] = {L.xq,  L.xqs,  L.hq,  L.hqs,  L.nvh,  L.nvsc, L.wgu1, L.wgu1s, L.wd2, L.wd2s, L.wnvgs, L.dyq,
+                        L.dyqs, L.daq, L.daqs, L.dbq, L.dbqs, L.wd3, L.wd3s, L.wg4, L.wg4s, L.wu4, L.wu4s};
+  for (int i = 0; i < 23; ++i) out[i] = static_cast<int64_t>(v[i]);
   return MOE_OK;
 }
 

@@ -77,11 +77,14 @@ struct Layout {
   bool mxw;  // MXFP8 mode with the weight-gradient GEMMs on MXFP8 as well
   bool w32;  // expert weight gradients written as fp32
   bool rslice;  // an expert slice (El < E): the router weight gradient runs over the listed tokens
-  bool nv;      // NVFP4 forward (moe_fwd_nvfp4): xq / xqs and hq / hqs hold E2M1 codes (two per byte)
-                // and E4M3 scale chunks (nv_sf_index), nvh the gate/up GEMM's fp32 H [RP, I], nvsc four
-                // words: amax(X), amax(H) (fp32 bits), then their global scales; the prepared weights
-                // are the two forward layouts and three global scales (wnvgs: gate, up, down)
-  size_t nvh, nvsc, wnvgs;
+  bool nv;      // NVFP4 (moe_fwd_nvfp4 / moe_bwd_nvfp4): xq / xqs, hq / hqs, dyq / dyqs, daq / daqs,
+                // dbq / dbqs hold E2M1 codes (two per byte) and E4M3 scale chunks (nv_sf_index); nvh the
+                // gate/up GEMM's fp32 H [RP, I], nvdab the dgrad of W_down's fp32 dA, dB; nvsc eight
+                // words: amax X, H, dY, [dA | dB] (fp32 bits) and their global scales, in the order
+                // amax X, amax H, gs X, gs H, amax dY, amax dAB, gs dY, gs dAB; the prepared weights are
+                // the five MXFP8 layouts in NVFP4 and the global scales gate, up, down, [gate | up]
+                // (wnvgs, then four amax words at +64)
+  size_t nvh, nvsc, wnvgs, nvdab;
   // prepared MXFP8 weights (moe_prepare_weights): fp8 codes and scale chunks
   size_t wgu1, wgu1s, wd2, wd2s, wd3, wd3s, wg4, wg4s, wu4, wu4s, wq_bytes;
 };
@@ -205,6 +208,8 @@ enum MxKind {
   MX_WGRAD_DOWN = 5,    // dW_down = Hgq^T dYq per expert
   NV_GATEUP = 6,        // NVFP4 (kind::mxf4nvf4): H = silu(A) B from Xq . [Wg|Wu]q, fp32 H and its amax out
   NV_DOWN = 7,          // NVFP4: O' = g * (Hq . Wd_q)
+  NV_DGRAD_DOWN = 8,    // NVFP4: dH' = dYq . Wd_q^T; SwiGLU backward; bf16 dA, dB, Hg and fp32 dA, dB (+ amax) out
+  NV_DGRAD_GATEUP = 9,  // NVFP4: dX_perm = [dA | dB]q . [Wg | Wu]q^T (K = 2I, one global scale per operand)
 };
 struct MxParams {
   CUtensorMap ta0, ta1, tb0, tb1;  // fp8 K-major operands, box {128 bytes of K, 128 rows (A) / mx_bn rows (B)}
@@ -250,17 +255,23 @@ struct MxParams {
   const float* gsb;
   float* hout;
   unsigned* amax;
+  float* hout2;  // NV_DGRAD_DOWN: fp32 dB beside hout's fp32 dA
 };
 __host__ __device__ constexpr bool mx_is_wgrad(int kind) { return kind == MX_WGRAD_GATEUP || kind == MX_WGRAD_DOWN; }
-__host__ __device__ constexpr bool mx_is_nv(int kind) { return kind == NV_GATEUP || kind == NV_DOWN; }
+__host__ __device__ constexpr bool mx_is_nv(int kind) {
+  return kind == NV_GATEUP || kind == NV_DOWN || kind == NV_DGRAD_DOWN || kind == NV_DGRAD_GATEUP;
+}
 // Tile width per kind: 128 x 256 tiles (one accumulator, four stages) keep 32 KB of fp8 weights
 // per stage in flight; the dgrad of W_down, whose epilogue reads and writes the most, keeps
 // 128 x 128 tiles with two accumulators (six stages) so that its epilogue overlaps the MMAs.
 // A stage = A tile (128 rows x 128 bytes of K), B tile (BN rows), the A scale chunk and BN/128
 // B scale chunks; stages start on 1 KB boundaries (128-byte swizzle atoms).
-__host__ __device__ constexpr int mx_bn(int kind) { return kind == MX_DGRAD_DOWN ? 128 : 256; }
+__host__ __device__ constexpr int mx_bn(int kind) { return kind == MX_DGRAD_DOWN || kind == NV_DGRAD_DOWN ? 128 : 256; }
 __host__ __device__ constexpr int mx_accs(int kind) { return mx_bn(kind) == 128 ? 2 : 1; }
-__host__ __device__ constexpr int mx_stages(int kind) { return mx_bn(kind) == 128 ? 6 : (mx_is_wgrad(kind) ? 3 : 4); }
+// (NVFP4 128 x 128: five stages, its 36 KB stages carrying four scale chunks per operand)
+__host__ __device__ constexpr int mx_stages(int kind) {
+  return mx_bn(kind) == 128 ? (mx_is_nv(kind) ? 5 : 6) : (mx_is_wgrad(kind) ? 3 : 4);
+}
 // Epilogue warps: with one accumulator the MMAs of the next tile wait for the epilogue, so it is
 // split over eight warps (two per TMEM lane quarter, each taking half of the columns); the
 // double-buffered 128 x 128 kind keeps four.
@@ -309,6 +320,7 @@ struct Ctx {  // typed views of ctx + ws for one shape
   uint8_t *xq, *xqs, *hq, *hqs, *dyq, *dyqs, *daq, *daqs, *dbq, *dbqs;  // MXFP8 operands and scales
   uint8_t *xqt, *xqts, *dyqt, *dyqts, *daqt, *daqts, *dbqt, *dbqts, *hgqt, *hgqts;  // MXFP8 weight-gradient operands
   float* nvh;       // NVFP4 forward: fp32 H [RP, I]
+  float* nvdab;     // NVFP4 backward: fp32 dA, then dB [2, RP, I]
   unsigned* nvsc;   // NVFP4 forward: amax(X), amax(H) (fp32 bits), gs_X, gs_H (fp32)
 };
 Ctx make_ctx(const Layout& L, void* ctx, void* ws);
@@ -365,8 +377,12 @@ cudaError_t launch_gather_quant2_range(const Layout& L, const Ctx& c, const __nv
 // otherwise W [El][K][N] to rows el * N + n), gs the device scale(s) of src0 (and src1)
 cudaError_t launch_nv_amax(const __nv_bfloat16* x, int64_t n, unsigned* amax, cudaStream_t st);
 cudaError_t launch_nv_scale(const unsigned* amax, float* gs, int n, cudaStream_t st);
+// (dst: the bf16 rows too, or NULL)
 cudaError_t launch_nv_gather_x(const Layout& L, const Ctx& c, const __nv_bfloat16* X, const float* gs, uint8_t* q,
-                               uint8_t* qs, cudaStream_t st);
+                               uint8_t* qs, __nv_bfloat16* dst, cudaStream_t st);
+// rows of a row-major bf16 [R, K] quantised along K (the backward's weight layouts)
+cudaError_t launch_nv_quant_rows(const __nv_bfloat16* src, int64_t R, int K, const float* gs, uint8_t* q, uint8_t* qs,
+                                 cudaStream_t st);
 cudaError_t launch_nv_quant_h(const Layout& L, const Ctx& c, const float* h, const float* gs, uint8_t* q, uint8_t* qs,
                               cudaStream_t st);
 cudaError_t launch_nv_quant_weight(bool paired, const __nv_bfloat16* src0, const __nv_bfloat16* src1, int El, int K,

@@ -68,12 +68,13 @@ __global__ void k_nv_scale(const unsigned* __restrict__ amax, float* __restrict_
 // One warp per padded row in [*lo, *hi); lane i takes the row's 16-value blocks i, i + 32, ...
 // (32 bytes of bf16 in, 8 bytes of codes out, contiguous across the warp).  Row R takes token
 // row_asg[R] / k; live pad rows get zero codes and scale 0; dead pad rows are skipped (the GEMM
-// reads them but no epilogue stores their rows).
+// reads them but no epilogue stores their rows).  With dst the bf16 row is stored there too
+// (the bf16 weight gradients' operand; live pad rows zero).
 __global__ void __launch_bounds__(256) k_nv_gather_x(const __nv_bfloat16* __restrict__ src,
                                                      const int* __restrict__ row_asg, const int* __restrict__ lo,
                                                      const int* __restrict__ hi, int k, int d,
                                                      const float* __restrict__ gsp, uint8_t* __restrict__ q,
-                                                     uint8_t* __restrict__ qs) {
+                                                     uint8_t* __restrict__ qs, __nv_bfloat16* __restrict__ dst) {
   const int r0 = __ldg(lo), r1 = __ldg(hi);
   const float gs = __ldg(gsp);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -84,14 +85,16 @@ __global__ void __launch_bounds__(256) k_nv_gather_x(const __nv_bfloat16* __rest
     if (a == ROW_DEAD) continue;
     const uint4* in = a >= 0 ? reinterpret_cast<const uint4*>(src + static_cast<size_t>(a / k) * d) : nullptr;
     uint2* qd = reinterpret_cast<uint2*>(q + R * (d / 2));
+    uint4* o = dst ? reinterpret_cast<uint4*>(dst + R * d) : nullptr;
     for (int c = lane; c < nb; c += 32) {
       float v[16];
-      if (in) {
-        unpack8_bf16(__ldg(in + 2 * c), v);
-        unpack8_bf16(__ldg(in + 2 * c + 1), v + 8);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+      const uint4 u0 = in ? __ldg(in + 2 * c) : make_uint4(0, 0, 0, 0);
+      const uint4 u1 = in ? __ldg(in + 2 * c + 1) : make_uint4(0, 0, 0, 0);
+      unpack8_bf16(u0, v);
+      unpack8_bf16(u1, v + 8);
+      if (o) {
+        o[2 * c] = u0;
+        o[2 * c + 1] = u1;
       }
       uint32_t w[2];
       const uint8_t sb = nv_quant16(v, gs, w);
@@ -130,6 +133,29 @@ __global__ void __launch_bounds__(256) k_nv_quant_h(const float* __restrict__ h,
       const uint8_t sb = nv_quant16(v, gs, w);
       qd[c] = make_uint2(w[0], w[1]);
       qs[nv_sf_index(static_cast<int>(R), 16 * c, I)] = sb;
+    }
+  }
+}
+
+// Rows of a row-major bf16 [R, K] quantised along K (no transpose: the backward's weight layouts
+// W_down [El*I, d], W_gate / W_up [El*d, I]); one warp per row, lanes over its 16-value blocks.
+__global__ void __launch_bounds__(256) k_nv_quant_rows(const __nv_bfloat16* __restrict__ src, int64_t R, int K,
+                                                       const float* __restrict__ gsp, uint8_t* __restrict__ q,
+                                                       uint8_t* __restrict__ qs) {
+  const float gs = __ldg(gsp);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nb = K / 16;
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + warp; r < R; r += static_cast<int64_t>(gridDim.x) * 8) {
+    const uint4* in = reinterpret_cast<const uint4*>(src + r * K);
+    uint2* qd = reinterpret_cast<uint2*>(q + r * (K / 2));
+    for (int c = lane; c < nb; c += 32) {
+      float v[16];
+      unpack8_bf16(__ldg(in + 2 * c), v);
+      unpack8_bf16(__ldg(in + 2 * c + 1), v + 8);
+      uint32_t w[2];
+      const uint8_t sb = nv_quant16(v, gs, w);
+      qd[c] = make_uint2(w[0], w[1]);
+      qs[nv_sf_index(static_cast<int>(r), 16 * c, K)] = sb;
     }
   }
 }
@@ -220,8 +246,14 @@ cudaError_t launch_nv_scale(const unsigned* amax, float* gs, int n, cudaStream_t
 }
 
 cudaError_t launch_nv_gather_x(const Layout& L, const Ctx& c, const __nv_bfloat16* X, const float* gs, uint8_t* q,
-                               uint8_t* qs, cudaStream_t st) {
-  k_nv_gather_x<<<nv_grid_rows(L.RP), 256, 0, st>>>(X, c.row_asg, c.poff, c.poff + L.El, L.k, L.d, gs, q, qs);
+                               uint8_t* qs, __nv_bfloat16* dst, cudaStream_t st) {
+  k_nv_gather_x<<<nv_grid_rows(L.RP), 256, 0, st>>>(X, c.row_asg, c.poff, c.poff + L.El, L.k, L.d, gs, q, qs, dst);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_nv_quant_rows(const __nv_bfloat16* src, int64_t R, int K, const float* gs, uint8_t* q, uint8_t* qs,
+                                 cudaStream_t st) {
+  k_nv_quant_rows<<<nv_grid_rows(R), 256, 0, st>>>(src, R, K, gs, q, qs);
   return cudaGetLastError();
 }
 

@@ -11,7 +11,10 @@
   a rounding boundary, so the bf16 tolerance holds; against the exact fp64 layer the error
   is the format's own (reported, bounded loosely);
 * two runs are bit-identical; an expert slice, a hot expert spanning tiles, an empty
-  expert and T = 0 run.
+  expert and T = 0 run;
+* backward: the backward's weight layouts and the dispatched dY bit-exact against the oracle
+  quantiser, dY's scale bit for bit, [dA | dB]'s within 1e-5 (fp32 against fp64 values), dX,
+  dW_r and the (bf16-operand) expert weight gradients within 2e-2 of backward_nv.
 """
 import numpy as np
 import pytest
@@ -46,7 +49,7 @@ def test_nvfp4_prepared_weights_only():
     torch.cuda.synchronize()
     Wg64, Wu64, Wd64 = to64(x["W_gate"]), to64(x["W_up"]), to64(x["W_down"])
     gsw = N.nv_weight_scales(Wg64, Wu64, Wd64)
-    assert [np.float32(v) for v in lay.scales()[1]] == list(gsw)
+    assert [np.float32(v) for v in lay.scales()[1]] == list(gsw) + [N.nv_weight_scales_bwd(Wg64, Wu64, Wd64)[0]]
     reg = lay.weight_regions()
     cg, sg = zip(*[N.nv_quantize(Wg64[e], gsw[0], axis=0) for e in range(E)])
     cu, su = zip(*[N.nv_quantize(Wu64[e], gsw[1], axis=0) for e in range(E)])
@@ -80,7 +83,7 @@ def _check(T, d, E, k, I, seed=0, bias=None, first=0, num=0):
     # global scales, bit for bit
     (gsx, gsh), gsw = lay.scales()
     want_w = N.nv_weight_scales(Wg64, Wu64, Wd64)
-    assert [np.float32(v) for v in gsw] == list(want_w)
+    assert [np.float32(v) for v in gsw[:3]] == list(want_w)
     assert np.float32(gsx) == N.nv_global_scale(f["X"])
 
     # prepared weights, bit for bit
@@ -173,7 +176,7 @@ def test_nvfp4_full_size_ep64_slice():
     # The EP64 per-rank slice at full size, as the bench runs it (epnv_n2368: 32768 tokens routed
     # top-8 over 384 experts, 6 local experts with 2368 rows each, one batch): every token's Y
     # (but the few near-tie tokens, whose fp64 routing differs) against the NVFP4 oracle's full
-    # forward, routing bit-exact on the GPU's logits, the global scales.
+    # forward, routing bit-exact on the GPU's logits, the global scales; then the backward.
     from mixture_experts_layer_27_b200 import inputs as IN
     w = IN.WORKLOADS["epnv_n2368"]
     x = IN.make_inputs(w, device="cuda")
@@ -187,7 +190,7 @@ def test_nvfp4_full_size_ep64_slice():
     f = {n: to64(x[n]) for n in ("X", "W_r", "bias")}
     W64 = [to64(t) for t in (Wg, Wu, Wd)]
     gs_w = N.nv_weight_scales(*W64)
-    assert [np.float32(v) for v in lay.scales()[1]] == list(gs_w)
+    assert [np.float32(v) for v in lay.scales()[1][:3]] == list(gs_w)
     Yq, info = N.forward_nv(f["X"], f["W_r"], f["bias"], W64[0], W64[1], W64[2], w.k, first_local=0,
                             num_local=El, gs_w=gs_w)
     r = lay.routing()
@@ -207,3 +210,92 @@ def test_nvfp4_full_size_ep64_slice():
     assert abs(float(lay.scales()[0][1]) / float(info["gs_h"]) - 1.0) < 1e-5
     err = relerr(to64(Y)[keep], Yq[keep])
     assert err <= TOL_BF16, err
+    # the backward at full size: dX off the near-tie tokens, dW_r and the local experts' weight
+    # gradients against backward_nv
+    g = lay.backward(x["X"], x["W_r"], x["dY"])
+    torch.cuda.synchronize()
+    assert lay.error() == B.MOE_OK
+    dY64 = to64(x["dY"])
+    go = N.backward_nv(info, f["X"], f["W_r"], W64[0], W64[1], W64[2], dY64)
+    assert np.float32(lay.bwd_scales()[0]) == go["gs_dy"]
+    errs = {"dX": relerr(to64(g["dX"])[keep], go["dX"][keep]), "dW_r": relerr(to64(g["dW_r"]), go["dW_r"])}
+    for n in ("dW_gate", "dW_up", "dW_down"):
+        errs[n] = relerr(to64(g[n]), np.stack([go[n][e] for e in range(El)]))
+    assert all(v <= TOL_BF16 for v in errs.values()), errs
+
+
+def test_nvfp4_backward_weights_only():
+    T, d, E, k, I = 64, 256, 4, 2, 512
+    w, x = make_case(T, d, E, k, I, seed=43)
+    lay = B.MoELayerNVFP4(T, d, E, I, k)
+    lay.prepare(x["W_gate"], x["W_up"], x["W_down"])
+    torch.cuda.synchronize()
+    Wg64, Wu64, Wd64 = to64(x["W_gate"]), to64(x["W_up"]), to64(x["W_down"])
+    gs_gu, gs_d = N.nv_weight_scales_bwd(Wg64, Wu64, Wd64)
+    reg = lay.bwd_weight_regions()
+    for name, W, gs in (("Wd3", Wd64, gs_d), ("Wg4", Wg64, gs_gu), ("Wu4", Wu64, gs_gu)):
+        c, sc = zip(*[N.nv_quantize(W[e], gs, axis=1) for e in range(E)])
+        assert np.array_equal(reg[name][0], np.concatenate(c)), name
+        assert np.array_equal(reg[name][1], np.concatenate(sc)), name
+
+
+def _check_bwd(T, d, E, k, I, seed=0, bias=None, first=0, num=0):
+    lay, x, Y, (Wg, Wu, Wd) = _run(T, d, E, k, I, seed, bias, first, num)
+    El = lay.El
+    g = lay.backward(x["X"], x["W_r"], x["dY"])
+    torch.cuda.synchronize()
+    assert lay.error() == B.MOE_OK
+    f = {n: (None if x[n] is None else to64(x[n])) for n in ("X", "W_r", "bias", "dY")}
+    W64 = [to64(t) for t in (x["W_gate"], x["W_up"], x["W_down"])]
+    _, info = N.forward_nv(f["X"], f["W_r"], f["bias"], *W64, k, first_local=first, num_local=El)
+    go = N.backward_nv(info, f["X"], f["W_r"], *W64, f["dY"])
+    gs_dy, gs_ab = lay.bwd_scales()
+    assert np.float32(gs_dy) == go["gs_dy"]
+    assert abs(float(gs_ab) / float(go["gs_ab"]) - 1.0) < 1e-5
+    # dispatched dY codes, bit for bit
+    r = lay.routing()
+    counts, offs = r["counts"].cpu().numpy(), r["offsets"].cpu().numpy()
+    poff, perm = r["padded_offsets"].cpu().numpy(), r["perm"].cpu().numpy()
+    yc, ys = lay.dy_operand()
+    cy, sy = N.nv_quantize(f["dY"], gs_dy, axis=1)
+    for e in range(El):
+        rows = poff[e] + np.arange(counts[e])
+        toks = perm[offs[e]:offs[e + 1]]
+        assert np.array_equal(yc[rows], cy[toks]) and np.array_equal(ys[rows], sy[toks]), e
+    errs = {"dX": relerr(to64(g["dX"]), go["dX"]), "dW_r": relerr(to64(g["dW_r"]), go["dW_r"])}
+    for n in ("dW_gate", "dW_up", "dW_down"):
+        errs[n] = relerr(to64(g[n]), np.stack([go[n][e + first] for e in range(El)]))
+    assert all(v <= TOL_BF16 for v in errs.values()), errs
+    g2 = lay.backward(x["X"], x["W_r"], x["dY"])
+    torch.cuda.synchronize()
+    for n in ("dX", "dW_gate", "dW_up", "dW_down", "dW_r"):
+        assert torch.equal(g[n], g2[n]), n
+    return errs
+
+
+def test_nvfp4_backward_tiny_config():
+    _check_bwd(128, 256, 8, 2, 512, seed=0)
+
+
+def test_nvfp4_backward_hot_expert_and_empty_expert():
+    bias = np.zeros(4, dtype=np.float32)
+    bias[0] = 8.0
+    bias[3] = -40.0
+    _check_bwd(600, 512, 4, 2, 512, bias=bias, seed=42)
+
+
+def test_nvfp4_backward_expert_slice_ragged_tokens():
+    _check_bwd(328, 768, 8, 3, 512, seed=7, first=2, num=4)
+
+
+def test_nvfp4_backward_empty_batch():
+    lay = B.MoELayerNVFP4(0, 256, 4, 512, 2)
+    w, x = make_case(8, 256, 4, 2, 512, seed=1)
+    lay.prepare(x["W_gate"], x["W_up"], x["W_down"])
+    g = {n: torch.full_like(x[n], 1.0) for n in ("W_gate", "W_up", "W_down")}
+    dWr = torch.ones(256, 4, dtype=torch.float32, device="cuda")
+    dX = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    B.check(B.moe_bwd_nvfp4(lay.shape, x["X"][:0], x["W_r"], lay.wq, x["dY"][:0], lay.ctx, dX, g["W_gate"], g["W_up"],
+                            g["W_down"], dWr, lay.ws), "empty")
+    torch.cuda.synchronize()
+    assert not dWr.any() and all(not t.any() for t in g.values())
