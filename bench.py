@@ -788,40 +788,49 @@ def run_moe(args, w: IN.Workload, world: int, rank: int, local: int):
 
 
 # ----------------------------------------------------------------------------
-# NVFP4 layer forward (moe_fwd_nvfp4): a step is one forward over the batch
+# NVFP4 layer (moe_fwd_nvfp4 + moe_bwd_nvfp4): a step is one forward + one backward
 # ----------------------------------------------------------------------------
-METRIC_NV = "MoE layer forward tokens/s and TFLOP/s, NVFP4 (% of B200 FP4 tensor peak)"
-NV_GEMMS = ("gemm_gateup_swiglu_nvfp4", "gemm_down_combw_nvfp4")
+METRIC_NV = METRIC
+NV_GEMMS = ("gemm_gateup_swiglu_nvfp4", "gemm_down_combw_nvfp4", "gemm_dgrad_down_swiglu_bwd_nvfp4",
+            "gemm_dgrad_gateup_nvfp4")
 
 
 def nv_algorithmic(w: IN.Workload) -> tuple:
-    """(bytes, flops) per launch of the NVFP4 forward's kernels: E2M1 codes at 1/2 byte and one
-    E4M3 scale per 16 values (9/16 byte per value), H in fp32 between the two passes."""
+    """(bytes, flops) per step of each kernel of the NVFP4 layer: E2M1 codes at 1/2 byte and one
+    E4M3 scale per 16 values (9/16 byte per value); H, dA and dB in fp32 between the two passes
+    of their quantisation; the router, combine, reverse dispatch and bf16 weight gradients as
+    in the bf16 layer."""
     T, d, E, I, k, El = w.tokens, w.d, w.E, w.I, w.k, w.El
     rows = local_rows(w)
     Tg = min(T, rows)
     q = 9 / 16
     W = El * d * I * q  # one weight tensor in NVFP4
-    by = {"nvfp4_amax_scale": T * d * 2, "dispatch": Tg * d * 2 + rows * d * q,
-          "gemm_gateup_swiglu_nvfp4": 2 * W + rows * d * q + rows * I * 4,
-          "nvfp4_quantize_h": rows * I * 4 + rows * I * q,
-          "gemm_down_combw_nvfp4": W + rows * I * q + rows * d * 2,
-          "combine": rows * d * 2 + T * d * 2,
-          "router_logits": T * d * 2 + d * E * 2 + T * E * 4}
-    fl = {"gemm_gateup_swiglu_nvfp4": 4 * d * I * rows, "gemm_down_combw_nvfp4": 2 * d * I * rows,
-          "router_logits": 2 * T * d * E}
+    by = algorithmic_bytes(w)
+    fl = algorithmic_flops(w)
+    by.update({"nvfp4_amax_scale": 2 * T * d * 2,  # X, then dY
+               "dispatch": Tg * d * 2 + rows * d * (q + 2),  # codes and the bf16 rows
+               "reverse_combine": Tg * d * 2 + rows * d * (q + 2),
+               "gemm_gateup_swiglu_nvfp4": 2 * W + rows * d * q + rows * I * (4 + 2 * 2),  # H fp32, A, B bf16
+               "nvfp4_quantize_h": rows * I * 4 + rows * I * q,
+               "gemm_down_combw_nvfp4": W + rows * I * q + rows * d * 2,
+               # dY codes, W_down, A and B in; dA, dB, Hg in bf16, dA and dB in fp32 and dg partials out
+               "gemm_dgrad_down_swiglu_bwd_nvfp4": W + rows * d * q + rows * I * (2 * 2 + 3 * 2 + 2 * 4)
+               + rows * (I // 128) * 4,
+               "nvfp4_quantize_da_db": 2 * rows * I * (4 + q),
+               "gemm_dgrad_gateup_nvfp4": 2 * W + 2 * rows * I * q + rows * d * 2})
+    fl.update({"gemm_gateup_swiglu_nvfp4": 4 * d * I * rows, "gemm_down_combw_nvfp4": 2 * d * I * rows,
+               "gemm_dgrad_down_swiglu_bwd_nvfp4": 2 * d * I * rows, "gemm_dgrad_gateup_nvfp4": 4 * d * I * rows})
     return by, fl
 
 
 def nv_config(w: IN.Workload) -> dict:
-    cfg = dict(workload_config(w), precision="nvfp4")
-    cfg["pass"] = "forward"
-    cfg["workload"] = cfg["workload"].replace(" bf16,", " nvfp4 forward,")
+    cfg = dict(workload_config(w), precision="nvfp4", wgrad_dtype="bf16", wgrad_gemms="bf16")
+    cfg["workload"] = cfg["workload"].replace(" bf16,", " nvfp4,")
     return cfg
 
 
 def nv_oracle_rate(w: IN.Workload, x_cpu: dict, steps: int) -> dict:
-    """The NVFP4 oracle forward on the sampled expert window (all tokens routed), timed."""
+    """The NVFP4 oracle forward + backward on the sampled expert window (all tokens routed), timed."""
     import numpy as np
     import oracle.nvfp4 as N
 
@@ -829,26 +838,30 @@ def nv_oracle_rate(w: IN.Workload, x_cpu: dict, steps: int) -> dict:
         return t.float().numpy().astype(np.float64)
 
     e0, m = x_cpu["window"]
-    X, Wr = f64(x_cpu["X"]), f64(x_cpu["W_r"])
+    X, Wr, dY = f64(x_cpu["X"]), f64(x_cpu["W_r"]), f64(x_cpu["dY"])
     b = None if x_cpu["bias"] is None else f64(x_cpu["bias"])
     Wg, Wu, Wd = (f64(x_cpu[n]) for n in ("W_gate", "W_up", "W_down"))
     first = w.first_local + e0
     gs_w = N.nv_weight_scales(Wg, Wu, Wd)  # over the window's experts
+    gs_b = N.nv_weight_scales_bwd(Wg, Wu, Wd)
     # weights rounded once, outside the timed step (the GPU path prepares them once per optimiser step)
     lay = {first + e: N.nv_weight_layouts(Wg[e], Wu[e], Wd[e], gs_w) for e in range(m)}
+    lay_b = {first + e: N.nv_weight_layouts_bwd(Wg[e], Wu[e], Wd[e], gs_b) for e in range(m)}
+    cg, cu, cd = (lambda e: Wg[e - first]), (lambda e: Wu[e - first]), (lambda e: Wd[e - first])
 
     def one():
         t0 = time.perf_counter()
-        _, info = N.forward_nv(X, Wr, b, lambda e: Wg[e - first], lambda e: Wu[e - first], lambda e: Wd[e - first],
-                               w.k, first_local=first, num_local=m, gs_w=gs_w, rounded=lay.__getitem__)
+        _, info = N.forward_nv(X, Wr, b, cg, cu, cd, w.k, first_local=first, num_local=m, gs_w=gs_w,
+                               rounded=lay.__getitem__)
+        N.backward_nv(info, X, Wr, cg, cu, cd, dY, gs_bwd=gs_b, rounded=lay_b.__getitem__)
         return time.perf_counter() - t0, int(info["sched"]["offsets"][-1])
 
     one()  # imports, BLAS start-up
     ts, asg = zip(*[one() for _ in range(steps)])
     med = statistics.median(ts)
     return {"value": asg[0] / w.k / med, "seconds": list(ts),
-            "sample": (f"fp64 numpy NVFP4 oracle forward, measured: each step routes all {w.tokens} tokens and "
-                       f"runs the forward of local experts {e0}..{e0 + m - 1} ({asg[0]} assignments; weights "
+            "sample": (f"fp64 numpy NVFP4 oracle, measured: each step routes all {w.tokens} tokens and "
+                       f"runs forward + backward of local experts {e0}..{e0 + m - 1} ({asg[0]} assignments; weights "
                        f"rounded once outside the step, global scales over the window); rate = assignments / "
                        f"top_k / the median of {steps} steps ({med:.2f} s)")}
 
@@ -865,6 +878,9 @@ def run_nvfp4(args, w: IN.Workload, world: int, rank: int, local: int):
     Wg, Wu, Wd = (x[n][w.first_local:w.first_local + El].contiguous() for n in ("W_gate", "W_up", "W_down"))
     NT = w.tokens
     Y = torch.empty(NT, w.d, dtype=torch.bfloat16, device=dev)
+    grads = dict(dX=torch.empty(NT, w.d, dtype=torch.bfloat16, device=dev), dW_gate=torch.empty_like(Wg),
+                 dW_up=torch.empty_like(Wu), dW_down=torch.empty_like(Wd),
+                 dW_r=torch.empty(w.d, w.E, dtype=torch.float32, device=dev))
     stream = torch.cuda.current_stream(dev)
     fp8_peak = measure_mxfp8_peak(dev)
     layer.prepare(Wg, Wu, Wd)
@@ -875,11 +891,12 @@ def run_nvfp4(args, w: IN.Workload, world: int, rank: int, local: int):
     torch.cuda.synchronize()
     prep_ms = pa.elapsed_time(pb)
 
-    def step(X, Yout):
+    def step(X, dY, Yout, g):
         layer.forward(X, x["W_r"], x["bias"], Y=Yout)
+        layer.backward(X, x["W_r"], dY, out=g)
 
     for _ in range(args.warmup):
-        step(x["X"], Y)
+        step(x["X"], x["dY"], Y, grads)
     torch.cuda.synchronize()
     if layer.error() != B.MOE_OK:
         raise RuntimeError("device error during warm-up")
@@ -892,7 +909,7 @@ def run_nvfp4(args, w: IN.Workload, world: int, rank: int, local: int):
     for _ in range(args.steps):
         if flush is not None:
             flush.fill_(1)
-        step(x["X"], Y)
+        step(x["X"], x["dY"], Y, grads)
     torch.cuda.synchronize()
     launches_per_step = (B.moe_kernel_launches() - launches0) // args.steps
     B.moe_profile_enable(False)
@@ -904,12 +921,12 @@ def run_nvfp4(args, w: IN.Workload, world: int, rank: int, local: int):
             side = torch.cuda.Stream(dev)
             side.wait_stream(stream)
             with torch.cuda.stream(side):
-                step(x["X"], Y)
+                step(x["X"], x["dY"], Y, grads)
             stream.wait_stream(side)
             torch.cuda.synchronize()
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph):
-                step(x["X"], Y)
+                step(x["X"], x["dY"], Y, grads)
             torch.cuda.synchronize()
         except Exception as ex:
             graph, launch_mode = None, f"direct (graph capture failed: {type(ex).__name__})"
@@ -920,7 +937,7 @@ def run_nvfp4(args, w: IN.Workload, world: int, rank: int, local: int):
         if graph is not None:
             graph.replay()
         else:
-            step(x["X"], Y)
+            step(x["X"], x["dY"], Y, grads)
 
     for _ in range(2):
         run_step()
@@ -944,18 +961,23 @@ def run_nvfp4(args, w: IN.Workload, world: int, rank: int, local: int):
         raise RuntimeError("device error in the timed region")
     t = max_over_ranks(t_local, world)
 
-    # end to end: X in from pinned host memory, Y out, every step (in line on the compute stream)
+    # end to end: X, dY in from pinned host memory, Y, dX out, every step (in line on the compute stream)
     hX = torch.empty(NT, w.d, dtype=torch.bfloat16, pin_memory=True)
+    hdY = torch.empty_like(hX, pin_memory=True)
     hY = torch.empty_like(hX, pin_memory=True)
+    hdX = torch.empty_like(hX, pin_memory=True)
     hX.copy_(x["X"].cpu())
-    Xd = torch.empty_like(x["X"])
+    hdY.copy_(x["dY"].cpu())
+    Xd, dYd = torch.empty_like(x["X"]), torch.empty_like(x["dY"])
     e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     e2.record(stream)
     for _ in range(args.steps):
         Xd.copy_(hX, non_blocking=True)
-        step(Xd, Y)
+        dYd.copy_(hdY, non_blocking=True)
+        step(Xd, dYd, Y, grads)
         hY.copy_(Y, non_blocking=True)
+        hdX.copy_(grads["dX"], non_blocking=True)
     e3.record(stream)
     torch.cuda.synchronize()
     t_e2e = max_over_ranks(e2.elapsed_time(e3) / 1e3, world)
@@ -995,20 +1017,21 @@ def run_nvfp4(args, w: IN.Workload, world: int, rank: int, local: int):
                 "frac": (ach / hbm) if ach else None, "traffic": ncu_traffic(top, w.name),
                 "peak_source": f"{peak_kind} HBM copy bandwidth" if peak_kind == "measured"
                 else "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"}
-    tflops = w.forward_flops() * args.steps * world / t / 1e12
+    tflops = w.model_flops() * args.steps * world / t / 1e12
     line = {
         "metric": METRIC_NV, "value": job_throughput(NT * args.steps, t, world), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "nvfp4 (e2m1 + e4m3 per 16 + fp32 per tensor)", "data": "synthetic (seeded, random-init weights)",
+        "dtype": "nvfp4 (e2m1 + e4m3 per 16 + fp32 per tensor) / bf16 wgrad", "data": "synthetic (seeded, random-init weights)",
         "config": nv_config(w),
         "tflops": tflops, "pct_of_fp4_peak": 100.0 * tflops / world / fp4, "fp4_peak_tflops": fp4,
-        "peak_note": "forward model FLOPs 6 d I per assignment + 2 T d E; fp4 peak = " + fp4_src,
+        "peak_note": ("model FLOPs 18 d I per assignment + 6 T d E per step; the four expert dgrad / forward "
+                      "GEMMs on NVFP4, the weight gradients and the router on bf16; fp4 peak = " + fp4_src),
         "roofline": roof,
         "e2e": {"value": job_throughput(NT * args.steps, t_e2e, world), "unit": "tokens/s",
-                "h2d_bytes_per_step": NT * w.d * 2, "d2h_bytes_per_step": NT * w.d * 2,
-                "note": "X copied in from pinned host memory and Y copied back every step, in line on the "
-                        "compute stream; prepared weights stay in HBM"},
+                "h2d_bytes_per_step": 2 * NT * w.d * 2, "d2h_bytes_per_step": 2 * NT * w.d * 2,
+                "note": "X, dY copied in from pinned host memory and Y, dX copied back every step, in line on "
+                        "the compute stream; prepared weights and the weight gradients stay in HBM"},
         "gpu_launches": int(launches_per_step * args.steps), "launch": launch_mode, "clocks": clk,
         "prepare_weights_ms": prep_ms, "mxfp8_peak": fp8_peak, "kernels": kern,
     }

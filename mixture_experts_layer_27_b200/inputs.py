@@ -47,7 +47,7 @@ class Workload:
     stream_M: int = 0           # > 0: M minibatches of T tokens through a ring of ring_bytes
     ring_bytes: int = 0
     local_tokens: int = 0       # streamed slice: assignments each local expert receives over the stream
-    nvfp4: bool = False         # NVFP4 layer forward (no NVFP4 backward exists)
+    nvfp4: bool = False         # NVFP4 layer (moe_fwd_nvfp4 / moe_bwd_nvfp4)
 
     @property
     def El(self) -> int:
@@ -107,7 +107,7 @@ for _n in (512, 2368, 4096, 8192):
 # epmx_n2368's expert work (6 local experts x 2368 rows, MXFP8) over 8192 tokens and 96 experts: the
 # same dispatched rows and GEMM tiles with a padded-row capacity (and workspace) a quarter of the
 # size, for profiler captures (a few GB on the device)
-# NVFP4 layer forward: the dsv3 and kimi configurations, the EP64 slice as one batch (where the
+# NVFP4 layer (forward and backward, bf16 weight gradients): the dsv3 and kimi configurations, the EP64 slice as one batch (where the
 # grouped GEMMs are tensor-bound), and two few-GB cases for profiler captures
 WORKLOADS["dsv3_nv"] = Workload("dsv3_nv", 2048, 7168, 256, 8, 2048, nvfp4=True)
 WORKLOADS["kimi_nv"] = Workload("kimi_nv", 4096, 7168, 384, 8, 2048, zipf=True, nvfp4=True)

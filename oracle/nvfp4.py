@@ -201,7 +201,14 @@ def nv_weight_scales_bwd(W_gate, W_up, W_down, first_local: int = 0, num_local: 
     return np.float32(min(g, u)), d
 
 
-def backward_nv(info, X, W_r, W_gate, W_up, W_down, dY, gs_bwd=None):
+def nv_weight_layouts_bwd(Wg, Wu, Wd, gs_bwd) -> dict:
+    """One expert's weights rounded for the backward's dgrad GEMMs (fp64): gate and up along I
+    under the joint [gate | up] scale, down along d."""
+    return dict(gate_i=nv_round(_f64(Wg), gs_bwd[0], axis=1), up_i=nv_round(_f64(Wu), gs_bwd[0], axis=1),
+                down_d=nv_round(_f64(Wd), gs_bwd[1], axis=1))
+
+
+def backward_nv(info, X, W_r, W_gate, W_up, W_down, dY, gs_bwd=None, rounded=None):
     """NVFP4 layer backward after forward_nv (its info): the dgrad GEMMs on NVFP4 operands,
     the weight gradients from the unrounded operands (as the MXFP8 layer with bf16 weight
     gradients does).
@@ -210,7 +217,8 @@ def backward_nv(info, X, W_r, W_gate, W_up, W_down, dY, gs_bwd=None):
     dgrad of gate/up (K = 2I): [dA | dB] rows along I under one scale over every assigned row's
     dA and dB, [W_gate | W_up] along I under one scale (nv_weight_scales_bwd).
     A and B are read as bf16 (the layer keeps them in bf16), H = silu(A) B recomputed from them.
-    gs_bwd: optional (gs_gate_up, gs_down) computed once by the caller."""
+    gs_bwd: optional (gs_gate_up, gs_down) computed once by the caller; rounded: optional
+    callable e -> nv_weight_layouts_bwd of expert e under gs_bwd (the same values, computed once)."""
     from .moe_oracle import bf16_round, silu_grad
     X64, dY64 = _f64(X), _f64(dY)
     ids, g, sched = info["ids"], info["g"], info["sched"]
@@ -236,7 +244,8 @@ def backward_nv(info, X, W_r, W_gate, W_up, W_down, dY, gs_bwd=None):
         ge = g[toks, slots]
         dYe = dY64[toks]
         H = silu(A) * B
-        dHp = nv_round(dYe, gs_dy, axis=1) @ nv_round(_expert(W_down, e), gs_d, axis=1).T  # K = d
+        Wdq = rounded(e)["down_d"] if rounded is not None else nv_round(_expert(W_down, e), gs_d, axis=1)
+        dHp = nv_round(dYe, gs_dy, axis=1) @ Wdq.T  # K = d
         dg[toks, slots] = np.sum(dHp * H, axis=1)
         dH = ge[:, None] * dHp
         dA = dH * B * silu_grad(A)
@@ -249,8 +258,12 @@ def backward_nv(info, X, W_r, W_gate, W_up, W_down, dY, gs_bwd=None):
     live = [np.abs(p[2]).max() for p in parts] + [np.abs(p[3]).max() for p in parts]
     gs_ab = nv_global_scale(np.array(live)) if live else np.float32(1.0)
     for e, toks, dA, dB in parts:  # K = I
-        dX[toks] += (nv_round(dA, gs_ab, axis=1) @ nv_round(_expert(W_gate, e), gs_gu, axis=1).T
-                     + nv_round(dB, gs_ab, axis=1) @ nv_round(_expert(W_up, e), gs_gu, axis=1).T)
+        if rounded is not None:
+            Wgq, Wuq = rounded(e)["gate_i"], rounded(e)["up_i"]
+        else:
+            Wgq = nv_round(_expert(W_gate, e), gs_gu, axis=1)
+            Wuq = nv_round(_expert(W_up, e), gs_gu, axis=1)
+        dX[toks] += nv_round(dA, gs_ab, axis=1) @ Wgq.T + nv_round(dB, gs_ab, axis=1) @ Wuq.T
     dl = np.zeros((T, E))
     s = np.sum(g * dg, axis=1, keepdims=True)
     np.put_along_axis(dl, ids.astype(np.int64), g * (dg - s), axis=1)

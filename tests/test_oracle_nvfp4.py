@@ -300,3 +300,20 @@ def test_backward_w_gate_up_rounded_along_i(which):
     g1 = N.backward_nv(info, X, W_r, W2 if which == "gate" else Wg, W2 if which == "up" else Wu, Wd, dY)
     assert not np.array_equal(g1["dX"][:, 19], g0["dX"][:, 19])
     np.testing.assert_array_equal(np.delete(g1["dX"], 19, axis=1), np.delete(g0["dX"], 19, axis=1))
+
+
+def test_weight_layout_caches_give_the_same_layer():
+    # the bench's CPU baseline rounds the weights once (nv_weight_layouts, nv_weight_layouts_bwd);
+    # the layer through those caches equals the layer rounding them inline
+    X, W_r, bias, Wg, Wu, Wd, k, dY = _bwd_case(25)
+    gs_w = N.nv_weight_scales(Wg, Wu, Wd)
+    gs_b = N.nv_weight_scales_bwd(Wg, Wu, Wd)
+    fw = {e: N.nv_weight_layouts(Wg[e], Wu[e], Wd[e], gs_w) for e in range(4)}
+    bw = {e: N.nv_weight_layouts_bwd(Wg[e], Wu[e], Wd[e], gs_b) for e in range(4)}
+    Y0, i0 = N.forward_nv(X, W_r, bias, Wg, Wu, Wd, k)
+    Y1, i1 = N.forward_nv(X, W_r, bias, Wg, Wu, Wd, k, gs_w=gs_w, rounded=fw.__getitem__)
+    np.testing.assert_array_equal(Y0, Y1)
+    g0 = N.backward_nv(i0, X, W_r, Wg, Wu, Wd, dY)
+    g1 = N.backward_nv(i1, X, W_r, Wg, Wu, Wd, dY, gs_bwd=gs_b, rounded=bw.__getitem__)
+    for n in ("dX", "dW_r"):
+        np.testing.assert_array_equal(g0[n], g1[n])
