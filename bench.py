@@ -1011,6 +1011,13 @@ def run_nvfp4(args, w: IN.Workload, world: int, rank: int, local: int):
         ach = kern[top]["achieved_TFLOPs"]
         roof = {"kernel": top, "bound": "tensor", "achieved": ach, "peak": fp4, "unit": "TFLOP/s",
                 "frac": ach / fp4, "traffic": ncu_traffic(top, w.name), "peak_source": fp4_src}
+    elif kern[top]["bound"] == "tensor":  # a bf16 GEMM (the weight gradients, the router)
+        bf16 = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        ach = kern[top]["achieved_TFLOPs"]
+        roof = {"kernel": top, "bound": "tensor", "achieved": ach, "peak": bf16, "unit": "TFLOP/s",
+                "frac": ach / bf16, "traffic": ncu_traffic(top, w.name),
+                "peak_source": "measured sustained bf16 GEMM (MEASURED_PEAKS.json bf16_tflops_sustained)"
+                if peak_kind == "measured" else "fallback 1.4 PFLOP/s sustained bf16 (no MEASURED_PEAKS.json)"}
     else:
         ach = kern[top].get("achieved_GBs")
         roof = {"kernel": top, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
