@@ -23,7 +23,7 @@ MOE_ERR_EXCHANGE = 7
 MOE_BF16 = 0
 MOE_MXFP8 = 1
 MOE_MXFP8_ALL = 2  # MOE_MXFP8 with the weight-gradient GEMMs on MXFP8 too (operands along tokens)
-MOE_NVFP4 = 3  # forward only: E2M1 operands, E4M3 scale per 16 along K, fp32 scale per tensor
+MOE_NVFP4 = 3  # E2M1 operands, E4M3 scale per 16 along K, fp32 scale per tensor (bf16 weight gradients)
 MOE_WGRAD_BF16 = 0
 MOE_WGRAD_FP32 = 1
 

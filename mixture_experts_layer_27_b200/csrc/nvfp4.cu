@@ -1,4 +1,4 @@
-// NVFP4 quantisation for the NVFP4 layer forward (page 1 of the MoK pages,
+// NVFP4 quantisation for the NVFP4 layer (page 1 of the MoK pages,
 // "MoE layer as the bottleneck", names NVFP4 training kernels as earlier work;
 // the format is NVIDIA's published one): E2M1 codes, one E4M3 scale per 16
 // values along a GEMM's contraction dimension and one fp32 scale per tensor,
@@ -11,7 +11,9 @@
 // Every tensor needs its amax before any of its blocks can be quantised, so
 // each operand takes two passes: an amax reduction (max is order-free, so the
 // atomicMax result is the same every run), then the quantisation.  For H the
-// first pass is the gate/up GEMM's own epilogue, which writes H in fp32.
+// first pass is the gate/up GEMM's own epilogue, which writes H in fp32; for dA
+// and dB (one tensor, the dgrad of gate/up's K = 2I operand) it is the dgrad of
+// W_down's epilogue.
 #include <cfloat>
 
 #include "moe_internal.cuh"

@@ -1,4 +1,4 @@
-"""Oracle of the NVFP4 layer forward (test infrastructure only).
+"""Oracle of the NVFP4 layer, forward and backward (test infrastructure only).
 
 TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import this module:
 only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg

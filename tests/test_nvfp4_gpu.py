@@ -1,4 +1,4 @@
-"""NVFP4 layer forward on the GPU, against the NVFP4 oracle (oracle/nvfp4.py).
+"""NVFP4 layer forward and backward on the GPU, against the NVFP4 oracle (oracle/nvfp4.py).
 
 * global scales: the three weight scales and X's equal the oracle's bit for bit (both
   compute 2688 / amax in fp32 on the same bf16 values);
@@ -122,7 +122,7 @@ def _check(T, d, E, k, I, seed=0, bias=None, first=0, num=0):
 
     # H: the device's codes are the oracle's quantiser on the device's fp32 H and scale
     if live.size:
-        H = lay.h_fp32().astype(np.float64)[live]
+        H = lay.h_fp32()[live].astype(np.float64)  # live rows only: dead pad rows hold stale bytes
         assert np.float32(gsh) == N.nv_global_scale(H)
         hc, hs = lay.h_operand()
         qc, qs = N.nv_quantize(H, gsh, axis=1)
