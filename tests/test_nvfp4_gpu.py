@@ -299,3 +299,34 @@ def test_nvfp4_backward_empty_batch():
                             g["W_down"], dWr, lay.ws), "empty")
     torch.cuda.synchronize()
     assert not dWr.any() and all(not t.any() for t in g.values())
+
+
+def test_nvfp4_step_replays_from_a_cuda_graph():
+    # the layer only enqueues work (no host sync, no allocation): one fwd+bwd step captured as a
+    # CUDA graph and replayed gives the direct launches' results bit for bit
+    lay, x, Y, _ = _run(256, 512, 8, 2, 512, seed=5)
+    g = lay.backward(x["X"], x["W_r"], x["dY"])
+    torch.cuda.synchronize()
+    ref = {"Y": Y.clone(), **{n: t.clone() for n, t in g.items()}}
+    Y2 = torch.empty_like(Y)
+    g2 = {n: torch.empty_like(t) for n, t in g.items()}
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm the capture stream
+        lay.forward(x["X"], x["W_r"], x["bias"], Y=Y2)
+        lay.backward(x["X"], x["W_r"], x["dY"], out=g2)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        lay.forward(x["X"], x["W_r"], x["bias"], Y=Y2)
+        lay.backward(x["X"], x["W_r"], x["dY"], out=g2)
+    Y2.zero_()
+    for t in g2.values():
+        t.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert lay.error() == B.MOE_OK
+    assert torch.equal(Y2, ref["Y"])
+    for n in g2:
+        assert torch.equal(g2[n], ref[n]), n
