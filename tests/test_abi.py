@@ -187,6 +187,38 @@ def test_mxfp8_sizes_and_argument_errors(lib):
     assert r == B.MOE_ERR_INVALID_ARG  # dY missing
 
 
+def test_nvfp4_sizes_and_argument_errors(lib):
+    nv = B.make_shape(256, 256, 8, 512, 2, prec=B.MOE_NVFP4)
+    mx = B.make_shape(256, 256, 8, 512, 2, prec=B.MOE_MXFP8)
+    bf = B.make_shape(256, 256, 8, 512, 2)
+    nq = B.moe_weights_size(nv)
+    # five prepared regions at half a byte per value and one scale byte per 16 values
+    assert nq >= 6 * 8 * 256 * 512 * 9 // 16 and nq < B.moe_weights_size(mx)
+    nc, nw = B.moe_ctx_size(nv), B.moe_workspace_size(nv)
+    assert nc > 0 and nw > B.moe_workspace_size(bf)  # fp32 H, dA, dB and the codes
+    offs = B.moe_debug_nv_offsets(nv)
+    assert len(offs) == 23 and all(o % 256 == 0 for o in offs)
+    assert max(offs[0:2]) < nc and max(offs[2:6] + offs[11:17]) < nw and max(offs[6:11] + offs[17:23]) < nq
+    with pytest.raises(B.MoeError):
+        B.moe_debug_nv_offsets(mx)
+    f = 1 << 20  # never dereferenced: every check below comes before any launch
+    by = ctypes.byref
+    assert lib.moe_prepare_weights(by(nv), f, f, None, f, nq, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_prepare_weights(by(nv), f, f, f, f, nq - 1, None) == B.MOE_ERR_WORKSPACE_TOO_SMALL
+    # the NVFP4 entry points refuse other precisions, and the MXFP8 / bf16 ones an NVFP4 shape
+    for other in (bf, mx):
+        assert lib.moe_fwd_nvfp4(by(other), f, f, None, f, nq, f, f, nc, f, nw, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_fwd_mx(by(nv), f, f, None, f, nq, f, f, nc, f, nw, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_fwd(by(nv), f, f, None, f, f, f, f, f, nc, f, nw, None) != B.MOE_OK
+    assert lib.moe_fwd_nvfp4(by(nv), f, f, None, f, nq - 1, f, f, nc, f, nw, None) == B.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert lib.moe_fwd_nvfp4(by(nv), f, f, None, f, nq, f, f, nc, f, nw - 1, None) == B.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert lib.moe_fwd_nvfp4(by(nv), f + 8, f, None, f, nq, f, f, nc, f, nw, None) == B.MOE_ERR_INVALID_ARG
+    r = lib.moe_bwd_nvfp4(by(nv), f, f, f, nq, None, f, nc, f, f, f, f, f, f, nw, None)
+    assert r == B.MOE_ERR_INVALID_ARG  # dY missing
+    r = lib.moe_bwd_nvfp4(by(nv), f, f, f, nq, f, f, nc - 1, f, f, f, f, f, f, nw, None)
+    assert r == B.MOE_ERR_WORKSPACE_TOO_SMALL
+
+
 def test_expert_parallel_sizes_and_argument_errors(lib):
     s = B.make_shape(64, 256, 8, 256, 2)
     assert B.moe_ep_buffer_size(s, 3) == 0 and B.moe_ep_ctx_size(s, 3) == 0  # E not a multiple of R
