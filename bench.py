@@ -813,10 +813,11 @@ def nv_algorithmic(w: IN.Workload) -> tuple:
                "gemm_gateup_swiglu_nvfp4": 2 * W + rows * d * q + rows * I * (4 + 2 * 2),  # H fp32, A, B bf16
                "nvfp4_quantize_h": rows * I * 4 + rows * I * q,
                "gemm_down_combw_nvfp4": W + rows * I * q + rows * d * 2,
-               # dY codes, W_down, A and B in; dA, dB, Hg in bf16, dA and dB in fp32 and dg partials out
-               "gemm_dgrad_down_swiglu_bwd_nvfp4": W + rows * d * q + rows * I * (2 * 2 + 3 * 2 + 2 * 4)
+               # dY codes, W_down, A and B in; Hg in bf16, dA and dB in fp32 and dg partials out
+               "gemm_dgrad_down_swiglu_bwd_nvfp4": W + rows * d * q + rows * I * (2 * 2 + 2 + 2 * 4)
                + rows * (I // 128) * 4,
-               "nvfp4_quantize_da_db": 2 * rows * I * (4 + q),
+               # dA, dB in fp32 in; their codes and their bf16 copies (the weight gradients' operands) out
+               "nvfp4_quantize_da_db": 2 * rows * I * (4 + q + 2),
                "gemm_dgrad_gateup_nvfp4": 2 * W + 2 * rows * I * q + rows * d * 2})
     fl.update({"gemm_gateup_swiglu_nvfp4": 4 * d * I * rows, "gemm_down_combw_nvfp4": 2 * d * I * rows,
                "gemm_dgrad_down_swiglu_bwd_nvfp4": 2 * d * I * rows, "gemm_dgrad_gateup_nvfp4": 4 * d * I * rows})

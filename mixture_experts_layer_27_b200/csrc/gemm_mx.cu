@@ -356,8 +356,9 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
     }
   } else if constexpr (KIND == NV_DGRAD_DOWN) {
     // dH' = acc / (gs_dY gs_down); the SwiGLU backward from the saved bf16 A, B as in
-    // MX_DGRAD_DOWN; bf16 dA, dB, Hg for the bf16 weight gradients, fp32 dA, dB for their NVFP4
-    // quantisation and the largest |dA|, |dB| of the warp's live rows into *amax
+    // MX_DGRAD_DOWN; bf16 Hg for the bf16 weight gradient of W_down, fp32 dA, dB for their NVFP4
+    // quantisation (which also writes their bf16 copies; out0 / out1 NULL) and the largest
+    // |dA|, |dB| of the warp's live rows into *amax
     const float al = __frcp_rn(__fmul_rn(__ldg(p.gsa), __ldg(p.gsb)));
     const float g = p.row_gate[R];
     float dg = 0.f, amx = 0.f;
@@ -387,8 +388,10 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const MxTile& tl,
         amx = fmaxf(amx, fmaxf(fabsf(a[i]), fabsf(b[i])));
       }
       if (live) {
-        mx_store_bf16_32(p.out0 + Rz * p.I + col, a);
-        mx_store_bf16_32(p.out1 + Rz * p.I + col, b);
+        if (p.out0) {
+          mx_store_bf16_32(p.out0 + Rz * p.I + col, a);
+          mx_store_bf16_32(p.out1 + Rz * p.I + col, b);
+        }
         mx_store_bf16_32(p.out2 + Rz * p.I + col, dh);
         float4* fa = reinterpret_cast<float4*>(p.hout + Rz * p.I + col);
         float4* fb = reinterpret_cast<float4*>(p.hout2 + Rz * p.I + col);

@@ -1577,7 +1577,7 @@ moe_status moe_fwd_nvfp4(const moe_shape* s, const void* X, const void* W_r, con
   }
   MOE_TRY(timed(K_NV_QUANT_H, st, [&] {
     const cudaError_t e = launch_nv_scale(amx + 1, gsv + 1, 1, st);
-    return e != cudaSuccess ? e : launch_nv_quant_h(L, c, c.nvh, gsv + 1, c.hq, c.hqs, st);
+    return e != cudaSuccess ? e : launch_nv_quant_h(L, c, c.nvh, gsv + 1, c.hq, c.hqs, nullptr, st);
   }));
   {
     MxParams p = mx_params(L, c, status);
@@ -1641,9 +1641,7 @@ moe_status moe_bwd_nvfp4(const moe_shape* s, const void* X, const void* W_r, con
     p.sfb0 = p.sfb1 = w + L.wd3s;
     p.in0 = c.abuf;
     p.in1 = c.bbuf;
-    p.out0 = c.dabuf;
-    p.out1 = c.dbbuf;
-    p.out2 = c.hgbuf;
+    p.out2 = c.hgbuf;  // dA, dB reach bf16 through their quantiser below
     p.hout = c.nvdab;
     p.hout2 = c.nvdab + RP * L.I;
     p.amax = amx + 1;
@@ -1658,8 +1656,8 @@ moe_status moe_bwd_nvfp4(const moe_shape* s, const void* X, const void* W_r, con
   }));
   MOE_TRY(timed(K_NV_QUANT_DAB, st, [&] {
     cudaError_t e = launch_nv_scale(amx + 1, gsv + 1, 1, st);
-    if (e == cudaSuccess) e = launch_nv_quant_h(L, c, c.nvdab, gsv + 1, c.daq, c.daqs, st);
-    if (e == cudaSuccess) e = launch_nv_quant_h(L, c, c.nvdab + RP * L.I, gsv + 1, c.dbq, c.dbqs, st);
+    if (e == cudaSuccess) e = launch_nv_quant_h(L, c, c.nvdab, gsv + 1, c.daq, c.daqs, c.dabuf, st);
+    if (e == cudaSuccess) e = launch_nv_quant_h(L, c, c.nvdab + RP * L.I, gsv + 1, c.dbq, c.dbqs, c.dbbuf, st);
     return e;
   }));
   {

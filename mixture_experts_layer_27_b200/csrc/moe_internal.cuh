@@ -384,7 +384,7 @@ cudaError_t launch_nv_gather_x(const Layout& L, const Ctx& c, const __nv_bfloat1
 cudaError_t launch_nv_quant_rows(const __nv_bfloat16* src, int64_t R, int K, const float* gs, uint8_t* q, uint8_t* qs,
                                  cudaStream_t st);
 cudaError_t launch_nv_quant_h(const Layout& L, const Ctx& c, const float* h, const float* gs, uint8_t* q, uint8_t* qs,
-                              cudaStream_t st);
+                              __nv_bfloat16* dst, cudaStream_t st);  // dst: the rows in bf16 too, or NULL
 cudaError_t launch_nv_quant_weight(bool paired, const __nv_bfloat16* src0, const __nv_bfloat16* src1, int El, int K,
                                    int N, const float* gs, uint8_t* q, uint8_t* qs, cudaStream_t st);
 cudaError_t launch_transpose_wr(const Layout& L, const __nv_bfloat16* W_r, __nv_bfloat16* W_rT, cudaStream_t st);

@@ -107,11 +107,12 @@ __global__ void __launch_bounds__(256) k_nv_gather_x(const __nv_bfloat16* __rest
 }
 
 // H (fp32 [RP, I], written by the gate/up GEMM for every live row) quantised along I; same
-// walk as k_nv_gather_x with 64 bytes of fp32 in per block.
+// walk as k_nv_gather_x with 64 bytes of fp32 in per block.  With dst (dA, dB in the backward)
+// the rows are also stored in bf16 (round to nearest even), the weight gradients' operand.
 __global__ void __launch_bounds__(256) k_nv_quant_h(const float* __restrict__ h, const int* __restrict__ row_asg,
                                                     const int* __restrict__ lo, const int* __restrict__ hi, int I,
                                                     const float* __restrict__ gsp, uint8_t* __restrict__ q,
-                                                    uint8_t* __restrict__ qs) {
+                                                    uint8_t* __restrict__ qs, __nv_bfloat16* __restrict__ dst) {
   const int r0 = __ldg(lo), r1 = __ldg(hi);
   const float gs = __ldg(gsp);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -121,6 +122,7 @@ __global__ void __launch_bounds__(256) k_nv_quant_h(const float* __restrict__ h,
     if (__ldg(row_asg + R) == ROW_DEAD) continue;
     const float4* in = reinterpret_cast<const float4*>(h + R * I);
     uint2* qd = reinterpret_cast<uint2*>(q + R * (I / 2));
+    uint4* o = dst ? reinterpret_cast<uint4*>(dst + R * I) : nullptr;
     for (int c = lane; c < nb; c += 32) {
       float v[16];
 #pragma unroll
@@ -130,6 +132,12 @@ __global__ void __launch_bounds__(256) k_nv_quant_h(const float* __restrict__ h,
         v[4 * j + 1] = f.y;
         v[4 * j + 2] = f.z;
         v[4 * j + 3] = f.w;
+      }
+      if (o) {
+        o[2 * c] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                              pack_bf16(v[6], v[7]));
+        o[2 * c + 1] = make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]), pack_bf16(v[12], v[13]),
+                                  pack_bf16(v[14], v[15]));
       }
       uint32_t w[2];
       const uint8_t sb = nv_quant16(v, gs, w);
@@ -260,8 +268,8 @@ cudaError_t launch_nv_quant_rows(const __nv_bfloat16* src, int64_t R, int K, con
 }
 
 cudaError_t launch_nv_quant_h(const Layout& L, const Ctx& c, const float* h, const float* gs, uint8_t* q, uint8_t* qs,
-                              cudaStream_t st) {
-  k_nv_quant_h<<<nv_grid_rows(L.RP), 256, 0, st>>>(h, c.row_asg, c.poff, c.poff + L.El, L.I, gs, q, qs);
+                              __nv_bfloat16* dst, cudaStream_t st) {
+  k_nv_quant_h<<<nv_grid_rows(L.RP), 256, 0, st>>>(h, c.row_asg, c.poff, c.poff + L.El, L.I, gs, q, qs, dst);
   return cudaGetLastError();
 }
 
