@@ -218,7 +218,8 @@ const char* moe_kernel_name(int kernel_id);
 unsigned long long moe_kernel_launches(void);
 
 /* ---------------------------------------------------------------------------
- * MXFP8 mode (page 1: "It supports BF16 and MXFP8 precision modes").  Shapes
+ * MXFP8 mode (page 1, closing paragraph of "Three design decisions that matter": the layer
+ * has a BF16 and an MXFP8 precision mode).  Shapes
  * carry prec = MOE_MXFP8.  E4M3 codes with one E8M0 scale per 32 values along
  * each GEMM's contraction dimension (OCP MX: scale exponent = floor(log2 amax)
  * - 8; codes rounded to nearest even, saturating at +-448).  The gate/up and

@@ -309,7 +309,8 @@ def token_forward_backward(t: int, X, W_r, bias, W_gate, W_up, W_down, top_k: in
 
 
 # ----------------------------------------------------------------------------
-# MXFP8 (page 1: "It supports BF16 and MXFP8 precision modes").  The block
+# MXFP8 (page 1, closing paragraph of "Three design decisions that matter": the layer has a
+# BF16 and an MXFP8 precision mode).  The block
 # format (E4M3 payload, one E8M0 power-of-two scale per 32 values along the
 # contraction dimension) is the OCP Microscaling v1.0 format; the scale rule is
 # that format's: shared exponent = floor(log2(amax)) - emax(E4M3) = ... - 8.
