@@ -54,3 +54,24 @@ def test_traffic_figure_only_for_the_captured_sources():
     assert t is None or (t == value and src == bench.gemm_source_hash())
     assert bench.ncu_traffic(key[0], key[1] + "+wgrad_fp32") is None
     assert bench.ncu_traffic("no_such_kernel", key[1]) is None
+
+
+def test_nvfp4_step_accounting():
+    # the NVFP4 step's four expert GEMMs carry the layer's forward and dgrad FLOPs (6 + 6 d I per
+    # assignment), the bf16 weight gradients the other 6; their weights stream at 9/16 byte per value
+    for name in ("dsv3_nv", "epnv_n2368"):
+        w = IN.WORKLOADS[name]
+        by, fl = bench.nv_algorithmic(w)
+        rows, d, I, El = bench.local_rows(w), w.d, w.I, w.El
+        nv = [fl[k] for k in bench.NV_GEMMS]
+        assert sum(nv) == 12 * d * I * rows
+        assert fl["gemm_wgrad_gateup"] + fl["gemm_wgrad_down"] == 6 * d * I * rows
+        assert sum(nv) + fl["gemm_wgrad_gateup"] + fl["gemm_wgrad_down"] == 18 * d * I * rows
+        W = El * d * I * 9 / 16
+        assert by["gemm_down_combw_nvfp4"] == W + rows * I * 9 / 16 + rows * d * 2
+        assert by["gemm_dgrad_gateup_nvfp4"] == 2 * W + 2 * rows * I * 9 / 16 + rows * d * 2
+        # the weight gradients are the bf16 layer's
+        assert by["gemm_wgrad_gateup"] == bench.algorithmic_bytes(w)["gemm_wgrad_gateup"]
+        cfg = bench.nv_config(w)
+        assert cfg["precision"] == "nvfp4" and cfg["wgrad_dtype"] == "bf16" and " nvfp4," in cfg["workload"]
+    assert IN.WORKLOADS["dsv3_nv"].model_flops() == IN.WORKLOADS["dsv3"].model_flops()
